@@ -1,0 +1,170 @@
+/*
+ * kd.h -- C ABI of the B200 (sm_100a) mixture-of-experts decode layer library
+ * (libkd.so).
+ *
+ * One call of kd_decode_layer runs one decode step of one transformer layer
+ * for M tokens (1..64), the chain described for vLLM's latency-specialised
+ * Kimi K3 decode path:
+ *   - fused QKV input projection            (wireai.ir "vLLM Blackwell Kimi decode",
+ *                                            section "4 key changes", item 1)
+ *   - output projection + residual add      (same section, item 2)
+ *   - router logits, top-k, renormalised    (same section, item 3;
+ *     softmax                                bigchange.ai "where the time went")
+ *   - shared SwiGLU expert on a second      (same section, item 3)
+ *     stream, overlapping the routed path
+ *   - routed SwiGLU experts over the active experts only, weighted combine
+ * and the multi-layer loop of a decode step captured in a CUDA graph with the
+ * next layer's static weights prefetched into L2 (same section, item 4, and
+ * section "extending the pattern to other models").
+ *
+ * Per token t, with x_t = hidden[t] and a_t = attn_out[t]:
+ *   qkv_t = Wqkv x_t ;  h1_t = x_t + Wo a_t ;  l_t = Wr h1_t + b
+ *   S_t   = top-k(l_t) (ties -> lower expert id)
+ *   g_e   = exp(l_e) / sum_{i in S_t} exp(l_i)            e in S_t
+ *   F(v)  = Wd (silu(Wg v) * (Wu v))
+ *   hidden[t] <- bf16( h1_t + F_shared(h1_t) + sum_{e in S_t} g_e F_e(h1_t) )
+ *
+ * Conventions
+ *   - Every function returns KD_OK (0) or a negative KD_E* code; the message
+ *     of the last failure on the calling thread is kd_last_error().
+ *   - Device pointers are plain CUDA device addresses on the layer's device.
+ *     `stream` arguments are cudaStream_t values passed as void* (NULL = the
+ *     legacy default stream).
+ *   - Nothing here falls back to another implementation: unsupported shapes
+ *     are rejected with KD_EINVAL / KD_ERANGE.
+ */
+#ifndef KD_H
+#define KD_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define KD_OK 0
+#define KD_EINVAL (-1)       /* null pointer, bad config field                  */
+#define KD_ERANGE (-2)       /* M outside 1..max_tokens                          */
+#define KD_ECUDA (-3)        /* a CUDA runtime call failed                       */
+#define KD_ENOMEM (-4)       /* device or host allocation failed                 */
+#define KD_ETIMEOUT (-5)     /* a kernel's bounded wait gave up (device error)   */
+#define KD_EDEVICE (-6)      /* other device-side error flag (bad routing)       */
+
+#define KD_WBF16 0           /* bf16 weights                                     */
+#define KD_WFP8 1            /* FP8 e4m3 weights, one fp32 scale per 128x128 block */
+
+typedef struct kd_config {
+  int hidden;        /* H; multiple of 128                                      */
+  int q_heads;       /* attention heads: attn_out width A = q_heads * head_dim  */
+  int kv_heads;      /* QKV width = (q_heads + 2 kv_heads) * head_dim            */
+  int head_dim;      /* A multiple of 128                                       */
+  int n_experts;     /* E routed experts, 1..1024                                */
+  int top_k;         /* k, 1..min(E, 16)                                          */
+  int n_shared;      /* shared experts: 0 or 1                                   */
+  int inter;         /* I expert intermediate size; multiple of 128              */
+  int wdtype;        /* KD_WBF16 or KD_WFP8                                      */
+  int layer_id;      /* id of the layer in the seeded weight generator           */
+  int max_tokens;    /* largest M a call may use, 1..64; sizes the workspaces    */
+  const float* router_bias; /* host [E] additive router bias, or NULL; copied    */
+} kd_config;
+
+typedef struct kd_layer kd_layer;
+typedef struct kd_stack kd_stack;
+
+/* Allocate one layer on the current CUDA device and generate its weights on
+ * the device from (seed, layer_id) with the counter-based generator of
+ * kdgen/kd_gen.h (synchronous).  The layer owns weights, workspaces, a side
+ * stream and events; *out receives the handle.  Errors: KD_EINVAL for a bad
+ * config, KD_ENOMEM, KD_ECUDA. */
+int kd_layer_create(const kd_config* cfg, uint64_t seed, kd_layer** out);
+
+/* Release everything kd_layer_create allocated (NULL is ignored).  The caller
+ * must make sure no call on the layer is still running on the device. */
+void kd_layer_destroy(kd_layer* layer);
+
+/* One decode step of the layer for M tokens, enqueued on `stream`.
+ *   hidden_inout  bf16 [M, H] device, row-major: the layer input x on entry,
+ *                 the layer output on exit (updated in place, stream-ordered)
+ *   attn_out      bf16 [M, q_heads*head_dim] device, row-major (read only)
+ * The call makes no host synchronisation and allocates nothing, so it can be
+ * captured into a CUDA graph.  Two calls on one layer must not overlap on the
+ * device (they share the layer's workspaces).  Errors: KD_EINVAL (null
+ * pointers), KD_ERANGE (M outside 1..max_tokens), KD_ECUDA (launch failure).
+ * Device-side failures are reported by kd_layer_check. */
+int kd_decode_layer(kd_layer* layer, void* hidden_inout, const void* attn_out, int M,
+                    void* stream);
+
+/* Synchronise the device and report (then clear) the layer's device error
+ * word: KD_OK, KD_ETIMEOUT (a bounded wait inside a kernel gave up) or
+ * KD_EDEVICE. */
+int kd_layer_check(kd_layer* layer);
+
+/* bf16 [M, (q_heads + 2 kv_heads) * head_dim] QKV projection of the last call
+ * (layer-owned device buffer, valid until the next call on the layer). */
+const void* kd_layer_qkv(const kd_layer* layer);
+
+/* Enqueue on `stream` an L2 prefetch of the layer's static weights (QKV,
+ * o-proj, router, shared expert), at most `max_bytes` of them in that order
+ * (0 = the device's L2 size).  Static weights only: activations are never
+ * prefetched (wireai.ir, section "validation of AI-generated kernels"). */
+int kd_layer_prefetch_l2(const kd_layer* layer, size_t max_bytes, void* stream);
+
+/* Intermediate device buffers of the last call, for tests and tools.
+ *   which: KD_T_H1F fp32 [M,H] | KD_T_H1B bf16 [M,H] | KD_T_LOGITS fp32 [M,E]
+ *          KD_T_IDX int32 [M,k] | KD_T_GATES fp32 [M,k]
+ *          KD_T_COUNTS int32 [E] | KD_T_NACTIVE int32 [1]
+ *          KD_T_YSHARED fp32 [M,H] | KD_T_YROUTED fp32 [M*k,H]
+ * *dev_ptr receives the layer-owned pointer. */
+#define KD_T_H1F 0
+#define KD_T_H1B 1
+#define KD_T_LOGITS 2
+#define KD_T_IDX 3
+#define KD_T_GATES 4
+#define KD_T_COUNTS 5
+#define KD_T_NACTIVE 6
+#define KD_T_YSHARED 7
+#define KD_T_YROUTED 8
+int kd_layer_debug_tensor(const kd_layer* layer, int which, void** dev_ptr);
+
+/* Device copy of one generated weight matrix in its LOGICAL layout, for
+ * checking the generator: kind 1 QKV [Nqkv,H], 2 o-proj [H,A], 3 router [E,H],
+ * 4 gate [I,H], 5 up [I,H], 6 down [H,I]; expert -1 = shared, else routed id.
+ * Copies rows [row0, row0+nrows) into dst (host memory): bf16 bits (2 bytes
+ * per element) or e4m3 codes (1 byte); for FP8 also the fp32 scales of the
+ * rows' 128-row blocks into dst_scales (host, may be NULL). */
+int kd_layer_read_weight(const kd_layer* layer, int kind, int expert, int row0, int nrows,
+                         void* dst, float* dst_scales);
+
+/* Byte counts used for the HBM roofline: static weight bytes (QKV, o-proj,
+ * router, shared expert, with FP8 scales) and the bytes of one routed expert. */
+int kd_layer_bytes(const kd_layer* layer, uint64_t* static_bytes, uint64_t* expert_bytes);
+
+/* Multi-layer decode step.  kd_stack_create records the layers (not owned)
+ * and the token count; kd_stack_run runs layer 0..n-1 in order on `stream`,
+ * reading attn_out for layer l at attn_out + l*M*A, and carrying hidden.
+ * On the first run (and whenever the pointers change) the sequence is
+ * captured into a CUDA graph, which later runs replay; with prefetch != 0,
+ * while layer l runs, a side stream prefetches layer l+1's static weights into
+ * L2.  The first run of a new pointer set must not itself be inside a stream
+ * capture. */
+int kd_stack_create(kd_layer* const* layers, int n_layers, int M, int prefetch, kd_stack** out);
+int kd_stack_run(kd_stack* stack, void* hidden_inout, const void* attn_out, void* stream);
+void kd_stack_destroy(kd_stack* stack);
+
+/* Profiling hook: with n_events == KD_N_TIMING_EVENTS, later kd_decode_layer
+ * calls record the caller's events (cudaEvent_t values created with timing)
+ * on the call's stream at: [0] start, [1] after the QKV + o-proj kernel,
+ * [2] after the router kernel, [3] after the routed gate/up kernel, [4] after
+ * the routed down kernel, [5] after the final combine.  n_events == 0 turns
+ * it off.  The events are not owned by the layer.  Errors: KD_EINVAL. */
+#define KD_N_TIMING_EVENTS 6
+int kd_layer_set_timing_events(kd_layer* layer, void* const* events, int n_events);
+
+/* Message of the last failure on the calling thread ("" if none). */
+const char* kd_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

@@ -1,0 +1,143 @@
+// kd_common.cuh -- sm_100a building blocks shared by the layer's kernels:
+// mbarriers with bounded waits, 1-D bulk TMA copies, L2 prefetch, the device
+// error word, and bf16 / e4m3 unpacking.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#define KD_DEV __device__ __forceinline__
+
+namespace kd {
+
+// Device error word bits (the layer's `err` buffer; read by kd_layer_check).
+enum : unsigned {
+  ERR_WAIT_FULL = 1u,   // consumer gave up waiting for a weight stage
+  ERR_WAIT_EMPTY = 2u,  // producer gave up waiting for a free stage
+  ERR_WAIT_MMA = 4u,    // tensor-core pipeline wait gave up
+  ERR_BAD_ROUTE = 8u,   // routing produced an out-of-range expert id
+};
+
+// Every spin-wait gives up after this many nanoseconds of %globaltimer.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+
+KD_DEV uint64_t globaltimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+KD_DEV uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+KD_DEV void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+KD_DEV void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+KD_DEV void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+KD_DEV void mbar_arrive(uint64_t* bar) {
+  asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}"
+               ::"r"(smem_u32(bar)) : "memory");
+}
+
+KD_DEV void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}"
+               ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+
+KD_DEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+  return ok != 0;
+}
+
+// Wait for phase `parity` of an mbarrier to complete; false after the time
+// limit (the caller records the error and stops its loop).
+KD_DEV bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  uint64_t t0 = globaltimer();
+  for (uint32_t it = 0;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 255u) == 255u && globaltimer() - t0 > kWaitLimitNs) return false;
+  }
+}
+
+// 1-D bulk copy global -> shared, completion counted on `bar` in bytes.
+// Both addresses 16-byte aligned, size a multiple of 16.
+KD_DEV void bulk_g2s(void* dst_smem, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(smem_u32(dst_smem)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
+}
+
+// Bring a global range into L2 without a destination (static weights only).
+KD_DEV void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
+KD_DEV void named_bar_sync(uint32_t id, uint32_t nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+KD_DEV void set_error(unsigned* err, unsigned bit) {
+  if (err) atomicOr(err, bit);
+}
+
+// Programmatic dependent launch: wait for the preceding grid's memory to be
+// visible / let the next grid start its prologue.
+KD_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+KD_DEV void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
+KD_DEV uint4 ld_nc_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+  return v;
+}
+
+KD_DEV uint4 lds_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(smem_u32(p)));
+  return v;
+}
+
+// bf16 pair packed in a u32 -> two fp32 (exact).
+KD_DEV float bf_lo(uint32_t u) { return __uint_as_float(u << 16); }
+KD_DEV float bf_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
+
+// Four e4m3 codes packed in a u32 -> four fp32 (exact, via f16x2).
+KD_DEV void e4m3x4_to_f32(uint32_t u, float& a, float& b, float& c, float& d) {
+  uint32_t lo, hi;
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, l;\n\tcvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+      : "=r"(lo), "=r"(hi) : "r"(u));
+  __half2 h0 = *reinterpret_cast<__half2*>(&lo);
+  __half2 h1 = *reinterpret_cast<__half2*>(&hi);
+  float2 f0 = __half22float2(h0), f1 = __half22float2(h1);
+  a = f0.x; b = f0.y; c = f1.x; d = f1.y;
+}
+
+KD_DEV uint16_t f32_to_bf16_bits(float f) {
+  __nv_bfloat16 b = __float2bfloat16_rn(f);
+  return *reinterpret_cast<uint16_t*>(&b);
+}
+
+KD_DEV float silu(float z) { return z / (1.0f + expf(-z)); }
+
+}  // namespace kd

@@ -1,0 +1,421 @@
+// kd_kernels.cuh -- the decode layer's kernels on CUDA cores (GEMV regime) and
+// the device-side weight generator.
+//
+//   gen_bf16_kernel / gen_fp8_kernel  weights from the seeded generator
+//   proj_kernel        fused QKV projection + o-proj with residual epilogue
+//   router_kernel      fp32 router logits, then (last CTA) top-k, renormalised
+//                      softmax and the per-expert token lists
+//   gateup_kernel      SwiGLU gate/up of the active experts (or the shared one)
+//   down_kernel        down projection of the active experts (or the shared one)
+//   combine_kernel     h1 + shared + gate-weighted routed outputs -> bf16
+#pragma once
+
+#include "../../kdgen/kd_gen.h"
+#include "kd_stream.cuh"
+
+namespace kd {
+
+// ------------------------------------------------------------------ generator
+
+// dst[(r*row_mult + row_off) * K + c] = bf16(value(stream, r*K + c)), r < R.
+__global__ void gen_bf16_kernel(uint16_t* __restrict__ dst, int R, int K, uint64_t stream,
+                                int row_mult, int row_off) {
+  const uint64_t n = (uint64_t)R * (uint64_t)K;
+  for (uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (uint64_t)gridDim.x * blockDim.x) {
+    const uint64_t r = i / (uint64_t)K, c = i - r * (uint64_t)K;
+    dst[(r * row_mult + row_off) * (uint64_t)K + c] = kdg_bf16(kdg_value(stream, i, KDG_W002));
+  }
+}
+
+// One 128x128 block per CTA (256 threads): amax -> scale -> e4m3 codes.
+// scales: [ceil(R/128), ceil(K/128)] table of this logical matrix.
+__global__ void __launch_bounds__(256) gen_fp8_kernel(uint8_t* __restrict__ dst,
+                                                      float* __restrict__ scales, int R, int K,
+                                                      uint64_t stream, int row_mult, int row_off) {
+  const int kb = blockIdx.x, rb = blockIdx.y, nkb = gridDim.x;
+  __shared__ float wmax[8];
+  float v[64];
+  float amax = 0.f;
+#pragma unroll
+  for (int q = 0; q < 64; ++q) {
+    const int e = threadIdx.x + 256 * q;
+    const int r = rb * 128 + (e >> 7), c = kb * 128 + (e & 127);
+    v[q] = 0.f;
+    if (r < R && c < K) {
+      v[q] = kdg_value(stream, (uint64_t)r * (uint64_t)K + (uint64_t)c, KDG_W002);
+      amax = fmaxf(amax, fabsf(v[q]));
+    }
+  }
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  amax = wmax[0];
+  for (int w = 1; w < 8; ++w) amax = fmaxf(amax, wmax[w]);
+  const float sc = kdg_fp8_scale(amax);
+  if (threadIdx.x == 0) scales[rb * nkb + kb] = sc;
+#pragma unroll
+  for (int q = 0; q < 64; ++q) {
+    const int e = threadIdx.x + 256 * q;
+    const int r = rb * 128 + (e >> 7), c = kb * 128 + (e & 127);
+    if (r < R && c < K)
+      dst[((uint64_t)r * row_mult + row_off) * (uint64_t)K + c] = kdg_e4m3(kdg_fp8_div(v[q], sc));
+  }
+}
+
+// ------------------------------------------------------------------ layer params
+
+struct LayerDev {
+  int H, A, Nqkv, E, k, I, S, eb;       // eb = weight element bytes (2 bf16, 1 fp8)
+  int nHb, nAb, nIb;                    // 128-blocks along H, A, I
+  // weights (physical layouts; see kd_layer.cu)
+  const uint8_t* wqkv; const uint8_t* wo; const uint8_t* wr;
+  const uint8_t* wgu_sh; const uint8_t* wd_sh;
+  const uint8_t* wgu; const uint8_t* wd;   // routed, expert-major
+  const float* sqkv; const float* so; const float* sr;
+  const float* sgu_sh; const float* sd_sh; const float* sgu; const float* sd;
+  const float* bias;                       // [E] or null
+  // workspaces
+  uint16_t* qkv; float* h1f; uint16_t* h1b;
+  float* logits; int* idx; float* gates;
+  int* counts; int* offsets; int* perm; int* active; int* n_active;
+  uint16_t* act; uint16_t* act_sh;         // [Mmax*k, I] by position, [Mmax, I]
+  float* yr; float* ysh;                   // [Mmax*k, H] by token*k+slot, [Mmax, H]
+  unsigned* counter;                       // router arrival counter (self-resetting)
+  unsigned* err;
+};
+
+struct Acts {                              // per-call activations
+  const uint16_t* x;                       // [M, H] (layer input)
+  const uint16_t* attn;                    // [M, A]
+  uint16_t* out;                           // [M, H] (layer output, = x in place)
+  int M;
+};
+
+KD_DEV int split_lo(int n, int parts, int i) { return (int)(((long long)n * i) / parts); }
+
+// ------------------------------------------------------------------ QKV + o-proj
+
+struct ProjPlan {
+  const LayerDev* L; Acts a;
+  int q0, q1, o0, o1;
+  KD_DEV int num_segments() const { return 2; }
+  KD_DEV Seg segment(int i) const {
+    Seg s;
+    if (i == 0) {
+      s.row_bytes = L->H * L->eb; s.w = L->wqkv + (size_t)q0 * s.row_bytes;
+      s.nrows = q1 - q0; s.row0 = q0;
+    } else {
+      s.row_bytes = L->A * L->eb; s.w = L->wo + (size_t)o0 * s.row_bytes;
+      s.nrows = o1 - o0; s.row0 = o0;
+    }
+    s.tok0 = 0; s.ntok = a.M; s.tag = i;
+    return s;
+  }
+  KD_DEV const void* act_row(const Seg& s, int j) const {
+    return s.tag == 0 ? (const void*)(a.x + (size_t)j * L->H) : (const void*)(a.attn + (size_t)j * L->A);
+  }
+  KD_DEV const float* scale_row(const Seg& s, int row) const {
+    return s.tag == 0 ? L->sqkv + (size_t)(row >> 7) * L->nHb : L->so + (size_t)(row >> 7) * L->nAb;
+  }
+  KD_DEV bool paired() const { return false; }
+  KD_DEV void epilogue(const Seg& s, int row, int j, float v) const {
+    if (s.tag == 0) {
+      L->qkv[(size_t)j * L->Nqkv + row] = f32_to_bf16_bits(v);
+    } else {
+      const size_t o = (size_t)j * L->H + row;
+      const float h = __uint_as_float((uint32_t)a.x[o] << 16) + v;
+      L->h1f[o] = h;
+      L->h1b[o] = f32_to_bf16_bits(h);
+    }
+  }
+  KD_DEV void epilogue2(const Seg&, int, int, float, float) const {}
+};
+
+template <int WT>
+__global__ void __launch_bounds__(kThreads, 1) proj_kernel(LayerDev L, Acts a) {
+  extern __shared__ uint8_t smem[];
+  ProjPlan p;
+  p.L = &L; p.a = a;
+  p.q0 = split_lo(L.Nqkv, gridDim.x, blockIdx.x); p.q1 = split_lo(L.Nqkv, gridDim.x, blockIdx.x + 1);
+  p.o0 = split_lo(L.H, gridDim.x, blockIdx.x); p.o1 = split_lo(L.H, gridDim.x, blockIdx.x + 1);
+  stream_run<WT, A_BF16>(p, smem, L.err);
+}
+
+// ------------------------------------------------------------------ router
+
+// Logits: one warp per (expert row, group of 8 tokens).  Then the last CTA to
+// finish selects the top-k per token (descending logit, ties -> lower id),
+// forms the renormalised softmax and builds the per-expert token lists:
+//   counts[e], offsets[e] (exclusive scan), perm[pos] = token*k + slot sorted
+//   by (expert, token*k + slot), active[a] = a-th expert with tokens, n_active.
+constexpr int kRouterThreads = 256;
+constexpr int kRouterTok = 8;
+
+template <int WT>
+__global__ void __launch_bounds__(kRouterThreads) router_kernel(LayerDev L, int M) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ngroups = (M + kRouterTok - 1) / kRouterTok;
+  const int units = L.E * ngroups;
+  const int row_bytes = L.H * L.eb;
+  const int epc = WT == W_BF16 ? 8 : 16;
+  const int nchunk = row_bytes / 16;
+  for (int u = blockIdx.x * (kRouterThreads / 32) + warp; u < units;
+       u += gridDim.x * (kRouterThreads / 32)) {
+    const int e = u / ngroups, g = u % ngroups;
+    const int t0 = g * kRouterTok, nt = M - t0 < kRouterTok ? M - t0 : kRouterTok;
+    float acc[kRouterTok];
+#pragma unroll
+    for (int t = 0; t < kRouterTok; ++t) acc[t] = 0.f;
+    const uint8_t* wrow = L.wr + (size_t)e * row_bytes;
+    const float* srow = WT == W_FP8 ? L.sr + (size_t)(e >> 7) * L.nHb : nullptr;
+    for (int c = lane; c < nchunk; c += 32) {
+      const uint4 wv = ld_nc_v4(wrow + (size_t)c * 16);
+      const int col = c * epc;
+      const void* arow[kTT];
+      for (int tq = 0; tq < nt; tq += kTT) {
+        const int ntq = nt - tq < kTT ? nt - tq : kTT;
+#pragma unroll
+        for (int t = 0; t < kTT; ++t)
+          arow[t] = L.h1f + (size_t)(t0 + tq + (t < ntq ? t : 0)) * L.H;
+        float part[kTT] = {0.f, 0.f, 0.f, 0.f};
+        chunk_fma<WT, A_F32>(wv, WT == W_FP8 ? srow[col >> 7] : 1.f, arow, col, ntq, part);
+#pragma unroll
+        for (int t = 0; t < kTT; ++t)
+          if (t < ntq) acc[tq + t] += part[t];
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < kRouterTok; ++t) {
+      float v = acc[t];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if (lane == 0 && t < nt) L.logits[(size_t)(t0 + t) * L.E + e] = v + (L.bias ? L.bias[e] : 0.f);
+    }
+  }
+
+  // ---- last CTA: selection and dispatch
+  __shared__ unsigned s_ticket;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) s_ticket = atomicAdd(L.counter, 1u);
+  __syncthreads();
+  if (s_ticket != gridDim.x - 1) return;
+  if (threadIdx.x == 0) *L.counter = 0u;  // ready for the next call / graph replay
+  __threadfence();
+
+  __shared__ int s_sel[64 * 16];
+  __shared__ int s_cnt[1024];
+  __shared__ int s_off[1025];
+  const int k = L.k, E = L.E;
+  // top-k: one warp per token; lane holds logits lane, lane+32, ...
+  for (int t = warp; t < M; t += kRouterThreads / 32) {
+    float lv[32];
+    const int per = (E + 31) / 32;
+#pragma unroll
+    for (int q = 0; q < 32; ++q) {
+      const int e = lane + 32 * q;
+      lv[q] = (q < per && e < E) ? __ldcg(L.logits + (size_t)t * E + e) : -INFINITY;
+    }
+    unsigned taken = 0u;  // bit q: lane's q-th logit already selected
+    float sel_v[16];
+    for (int j = 0; j < k; ++j) {
+      // lane-local best not yet taken: larger value, then lower expert id
+      float bv = -INFINITY; int be = 0x7fffffff;
+#pragma unroll
+      for (int q = 0; q < 32; ++q) {
+        const int e = lane + 32 * q;
+        if (q < per && e < E && !(taken >> q & 1u) && (lv[q] > bv || (lv[q] == bv && e < be))) {
+          bv = lv[q]; be = e;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+        if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
+      }
+      if ((be & 31) == lane) taken |= 1u << (be >> 5);
+      sel_v[j] = bv;
+      if (lane == 0) s_sel[t * k + j] = be;
+    }
+    if (lane == 0) {
+      float den = 0.f;
+      for (int j = 0; j < k; ++j) den += expf(sel_v[j] - sel_v[0]);
+      for (int j = 0; j < k; ++j) {
+        L.idx[t * k + j] = s_sel[t * k + j];
+        L.gates[t * k + j] = expf(sel_v[j] - sel_v[0]) / den;
+      }
+    }
+  }
+  for (int e = threadIdx.x; e < E; e += kRouterThreads) s_cnt[e] = 0;
+  __syncthreads();
+  const int ncode = M * k;
+  for (int c = threadIdx.x; c < ncode; c += kRouterThreads) {
+    const int e = s_sel[c];
+    if (e < 0 || e >= E) set_error(L.err, ERR_BAD_ROUTE);
+    else atomicAdd(&s_cnt[e], 1);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int run = 0, na = 0;
+    for (int e = 0; e < E; ++e) {
+      s_off[e] = run;
+      run += s_cnt[e];
+      if (s_cnt[e] > 0) L.active[na++] = e;
+    }
+    s_off[E] = run;
+    *L.n_active = na;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += kRouterThreads) {
+    L.counts[e] = s_cnt[e];
+    L.offsets[e] = s_off[e];
+  }
+  if (threadIdx.x == 0) L.offsets[E] = s_off[E];
+  for (int c = threadIdx.x; c < ncode; c += kRouterThreads) {
+    const int e = s_sel[c];
+    if (e < 0 || e >= E) continue;
+    int rank = 0;
+    for (int c2 = 0; c2 < c; ++c2) rank += (s_sel[c2] == e);
+    L.perm[s_off[e] + rank] = c;
+  }
+}
+
+// ------------------------------------------------------------------ experts
+
+// Routed mode: CTA b takes pairs / rows [lo, hi) of the concatenation over
+// active experts (in expert-id order).  Shared mode: one expert, all tokens.
+struct ExpertRange {
+  int n_act, per, lo, hi;   // per = units per expert
+  KD_DEV int num_segments() const {
+    if (hi <= lo) return 0;
+    return (hi - 1) / per - lo / per + 1;
+  }
+  KD_DEV void seg(int i, int& a, int& u0, int& u1) const {
+    a = lo / per + i;
+    const int b0 = a * per, b1 = b0 + per;
+    u0 = (lo > b0 ? lo : b0) - b0;
+    u1 = (hi < b1 ? hi : b1) - b0;
+  }
+};
+
+struct GateUpPlan {
+  const LayerDev* L; int M; bool shared; ExpertRange R;
+  KD_DEV int num_segments() const { return R.num_segments(); }
+  KD_DEV Seg segment(int i) const {
+    int a, u0, u1;
+    R.seg(i, a, u0, u1);
+    Seg s;
+    s.row_bytes = L->H * L->eb;
+    const size_t estride = (size_t)2 * L->I * s.row_bytes;
+    if (shared) {
+      s.tag = -1; s.w = L->wgu_sh; s.tok0 = 0; s.ntok = M;
+    } else {
+      const int e = L->active[a];
+      s.tag = e; s.w = L->wgu + (size_t)e * estride;
+      s.tok0 = L->offsets[e]; s.ntok = L->counts[e];
+    }
+    s.w += (size_t)(2 * u0) * s.row_bytes;
+    s.row0 = 2 * u0;
+    s.nrows = 2 * (u1 - u0);
+    return s;
+  }
+  KD_DEV const void* act_row(const Seg& s, int j) const {
+    const int t = shared ? j : L->perm[s.tok0 + j] / L->k;
+    return L->h1b + (size_t)t * L->H;
+  }
+  KD_DEV const float* scale_row(const Seg& s, int prow) const {
+    const float* base = shared ? L->sgu_sh : L->sgu + (size_t)s.tag * 2 * L->nIb * L->nHb;
+    return base + (size_t)((prow & 1) * L->nIb + ((prow >> 1) >> 7)) * L->nHb;
+  }
+  KD_DEV bool paired() const { return true; }
+  KD_DEV void epilogue(const Seg&, int, int, float) const {}
+  KD_DEV void epilogue2(const Seg& s, int i, int j, float g, float u) const {
+    const float v = silu(g) * u;
+    uint16_t* dst = shared ? L->act_sh + (size_t)j * L->I : L->act + (size_t)(s.tok0 + j) * L->I;
+    dst[i] = f32_to_bf16_bits(v);
+  }
+};
+
+struct DownPlan {
+  const LayerDev* L; int M; bool shared; ExpertRange R;
+  KD_DEV int num_segments() const { return R.num_segments(); }
+  KD_DEV Seg segment(int i) const {
+    int a, u0, u1;
+    R.seg(i, a, u0, u1);
+    Seg s;
+    s.row_bytes = L->I * L->eb;
+    const size_t estride = (size_t)L->H * s.row_bytes;
+    if (shared) {
+      s.tag = -1; s.w = L->wd_sh; s.tok0 = 0; s.ntok = M;
+    } else {
+      const int e = L->active[a];
+      s.tag = e; s.w = L->wd + (size_t)e * estride;
+      s.tok0 = L->offsets[e]; s.ntok = L->counts[e];
+    }
+    s.w += (size_t)u0 * s.row_bytes;
+    s.row0 = u0;
+    s.nrows = u1 - u0;
+    return s;
+  }
+  KD_DEV const void* act_row(const Seg& s, int j) const {
+    return shared ? L->act_sh + (size_t)j * L->I : L->act + (size_t)(s.tok0 + j) * L->I;
+  }
+  KD_DEV const float* scale_row(const Seg& s, int row) const {
+    const float* base = shared ? L->sd_sh : L->sd + (size_t)s.tag * L->nHb * L->nIb;
+    return base + (size_t)(row >> 7) * L->nIb;
+  }
+  KD_DEV bool paired() const { return false; }
+  KD_DEV void epilogue(const Seg& s, int h, int j, float v) const {
+    if (shared) L->ysh[(size_t)j * L->H + h] = v;
+    else L->yr[(size_t)L->perm[s.tok0 + j] * L->H + h] = v;
+  }
+  KD_DEV void epilogue2(const Seg&, int, int, float, float) const {}
+};
+
+KD_DEV ExpertRange expert_range(int n_act, int per) {
+  ExpertRange r;
+  r.n_act = n_act; r.per = per;
+  const int total = n_act * per;
+  r.lo = split_lo(total, gridDim.x, blockIdx.x);
+  r.hi = split_lo(total, gridDim.x, blockIdx.x + 1);
+  return r;
+}
+
+template <int WT>
+__global__ void __launch_bounds__(kThreads, 1) gateup_kernel(LayerDev L, int M, int shared) {
+  extern __shared__ uint8_t smem[];
+  GateUpPlan p;
+  p.L = &L; p.M = M; p.shared = shared != 0;
+  const int n_act = shared ? 1 : *(volatile int*)L.n_active;
+  p.R = expert_range(n_act, L.I);
+  stream_run<WT, A_BF16>(p, smem, L.err);
+}
+
+template <int WT>
+__global__ void __launch_bounds__(kThreads, 1) down_kernel(LayerDev L, int M, int shared) {
+  extern __shared__ uint8_t smem[];
+  DownPlan p;
+  p.L = &L; p.M = M; p.shared = shared != 0;
+  const int n_act = shared ? 1 : *(volatile int*)L.n_active;
+  p.R = expert_range(n_act, L.H);
+  stream_run<WT, A_BF16>(p, smem, L.err);
+}
+
+// ------------------------------------------------------------------ combine
+
+__global__ void combine_kernel(LayerDev L, Acts a) {
+  const size_t n = (size_t)a.M * L.H;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (size_t)gridDim.x * blockDim.x) {
+    const int t = (int)(i / L.H), h = (int)(i % L.H);
+    float v = L.h1f[i];
+    if (L.S) v += L.ysh[i];
+    for (int j = 0; j < L.k; ++j)
+      v += L.gates[t * L.k + j] * L.yr[((size_t)t * L.k + j) * L.H + h];
+    a.out[i] = f32_to_bf16_bits(v);
+  }
+}
+
+}  // namespace kd

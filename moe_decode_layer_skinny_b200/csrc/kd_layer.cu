@@ -1,0 +1,587 @@
+// kd_layer.cu -- runtime of the decode layer and its C ABI (include/kd.h).
+//
+// HBM layout of one layer (all row-major, K contiguous; elem = 2 bytes bf16
+// or 1 byte e4m3; FP8 scales are fp32 per logical 128x128 block):
+//   wqkv  [Nqkv, H]          sqkv [Nqkv/128, H/128]
+//   wo    [H, A]             so   [H/128, A/128]
+//   wr    [E, H]             sr   [ceil(E/128), H/128]
+//   wgu   [E][2I, H]  physical row 2i = gate row i, 2i+1 = up row i
+//                            sgu  [E][2][I/128][H/128]   (gate blocks, then up)
+//   wd    [E][H, I]          sd   [E][H/128][I/128]
+//   shared expert: wgu_sh [2I, H], wd_sh [H, I] (same layouts, own scales)
+// Workspaces are sized for max_tokens and owned by the layer.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <vector>
+
+#include "../../include/kd.h"
+#include "kd_kernels.cuh"
+
+using namespace kd;
+
+static thread_local std::string g_err;
+
+static int fail(int code, const char* fmt, const char* a = "", long b = 0) {
+  char buf[512];
+  snprintf(buf, sizeof buf, fmt, a, b);
+  g_err = buf;
+  return code;
+}
+
+#define KD_CUDA(call)                                                                   \
+  do {                                                                                  \
+    cudaError_t e_ = (call);                                                            \
+    if (e_ != cudaSuccess) return fail(KD_ECUDA, "%s (line %ld)", cudaGetErrorString(e_), __LINE__); \
+  } while (0)
+
+struct kd_layer {
+  kd_config cfg{};
+  int dev = 0, nsm = 0, maxM = 0;
+  size_t l2_bytes = 0;
+  LayerDev d{};
+  std::vector<void*> allocs;
+  cudaStream_t side = nullptr;
+  cudaEvent_t ev_h1 = nullptr, ev_sh = nullptr;
+  uint64_t static_bytes = 0, expert_bytes = 0;
+  int Nqkv = 0, A = 0;
+  cudaEvent_t tev[KD_N_TIMING_EVENTS] = {};
+  bool timing = false;
+};
+
+struct kd_stack {
+  std::vector<kd_layer*> layers;
+  int M = 0, prefetch = 0;
+  cudaStream_t cap = nullptr, pf = nullptr;
+  std::vector<cudaEvent_t> ev_fork, ev_join;
+  cudaGraph_t graph = nullptr;
+  cudaGraphExec_t exec = nullptr;
+  void* hidden = nullptr;
+  const void* attn = nullptr;
+};
+
+extern "C" const char* kd_last_error(void) { return g_err.c_str(); }
+
+// ------------------------------------------------------------------ helpers
+
+static int dalloc(kd_layer* L, size_t bytes, void** p) {
+  if (bytes == 0) bytes = 16;
+  cudaError_t e = cudaMalloc(p, bytes);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    *p = nullptr;
+    return fail(KD_ENOMEM, "cudaMalloc of %s%ld bytes failed", "", (long)bytes);
+  }
+  L->allocs.push_back(*p);
+  return KD_OK;
+}
+
+template <class T>
+static int dalloc_t(kd_layer* L, size_t n, T** p) {
+  void* v = nullptr;
+  int rc = dalloc(L, n * sizeof(T), &v);
+  *p = static_cast<T*>(v);
+  return rc;
+}
+
+static int ceil128(int x) { return (x + 127) / 128; }
+
+// Generate one logical [R, K] matrix into `dst` with row stride multiplier
+// (physical row = r*mult + off); FP8 writes its block scales to `scales`.
+static int gen_matrix(const kd_layer* L, uint8_t* dst, float* scales, int R, int K, uint64_t seed,
+                      uint32_t kind, uint32_t slot, int mult, int off, cudaStream_t s) {
+  const uint64_t st = kdg_stream(seed, kdg_uid((uint32_t)L->cfg.layer_id, kind, slot));
+  if (L->cfg.wdtype == KD_WBF16) {
+    gen_bf16_kernel<<<L->nsm * 8, 256, 0, s>>>(reinterpret_cast<uint16_t*>(dst), R, K, st, mult, off);
+  } else {
+    gen_fp8_kernel<<<dim3(ceil128(K), ceil128(R)), 256, 0, s>>>(dst, scales, R, K, st, mult, off);
+  }
+  KD_CUDA(cudaGetLastError());
+  return KD_OK;
+}
+
+static void free_layer(kd_layer* L) {
+  if (!L) return;
+  for (void* p : L->allocs) cudaFree(p);
+  if (L->side) cudaStreamDestroy(L->side);
+  if (L->ev_h1) cudaEventDestroy(L->ev_h1);
+  if (L->ev_sh) cudaEventDestroy(L->ev_sh);
+  delete L;
+}
+
+static bool stream_kernels_configured = false;
+
+static int configure_kernels() {
+  if (stream_kernels_configured) return KD_OK;
+  const int smem = (int)kStreamSmem;
+  KD_CUDA(cudaFuncSetAttribute(proj_kernel<W_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  KD_CUDA(cudaFuncSetAttribute(proj_kernel<W_FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  KD_CUDA(cudaFuncSetAttribute(gateup_kernel<W_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  KD_CUDA(cudaFuncSetAttribute(gateup_kernel<W_FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  KD_CUDA(cudaFuncSetAttribute(down_kernel<W_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  KD_CUDA(cudaFuncSetAttribute(down_kernel<W_FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  stream_kernels_configured = true;
+  return KD_OK;
+}
+
+// ------------------------------------------------------------------ create
+
+extern "C" int kd_layer_create(const kd_config* cfg, uint64_t seed, kd_layer** out) {
+  if (!cfg || !out) return fail(KD_EINVAL, "kd_layer_create: null argument%s", "");
+  *out = nullptr;
+  const kd_config& c = *cfg;
+  const int A = c.q_heads * c.head_dim, Nqkv = (c.q_heads + 2 * c.kv_heads) * c.head_dim;
+  if (c.hidden <= 0 || c.hidden % 128 || c.q_heads <= 0 || c.kv_heads < 0 || c.head_dim <= 0 ||
+      A % 128 || Nqkv % 128 || c.n_experts < 1 || c.n_experts > 1024 || c.top_k < 1 ||
+      c.top_k > 16 || c.top_k > c.n_experts || c.n_shared < 0 || c.n_shared > 1 || c.inter <= 0 ||
+      c.inter % 128 || (c.wdtype != KD_WBF16 && c.wdtype != KD_WFP8) || c.max_tokens < 1 ||
+      c.max_tokens > 64 || c.layer_id < 0)
+    return fail(KD_EINVAL, "kd_layer_create: unsupported configuration%s", "");
+  if (c.hidden * 2 > kStageBytes || A * 2 > kStageBytes || c.inter * 2 > kStageBytes)
+    return fail(KD_EINVAL, "kd_layer_create: a weight row exceeds one %s%ld-byte stage", "",
+                (long)kStageBytes);
+
+  kd_layer* L = new kd_layer();
+  L->cfg = c;
+  L->cfg.router_bias = nullptr;
+  L->maxM = c.max_tokens;
+  L->Nqkv = Nqkv;
+  L->A = A;
+  int rc = KD_OK;
+#define TRY(x)                 \
+  do {                         \
+    rc = (x);                  \
+    if (rc != KD_OK) {         \
+      free_layer(L);           \
+      return rc;               \
+    }                          \
+  } while (0)
+#define TRYC(x)                                                                      \
+  do {                                                                               \
+    cudaError_t e_ = (x);                                                            \
+    if (e_ != cudaSuccess) {                                                         \
+      free_layer(L);                                                                 \
+      return fail(KD_ECUDA, "%s (line %ld)", cudaGetErrorString(e_), __LINE__);      \
+    }                                                                                \
+  } while (0)
+  TRYC(cudaGetDevice(&L->dev));
+  TRYC(cudaDeviceGetAttribute(&L->nsm, cudaDevAttrMultiProcessorCount, L->dev));
+  int l2 = 0;
+  TRYC(cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, L->dev));
+  L->l2_bytes = (size_t)l2;
+  TRY(configure_kernels());
+
+  LayerDev& d = L->d;
+  const int H = c.hidden, E = c.n_experts, I = c.inter, k = c.top_k, M = c.max_tokens;
+  const int eb = c.wdtype == KD_WBF16 ? 2 : 1;
+  const bool fp8 = c.wdtype == KD_WFP8;
+  d.H = H; d.A = A; d.Nqkv = Nqkv; d.E = E; d.k = k; d.I = I; d.S = c.n_shared; d.eb = eb;
+  d.nHb = ceil128(H); d.nAb = ceil128(A); d.nIb = ceil128(I);
+
+  uint8_t *wqkv, *wo, *wr, *wgu_sh = nullptr, *wd_sh = nullptr, *wgu, *wd;
+  float *sqkv = nullptr, *so = nullptr, *sr = nullptr, *sgu_sh = nullptr, *sd_sh = nullptr,
+        *sgu = nullptr, *sd = nullptr;
+  TRY(dalloc_t(L, (size_t)Nqkv * H * eb, &wqkv));
+  TRY(dalloc_t(L, (size_t)H * A * eb, &wo));
+  TRY(dalloc_t(L, (size_t)E * H * eb, &wr));
+  const size_t gu_bytes = (size_t)2 * I * H * eb, dn_bytes = (size_t)H * I * eb;
+  if (c.n_shared) {
+    TRY(dalloc_t(L, gu_bytes, &wgu_sh));
+    TRY(dalloc_t(L, dn_bytes, &wd_sh));
+  }
+  TRY(dalloc_t(L, gu_bytes * E, &wgu));
+  TRY(dalloc_t(L, dn_bytes * E, &wd));
+  const size_t n_sgu = (size_t)2 * d.nIb * d.nHb, n_sd = (size_t)d.nHb * d.nIb;
+  if (fp8) {
+    TRY(dalloc_t(L, (size_t)ceil128(Nqkv) * d.nHb, &sqkv));
+    TRY(dalloc_t(L, (size_t)d.nHb * d.nAb, &so));
+    TRY(dalloc_t(L, (size_t)ceil128(E) * d.nHb, &sr));
+    if (c.n_shared) {
+      TRY(dalloc_t(L, n_sgu, &sgu_sh));
+      TRY(dalloc_t(L, n_sd, &sd_sh));
+    }
+    TRY(dalloc_t(L, n_sgu * E, &sgu));
+    TRY(dalloc_t(L, n_sd * E, &sd));
+  }
+  d.wqkv = wqkv; d.wo = wo; d.wr = wr; d.wgu_sh = wgu_sh; d.wd_sh = wd_sh; d.wgu = wgu; d.wd = wd;
+  d.sqkv = sqkv; d.so = so; d.sr = sr; d.sgu_sh = sgu_sh; d.sd_sh = sd_sh; d.sgu = sgu; d.sd = sd;
+
+  const size_t sc = fp8 ? sizeof(float) : 0;
+  L->static_bytes = (size_t)Nqkv * H * eb + (size_t)H * A * eb + (size_t)E * H * eb +
+                    (c.n_shared ? gu_bytes + dn_bytes : 0) +
+                    sc * ((size_t)ceil128(Nqkv) * d.nHb + (size_t)d.nHb * d.nAb +
+                          (size_t)ceil128(E) * d.nHb + (c.n_shared ? n_sgu + n_sd : 0));
+  L->expert_bytes = gu_bytes + dn_bytes + sc * (n_sgu + n_sd);
+
+  float* bias = nullptr;
+  if (cfg->router_bias) {
+    TRY(dalloc_t(L, (size_t)E, &bias));
+    TRYC(cudaMemcpy(bias, cfg->router_bias, sizeof(float) * E, cudaMemcpyHostToDevice));
+  }
+  d.bias = bias;
+
+  TRY(dalloc_t(L, (size_t)M * Nqkv, &d.qkv));
+  TRY(dalloc_t(L, (size_t)M * H, &d.h1f));
+  TRY(dalloc_t(L, (size_t)M * H, &d.h1b));
+  TRY(dalloc_t(L, (size_t)M * E, &d.logits));
+  TRY(dalloc_t(L, (size_t)M * k, &d.idx));
+  TRY(dalloc_t(L, (size_t)M * k, &d.gates));
+  TRY(dalloc_t(L, (size_t)E, &d.counts));
+  TRY(dalloc_t(L, (size_t)E + 1, &d.offsets));
+  TRY(dalloc_t(L, (size_t)M * k, &d.perm));
+  TRY(dalloc_t(L, (size_t)E, &d.active));
+  TRY(dalloc_t(L, 1, &d.n_active));
+  TRY(dalloc_t(L, (size_t)M * k * I, &d.act));
+  TRY(dalloc_t(L, (size_t)M * I, &d.act_sh));
+  TRY(dalloc_t(L, (size_t)M * k * H, &d.yr));
+  TRY(dalloc_t(L, (size_t)M * H, &d.ysh));
+  TRY(dalloc_t(L, 1, &d.counter));
+  TRY(dalloc_t(L, 1, &d.err));
+  TRYC(cudaMemset(d.counter, 0, sizeof(unsigned)));
+  TRYC(cudaMemset(d.err, 0, sizeof(unsigned)));
+  TRYC(cudaMemset(d.n_active, 0, sizeof(int)));
+  TRYC(cudaMemset(d.ysh, 0, sizeof(float) * (size_t)M * H));
+
+  // weights from the seeded generator
+  cudaStream_t gs = nullptr;
+  TRYC(cudaStreamCreateWithFlags(&gs, cudaStreamNonBlocking));
+  auto gen = [&](uint8_t* dst, float* s, int R, int K, uint32_t kind, uint32_t slot, int mult,
+                 int off) { return gen_matrix(L, dst, s, R, K, seed, kind, slot, mult, off, gs); };
+  rc = gen(wqkv, sqkv, Nqkv, H, KDG_QKV, 0, 1, 0);
+  if (rc == KD_OK) rc = gen(wo, so, H, A, KDG_OPROJ, 0, 1, 0);
+  if (rc == KD_OK) rc = gen(wr, sr, E, H, KDG_ROUTER, 0, 1, 0);
+  for (int e = (c.n_shared ? -1 : 0); e < E && rc == KD_OK; ++e) {
+    uint8_t* gu = e < 0 ? wgu_sh : wgu + (size_t)e * gu_bytes;
+    uint8_t* dn = e < 0 ? wd_sh : wd + (size_t)e * dn_bytes;
+    float* sg = fp8 ? (e < 0 ? sgu_sh : sgu + (size_t)e * n_sgu) : nullptr;
+    float* sdn = fp8 ? (e < 0 ? sd_sh : sd + (size_t)e * n_sd) : nullptr;
+    const uint32_t slot = (uint32_t)(e + 1);
+    rc = gen(gu, sg, I, H, KDG_GATE, slot, 2, 0);
+    if (rc == KD_OK) rc = gen(gu, sg ? sg + (size_t)d.nIb * d.nHb : nullptr, I, H, KDG_UP, slot, 2, 1);
+    if (rc == KD_OK) rc = gen(dn, sdn, H, I, KDG_DOWN, slot, 1, 0);
+  }
+  cudaError_t se = cudaStreamSynchronize(gs);
+  cudaStreamDestroy(gs);
+  if (rc != KD_OK) { free_layer(L); return rc; }
+  TRYC(se);
+
+  TRYC(cudaStreamCreateWithFlags(&L->side, cudaStreamNonBlocking));
+  TRYC(cudaEventCreateWithFlags(&L->ev_h1, cudaEventDisableTiming));
+  TRYC(cudaEventCreateWithFlags(&L->ev_sh, cudaEventDisableTiming));
+  d.err = d.err;
+  *out = L;
+  return KD_OK;
+#undef TRY
+#undef TRYC
+}
+
+extern "C" void kd_layer_destroy(kd_layer* L) {
+  if (!L) return;
+  cudaDeviceSynchronize();
+  free_layer(L);
+}
+
+// ------------------------------------------------------------------ decode
+
+static int launch_layer(kd_layer* L, void* hidden, const void* attn, int M, cudaStream_t s,
+                        const kd_layer* prefetch_next, cudaStream_t pf, cudaEvent_t ev_fork,
+                        cudaEvent_t ev_join);
+
+extern "C" int kd_decode_layer(kd_layer* L, void* hidden, const void* attn, int M, void* stream) {
+  if (!L || !hidden || !attn) return fail(KD_EINVAL, "kd_decode_layer: null argument%s", "");
+  if (M < 1 || M > L->maxM)
+    return fail(KD_ERANGE, "kd_decode_layer: M=%s%ld outside 1..max_tokens", "", (long)M);
+  return launch_layer(L, hidden, attn, M, static_cast<cudaStream_t>(stream), nullptr, nullptr,
+                      nullptr, nullptr);
+}
+
+static int prefetch_static(const kd_layer* L, size_t max_bytes, cudaStream_t s);
+
+static int launch_layer(kd_layer* L, void* hidden, const void* attn, int M, cudaStream_t s,
+                        const kd_layer* next, cudaStream_t pf, cudaEvent_t ev_fork,
+                        cudaEvent_t ev_join) {
+  const LayerDev& d = L->d;
+  const bool fp8 = L->cfg.wdtype == KD_WFP8;
+  Acts a;
+  a.x = static_cast<const uint16_t*>(hidden);
+  a.attn = static_cast<const uint16_t*>(attn);
+  a.out = static_cast<uint16_t*>(hidden);
+  a.M = M;
+  const int G = L->nsm;
+  const size_t sm = kStreamSmem;
+  if (L->timing) KD_CUDA(cudaEventRecord(L->tev[0], s));
+  if (fp8) proj_kernel<W_FP8><<<G, kThreads, sm, s>>>(d, a);
+  else proj_kernel<W_BF16><<<G, kThreads, sm, s>>>(d, a);
+  KD_CUDA(cudaGetLastError());
+  if (L->timing) KD_CUDA(cudaEventRecord(L->tev[1], s));
+  if (d.S) {
+    KD_CUDA(cudaEventRecord(L->ev_h1, s));
+    KD_CUDA(cudaStreamWaitEvent(L->side, L->ev_h1, 0));
+    if (fp8) {
+      gateup_kernel<W_FP8><<<G, kThreads, sm, L->side>>>(d, M, 1);
+      down_kernel<W_FP8><<<G, kThreads, sm, L->side>>>(d, M, 1);
+    } else {
+      gateup_kernel<W_BF16><<<G, kThreads, sm, L->side>>>(d, M, 1);
+      down_kernel<W_BF16><<<G, kThreads, sm, L->side>>>(d, M, 1);
+    }
+    KD_CUDA(cudaGetLastError());
+    KD_CUDA(cudaEventRecord(L->ev_sh, L->side));
+  }
+  const int units = d.E * ((M + kRouterTok - 1) / kRouterTok);
+  const int rgrid = std::max(1, std::min((units + 7) / 8, G * 4));
+  if (fp8) router_kernel<W_FP8><<<rgrid, kRouterThreads, 0, s>>>(d, M);
+  else router_kernel<W_BF16><<<rgrid, kRouterThreads, 0, s>>>(d, M);
+  KD_CUDA(cudaGetLastError());
+  if (L->timing) KD_CUDA(cudaEventRecord(L->tev[2], s));
+  if (fp8) gateup_kernel<W_FP8><<<G, kThreads, sm, s>>>(d, M, 0);
+  else gateup_kernel<W_BF16><<<G, kThreads, sm, s>>>(d, M, 0);
+  KD_CUDA(cudaGetLastError());
+  if (L->timing) KD_CUDA(cudaEventRecord(L->tev[3], s));
+  if (fp8) down_kernel<W_FP8><<<G, kThreads, sm, s>>>(d, M, 0);
+  else down_kernel<W_BF16><<<G, kThreads, sm, s>>>(d, M, 0);
+  KD_CUDA(cudaGetLastError());
+  if (L->timing) KD_CUDA(cudaEventRecord(L->tev[4], s));
+  if (next && pf) {
+    // the next layer's static weights into L2 while this layer finishes
+    KD_CUDA(cudaEventRecord(ev_fork, s));
+    KD_CUDA(cudaStreamWaitEvent(pf, ev_fork, 0));
+    int rc = prefetch_static(next, 0, pf);
+    if (rc != KD_OK) return rc;
+    KD_CUDA(cudaEventRecord(ev_join, pf));
+  }
+  if (d.S) KD_CUDA(cudaStreamWaitEvent(s, L->ev_sh, 0));
+  const size_t n = (size_t)M * d.H;
+  const int cgrid = (int)std::min<size_t>((n + 255) / 256, (size_t)G * 8);
+  combine_kernel<<<cgrid, 256, 0, s>>>(d, a);
+  KD_CUDA(cudaGetLastError());
+  if (L->timing) KD_CUDA(cudaEventRecord(L->tev[5], s));
+  if (next && pf) KD_CUDA(cudaStreamWaitEvent(s, ev_join, 0));
+  return KD_OK;
+}
+
+extern "C" int kd_layer_check(kd_layer* L) {
+  if (!L) return fail(KD_EINVAL, "kd_layer_check: null layer%s", "");
+  KD_CUDA(cudaDeviceSynchronize());
+  unsigned e = 0;
+  KD_CUDA(cudaMemcpy(&e, L->d.err, sizeof e, cudaMemcpyDeviceToHost));
+  if (e == 0) return KD_OK;
+  KD_CUDA(cudaMemset(L->d.err, 0, sizeof(unsigned)));
+  if (e & (ERR_WAIT_FULL | ERR_WAIT_EMPTY | ERR_WAIT_MMA))
+    return fail(KD_ETIMEOUT, "device: a bounded wait gave up (flags %s0x%lx)", "", (long)e);
+  return fail(KD_EDEVICE, "device error flags %s0x%lx", "", (long)e);
+}
+
+extern "C" int kd_layer_set_timing_events(kd_layer* L, void* const* events, int n) {
+  if (!L || (n != 0 && n != KD_N_TIMING_EVENTS) || (n && !events))
+    return fail(KD_EINVAL, "kd_layer_set_timing_events: bad arguments%s", "");
+  L->timing = n != 0;
+  for (int i = 0; i < KD_N_TIMING_EVENTS; ++i)
+    L->tev[i] = n ? static_cast<cudaEvent_t>(events[i]) : nullptr;
+  return KD_OK;
+}
+
+extern "C" const void* kd_layer_qkv(const kd_layer* L) { return L ? L->d.qkv : nullptr; }
+
+// ------------------------------------------------------------------ L2 prefetch
+
+__global__ void prefetch_kernel(const uint8_t* p0, size_t n0, const uint8_t* p1, size_t n1,
+                                const uint8_t* p2, size_t n2, const uint8_t* p3, size_t n3,
+                                size_t budget) {
+  constexpr size_t kChunk = 32768;
+  const uint8_t* ps[4] = {p0, p1, p2, p3};
+  size_t ns[4] = {n0, n1, n2, n3};
+  size_t base = 0;
+  const size_t tid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const size_t nth = (size_t)gridDim.x * blockDim.x;
+  for (int r = 0; r < 4; ++r) {
+    if (!ps[r]) continue;
+    size_t n = ns[r];
+    if (base + n > budget) n = budget > base ? budget - base : 0;
+    const size_t nch = (n + kChunk - 1) / kChunk;
+    for (size_t c = tid; c < nch; c += nth) {
+      const size_t off = c * kChunk;
+      size_t len = n - off < kChunk ? n - off : kChunk;
+      len &= ~size_t(15);
+      if (len) bulk_prefetch_l2(ps[r] + off, (uint32_t)len);
+    }
+    base += ns[r];
+  }
+}
+
+static int prefetch_static(const kd_layer* L, size_t max_bytes, cudaStream_t s) {
+  const LayerDev& d = L->d;
+  const size_t budget = max_bytes ? max_bytes : L->l2_bytes;
+  const size_t bqkv = (size_t)d.Nqkv * d.H * d.eb, bo = (size_t)d.H * d.A * d.eb,
+               br = (size_t)d.E * d.H * d.eb, bsh = (size_t)2 * d.I * d.H * d.eb;
+  prefetch_kernel<<<L->nsm, 128, 0, s>>>(d.wqkv, bqkv, d.wo, bo, d.wr, br, d.wgu_sh,
+                                         d.S ? bsh : 0, budget);
+  KD_CUDA(cudaGetLastError());
+  return KD_OK;
+}
+
+extern "C" int kd_layer_prefetch_l2(const kd_layer* L, size_t max_bytes, void* stream) {
+  if (!L) return fail(KD_EINVAL, "kd_layer_prefetch_l2: null layer%s", "");
+  return prefetch_static(L, max_bytes, static_cast<cudaStream_t>(stream));
+}
+
+// ------------------------------------------------------------------ introspection
+
+extern "C" int kd_layer_debug_tensor(const kd_layer* L, int which, void** p) {
+  if (!L || !p) return fail(KD_EINVAL, "kd_layer_debug_tensor: null argument%s", "");
+  const LayerDev& d = L->d;
+  switch (which) {
+    case KD_T_H1F: *p = d.h1f; break;
+    case KD_T_H1B: *p = d.h1b; break;
+    case KD_T_LOGITS: *p = d.logits; break;
+    case KD_T_IDX: *p = d.idx; break;
+    case KD_T_GATES: *p = d.gates; break;
+    case KD_T_COUNTS: *p = d.counts; break;
+    case KD_T_NACTIVE: *p = d.n_active; break;
+    case KD_T_YSHARED: *p = d.ysh; break;
+    case KD_T_YROUTED: *p = d.yr; break;
+    default: return fail(KD_EINVAL, "kd_layer_debug_tensor: unknown tensor %s%ld", "", (long)which);
+  }
+  return KD_OK;
+}
+
+extern "C" int kd_layer_read_weight(const kd_layer* L, int kind, int expert, int row0, int nrows,
+                                    void* dst, float* dst_scales) {
+  if (!L || !dst) return fail(KD_EINVAL, "kd_layer_read_weight: null argument%s", "");
+  const LayerDev& d = L->d;
+  const int eb = d.eb;
+  const bool fp8 = eb == 1;
+  const uint8_t* base = nullptr;
+  const float* sbase = nullptr;
+  int R = 0, K = 0, mult = 1, off = 0;
+  if (expert < -1 || expert >= d.E || (expert == -1 && kind >= 4 && !d.S))
+    return fail(KD_EINVAL, "kd_layer_read_weight: bad expert %s%ld", "", (long)expert);
+  const size_t gu = (size_t)2 * d.I * d.H * eb, dn = (size_t)d.H * d.I * eb;
+  const size_t n_sgu = (size_t)2 * d.nIb * d.nHb, n_sd = (size_t)d.nHb * d.nIb;
+  switch (kind) {
+    case 1: base = d.wqkv; sbase = d.sqkv; R = d.Nqkv; K = d.H; break;
+    case 2: base = d.wo; sbase = d.so; R = d.H; K = d.A; break;
+    case 3: base = d.wr; sbase = d.sr; R = d.E; K = d.H; break;
+    case 4:
+    case 5:
+      base = expert < 0 ? d.wgu_sh : d.wgu + (size_t)expert * gu;
+      sbase = expert < 0 ? d.sgu_sh : (d.sgu ? d.sgu + (size_t)expert * n_sgu : nullptr);
+      if (sbase && kind == 5) sbase += (size_t)d.nIb * d.nHb;
+      R = d.I; K = d.H; mult = 2; off = kind == 5 ? 1 : 0;
+      break;
+    case 6:
+      base = expert < 0 ? d.wd_sh : d.wd + (size_t)expert * dn;
+      sbase = expert < 0 ? d.sd_sh : (d.sd ? d.sd + (size_t)expert * n_sd : nullptr);
+      R = d.H; K = d.I;
+      break;
+    default: return fail(KD_EINVAL, "kd_layer_read_weight: bad kind %s%ld", "", (long)kind);
+  }
+  if (row0 < 0 || nrows < 0 || row0 + nrows > R)
+    return fail(KD_EINVAL, "kd_layer_read_weight: rows out of range%s", "");
+  if (nrows == 0) return KD_OK;
+  const size_t rb = (size_t)K * eb;
+  KD_CUDA(cudaMemcpy2D(dst, rb, base + ((size_t)row0 * mult + off) * rb, rb * mult, rb, nrows,
+                       cudaMemcpyDeviceToHost));
+  if (fp8 && dst_scales) {
+    const int b0 = row0 / 128, b1 = (row0 + nrows - 1) / 128, nkb = ceil128(K);
+    KD_CUDA(cudaMemcpy(dst_scales, sbase + (size_t)b0 * nkb, sizeof(float) * (b1 - b0 + 1) * nkb,
+                       cudaMemcpyDeviceToHost));
+  }
+  return KD_OK;
+}
+
+extern "C" int kd_layer_bytes(const kd_layer* L, uint64_t* static_bytes, uint64_t* expert_bytes) {
+  if (!L) return fail(KD_EINVAL, "kd_layer_bytes: null layer%s", "");
+  if (static_bytes) *static_bytes = L->static_bytes;
+  if (expert_bytes) *expert_bytes = L->expert_bytes;
+  return KD_OK;
+}
+
+// ------------------------------------------------------------------ stack + graph
+
+extern "C" int kd_stack_create(kd_layer* const* layers, int n, int M, int prefetch, kd_stack** out) {
+  if (!layers || !out || n < 1) return fail(KD_EINVAL, "kd_stack_create: bad arguments%s", "");
+  *out = nullptr;
+  for (int i = 0; i < n; ++i) {
+    if (!layers[i]) return fail(KD_EINVAL, "kd_stack_create: null layer%s", "");
+    if (M < 1 || M > layers[i]->maxM)
+      return fail(KD_ERANGE, "kd_stack_create: M=%s%ld outside a layer's 1..max_tokens", "", (long)M);
+    if (layers[i]->d.H != layers[0]->d.H || layers[i]->d.A != layers[0]->d.A)
+      return fail(KD_EINVAL, "kd_stack_create: layers of different widths%s", "");
+  }
+  kd_stack* S = new kd_stack();
+  S->layers.assign(layers, layers + n);
+  S->M = M;
+  S->prefetch = prefetch;
+  auto bad = [&](cudaError_t e) {
+    if (S->cap) cudaStreamDestroy(S->cap);
+    if (S->pf) cudaStreamDestroy(S->pf);
+    for (auto ev : S->ev_fork) cudaEventDestroy(ev);
+    for (auto ev : S->ev_join) cudaEventDestroy(ev);
+    delete S;
+    return fail(KD_ECUDA, "kd_stack_create: %s", cudaGetErrorString(e));
+  };
+  cudaError_t e;
+  if ((e = cudaStreamCreateWithFlags(&S->cap, cudaStreamNonBlocking)) != cudaSuccess) return bad(e);
+  if ((e = cudaStreamCreateWithFlags(&S->pf, cudaStreamNonBlocking)) != cudaSuccess) return bad(e);
+  for (int i = 0; i < n; ++i) {
+    cudaEvent_t a, b;
+    if ((e = cudaEventCreateWithFlags(&a, cudaEventDisableTiming)) != cudaSuccess) return bad(e);
+    S->ev_fork.push_back(a);
+    if ((e = cudaEventCreateWithFlags(&b, cudaEventDisableTiming)) != cudaSuccess) return bad(e);
+    S->ev_join.push_back(b);
+  }
+  *out = S;
+  return KD_OK;
+}
+
+static void stack_drop_graph(kd_stack* S) {
+  if (S->exec) cudaGraphExecDestroy(S->exec);
+  if (S->graph) cudaGraphDestroy(S->graph);
+  S->exec = nullptr;
+  S->graph = nullptr;
+}
+
+extern "C" int kd_stack_run(kd_stack* S, void* hidden, const void* attn, void* stream) {
+  if (!S || !hidden || !attn) return fail(KD_EINVAL, "kd_stack_run: null argument%s", "");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (!S->exec || S->hidden != hidden || S->attn != attn) {
+    stack_drop_graph(S);
+    KD_CUDA(cudaStreamBeginCapture(S->cap, cudaStreamCaptureModeThreadLocal));
+    const int n = (int)S->layers.size();
+    int rc = KD_OK;
+    for (int l = 0; l < n && rc == KD_OK; ++l) {
+      kd_layer* L = S->layers[l];
+      const uint8_t* a = static_cast<const uint8_t*>(attn) + (size_t)l * S->M * L->d.A * 2;
+      const kd_layer* next = (S->prefetch && l + 1 < n) ? S->layers[l + 1] : nullptr;
+      rc = launch_layer(L, hidden, a, S->M, S->cap, next, next ? S->pf : nullptr, S->ev_fork[l],
+                        S->ev_join[l]);
+    }
+    cudaGraph_t g = nullptr;
+    cudaError_t ce = cudaStreamEndCapture(S->cap, &g);
+    if (rc != KD_OK) {
+      if (g) cudaGraphDestroy(g);
+      return rc;
+    }
+    KD_CUDA(ce);
+    S->graph = g;
+    KD_CUDA(cudaGraphInstantiate(&S->exec, g, 0));
+    S->hidden = hidden;
+    S->attn = attn;
+  }
+  KD_CUDA(cudaGraphLaunch(S->exec, s));
+  return KD_OK;
+}
+
+extern "C" void kd_stack_destroy(kd_stack* S) {
+  if (!S) return;
+  cudaDeviceSynchronize();
+  stack_drop_graph(S);
+  if (S->cap) cudaStreamDestroy(S->cap);
+  if (S->pf) cudaStreamDestroy(S->pf);
+  for (auto ev : S->ev_fork) cudaEventDestroy(ev);
+  for (auto ev : S->ev_join) cudaEventDestroy(ev);
+  delete S;
+}

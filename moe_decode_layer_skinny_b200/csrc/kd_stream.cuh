@@ -1,0 +1,303 @@
+// kd_stream.cuh -- weight-streaming GEMV engine on CUDA cores.
+//
+// One CTA per SM.  A producer warp streams contiguous runs of weight rows from
+// HBM into a ring of shared-memory stages with 1-D bulk TMA copies
+// (cp.async.bulk, completion counted on an mbarrier); eight consumer warps
+// take each stage as it lands, form dot products of its rows with a few token
+// activation rows (read through L1), reduce across lanes and warps in a fixed
+// order (deterministic), and hand each (row, token) sum to an epilogue.
+//
+// The work of a launch is a sequence of "segments" (a run of rows of one
+// weight matrix against one token list) that producer and consumers both
+// enumerate from the same plan object, so they agree on stage order without
+// talking to each other beyond the full / empty barriers.
+#pragma once
+
+#include "kd_common.cuh"
+
+namespace kd {
+
+constexpr int kCW = 8;                        // consumer warps
+constexpr int kThreads = (kCW + 1) * 32;      // + one producer warp
+constexpr int kStageBytes = 32768;
+constexpr int kStages = 6;
+constexpr int kTokBlk = 16;                   // tokens reduced per pass over a stage
+constexpr int kTT = 4;                        // tokens accumulated in registers at once
+constexpr int kMaxRps = 64;                   // rows per stage cap
+constexpr int kRedFloats = kMaxRps * kTokBlk; // rows x slices <= kMaxRps
+constexpr size_t kStreamSmem =
+    (size_t)kStages * kStageBytes + 2 * kRedFloats * sizeof(float) + 2 * kStages * 8 + 16 + 128;
+
+enum WType { W_BF16 = 0, W_FP8 = 1 };
+enum AType { A_BF16 = 0, A_F32 = 1 };
+
+// One run of rows.  Rows are contiguous in memory (row stride = row_bytes).
+struct Seg {
+  const uint8_t* w;     // first row
+  int row_bytes;        // bytes of one row (multiple of 256)
+  int nrows;            // rows in the run (even for paired gate/up runs)
+  int row0;             // index of the first row within its matrix (physical)
+  int tok0, ntok;       // token list range (meaning is the plan's)
+  int tag;              // plan-defined (expert id, matrix id ...)
+};
+
+struct StreamShared {
+  uint8_t* stage;       // kStages * kStageBytes
+  float* red;           // [2][kRedFloats]
+  uint64_t* full;
+  uint64_t* empty;
+  int* abort_flag;
+};
+
+KD_DEV StreamShared carve_stream_smem(uint8_t* base) {
+  StreamShared s;
+  uintptr_t p = (reinterpret_cast<uintptr_t>(base) + 127) & ~uintptr_t(127);
+  s.stage = reinterpret_cast<uint8_t*>(p);
+  p += (size_t)kStages * kStageBytes;
+  s.red = reinterpret_cast<float*>(p);
+  p += 2 * kRedFloats * sizeof(float);
+  s.full = reinterpret_cast<uint64_t*>(p);
+  s.empty = s.full + kStages;
+  s.abort_flag = reinterpret_cast<int*>(s.empty + kStages);
+  return s;
+}
+
+// Bounded wait that gives up immediately once any thread of the CTA aborted.
+KD_DEV bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                          unsigned* err, unsigned bit) {
+  if (*abort_flag) return false;
+  if (mbar_wait(bar, parity)) return true;
+  *abort_flag = 1;
+  set_error(err, bit);
+  return false;
+}
+
+// rows per stage for a row of `row_bytes` (power of two, <= kMaxRps)
+KD_DEV int rows_per_stage(int row_bytes) {
+  int r = kStageBytes / row_bytes;
+  int p = 1;
+  while (p * 2 <= r && p * 2 <= kMaxRps) p *= 2;
+  return p;
+}
+
+// ---------------------------------------------------------------- producer
+
+template <class Plan>
+KD_DEV void stream_produce(const Plan& plan, StreamShared& sh, unsigned* err) {
+  uint32_t it = 0;
+  const int nseg = plan.num_segments();
+  for (int si = 0; si < nseg; ++si) {
+    Seg s = plan.segment(si);
+    const int row_bytes = s.row_bytes;
+    const int rps = rows_per_stage(row_bytes);
+    for (int r = 0; r < s.nrows; r += rps, ++it) {
+      int n = s.nrows - r < rps ? s.nrows - r : rps;
+      int slot = it % kStages;
+      uint32_t ph = (it / kStages) & 1u;
+      wait_or_abort(&sh.empty[slot], ph ^ 1u, sh.abort_flag, err, ERR_WAIT_EMPTY);
+      uint32_t bytes = (uint32_t)n * (uint32_t)row_bytes;
+      mbar_arrive_expect_tx(&sh.full[slot], bytes);
+      bulk_g2s(sh.stage + (size_t)slot * kStageBytes, s.w + (size_t)r * row_bytes, bytes,
+               &sh.full[slot]);
+    }
+  }
+  // drain: the last stages must have been consumed before the CTA may exit
+  for (uint32_t j = it > kStages ? it - kStages : 0; j < it; ++j)
+    wait_or_abort(&sh.empty[j % kStages], (j / kStages) & 1u, sh.abort_flag, err, ERR_WAIT_EMPTY);
+}
+
+// ---------------------------------------------------------------- consumer
+
+// Accumulate dot products of weight chunk (16 bytes at `wp`) with tokens.
+template <int WT, int AT>
+KD_DEV void chunk_fma(const uint4 wv, float scale, const void* const* arow, int col, int nt,
+                      float* acc) {
+  if constexpr (WT == W_BF16) {
+    float w[8] = {bf_lo(wv.x), bf_hi(wv.x), bf_lo(wv.y), bf_hi(wv.y),
+                  bf_lo(wv.z), bf_hi(wv.z), bf_lo(wv.w), bf_hi(wv.w)};
+#pragma unroll
+    for (int t = 0; t < kTT; ++t) {
+      if (t < nt) {
+        float s = 0.f;
+        if constexpr (AT == A_BF16) {
+          uint4 a = ld_nc_v4(static_cast<const uint16_t*>(arow[t]) + col);
+          s = fmaf(w[0], bf_lo(a.x), s); s = fmaf(w[1], bf_hi(a.x), s);
+          s = fmaf(w[2], bf_lo(a.y), s); s = fmaf(w[3], bf_hi(a.y), s);
+          s = fmaf(w[4], bf_lo(a.z), s); s = fmaf(w[5], bf_hi(a.z), s);
+          s = fmaf(w[6], bf_lo(a.w), s); s = fmaf(w[7], bf_hi(a.w), s);
+        } else {
+          const float* ap = static_cast<const float*>(arow[t]) + col;
+          uint4 a0 = ld_nc_v4(ap), a1 = ld_nc_v4(ap + 4);
+          s = fmaf(w[0], __uint_as_float(a0.x), s); s = fmaf(w[1], __uint_as_float(a0.y), s);
+          s = fmaf(w[2], __uint_as_float(a0.z), s); s = fmaf(w[3], __uint_as_float(a0.w), s);
+          s = fmaf(w[4], __uint_as_float(a1.x), s); s = fmaf(w[5], __uint_as_float(a1.y), s);
+          s = fmaf(w[6], __uint_as_float(a1.z), s); s = fmaf(w[7], __uint_as_float(a1.w), s);
+        }
+        acc[t] += s;
+      }
+    }
+  } else {
+    float w[16];
+    e4m3x4_to_f32(wv.x, w[0], w[1], w[2], w[3]);
+    e4m3x4_to_f32(wv.y, w[4], w[5], w[6], w[7]);
+    e4m3x4_to_f32(wv.z, w[8], w[9], w[10], w[11]);
+    e4m3x4_to_f32(wv.w, w[12], w[13], w[14], w[15]);
+#pragma unroll
+    for (int t = 0; t < kTT; ++t) {
+      if (t < nt) {
+        float s = 0.f;
+        if constexpr (AT == A_BF16) {
+          const uint16_t* ap = static_cast<const uint16_t*>(arow[t]) + col;
+          uint4 a0 = ld_nc_v4(ap), a1 = ld_nc_v4(ap + 8);
+          s = fmaf(w[0], bf_lo(a0.x), s); s = fmaf(w[1], bf_hi(a0.x), s);
+          s = fmaf(w[2], bf_lo(a0.y), s); s = fmaf(w[3], bf_hi(a0.y), s);
+          s = fmaf(w[4], bf_lo(a0.z), s); s = fmaf(w[5], bf_hi(a0.z), s);
+          s = fmaf(w[6], bf_lo(a0.w), s); s = fmaf(w[7], bf_hi(a0.w), s);
+          s = fmaf(w[8], bf_lo(a1.x), s); s = fmaf(w[9], bf_hi(a1.x), s);
+          s = fmaf(w[10], bf_lo(a1.y), s); s = fmaf(w[11], bf_hi(a1.y), s);
+          s = fmaf(w[12], bf_lo(a1.z), s); s = fmaf(w[13], bf_hi(a1.z), s);
+          s = fmaf(w[14], bf_lo(a1.w), s); s = fmaf(w[15], bf_hi(a1.w), s);
+        } else {
+          const float* ap = static_cast<const float*>(arow[t]) + col;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint4 a = ld_nc_v4(ap + 4 * q);
+            s = fmaf(w[4 * q + 0], __uint_as_float(a.x), s);
+            s = fmaf(w[4 * q + 1], __uint_as_float(a.y), s);
+            s = fmaf(w[4 * q + 2], __uint_as_float(a.z), s);
+            s = fmaf(w[4 * q + 3], __uint_as_float(a.w), s);
+          }
+        }
+        acc[t] = fmaf(s, scale, acc[t]);
+      }
+    }
+  }
+}
+
+// Consumer side.  Plan must provide:
+//   int num_segments(), Seg segment(int)
+//   const void* act_row(const Seg&, int j)        activation row of token j of the segment
+//   const float* scale_row(const Seg&, int row)   FP8: scales of this physical row's block
+//   bool paired()                                 rows come in (gate, up) pairs
+//   void epilogue(const Seg&, int row, int j, float sum)            unpaired
+//   void epilogue2(const Seg&, int pair_row, int j, float g, float u) paired
+template <int WT, int AT, class Plan>
+KD_DEV void stream_consume(const Plan& plan, StreamShared& sh, unsigned* err) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ctid = threadIdx.x;  // 0 .. kCW*32-1
+  const int epc = WT == W_BF16 ? 8 : 16;        // elements per 16-byte chunk
+  uint32_t it = 0;
+  int rb = 0;  // reduction buffer parity
+  const int nseg = plan.num_segments();
+  for (int si = 0; si < nseg; ++si) {
+    Seg s = plan.segment(si);
+    const int row_bytes = s.row_bytes;
+    const int rps = rows_per_stage(row_bytes);
+    const int wpr = rps >= kCW ? 1 : kCW / rps;   // warps per row
+    const int rpw = rps >= kCW ? rps / kCW : 1;   // rows per warp
+    const int slices = wpr;
+    const int chunks_row = row_bytes / 16;
+    const int chunks_slice = chunks_row / wpr;
+    const int my_slice = warp % wpr;
+    const int my_row0 = (warp / wpr) * rpw;
+    for (int r0 = 0; r0 < s.nrows; r0 += rps, ++it) {
+      const int n = s.nrows - r0 < rps ? s.nrows - r0 : rps;
+      const int slot = it % kStages;
+      const uint32_t ph = (it / kStages) & 1u;
+      wait_or_abort(&sh.full[slot], ph, sh.abort_flag, err, ERR_WAIT_FULL);
+      const uint8_t* st = sh.stage + (size_t)slot * kStageBytes;
+      for (int tb = 0; tb < s.ntok; tb += kTokBlk) {
+        const int ntb = s.ntok - tb < kTokBlk ? s.ntok - tb : kTokBlk;
+        float* red = sh.red + rb * kRedFloats;
+        for (int rr = 0; rr < rpw; ++rr) {
+          const int row = my_row0 + rr;
+          if (row >= n) break;
+          const float* srow = nullptr;
+          if constexpr (WT == W_FP8) srow = plan.scale_row(s, s.row0 + r0 + row);
+          for (int tg = 0; tg < ntb; tg += kTT) {
+            const int nt = ntb - tg < kTT ? ntb - tg : kTT;
+            const void* arow[kTT];
+#pragma unroll
+            for (int t = 0; t < kTT; ++t) arow[t] = plan.act_row(s, tb + tg + (t < nt ? t : 0));
+            float acc[kTT];
+#pragma unroll
+            for (int t = 0; t < kTT; ++t) acc[t] = 0.f;
+            const uint8_t* wrow = st + (size_t)row * row_bytes;
+            for (int c = lane; c < chunks_slice; c += 32) {
+              const int ci = my_slice * chunks_slice + c;
+              const int col = ci * epc;
+              uint4 wv = lds_v4(wrow + (size_t)ci * 16);
+              float scale = 1.f;
+              if constexpr (WT == W_FP8) scale = srow[col >> 7];
+              chunk_fma<WT, AT>(wv, scale, arow, col, nt, acc);
+            }
+#pragma unroll
+            for (int t = 0; t < kTT; ++t) {
+              float v = acc[t];
+#pragma unroll
+              for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+              acc[t] = v;
+            }
+            if (lane == 0) {
+#pragma unroll
+              for (int t = 0; t < kTT; ++t)
+                if (t < nt) red[(row * slices + my_slice) * kTokBlk + tg + t] = acc[t];
+            }
+          }
+        }
+        if (tb + kTokBlk >= s.ntok) {
+          // all reads of this stage are done: release it to the producer
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sh.empty[slot]);
+        }
+        named_bar_sync(1, kCW * 32);
+        if (plan.paired()) {
+          const int npair = n >> 1;
+          for (int q = ctid; q < npair * ntb; q += kCW * 32) {
+            const int p = q / ntb, j = q % ntb;
+            float g = 0.f, u = 0.f;
+            for (int sl = 0; sl < slices; ++sl) {
+              g += red[((2 * p) * slices + sl) * kTokBlk + j];
+              u += red[((2 * p + 1) * slices + sl) * kTokBlk + j];
+            }
+            plan.epilogue2(s, (s.row0 + r0) / 2 + p, tb + j, g, u);
+          }
+        } else {
+          for (int q = ctid; q < n * ntb; q += kCW * 32) {
+            const int row = q / ntb, j = q % ntb;
+            float v = 0.f;
+            for (int sl = 0; sl < slices; ++sl) v += red[(row * slices + sl) * kTokBlk + j];
+            plan.epilogue(s, s.row0 + r0 + row, tb + j, v);
+          }
+        }
+        rb ^= 1;
+      }
+      if (s.ntok == 0) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh.empty[slot]);
+      }
+    }
+  }
+}
+
+// Shared body of every streaming kernel.
+template <int WT, int AT, class Plan>
+KD_DEV void stream_run(const Plan& plan, uint8_t* smem_raw, unsigned* err) {
+  StreamShared sh = carve_stream_smem(smem_raw);
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&sh.full[i], 1);
+      mbar_init(&sh.empty[i], kCW);
+    }
+    *sh.abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if ((threadIdx.x >> 5) == kCW) {
+    if ((threadIdx.x & 31) == 0) stream_produce(plan, sh, err);
+  } else {
+    stream_consume<WT, AT>(plan, sh, err);
+  }
+}
+
+}  // namespace kd

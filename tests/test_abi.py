@@ -1,0 +1,79 @@
+"""The C ABI library loads on a machine without a GPU, exports every symbol
+include/kd.h declares, and rejects bad arguments on the host (no device
+calls are made on these paths)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def kd():
+    from moe_decode_layer_skinny_b200 import build
+    build.build()
+    import moe_decode_layer_skinny_b200 as kd
+    kd.lib()
+    return kd
+
+
+def declared_functions():
+    src = ""
+    for f in os.listdir(os.path.join(ROOT, "include")):
+        if f.endswith(".h"):
+            src += open(os.path.join(ROOT, "include", f)).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[\w\s\*]+?\b(kd_\w+)\s*\(", src, flags=re.M)))
+
+
+def test_header_declares_the_binding_exports(kd):
+    decl = declared_functions()
+    assert "kd_decode_layer" in decl and "kd_layer_create" in decl
+    assert set(decl) == set(kd.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(kd):
+    L = ctypes.CDLL(kd.SO_PATH)
+    for name in declared_functions():
+        assert hasattr(L, name), name
+
+
+def test_host_side_argument_errors(kd):
+    L = kd.lib()
+    h = ctypes.c_void_p()
+    assert L.kd_layer_create(None, 0, ctypes.byref(h)) == kd.KD_EINVAL
+    # invalid configurations are rejected before any device call
+    bad = [dict(hidden=100), dict(top_k=0), dict(top_k=9, n_experts=8), dict(max_tokens=65),
+           dict(max_tokens=0), dict(wdtype=7), dict(n_shared=2), dict(inter=96), dict(n_experts=2000),
+           dict(hidden=32768)]
+    for b in bad:
+        f = dict(hidden=256, q_heads=4, kv_heads=1, head_dim=64, n_experts=8, top_k=2,
+                 n_shared=1, inter=128, wdtype=0, layer_id=0, max_tokens=4, router_bias=None)
+        f.update(b)
+        cfg = kd._Config(**f)
+        assert L.kd_layer_create(ctypes.byref(cfg), 0, ctypes.byref(h)) == kd.KD_EINVAL, b
+        assert kd.lib().kd_last_error().decode()
+    assert L.kd_decode_layer(None, None, None, 1, None) == kd.KD_EINVAL
+    assert L.kd_layer_check(None) == kd.KD_EINVAL
+    assert L.kd_layer_qkv(None) is None
+    assert L.kd_layer_bytes(None, None, None) == kd.KD_EINVAL
+    assert L.kd_layer_prefetch_l2(None, 0, None) == kd.KD_EINVAL
+    assert L.kd_layer_set_timing_events(None, None, 0) == kd.KD_EINVAL
+    assert L.kd_stack_create(None, 0, 1, 0, ctypes.byref(h)) == kd.KD_EINVAL
+    assert L.kd_stack_run(None, None, None, None) == kd.KD_EINVAL
+    L.kd_layer_destroy(None)
+    L.kd_stack_destroy(None)
+    assert "kd_stack_run" in kd.lib().kd_last_error().decode()
+
+
+def test_product_path_does_not_touch_the_oracle():
+    # the package and bench's GPU arm never import oracle/; only tests, smoke
+    # and the CPU-baseline leg do
+    pkg = os.path.join(ROOT, "moe_decode_layer_skinny_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                txt = open(os.path.join(dirpath, f)).read()
+                assert "import oracle" not in txt and "orc.h" not in txt, f
