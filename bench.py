@@ -263,15 +263,19 @@ def time_layer_e2e(layer, x_bits, a_bits, steps, warmup, flush, pg, local):
     return times, hx.numel() * 2 + ha.numel() * 2, hout.numel() * 2
 
 
+class _DeviceView:
+    def __init__(self, ptr: int, n: int):
+        self.__cuda_array_interface__ = {"shape": (n,), "typestr": "<i4", "data": (int(ptr), False),
+                                         "version": 3, "strides": None}
+
+
 def n_active_of(layer) -> int:
+    """Experts the last call touched (layer-owned device counter)."""
     import torch
 
     import moe_decode_layer_skinny_b200 as kd
     torch.cuda.synchronize()
-    buf = np.zeros(1, np.int32)
-    cudart = torch.cuda.cudart()
-    cudart.cudaMemcpy(buf.ctypes.data, layer.debug_ptr(kd.T_NACTIVE), 4, 2)
-    return int(buf[0])
+    return int(torch.as_tensor(_DeviceView(layer.debug_ptr(kd.T_NACTIVE), 1), device="cuda").item())
 
 
 def make_layer(w, layer_id=0):

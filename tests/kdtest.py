@@ -23,8 +23,27 @@ def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
 
 
 def rel_err(gpu: np.ndarray, ref: np.ndarray) -> float:
+    """max|gpu - ref| / rms(ref)."""
     rms = float(np.sqrt(np.mean(ref.astype(np.float64) ** 2)))
     return float(np.max(np.abs(gpu.astype(np.float64) - ref))) / max(rms, 1e-300)
+
+
+def bf16_half_ulp(x: np.ndarray) -> np.ndarray:
+    """Largest error of round-to-nearest into bf16 (8 significant bits) at x."""
+    ax = np.abs(x.astype(np.float64))
+    e = np.floor(np.log2(np.where(ax > 0, ax, 1.0)))
+    return np.where(ax > 0, np.exp2(e - 8), 0.0)
+
+
+def rel_err_bf16(gpu: np.ndarray, ref: np.ndarray) -> float:
+    """max over elements of (|gpu - ref| - half-ulp_bf16(ref))+ / rms(ref).
+
+    A bf16 result cannot be closer to the exact value than the rounding of
+    that value into bf16; this measures the error beyond that storage
+    rounding (which alone is ~1% of rms where max|x| ~ 4 rms)."""
+    rms = float(np.sqrt(np.mean(ref.astype(np.float64) ** 2)))
+    ex = np.abs(gpu.astype(np.float64) - ref) - bf16_half_ulp(ref)
+    return float(max(np.max(ex), 0.0)) / max(rms, 1e-300)
 
 
 def torch_bf16(bits: np.ndarray, device="cuda"):
@@ -37,20 +56,23 @@ def torch_bits(t) -> np.ndarray:
     return t.detach().view(torch.int16).cpu().numpy().view(np.uint16)
 
 
+class _DeviceView:
+    """A raw device pointer seen through __cuda_array_interface__."""
+
+    def __init__(self, ptr: int, shape, typestr: str):
+        self.__cuda_array_interface__ = {"shape": tuple(shape), "typestr": typestr,
+                                         "data": (int(ptr), False), "version": 3, "strides": None}
+
+
 def fetch(ptr: int, shape, dtype):
     """Copy a device buffer (raw pointer) to host numpy."""
-    import ctypes
-
     import torch
-    n = int(np.prod(shape))
-    out = np.empty(shape, dtype)
+    dtype = np.dtype(dtype)
+    code = {np.dtype(np.uint16): "<i2", np.dtype(np.int16): "<i2", np.dtype(np.float32): "<f4",
+            np.dtype(np.int32): "<i4", np.dtype(np.uint8): "|u1"}[dtype]
     torch.cuda.synchronize()
-    cudart = torch.cuda.cudart()
-    rc = cudart.cudaMemcpy(out.ctypes.data, ptr, n * out.itemsize, 2)  # DeviceToHost
-    if hasattr(rc, "value"):
-        rc = rc.value
-    assert int(rc) == 0, f"cudaMemcpy failed: {rc}"
-    return out
+    t = torch.as_tensor(_DeviceView(ptr, shape, code), device="cuda")
+    return t.cpu().numpy().view(dtype).reshape(shape).copy()
 
 
 def run_gpu_layer(layer, x_bits: np.ndarray, a_bits: np.ndarray, with_debug: bool = True) -> dict:
@@ -124,9 +146,12 @@ def compare_layer(dims, gpu: dict, x_bits, a_bits, *, wdtype=0, layer_id=0, seed
         assert report["h1"] < 1e-4, report
         assert report["logits"] < 1e-3, report
     out = bf16_to_f64(g["out"])
-    report["out"] = rel_err(out, ref["out"])
+    report["out_raw"] = rel_err(out, ref["out"])
+    report["out"] = rel_err_bf16(out, ref["out"])
     assert report["out"] <= tol, report
     if check_qkv:
-        report["qkv"] = rel_err(bf16_to_f64(g["qkv"]), ref["qkv"])
+        q = bf16_to_f64(g["qkv"])
+        report["qkv_raw"] = rel_err(q, ref["qkv"])
+        report["qkv"] = rel_err_bf16(q, ref["qkv"])
         assert report["qkv"] <= tol, report
     return report

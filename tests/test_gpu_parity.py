@@ -11,8 +11,8 @@ import pytest
 import kdgen
 import oracle
 from kdgen import K2, TINY, WORKLOADS
-from kdtest import (TOL, bf16_to_f64, compare_layer, fetch, rel_err, run_gpu_layer, torch_bf16,
-                    torch_bits)
+from kdtest import (TOL, bf16_to_f64, compare_layer, fetch, rel_err_bf16, run_gpu_layer,
+                    torch_bf16, torch_bits)
 
 pytestmark = pytest.mark.gpu
 
@@ -227,7 +227,7 @@ def test_stack4_fp8(kd):
             xl = bf16_to_f64(hs[l])[rows]
             al = bf16_to_f64(attn[l])[rows]
             ref = oracle.layer(K2, xl, al, wdtype=1, layer_id=l, want_qkv=False)
-            err = rel_err(bf16_to_f64(hs[l + 1])[rows], ref["out"])
+            err = rel_err_bf16(bf16_to_f64(hs[l + 1])[rows], ref["out"])
             assert err <= TOL[1], (l, err)
         # the graph-captured stack (with and without L2 prefetch) gives the
         # same bits as the eager sequence
