@@ -79,7 +79,7 @@ struct LayerDev {
   uint16_t* qkv; float* h1f; uint16_t* h1b;
   float* logits; int* idx; float* gates;
   int* counts; int* offsets; int* perm; int* active; int* n_active;
-  uint16_t* act; uint16_t* act_sh;         // [Mmax*k, I] by position, [Mmax, I]
+  float* act; float* act_sh;               // [Mmax*k, I] by position, [Mmax, I] (fp32)
   float* yr; float* ysh;                   // [Mmax*k, H] by token*k+slot, [Mmax, H]
   unsigned* counter;                       // router arrival counter (self-resetting)
   unsigned* err;
@@ -323,7 +323,7 @@ struct GateUpPlan {
   }
   KD_DEV const void* act_row(const Seg& s, int j) const {
     const int t = shared ? j : L->perm[s.tok0 + j] / L->k;
-    return L->h1b + (size_t)t * L->H;
+    return L->h1f + (size_t)t * L->H;
   }
   KD_DEV const float* scale_row(const Seg& s, int prow) const {
     const float* base = shared ? L->sgu_sh : L->sgu + (size_t)s.tag * 2 * L->nIb * L->nHb;
@@ -332,9 +332,8 @@ struct GateUpPlan {
   KD_DEV bool paired() const { return true; }
   KD_DEV void epilogue(const Seg&, int, int, float) const {}
   KD_DEV void epilogue2(const Seg& s, int i, int j, float g, float u) const {
-    const float v = silu(g) * u;
-    uint16_t* dst = shared ? L->act_sh + (size_t)j * L->I : L->act + (size_t)(s.tok0 + j) * L->I;
-    dst[i] = f32_to_bf16_bits(v);
+    float* dst = shared ? L->act_sh + (size_t)j * L->I : L->act + (size_t)(s.tok0 + j) * L->I;
+    dst[i] = silu(g) * u;
   }
 };
 
@@ -390,7 +389,7 @@ __global__ void __launch_bounds__(kThreads, 1) gateup_kernel(LayerDev L, int M, 
   p.L = &L; p.M = M; p.shared = shared != 0;
   const int n_act = shared ? 1 : *(volatile int*)L.n_active;
   p.R = expert_range(n_act, L.I);
-  stream_run<WT, A_BF16>(p, smem, L.err);
+  stream_run<WT, A_F32>(p, smem, L.err);
 }
 
 template <int WT>
@@ -400,7 +399,7 @@ __global__ void __launch_bounds__(kThreads, 1) down_kernel(LayerDev L, int M, in
   p.L = &L; p.M = M; p.shared = shared != 0;
   const int n_act = shared ? 1 : *(volatile int*)L.n_active;
   p.R = expert_range(n_act, L.H);
-  stream_run<WT, A_BF16>(p, smem, L.err);
+  stream_run<WT, A_F32>(p, smem, L.err);
 }
 
 // ------------------------------------------------------------------ combine

@@ -191,8 +191,9 @@ def test_batch64_zipf_parity_sampled(kd):
         assert np.allclose(g["gates"].sum(1), 1.0, atol=1e-5)
         assert all(len(set(row)) == k for row in g["idx"].tolist())
         assert g["counts"].sum() == M * k
-        assert g["counts"].max() > 20          # skewed load from the Zipf bias
-        assert g["counts"][0] == g["counts"].max() or g["counts"][:4].max() == g["counts"].max()
+        # skewed load from the Zipf bias: the hottest experts are the low ids
+        assert g["counts"].max() >= 4 * (M * k) / K2.n_experts
+        assert g["counts"][:4].max() == g["counts"].max()
         # selected logits dominate the rest, per token
         for t in range(M):
             sel = g["logits"][t, g["idx"][t]]
