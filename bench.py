@@ -206,6 +206,10 @@ def time_layer(layer, x_bits, a_bits, steps, warmup, flush, pg, local, per_kerne
     end = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     kev = [[torch.cuda.Event(enable_timing=True) for _ in range(kd.N_TIMING_EVENTS)]
            for _ in range(steps)] if per_kernel else None
+    if per_kernel:
+        for evs in kev:          # torch creates the CUDA event on its first record
+            for e in evs:
+                e.record(s)
     barrier(pg, local)
     for i in range(steps):
         hidden.copy_(x0)

@@ -167,6 +167,8 @@ class Layer:
         if not events:
             _check(lib().kd_layer_set_timing_events(self._h, None, 0))
             return
+        if any(not e.cuda_event for e in events):
+            raise ValueError("timing events must have been recorded once (torch creates them lazily)")
         arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
         _check(lib().kd_layer_set_timing_events(self._h, arr, len(events)))
 
