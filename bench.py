@@ -151,15 +151,23 @@ def to_dev_bf16(bits: np.ndarray):
 
 
 class L2Flush:
+    """Write a buffer of 2x L2, then read another one, so that the step starts
+    with no useful line in L2 and no dirty line left to write back."""
+
     def __init__(self):
         import torch
         l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
-        self.buf = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device="cuda")
+        n = max(2 * l2, 256 << 20)
+        self.buf = torch.empty(n, dtype=torch.uint8, device="cuda")
+        self.buf2 = torch.ones(n // 4, dtype=torch.float32, device="cuda")
+        self.sink = torch.empty((), dtype=torch.float32, device="cuda")
         self.n = 0
 
     def __call__(self):
+        import torch
         self.n += 1
         self.buf.fill_(self.n & 0xFF)
+        torch.amax(self.buf2, dim=0, out=self.sink)
 
 
 def layer_bytes(layer, n_active: int) -> int:

@@ -103,19 +103,14 @@ KD_DEV void set_error(unsigned* err, unsigned bit) {
 KD_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 KD_DEV void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" :::); }
 
-KD_DEV uint4 ld_nc_v4(const void* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
-  return v;
-}
+// Read-only global load (activations written by an earlier kernel; weights).
+// A plain intrinsic so the compiler may batch independent loads.
+KD_DEV uint4 ld_nc_v4(const void* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
 
-KD_DEV uint4 lds_v4(const void* p) {
-  uint4 v;
-  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(smem_u32(p)));
-  return v;
-}
+// Shared-memory load of a stage written by the bulk-copy engine.  An ordinary
+// C++ load: the "memory" clobber of the mbarrier wait that precedes it keeps
+// the compiler from hoisting it above the wait.
+KD_DEV uint4 lds_v4(const void* p) { return *reinterpret_cast<const uint4*>(p); }
 
 // bf16 pair packed in a u32 -> two fp32 (exact).
 KD_DEV float bf_lo(uint32_t u) { return __uint_as_float(u << 16); }

@@ -133,7 +133,7 @@ struct ProjPlan {
 };
 
 template <int WT>
-__global__ void __launch_bounds__(kThreads, 1) proj_kernel(LayerDev L, Acts a) {
+__global__ void __maxnreg__(224) proj_kernel(LayerDev L, Acts a) {
   extern __shared__ uint8_t smem[];
   ProjPlan p;
   p.L = &L; p.a = a;
@@ -144,54 +144,67 @@ __global__ void __launch_bounds__(kThreads, 1) proj_kernel(LayerDev L, Acts a) {
 
 // ------------------------------------------------------------------ router
 
-// Logits: one warp per (expert row, group of 8 tokens).  Then the last CTA to
-// finish selects the top-k per token (descending logit, ties -> lower id),
-// forms the renormalised softmax and builds the per-expert token lists:
+// Logits: CTA b owns expert rows 2b and 2b+1; warp w takes row 2b + w/4 and
+// the (w%4)-th quarter of its columns.  Each lane issues all of its weight
+// loads (16 bytes each, up to 8) before using any, then forms partial dot
+// products with the fp32 h1 rows of 4 tokens at a time; the four quarters are
+// added in a fixed order.  The last CTA to finish (arrival counter) selects
+// the top-k of every token (descending logit, ties -> lower id), forms the
+// softmax renormalised over the selection and builds the per-expert lists:
 //   counts[e], offsets[e] (exclusive scan), perm[pos] = token*k + slot sorted
 //   by (expert, token*k + slot), active[a] = a-th expert with tokens, n_active.
 constexpr int kRouterThreads = 256;
-constexpr int kRouterTok = 8;
+constexpr int kRouterRows = 2;
 
 template <int WT>
 __global__ void __launch_bounds__(kRouterThreads) router_kernel(LayerDev L, int M) {
+  constexpr int EPC = WT == W_BF16 ? 8 : 16;
+  constexpr int kRouterWChunks = WT == W_BF16 ? 8 : 4;  // 16-byte chunks per lane, H <= 8192
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int ngroups = (M + kRouterTok - 1) / kRouterTok;
-  const int units = L.E * ngroups;
-  const int row_bytes = L.H * L.eb;
-  const int epc = WT == W_BF16 ? 8 : 16;
-  const int nchunk = row_bytes / 16;
-  for (int u = blockIdx.x * (kRouterThreads / 32) + warp; u < units;
-       u += gridDim.x * (kRouterThreads / 32)) {
-    const int e = u / ngroups, g = u % ngroups;
-    const int t0 = g * kRouterTok, nt = M - t0 < kRouterTok ? M - t0 : kRouterTok;
-    float acc[kRouterTok];
+  const int rloc = warp >> 2, q = warp & 3;
+  const int row = blockIdx.x * kRouterRows + rloc;
+  const int cq = (L.H * L.eb / 16) / 4;   // chunks per quarter row
+  __shared__ float part[kRouterRows][4][64];
+  if (row < L.E) {
+    const uint8_t* wrow = L.wr + (size_t)row * L.H * L.eb;
+    uint4 w[kRouterWChunks];
+    float sc[kRouterWChunks];
 #pragma unroll
-    for (int t = 0; t < kRouterTok; ++t) acc[t] = 0.f;
-    const uint8_t* wrow = L.wr + (size_t)e * row_bytes;
-    const float* srow = WT == W_FP8 ? L.sr + (size_t)(e >> 7) * L.nHb : nullptr;
-    for (int c = lane; c < nchunk; c += 32) {
-      const uint4 wv = ld_nc_v4(wrow + (size_t)c * 16);
-      const int col = c * epc;
-      const void* arow[kTT];
-      for (int tq = 0; tq < nt; tq += kTT) {
-        const int ntq = nt - tq < kTT ? nt - tq : kTT;
-#pragma unroll
-        for (int t = 0; t < kTT; ++t)
-          arow[t] = L.h1f + (size_t)(t0 + tq + (t < ntq ? t : 0)) * L.H;
-        float part[kTT] = {0.f, 0.f, 0.f, 0.f};
-        chunk_fma<WT, A_F32>(wv, WT == W_FP8 ? srow[col >> 7] : 1.f, arow, col, ntq, part);
-#pragma unroll
-        for (int t = 0; t < kTT; ++t)
-          if (t < ntq) acc[tq + t] += part[t];
+    for (int i = 0; i < kRouterWChunks; ++i) {
+      const int c = lane + 32 * i;
+      if (c < cq) {
+        const int ci = q * cq + c;
+        w[i] = ld_nc_v4(wrow + (size_t)ci * 16);
+        sc[i] = WT == W_FP8 ? __ldg(L.sr + (size_t)(row >> 7) * L.nHb + ((ci * EPC) >> 7)) : 1.f;
       }
     }
+    for (int t0 = 0; t0 < M; t0 += kTT) {
+      const int nt = M - t0 < kTT ? M - t0 : kTT;
+      const void* arow[kTT];
 #pragma unroll
-    for (int t = 0; t < kRouterTok; ++t) {
-      float v = acc[t];
+      for (int t = 0; t < kTT; ++t) arow[t] = L.h1f + (size_t)(t0 + (t < nt ? t : 0)) * L.H;
+      float acc[kTT] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      if (lane == 0 && t < nt) L.logits[(size_t)(t0 + t) * L.E + e] = v + (L.bias ? L.bias[e] : 0.f);
+      for (int i = 0; i < kRouterWChunks; ++i) {
+        const int c = lane + 32 * i;
+        if (c < cq) chunk_fma<WT, A_F32>(w[i], sc[i], arow, (q * cq + c) * EPC, nt, acc);
+      }
+#pragma unroll
+      for (int t = 0; t < kTT; ++t) {
+        float v = acc[t];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == 0 && t < nt) part[rloc][q][t0 + t] = v;
+      }
     }
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < kRouterRows * M; i += kRouterThreads) {
+    const int r = i / M, t = i % M, e = blockIdx.x * kRouterRows + r;
+    if (e < L.E)
+      L.logits[(size_t)t * L.E + e] =
+          ((part[r][0][t] + part[r][1][t]) + (part[r][2][t] + part[r][3][t])) +
+          (L.bias ? L.bias[e] : 0.f);
   }
 
   // ---- last CTA: selection and dispatch
@@ -206,27 +219,29 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(LayerDev L, int 
 
   __shared__ int s_sel[64 * 16];
   __shared__ int s_cnt[1024];
-  __shared__ int s_off[1025];
+  __shared__ int s_off[1024];
+  __shared__ int s_wsum[2][kRouterThreads / 32];
   const int k = L.k, E = L.E;
   // top-k: one warp per token; lane holds logits lane, lane+32, ...
   for (int t = warp; t < M; t += kRouterThreads / 32) {
     float lv[32];
     const int per = (E + 31) / 32;
 #pragma unroll
-    for (int q = 0; q < 32; ++q) {
-      const int e = lane + 32 * q;
-      lv[q] = (q < per && e < E) ? __ldcg(L.logits + (size_t)t * E + e) : -INFINITY;
+    for (int qq = 0; qq < 32; ++qq) {
+      const int e = lane + 32 * qq;
+      lv[qq] = (qq < per && e < E) ? __ldcg(L.logits + (size_t)t * E + e) : -INFINITY;
     }
-    unsigned taken = 0u;  // bit q: lane's q-th logit already selected
-    float sel_v[16];
+    unsigned taken = 0u;
+    float top = 0.f, den = 0.f, selv[16];
     for (int j = 0; j < k; ++j) {
-      // lane-local best not yet taken: larger value, then lower expert id
-      float bv = -INFINITY; int be = 0x7fffffff;
+      float bv = -INFINITY;
+      int be = 0x7fffffff;
 #pragma unroll
-      for (int q = 0; q < 32; ++q) {
-        const int e = lane + 32 * q;
-        if (q < per && e < E && !(taken >> q & 1u) && (lv[q] > bv || (lv[q] == bv && e < be))) {
-          bv = lv[q]; be = e;
+      for (int qq = 0; qq < 32; ++qq) {
+        const int e = lane + 32 * qq;
+        if (qq < per && e < E && !((taken >> qq) & 1u) && (lv[qq] > bv || (lv[qq] == bv && e < be))) {
+          bv = lv[qq];
+          be = e;
         }
       }
 #pragma unroll
@@ -236,16 +251,16 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(LayerDev L, int 
         if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
       }
       if ((be & 31) == lane) taken |= 1u << (be >> 5);
-      sel_v[j] = bv;
+      if (j == 0) top = bv;
+      selv[j] = bv;
+      den += expf(bv - top);
       if (lane == 0) s_sel[t * k + j] = be;
     }
-    if (lane == 0) {
-      float den = 0.f;
-      for (int j = 0; j < k; ++j) den += expf(sel_v[j] - sel_v[0]);
-      for (int j = 0; j < k; ++j) {
-        L.idx[t * k + j] = s_sel[t * k + j];
-        L.gates[t * k + j] = expf(sel_v[j] - sel_v[0]) / den;
-      }
+    if (lane < k) {
+      float v = 0.f;
+      for (int j = 0; j < k; ++j) if (j == lane) v = selv[j];
+      L.idx[t * k + lane] = s_sel[t * k + lane];
+      L.gates[t * k + lane] = expf(v - top) / den;
     }
   }
   for (int e = threadIdx.x; e < E; e += kRouterThreads) s_cnt[e] = 0;
@@ -257,28 +272,59 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(LayerDev L, int 
     else atomicAdd(&s_cnt[e], 1);
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    int run = 0, na = 0;
-    for (int e = 0; e < E; ++e) {
-      s_off[e] = run;
-      run += s_cnt[e];
-      if (s_cnt[e] > 0) L.active[na++] = e;
+  // block-wide exclusive scans of counts and of (count > 0): each thread owns
+  // experts [4*tid, 4*tid+4)
+  {
+    int c4[4], a4[4], cs = 0, as = 0;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int e = 4 * threadIdx.x + u;
+      c4[u] = e < E ? s_cnt[e] : 0;
+      a4[u] = c4[u] > 0;
+      cs += c4[u];
+      as += a4[u];
     }
-    s_off[E] = run;
-    *L.n_active = na;
+    int ci = cs, ai = as;  // inclusive warp scans
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int cv = __shfl_up_sync(0xffffffffu, ci, o), av = __shfl_up_sync(0xffffffffu, ai, o);
+      if (lane >= o) { ci += cv; ai += av; }
+    }
+    if (lane == 31) { s_wsum[0][warp] = ci; s_wsum[1][warp] = ai; }
+    __syncthreads();
+    int cb = 0, ab = 0;
+    for (int w2 = 0; w2 < warp; ++w2) { cb += s_wsum[0][w2]; ab += s_wsum[1][w2]; }
+    int run = cb + ci - cs, arun = ab + ai - as;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int e = 4 * threadIdx.x + u;
+      if (e < E) {
+        s_off[e] = run;
+        L.counts[e] = c4[u];
+        L.offsets[e] = run;
+        if (a4[u]) L.active[arun] = e;
+      }
+      run += c4[u];
+      arun += a4[u];
+    }
+    if (threadIdx.x == kRouterThreads - 1) {
+      L.offsets[E] = run;
+      *L.n_active = arun;
+    }
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < E; e += kRouterThreads) {
-    L.counts[e] = s_cnt[e];
-    L.offsets[e] = s_off[e];
-  }
-  if (threadIdx.x == 0) L.offsets[E] = s_off[E];
-  for (int c = threadIdx.x; c < ncode; c += kRouterThreads) {
-    const int e = s_sel[c];
-    if (e < 0 || e >= E) continue;
-    int rank = 0;
-    for (int c2 = 0; c2 < c; ++c2) rank += (s_sel[c2] == e);
-    L.perm[s_off[e] + rank] = c;
+  // positions in (expert, code) order: one warp walks the codes 32 at a time
+  if (warp == 0) {
+    for (int c0 = 0; c0 < ncode; c0 += 32) {
+      const int c = c0 + lane;
+      const int e = c < ncode ? s_sel[c] : -1 - lane;  // unique dummies
+      const unsigned same = __match_any_sync(0xffffffffu, e);
+      const int rank = __popc(same & ((1u << lane) - 1u));
+      if (c < ncode && e >= 0 && e < E) L.perm[s_off[e] + rank] = c;
+      __syncwarp();
+      if (c < ncode && e >= 0 && e < E && rank == 0) s_off[e] += __popc(same);
+      __syncwarp();
+    }
   }
 }
 
@@ -383,7 +429,7 @@ KD_DEV ExpertRange expert_range(int n_act, int per) {
 }
 
 template <int WT>
-__global__ void __launch_bounds__(kThreads, 1) gateup_kernel(LayerDev L, int M, int shared) {
+__global__ void __maxnreg__(224) gateup_kernel(LayerDev L, int M, int shared) {
   extern __shared__ uint8_t smem[];
   GateUpPlan p;
   p.L = &L; p.M = M; p.shared = shared != 0;
@@ -393,7 +439,7 @@ __global__ void __launch_bounds__(kThreads, 1) gateup_kernel(LayerDev L, int M, 
 }
 
 template <int WT>
-__global__ void __launch_bounds__(kThreads, 1) down_kernel(LayerDev L, int M, int shared) {
+__global__ void __maxnreg__(224) down_kernel(LayerDev L, int M, int shared) {
   extern __shared__ uint8_t smem[];
   DownPlan p;
   p.L = &L; p.M = M; p.shared = shared != 0;

@@ -140,7 +140,8 @@ extern "C" int kd_layer_create(const kd_config* cfg, uint64_t seed, kd_layer** o
       c.inter % 128 || (c.wdtype != KD_WBF16 && c.wdtype != KD_WFP8) || c.max_tokens < 1 ||
       c.max_tokens > 64 || c.layer_id < 0)
     return fail(KD_EINVAL, "kd_layer_create: unsupported configuration%s", "");
-  if (c.hidden * 2 > kStageBytes || A * 2 > kStageBytes || c.inter * 2 > kStageBytes)
+  if (c.hidden * 2 > kStageBytes || A * 2 > kStageBytes || c.inter * 2 > kStageBytes ||
+      c.hidden > 8192 || A > 8192)
     return fail(KD_EINVAL, "kd_layer_create: a weight row exceeds one %s%ld-byte stage", "",
                 (long)kStageBytes);
 
@@ -330,8 +331,7 @@ static int launch_layer(kd_layer* L, void* hidden, const void* attn, int M, cuda
     KD_CUDA(cudaGetLastError());
     KD_CUDA(cudaEventRecord(L->ev_sh, L->side));
   }
-  const int units = d.E * ((M + kRouterTok - 1) / kRouterTok);
-  const int rgrid = std::max(1, std::min((units + 7) / 8, G * 4));
+  const int rgrid = (d.E + kRouterRows - 1) / kRouterRows;
   if (fp8) router_kernel<W_FP8><<<rgrid, kRouterThreads, 0, s>>>(d, M);
   else router_kernel<W_BF16><<<rgrid, kRouterThreads, 0, s>>>(d, M);
   KD_CUDA(cudaGetLastError());

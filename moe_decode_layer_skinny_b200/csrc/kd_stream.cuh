@@ -181,101 +181,253 @@ KD_DEV void chunk_fma(const uint4 wv, float scale, const void* const* arow, int 
 //   bool paired()                                 rows come in (gate, up) pairs
 //   void epilogue(const Seg&, int row, int j, float sum)            unpaired
 //   void epilogue2(const Seg&, int pair_row, int j, float g, float u) paired
+
+// Geometry of one segment as seen by one consumer warp.
+struct SegGeom {
+  int rps;            // rows per stage
+  int wpr;            // warps per row (= K slices)
+  int rpw;            // rows per warp
+  int chunks_slice;   // 16-byte chunks of one row slice
+  int my_slice, my_row0;
+};
+
+KD_DEV SegGeom seg_geom(int row_bytes, int warp) {
+  SegGeom g;
+  g.rps = rows_per_stage(row_bytes);
+  g.wpr = g.rps >= kCW ? 1 : kCW / g.rps;
+  g.rpw = g.rps >= kCW ? g.rps / kCW : 1;
+  g.chunks_slice = (row_bytes / 16) / g.wpr;
+  g.my_slice = warp % g.wpr;
+  g.my_row0 = (warp / g.wpr) * g.rpw;
+  return g;
+}
+
+// After every warp wrote its partial sums of a stage into `red`: sum the
+// slices in a fixed order and run the epilogue.
+template <class Plan>
+KD_DEV void stage_epilogue(const Plan& plan, const Seg& s, const float* red, int n, int slices,
+                           int stage_row0, int tb, int ntb) {
+  const int ctid = threadIdx.x;
+  if (plan.paired()) {
+    const int npair = n >> 1;
+    for (int q = ctid; q < npair * ntb; q += kCW * 32) {
+      const int p = q / ntb, j = q % ntb;
+      float g = 0.f, u = 0.f;
+      for (int sl = 0; sl < slices; ++sl) {
+        g += red[((2 * p) * slices + sl) * kTokBlk + j];
+        u += red[((2 * p + 1) * slices + sl) * kTokBlk + j];
+      }
+      plan.epilogue2(s, (s.row0 + stage_row0) / 2 + p, tb + j, g, u);
+    }
+  } else {
+    for (int q = ctid; q < n * ntb; q += kCW * 32) {
+      const int row = q / ntb, j = q % ntb;
+      float v = 0.f;
+      for (int sl = 0; sl < slices; ++sl) v += red[(row * slices + sl) * kTokBlk + j];
+      plan.epilogue(s, s.row0 + stage_row0 + row, tb + j, v);
+    }
+  }
+}
+
+constexpr int kMaxChunksLane = 8;   // 16-byte chunks per lane per row slice (K <= 8192 bf16)
+
+// Register path: the segment's T (<= 2) activation rows, restricted to this
+// lane's columns, live in registers for the whole segment; each stage costs
+// one 16-byte shared load per chunk and T x 8 (or 16) FMAs.
+template <int WT, int AT, int T, class Plan>
+KD_DEV void consume_segment_reg(const Plan& plan, StreamShared& sh, const Seg& s, uint32_t& it,
+                                int& rb, unsigned* err) {
+  constexpr int EPC = WT == W_BF16 ? 8 : 16;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const SegGeom g = seg_geom(s.row_bytes, warp);
+  float areg[T][kMaxChunksLane][EPC];
+#pragma unroll
+  for (int t = 0; t < T; ++t) {
+    const void* ar = plan.act_row(s, t);
+#pragma unroll
+    for (int i = 0; i < kMaxChunksLane; ++i) {
+      const int c = lane + 32 * i;
+      if (c < g.chunks_slice) {
+        const int col = (g.my_slice * g.chunks_slice + c) * EPC;
+#pragma unroll
+        for (int q = 0; q < EPC / 8; ++q) {
+          if constexpr (AT == A_BF16) {
+            const uint4 v = ld_nc_v4(static_cast<const uint16_t*>(ar) + col + 8 * q);
+            areg[t][i][8 * q + 0] = bf_lo(v.x); areg[t][i][8 * q + 1] = bf_hi(v.x);
+            areg[t][i][8 * q + 2] = bf_lo(v.y); areg[t][i][8 * q + 3] = bf_hi(v.y);
+            areg[t][i][8 * q + 4] = bf_lo(v.z); areg[t][i][8 * q + 5] = bf_hi(v.z);
+            areg[t][i][8 * q + 6] = bf_lo(v.w); areg[t][i][8 * q + 7] = bf_hi(v.w);
+          } else {
+            const float* ap = static_cast<const float*>(ar) + col + 8 * q;
+            const uint4 v0 = ld_nc_v4(ap), v1 = ld_nc_v4(ap + 4);
+            areg[t][i][8 * q + 0] = __uint_as_float(v0.x); areg[t][i][8 * q + 1] = __uint_as_float(v0.y);
+            areg[t][i][8 * q + 2] = __uint_as_float(v0.z); areg[t][i][8 * q + 3] = __uint_as_float(v0.w);
+            areg[t][i][8 * q + 4] = __uint_as_float(v1.x); areg[t][i][8 * q + 5] = __uint_as_float(v1.y);
+            areg[t][i][8 * q + 6] = __uint_as_float(v1.z); areg[t][i][8 * q + 7] = __uint_as_float(v1.w);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < EPC; ++e) areg[t][i][e] = 0.f;
+      }
+    }
+  }
+  for (int r0 = 0; r0 < s.nrows; r0 += g.rps, ++it) {
+    const int n = s.nrows - r0 < g.rps ? s.nrows - r0 : g.rps;
+    const int slot = it % kStages;
+    const uint32_t ph = (it / kStages) & 1u;
+    // FP8 block scales of this warp's rows: static weights, so they may be
+    // read before the stage's wait.
+    float sc[2][kMaxChunksLane];
+    if constexpr (WT == W_FP8) {
+#pragma unroll
+      for (int rr = 0; rr < 2; ++rr) {
+        const int row = g.my_row0 + rr;
+        const float* srow = (rr < g.rpw && row < n) ? plan.scale_row(s, s.row0 + r0 + row) : nullptr;
+#pragma unroll
+        for (int i = 0; i < kMaxChunksLane; ++i) {
+          const int c = lane + 32 * i;
+          sc[rr][i] = (srow && c < g.chunks_slice) ? __ldg(srow + (((g.my_slice * g.chunks_slice + c) * EPC) >> 7)) : 0.f;
+        }
+      }
+    }
+    wait_or_abort(&sh.full[slot], ph, sh.abort_flag, err, ERR_WAIT_FULL);
+    const uint8_t* st = sh.stage + (size_t)slot * kStageBytes;
+    float* red = sh.red + rb * kRedFloats;
+    for (int rr = 0; rr < g.rpw; ++rr) {
+      const int row = g.my_row0 + rr;
+      if (row >= n) break;
+      const uint8_t* wrow = st + (size_t)row * s.row_bytes + (size_t)g.my_slice * g.chunks_slice * 16;
+      float acc[T];
+#pragma unroll
+      for (int t = 0; t < T; ++t) acc[t] = 0.f;
+#pragma unroll
+      for (int i = 0; i < kMaxChunksLane; ++i) {
+        const int c = lane + 32 * i;
+        if (c < g.chunks_slice) {
+          const uint4 wv = lds_v4(wrow + (size_t)c * 16);
+          if constexpr (WT == W_BF16) {
+            const float w[8] = {bf_lo(wv.x), bf_hi(wv.x), bf_lo(wv.y), bf_hi(wv.y),
+                                bf_lo(wv.z), bf_hi(wv.z), bf_lo(wv.w), bf_hi(wv.w)};
+#pragma unroll
+            for (int t = 0; t < T; ++t)
+#pragma unroll
+              for (int e = 0; e < 8; ++e) acc[t] = fmaf(w[e], areg[t][i][e], acc[t]);
+          } else {
+            float w[16];
+            e4m3x4_to_f32(wv.x, w[0], w[1], w[2], w[3]);
+            e4m3x4_to_f32(wv.y, w[4], w[5], w[6], w[7]);
+            e4m3x4_to_f32(wv.z, w[8], w[9], w[10], w[11]);
+            e4m3x4_to_f32(wv.w, w[12], w[13], w[14], w[15]);
+            const float scl = rr == 0 ? sc[0][i] : sc[1][i];
+#pragma unroll
+            for (int t = 0; t < T; ++t) {
+              float p = 0.f;
+#pragma unroll
+              for (int e = 0; e < 16; ++e) p = fmaf(w[e], areg[t][i][e], p);
+              acc[t] = fmaf(p, scl, acc[t]);
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int t = 0; t < T; ++t) {
+        float v = acc[t];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == 0) red[(row * g.wpr + g.my_slice) * kTokBlk + t] = v;
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sh.empty[slot]);
+    named_bar_sync(1, kCW * 32);
+    stage_epilogue(plan, s, red, n, g.wpr, r0, 0, T);
+    rb ^= 1;
+  }
+}
+
+// General path (any token count): activations read through L1 per stage.
+template <int WT, int AT, class Plan>
+KD_DEV void consume_segment_l1(const Plan& plan, StreamShared& sh, const Seg& s, uint32_t& it,
+                               int& rb, unsigned* err) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int epc = WT == W_BF16 ? 8 : 16;
+  const SegGeom g = seg_geom(s.row_bytes, warp);
+  for (int r0 = 0; r0 < s.nrows; r0 += g.rps, ++it) {
+    const int n = s.nrows - r0 < g.rps ? s.nrows - r0 : g.rps;
+    const int slot = it % kStages;
+    const uint32_t ph = (it / kStages) & 1u;
+    wait_or_abort(&sh.full[slot], ph, sh.abort_flag, err, ERR_WAIT_FULL);
+    const uint8_t* st = sh.stage + (size_t)slot * kStageBytes;
+    for (int tb = 0; tb < s.ntok; tb += kTokBlk) {
+      const int ntb = s.ntok - tb < kTokBlk ? s.ntok - tb : kTokBlk;
+      float* red = sh.red + rb * kRedFloats;
+      for (int rr = 0; rr < g.rpw; ++rr) {
+        const int row = g.my_row0 + rr;
+        if (row >= n) break;
+        const float* srow = nullptr;
+        if constexpr (WT == W_FP8) srow = plan.scale_row(s, s.row0 + r0 + row);
+        for (int tg = 0; tg < ntb; tg += kTT) {
+          const int nt = ntb - tg < kTT ? ntb - tg : kTT;
+          const void* arow[kTT];
+#pragma unroll
+          for (int t = 0; t < kTT; ++t) arow[t] = plan.act_row(s, tb + tg + (t < nt ? t : 0));
+          float acc[kTT];
+#pragma unroll
+          for (int t = 0; t < kTT; ++t) acc[t] = 0.f;
+          const uint8_t* wrow = st + (size_t)row * s.row_bytes;
+          for (int c = lane; c < g.chunks_slice; c += 32) {
+            const int ci = g.my_slice * g.chunks_slice + c;
+            const int col = ci * epc;
+            const uint4 wv = lds_v4(wrow + (size_t)ci * 16);
+            float scale = 1.f;
+            if constexpr (WT == W_FP8) scale = srow[col >> 7];
+            chunk_fma<WT, AT>(wv, scale, arow, col, nt, acc);
+          }
+#pragma unroll
+          for (int t = 0; t < kTT; ++t) {
+            float v = acc[t];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+            acc[t] = v;
+          }
+          if (lane == 0) {
+#pragma unroll
+            for (int t = 0; t < kTT; ++t)
+              if (t < nt) red[(row * g.wpr + g.my_slice) * kTokBlk + tg + t] = acc[t];
+          }
+        }
+      }
+      if (tb + kTokBlk >= s.ntok) {
+        // all reads of this stage are done: release it to the producer
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh.empty[slot]);
+      }
+      named_bar_sync(1, kCW * 32);
+      stage_epilogue(plan, s, red, n, g.wpr, r0, tb, ntb);
+      rb ^= 1;
+    }
+    if (s.ntok == 0) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.empty[slot]);
+    }
+  }
+}
+
 template <int WT, int AT, class Plan>
 KD_DEV void stream_consume(const Plan& plan, StreamShared& sh, unsigned* err) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int ctid = threadIdx.x;  // 0 .. kCW*32-1
-  const int epc = WT == W_BF16 ? 8 : 16;        // elements per 16-byte chunk
   uint32_t it = 0;
   int rb = 0;  // reduction buffer parity
   const int nseg = plan.num_segments();
   for (int si = 0; si < nseg; ++si) {
-    Seg s = plan.segment(si);
-    const int row_bytes = s.row_bytes;
-    const int rps = rows_per_stage(row_bytes);
-    const int wpr = rps >= kCW ? 1 : kCW / rps;   // warps per row
-    const int rpw = rps >= kCW ? rps / kCW : 1;   // rows per warp
-    const int slices = wpr;
-    const int chunks_row = row_bytes / 16;
-    const int chunks_slice = chunks_row / wpr;
-    const int my_slice = warp % wpr;
-    const int my_row0 = (warp / wpr) * rpw;
-    for (int r0 = 0; r0 < s.nrows; r0 += rps, ++it) {
-      const int n = s.nrows - r0 < rps ? s.nrows - r0 : rps;
-      const int slot = it % kStages;
-      const uint32_t ph = (it / kStages) & 1u;
-      wait_or_abort(&sh.full[slot], ph, sh.abort_flag, err, ERR_WAIT_FULL);
-      const uint8_t* st = sh.stage + (size_t)slot * kStageBytes;
-      for (int tb = 0; tb < s.ntok; tb += kTokBlk) {
-        const int ntb = s.ntok - tb < kTokBlk ? s.ntok - tb : kTokBlk;
-        float* red = sh.red + rb * kRedFloats;
-        for (int rr = 0; rr < rpw; ++rr) {
-          const int row = my_row0 + rr;
-          if (row >= n) break;
-          const float* srow = nullptr;
-          if constexpr (WT == W_FP8) srow = plan.scale_row(s, s.row0 + r0 + row);
-          for (int tg = 0; tg < ntb; tg += kTT) {
-            const int nt = ntb - tg < kTT ? ntb - tg : kTT;
-            const void* arow[kTT];
-#pragma unroll
-            for (int t = 0; t < kTT; ++t) arow[t] = plan.act_row(s, tb + tg + (t < nt ? t : 0));
-            float acc[kTT];
-#pragma unroll
-            for (int t = 0; t < kTT; ++t) acc[t] = 0.f;
-            const uint8_t* wrow = st + (size_t)row * row_bytes;
-            for (int c = lane; c < chunks_slice; c += 32) {
-              const int ci = my_slice * chunks_slice + c;
-              const int col = ci * epc;
-              uint4 wv = lds_v4(wrow + (size_t)ci * 16);
-              float scale = 1.f;
-              if constexpr (WT == W_FP8) scale = srow[col >> 7];
-              chunk_fma<WT, AT>(wv, scale, arow, col, nt, acc);
-            }
-#pragma unroll
-            for (int t = 0; t < kTT; ++t) {
-              float v = acc[t];
-#pragma unroll
-              for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-              acc[t] = v;
-            }
-            if (lane == 0) {
-#pragma unroll
-              for (int t = 0; t < kTT; ++t)
-                if (t < nt) red[(row * slices + my_slice) * kTokBlk + tg + t] = acc[t];
-            }
-          }
-        }
-        if (tb + kTokBlk >= s.ntok) {
-          // all reads of this stage are done: release it to the producer
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sh.empty[slot]);
-        }
-        named_bar_sync(1, kCW * 32);
-        if (plan.paired()) {
-          const int npair = n >> 1;
-          for (int q = ctid; q < npair * ntb; q += kCW * 32) {
-            const int p = q / ntb, j = q % ntb;
-            float g = 0.f, u = 0.f;
-            for (int sl = 0; sl < slices; ++sl) {
-              g += red[((2 * p) * slices + sl) * kTokBlk + j];
-              u += red[((2 * p + 1) * slices + sl) * kTokBlk + j];
-            }
-            plan.epilogue2(s, (s.row0 + r0) / 2 + p, tb + j, g, u);
-          }
-        } else {
-          for (int q = ctid; q < n * ntb; q += kCW * 32) {
-            const int row = q / ntb, j = q % ntb;
-            float v = 0.f;
-            for (int sl = 0; sl < slices; ++sl) v += red[(row * slices + sl) * kTokBlk + j];
-            plan.epilogue(s, s.row0 + r0 + row, tb + j, v);
-          }
-        }
-        rb ^= 1;
-      }
-      if (s.ntok == 0) {
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sh.empty[slot]);
-      }
+    const Seg s = plan.segment(si);
+    const bool fits = (s.row_bytes / 16) / seg_geom(s.row_bytes, 0).wpr <= 32 * kMaxChunksLane;
+    if (fits && s.ntok == 1) {
+      consume_segment_reg<WT, AT, 1>(plan, sh, s, it, rb, err);
+    } else if (WT == W_BF16 && fits && s.ntok == 2) {
+      consume_segment_reg<WT, AT, 2>(plan, sh, s, it, rb, err);
+    } else {
+      consume_segment_l1<WT, AT>(plan, sh, s, it, rb, err);
     }
   }
 }
