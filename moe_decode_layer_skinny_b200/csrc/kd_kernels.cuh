@@ -133,7 +133,7 @@ struct ProjPlan {
 };
 
 template <int WT>
-__global__ void __maxnreg__(224) proj_kernel(LayerDev L, Acts a) {
+__global__ void __launch_bounds__(kThreads, 1) proj_kernel(LayerDev L, Acts a) {
   extern __shared__ uint8_t smem[];
   ProjPlan p;
   p.L = &L; p.a = a;
@@ -429,7 +429,7 @@ KD_DEV ExpertRange expert_range(int n_act, int per) {
 }
 
 template <int WT>
-__global__ void __maxnreg__(224) gateup_kernel(LayerDev L, int M, int shared) {
+__global__ void __launch_bounds__(kThreads, 1) gateup_kernel(LayerDev L, int M, int shared) {
   extern __shared__ uint8_t smem[];
   GateUpPlan p;
   p.L = &L; p.M = M; p.shared = shared != 0;
@@ -439,7 +439,7 @@ __global__ void __maxnreg__(224) gateup_kernel(LayerDev L, int M, int shared) {
 }
 
 template <int WT>
-__global__ void __maxnreg__(224) down_kernel(LayerDev L, int M, int shared) {
+__global__ void __launch_bounds__(kThreads, 1) down_kernel(LayerDev L, int M, int shared) {
   extern __shared__ uint8_t smem[];
   DownPlan p;
   p.L = &L; p.M = M; p.shared = shared != 0;

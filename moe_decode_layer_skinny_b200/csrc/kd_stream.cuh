@@ -1,24 +1,27 @@
 // kd_stream.cuh -- weight-streaming GEMV engine on CUDA cores.
 //
-// One CTA per SM.  A producer warp streams contiguous runs of weight rows from
+// One CTA of eight warps per SM.  Contiguous runs of weight rows stream from
 // HBM into a ring of shared-memory stages with 1-D bulk TMA copies
-// (cp.async.bulk, completion counted on an mbarrier); eight consumer warps
-// take each stage as it lands, form dot products of its rows with a few token
-// activation rows (read through L1), reduce across lanes and warps in a fixed
-// order (deterministic), and hand each (row, token) sum to an epilogue.
+// (cp.async.bulk, completion counted on one mbarrier per stage).  All eight
+// warps take each stage as it lands, form dot products of its rows with a few
+// token activation rows (kept in registers when there are one or two), reduce
+// across lanes and warps in a fixed order (deterministic), and hand each
+// (row, token) sum to an epilogue.  The named barrier that closes a stage also
+// frees its slot, and thread 0 immediately refills it with the stage
+// kStages ahead, so no producer warp or "empty" barrier is needed and each
+// thread can hold up to 255 registers.
 //
 // The work of a launch is a sequence of "segments" (a run of rows of one
-// weight matrix against one token list) that producer and consumers both
-// enumerate from the same plan object, so they agree on stage order without
-// talking to each other beyond the full / empty barriers.
+// weight matrix against one token list) that the issuing thread and the
+// consumers both enumerate from the same plan object.
 #pragma once
 
 #include "kd_common.cuh"
 
 namespace kd {
 
-constexpr int kCW = 8;                        // consumer warps
-constexpr int kThreads = (kCW + 1) * 32;      // + one producer warp
+constexpr int kCW = 8;                        // warps per CTA (all consume)
+constexpr int kThreads = kCW * 32;
 constexpr int kStageBytes = 32768;
 constexpr int kStages = 6;
 constexpr int kTokBlk = 16;                   // tokens reduced per pass over a stage
@@ -26,7 +29,7 @@ constexpr int kTT = 4;                        // tokens accumulated in registers
 constexpr int kMaxRps = 64;                   // rows per stage cap
 constexpr int kRedFloats = kMaxRps * kTokBlk; // rows x slices <= kMaxRps
 constexpr size_t kStreamSmem =
-    (size_t)kStages * kStageBytes + 2 * kRedFloats * sizeof(float) + 2 * kStages * 8 + 16 + 128;
+    (size_t)kStages * kStageBytes + 2 * kRedFloats * sizeof(float) + kStages * 8 + 16 + 128;
 
 enum WType { W_BF16 = 0, W_FP8 = 1 };
 enum AType { A_BF16 = 0, A_F32 = 1 };
@@ -44,8 +47,7 @@ struct Seg {
 struct StreamShared {
   uint8_t* stage;       // kStages * kStageBytes
   float* red;           // [2][kRedFloats]
-  uint64_t* full;
-  uint64_t* empty;
+  uint64_t* full;       // [kStages] stage landed (bulk-copy byte count)
   int* abort_flag;
 };
 
@@ -57,8 +59,7 @@ KD_DEV StreamShared carve_stream_smem(uint8_t* base) {
   s.red = reinterpret_cast<float*>(p);
   p += 2 * kRedFloats * sizeof(float);
   s.full = reinterpret_cast<uint64_t*>(p);
-  s.empty = s.full + kStages;
-  s.abort_flag = reinterpret_cast<int*>(s.empty + kStages);
+  s.abort_flag = reinterpret_cast<int*>(s.full + kStages);
   return s;
 }
 
@@ -80,31 +81,43 @@ KD_DEV int rows_per_stage(int row_bytes) {
   return p;
 }
 
-// ---------------------------------------------------------------- producer
+// ---------------------------------------------------------------- issuer
 
-template <class Plan>
-KD_DEV void stream_produce(const Plan& plan, StreamShared& sh, unsigned* err) {
-  uint32_t it = 0;
-  const int nseg = plan.num_segments();
-  for (int si = 0; si < nseg; ++si) {
-    Seg s = plan.segment(si);
-    const int row_bytes = s.row_bytes;
-    const int rps = rows_per_stage(row_bytes);
-    for (int r = 0; r < s.nrows; r += rps, ++it) {
-      int n = s.nrows - r < rps ? s.nrows - r : rps;
-      int slot = it % kStages;
-      uint32_t ph = (it / kStages) & 1u;
-      wait_or_abort(&sh.empty[slot], ph ^ 1u, sh.abort_flag, err, ERR_WAIT_EMPTY);
-      uint32_t bytes = (uint32_t)n * (uint32_t)row_bytes;
-      mbar_arrive_expect_tx(&sh.full[slot], bytes);
-      bulk_g2s(sh.stage + (size_t)slot * kStageBytes, s.w + (size_t)r * row_bytes, bytes,
-               &sh.full[slot]);
-    }
+// Thread 0's cursor over the stage sequence: (segment, first row) pairs in the
+// order the consumers take them.
+struct Issuer {
+  int si = -1, nseg = 0, r = 0, rps = 1;
+  uint32_t n = 0;       // stages issued so far
+  Seg s;
+
+  template <class Plan>
+  KD_DEV void start(const Plan& plan) {
+    nseg = plan.num_segments();
+    si = -1;
+    r = 0;
+    s.nrows = 0;
   }
-  // drain: the last stages must have been consumed before the CTA may exit
-  for (uint32_t j = it > kStages ? it - kStages : 0; j < it; ++j)
-    wait_or_abort(&sh.empty[j % kStages], (j / kStages) & 1u, sh.abort_flag, err, ERR_WAIT_EMPTY);
-}
+
+  // Issue the next stage into slot n % kStages; false when none is left.
+  template <class Plan>
+  KD_DEV bool next(const Plan& plan, StreamShared& sh) {
+    while (r >= s.nrows) {
+      if (++si >= nseg) return false;
+      s = plan.segment(si);
+      rps = rows_per_stage(s.row_bytes);
+      r = 0;
+    }
+    const int rows = s.nrows - r < rps ? s.nrows - r : rps;
+    const int slot = n % kStages;
+    const uint32_t bytes = (uint32_t)rows * (uint32_t)s.row_bytes;
+    mbar_arrive_expect_tx(&sh.full[slot], bytes);
+    bulk_g2s(sh.stage + (size_t)slot * kStageBytes, s.w + (size_t)r * s.row_bytes, bytes,
+             &sh.full[slot]);
+    r += rps;
+    ++n;
+    return true;
+  }
+};
 
 // ---------------------------------------------------------------- consumer
 
@@ -235,8 +248,8 @@ constexpr int kMaxChunksLane = 8;   // 16-byte chunks per lane per row slice (K 
 // lane's columns, live in registers for the whole segment; each stage costs
 // one 16-byte shared load per chunk and T x 8 (or 16) FMAs.
 template <int WT, int AT, int T, class Plan>
-KD_DEV void consume_segment_reg(const Plan& plan, StreamShared& sh, const Seg& s, uint32_t& it,
-                                int& rb, unsigned* err) {
+KD_DEV void consume_segment_reg(const Plan& plan, StreamShared& sh, Issuer& iss, const Seg& s,
+                                uint32_t& it, int& rb, unsigned* err) {
   constexpr int EPC = WT == W_BF16 ? 8 : 16;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const SegGeom g = seg_geom(s.row_bytes, warp);
@@ -338,9 +351,8 @@ KD_DEV void consume_segment_reg(const Plan& plan, StreamShared& sh, const Seg& s
         if (lane == 0) red[(row * g.wpr + g.my_slice) * kTokBlk + t] = v;
       }
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&sh.empty[slot]);
     named_bar_sync(1, kCW * 32);
+    if (threadIdx.x == 0) iss.next(plan, sh);   // the slot is free: refill it
     stage_epilogue(plan, s, red, n, g.wpr, r0, 0, T);
     rb ^= 1;
   }
@@ -348,8 +360,8 @@ KD_DEV void consume_segment_reg(const Plan& plan, StreamShared& sh, const Seg& s
 
 // General path (any token count): activations read through L1 per stage.
 template <int WT, int AT, class Plan>
-KD_DEV void consume_segment_l1(const Plan& plan, StreamShared& sh, const Seg& s, uint32_t& it,
-                               int& rb, unsigned* err) {
+KD_DEV void consume_segment_l1(const Plan& plan, StreamShared& sh, Issuer& iss, const Seg& s,
+                               uint32_t& it, int& rb, unsigned* err) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int epc = WT == W_BF16 ? 8 : 16;
   const SegGeom g = seg_geom(s.row_bytes, warp);
@@ -398,24 +410,21 @@ KD_DEV void consume_segment_l1(const Plan& plan, StreamShared& sh, const Seg& s,
           }
         }
       }
-      if (tb + kTokBlk >= s.ntok) {
-        // all reads of this stage are done: release it to the producer
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sh.empty[slot]);
-      }
       named_bar_sync(1, kCW * 32);
+      // after the stage's last token block no thread reads it again: refill
+      if (threadIdx.x == 0 && tb + kTokBlk >= s.ntok) iss.next(plan, sh);
       stage_epilogue(plan, s, red, n, g.wpr, r0, tb, ntb);
       rb ^= 1;
     }
     if (s.ntok == 0) {
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sh.empty[slot]);
+      named_bar_sync(1, kCW * 32);
+      if (threadIdx.x == 0) iss.next(plan, sh);
     }
   }
 }
 
 template <int WT, int AT, class Plan>
-KD_DEV void stream_consume(const Plan& plan, StreamShared& sh, unsigned* err) {
+KD_DEV void stream_consume(const Plan& plan, StreamShared& sh, Issuer& iss, unsigned* err) {
   uint32_t it = 0;
   int rb = 0;  // reduction buffer parity
   const int nseg = plan.num_segments();
@@ -423,11 +432,11 @@ KD_DEV void stream_consume(const Plan& plan, StreamShared& sh, unsigned* err) {
     const Seg s = plan.segment(si);
     const bool fits = (s.row_bytes / 16) / seg_geom(s.row_bytes, 0).wpr <= 32 * kMaxChunksLane;
     if (fits && s.ntok == 1) {
-      consume_segment_reg<WT, AT, 1>(plan, sh, s, it, rb, err);
+      consume_segment_reg<WT, AT, 1>(plan, sh, iss, s, it, rb, err);
     } else if (WT == W_BF16 && fits && s.ntok == 2) {
-      consume_segment_reg<WT, AT, 2>(plan, sh, s, it, rb, err);
+      consume_segment_reg<WT, AT, 2>(plan, sh, iss, s, it, rb, err);
     } else {
-      consume_segment_l1<WT, AT>(plan, sh, s, it, rb, err);
+      consume_segment_l1<WT, AT>(plan, sh, iss, s, it, rb, err);
     }
   }
 }
@@ -436,20 +445,17 @@ KD_DEV void stream_consume(const Plan& plan, StreamShared& sh, unsigned* err) {
 template <int WT, int AT, class Plan>
 KD_DEV void stream_run(const Plan& plan, uint8_t* smem_raw, unsigned* err) {
   StreamShared sh = carve_stream_smem(smem_raw);
+  Issuer iss;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; ++i) {
-      mbar_init(&sh.full[i], 1);
-      mbar_init(&sh.empty[i], kCW);
-    }
+    for (int i = 0; i < kStages; ++i) mbar_init(&sh.full[i], 1);
     *sh.abort_flag = 0;
     fence_mbar_init();
+    iss.start(plan);
+    for (int i = 0; i < kStages; ++i)
+      if (!iss.next(plan, sh)) break;
   }
   __syncthreads();
-  if ((threadIdx.x >> 5) == kCW) {
-    if ((threadIdx.x & 31) == 0) stream_produce(plan, sh, err);
-  } else {
-    stream_consume<WT, AT>(plan, sh, err);
-  }
+  stream_consume<WT, AT>(plan, sh, iss, err);
 }
 
 }  // namespace kd
