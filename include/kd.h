@@ -156,7 +156,7 @@ void kd_stack_destroy(kd_stack* stack);
  * calls record the caller's events (cudaEvent_t values created with timing)
  * on the call's stream at: [0] start, [1] after the QKV + o-proj kernel,
  * [2] after the router kernel, [3] after the routed gate/up kernel, [4] after
- * the routed down kernel, [5] after the final combine.  n_events == 0 turns
+ * the down kernel (routed experts + shared expert), [5] after the final combine.  n_events == 0 turns
  * it off.  The events are not owned by the layer.  Errors: KD_EINVAL. */
 #define KD_N_TIMING_EVENTS 6
 int kd_layer_set_timing_events(kd_layer* layer, void* const* events, int n_events);

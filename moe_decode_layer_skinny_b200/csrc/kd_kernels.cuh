@@ -6,7 +6,7 @@
 //   router_kernel      fp32 router logits, then (last CTA) top-k, renormalised
 //                      softmax and the per-expert token lists
 //   gateup_kernel      SwiGLU gate/up of the active experts (or the shared one)
-//   down_kernel        down projection of the active experts (or the shared one)
+//   down_kernel        down projection of the active experts and the shared one
 //   combine_kernel     h1 + shared + gate-weighted routed outputs -> bf16
 #pragma once
 
@@ -156,6 +156,39 @@ __global__ void __launch_bounds__(kThreads, 1) proj_kernel(LayerDev L, Acts a) {
 constexpr int kRouterThreads = 256;
 constexpr int kRouterRows = 2;
 
+// Accumulate one 16-byte weight chunk against up to kTT fp32 activation rows.
+template <int WT>
+KD_DEV void router_chunk(const uint4 wv, float scale, const float* const* arow, int col, int nt,
+                         float* acc) {
+  float w[16];
+  if constexpr (WT == W_BF16) {
+    w[0] = bf_lo(wv.x); w[1] = bf_hi(wv.x); w[2] = bf_lo(wv.y); w[3] = bf_hi(wv.y);
+    w[4] = bf_lo(wv.z); w[5] = bf_hi(wv.z); w[6] = bf_lo(wv.w); w[7] = bf_hi(wv.w);
+  } else {
+    e4m3x4_to_f32(wv.x, w[0], w[1], w[2], w[3]);
+    e4m3x4_to_f32(wv.y, w[4], w[5], w[6], w[7]);
+    e4m3x4_to_f32(wv.z, w[8], w[9], w[10], w[11]);
+    e4m3x4_to_f32(wv.w, w[12], w[13], w[14], w[15]);
+  }
+  constexpr int EPC = WTraits<WT>::EPC;
+#pragma unroll
+  for (int t = 0; t < kTT; ++t) {
+    if (t < nt) {
+      const float* ap = arow[t] + col;
+      float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+      for (int q = 0; q < EPC / 4; ++q) {
+        const uint4 a = ld_nc_v4(ap + 4 * q);
+        a0 = fmaf(w[4 * q + 0], __uint_as_float(a.x), a0);
+        a1 = fmaf(w[4 * q + 1], __uint_as_float(a.y), a1);
+        a0 = fmaf(w[4 * q + 2], __uint_as_float(a.z), a0);
+        a1 = fmaf(w[4 * q + 3], __uint_as_float(a.w), a1);
+      }
+      acc[t] = fmaf(a0 + a1, scale, acc[t]);
+    }
+  }
+}
+
 template <int WT>
 __global__ void __launch_bounds__(kRouterThreads) router_kernel(LayerDev L, int M) {
   constexpr int EPC = WT == W_BF16 ? 8 : 16;
@@ -180,14 +213,14 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(LayerDev L, int 
     }
     for (int t0 = 0; t0 < M; t0 += kTT) {
       const int nt = M - t0 < kTT ? M - t0 : kTT;
-      const void* arow[kTT];
+      const float* arow[kTT];
 #pragma unroll
       for (int t = 0; t < kTT; ++t) arow[t] = L.h1f + (size_t)(t0 + (t < nt ? t : 0)) * L.H;
       float acc[kTT] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int i = 0; i < kRouterWChunks; ++i) {
         const int c = lane + 32 * i;
-        if (c < cq) chunk_fma<WT, A_F32>(w[i], sc[i], arow, (q * cq + c) * EPC, nt, acc);
+        if (c < cq) router_chunk<WT>(w[i], sc[i], arow, (q * cq + c) * EPC, nt, acc);
       }
 #pragma unroll
       for (int t = 0; t < kTT; ++t) {
@@ -383,8 +416,10 @@ struct GateUpPlan {
   }
 };
 
+// Down projection of every active routed expert and (entry n_act) the shared
+// expert, in one launch.
 struct DownPlan {
-  const LayerDev* L; int M; bool shared; ExpertRange R;
+  const LayerDev* L; int M; int n_act; ExpertRange R;
   KD_DEV int num_segments() const { return R.num_segments(); }
   KD_DEV Seg segment(int i) const {
     int a, u0, u1;
@@ -392,7 +427,7 @@ struct DownPlan {
     Seg s;
     s.row_bytes = L->I * L->eb;
     const size_t estride = (size_t)L->H * s.row_bytes;
-    if (shared) {
+    if (a >= n_act) {
       s.tag = -1; s.w = L->wd_sh; s.tok0 = 0; s.ntok = M;
     } else {
       const int e = L->active[a];
@@ -405,15 +440,15 @@ struct DownPlan {
     return s;
   }
   KD_DEV const void* act_row(const Seg& s, int j) const {
-    return shared ? L->act_sh + (size_t)j * L->I : L->act + (size_t)(s.tok0 + j) * L->I;
+    return s.tag < 0 ? L->act_sh + (size_t)j * L->I : L->act + (size_t)(s.tok0 + j) * L->I;
   }
   KD_DEV const float* scale_row(const Seg& s, int row) const {
-    const float* base = shared ? L->sd_sh : L->sd + (size_t)s.tag * L->nHb * L->nIb;
+    const float* base = s.tag < 0 ? L->sd_sh : L->sd + (size_t)s.tag * L->nHb * L->nIb;
     return base + (size_t)(row >> 7) * L->nIb;
   }
   KD_DEV bool paired() const { return false; }
   KD_DEV void epilogue(const Seg& s, int h, int j, float v) const {
-    if (shared) L->ysh[(size_t)j * L->H + h] = v;
+    if (s.tag < 0) L->ysh[(size_t)j * L->H + h] = v;
     else L->yr[(size_t)L->perm[s.tok0 + j] * L->H + h] = v;
   }
   KD_DEV void epilogue2(const Seg&, int, int, float, float) const {}
@@ -439,12 +474,12 @@ __global__ void __launch_bounds__(kThreads, 1) gateup_kernel(LayerDev L, int M, 
 }
 
 template <int WT>
-__global__ void __launch_bounds__(kThreads, 1) down_kernel(LayerDev L, int M, int shared) {
+__global__ void __launch_bounds__(kThreads, 1) down_kernel(LayerDev L, int M) {
   extern __shared__ uint8_t smem[];
   DownPlan p;
-  p.L = &L; p.M = M; p.shared = shared != 0;
-  const int n_act = shared ? 1 : *(volatile int*)L.n_active;
-  p.R = expert_range(n_act, L.H);
+  p.L = &L; p.M = M;
+  p.n_act = *(volatile int*)L.n_active;
+  p.R = expert_range(p.n_act + L.S, L.H);
   stream_run<WT, A_F32>(p, smem, L.err);
 }
 

@@ -141,7 +141,7 @@ extern "C" int kd_layer_create(const kd_config* cfg, uint64_t seed, kd_layer** o
       c.max_tokens > 64 || c.layer_id < 0)
     return fail(KD_EINVAL, "kd_layer_create: unsupported configuration%s", "");
   if (c.hidden * 2 > kStageBytes || A * 2 > kStageBytes || c.inter * 2 > kStageBytes ||
-      c.hidden > 8192 || A > 8192)
+      c.hidden > 8192 || A > 8192 || c.inter > 8192)
     return fail(KD_EINVAL, "kd_layer_create: a weight row exceeds one %s%ld-byte stage", "",
                 (long)kStageBytes);
 
@@ -318,30 +318,28 @@ static int launch_layer(kd_layer* L, void* hidden, const void* attn, int M, cuda
   else proj_kernel<W_BF16><<<G, kThreads, sm, s>>>(d, a);
   KD_CUDA(cudaGetLastError());
   if (L->timing) KD_CUDA(cudaEventRecord(L->tev[1], s));
-  if (d.S) {
-    KD_CUDA(cudaEventRecord(L->ev_h1, s));
-    KD_CUDA(cudaStreamWaitEvent(L->side, L->ev_h1, 0));
-    if (fp8) {
-      gateup_kernel<W_FP8><<<G, kThreads, sm, L->side>>>(d, M, 1);
-      down_kernel<W_FP8><<<G, kThreads, sm, L->side>>>(d, M, 1);
-    } else {
-      gateup_kernel<W_BF16><<<G, kThreads, sm, L->side>>>(d, M, 1);
-      down_kernel<W_BF16><<<G, kThreads, sm, L->side>>>(d, M, 1);
-    }
-    KD_CUDA(cudaGetLastError());
-    KD_CUDA(cudaEventRecord(L->ev_sh, L->side));
-  }
+  if (d.S) KD_CUDA(cudaEventRecord(L->ev_h1, s));
+  // the router goes first so that its CTAs get SMs before the shared
+  // expert's gate/up (on the side stream) fills them
   const int rgrid = (d.E + kRouterRows - 1) / kRouterRows;
   if (fp8) router_kernel<W_FP8><<<rgrid, kRouterThreads, 0, s>>>(d, M);
   else router_kernel<W_BF16><<<rgrid, kRouterThreads, 0, s>>>(d, M);
   KD_CUDA(cudaGetLastError());
+  if (d.S) {
+    KD_CUDA(cudaStreamWaitEvent(L->side, L->ev_h1, 0));
+    if (fp8) gateup_kernel<W_FP8><<<G, kThreads, sm, L->side>>>(d, M, 1);
+    else gateup_kernel<W_BF16><<<G, kThreads, sm, L->side>>>(d, M, 1);
+    KD_CUDA(cudaGetLastError());
+    KD_CUDA(cudaEventRecord(L->ev_sh, L->side));
+  }
   if (L->timing) KD_CUDA(cudaEventRecord(L->tev[2], s));
   if (fp8) gateup_kernel<W_FP8><<<G, kThreads, sm, s>>>(d, M, 0);
   else gateup_kernel<W_BF16><<<G, kThreads, sm, s>>>(d, M, 0);
   KD_CUDA(cudaGetLastError());
   if (L->timing) KD_CUDA(cudaEventRecord(L->tev[3], s));
-  if (fp8) down_kernel<W_FP8><<<G, kThreads, sm, s>>>(d, M, 0);
-  else down_kernel<W_BF16><<<G, kThreads, sm, s>>>(d, M, 0);
+  if (d.S) KD_CUDA(cudaStreamWaitEvent(s, L->ev_sh, 0));
+  if (fp8) down_kernel<W_FP8><<<G, kThreads, sm, s>>>(d, M);
+  else down_kernel<W_BF16><<<G, kThreads, sm, s>>>(d, M);
   KD_CUDA(cudaGetLastError());
   if (L->timing) KD_CUDA(cudaEventRecord(L->tev[4], s));
   if (next && pf) {
@@ -352,7 +350,6 @@ static int launch_layer(kd_layer* L, void* hidden, const void* attn, int M, cuda
     if (rc != KD_OK) return rc;
     KD_CUDA(cudaEventRecord(ev_join, pf));
   }
-  if (d.S) KD_CUDA(cudaStreamWaitEvent(s, L->ev_sh, 0));
   const size_t n = (size_t)M * d.H;
   const int cgrid = (int)std::min<size_t>((n + 255) / 256, (size_t)G * 8);
   combine_kernel<<<cgrid, 256, 0, s>>>(d, a);

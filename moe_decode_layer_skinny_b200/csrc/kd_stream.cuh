@@ -2,14 +2,16 @@
 //
 // One CTA of eight warps per SM.  Contiguous runs of weight rows stream from
 // HBM into a ring of shared-memory stages with 1-D bulk TMA copies
-// (cp.async.bulk, completion counted on one mbarrier per stage).  All eight
-// warps take each stage as it lands, form dot products of its rows with a few
-// token activation rows (kept in registers when there are one or two), reduce
-// across lanes and warps in a fixed order (deterministic), and hand each
-// (row, token) sum to an epilogue.  The named barrier that closes a stage also
-// frees its slot, and thread 0 immediately refills it with the stage
-// kStages ahead, so no producer warp or "empty" barrier is needed and each
-// thread can hold up to 255 registers.
+// (cp.async.bulk, completion counted on one mbarrier per stage).  Each stage
+// holds several whole rows; warp w owns the w-th eighth of the columns of
+// every row, so the activation values it needs are the same for every row and
+// stay in registers for a whole segment (up to 4 tokens).  Per stage a warp
+// forms its partial dot products for all rows, reduces across lanes, and
+// writes one partial per (row, token); after the CTA barrier that closes the
+// stage the eight partials are added in a fixed order (deterministic) and
+// handed to the plan's epilogue.  The same barrier frees the stage's slot and
+// thread 0 immediately refills it with the stage kStages ahead, so there is no
+// producer warp and no "empty" barrier.
 //
 // The work of a launch is a sequence of "segments" (a run of rows of one
 // weight matrix against one token list) that the issuing thread and the
@@ -20,19 +22,25 @@
 
 namespace kd {
 
-constexpr int kCW = 8;                        // warps per CTA (all consume)
+constexpr int kCW = 8;                        // warps per CTA = column slices per row
 constexpr int kThreads = kCW * 32;
-constexpr int kStageBytes = 32768;
-constexpr int kStages = 6;
-constexpr int kTokBlk = 16;                   // tokens reduced per pass over a stage
-constexpr int kTT = 4;                        // tokens accumulated in registers at once
+constexpr int kStageBytes = 57344;            // 56 KB: 4 rows of 7168 bf16
+constexpr int kStages = 3;
 constexpr int kMaxRps = 64;                   // rows per stage cap
-constexpr int kRedFloats = kMaxRps * kTokBlk; // rows x slices <= kMaxRps
+constexpr int kTT = 4;                        // tokens per register pass
+constexpr int kRedFloats = kMaxRps * kCW * kTT;
+constexpr int kMaxChunksLane = 4;             // 16-byte chunks per lane per row (K <= 8192 bf16)
 constexpr size_t kStreamSmem =
     (size_t)kStages * kStageBytes + 2 * kRedFloats * sizeof(float) + kStages * 8 + 16 + 128;
 
 enum WType { W_BF16 = 0, W_FP8 = 1 };
 enum AType { A_BF16 = 0, A_F32 = 1 };
+
+template <int WT>
+struct WTraits {
+  static constexpr int EPC = WT == W_BF16 ? 8 : 16;   // elements per 16-byte chunk
+  static constexpr int TT = WT == W_BF16 ? 4 : 2;     // tokens held in registers at once
+};
 
 // One run of rows.  Rows are contiguous in memory (row stride = row_bytes).
 struct Seg {
@@ -73,12 +81,12 @@ KD_DEV bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_fl
   return false;
 }
 
-// rows per stage for a row of `row_bytes` (power of two, <= kMaxRps)
-KD_DEV int rows_per_stage(int row_bytes) {
+// Rows per stage for a row of `row_bytes` (even when rows come in pairs).
+KD_DEV int rows_per_stage(int row_bytes, bool paired) {
   int r = kStageBytes / row_bytes;
-  int p = 1;
-  while (p * 2 <= r && p * 2 <= kMaxRps) p *= 2;
-  return p;
+  if (r > kMaxRps) r = kMaxRps;
+  if (paired) r &= ~1;
+  return r;
 }
 
 // ---------------------------------------------------------------- issuer
@@ -104,7 +112,7 @@ struct Issuer {
     while (r >= s.nrows) {
       if (++si >= nseg) return false;
       s = plan.segment(si);
-      rps = rows_per_stage(s.row_bytes);
+      rps = rows_per_stage(s.row_bytes, plan.paired());
       r = 0;
     }
     const int rows = s.nrows - r < rps ? s.nrows - r : rps;
@@ -120,74 +128,8 @@ struct Issuer {
 };
 
 // ---------------------------------------------------------------- consumer
-
-// Accumulate dot products of weight chunk (16 bytes at `wp`) with tokens.
-template <int WT, int AT>
-KD_DEV void chunk_fma(const uint4 wv, float scale, const void* const* arow, int col, int nt,
-                      float* acc) {
-  if constexpr (WT == W_BF16) {
-    float w[8] = {bf_lo(wv.x), bf_hi(wv.x), bf_lo(wv.y), bf_hi(wv.y),
-                  bf_lo(wv.z), bf_hi(wv.z), bf_lo(wv.w), bf_hi(wv.w)};
-#pragma unroll
-    for (int t = 0; t < kTT; ++t) {
-      if (t < nt) {
-        float s = 0.f;
-        if constexpr (AT == A_BF16) {
-          uint4 a = ld_nc_v4(static_cast<const uint16_t*>(arow[t]) + col);
-          s = fmaf(w[0], bf_lo(a.x), s); s = fmaf(w[1], bf_hi(a.x), s);
-          s = fmaf(w[2], bf_lo(a.y), s); s = fmaf(w[3], bf_hi(a.y), s);
-          s = fmaf(w[4], bf_lo(a.z), s); s = fmaf(w[5], bf_hi(a.z), s);
-          s = fmaf(w[6], bf_lo(a.w), s); s = fmaf(w[7], bf_hi(a.w), s);
-        } else {
-          const float* ap = static_cast<const float*>(arow[t]) + col;
-          uint4 a0 = ld_nc_v4(ap), a1 = ld_nc_v4(ap + 4);
-          s = fmaf(w[0], __uint_as_float(a0.x), s); s = fmaf(w[1], __uint_as_float(a0.y), s);
-          s = fmaf(w[2], __uint_as_float(a0.z), s); s = fmaf(w[3], __uint_as_float(a0.w), s);
-          s = fmaf(w[4], __uint_as_float(a1.x), s); s = fmaf(w[5], __uint_as_float(a1.y), s);
-          s = fmaf(w[6], __uint_as_float(a1.z), s); s = fmaf(w[7], __uint_as_float(a1.w), s);
-        }
-        acc[t] += s;
-      }
-    }
-  } else {
-    float w[16];
-    e4m3x4_to_f32(wv.x, w[0], w[1], w[2], w[3]);
-    e4m3x4_to_f32(wv.y, w[4], w[5], w[6], w[7]);
-    e4m3x4_to_f32(wv.z, w[8], w[9], w[10], w[11]);
-    e4m3x4_to_f32(wv.w, w[12], w[13], w[14], w[15]);
-#pragma unroll
-    for (int t = 0; t < kTT; ++t) {
-      if (t < nt) {
-        float s = 0.f;
-        if constexpr (AT == A_BF16) {
-          const uint16_t* ap = static_cast<const uint16_t*>(arow[t]) + col;
-          uint4 a0 = ld_nc_v4(ap), a1 = ld_nc_v4(ap + 8);
-          s = fmaf(w[0], bf_lo(a0.x), s); s = fmaf(w[1], bf_hi(a0.x), s);
-          s = fmaf(w[2], bf_lo(a0.y), s); s = fmaf(w[3], bf_hi(a0.y), s);
-          s = fmaf(w[4], bf_lo(a0.z), s); s = fmaf(w[5], bf_hi(a0.z), s);
-          s = fmaf(w[6], bf_lo(a0.w), s); s = fmaf(w[7], bf_hi(a0.w), s);
-          s = fmaf(w[8], bf_lo(a1.x), s); s = fmaf(w[9], bf_hi(a1.x), s);
-          s = fmaf(w[10], bf_lo(a1.y), s); s = fmaf(w[11], bf_hi(a1.y), s);
-          s = fmaf(w[12], bf_lo(a1.z), s); s = fmaf(w[13], bf_hi(a1.z), s);
-          s = fmaf(w[14], bf_lo(a1.w), s); s = fmaf(w[15], bf_hi(a1.w), s);
-        } else {
-          const float* ap = static_cast<const float*>(arow[t]) + col;
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint4 a = ld_nc_v4(ap + 4 * q);
-            s = fmaf(w[4 * q + 0], __uint_as_float(a.x), s);
-            s = fmaf(w[4 * q + 1], __uint_as_float(a.y), s);
-            s = fmaf(w[4 * q + 2], __uint_as_float(a.z), s);
-            s = fmaf(w[4 * q + 3], __uint_as_float(a.w), s);
-          }
-        }
-        acc[t] = fmaf(s, scale, acc[t]);
-      }
-    }
-  }
-}
-
-// Consumer side.  Plan must provide:
+//
+// Plan must provide:
 //   int num_segments(), Seg segment(int)
 //   const void* act_row(const Seg&, int j)        activation row of token j of the segment
 //   const float* scale_row(const Seg&, int row)   FP8: scales of this physical row's block
@@ -195,73 +137,23 @@ KD_DEV void chunk_fma(const uint4 wv, float scale, const void* const* arow, int 
 //   void epilogue(const Seg&, int row, int j, float sum)            unpaired
 //   void epilogue2(const Seg&, int pair_row, int j, float g, float u) paired
 
-// Geometry of one segment as seen by one consumer warp.
-struct SegGeom {
-  int rps;            // rows per stage
-  int wpr;            // warps per row (= K slices)
-  int rpw;            // rows per warp
-  int chunks_slice;   // 16-byte chunks of one row slice
-  int my_slice, my_row0;
-};
+template <int WT>
+using ActRegs = float[WTraits<WT>::TT][kMaxChunksLane][WTraits<WT>::EPC];
 
-KD_DEV SegGeom seg_geom(int row_bytes, int warp) {
-  SegGeom g;
-  g.rps = rows_per_stage(row_bytes);
-  g.wpr = g.rps >= kCW ? 1 : kCW / g.rps;
-  g.rpw = g.rps >= kCW ? g.rps / kCW : 1;
-  g.chunks_slice = (row_bytes / 16) / g.wpr;
-  g.my_slice = warp % g.wpr;
-  g.my_row0 = (warp / g.wpr) * g.rpw;
-  return g;
-}
-
-// After every warp wrote its partial sums of a stage into `red`: sum the
-// slices in a fixed order and run the epilogue.
-template <class Plan>
-KD_DEV void stage_epilogue(const Plan& plan, const Seg& s, const float* red, int n, int slices,
-                           int stage_row0, int tb, int ntb) {
-  const int ctid = threadIdx.x;
-  if (plan.paired()) {
-    const int npair = n >> 1;
-    for (int q = ctid; q < npair * ntb; q += kCW * 32) {
-      const int p = q / ntb, j = q % ntb;
-      float g = 0.f, u = 0.f;
-      for (int sl = 0; sl < slices; ++sl) {
-        g += red[((2 * p) * slices + sl) * kTokBlk + j];
-        u += red[((2 * p + 1) * slices + sl) * kTokBlk + j];
-      }
-      plan.epilogue2(s, (s.row0 + stage_row0) / 2 + p, tb + j, g, u);
-    }
-  } else {
-    for (int q = ctid; q < n * ntb; q += kCW * 32) {
-      const int row = q / ntb, j = q % ntb;
-      float v = 0.f;
-      for (int sl = 0; sl < slices; ++sl) v += red[(row * slices + sl) * kTokBlk + j];
-      plan.epilogue(s, s.row0 + stage_row0 + row, tb + j, v);
-    }
-  }
-}
-
-constexpr int kMaxChunksLane = 8;   // 16-byte chunks per lane per row slice (K <= 8192 bf16)
-
-// Register path: the segment's T (<= 2) activation rows, restricted to this
-// lane's columns, live in registers for the whole segment; each stage costs
-// one 16-byte shared load per chunk and T x 8 (or 16) FMAs.
-template <int WT, int AT, int T, class Plan>
-KD_DEV void consume_segment_reg(const Plan& plan, StreamShared& sh, Issuer& iss, const Seg& s,
-                                uint32_t& it, int& rb, unsigned* err) {
-  constexpr int EPC = WT == W_BF16 ? 8 : 16;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const SegGeom g = seg_geom(s.row_bytes, warp);
-  float areg[T][kMaxChunksLane][EPC];
+// Activation values of `nt` tokens at this lane's columns, into registers.
+template <int WT, int AT, class Plan>
+KD_DEV void load_act_regs(const Plan& plan, const Seg& s, int tok, int nt, int slice0, int cpl,
+                          ActRegs<WT>& areg) {
+  constexpr int EPC = WTraits<WT>::EPC;
+  const int lane = threadIdx.x & 31;
 #pragma unroll
-  for (int t = 0; t < T; ++t) {
-    const void* ar = plan.act_row(s, t);
+  for (int t = 0; t < WTraits<WT>::TT; ++t) {
+    const void* ar = plan.act_row(s, tok + (t < nt ? t : 0));
 #pragma unroll
     for (int i = 0; i < kMaxChunksLane; ++i) {
       const int c = lane + 32 * i;
-      if (c < g.chunks_slice) {
-        const int col = (g.my_slice * g.chunks_slice + c) * EPC;
+      if (t < nt && c < cpl) {
+        const int col = (slice0 + c) * EPC;
 #pragma unroll
         for (int q = 0; q < EPC / 8; ++q) {
           if constexpr (AT == A_BF16) {
@@ -285,139 +177,153 @@ KD_DEV void consume_segment_reg(const Plan& plan, StreamShared& sh, Issuer& iss,
       }
     }
   }
-  for (int r0 = 0; r0 < s.nrows; r0 += g.rps, ++it) {
-    const int n = s.nrows - r0 < g.rps ? s.nrows - r0 : g.rps;
-    const int slot = it % kStages;
-    const uint32_t ph = (it / kStages) & 1u;
-    // FP8 block scales of this warp's rows: static weights, so they may be
-    // read before the stage's wait.
-    float sc[2][kMaxChunksLane];
-    if constexpr (WT == W_FP8) {
+}
+
+// Partial dot products of one row slice (this lane's chunks) with NT tokens,
+// reduced over the warp's lanes.  Independent accumulators per chunk and two
+// interleaved FMA chains per chunk keep the FMA pipe busy.
+template <int WT, int NT>
+KD_DEV void row_dot(const uint8_t* wslice, const float (&sc)[kMaxChunksLane], int cpl,
+                    const ActRegs<WT>& areg, float (&out)[kTT]) {
+  const int lane = threadIdx.x & 31;
+  float acc[kMaxChunksLane][NT];
 #pragma unroll
-      for (int rr = 0; rr < 2; ++rr) {
-        const int row = g.my_row0 + rr;
-        const float* srow = (rr < g.rpw && row < n) ? plan.scale_row(s, s.row0 + r0 + row) : nullptr;
+  for (int i = 0; i < kMaxChunksLane; ++i)
 #pragma unroll
-        for (int i = 0; i < kMaxChunksLane; ++i) {
-          const int c = lane + 32 * i;
-          sc[rr][i] = (srow && c < g.chunks_slice) ? __ldg(srow + (((g.my_slice * g.chunks_slice + c) * EPC) >> 7)) : 0.f;
+    for (int t = 0; t < NT; ++t) acc[i][t] = 0.f;
+#pragma unroll
+  for (int i = 0; i < kMaxChunksLane; ++i) {
+    const int c = lane + 32 * i;
+    if (c < cpl) {
+      const uint4 wv = lds_v4(wslice + (size_t)c * 16);
+      if constexpr (WT == W_BF16) {
+        const float w[8] = {bf_lo(wv.x), bf_hi(wv.x), bf_lo(wv.y), bf_hi(wv.y),
+                            bf_lo(wv.z), bf_hi(wv.z), bf_lo(wv.w), bf_hi(wv.w)};
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+          float a0 = w[0] * areg[t][i][0], a1 = w[1] * areg[t][i][1];
+          a0 = fmaf(w[2], areg[t][i][2], a0); a1 = fmaf(w[3], areg[t][i][3], a1);
+          a0 = fmaf(w[4], areg[t][i][4], a0); a1 = fmaf(w[5], areg[t][i][5], a1);
+          a0 = fmaf(w[6], areg[t][i][6], a0); a1 = fmaf(w[7], areg[t][i][7], a1);
+          acc[i][t] = a0 + a1;
         }
-      }
-    }
-    wait_or_abort(&sh.full[slot], ph, sh.abort_flag, err, ERR_WAIT_FULL);
-    const uint8_t* st = sh.stage + (size_t)slot * kStageBytes;
-    float* red = sh.red + rb * kRedFloats;
-    for (int rr = 0; rr < g.rpw; ++rr) {
-      const int row = g.my_row0 + rr;
-      if (row >= n) break;
-      const uint8_t* wrow = st + (size_t)row * s.row_bytes + (size_t)g.my_slice * g.chunks_slice * 16;
-      float acc[T];
+      } else {
+        float w[16];
+        e4m3x4_to_f32(wv.x, w[0], w[1], w[2], w[3]);
+        e4m3x4_to_f32(wv.y, w[4], w[5], w[6], w[7]);
+        e4m3x4_to_f32(wv.z, w[8], w[9], w[10], w[11]);
+        e4m3x4_to_f32(wv.w, w[12], w[13], w[14], w[15]);
 #pragma unroll
-      for (int t = 0; t < T; ++t) acc[t] = 0.f;
+        for (int t = 0; t < NT; ++t) {
+          float a0 = w[0] * areg[t][i][0], a1 = w[1] * areg[t][i][1];
 #pragma unroll
-      for (int i = 0; i < kMaxChunksLane; ++i) {
-        const int c = lane + 32 * i;
-        if (c < g.chunks_slice) {
-          const uint4 wv = lds_v4(wrow + (size_t)c * 16);
-          if constexpr (WT == W_BF16) {
-            const float w[8] = {bf_lo(wv.x), bf_hi(wv.x), bf_lo(wv.y), bf_hi(wv.y),
-                                bf_lo(wv.z), bf_hi(wv.z), bf_lo(wv.w), bf_hi(wv.w)};
-#pragma unroll
-            for (int t = 0; t < T; ++t)
-#pragma unroll
-              for (int e = 0; e < 8; ++e) acc[t] = fmaf(w[e], areg[t][i][e], acc[t]);
-          } else {
-            float w[16];
-            e4m3x4_to_f32(wv.x, w[0], w[1], w[2], w[3]);
-            e4m3x4_to_f32(wv.y, w[4], w[5], w[6], w[7]);
-            e4m3x4_to_f32(wv.z, w[8], w[9], w[10], w[11]);
-            e4m3x4_to_f32(wv.w, w[12], w[13], w[14], w[15]);
-            const float scl = rr == 0 ? sc[0][i] : sc[1][i];
-#pragma unroll
-            for (int t = 0; t < T; ++t) {
-              float p = 0.f;
-#pragma unroll
-              for (int e = 0; e < 16; ++e) p = fmaf(w[e], areg[t][i][e], p);
-              acc[t] = fmaf(p, scl, acc[t]);
-            }
+          for (int e = 2; e < 16; e += 2) {
+            a0 = fmaf(w[e], areg[t][i][e], a0);
+            a1 = fmaf(w[e + 1], areg[t][i][e + 1], a1);
           }
+          acc[i][t] = (a0 + a1) * sc[i];
         }
       }
-#pragma unroll
-      for (int t = 0; t < T; ++t) {
-        float v = acc[t];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if (lane == 0) red[(row * g.wpr + g.my_slice) * kTokBlk + t] = v;
-      }
     }
-    named_bar_sync(1, kCW * 32);
-    if (threadIdx.x == 0) iss.next(plan, sh);   // the slot is free: refill it
-    stage_epilogue(plan, s, red, n, g.wpr, r0, 0, T);
-    rb ^= 1;
+  }
+#pragma unroll
+  for (int t = 0; t < NT; ++t) {
+    float v = acc[0][t];
+#pragma unroll
+    for (int i = 1; i < kMaxChunksLane; ++i) v += acc[i][t];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    out[t] = v;
   }
 }
 
-// General path (any token count): activations read through L1 per stage.
+// After every warp wrote its partials of a stage into `red` ([row][slice][t]):
+// sum the slices in a fixed order and run the epilogue.
+template <class Plan>
+KD_DEV void stage_epilogue(const Plan& plan, const Seg& s, const float* red, int n, int stage_row0,
+                           int tok, int nt) {
+  const int ctid = threadIdx.x;
+  if (plan.paired()) {
+    const int npair = n >> 1;
+    for (int q = ctid; q < npair * nt; q += kThreads) {
+      const int p = q / nt, j = q % nt;
+      float g = 0.f, u = 0.f;
+#pragma unroll
+      for (int sl = 0; sl < kCW; ++sl) {
+        g += red[((2 * p) * kCW + sl) * kTT + j];
+        u += red[((2 * p + 1) * kCW + sl) * kTT + j];
+      }
+      plan.epilogue2(s, (s.row0 + stage_row0) / 2 + p, tok + j, g, u);
+    }
+  } else {
+    for (int q = ctid; q < n * nt; q += kThreads) {
+      const int row = q / nt, j = q % nt;
+      float v = 0.f;
+#pragma unroll
+      for (int sl = 0; sl < kCW; ++sl) v += red[(row * kCW + sl) * kTT + j];
+      plan.epilogue(s, s.row0 + stage_row0 + row, tok + j, v);
+    }
+  }
+}
+
+// One segment.  Tokens are processed TT at a time (4 for bf16 weights, 2 for
+// FP8): with at most TT tokens (the common case) their activations are loaded
+// once for the whole segment; with more, the stage is swept once per group of
+// TT tokens, reloading the activations (through L1) for every group.
 template <int WT, int AT, class Plan>
-KD_DEV void consume_segment_l1(const Plan& plan, StreamShared& sh, Issuer& iss, const Seg& s,
-                               uint32_t& it, int& rb, unsigned* err) {
+KD_DEV void consume_segment(const Plan& plan, StreamShared& sh, Issuer& iss, const Seg& s,
+                            uint32_t& it, int& rb, unsigned* err) {
+  constexpr int EPC = WTraits<WT>::EPC;
+  constexpr int TT = WTraits<WT>::TT;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int epc = WT == W_BF16 ? 8 : 16;
-  const SegGeom g = seg_geom(s.row_bytes, warp);
-  for (int r0 = 0; r0 < s.nrows; r0 += g.rps, ++it) {
-    const int n = s.nrows - r0 < g.rps ? s.nrows - r0 : g.rps;
+  const int rps = rows_per_stage(s.row_bytes, plan.paired());
+  const int cpl = (s.row_bytes / 16) / kCW;       // chunks per slice (<= 32*kMaxChunksLane)
+  const int slice0 = warp * cpl;
+  ActRegs<WT> areg;
+  const bool single_pass = s.ntok <= TT;
+  if (single_pass) load_act_regs<WT, AT>(plan, s, 0, s.ntok, slice0, cpl, areg);
+  for (int r0 = 0; r0 < s.nrows; r0 += rps, ++it) {
+    const int n = s.nrows - r0 < rps ? s.nrows - r0 : rps;
     const int slot = it % kStages;
     const uint32_t ph = (it / kStages) & 1u;
     wait_or_abort(&sh.full[slot], ph, sh.abort_flag, err, ERR_WAIT_FULL);
-    const uint8_t* st = sh.stage + (size_t)slot * kStageBytes;
-    for (int tb = 0; tb < s.ntok; tb += kTokBlk) {
-      const int ntb = s.ntok - tb < kTokBlk ? s.ntok - tb : kTokBlk;
+    const uint8_t* st = sh.stage + (size_t)slot * kStageBytes + (size_t)slice0 * 16;
+    for (int tok = 0; tok < s.ntok; tok += TT) {
+      const int nt = s.ntok - tok < TT ? s.ntok - tok : TT;
+      if (!single_pass) load_act_regs<WT, AT>(plan, s, tok, nt, slice0, cpl, areg);
       float* red = sh.red + rb * kRedFloats;
-      for (int rr = 0; rr < g.rpw; ++rr) {
-        const int row = g.my_row0 + rr;
-        if (row >= n) break;
-        const float* srow = nullptr;
-        if constexpr (WT == W_FP8) srow = plan.scale_row(s, s.row0 + r0 + row);
-        for (int tg = 0; tg < ntb; tg += kTT) {
-          const int nt = ntb - tg < kTT ? ntb - tg : kTT;
-          const void* arow[kTT];
+      for (int row = 0; row < n; ++row) {
+        // FP8 block scales of this row at this lane's chunks (static weights)
+        float sc[kMaxChunksLane];
 #pragma unroll
-          for (int t = 0; t < kTT; ++t) arow[t] = plan.act_row(s, tb + tg + (t < nt ? t : 0));
-          float acc[kTT];
+        for (int i = 0; i < kMaxChunksLane; ++i) sc[i] = 1.f;
+        if constexpr (WT == W_FP8) {
+          const float* srow = plan.scale_row(s, s.row0 + r0 + row);
 #pragma unroll
-          for (int t = 0; t < kTT; ++t) acc[t] = 0.f;
-          const uint8_t* wrow = st + (size_t)row * s.row_bytes;
-          for (int c = lane; c < g.chunks_slice; c += 32) {
-            const int ci = g.my_slice * g.chunks_slice + c;
-            const int col = ci * epc;
-            const uint4 wv = lds_v4(wrow + (size_t)ci * 16);
-            float scale = 1.f;
-            if constexpr (WT == W_FP8) scale = srow[col >> 7];
-            chunk_fma<WT, AT>(wv, scale, arow, col, nt, acc);
-          }
-#pragma unroll
-          for (int t = 0; t < kTT; ++t) {
-            float v = acc[t];
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-            acc[t] = v;
-          }
-          if (lane == 0) {
-#pragma unroll
-            for (int t = 0; t < kTT; ++t)
-              if (t < nt) red[(row * g.wpr + g.my_slice) * kTokBlk + tg + t] = acc[t];
+          for (int i = 0; i < kMaxChunksLane; ++i) {
+            const int c = lane + 32 * i;
+            sc[i] = c < cpl ? __ldg(srow + (((slice0 + c) * EPC) >> 7)) : 0.f;
           }
         }
+        float part[kTT];
+        const uint8_t* wrow = st + (size_t)row * s.row_bytes;
+        if (nt == 1) row_dot<WT, 1>(wrow, sc, cpl, areg, part);
+        else if (TT == 2 || nt == 2) row_dot<WT, 2>(wrow, sc, cpl, areg, part);
+        else row_dot<WT, TT>(wrow, sc, cpl, areg, part);
+        if (lane == 0) {
+#pragma unroll
+          for (int t = 0; t < kTT; ++t)
+            if (t < nt) red[(row * kCW + warp) * kTT + t] = part[t];
+        }
       }
-      named_bar_sync(1, kCW * 32);
-      // after the stage's last token block no thread reads it again: refill
-      if (threadIdx.x == 0 && tb + kTokBlk >= s.ntok) iss.next(plan, sh);
-      stage_epilogue(plan, s, red, n, g.wpr, r0, tb, ntb);
+      named_bar_sync(1, kThreads);
+      // after the stage's last token group no thread reads it again: refill
+      if (threadIdx.x == 0 && tok + TT >= s.ntok) iss.next(plan, sh);
+      stage_epilogue(plan, s, red, n, r0, tok, nt);
       rb ^= 1;
     }
     if (s.ntok == 0) {
-      named_bar_sync(1, kCW * 32);
+      named_bar_sync(1, kThreads);
       if (threadIdx.x == 0) iss.next(plan, sh);
     }
   }
@@ -430,14 +336,7 @@ KD_DEV void stream_consume(const Plan& plan, StreamShared& sh, Issuer& iss, unsi
   const int nseg = plan.num_segments();
   for (int si = 0; si < nseg; ++si) {
     const Seg s = plan.segment(si);
-    const bool fits = (s.row_bytes / 16) / seg_geom(s.row_bytes, 0).wpr <= 32 * kMaxChunksLane;
-    if (fits && s.ntok == 1) {
-      consume_segment_reg<WT, AT, 1>(plan, sh, iss, s, it, rb, err);
-    } else if (WT == W_BF16 && fits && s.ntok == 2) {
-      consume_segment_reg<WT, AT, 2>(plan, sh, iss, s, it, rb, err);
-    } else {
-      consume_segment_l1<WT, AT>(plan, sh, iss, s, it, rb, err);
-    }
+    consume_segment<WT, AT>(plan, sh, iss, s, it, rb, err);
   }
 }
 
