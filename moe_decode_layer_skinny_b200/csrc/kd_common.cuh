@@ -135,4 +135,29 @@ KD_DEV uint16_t f32_to_bf16_bits(float f) {
 
 KD_DEV float silu(float z) { return z / (1.0f + expf(-z)); }
 
+// Two fp32 values in one 64-bit register, for the packed fp32 FMA of sm_100
+// (fma.rn.f32x2: two IEEE fp32 FMAs per instruction).
+typedef unsigned long long f32x2;
+
+KD_DEV f32x2 pack2(float lo, float hi) {
+  f32x2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+
+KD_DEV float2 unpack2(f32x2 v) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+  return r;
+}
+
+KD_DEV f32x2 ffma2(f32x2 a, f32x2 b, f32x2 c) {
+  f32x2 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
+// bf16 pair (u32) -> packed fp32 pair (exact).
+KD_DEV f32x2 bf2_to_f2(uint32_t u) { return pack2(bf_lo(u), bf_hi(u)); }
+
 }  // namespace kd

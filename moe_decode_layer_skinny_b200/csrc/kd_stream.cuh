@@ -3,13 +3,13 @@
 // One CTA of eight warps per SM.  Contiguous runs of weight rows stream from
 // HBM into a ring of shared-memory stages with 1-D bulk TMA copies
 // (cp.async.bulk, completion counted on one mbarrier per stage).  Each stage
-// holds several whole rows; warp w owns the w-th eighth of the columns of
-// every row, so the activation values it needs are the same for every row and
-// stay in registers for a whole segment (up to 4 tokens).  Per stage a warp
-// forms its partial dot products for all rows, reduces across lanes, and
-// writes one partial per (row, token); after the CTA barrier that closes the
-// stage the eight partials are added in a fixed order (deterministic) and
-// handed to the plan's epilogue.  The same barrier frees the stage's slot and
+// holds several whole rows; a warp owns one column slice of a subset of them,
+// so the activation values it needs are the same for every row and stay in
+// registers for a whole segment (up to 4 tokens), and the products use the
+// packed fp32 FMA (two IEEE fp32 FMAs per instruction).  Per stage a warp
+// writes one lane-reduced partial per (row, slice, token); after the CTA
+// barrier that closes the stage the slices are added in a fixed order
+// (deterministic) and handed to the plan's epilogue.  The same barrier frees the stage's slot and
 // thread 0 immediately refills it with the stage kStages ahead, so there is no
 // producer warp and no "empty" barrier.
 //
@@ -28,7 +28,7 @@ constexpr int kStageBytes = 57344;            // 56 KB: 4 rows of 7168 bf16
 constexpr int kStages = 3;
 constexpr int kMaxRps = 64;                   // rows per stage cap
 constexpr int kTT = 4;                        // tokens per register pass
-constexpr int kRedFloats = kMaxRps * kCW * kTT;
+constexpr int kRedFloats = kMaxRps * kCW * kTT;   // [row][slice][token], S*rows <= 8*rps
 constexpr int kMaxChunksLane = 4;             // 16-byte chunks per lane per row (K <= 8192 bf16)
 constexpr size_t kStreamSmem =
     (size_t)kStages * kStageBytes + 2 * kRedFloats * sizeof(float) + kStages * 8 + 16 + 128;
@@ -136,9 +136,23 @@ struct Issuer {
 //   bool paired()                                 rows come in (gate, up) pairs
 //   void epilogue(const Seg&, int row, int j, float sum)            unpaired
 //   void epilogue2(const Seg&, int pair_row, int j, float g, float u) paired
+//
+// Geometry of a segment: each row is cut into S column slices (the smallest
+// power of two that leaves <= 32*kMaxChunksLane 16-byte chunks per slice);
+// warp w takes slice w % S of rows w / S, w / S + G, ... (G = 8 / S row
+// groups).  A warp handles its rows four at a time and reduces the four
+// partial sums across its lanes together (a transposing butterfly: 6 shuffles
+// instead of 20).
+
+KD_DEV int slices_per_row(int row_bytes) {
+  const int chunks = row_bytes / 16;
+  int S = 1;
+  while (S < kCW && chunks / S > 32 * kMaxChunksLane) S *= 2;
+  return S;
+}
 
 template <int WT>
-using ActRegs = float[WTraits<WT>::TT][kMaxChunksLane][WTraits<WT>::EPC];
+using ActRegs = f32x2[WTraits<WT>::TT][kMaxChunksLane][WTraits<WT>::EPC / 2];
 
 // Activation values of `nt` tokens at this lane's columns, into registers.
 template <int WT, int AT, class Plan>
@@ -158,100 +172,127 @@ KD_DEV void load_act_regs(const Plan& plan, const Seg& s, int tok, int nt, int s
         for (int q = 0; q < EPC / 8; ++q) {
           if constexpr (AT == A_BF16) {
             const uint4 v = ld_nc_v4(static_cast<const uint16_t*>(ar) + col + 8 * q);
-            areg[t][i][8 * q + 0] = bf_lo(v.x); areg[t][i][8 * q + 1] = bf_hi(v.x);
-            areg[t][i][8 * q + 2] = bf_lo(v.y); areg[t][i][8 * q + 3] = bf_hi(v.y);
-            areg[t][i][8 * q + 4] = bf_lo(v.z); areg[t][i][8 * q + 5] = bf_hi(v.z);
-            areg[t][i][8 * q + 6] = bf_lo(v.w); areg[t][i][8 * q + 7] = bf_hi(v.w);
+            areg[t][i][4 * q + 0] = bf2_to_f2(v.x);
+            areg[t][i][4 * q + 1] = bf2_to_f2(v.y);
+            areg[t][i][4 * q + 2] = bf2_to_f2(v.z);
+            areg[t][i][4 * q + 3] = bf2_to_f2(v.w);
           } else {
             const float* ap = static_cast<const float*>(ar) + col + 8 * q;
             const uint4 v0 = ld_nc_v4(ap), v1 = ld_nc_v4(ap + 4);
-            areg[t][i][8 * q + 0] = __uint_as_float(v0.x); areg[t][i][8 * q + 1] = __uint_as_float(v0.y);
-            areg[t][i][8 * q + 2] = __uint_as_float(v0.z); areg[t][i][8 * q + 3] = __uint_as_float(v0.w);
-            areg[t][i][8 * q + 4] = __uint_as_float(v1.x); areg[t][i][8 * q + 5] = __uint_as_float(v1.y);
-            areg[t][i][8 * q + 6] = __uint_as_float(v1.z); areg[t][i][8 * q + 7] = __uint_as_float(v1.w);
+            areg[t][i][4 * q + 0] = pack2(__uint_as_float(v0.x), __uint_as_float(v0.y));
+            areg[t][i][4 * q + 1] = pack2(__uint_as_float(v0.z), __uint_as_float(v0.w));
+            areg[t][i][4 * q + 2] = pack2(__uint_as_float(v1.x), __uint_as_float(v1.y));
+            areg[t][i][4 * q + 3] = pack2(__uint_as_float(v1.z), __uint_as_float(v1.w));
           }
         }
       } else {
 #pragma unroll
-        for (int e = 0; e < EPC; ++e) areg[t][i][e] = 0.f;
+        for (int e = 0; e < EPC / 2; ++e) areg[t][i][e] = 0ull;
       }
     }
   }
 }
 
-// Partial dot products of one row slice (this lane's chunks) with NT tokens,
-// reduced over the warp's lanes.  Independent accumulators per chunk and two
-// interleaved FMA chains per chunk keep the FMA pipe busy.
-template <int WT, int NT>
-KD_DEV void row_dot(const uint8_t* wslice, const float (&sc)[kMaxChunksLane], int cpl,
-                    const ActRegs<WT>& areg, float (&out)[kTT]) {
+// Sum of four per-lane values over the warp, transposed: lane l receives the
+// total of value (l >> 3) & 3.
+KD_DEV float reduce4_transposed(float v0, float v1, float v2, float v3) {
   const int lane = threadIdx.x & 31;
-  float acc[kMaxChunksLane][NT];
+  const bool b4 = lane & 16, b3 = lane & 8;
+  float k0 = b4 ? v2 : v0, k1 = b4 ? v3 : v1;
+  const float s0 = b4 ? v0 : v2, s1 = b4 ? v1 : v3;
+  k0 += __shfl_xor_sync(0xffffffffu, s0, 16);
+  k1 += __shfl_xor_sync(0xffffffffu, s1, 16);
+  float k = b3 ? k1 : k0;
+  const float sx = b3 ? k0 : k1;
+  k += __shfl_xor_sync(0xffffffffu, sx, 8);
+  k += __shfl_xor_sync(0xffffffffu, k, 4);
+  k += __shfl_xor_sync(0xffffffffu, k, 2);
+  k += __shfl_xor_sync(0xffffffffu, k, 1);
+  return k;
+}
+
+// Dot products of up to four rows (stage rows rows[j], -1 = none) with NT
+// tokens over this lane's chunks, reduced over the warp: lane l returns the
+// sums of row j = (l >> 3) & 3 in res[].
+template <int WT, int NT, class Plan>
+KD_DEV void batch_dot(const Plan& plan, const Seg& s, int stage_row0, const uint8_t* st,
+                      const int (&rows)[4], int slice0, int cpl, const ActRegs<WT>& areg,
+                      float (&res)[kTT]) {
+  constexpr int EPC = WTraits<WT>::EPC;
+  const int lane = threadIdx.x & 31;
+  f32x2 acc[4][NT];
 #pragma unroll
-  for (int i = 0; i < kMaxChunksLane; ++i)
+  for (int j = 0; j < 4; ++j)
 #pragma unroll
-    for (int t = 0; t < NT; ++t) acc[i][t] = 0.f;
+    for (int t = 0; t < NT; ++t) acc[j][t] = 0ull;
 #pragma unroll
-  for (int i = 0; i < kMaxChunksLane; ++i) {
-    const int c = lane + 32 * i;
-    if (c < cpl) {
-      const uint4 wv = lds_v4(wslice + (size_t)c * 16);
-      if constexpr (WT == W_BF16) {
-        const float w[8] = {bf_lo(wv.x), bf_hi(wv.x), bf_lo(wv.y), bf_hi(wv.y),
-                            bf_lo(wv.z), bf_hi(wv.z), bf_lo(wv.w), bf_hi(wv.w)};
+  for (int j = 0; j < 4; ++j) {
+    if (rows[j] < 0) continue;
+    const uint8_t* wrow = st + (size_t)rows[j] * s.row_bytes + (size_t)slice0 * 16;
+    const float* srow = nullptr;
+    if constexpr (WT == W_FP8) srow = plan.scale_row(s, s.row0 + stage_row0 + rows[j]);
 #pragma unroll
-        for (int t = 0; t < NT; ++t) {
-          float a0 = w[0] * areg[t][i][0], a1 = w[1] * areg[t][i][1];
-          a0 = fmaf(w[2], areg[t][i][2], a0); a1 = fmaf(w[3], areg[t][i][3], a1);
-          a0 = fmaf(w[4], areg[t][i][4], a0); a1 = fmaf(w[5], areg[t][i][5], a1);
-          a0 = fmaf(w[6], areg[t][i][6], a0); a1 = fmaf(w[7], areg[t][i][7], a1);
-          acc[i][t] = a0 + a1;
-        }
-      } else {
-        float w[16];
-        e4m3x4_to_f32(wv.x, w[0], w[1], w[2], w[3]);
-        e4m3x4_to_f32(wv.y, w[4], w[5], w[6], w[7]);
-        e4m3x4_to_f32(wv.z, w[8], w[9], w[10], w[11]);
-        e4m3x4_to_f32(wv.w, w[12], w[13], w[14], w[15]);
+    for (int i = 0; i < kMaxChunksLane; ++i) {
+      const int c = lane + 32 * i;
+      if (c < cpl) {
+        const uint4 wv = lds_v4(wrow + (size_t)c * 16);
+        if constexpr (WT == W_BF16) {
+          const f32x2 w0 = bf2_to_f2(wv.x), w1 = bf2_to_f2(wv.y), w2 = bf2_to_f2(wv.z),
+                      w3 = bf2_to_f2(wv.w);
 #pragma unroll
-        for (int t = 0; t < NT; ++t) {
-          float a0 = w[0] * areg[t][i][0], a1 = w[1] * areg[t][i][1];
-#pragma unroll
-          for (int e = 2; e < 16; e += 2) {
-            a0 = fmaf(w[e], areg[t][i][e], a0);
-            a1 = fmaf(w[e + 1], areg[t][i][e + 1], a1);
+          for (int t = 0; t < NT; ++t) {
+            f32x2 a = acc[j][t];
+            a = ffma2(w0, areg[t][i][0], a);
+            a = ffma2(w1, areg[t][i][1], a);
+            a = ffma2(w2, areg[t][i][2], a);
+            a = ffma2(w3, areg[t][i][3], a);
+            acc[j][t] = a;
           }
-          acc[i][t] = (a0 + a1) * sc[i];
+        } else {
+          float w[16];
+          e4m3x4_to_f32(wv.x, w[0], w[1], w[2], w[3]);
+          e4m3x4_to_f32(wv.y, w[4], w[5], w[6], w[7]);
+          e4m3x4_to_f32(wv.z, w[8], w[9], w[10], w[11]);
+          e4m3x4_to_f32(wv.w, w[12], w[13], w[14], w[15]);
+          const float sc = __ldg(srow + (((slice0 + c) * EPC) >> 7));
+          const f32x2 sc2 = pack2(sc, sc);
+#pragma unroll
+          for (int t = 0; t < NT; ++t) {
+            f32x2 p = 0ull;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) p = ffma2(pack2(w[2 * e], w[2 * e + 1]), areg[t][i][e], p);
+            acc[j][t] = ffma2(p, sc2, acc[j][t]);
+          }
         }
       }
     }
   }
 #pragma unroll
   for (int t = 0; t < NT; ++t) {
-    float v = acc[0][t];
+    float v[4];
 #pragma unroll
-    for (int i = 1; i < kMaxChunksLane; ++i) v += acc[i][t];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    out[t] = v;
+    for (int j = 0; j < 4; ++j) {
+      const float2 p = unpack2(acc[j][t]);
+      v[j] = p.x + p.y;
+    }
+    res[t] = reduce4_transposed(v[0], v[1], v[2], v[3]);
   }
 }
 
 // After every warp wrote its partials of a stage into `red` ([row][slice][t]):
-// sum the slices in a fixed order and run the epilogue.
+// sum the S slices in a fixed order and run the epilogue.
 template <class Plan>
-KD_DEV void stage_epilogue(const Plan& plan, const Seg& s, const float* red, int n, int stage_row0,
-                           int tok, int nt) {
+KD_DEV void stage_epilogue(const Plan& plan, const Seg& s, const float* red, int n, int S,
+                           int stage_row0, int tok, int nt) {
   const int ctid = threadIdx.x;
   if (plan.paired()) {
     const int npair = n >> 1;
     for (int q = ctid; q < npair * nt; q += kThreads) {
       const int p = q / nt, j = q % nt;
       float g = 0.f, u = 0.f;
-#pragma unroll
-      for (int sl = 0; sl < kCW; ++sl) {
-        g += red[((2 * p) * kCW + sl) * kTT + j];
-        u += red[((2 * p + 1) * kCW + sl) * kTT + j];
+      for (int sl = 0; sl < S; ++sl) {
+        g += red[((2 * p) * S + sl) * kTT + j];
+        u += red[((2 * p + 1) * S + sl) * kTT + j];
       }
       plan.epilogue2(s, (s.row0 + stage_row0) / 2 + p, tok + j, g, u);
     }
@@ -259,8 +300,7 @@ KD_DEV void stage_epilogue(const Plan& plan, const Seg& s, const float* red, int
     for (int q = ctid; q < n * nt; q += kThreads) {
       const int row = q / nt, j = q % nt;
       float v = 0.f;
-#pragma unroll
-      for (int sl = 0; sl < kCW; ++sl) v += red[(row * kCW + sl) * kTT + j];
+      for (int sl = 0; sl < S; ++sl) v += red[(row * S + sl) * kTT + j];
       plan.epilogue(s, s.row0 + stage_row0 + row, tok + j, v);
     }
   }
@@ -273,12 +313,13 @@ KD_DEV void stage_epilogue(const Plan& plan, const Seg& s, const float* red, int
 template <int WT, int AT, class Plan>
 KD_DEV void consume_segment(const Plan& plan, StreamShared& sh, Issuer& iss, const Seg& s,
                             uint32_t& it, int& rb, unsigned* err) {
-  constexpr int EPC = WTraits<WT>::EPC;
   constexpr int TT = WTraits<WT>::TT;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rps = rows_per_stage(s.row_bytes, plan.paired());
-  const int cpl = (s.row_bytes / 16) / kCW;       // chunks per slice (<= 32*kMaxChunksLane)
-  const int slice0 = warp * cpl;
+  const int S = slices_per_row(s.row_bytes), G = kCW / S;
+  const int cpl = (s.row_bytes / 16) / S;         // chunks per slice (<= 32*kMaxChunksLane)
+  const int my_slice = warp % S, my_group = warp / S;
+  const int slice0 = my_slice * cpl;
   ActRegs<WT> areg;
   const bool single_pass = s.ntok <= TT;
   if (single_pass) load_act_regs<WT, AT>(plan, s, 0, s.ntok, slice0, cpl, areg);
@@ -287,39 +328,30 @@ KD_DEV void consume_segment(const Plan& plan, StreamShared& sh, Issuer& iss, con
     const int slot = it % kStages;
     const uint32_t ph = (it / kStages) & 1u;
     wait_or_abort(&sh.full[slot], ph, sh.abort_flag, err, ERR_WAIT_FULL);
-    const uint8_t* st = sh.stage + (size_t)slot * kStageBytes + (size_t)slice0 * 16;
+    const uint8_t* st = sh.stage + (size_t)slot * kStageBytes;
     for (int tok = 0; tok < s.ntok; tok += TT) {
       const int nt = s.ntok - tok < TT ? s.ntok - tok : TT;
       if (!single_pass) load_act_regs<WT, AT>(plan, s, tok, nt, slice0, cpl, areg);
       float* red = sh.red + rb * kRedFloats;
-      for (int row = 0; row < n; ++row) {
-        // FP8 block scales of this row at this lane's chunks (static weights)
-        float sc[kMaxChunksLane];
+      for (int rbase = my_group; rbase < n; rbase += 4 * G) {
+        int rows[4];
 #pragma unroll
-        for (int i = 0; i < kMaxChunksLane; ++i) sc[i] = 1.f;
-        if constexpr (WT == W_FP8) {
-          const float* srow = plan.scale_row(s, s.row0 + r0 + row);
-#pragma unroll
-          for (int i = 0; i < kMaxChunksLane; ++i) {
-            const int c = lane + 32 * i;
-            sc[i] = c < cpl ? __ldg(srow + (((slice0 + c) * EPC) >> 7)) : 0.f;
-          }
-        }
-        float part[kTT];
-        const uint8_t* wrow = st + (size_t)row * s.row_bytes;
-        if (nt == 1) row_dot<WT, 1>(wrow, sc, cpl, areg, part);
-        else if (TT == 2 || nt == 2) row_dot<WT, 2>(wrow, sc, cpl, areg, part);
-        else row_dot<WT, TT>(wrow, sc, cpl, areg, part);
-        if (lane == 0) {
+        for (int j = 0; j < 4; ++j) rows[j] = rbase + j * G < n ? rbase + j * G : -1;
+        float res[kTT];
+        if (nt == 1) batch_dot<WT, 1>(plan, s, r0, st, rows, slice0, cpl, areg, res);
+        else if (TT == 2 || nt == 2) batch_dot<WT, 2>(plan, s, r0, st, rows, slice0, cpl, areg, res);
+        else batch_dot<WT, TT>(plan, s, r0, st, rows, slice0, cpl, areg, res);
+        const int myrow = rbase + ((lane >> 3) & 3) * G;   // the row this lane's sums belong to
+        if ((lane & 7) == 0 && myrow < n) {
 #pragma unroll
           for (int t = 0; t < kTT; ++t)
-            if (t < nt) red[(row * kCW + warp) * kTT + t] = part[t];
+            if (t < nt) red[(myrow * S + my_slice) * kTT + t] = res[t];
         }
       }
       named_bar_sync(1, kThreads);
       // after the stage's last token group no thread reads it again: refill
       if (threadIdx.x == 0 && tok + TT >= s.ntok) iss.next(plan, sh);
-      stage_epilogue(plan, s, red, n, r0, tok, nt);
+      stage_epilogue(plan, s, red, n, S, r0, tok, nt);
       rb ^= 1;
     }
     if (s.ntok == 0) {
