@@ -187,12 +187,11 @@ def kernel_bytes(spec, n_active: int) -> dict:
         "proj": (nq * H + H * A) * eb + blk(nq, H) + blk(H, A),
         "router": E * H * eb + blk(E, H),
         "gateup": n_active * (2 * I * H * eb + 2 * blk(I, H)),
-        "down": n_active * (H * I * eb + blk(H, I)),
-        "combine": 0,
+        "down": (n_active + spec.n_shared) * (H * I * eb + blk(H, I)),
     }
 
 
-KNAMES = ("proj", "router", "gateup", "down", "combine")
+KNAMES = ("proj", "router", "gateup", "down")
 
 
 def time_layer(layer, x_bits, a_bits, steps, warmup, flush, pg, local, per_kernel=True):
@@ -301,7 +300,11 @@ def bench_single(w, steps, warmup, flush, pg, local, peak):
     layer = make_layer(w)
     try:
         x, a = w.hidden_in(), w.attn_out()
-        times, kt = time_layer(layer, x, a, steps, warmup, flush, pg, local)
+        # the layer as it runs (kernels chained by programmatic dependent launch)
+        times, _ = time_layer(layer, x, a, steps, warmup, flush, pg, local, per_kernel=False)
+        # per-kernel durations from a separate pass with events between kernels
+        # (the hook launches each kernel only after the previous one finished)
+        _, kt = time_layer(layer, x, a, max(steps // 4, 5), 2, flush, pg, local, per_kernel=True)
         na = n_active_of(layer)
         ms = statistics.mean(times)
         byts = layer_bytes(layer, na)
@@ -411,7 +414,7 @@ def run_kd(args):
     clocks = cs.summary()
     e2e_times, h2d, d2h = time_layer_e2e(layer, x, a, min(args.steps, 200), args.warmup, flush, pg,
                                          local)
-    launches_per_step = 5 + (2 if main.dims.n_shared else 0)
+    launches_per_step = 4 + (1 if main.dims.n_shared else 0)
     layer.close()
     ms = res["us_per_layer"] / 1e3
     ms_max = max_over_ranks(pg, ms)

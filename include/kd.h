@@ -156,9 +156,11 @@ void kd_stack_destroy(kd_stack* stack);
  * calls record the caller's events (cudaEvent_t values created with timing)
  * on the call's stream at: [0] start, [1] after the QKV + o-proj kernel,
  * [2] after the router kernel, [3] after the routed gate/up kernel, [4] after
- * the down kernel (routed experts + shared expert), [5] after the final combine.  n_events == 0 turns
- * it off.  The events are not owned by the layer.  Errors: KD_EINVAL. */
-#define KD_N_TIMING_EVENTS 6
+ * the down kernel (routed + shared experts, with the final combine).  While
+ * it is on, kernels of the call are not launched as programmatic dependents,
+ * so that each interval covers one kernel.  n_events == 0 turns it off.  The
+ * events are not owned by the layer.  Errors: KD_EINVAL. */
+#define KD_N_TIMING_EVENTS 5
 int kd_layer_set_timing_events(kd_layer* layer, void* const* events, int n_events);
 
 /* Message of the last failure on the calling thread ("" if none). */

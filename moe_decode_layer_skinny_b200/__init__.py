@@ -25,7 +25,7 @@ EXPORTS = ("kd_layer_create", "kd_layer_destroy", "kd_decode_layer", "kd_layer_c
            "kd_layer_qkv", "kd_layer_prefetch_l2", "kd_layer_debug_tensor", "kd_layer_read_weight",
            "kd_layer_bytes", "kd_layer_set_timing_events", "kd_stack_create", "kd_stack_run",
            "kd_stack_destroy", "kd_last_error")
-N_TIMING_EVENTS = 6
+N_TIMING_EVENTS = 5
 
 
 class KdError(RuntimeError):

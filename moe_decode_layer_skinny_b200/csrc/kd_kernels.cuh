@@ -6,8 +6,10 @@
 //   router_kernel      fp32 router logits, then (last CTA) top-k, renormalised
 //                      softmax and the per-expert token lists
 //   gateup_kernel      SwiGLU gate/up of the active experts (or the shared one)
-//   down_kernel        down projection of the active experts and the shared one
-//   combine_kernel     h1 + shared + gate-weighted routed outputs -> bf16
+//   down_kernel        down projection of the active experts and the shared one,
+//                      with the final combine h1 + shared + gate-weighted routed
+//                      outputs -> bf16 done per 64-row block by the CTA that
+//                      completes the block
 #pragma once
 
 #include "../../kdgen/kd_gen.h"
@@ -82,6 +84,7 @@ struct LayerDev {
   float* act; float* act_sh;               // [Mmax*k, I] by position, [Mmax, I] (fp32)
   float* yr; float* ysh;                   // [Mmax*k, H] by token*k+slot, [Mmax, H]
   unsigned* counter;                       // router arrival counter (self-resetting)
+  unsigned* hcnt;                          // [H/64] down rows done per block (self-resetting)
   unsigned* err;
 };
 
@@ -130,8 +133,13 @@ struct ProjPlan {
     }
   }
   KD_DEV void epilogue2(const Seg&, int, int, float, float) const {}
+  KD_DEV bool wants_segment_done() const { return false; }
+  KD_DEV void segment_done(const Seg&) const {}
 };
 
+// The weights are static, so the first stages are requested before waiting
+// for the preceding kernel (programmatic dependent launch); x and attn_out
+// are read only after the wait.
 template <int WT>
 __global__ void __launch_bounds__(kThreads, 1) proj_kernel(LayerDev L, Acts a) {
   extern __shared__ uint8_t smem[];
@@ -139,7 +147,7 @@ __global__ void __launch_bounds__(kThreads, 1) proj_kernel(LayerDev L, Acts a) {
   p.L = &L; p.a = a;
   p.q0 = split_lo(L.Nqkv, gridDim.x, blockIdx.x); p.q1 = split_lo(L.Nqkv, gridDim.x, blockIdx.x + 1);
   p.o0 = split_lo(L.H, gridDim.x, blockIdx.x); p.o1 = split_lo(L.H, gridDim.x, blockIdx.x + 1);
-  stream_run<WT, A_BF16>(p, smem, L.err);
+  stream_run<WT, A_BF16>(p, smem, L.err, true);
 }
 
 // ------------------------------------------------------------------ router
@@ -198,10 +206,11 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(LayerDev L, int 
   const int row = blockIdx.x * kRouterRows + rloc;
   const int cq = (L.H * L.eb / 16) / 4;   // chunks per quarter row
   __shared__ float part[kRouterRows][4][64];
+  // the router weights are static: load them before waiting for h1
+  uint4 w[kRouterWChunks];
+  float sc[kRouterWChunks];
   if (row < L.E) {
     const uint8_t* wrow = L.wr + (size_t)row * L.H * L.eb;
-    uint4 w[kRouterWChunks];
-    float sc[kRouterWChunks];
 #pragma unroll
     for (int i = 0; i < kRouterWChunks; ++i) {
       const int c = lane + 32 * i;
@@ -211,6 +220,10 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(LayerDev L, int 
         sc[i] = WT == W_FP8 ? __ldg(L.sr + (size_t)(row >> 7) * L.nHb + ((ci * EPC) >> 7)) : 1.f;
       }
     }
+  }
+  pdl_wait();
+  pdl_launch_dependents();
+  if (row < L.E) {
     for (int t0 = 0; t0 < M; t0 += kTT) {
       const int nt = M - t0 < kTT ? M - t0 : kTT;
       const float* arow[kTT];
@@ -414,12 +427,16 @@ struct GateUpPlan {
     float* dst = shared ? L->act_sh + (size_t)j * L->I : L->act + (size_t)(s.tok0 + j) * L->I;
     dst[i] = silu(g) * u;
   }
+  KD_DEV bool wants_segment_done() const { return false; }
+  KD_DEV void segment_done(const Seg&) const {}
 };
 
 // Down projection of every active routed expert and (entry n_act) the shared
 // expert, in one launch.
 struct DownPlan {
   const LayerDev* L; int M; int n_act; ExpertRange R;
+  uint16_t* out;                 // layer output [M, H] bf16
+  int* s_list; int* s_n;         // shared scratch: blocks this CTA completes
   KD_DEV int num_segments() const { return R.num_segments(); }
   KD_DEV Seg segment(int i) const {
     int a, u0, u1;
@@ -452,6 +469,45 @@ struct DownPlan {
     else L->yr[(size_t)L->perm[s.tok0 + j] * L->H + h] = v;
   }
   KD_DEV void epilogue2(const Seg&, int, int, float, float) const {}
+  KD_DEV bool wants_segment_done() const { return true; }
+
+  // Count the segment's rows into their 64-row blocks; the CTA whose rows
+  // complete a block (every routed entry and the shared one) writes that
+  // block of the layer output:
+  //   out[t, h] = bf16(h1[t, h] + ysh[t, h] + sum_j g[t, j] yr[t*k + j, h])
+  // with the terms added in this fixed order.
+  KD_DEV void segment_done(const Seg& s) const {
+    const int target = 64 * (n_act + L->S);
+    if (threadIdx.x == 0) {
+      *s_n = 0;
+      __threadfence();
+      for (int b = s.row0 / 64; b * 64 < s.row0 + s.nrows; ++b) {
+        const int lo = b * 64 > s.row0 ? b * 64 : s.row0;
+        const int hi = (b + 1) * 64 < s.row0 + s.nrows ? (b + 1) * 64 : s.row0 + s.nrows;
+        const unsigned prev = atomicAdd(L->hcnt + b, (unsigned)(hi - lo));
+        if (prev + (unsigned)(hi - lo) == (unsigned)target) {
+          L->hcnt[b] = 0u;  // every contribution is in: ready for the next call
+          s_list[(*s_n)++] = b;
+        }
+      }
+      __threadfence();
+    }
+    named_bar_sync(1, kThreads);
+    const int nb = *s_n;
+    for (int q = 0; q < nb; ++q) {
+      const int b = s_list[q];
+      for (int e = threadIdx.x; e < 64 * M; e += kThreads) {
+        const int t = e / 64, h = b * 64 + e % 64;
+        const size_t o = (size_t)t * L->H + h;
+        float v = L->h1f[o];
+        if (L->S) v += __ldcg(L->ysh + o);
+        for (int j = 0; j < L->k; ++j)
+          v += L->gates[t * L->k + j] * __ldcg(L->yr + ((size_t)t * L->k + j) * L->H + h);
+        out[o] = f32_to_bf16_bits(v);
+      }
+    }
+    named_bar_sync(1, kThreads);  // s_list / s_n are reused by the next segment
+  }
 };
 
 KD_DEV ExpertRange expert_range(int n_act, int per) {
@@ -463,39 +519,35 @@ KD_DEV ExpertRange expert_range(int n_act, int per) {
   return r;
 }
 
+// Routed experts are known only after the router, so the routed launches
+// wait for the preceding kernel before reading the routing (and before their
+// first weight request); the shared expert's weights are static.
 template <int WT>
 __global__ void __launch_bounds__(kThreads, 1) gateup_kernel(LayerDev L, int M, int shared) {
   extern __shared__ uint8_t smem[];
   GateUpPlan p;
   p.L = &L; p.M = M; p.shared = shared != 0;
+  if (!shared) {
+    pdl_wait();
+    pdl_launch_dependents();
+  }
   const int n_act = shared ? 1 : *(volatile int*)L.n_active;
   p.R = expert_range(n_act, L.I);
-  stream_run<WT, A_F32>(p, smem, L.err);
+  stream_run<WT, A_F32>(p, smem, L.err, shared != 0);
 }
 
 template <int WT>
-__global__ void __launch_bounds__(kThreads, 1) down_kernel(LayerDev L, int M) {
+__global__ void __launch_bounds__(kThreads, 1) down_kernel(LayerDev L, int M, uint16_t* out) {
   extern __shared__ uint8_t smem[];
+  __shared__ int s_list[128];
+  __shared__ int s_n;
+  pdl_wait();
+  pdl_launch_dependents();
   DownPlan p;
-  p.L = &L; p.M = M;
+  p.L = &L; p.M = M; p.out = out; p.s_list = s_list; p.s_n = &s_n;
   p.n_act = *(volatile int*)L.n_active;
   p.R = expert_range(p.n_act + L.S, L.H);
-  stream_run<WT, A_F32>(p, smem, L.err);
-}
-
-// ------------------------------------------------------------------ combine
-
-__global__ void combine_kernel(LayerDev L, Acts a) {
-  const size_t n = (size_t)a.M * L.H;
-  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
-       i += (size_t)gridDim.x * blockDim.x) {
-    const int t = (int)(i / L.H), h = (int)(i % L.H);
-    float v = L.h1f[i];
-    if (L.S) v += L.ysh[i];
-    for (int j = 0; j < L.k; ++j)
-      v += L.gates[t * L.k + j] * L.yr[((size_t)t * L.k + j) * L.H + h];
-    a.out[i] = f32_to_bf16_bits(v);
-  }
+  stream_run<WT, A_F32>(p, smem, L.err, false);
 }
 
 }  // namespace kd

@@ -48,7 +48,7 @@ struct kd_layer {
   cudaEvent_t ev_h1 = nullptr, ev_sh = nullptr;
   uint64_t static_bytes = 0, expert_bytes = 0;
   int Nqkv = 0, A = 0;
-  cudaEvent_t tev[KD_N_TIMING_EVENTS] = {};
+  cudaEvent_t tev[KD_N_TIMING_EVENTS] = {};  // profiling hook (kd_layer_set_timing_events)
   bool timing = false;
 };
 
@@ -240,6 +240,8 @@ extern "C" int kd_layer_create(const kd_config* cfg, uint64_t seed, kd_layer** o
   TRY(dalloc_t(L, (size_t)M * k * H, &d.yr));
   TRY(dalloc_t(L, (size_t)M * H, &d.ysh));
   TRY(dalloc_t(L, 1, &d.counter));
+  TRY(dalloc_t(L, (size_t)H / 64, &d.hcnt));
+  TRYC(cudaMemset(d.hcnt, 0, sizeof(unsigned) * (H / 64)));
   TRY(dalloc_t(L, 1, &d.err));
   TRYC(cudaMemset(d.counter, 0, sizeof(unsigned)));
   TRYC(cudaMemset(d.err, 0, sizeof(unsigned)));
@@ -287,23 +289,42 @@ extern "C" void kd_layer_destroy(kd_layer* L) {
 
 // ------------------------------------------------------------------ decode
 
+static int prefetch_static(const kd_layer* L, size_t max_bytes, cudaStream_t s);
+
+// Launch with programmatic stream serialization: the kernel may start while
+// the preceding kernel in the stream finishes; it waits (griddepcontrol.wait)
+// before reading anything that kernel wrote.
+template <typename... KArgs, typename... Args>
+static cudaError_t launch(void (*kernel)(KArgs...), int grid, int block, size_t smem,
+                          cudaStream_t s, bool pdl, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 static int launch_layer(kd_layer* L, void* hidden, const void* attn, int M, cudaStream_t s,
                         const kd_layer* prefetch_next, cudaStream_t pf, cudaEvent_t ev_fork,
-                        cudaEvent_t ev_join);
+                        cudaEvent_t ev_join, bool pdl_first);
 
 extern "C" int kd_decode_layer(kd_layer* L, void* hidden, const void* attn, int M, void* stream) {
   if (!L || !hidden || !attn) return fail(KD_EINVAL, "kd_decode_layer: null argument%s", "");
   if (M < 1 || M > L->maxM)
     return fail(KD_ERANGE, "kd_decode_layer: M=%s%ld outside 1..max_tokens", "", (long)M);
   return launch_layer(L, hidden, attn, M, static_cast<cudaStream_t>(stream), nullptr, nullptr,
-                      nullptr, nullptr);
+                      nullptr, nullptr, false);
 }
-
-static int prefetch_static(const kd_layer* L, size_t max_bytes, cudaStream_t s);
 
 static int launch_layer(kd_layer* L, void* hidden, const void* attn, int M, cudaStream_t s,
                         const kd_layer* next, cudaStream_t pf, cudaEvent_t ev_fork,
-                        cudaEvent_t ev_join) {
+                        cudaEvent_t ev_join, bool pdl_first) {
   const LayerDev& d = L->d;
   const bool fp8 = L->cfg.wdtype == KD_WFP8;
   Acts a;
@@ -314,34 +335,25 @@ static int launch_layer(kd_layer* L, void* hidden, const void* attn, int M, cuda
   const int G = L->nsm;
   const size_t sm = kStreamSmem;
   if (L->timing) KD_CUDA(cudaEventRecord(L->tev[0], s));
-  if (fp8) proj_kernel<W_FP8><<<G, kThreads, sm, s>>>(d, a);
-  else proj_kernel<W_BF16><<<G, kThreads, sm, s>>>(d, a);
-  KD_CUDA(cudaGetLastError());
+  KD_CUDA(launch(fp8 ? proj_kernel<W_FP8> : proj_kernel<W_BF16>, G, kThreads, sm, s, pdl_first, d, a));
   if (L->timing) KD_CUDA(cudaEventRecord(L->tev[1], s));
   if (d.S) KD_CUDA(cudaEventRecord(L->ev_h1, s));
   // the router goes first so that its CTAs get SMs before the shared
   // expert's gate/up (on the side stream) fills them
   const int rgrid = (d.E + kRouterRows - 1) / kRouterRows;
-  if (fp8) router_kernel<W_FP8><<<rgrid, kRouterThreads, 0, s>>>(d, M);
-  else router_kernel<W_BF16><<<rgrid, kRouterThreads, 0, s>>>(d, M);
-  KD_CUDA(cudaGetLastError());
+  KD_CUDA(launch(fp8 ? router_kernel<W_FP8> : router_kernel<W_BF16>, rgrid, kRouterThreads, 0, s,
+                 !L->timing, d, M));
   if (d.S) {
     KD_CUDA(cudaStreamWaitEvent(L->side, L->ev_h1, 0));
-    if (fp8) gateup_kernel<W_FP8><<<G, kThreads, sm, L->side>>>(d, M, 1);
-    else gateup_kernel<W_BF16><<<G, kThreads, sm, L->side>>>(d, M, 1);
-    KD_CUDA(cudaGetLastError());
+    KD_CUDA(launch(fp8 ? gateup_kernel<W_FP8> : gateup_kernel<W_BF16>, G, kThreads, sm, L->side,
+                   false, d, M, 1));
     KD_CUDA(cudaEventRecord(L->ev_sh, L->side));
   }
   if (L->timing) KD_CUDA(cudaEventRecord(L->tev[2], s));
-  if (fp8) gateup_kernel<W_FP8><<<G, kThreads, sm, s>>>(d, M, 0);
-  else gateup_kernel<W_BF16><<<G, kThreads, sm, s>>>(d, M, 0);
-  KD_CUDA(cudaGetLastError());
+  KD_CUDA(launch(fp8 ? gateup_kernel<W_FP8> : gateup_kernel<W_BF16>, G, kThreads, sm, s,
+                 !L->timing, d, M, 0));
   if (L->timing) KD_CUDA(cudaEventRecord(L->tev[3], s));
   if (d.S) KD_CUDA(cudaStreamWaitEvent(s, L->ev_sh, 0));
-  if (fp8) down_kernel<W_FP8><<<G, kThreads, sm, s>>>(d, M);
-  else down_kernel<W_BF16><<<G, kThreads, sm, s>>>(d, M);
-  KD_CUDA(cudaGetLastError());
-  if (L->timing) KD_CUDA(cudaEventRecord(L->tev[4], s));
   if (next && pf) {
     // the next layer's static weights into L2 while this layer finishes
     KD_CUDA(cudaEventRecord(ev_fork, s));
@@ -350,11 +362,9 @@ static int launch_layer(kd_layer* L, void* hidden, const void* attn, int M, cuda
     if (rc != KD_OK) return rc;
     KD_CUDA(cudaEventRecord(ev_join, pf));
   }
-  const size_t n = (size_t)M * d.H;
-  const int cgrid = (int)std::min<size_t>((n + 255) / 256, (size_t)G * 8);
-  combine_kernel<<<cgrid, 256, 0, s>>>(d, a);
-  KD_CUDA(cudaGetLastError());
-  if (L->timing) KD_CUDA(cudaEventRecord(L->tev[5], s));
+  KD_CUDA(launch(fp8 ? down_kernel<W_FP8> : down_kernel<W_BF16>, G, kThreads, sm, s,
+                 !L->timing && !d.S, d, M, a.out));
+  if (L->timing) KD_CUDA(cudaEventRecord(L->tev[4], s));
   if (next && pf) KD_CUDA(cudaStreamWaitEvent(s, ev_join, 0));
   return KD_OK;
 }
@@ -366,6 +376,9 @@ extern "C" int kd_layer_check(kd_layer* L) {
   KD_CUDA(cudaMemcpy(&e, L->d.err, sizeof e, cudaMemcpyDeviceToHost));
   if (e == 0) return KD_OK;
   KD_CUDA(cudaMemset(L->d.err, 0, sizeof(unsigned)));
+  // an aborted call may have left arrival counters part-way
+  KD_CUDA(cudaMemset(L->d.counter, 0, sizeof(unsigned)));
+  KD_CUDA(cudaMemset(L->d.hcnt, 0, sizeof(unsigned) * (L->d.H / 64)));
   if (e & (ERR_WAIT_FULL | ERR_WAIT_EMPTY | ERR_WAIT_MMA))
     return fail(KD_ETIMEOUT, "device: a bounded wait gave up (flags %s0x%lx)", "", (long)e);
   return fail(KD_EDEVICE, "device error flags %s0x%lx", "", (long)e);
@@ -554,7 +567,7 @@ extern "C" int kd_stack_run(kd_stack* S, void* hidden, const void* attn, void* s
       const uint8_t* a = static_cast<const uint8_t*>(attn) + (size_t)l * S->M * L->d.A * 2;
       const kd_layer* next = (S->prefetch && l + 1 < n) ? S->layers[l + 1] : nullptr;
       rc = launch_layer(L, hidden, a, S->M, S->cap, next, next ? S->pf : nullptr, S->ev_fork[l],
-                        S->ev_join[l]);
+                        S->ev_join[l], l > 0);
     }
     cudaGraph_t g = nullptr;
     cudaError_t ce = cudaStreamEndCapture(S->cap, &g);

@@ -136,6 +136,9 @@ struct Issuer {
 //   bool paired()                                 rows come in (gate, up) pairs
 //   void epilogue(const Seg&, int row, int j, float sum)            unpaired
 //   void epilogue2(const Seg&, int pair_row, int j, float g, float u) paired
+//   bool wants_segment_done(); void segment_done(const Seg&)
+//                                                 called by all threads after a CTA
+//                                                 barrier that follows a segment
 //
 // Geometry of a segment: each row is cut into S column slices (the smallest
 // power of two that leaves <= 32*kMaxChunksLane 16-byte chunks per slice);
@@ -220,11 +223,16 @@ KD_DEV void batch_dot(const Plan& plan, const Seg& s, int stage_row0, const uint
                       float (&res)[kTT]) {
   constexpr int EPC = WTraits<WT>::EPC;
   const int lane = threadIdx.x & 31;
-  f32x2 acc[4][NT];
+  // one accumulator per (row, token); with a single token, one per (row,
+  // chunk pair) so that 8 independent FMA chains are in flight
+  constexpr int NA = NT == 1 ? 2 : 1;
+  f32x2 acc[4][NT][NA];
 #pragma unroll
   for (int j = 0; j < 4; ++j)
 #pragma unroll
-    for (int t = 0; t < NT; ++t) acc[j][t] = 0ull;
+    for (int t = 0; t < NT; ++t)
+#pragma unroll
+      for (int u = 0; u < NA; ++u) acc[j][t][u] = 0ull;
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     if (rows[j] < 0) continue;
@@ -241,12 +249,12 @@ KD_DEV void batch_dot(const Plan& plan, const Seg& s, int stage_row0, const uint
                       w3 = bf2_to_f2(wv.w);
 #pragma unroll
           for (int t = 0; t < NT; ++t) {
-            f32x2 a = acc[j][t];
+            f32x2 a = acc[j][t][i % NA];
             a = ffma2(w0, areg[t][i][0], a);
             a = ffma2(w1, areg[t][i][1], a);
             a = ffma2(w2, areg[t][i][2], a);
             a = ffma2(w3, areg[t][i][3], a);
-            acc[j][t] = a;
+            acc[j][t][i % NA] = a;
           }
         } else {
           float w[16];
@@ -261,7 +269,7 @@ KD_DEV void batch_dot(const Plan& plan, const Seg& s, int stage_row0, const uint
             f32x2 p = 0ull;
 #pragma unroll
             for (int e = 0; e < 8; ++e) p = ffma2(pack2(w[2 * e], w[2 * e + 1]), areg[t][i][e], p);
-            acc[j][t] = ffma2(p, sc2, acc[j][t]);
+            acc[j][t][i % NA] = ffma2(p, sc2, acc[j][t][i % NA]);
           }
         }
       }
@@ -272,7 +280,12 @@ KD_DEV void batch_dot(const Plan& plan, const Seg& s, int stage_row0, const uint
     float v[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const float2 p = unpack2(acc[j][t]);
+      float2 p = unpack2(acc[j][t][0]);
+      if (NA == 2) {
+        const float2 q = unpack2(acc[j][t][NA - 1]);
+        p.x += q.x;
+        p.y += q.y;
+      }
       v[j] = p.x + p.y;
     }
     res[t] = reduce4_transposed(v[0], v[1], v[2], v[3]);
@@ -369,18 +382,37 @@ KD_DEV void stream_consume(const Plan& plan, StreamShared& sh, Issuer& iss, unsi
   for (int si = 0; si < nseg; ++si) {
     const Seg s = plan.segment(si);
     consume_segment<WT, AT>(plan, sh, iss, s, it, rb, err);
+    if (plan.wants_segment_done()) {
+      named_bar_sync(1, kThreads);  // every epilogue write of the segment is done
+      plan.segment_done(s);
+    }
   }
 }
 
-// Shared body of every streaming kernel.
+// Shared body of every streaming kernel.  With `weights_before_wait` the
+// first kStages stages are requested before the programmatic-launch wait:
+// only for plans whose segments are static weights known without reading
+// anything a preceding kernel writes (activations are read after the wait).
 template <int WT, int AT, class Plan>
-KD_DEV void stream_run(const Plan& plan, uint8_t* smem_raw, unsigned* err) {
+KD_DEV void stream_run(const Plan& plan, uint8_t* smem_raw, unsigned* err,
+                       bool weights_before_wait) {
   StreamShared sh = carve_stream_smem(smem_raw);
   Issuer iss;
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) mbar_init(&sh.full[i], 1);
     *sh.abort_flag = 0;
     fence_mbar_init();
+    if (weights_before_wait) {
+      iss.start(plan);
+      for (int i = 0; i < kStages; ++i)
+        if (!iss.next(plan, sh)) break;
+    }
+  }
+  if (weights_before_wait) {
+    pdl_wait();
+    pdl_launch_dependents();
+  }
+  if (threadIdx.x == 0 && !weights_before_wait) {
     iss.start(plan);
     for (int i = 0; i < kStages; ++i)
       if (!iss.next(plan, sh)) break;
