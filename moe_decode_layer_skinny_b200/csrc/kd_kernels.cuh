@@ -83,7 +83,6 @@ struct LayerDev {
   int* counts; int* offsets; int* perm; int* active; int* n_active;
   float* act; float* act_sh;               // [Mmax*k, I] by position, [Mmax, I] (fp32)
   float* yr; float* ysh;                   // [Mmax*k, H] by token*k+slot, [Mmax, H]
-  unsigned* counter;                       // router arrival counter (self-resetting)
   unsigned* hcnt;                          // [H/64] down rows done per block (self-resetting)
   unsigned* err;
 };
@@ -152,15 +151,13 @@ __global__ void __launch_bounds__(kThreads, 1) proj_kernel(LayerDev L, Acts a) {
 
 // ------------------------------------------------------------------ router
 
-// Logits: CTA b owns expert rows 2b and 2b+1; warp w takes row 2b + w/4 and
-// the (w%4)-th quarter of its columns.  Each lane issues all of its weight
-// loads (16 bytes each, up to 8) before using any, then forms partial dot
-// products with the fp32 h1 rows of 4 tokens at a time; the four quarters are
-// added in a fixed order.  The last CTA to finish (arrival counter) selects
-// the top-k of every token (descending logit, ties -> lower id), forms the
-// softmax renormalised over the selection and builds the per-expert lists:
-//   counts[e], offsets[e] (exclusive scan), perm[pos] = token*k + slot sorted
-//   by (expert, token*k + slot), active[a] = a-th expert with tokens, n_active.
+// Router logits l = Wr h1 + b from the fp32 h1: CTA b owns expert rows 2b and
+// 2b+1; warp w takes row 2b + w/4 and the (w%4)-th quarter of its columns.
+// Each lane loads its weight chunks (16 bytes each, up to 8) before waiting
+// for h1 (the router weights are static), then forms partial dot products
+// with the h1 rows of 4 tokens at a time; the four quarters are added in a
+// fixed order.  The selection itself (route_tokens) runs at the start of the
+// routed-expert kernel.
 constexpr int kRouterThreads = 256;
 constexpr int kRouterRows = 2;
 
@@ -253,32 +250,54 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(LayerDev L, int 
           (L.bias ? L.bias[e] : 0.f);
   }
 
-  // ---- last CTA: selection and dispatch
-  __shared__ unsigned s_ticket;
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) s_ticket = atomicAdd(L.counter, 1u);
-  __syncthreads();
-  if (s_ticket != gridDim.x - 1) return;
-  if (threadIdx.x == 0) *L.counter = 0u;  // ready for the next call / graph replay
-  __threadfence();
+}
 
-  __shared__ int s_sel[64 * 16];
-  __shared__ int s_cnt[1024];
-  __shared__ int s_off[1024];
-  __shared__ int s_wsum[2][kRouterThreads / 32];
+// ------------------------------------------------------------------ selection + dispatch
+
+// Routing of the call in shared memory, built by every routed-expert CTA from
+// the logits (redundantly: no grid-wide serialisation); CTA 0 also writes it
+// to global memory for the down kernel and for inspection.
+struct Route {
+  int* sel;      // [M*k] selected expert of (token, slot), descending logit
+  int* cnt;      // [E] tokens per expert
+  int* off;      // [E] exclusive scan of cnt
+  int* act;      // [E] active experts in id order
+  int* perm;     // [M*k] token*k + slot, sorted by (expert, token*k + slot)
+  int* n_act;    // [1]
+  int* wsum;     // [2][8] scan scratch
+};
+
+constexpr size_t kRouteSmemInts(int E, int Mk) { return (size_t)3 * E + 2 * Mk + 1 + 16; }
+
+KD_DEV Route carve_route(int* base, int E, int Mk) {
+  Route r;
+  r.sel = base;
+  r.perm = r.sel + Mk;
+  r.cnt = r.perm + Mk;
+  r.off = r.cnt + E;
+  r.act = r.off + E;
+  r.n_act = r.act + E;
+  r.wsum = r.n_act + 1;
+  return r;
+}
+
+// Top-k of every token (descending logit, ties -> lower expert id), the
+// softmax renormalised over the selection, and the per-expert token lists.
+KD_DEV void route_tokens(const LayerDev& L, int M, const Route& R, bool write_global) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nw = blockDim.x >> 5;
   const int k = L.k, E = L.E;
   // top-k: one warp per token; lane holds logits lane, lane+32, ...
-  for (int t = warp; t < M; t += kRouterThreads / 32) {
+  for (int t = warp; t < M; t += nw) {
     float lv[32];
     const int per = (E + 31) / 32;
 #pragma unroll
     for (int qq = 0; qq < 32; ++qq) {
       const int e = lane + 32 * qq;
-      lv[qq] = (qq < per && e < E) ? __ldcg(L.logits + (size_t)t * E + e) : -INFINITY;
+      lv[qq] = (qq < per && e < E) ? L.logits[(size_t)t * E + e] : -INFINITY;
     }
     unsigned taken = 0u;
-    float top = 0.f, den = 0.f, selv[16];
+    float top = 0.f, den = 0.f, mysel = 0.f;
     for (int j = 0; j < k; ++j) {
       float bv = -INFINITY;
       int be = 0x7fffffff;
@@ -298,34 +317,33 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(LayerDev L, int 
       }
       if ((be & 31) == lane) taken |= 1u << (be >> 5);
       if (j == 0) top = bv;
-      selv[j] = bv;
+      if (j == lane) mysel = bv;
       den += expf(bv - top);
-      if (lane == 0) s_sel[t * k + j] = be;
+      if (lane == 0) R.sel[t * k + j] = be;
     }
-    if (lane < k) {
-      float v = 0.f;
-      for (int j = 0; j < k; ++j) if (j == lane) v = selv[j];
-      L.idx[t * k + lane] = s_sel[t * k + lane];
-      L.gates[t * k + lane] = expf(v - top) / den;
+    __syncwarp();
+    if (write_global && lane < k) {
+      L.idx[t * k + lane] = R.sel[t * k + lane];
+      L.gates[t * k + lane] = expf(mysel - top) / den;
     }
   }
-  for (int e = threadIdx.x; e < E; e += kRouterThreads) s_cnt[e] = 0;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) R.cnt[e] = 0;
   __syncthreads();
   const int ncode = M * k;
-  for (int c = threadIdx.x; c < ncode; c += kRouterThreads) {
-    const int e = s_sel[c];
+  for (int c = threadIdx.x; c < ncode; c += blockDim.x) {
+    const int e = R.sel[c];
     if (e < 0 || e >= E) set_error(L.err, ERR_BAD_ROUTE);
-    else atomicAdd(&s_cnt[e], 1);
+    else atomicAdd(&R.cnt[e], 1);
   }
   __syncthreads();
-  // block-wide exclusive scans of counts and of (count > 0): each thread owns
-  // experts [4*tid, 4*tid+4)
+  // block-wide exclusive scans of cnt and of (cnt > 0): each thread owns
+  // experts [4*tid, 4*tid+4)  (E <= 4 * blockDim.x)
   {
     int c4[4], a4[4], cs = 0, as = 0;
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int e = 4 * threadIdx.x + u;
-      c4[u] = e < E ? s_cnt[e] : 0;
+      c4[u] = e < E ? R.cnt[e] : 0;
       a4[u] = c4[u] > 0;
       cs += c4[u];
       as += a4[u];
@@ -336,26 +354,32 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(LayerDev L, int 
       const int cv = __shfl_up_sync(0xffffffffu, ci, o), av = __shfl_up_sync(0xffffffffu, ai, o);
       if (lane >= o) { ci += cv; ai += av; }
     }
-    if (lane == 31) { s_wsum[0][warp] = ci; s_wsum[1][warp] = ai; }
+    if (lane == 31) { R.wsum[warp] = ci; R.wsum[8 + warp] = ai; }
     __syncthreads();
     int cb = 0, ab = 0;
-    for (int w2 = 0; w2 < warp; ++w2) { cb += s_wsum[0][w2]; ab += s_wsum[1][w2]; }
+    for (int w2 = 0; w2 < warp; ++w2) { cb += R.wsum[w2]; ab += R.wsum[8 + w2]; }
     int run = cb + ci - cs, arun = ab + ai - as;
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int e = 4 * threadIdx.x + u;
       if (e < E) {
-        s_off[e] = run;
-        L.counts[e] = c4[u];
-        L.offsets[e] = run;
-        if (a4[u]) L.active[arun] = e;
+        R.off[e] = run;
+        if (a4[u]) R.act[arun] = e;
+        if (write_global) {
+          L.counts[e] = c4[u];
+          L.offsets[e] = run;
+          if (a4[u]) L.active[arun] = e;
+        }
       }
       run += c4[u];
       arun += a4[u];
     }
-    if (threadIdx.x == kRouterThreads - 1) {
-      L.offsets[E] = run;
-      *L.n_active = arun;
+    if (threadIdx.x == blockDim.x - 1) {
+      *R.n_act = arun;
+      if (write_global) {
+        L.offsets[E] = run;
+        *L.n_active = arun;
+      }
     }
   }
   __syncthreads();
@@ -363,15 +387,23 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(LayerDev L, int 
   if (warp == 0) {
     for (int c0 = 0; c0 < ncode; c0 += 32) {
       const int c = c0 + lane;
-      const int e = c < ncode ? s_sel[c] : -1 - lane;  // unique dummies
+      const int e = c < ncode ? R.sel[c] : -1 - lane;  // unique dummies
       const unsigned same = __match_any_sync(0xffffffffu, e);
       const int rank = __popc(same & ((1u << lane) - 1u));
-      if (c < ncode && e >= 0 && e < E) L.perm[s_off[e] + rank] = c;
+      const int base = (c < ncode && e >= 0 && e < E) ? R.off[e] : 0;
       __syncwarp();
-      if (c < ncode && e >= 0 && e < E && rank == 0) s_off[e] += __popc(same);
+      if (c < ncode && e >= 0 && e < E) {
+        R.perm[base + rank] = c;
+        if (write_global) L.perm[base + rank] = c;
+        if (rank == 0) R.off[e] = base + __popc(same);
+      }
       __syncwarp();
     }
   }
+  __syncthreads();
+  // restore the exclusive offsets (the walk advanced them to the ends)
+  for (int e = threadIdx.x; e < E; e += blockDim.x) R.off[e] -= R.cnt[e];
+  __syncthreads();
 }
 
 // ------------------------------------------------------------------ experts
@@ -394,6 +426,7 @@ struct ExpertRange {
 
 struct GateUpPlan {
   const LayerDev* L; int M; bool shared; ExpertRange R;
+  Route rt;                      // routing of the call (shared memory)
   KD_DEV int num_segments() const { return R.num_segments(); }
   KD_DEV Seg segment(int i) const {
     int a, u0, u1;
@@ -404,9 +437,9 @@ struct GateUpPlan {
     if (shared) {
       s.tag = -1; s.w = L->wgu_sh; s.tok0 = 0; s.ntok = M;
     } else {
-      const int e = L->active[a];
+      const int e = rt.act[a];
       s.tag = e; s.w = L->wgu + (size_t)e * estride;
-      s.tok0 = L->offsets[e]; s.ntok = L->counts[e];
+      s.tok0 = rt.off[e]; s.ntok = rt.cnt[e];
     }
     s.w += (size_t)(2 * u0) * s.row_bytes;
     s.row0 = 2 * u0;
@@ -414,7 +447,7 @@ struct GateUpPlan {
     return s;
   }
   KD_DEV const void* act_row(const Seg& s, int j) const {
-    const int t = shared ? j : L->perm[s.tok0 + j] / L->k;
+    const int t = shared ? j : rt.perm[s.tok0 + j] / L->k;
     return L->h1f + (size_t)t * L->H;
   }
   KD_DEV const float* scale_row(const Seg& s, int prow) const {
@@ -527,11 +560,14 @@ __global__ void __launch_bounds__(kThreads, 1) gateup_kernel(LayerDev L, int M, 
   extern __shared__ uint8_t smem[];
   GateUpPlan p;
   p.L = &L; p.M = M; p.shared = shared != 0;
+  int n_act = 1;
   if (!shared) {
     pdl_wait();
     pdl_launch_dependents();
+    p.rt = carve_route(reinterpret_cast<int*>(smem + kStreamSmem), L.E, M * L.k);
+    route_tokens(L, M, p.rt, blockIdx.x == 0);
+    n_act = *p.rt.n_act;
   }
-  const int n_act = shared ? 1 : *(volatile int*)L.n_active;
   p.R = expert_range(n_act, L.I);
   stream_run<WT, A_F32>(p, smem, L.err, shared != 0);
 }

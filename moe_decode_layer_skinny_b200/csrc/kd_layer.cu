@@ -114,9 +114,15 @@ static void free_layer(kd_layer* L) {
 
 static bool stream_kernels_configured = false;
 
+// Routed gate/up CTAs keep the call's routing after the stream area.
+static size_t gateup_smem(const LayerDev& d, int M) {
+  return kStreamSmem + 16 + sizeof(int) * kRouteSmemInts(d.E, M * d.k);
+}
+static const size_t kMaxGateupSmem = kStreamSmem + 16 + sizeof(int) * kRouteSmemInts(1024, 64 * 16);
+
 static int configure_kernels() {
   if (stream_kernels_configured) return KD_OK;
-  const int smem = (int)kStreamSmem;
+  const int smem = (int)kMaxGateupSmem;
   KD_CUDA(cudaFuncSetAttribute(proj_kernel<W_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   KD_CUDA(cudaFuncSetAttribute(proj_kernel<W_FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   KD_CUDA(cudaFuncSetAttribute(gateup_kernel<W_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
@@ -239,11 +245,9 @@ extern "C" int kd_layer_create(const kd_config* cfg, uint64_t seed, kd_layer** o
   TRY(dalloc_t(L, (size_t)M * I, &d.act_sh));
   TRY(dalloc_t(L, (size_t)M * k * H, &d.yr));
   TRY(dalloc_t(L, (size_t)M * H, &d.ysh));
-  TRY(dalloc_t(L, 1, &d.counter));
   TRY(dalloc_t(L, (size_t)H / 64, &d.hcnt));
   TRYC(cudaMemset(d.hcnt, 0, sizeof(unsigned) * (H / 64)));
   TRY(dalloc_t(L, 1, &d.err));
-  TRYC(cudaMemset(d.counter, 0, sizeof(unsigned)));
   TRYC(cudaMemset(d.err, 0, sizeof(unsigned)));
   TRYC(cudaMemset(d.n_active, 0, sizeof(int)));
   TRYC(cudaMemset(d.ysh, 0, sizeof(float) * (size_t)M * H));
@@ -350,8 +354,8 @@ static int launch_layer(kd_layer* L, void* hidden, const void* attn, int M, cuda
     KD_CUDA(cudaEventRecord(L->ev_sh, L->side));
   }
   if (L->timing) KD_CUDA(cudaEventRecord(L->tev[2], s));
-  KD_CUDA(launch(fp8 ? gateup_kernel<W_FP8> : gateup_kernel<W_BF16>, G, kThreads, sm, s,
-                 !L->timing, d, M, 0));
+  KD_CUDA(launch(fp8 ? gateup_kernel<W_FP8> : gateup_kernel<W_BF16>, G, kThreads,
+                 gateup_smem(d, M), s, !L->timing, d, M, 0));
   if (L->timing) KD_CUDA(cudaEventRecord(L->tev[3], s));
   if (d.S) KD_CUDA(cudaStreamWaitEvent(s, L->ev_sh, 0));
   if (next && pf) {
@@ -377,7 +381,6 @@ extern "C" int kd_layer_check(kd_layer* L) {
   if (e == 0) return KD_OK;
   KD_CUDA(cudaMemset(L->d.err, 0, sizeof(unsigned)));
   // an aborted call may have left arrival counters part-way
-  KD_CUDA(cudaMemset(L->d.counter, 0, sizeof(unsigned)));
   KD_CUDA(cudaMemset(L->d.hcnt, 0, sizeof(unsigned) * (L->d.H / 64)));
   if (e & (ERR_WAIT_FULL | ERR_WAIT_EMPTY | ERR_WAIT_MMA))
     return fail(KD_ETIMEOUT, "device: a bounded wait gave up (flags %s0x%lx)", "", (long)e);
