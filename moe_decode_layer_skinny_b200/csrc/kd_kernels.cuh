@@ -264,10 +264,10 @@ struct Route {
   int* act;      // [E] active experts in id order
   int* perm;     // [M*k] token*k + slot, sorted by (expert, token*k + slot)
   int* n_act;    // [1]
-  int* wsum;     // [2][8] scan scratch
+  int* wsum;     // [2][32] scan scratch
 };
 
-constexpr size_t kRouteSmemInts(int E, int Mk) { return (size_t)3 * E + 2 * Mk + 1 + 16; }
+constexpr size_t kRouteSmemInts(int E, int Mk) { return (size_t)3 * E + 2 * Mk + 1 + 64; }
 
 KD_DEV Route carve_route(int* base, int E, int Mk) {
   Route r;
@@ -354,10 +354,10 @@ KD_DEV void route_tokens(const LayerDev& L, int M, const Route& R, bool write_gl
       const int cv = __shfl_up_sync(0xffffffffu, ci, o), av = __shfl_up_sync(0xffffffffu, ai, o);
       if (lane >= o) { ci += cv; ai += av; }
     }
-    if (lane == 31) { R.wsum[warp] = ci; R.wsum[8 + warp] = ai; }
+    if (lane == 31) { R.wsum[warp] = ci; R.wsum[32 + warp] = ai; }
     __syncthreads();
     int cb = 0, ab = 0;
-    for (int w2 = 0; w2 < warp; ++w2) { cb += R.wsum[w2]; ab += R.wsum[8 + w2]; }
+    for (int w2 = 0; w2 < warp; ++w2) { cb += R.wsum[w2]; ab += R.wsum[32 + w2]; }
     int run = cb + ci - cs, arun = ab + ai - as;
 #pragma unroll
     for (int u = 0; u < 4; ++u) {

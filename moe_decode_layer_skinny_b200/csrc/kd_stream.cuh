@@ -1,6 +1,6 @@
 // kd_stream.cuh -- weight-streaming GEMV engine on CUDA cores.
 //
-// One CTA of eight warps per SM.  Contiguous runs of weight rows stream from
+// One CTA of sixteen warps per SM.  Contiguous runs of weight rows stream from
 // HBM into a ring of shared-memory stages with 1-D bulk TMA copies
 // (cp.async.bulk, completion counted on one mbarrier per stage).  Each stage
 // holds several whole rows; a warp owns one column slice of a subset of them,
@@ -22,14 +22,14 @@
 
 namespace kd {
 
-constexpr int kCW = 8;                        // warps per CTA = column slices per row
+constexpr int kCW = 16;                       // warps per CTA (max column slices per row)
 constexpr int kThreads = kCW * 32;
 constexpr int kStageBytes = 57344;            // 56 KB: 4 rows of 7168 bf16
 constexpr int kStages = 3;
 constexpr int kMaxRps = 64;                   // rows per stage cap
 constexpr int kTT = 4;                        // tokens per register pass
 constexpr int kRedFloats = kMaxRps * kCW * kTT;   // [row][slice][token], S*rows <= 8*rps
-constexpr int kMaxChunksLane = 4;             // 16-byte chunks per lane per row (K <= 8192 bf16)
+constexpr int kMaxChunksLane = 2;             // 16-byte chunks per lane per row slice
 constexpr size_t kStreamSmem =
     (size_t)kStages * kStageBytes + 2 * kRedFloats * sizeof(float) + kStages * 8 + 16 + 128;
 
@@ -39,7 +39,7 @@ enum AType { A_BF16 = 0, A_F32 = 1 };
 template <int WT>
 struct WTraits {
   static constexpr int EPC = WT == W_BF16 ? 8 : 16;   // elements per 16-byte chunk
-  static constexpr int TT = WT == W_BF16 ? 4 : 2;     // tokens held in registers at once
+  static constexpr int TT = 2;                        // tokens held in registers at once
 };
 
 // One run of rows.  Rows are contiguous in memory (row stride = row_bytes).
@@ -142,7 +142,7 @@ struct Issuer {
 //
 // Geometry of a segment: each row is cut into S column slices (the smallest
 // power of two that leaves <= 32*kMaxChunksLane 16-byte chunks per slice);
-// warp w takes slice w % S of rows w / S, w / S + G, ... (G = 8 / S row
+// warp w takes slice w % S of rows w / S, w / S + G, ... (G = 16 / S row
 // groups).  A warp handles its rows four at a time and reduces the four
 // partial sums across its lanes together (a transposing butterfly: 6 shuffles
 // instead of 20).
