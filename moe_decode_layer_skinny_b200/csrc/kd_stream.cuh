@@ -24,6 +24,7 @@ namespace kd {
 
 constexpr int kCW = 16;                       // warps per CTA (max column slices per row)
 constexpr int kThreads = kCW * 32;
+constexpr int kIssuer = kThreads - 32;        // lane 0 of the last warp issues the bulk copies
 constexpr int kStageBytes = 57344;            // 56 KB: 4 rows of 7168 bf16
 constexpr int kStages = 3;
 constexpr int kMaxRps = 64;                   // rows per stage cap
@@ -293,28 +294,36 @@ KD_DEV void batch_dot(const Plan& plan, const Seg& s, int stage_row0, const uint
 }
 
 // After every warp wrote its partials of a stage into `red` ([row][slice][t]):
-// sum the S slices in a fixed order and run the epilogue.
+// add the S slices of each (row, token) with a fixed shuffle tree over S
+// consecutive lanes (S is a power of two <= 16) and run the epilogue.  Paired
+// plans first park the sums at the top of `red` (above every partial: rows *
+// slices <= 112 here) and then combine (gate, up) rows.
 template <class Plan>
-KD_DEV void stage_epilogue(const Plan& plan, const Seg& s, const float* red, int n, int S,
+KD_DEV void stage_epilogue(const Plan& plan, const Seg& s, float* red, int n, int S,
                            int stage_row0, int tok, int nt) {
   const int ctid = threadIdx.x;
-  if (plan.paired()) {
+  const bool paired = plan.paired();
+  const int nsum = n * nt;
+  float* sums = red + kRedFloats - nsum;
+  for (int base = 0; base < nsum * S; base += kThreads) {
+    const int q = base + ctid;
+    const bool live = q < nsum * S;
+    const int idx = q / S, sl = q % S;                // sum index (row * nt + j), slice
+    const int row = idx / nt, j = idx % nt;
+    float v = live ? red[(row * S + sl) * kTT + j] : 0.f;
+    for (int o = S >> 1; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (live && sl == 0) {
+      if (paired) sums[idx] = v;
+      else plan.epilogue(s, s.row0 + stage_row0 + row, tok + j, v);
+    }
+  }
+  if (paired) {
+    named_bar_sync(2, kThreads);
     const int npair = n >> 1;
     for (int q = ctid; q < npair * nt; q += kThreads) {
       const int p = q / nt, j = q % nt;
-      float g = 0.f, u = 0.f;
-      for (int sl = 0; sl < S; ++sl) {
-        g += red[((2 * p) * S + sl) * kTT + j];
-        u += red[((2 * p + 1) * S + sl) * kTT + j];
-      }
-      plan.epilogue2(s, (s.row0 + stage_row0) / 2 + p, tok + j, g, u);
-    }
-  } else {
-    for (int q = ctid; q < n * nt; q += kThreads) {
-      const int row = q / nt, j = q % nt;
-      float v = 0.f;
-      for (int sl = 0; sl < S; ++sl) v += red[(row * S + sl) * kTT + j];
-      plan.epilogue(s, s.row0 + stage_row0 + row, tok + j, v);
+      plan.epilogue2(s, (s.row0 + stage_row0) / 2 + p, tok + j, sums[(2 * p) * nt + j],
+                     sums[(2 * p + 1) * nt + j]);
     }
   }
 }
@@ -363,13 +372,14 @@ KD_DEV void consume_segment(const Plan& plan, StreamShared& sh, Issuer& iss, con
       }
       named_bar_sync(1, kThreads);
       // after the stage's last token group no thread reads it again: refill
-      if (threadIdx.x == 0 && tok + TT >= s.ntok) iss.next(plan, sh);
+      // (from the last warp, which has no epilogue work when rows are few)
+      if (threadIdx.x == kIssuer && tok + TT >= s.ntok) iss.next(plan, sh);
       stage_epilogue(plan, s, red, n, S, r0, tok, nt);
       rb ^= 1;
     }
     if (s.ntok == 0) {
       named_bar_sync(1, kThreads);
-      if (threadIdx.x == 0) iss.next(plan, sh);
+      if (threadIdx.x == kIssuer) iss.next(plan, sh);
     }
   }
 }
@@ -398,7 +408,7 @@ KD_DEV void stream_run(const Plan& plan, uint8_t* smem_raw, unsigned* err,
                        bool weights_before_wait) {
   StreamShared sh = carve_stream_smem(smem_raw);
   Issuer iss;
-  if (threadIdx.x == 0) {
+  if (threadIdx.x == kIssuer) {
     for (int i = 0; i < kStages; ++i) mbar_init(&sh.full[i], 1);
     *sh.abort_flag = 0;
     fence_mbar_init();
@@ -412,7 +422,7 @@ KD_DEV void stream_run(const Plan& plan, uint8_t* smem_raw, unsigned* err,
     pdl_wait();
     pdl_launch_dependents();
   }
-  if (threadIdx.x == 0 && !weights_before_wait) {
+  if (threadIdx.x == kIssuer && !weights_before_wait) {
     iss.start(plan);
     for (int i = 0; i < kStages; ++i)
       if (!iss.next(plan, sh)) break;
