@@ -32,7 +32,7 @@ constexpr int kTT = 4;                        // tokens per register pass
 constexpr int kRedFloats = kMaxRps * kCW * kTT;   // [row][slice][token], S*rows <= 8*rps
 constexpr int kMaxChunksLane = 2;             // 16-byte chunks per lane per row slice
 constexpr size_t kStreamSmem =
-    (size_t)kStages * kStageBytes + 2 * kRedFloats * sizeof(float) + kStages * 8 + 16 + 128;
+    (size_t)kStages * kStageBytes + 2 * kRedFloats * sizeof(float) + 2 * kStages * 8 + 16 + 128;
 
 enum WType { W_BF16 = 0, W_FP8 = 1 };
 enum AType { A_BF16 = 0, A_F32 = 1 };
@@ -57,6 +57,7 @@ struct StreamShared {
   uint8_t* stage;       // kStages * kStageBytes
   float* red;           // [2][kRedFloats]
   uint64_t* full;       // [kStages] stage landed (bulk-copy byte count)
+  uint64_t* empty;      // [kStages] every warp finished reading the stage
   int* abort_flag;
 };
 
@@ -68,7 +69,8 @@ KD_DEV StreamShared carve_stream_smem(uint8_t* base) {
   s.red = reinterpret_cast<float*>(p);
   p += 2 * kRedFloats * sizeof(float);
   s.full = reinterpret_cast<uint64_t*>(p);
-  s.abort_flag = reinterpret_cast<int*>(s.full + kStages);
+  s.empty = s.full + kStages;
+  s.abort_flag = reinterpret_cast<int*>(s.empty + kStages);
   return s;
 }
 
@@ -303,13 +305,14 @@ KD_DEV void stage_epilogue(const Plan& plan, const Seg& s, float* red, int n, in
                            int stage_row0, int tok, int nt) {
   const int ctid = threadIdx.x;
   const bool paired = plan.paired();
-  const int nsum = n * nt;
+  const int nsum = n * nt;                            // nt is 1 or 2
+  const int sshift = 31 - __clz(S);
   float* sums = red + kRedFloats - nsum;
   for (int base = 0; base < nsum * S; base += kThreads) {
     const int q = base + ctid;
     const bool live = q < nsum * S;
-    const int idx = q / S, sl = q % S;                // sum index (row * nt + j), slice
-    const int row = idx / nt, j = idx % nt;
+    const int idx = q >> sshift, sl = q & (S - 1);    // sum index (row * nt + j), slice
+    const int row = nt == 1 ? idx : idx >> 1, j = nt == 1 ? 0 : idx & 1;
     float v = live ? red[(row * S + sl) * kTT + j] : 0.f;
     for (int o = S >> 1; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     if (live && sl == 0) {
@@ -321,11 +324,26 @@ KD_DEV void stage_epilogue(const Plan& plan, const Seg& s, float* red, int n, in
     named_bar_sync(2, kThreads);
     const int npair = n >> 1;
     for (int q = ctid; q < npair * nt; q += kThreads) {
-      const int p = q / nt, j = q % nt;
+      const int p = nt == 1 ? q : q >> 1, j = nt == 1 ? 0 : q & 1;
       plan.epilogue2(s, (s.row0 + stage_row0) / 2 + p, tok + j, sums[(2 * p) * nt + j],
                      sums[(2 * p + 1) * nt + j]);
     }
   }
+}
+
+// A warp is done reading a stage: count it on the stage's "empty" barrier.
+// The issuing lane waits for all warps and refills the slot at once, without
+// waiting for the reductions and the epilogue of the stage.
+template <class Plan>
+KD_DEV void release_stage(const Plan& plan, StreamShared& sh, Issuer& iss, int slot, uint32_t ph,
+                          unsigned* err) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(&sh.empty[slot]);
+  if (threadIdx.x == kIssuer) {
+    wait_or_abort(&sh.empty[slot], ph, sh.abort_flag, err, ERR_WAIT_EMPTY);
+    iss.next(plan, sh);
+  }
+  __syncwarp();  // the issuing lane rejoins its warp before any CTA barrier
 }
 
 // One segment.  Tokens are processed TT at a time (4 for bf16 weights, 2 for
@@ -370,17 +388,12 @@ KD_DEV void consume_segment(const Plan& plan, StreamShared& sh, Issuer& iss, con
             if (t < nt) red[(myrow * S + my_slice) * kTT + t] = res[t];
         }
       }
+      if (tok + TT >= s.ntok) release_stage(plan, sh, iss, slot, ph, err);
       named_bar_sync(1, kThreads);
-      // after the stage's last token group no thread reads it again: refill
-      // (from the last warp, which has no epilogue work when rows are few)
-      if (threadIdx.x == kIssuer && tok + TT >= s.ntok) iss.next(plan, sh);
       stage_epilogue(plan, s, red, n, S, r0, tok, nt);
       rb ^= 1;
     }
-    if (s.ntok == 0) {
-      named_bar_sync(1, kThreads);
-      if (threadIdx.x == kIssuer) iss.next(plan, sh);
-    }
+    if (s.ntok == 0) release_stage(plan, sh, iss, slot, ph, err);
   }
 }
 
@@ -409,7 +422,10 @@ KD_DEV void stream_run(const Plan& plan, uint8_t* smem_raw, unsigned* err,
   StreamShared sh = carve_stream_smem(smem_raw);
   Issuer iss;
   if (threadIdx.x == kIssuer) {
-    for (int i = 0; i < kStages; ++i) mbar_init(&sh.full[i], 1);
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&sh.full[i], 1);
+      mbar_init(&sh.empty[i], kCW);
+    }
     *sh.abort_flag = 0;
     fence_mbar_init();
     if (weights_before_wait) {
