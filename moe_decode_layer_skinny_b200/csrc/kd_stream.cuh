@@ -29,10 +29,12 @@ constexpr int kStageBytes = 57344;            // 56 KB: 4 rows of 7168 bf16
 constexpr int kStages = 3;
 constexpr int kMaxRps = 64;                   // rows per stage cap
 constexpr int kTT = 4;                        // tokens per register pass
-constexpr int kRedFloats = kMaxRps * kCW * kTT;   // [row][slice][token], S*rows <= 8*rps
+constexpr int kRedFloats = 1024;              // [row][slice][token]: rows*slices <= 112, + parked sums
+constexpr int kSumCap = 2048;                 // reduced (row, token) sums held until the epilogue
 constexpr int kMaxChunksLane = 2;             // 16-byte chunks per lane per row slice
 constexpr size_t kStreamSmem =
-    (size_t)kStages * kStageBytes + 2 * kRedFloats * sizeof(float) + 2 * kStages * 8 + 16 + 128;
+    (size_t)kStages * kStageBytes + (2 * kRedFloats + kSumCap) * sizeof(float) + 2 * kStages * 8 +
+    16 + 128;
 
 enum WType { W_BF16 = 0, W_FP8 = 1 };
 enum AType { A_BF16 = 0, A_F32 = 1 };
@@ -56,6 +58,7 @@ struct Seg {
 struct StreamShared {
   uint8_t* stage;       // kStages * kStageBytes
   float* red;           // [2][kRedFloats]
+  float* sums;          // [kSumCap] reduced sums of the rows since the last epilogue
   uint64_t* full;       // [kStages] stage landed (bulk-copy byte count)
   uint64_t* empty;      // [kStages] every warp finished reading the stage
   int* abort_flag;
@@ -68,6 +71,8 @@ KD_DEV StreamShared carve_stream_smem(uint8_t* base) {
   p += (size_t)kStages * kStageBytes;
   s.red = reinterpret_cast<float*>(p);
   p += 2 * kRedFloats * sizeof(float);
+  s.sums = reinterpret_cast<float*>(p);
+  p += kSumCap * sizeof(float);
   s.full = reinterpret_cast<uint64_t*>(p);
   s.empty = s.full + kStages;
   s.abort_flag = reinterpret_cast<int*>(s.empty + kStages);
@@ -297,36 +302,37 @@ KD_DEV void batch_dot(const Plan& plan, const Seg& s, int stage_row0, const uint
 
 // After every warp wrote its partials of a stage into `red` ([row][slice][t]):
 // add the S slices of each (row, token) with a fixed shuffle tree over S
-// consecutive lanes (S is a power of two <= 16) and run the epilogue.  Paired
-// plans first park the sums at the top of `red` (above every partial: rows *
-// slices <= 112 here) and then combine (gate, up) rows.
-template <class Plan>
-KD_DEV void stage_epilogue(const Plan& plan, const Seg& s, float* red, int n, int S,
-                           int stage_row0, int tok, int nt) {
-  const int ctid = threadIdx.x;
-  const bool paired = plan.paired();
+// consecutive lanes (S is a power of two <= 16) into dst[row * nt + j].
+KD_DEV void reduce_slices(const float* red, float* dst, int n, int S, int nt) {
   const int nsum = n * nt;                            // nt is 1 or 2
   const int sshift = 31 - __clz(S);
-  float* sums = red + kRedFloats - nsum;
   for (int base = 0; base < nsum * S; base += kThreads) {
-    const int q = base + ctid;
+    const int q = base + threadIdx.x;
     const bool live = q < nsum * S;
     const int idx = q >> sshift, sl = q & (S - 1);    // sum index (row * nt + j), slice
     const int row = nt == 1 ? idx : idx >> 1, j = nt == 1 ? 0 : idx & 1;
     float v = live ? red[(row * S + sl) * kTT + j] : 0.f;
     for (int o = S >> 1; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if (live && sl == 0) {
-      if (paired) sums[idx] = v;
-      else plan.epilogue(s, s.row0 + stage_row0 + row, tok + j, v);
-    }
+    if (live && sl == 0) dst[idx] = v;
   }
-  if (paired) {
-    named_bar_sync(2, kThreads);
+}
+
+// Epilogue of `n` consecutive rows starting at segment row `row0` whose sums
+// are sums[row * nt + j] (rows relative to row0), tokens tok .. tok+nt-1.
+template <class Plan>
+KD_DEV void run_epilogue(const Plan& plan, const Seg& s, const float* sums, int row0, int n,
+                         int tok, int nt) {
+  if (plan.paired()) {
     const int npair = n >> 1;
-    for (int q = ctid; q < npair * nt; q += kThreads) {
+    for (int q = threadIdx.x; q < npair * nt; q += kThreads) {
       const int p = nt == 1 ? q : q >> 1, j = nt == 1 ? 0 : q & 1;
-      plan.epilogue2(s, (s.row0 + stage_row0) / 2 + p, tok + j, sums[(2 * p) * nt + j],
+      plan.epilogue2(s, (s.row0 + row0) / 2 + p, tok + j, sums[(2 * p) * nt + j],
                      sums[(2 * p + 1) * nt + j]);
+    }
+  } else {
+    for (int q = threadIdx.x; q < n * nt; q += kThreads) {
+      const int row = nt == 1 ? q : q >> 1, j = nt == 1 ? 0 : q & 1;
+      plan.epilogue(s, s.row0 + row0 + row, tok + j, sums[q]);
     }
   }
 }
@@ -346,10 +352,13 @@ KD_DEV void release_stage(const Plan& plan, StreamShared& sh, Issuer& iss, int s
   __syncwarp();  // the issuing lane rejoins its warp before any CTA barrier
 }
 
-// One segment.  Tokens are processed TT at a time (4 for bf16 weights, 2 for
-// FP8): with at most TT tokens (the common case) their activations are loaded
-// once for the whole segment; with more, the stage is swept once per group of
-// TT tokens, reloading the activations (through L1) for every group.
+// One segment.  Tokens are processed TT (= 2) at a time.  With at most TT
+// tokens (the common case) their activations are loaded once for the whole
+// segment and the reduced sums of consecutive stages are held in shared
+// memory, so the epilogue (and any global loads it makes) runs once per
+// kSumCap sums instead of once per stage.  With more tokens the stage is
+// swept once per group of TT tokens, reloading the activations (through L1)
+// for every group, and each group's epilogue runs at once.
 template <int WT, int AT, class Plan>
 KD_DEV void consume_segment(const Plan& plan, StreamShared& sh, Issuer& iss, const Seg& s,
                             uint32_t& it, int& rb, unsigned* err) {
@@ -363,6 +372,7 @@ KD_DEV void consume_segment(const Plan& plan, StreamShared& sh, Issuer& iss, con
   ActRegs<WT> areg;
   const bool single_pass = s.ntok <= TT;
   if (single_pass) load_act_regs<WT, AT>(plan, s, 0, s.ntok, slice0, cpl, areg);
+  int held0 = 0;  // first segment row whose sums wait in sh.sums (single pass)
   for (int r0 = 0; r0 < s.nrows; r0 += rps, ++it) {
     const int n = s.nrows - r0 < rps ? s.nrows - r0 : rps;
     const int slot = it % kStages;
@@ -379,7 +389,6 @@ KD_DEV void consume_segment(const Plan& plan, StreamShared& sh, Issuer& iss, con
         for (int j = 0; j < 4; ++j) rows[j] = rbase + j * G < n ? rbase + j * G : -1;
         float res[kTT];
         if (nt == 1) batch_dot<WT, 1>(plan, s, r0, st, rows, slice0, cpl, areg, res);
-        else if (TT == 2 || nt == 2) batch_dot<WT, 2>(plan, s, r0, st, rows, slice0, cpl, areg, res);
         else batch_dot<WT, TT>(plan, s, r0, st, rows, slice0, cpl, areg, res);
         const int myrow = rbase + ((lane >> 3) & 3) * G;   // the row this lane's sums belong to
         if ((lane & 7) == 0 && myrow < n) {
@@ -390,7 +399,21 @@ KD_DEV void consume_segment(const Plan& plan, StreamShared& sh, Issuer& iss, con
       }
       if (tok + TT >= s.ntok) release_stage(plan, sh, iss, slot, ph, err);
       named_bar_sync(1, kThreads);
-      stage_epilogue(plan, s, red, n, S, r0, tok, nt);
+      if (single_pass) {
+        reduce_slices(red, sh.sums + (r0 - held0) * nt, n, S, nt);
+        const bool last = r0 + rps >= s.nrows;
+        if (last || (r0 + n + rps - held0) * nt > kSumCap) {
+          named_bar_sync(1, kThreads);
+          run_epilogue(plan, s, sh.sums, held0, r0 + n - held0, 0, nt);
+          named_bar_sync(1, kThreads);  // sums are reused from the start
+          held0 = r0 + n;
+        }
+      } else {
+        float* dst = red + kRedFloats - n * nt;   // above every partial of the stage
+        reduce_slices(red, dst, n, S, nt);
+        named_bar_sync(1, kThreads);
+        run_epilogue(plan, s, dst, r0, n, tok, nt);
+      }
       rb ^= 1;
     }
     if (s.ntok == 0) release_stage(plan, sh, iss, slot, ph, err);
