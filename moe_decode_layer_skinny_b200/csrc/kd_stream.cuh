@@ -29,12 +29,10 @@ constexpr int kStageBytes = 57344;            // 56 KB: 4 rows of 7168 bf16
 constexpr int kStages = 3;
 constexpr int kMaxRps = 64;                   // rows per stage cap
 constexpr int kTT = 4;                        // tokens per register pass
-constexpr int kRedFloats = 1024;              // [row][slice][token]: rows*slices <= 112, + parked sums
-constexpr int kSumCap = 2048;                 // reduced (row, token) sums held until the epilogue
+constexpr int kPartCap = 8192;                // per-warp partial sums held until the epilogue
 constexpr int kMaxChunksLane = 2;             // 16-byte chunks per lane per row slice
 constexpr size_t kStreamSmem =
-    (size_t)kStages * kStageBytes + (2 * kRedFloats + kSumCap) * sizeof(float) + 2 * kStages * 8 +
-    16 + 128;
+    (size_t)kStages * kStageBytes + kPartCap * sizeof(float) + 2 * kStages * 8 + 16 + 128;
 
 enum WType { W_BF16 = 0, W_FP8 = 1 };
 enum AType { A_BF16 = 0, A_F32 = 1 };
@@ -57,8 +55,7 @@ struct Seg {
 
 struct StreamShared {
   uint8_t* stage;       // kStages * kStageBytes
-  float* red;           // [2][kRedFloats]
-  float* sums;          // [kSumCap] reduced sums of the rows since the last epilogue
+  float* part;          // [kPartCap] partials [row][slice][token] since the last epilogue
   uint64_t* full;       // [kStages] stage landed (bulk-copy byte count)
   uint64_t* empty;      // [kStages] every warp finished reading the stage
   int* abort_flag;
@@ -69,10 +66,8 @@ KD_DEV StreamShared carve_stream_smem(uint8_t* base) {
   uintptr_t p = (reinterpret_cast<uintptr_t>(base) + 127) & ~uintptr_t(127);
   s.stage = reinterpret_cast<uint8_t*>(p);
   p += (size_t)kStages * kStageBytes;
-  s.red = reinterpret_cast<float*>(p);
-  p += 2 * kRedFloats * sizeof(float);
-  s.sums = reinterpret_cast<float*>(p);
-  p += kSumCap * sizeof(float);
+  s.part = reinterpret_cast<float*>(p);
+  p += kPartCap * sizeof(float);
   s.full = reinterpret_cast<uint64_t*>(p);
   s.empty = s.full + kStages;
   s.abort_flag = reinterpret_cast<int*>(s.empty + kStages);
@@ -300,39 +295,28 @@ KD_DEV void batch_dot(const Plan& plan, const Seg& s, int stage_row0, const uint
   }
 }
 
-// After every warp wrote its partials of a stage into `red` ([row][slice][t]):
-// add the S slices of each (row, token) with a fixed shuffle tree over S
-// consecutive lanes (S is a power of two <= 16) into dst[row * nt + j].
-KD_DEV void reduce_slices(const float* red, float* dst, int n, int S, int nt) {
-  const int nsum = n * nt;                            // nt is 1 or 2
-  const int sshift = 31 - __clz(S);
-  for (int base = 0; base < nsum * S; base += kThreads) {
-    const int q = base + threadIdx.x;
-    const bool live = q < nsum * S;
-    const int idx = q >> sshift, sl = q & (S - 1);    // sum index (row * nt + j), slice
-    const int row = nt == 1 ? idx : idx >> 1, j = nt == 1 ? 0 : idx & 1;
-    float v = live ? red[(row * S + sl) * kTT + j] : 0.f;
-    for (int o = S >> 1; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if (live && sl == 0) dst[idx] = v;
-  }
-}
-
-// Epilogue of `n` consecutive rows starting at segment row `row0` whose sums
-// are sums[row * nt + j] (rows relative to row0), tokens tok .. tok+nt-1.
+// Epilogue of `n` consecutive rows starting at segment row `row0`, whose lane-
+// reduced partials are part[(row * S + slice) * nt + j] (rows relative to
+// row0): each sum adds its S slices in a fixed order (deterministic).
 template <class Plan>
-KD_DEV void run_epilogue(const Plan& plan, const Seg& s, const float* sums, int row0, int n,
-                         int tok, int nt) {
+KD_DEV void reduce_epilogue(const Plan& plan, const Seg& s, const float* part, int row0, int n,
+                            int S, int tok, int nt) {
+  auto sum = [&](int row, int j) {
+    const float* p = part + (size_t)row * S * nt + j;
+    float v = 0.f;
+    for (int sl = 0; sl < S; ++sl) v += p[sl * nt];
+    return v;
+  };
   if (plan.paired()) {
     const int npair = n >> 1;
     for (int q = threadIdx.x; q < npair * nt; q += kThreads) {
       const int p = nt == 1 ? q : q >> 1, j = nt == 1 ? 0 : q & 1;
-      plan.epilogue2(s, (s.row0 + row0) / 2 + p, tok + j, sums[(2 * p) * nt + j],
-                     sums[(2 * p + 1) * nt + j]);
+      plan.epilogue2(s, (s.row0 + row0) / 2 + p, tok + j, sum(2 * p, j), sum(2 * p + 1, j));
     }
   } else {
     for (int q = threadIdx.x; q < n * nt; q += kThreads) {
       const int row = nt == 1 ? q : q >> 1, j = nt == 1 ? 0 : q & 1;
-      plan.epilogue(s, s.row0 + row0 + row, tok + j, sums[q]);
+      plan.epilogue(s, s.row0 + row0 + row, tok + j, sum(row, j));
     }
   }
 }
@@ -354,14 +338,15 @@ KD_DEV void release_stage(const Plan& plan, StreamShared& sh, Issuer& iss, int s
 
 // One segment.  Tokens are processed TT (= 2) at a time.  With at most TT
 // tokens (the common case) their activations are loaded once for the whole
-// segment and the reduced sums of consecutive stages are held in shared
-// memory, so the epilogue (and any global loads it makes) runs once per
-// kSumCap sums instead of once per stage.  With more tokens the stage is
-// swept once per group of TT tokens, reloading the activations (through L1)
-// for every group, and each group's epilogue runs at once.
+// segment and the warps run through the stages without any CTA barrier: each
+// writes its lane-reduced partials into shared memory, and only when
+// kPartCap is about to fill (or at the end of the segment) do all warps meet
+// to reduce them and run the epilogue.  With more tokens the stage is swept
+// once per group of TT tokens, reloading the activations (through L1) for
+// every group, and each group is reduced at once.
 template <int WT, int AT, class Plan>
 KD_DEV void consume_segment(const Plan& plan, StreamShared& sh, Issuer& iss, const Seg& s,
-                            uint32_t& it, int& rb, unsigned* err) {
+                            uint32_t& it, unsigned* err) {
   constexpr int TT = WTraits<WT>::TT;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rps = rows_per_stage(s.row_bytes, plan.paired());
@@ -371,18 +356,20 @@ KD_DEV void consume_segment(const Plan& plan, StreamShared& sh, Issuer& iss, con
   const int slice0 = my_slice * cpl;
   ActRegs<WT> areg;
   const bool single_pass = s.ntok <= TT;
+  const int ntp = single_pass ? (s.ntok > 0 ? s.ntok : 1) : TT;  // token stride of the partials
   if (single_pass) load_act_regs<WT, AT>(plan, s, 0, s.ntok, slice0, cpl, areg);
-  int held0 = 0;  // first segment row whose sums wait in sh.sums (single pass)
+  int held0 = 0;  // first segment row whose partials wait in sh.part
   for (int r0 = 0; r0 < s.nrows; r0 += rps, ++it) {
     const int n = s.nrows - r0 < rps ? s.nrows - r0 : rps;
     const int slot = it % kStages;
     const uint32_t ph = (it / kStages) & 1u;
     wait_or_abort(&sh.full[slot], ph, sh.abort_flag, err, ERR_WAIT_FULL);
     const uint8_t* st = sh.stage + (size_t)slot * kStageBytes;
+    if (!single_pass) held0 = r0;
+    float* part = sh.part + (size_t)(r0 - held0) * S * ntp;
     for (int tok = 0; tok < s.ntok; tok += TT) {
       const int nt = s.ntok - tok < TT ? s.ntok - tok : TT;
       if (!single_pass) load_act_regs<WT, AT>(plan, s, tok, nt, slice0, cpl, areg);
-      float* red = sh.red + rb * kRedFloats;
       for (int rbase = my_group; rbase < n; rbase += 4 * G) {
         int rows[4];
 #pragma unroll
@@ -393,41 +380,37 @@ KD_DEV void consume_segment(const Plan& plan, StreamShared& sh, Issuer& iss, con
         const int myrow = rbase + ((lane >> 3) & 3) * G;   // the row this lane's sums belong to
         if ((lane & 7) == 0 && myrow < n) {
 #pragma unroll
-          for (int t = 0; t < kTT; ++t)
-            if (t < nt) red[(myrow * S + my_slice) * kTT + t] = res[t];
+          for (int t = 0; t < TT; ++t)
+            if (t < nt) part[(myrow * S + my_slice) * ntp + t] = res[t];
         }
       }
       if (tok + TT >= s.ntok) release_stage(plan, sh, iss, slot, ph, err);
-      named_bar_sync(1, kThreads);
-      if (single_pass) {
-        reduce_slices(red, sh.sums + (r0 - held0) * nt, n, S, nt);
-        const bool last = r0 + rps >= s.nrows;
-        if (last || (r0 + n + rps - held0) * nt > kSumCap) {
-          named_bar_sync(1, kThreads);
-          run_epilogue(plan, s, sh.sums, held0, r0 + n - held0, 0, nt);
-          named_bar_sync(1, kThreads);  // sums are reused from the start
-          held0 = r0 + n;
-        }
-      } else {
-        float* dst = red + kRedFloats - n * nt;   // above every partial of the stage
-        reduce_slices(red, dst, n, S, nt);
+      if (!single_pass) {
         named_bar_sync(1, kThreads);
-        run_epilogue(plan, s, dst, r0, n, tok, nt);
+        reduce_epilogue(plan, s, sh.part, r0, n, S, tok, nt);
+        named_bar_sync(1, kThreads);
       }
-      rb ^= 1;
     }
     if (s.ntok == 0) release_stage(plan, sh, iss, slot, ph, err);
+    if (single_pass && s.ntok > 0) {
+      const bool last = r0 + rps >= s.nrows;
+      if (last || (r0 + n + rps - held0) * S * ntp > kPartCap) {
+        named_bar_sync(1, kThreads);
+        reduce_epilogue(plan, s, sh.part, held0, r0 + n - held0, S, 0, s.ntok);
+        named_bar_sync(1, kThreads);  // the partials buffer is reused from the start
+        held0 = r0 + n;
+      }
+    }
   }
 }
 
 template <int WT, int AT, class Plan>
 KD_DEV void stream_consume(const Plan& plan, StreamShared& sh, Issuer& iss, unsigned* err) {
   uint32_t it = 0;
-  int rb = 0;  // reduction buffer parity
   const int nseg = plan.num_segments();
   for (int si = 0; si < nseg; ++si) {
     const Seg s = plan.segment(si);
-    consume_segment<WT, AT>(plan, sh, iss, s, it, rb, err);
+    consume_segment<WT, AT>(plan, sh, iss, s, it, err);
     if (plan.wants_segment_done()) {
       named_bar_sync(1, kThreads);  // every epilogue write of the segment is done
       plan.segment_done(s);
