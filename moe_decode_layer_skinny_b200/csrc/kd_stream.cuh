@@ -296,15 +296,16 @@ KD_DEV void batch_dot(const Plan& plan, const Seg& s, int stage_row0, const uint
 }
 
 // Epilogue of `n` consecutive rows starting at segment row `row0`, whose lane-
-// reduced partials are part[(row * S + slice) * nt + j] (rows relative to
-// row0): each sum adds its S slices in a fixed order (deterministic).
+// reduced partials are part[(row * S + slice) * ts + j] (rows relative to
+// row0, ts >= nt the token stride): each sum adds its S slices in a fixed
+// order (deterministic).
 template <class Plan>
 KD_DEV void reduce_epilogue(const Plan& plan, const Seg& s, const float* part, int row0, int n,
-                            int S, int tok, int nt) {
+                            int S, int tok, int nt, int ts) {
   auto sum = [&](int row, int j) {
-    const float* p = part + (size_t)row * S * nt + j;
+    const float* p = part + (size_t)row * S * ts + j;
     float v = 0.f;
-    for (int sl = 0; sl < S; ++sl) v += p[sl * nt];
+    for (int sl = 0; sl < S; ++sl) v += p[sl * ts];
     return v;
   };
   if (plan.paired()) {
@@ -387,7 +388,7 @@ KD_DEV void consume_segment(const Plan& plan, StreamShared& sh, Issuer& iss, con
       if (tok + TT >= s.ntok) release_stage(plan, sh, iss, slot, ph, err);
       if (!single_pass) {
         named_bar_sync(1, kThreads);
-        reduce_epilogue(plan, s, sh.part, r0, n, S, tok, nt);
+        reduce_epilogue(plan, s, sh.part, r0, n, S, tok, nt, ntp);
         named_bar_sync(1, kThreads);
       }
     }
@@ -396,7 +397,7 @@ KD_DEV void consume_segment(const Plan& plan, StreamShared& sh, Issuer& iss, con
       const bool last = r0 + rps >= s.nrows;
       if (last || (r0 + n + rps - held0) * S * ntp > kPartCap) {
         named_bar_sync(1, kThreads);
-        reduce_epilogue(plan, s, sh.part, held0, r0 + n - held0, S, 0, s.ntok);
+        reduce_epilogue(plan, s, sh.part, held0, r0 + n - held0, S, 0, s.ntok, ntp);
         named_bar_sync(1, kThreads);  // the partials buffer is reused from the start
         held0 = r0 + n;
       }
