@@ -163,6 +163,38 @@ void kd_stack_destroy(kd_stack* stack);
 #define KD_N_TIMING_EVENTS 5
 int kd_layer_set_timing_events(kd_layer* layer, void* const* events, int n_events);
 
+/* Router top-k without any device allocation (the pages have no counterpart
+ * of this entry point).  For callers that cannot call cudaMalloc from where
+ * they run it -- e.g. a host runtime whose device memory all belongs to
+ * another allocator, or a plugin that is handed only its input and output
+ * buffers: the scratch this computation needs between its two kernels
+ * (router logits and per-expert lists) lives in a file-scope __device__
+ * array of fixed size in the library, held by every GPU that loads it until
+ * the process exits, instead of a cudaMalloc'd workspace.
+ *   router_w      device, [n_experts, hidden] bf16 (wdtype KD_WBF16) or e4m3
+ *                 codes (KD_WFP8), row-major
+ *   router_scales device fp32 [ceil(n_experts/128), hidden/128] for KD_WFP8,
+ *                 else ignored (may be NULL)
+ *   router_bias   device fp32 [n_experts] added to the logits, or NULL
+ *   h1            device fp32 [M, hidden]
+ *   idx_out       device int32 [M, top_k]: selected experts, descending logit,
+ *                 ties -> lower id
+ *   gates_out     device fp32 [M, top_k]: softmax renormalised over the top_k
+ * Same arithmetic as the router of kd_decode_layer.  Limits: M <= 64
+ * (KD_STATIC_MAX_TOKENS), n_experts <= 1024 (KD_STATIC_MAX_EXPERTS),
+ * top_k <= 16, hidden a multiple of 128 and <= 8192; larger sizes return
+ * KD_ERANGE, bad pointers or shapes KD_EINVAL.  Calls no cudaMalloc /
+ * cudaFree.  The first call on a device looks up the scratch's device
+ * address (cudaGetSymbolAddress) for that device and caches it, so make that
+ * first call before any stream capture.  All calls share the scratch and it
+ * keeps the last call's contents; calls that overlap on the GPU (other
+ * streams, other threads) race on it. */
+#define KD_STATIC_MAX_TOKENS 64
+#define KD_STATIC_MAX_EXPERTS 1024
+int kd_router_topk_static(const void* router_w, const float* router_scales, int wdtype,
+                          const float* router_bias, const float* h1, int M, int hidden,
+                          int n_experts, int top_k, int* idx_out, float* gates_out, void* stream);
+
 /* Message of the last failure on the calling thread ("" if none). */
 const char* kd_last_error(void);
 

@@ -24,7 +24,7 @@ T_H1F, T_H1B, T_LOGITS, T_IDX, T_GATES, T_COUNTS, T_NACTIVE, T_YSHARED, T_YROUTE
 EXPORTS = ("kd_layer_create", "kd_layer_destroy", "kd_decode_layer", "kd_layer_check",
            "kd_layer_qkv", "kd_layer_prefetch_l2", "kd_layer_debug_tensor", "kd_layer_read_weight",
            "kd_layer_bytes", "kd_layer_set_timing_events", "kd_stack_create", "kd_stack_run",
-           "kd_stack_destroy", "kd_last_error")
+           "kd_stack_destroy", "kd_router_topk_static", "kd_last_error")
 N_TIMING_EVENTS = 5
 
 
@@ -69,6 +69,7 @@ def lib() -> ctypes.CDLL:
         L.kd_stack_run.argtypes = [vp, vp, vp, vp]
         L.kd_stack_destroy.argtypes = [vp]
         L.kd_stack_destroy.restype = None
+        L.kd_router_topk_static.argtypes = [vp, vp, i32, vp, vp, i32, i32, i32, i32, vp, vp, vp]
         L.kd_last_error.restype = ctypes.c_char_p
         _lib = L
     return _lib
@@ -193,6 +194,17 @@ class Layer:
         _check(lib().kd_layer_read_weight(self._h, kind, expert, row0, nrows, out.ctypes.data,
                                           sc.ctypes.data))
         return out, sc
+
+
+def router_topk_static(router_w, router_scales, wdtype: int, router_bias, h1, M: int,
+                       hidden: int, n_experts: int, top_k: int, idx_out, gates_out,
+                       stream=None) -> None:
+    """kd_router_topk_static on torch CUDA tensors (or None for the optional
+    ones); allocates no device memory."""
+    ptr = lambda t: None if t is None else t.data_ptr()
+    _check(lib().kd_router_topk_static(ptr(router_w), ptr(router_scales), wdtype, ptr(router_bias),
+                                       ptr(h1), M, hidden, n_experts, top_k, ptr(idx_out),
+                                       ptr(gates_out), _stream_ptr(stream)))
 
 
 class Stack:

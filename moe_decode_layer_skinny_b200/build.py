@@ -30,7 +30,8 @@ def build(force: bool = False, verbose: bool = False) -> str:
     if not (force or stale()):
         return SO
     nvcc = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
-    cmd = [nvcc, *NVCC_FLAGS, "-o", SO, os.path.join(HERE, "csrc", "kd_layer.cu")]
+    cmd = [nvcc, *NVCC_FLAGS, "-o", SO, os.path.join(HERE, "csrc", "kd_layer.cu"),
+           os.path.join(HERE, "csrc", "kd_static.cu")]
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     subprocess.check_call(cmd)

@@ -20,7 +20,7 @@ namespace kd {
 // ------------------------------------------------------------------ generator
 
 // dst[(r*row_mult + row_off) * K + c] = bf16(value(stream, r*K + c)), r < R.
-__global__ void gen_bf16_kernel(uint16_t* __restrict__ dst, int R, int K, uint64_t stream,
+static __global__ void gen_bf16_kernel(uint16_t* __restrict__ dst, int R, int K, uint64_t stream,
                                 int row_mult, int row_off) {
   const uint64_t n = (uint64_t)R * (uint64_t)K;
   for (uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
@@ -32,7 +32,7 @@ __global__ void gen_bf16_kernel(uint16_t* __restrict__ dst, int R, int K, uint64
 
 // One 128x128 block per CTA (256 threads): amax -> scale -> e4m3 codes.
 // scales: [ceil(R/128), ceil(K/128)] table of this logical matrix.
-__global__ void __launch_bounds__(256) gen_fp8_kernel(uint8_t* __restrict__ dst,
+static __global__ void __launch_bounds__(256) gen_fp8_kernel(uint8_t* __restrict__ dst,
                                                       float* __restrict__ scales, int R, int K,
                                                       uint64_t stream, int row_mult, int row_off) {
   const int kb = blockIdx.x, rb = blockIdx.y, nkb = gridDim.x;

@@ -65,6 +65,9 @@ struct kd_stack {
 
 extern "C" const char* kd_last_error(void) { return g_err.c_str(); }
 
+// Shared with the other entry-point files of the library.
+void kd_set_last_error(const char* msg) { g_err = msg; }
+
 // ------------------------------------------------------------------ helpers
 
 static int dalloc(kd_layer* L, size_t bytes, void** p) {

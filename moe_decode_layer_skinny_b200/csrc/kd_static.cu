@@ -1,0 +1,137 @@
+// kd_static.cu -- router top-k entry point that allocates no device memory.
+//
+// For callers that cannot call cudaMalloc from where they run this code: for
+// example a host runtime whose device memory is entirely owned by another
+// allocator (a framework's caching allocator, an inference engine that hands
+// plugins only their input and output buffers), or code that may only enqueue
+// work.  The logits and the per-expert lists this router needs between its
+// two kernels live in one file-scope __device__ array of fixed size instead
+// of a cudaMalloc'd workspace.
+//
+// The array exists once per device for the life of the process.  Host code
+// may not pass the array's name to a kernel (on the host it names a stand-in,
+// not the device address): the device address is looked up with
+// cudaGetSymbolAddress on the first call on each device, with that device
+// current, and cached.  All calls share the array: two calls that overlap on
+// the GPU (different streams, or different host threads) race on it.
+#include <cuda_runtime.h>
+
+#include <cstdio>
+#include <mutex>
+
+#include "../../include/kd.h"
+#include "kd_kernels.cuh"
+
+using namespace kd;
+
+namespace {
+
+constexpr int kMaxTok = KD_STATIC_MAX_TOKENS;
+constexpr int kMaxExp = KD_STATIC_MAX_EXPERTS;
+constexpr int kMaxK = 16;
+
+// logits [64 x 1024] | counts [1024] | offsets [1025] | active [1024]
+// | perm [64 x 16] | n_active [1] | err [1]       (4-byte words)
+constexpr size_t kWords = (size_t)kMaxTok * kMaxExp + kMaxExp + (kMaxExp + 1) + kMaxExp +
+                          (size_t)kMaxTok * kMaxK + 2;
+
+static __device__ __align__(256) float g_router_scratch[kWords];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+thread_local char g_msg[256];
+
+// Every scratch word is written before it is read within a call (logits by
+// the logit kernel, lists by the selection), so nothing needs clearing.
+__global__ void __launch_bounds__(256) topk_kernel(LayerDev L, int M) {
+  extern __shared__ int route_smem[];
+  const Route R = carve_route(route_smem, L.E, M * L.k);
+  route_tokens(L, M, R, true);
+}
+
+}  // namespace
+
+// kd_last_error() reports these messages too (defined with the layer API).
+void kd_set_last_error(const char* msg);
+
+namespace {
+int fail_static(int code) {
+  kd_set_last_error(g_msg);
+  return code;
+}
+}  // namespace
+
+extern "C" int kd_router_topk_static(const void* router_w, const float* router_scales,
+                                     int wdtype, const float* router_bias, const float* h1,
+                                     int M, int hidden, int n_experts, int top_k, int* idx_out,
+                                     float* gates_out, void* stream) {
+  if (!router_w || !h1 || !idx_out || !gates_out || (wdtype == KD_WFP8 && !router_scales) ||
+      (wdtype != KD_WBF16 && wdtype != KD_WFP8) || hidden <= 0 || hidden % 128 ||
+      hidden > 8192 || top_k < 1) {
+    snprintf(g_msg, sizeof g_msg, "kd_router_topk_static: null pointer or unsupported shape");
+    return fail_static(KD_EINVAL);
+  }
+  if (M < 1 || M > kMaxTok || n_experts < top_k || n_experts > kMaxExp || top_k > kMaxK) {
+    snprintf(g_msg, sizeof g_msg,
+             "kd_router_topk_static: M=%d experts=%d top_k=%d beyond the static limits "
+             "(M <= %d, top_k <= experts <= %d, top_k <= %d)",
+             M, n_experts, top_k, kMaxTok, kMaxExp, kMaxK);
+    return fail_static(KD_ERANGE);
+  }
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    snprintf(g_msg, sizeof g_msg, "kd_router_topk_static: no usable current device");
+    return fail_static(KD_ECUDA);
+  }
+  void* base = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_scratch_ptr[dev]) {
+      void* p = nullptr;
+      cudaError_t e = cudaGetSymbolAddress(&p, g_router_scratch);
+      if (e != cudaSuccess) {
+        snprintf(g_msg, sizeof g_msg, "kd_router_topk_static: cudaGetSymbolAddress: %s",
+                 cudaGetErrorString(e));
+        return fail_static(KD_ECUDA);
+      }
+      g_scratch_ptr[dev] = p;
+    }
+    base = g_scratch_ptr[dev];
+  }
+  float* f = static_cast<float*>(base);
+  int* w = reinterpret_cast<int*>(f);
+  size_t o = (size_t)kMaxTok * kMaxExp;
+  LayerDev d{};
+  d.H = hidden;
+  d.E = n_experts;
+  d.k = top_k;
+  d.eb = wdtype == KD_WBF16 ? 2 : 1;
+  d.nHb = hidden / 128;
+  d.wr = static_cast<const uint8_t*>(router_w);
+  d.sr = router_scales;
+  d.bias = router_bias;
+  d.h1f = const_cast<float*>(h1);
+  d.logits = f;
+  d.idx = idx_out;
+  d.gates = gates_out;
+  d.counts = w + o; o += kMaxExp;
+  d.offsets = w + o; o += kMaxExp + 1;
+  d.active = w + o; o += kMaxExp;
+  d.perm = w + o; o += (size_t)kMaxTok * kMaxK;
+  d.n_active = w + o; o += 1;
+  d.err = reinterpret_cast<unsigned*>(w + o);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int rgrid = (n_experts + kRouterRows - 1) / kRouterRows;
+  if (wdtype == KD_WFP8) router_kernel<W_FP8><<<rgrid, kRouterThreads, 0, s>>>(d, M);
+  else router_kernel<W_BF16><<<rgrid, kRouterThreads, 0, s>>>(d, M);
+  const size_t smem = sizeof(int) * kRouteSmemInts(n_experts, M * top_k);
+  topk_kernel<<<1, 256, smem, s>>>(d, M);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    snprintf(g_msg, sizeof g_msg, "kd_router_topk_static: launch: %s", cudaGetErrorString(e));
+    return fail_static(KD_ECUDA);
+  }
+  return KD_OK;
+}

@@ -63,9 +63,10 @@ def test_host_side_argument_errors(kd):
     assert L.kd_layer_set_timing_events(None, None, 0) == kd.KD_EINVAL
     assert L.kd_stack_create(None, 0, 1, 0, ctypes.byref(h)) == kd.KD_EINVAL
     assert L.kd_stack_run(None, None, None, None) == kd.KD_EINVAL
+    assert L.kd_router_topk_static(None, None, 0, None, None, 1, 256, 8, 2, None, None, None) == kd.KD_EINVAL
     L.kd_layer_destroy(None)
     L.kd_stack_destroy(None)
-    assert "kd_stack_run" in kd.lib().kd_last_error().decode()
+    assert "kd_router_topk_static" in kd.lib().kd_last_error().decode()
 
 
 def test_product_path_does_not_touch_the_oracle():
