@@ -67,6 +67,9 @@ typedef struct kd_config {
   int layer_id;      /* id of the layer in the seeded weight generator           */
   int max_tokens;    /* largest M a call may use, 1..64; sizes the workspaces    */
   const float* router_bias; /* host [E] additive router bias, or NULL; copied    */
+  int mma_min_tokens;/* calls with M >= this use the tensor-core (tcgen05) kernels,
+                        smaller M the CUDA-core streaming kernels; 0 = default (4),
+                        > 64 = never.  bf16 weights only (FP8 always streams).    */
 } kd_config;
 
 typedef struct kd_layer kd_layer;

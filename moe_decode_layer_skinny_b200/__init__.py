@@ -39,7 +39,7 @@ class _Config(ctypes.Structure):
                 ("head_dim", ctypes.c_int), ("n_experts", ctypes.c_int), ("top_k", ctypes.c_int),
                 ("n_shared", ctypes.c_int), ("inter", ctypes.c_int), ("wdtype", ctypes.c_int),
                 ("layer_id", ctypes.c_int), ("max_tokens", ctypes.c_int),
-                ("router_bias", ctypes.c_void_p)]
+                ("router_bias", ctypes.c_void_p), ("mma_min_tokens", ctypes.c_int)]
 
 
 _lib = None
@@ -101,6 +101,7 @@ class LayerSpec:
     layer_id: int = 0
     max_tokens: int = 64
     router_bias: np.ndarray | None = None
+    mma_min_tokens: int = 0
 
     @classmethod
     def from_dims(cls, dims, **kw) -> "LayerSpec":
@@ -118,7 +119,8 @@ class Layer:
             bias = np.ascontiguousarray(spec.router_bias, np.float32)
         cfg = _Config(spec.hidden, spec.q_heads, spec.kv_heads, spec.head_dim, spec.n_experts,
                       spec.top_k, spec.n_shared, spec.inter, spec.wdtype, spec.layer_id,
-                      spec.max_tokens, None if bias is None else bias.ctypes.data)
+                      spec.max_tokens, None if bias is None else bias.ctypes.data,
+                      spec.mma_min_tokens)
         h = ctypes.c_void_p()
         _check(lib().kd_layer_create(ctypes.byref(cfg), seed, ctypes.byref(h)))
         self._h = h

@@ -82,6 +82,11 @@ struct LayerDev {
   float* logits; int* idx; float* gates;
   int* counts; int* offsets; int* perm; int* active; int* n_active;
   float* act; float* act_sh;               // [Mmax*k, I] by position, [Mmax, I] (fp32)
+  uint16_t* h1lo;                          // [Mmax, H] bf16(h1 - bf16(h1))   (tensor-core path)
+  uint16_t* act_hi; uint16_t* act_lo;      // [Mmax*k, I] bf16 pair of act    (tensor-core path)
+  uint16_t* act_sh_hi; uint16_t* act_sh_lo;// [Mmax, I]
+  float* ws_main; float* ws_side;          // split-K partials, main / side stream launches
+  unsigned* tcnt_main; unsigned* tcnt_side;// split-K tile arrivals (self-resetting)
   float* yr; float* ysh;                   // [Mmax*k, H] by token*k+slot, [Mmax, H]
   unsigned* hcnt;                          // [H/64] down rows done per block (self-resetting)
   unsigned* err;

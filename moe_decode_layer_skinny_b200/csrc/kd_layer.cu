@@ -20,6 +20,7 @@
 
 #include "../../include/kd.h"
 #include "kd_kernels.cuh"
+#include "kd_mma_kernels.cuh"
 
 using namespace kd;
 
@@ -50,6 +51,9 @@ struct kd_layer {
   int Nqkv = 0, A = 0;
   cudaEvent_t tev[KD_N_TIMING_EVENTS] = {};  // profiling hook (kd_layer_set_timing_events)
   bool timing = false;
+  int mma_min = 4;       // calls with M >= mma_min use the tensor-core kernels
+  bool has_maps = false;
+  MmaMaps maps{};
 };
 
 struct kd_stack {
@@ -92,6 +96,37 @@ static int dalloc_t(kd_layer* L, size_t n, T** p) {
 
 static int ceil128(int x) { return (x + 127) / 128; }
 
+// cuTensorMapEncodeTiled, looked up through the runtime (no libcuda link).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess && q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D map of a row-major bf16 matrix [rows, K]: box 64 K x 128 rows, 128B swizzle.
+static bool encode_bf16_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t K) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {K, rows};
+  const cuuint64_t strides[1] = {K * 2};
+  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Generate one logical [R, K] matrix into `dst` with row stride multiplier
 // (physical row = r*mult + off); FP8 writes its block scales to `scales`.
 static int gen_matrix(const kd_layer* L, uint8_t* dst, float* scales, int R, int K, uint64_t seed,
@@ -132,6 +167,10 @@ static int configure_kernels() {
   KD_CUDA(cudaFuncSetAttribute(gateup_kernel<W_FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   KD_CUDA(cudaFuncSetAttribute(down_kernel<W_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   KD_CUDA(cudaFuncSetAttribute(down_kernel<W_FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  const int msmem = (int)(kMmaSmem + 16 + sizeof(int) * kRouteSmemInts(1024, 64 * 16));
+  KD_CUDA(cudaFuncSetAttribute(mma_proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem));
+  KD_CUDA(cudaFuncSetAttribute(mma_gateup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem));
+  KD_CUDA(cudaFuncSetAttribute(mma_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem));
   stream_kernels_configured = true;
   return KD_OK;
 }
@@ -147,7 +186,7 @@ extern "C" int kd_layer_create(const kd_config* cfg, uint64_t seed, kd_layer** o
       A % 128 || Nqkv % 128 || c.n_experts < 1 || c.n_experts > 1024 || c.top_k < 1 ||
       c.top_k > 16 || c.top_k > c.n_experts || c.n_shared < 0 || c.n_shared > 1 || c.inter <= 0 ||
       c.inter % 128 || (c.wdtype != KD_WBF16 && c.wdtype != KD_WFP8) || c.max_tokens < 1 ||
-      c.max_tokens > 64 || c.layer_id < 0)
+      c.max_tokens > 64 || c.layer_id < 0 || c.mma_min_tokens < 0)
     return fail(KD_EINVAL, "kd_layer_create: unsupported configuration%s", "");
   if (c.hidden * 2 > kStageBytes || A * 2 > kStageBytes || c.inter * 2 > kStageBytes ||
       c.hidden > 8192 || A > 8192 || c.inter > 8192)
@@ -158,6 +197,7 @@ extern "C" int kd_layer_create(const kd_config* cfg, uint64_t seed, kd_layer** o
   L->cfg = c;
   L->cfg.router_bias = nullptr;
   L->maxM = c.max_tokens;
+  L->mma_min = c.mma_min_tokens > 0 ? c.mma_min_tokens : 4;
   L->Nqkv = Nqkv;
   L->A = A;
   int rc = KD_OK;
@@ -249,6 +289,21 @@ extern "C" int kd_layer_create(const kd_config* cfg, uint64_t seed, kd_layer** o
   TRY(dalloc_t(L, (size_t)M * k * H, &d.yr));
   TRY(dalloc_t(L, (size_t)M * H, &d.ysh));
   TRY(dalloc_t(L, (size_t)H / 64, &d.hcnt));
+  TRY(dalloc_t(L, (size_t)M * H, &d.h1lo));
+  TRY(dalloc_t(L, (size_t)M * k * I, &d.act_hi));
+  TRY(dalloc_t(L, (size_t)M * k * I, &d.act_lo));
+  TRY(dalloc_t(L, (size_t)M * I, &d.act_sh_hi));
+  TRY(dalloc_t(L, (size_t)M * I, &d.act_sh_lo));
+  TRY(dalloc_t(L, (size_t)L->nsm * kWsFloatsPerCta, &d.ws_main));
+  TRY(dalloc_t(L, (size_t)L->nsm * kWsFloatsPerCta, &d.ws_side));
+  {
+    const size_t ntile = std::max<size_t>({(size_t)(E + 1) * (H / 128), (size_t)E * (2 * I / 128),
+                                           (size_t)(Nqkv + H) / 128});
+    TRY(dalloc_t(L, ntile, &d.tcnt_main));
+    TRY(dalloc_t(L, ntile, &d.tcnt_side));
+    TRYC(cudaMemset(d.tcnt_main, 0, sizeof(unsigned) * ntile));
+    TRYC(cudaMemset(d.tcnt_side, 0, sizeof(unsigned) * ntile));
+  }
   TRYC(cudaMemset(d.hcnt, 0, sizeof(unsigned) * (H / 64)));
   TRY(dalloc_t(L, 1, &d.err));
   TRYC(cudaMemset(d.err, 0, sizeof(unsigned)));
@@ -277,6 +332,15 @@ extern "C" int kd_layer_create(const kd_config* cfg, uint64_t seed, kd_layer** o
   cudaStreamDestroy(gs);
   if (rc != KD_OK) { free_layer(L); return rc; }
   TRYC(se);
+
+  if (!fp8) {
+    bool ok = encode_bf16_map(&L->maps.m[0], wqkv, Nqkv, H) && encode_bf16_map(&L->maps.m[1], wo, H, A) &&
+              encode_bf16_map(&L->maps.m[2], wgu, (uint64_t)E * 2 * I, H) &&
+              encode_bf16_map(&L->maps.m[3], wd, (uint64_t)E * H, I);
+    if (ok && c.n_shared)
+      ok = encode_bf16_map(&L->maps.m[4], wgu_sh, 2 * I, H) && encode_bf16_map(&L->maps.m[5], wd_sh, H, I);
+    L->has_maps = ok;
+  }
 
   TRYC(cudaStreamCreateWithFlags(&L->side, cudaStreamNonBlocking));
   TRYC(cudaEventCreateWithFlags(&L->ev_h1, cudaEventDisableTiming));
@@ -341,8 +405,14 @@ static int launch_layer(kd_layer* L, void* hidden, const void* attn, int M, cuda
   a.M = M;
   const int G = L->nsm;
   const size_t sm = kStreamSmem;
+  const bool mma = L->has_maps && M >= L->mma_min;
+  const size_t msm = kMmaSmem;
+  const size_t mroute = kMmaSmem + 16 + sizeof(int) * kRouteSmemInts(d.E, M * d.k);
   if (L->timing) KD_CUDA(cudaEventRecord(L->tev[0], s));
-  KD_CUDA(launch(fp8 ? proj_kernel<W_FP8> : proj_kernel<W_BF16>, G, kThreads, sm, s, pdl_first, d, a));
+  if (mma)
+    KD_CUDA(launch(mma_proj_kernel, G, kMThreads, msm, s, pdl_first, d, a, L->maps));
+  else
+    KD_CUDA(launch(fp8 ? proj_kernel<W_FP8> : proj_kernel<W_BF16>, G, kThreads, sm, s, pdl_first, d, a));
   if (L->timing) KD_CUDA(cudaEventRecord(L->tev[1], s));
   if (d.S) KD_CUDA(cudaEventRecord(L->ev_h1, s));
   // the router goes first so that its CTAs get SMs before the shared
@@ -352,13 +422,19 @@ static int launch_layer(kd_layer* L, void* hidden, const void* attn, int M, cuda
                  !L->timing, d, M));
   if (d.S) {
     KD_CUDA(cudaStreamWaitEvent(L->side, L->ev_h1, 0));
-    KD_CUDA(launch(fp8 ? gateup_kernel<W_FP8> : gateup_kernel<W_BF16>, G, kThreads, sm, L->side,
-                   false, d, M, 1));
+    if (mma)
+      KD_CUDA(launch(mma_gateup_kernel, G, kMThreads, msm, L->side, false, d, M, 1, L->maps));
+    else
+      KD_CUDA(launch(fp8 ? gateup_kernel<W_FP8> : gateup_kernel<W_BF16>, G, kThreads, sm, L->side,
+                     false, d, M, 1));
     KD_CUDA(cudaEventRecord(L->ev_sh, L->side));
   }
   if (L->timing) KD_CUDA(cudaEventRecord(L->tev[2], s));
-  KD_CUDA(launch(fp8 ? gateup_kernel<W_FP8> : gateup_kernel<W_BF16>, G, kThreads,
-                 gateup_smem(d, M), s, !L->timing, d, M, 0));
+  if (mma)
+    KD_CUDA(launch(mma_gateup_kernel, G, kMThreads, mroute, s, !L->timing, d, M, 0, L->maps));
+  else
+    KD_CUDA(launch(fp8 ? gateup_kernel<W_FP8> : gateup_kernel<W_BF16>, G, kThreads,
+                   gateup_smem(d, M), s, !L->timing, d, M, 0));
   if (L->timing) KD_CUDA(cudaEventRecord(L->tev[3], s));
   if (d.S) KD_CUDA(cudaStreamWaitEvent(s, L->ev_sh, 0));
   if (next && pf) {
@@ -369,8 +445,11 @@ static int launch_layer(kd_layer* L, void* hidden, const void* attn, int M, cuda
     if (rc != KD_OK) return rc;
     KD_CUDA(cudaEventRecord(ev_join, pf));
   }
-  KD_CUDA(launch(fp8 ? down_kernel<W_FP8> : down_kernel<W_BF16>, G, kThreads, sm, s,
-                 !L->timing && !d.S, d, M, a.out));
+  if (mma)
+    KD_CUDA(launch(mma_down_kernel, G, kMThreads, msm, s, !L->timing && !d.S, d, M, a.out, L->maps));
+  else
+    KD_CUDA(launch(fp8 ? down_kernel<W_FP8> : down_kernel<W_BF16>, G, kThreads, sm, s,
+                   !L->timing && !d.S, d, M, a.out));
   if (L->timing) KD_CUDA(cudaEventRecord(L->tev[4], s));
   if (next && pf) KD_CUDA(cudaStreamWaitEvent(s, ev_join, 0));
   return KD_OK;

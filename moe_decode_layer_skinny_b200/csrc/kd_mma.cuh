@@ -1,0 +1,420 @@
+// kd_mma.cuh -- tensor-core engine (tcgen05) for token counts where the
+// projections are real dense contractions (M >= a few tokens).
+//
+// Swap-AB: a 128-row weight tile is the MMA's A operand (M = 128) and the
+// tokens are its N (padded to a multiple of 16), so one kind::f16 MMA of
+// 128 x N x 16 consumes 4 KB of weights.  Per CTA (one per SM), warp roles:
+//   warp 0      TMA producer: 2-D tiled loads (128B swizzle) of the weight tile
+//               [128 rows x 64 K] into a ring of stages
+//   warp 1      MMA issuer: owns the TMEM accumulators (two buffers of N fp32
+//               columns), issues tcgen05.mma, commits stage releases
+//   warps 2-3   B producers: gather the tokens' bf16 rows (64 K at a time)
+//               into the stage in the same swizzled K-major layout
+//   warps 4-7   epilogue: tcgen05.ld of the accumulator (lane = weight row),
+//               then the plan's epilogue, or a split-K partial
+// Activations that must stay fp32-accurate (h1, the SwiGLU activations) come
+// as a bf16 pair hi + lo (hi = bf16(v), lo = bf16(v - hi)); both are
+// multiplied into the same accumulator, which keeps ~16 significant bits.
+// Work units are (weight tile, K part); a tile split over several parts is
+// summed in part order by the unit that completes it (deterministic).
+#pragma once
+
+#include <cuda.h>
+
+#include "kd_common.cuh"
+
+namespace kd {
+
+// ------------------------------------------------------------------ PTX
+
+KD_DEV void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];"
+      ::"r"(smem_u32(dst)), "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar)) : "memory");
+}
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
+// 1024 bytes apart (stride byte offset), version 1.
+KD_DEV uint64_t sw128_desc(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);           // start address
+  d |= (uint64_t)1u << 16;                            // leading byte offset (16 B, unused)
+  d |= (uint64_t)(1024u >> 4) << 32;                  // stride byte offset
+  d |= (uint64_t)1u << 46;                            // version
+  d |= (uint64_t)2u << 61;                            // layout: 128-byte swizzle
+  return d;
+}
+
+// Instruction descriptor, kind::f16: bf16 A and B (K-major), fp32 D, M = 128.
+KD_DEV uint32_t idesc_bf16(int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((128u >> 4) << 24);
+}
+
+KD_DEV void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+KD_DEV void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+KD_DEV void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+               ::"r"(smem_u32(dst_smem)), "r"(ncols) : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+KD_DEV void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+
+KD_DEV void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, bool acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"((uint32_t)acc) : "memory");
+}
+
+// Arrive once on `bar` when every MMA issued so far by this thread completed.
+KD_DEV void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+               ::"r"(smem_u32(bar)) : "memory");
+}
+
+KD_DEV void tmem_ld16(uint32_t taddr, float* v) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+KD_DEV void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// ------------------------------------------------------------------ engine
+
+constexpr int kMThreads = 256;
+constexpr int kMStages = 6;
+constexpr int kATileBytes = 128 * 128;                // 128 rows x 64 bf16
+constexpr int kBTileBytes = 64 * 128 * 2;             // up to 64 tokens x 64 bf16, hi + lo
+constexpr int kMStageBytes = kATileBytes + kBTileBytes;
+constexpr int kMaxN = 64;                             // tokens per MMA (N)
+constexpr int kKChunk = 64;                           // K elements per stage
+constexpr size_t kWsFloatsPerCta = 2 * 128 * 64;     // split-K partial slots of one CTA
+constexpr size_t kMmaSmem = (size_t)kMStages * kMStageBytes + 1024 /*align*/ + 1024 /*barriers, lists*/;
+
+// One unit of work: K chunks [kc0, kc0 + nkc) of a 128-row weight tile.
+struct MUnit {
+  int map;        // tensor map index (plan-defined)
+  int row;        // first row of the tile in the tensor map
+  int kc0, nkc;   // K chunks (64 elements each)
+  int tile;       // tile id within the launch (split-K bookkeeping)
+  int part, nparts;
+  int tok0, ntok; // token list range (plan-defined meaning)
+  int tag;        // plan-defined (matrix, expert)
+  int lrow;       // first row of the tile in its logical output (epilogue index)
+};
+
+KD_DEV int pad16(int n) { return (n + 15) & ~15; }
+
+// Stream-K partition of a launch: the K chunks of all tiles, concatenated in
+// tile order, are cut into gridDim.x equal ranges; CTA b takes range b.  A
+// tile that straddles ranges is computed in parts (one per CTA, part p by
+// CTA first_owner + p) and summed, in part order, by the part that finishes
+// last.  Only a CTA's first and last unit can be partial, so the partials
+// live in two slots per CTA: the tile's part 0 in slot 1 (the end of the
+// first owner's range), every later part in slot 0 (the start of its range).  Plan: int num_tiles(); long long
+// tile_start(int t) (first chunk of tile t, non-decreasing, tile_start(n) =
+// total); MUnit tile_unit(int t) (map, row, tag, lrow, tok0, ntok filled).
+template <class Plan>
+struct CtaUnits {
+  const Plan& plan;
+  long long T, lo, hi;
+  int t, nt;
+  KD_DEV explicit CtaUnits(const Plan& p) : plan(p) {
+    nt = plan.num_tiles();
+    T = plan.tile_start(nt);
+    const long long G = gridDim.x, b = blockIdx.x;
+    lo = b * T / G;
+    hi = (b + 1) * T / G;
+    // first tile whose chunk range reaches past lo
+    int a = 0, z = nt;
+    while (a < z) {
+      const int mid = (a + z) >> 1;
+      if (plan.tile_start(mid + 1) <= lo) a = mid + 1;
+      else z = mid;
+    }
+    t = a;
+  }
+  // CTA owning chunk c: the largest b with floor(b*T/G) <= c
+  KD_DEV long long owner(long long c) const {
+    const long long G = gridDim.x;
+    return ((c + 1) * G + T - 1) / T - 1;
+  }
+  KD_DEV bool next(MUnit& m) {
+    if (lo >= hi) return false;
+    long long cs = 0, ce = 0;
+    for (;; ++t) {
+      if (t >= nt) return false;
+      cs = plan.tile_start(t);
+      ce = plan.tile_start(t + 1);
+      if (cs >= hi) return false;
+      if (ce > cs) break;
+    }
+    m = plan.tile_unit(t);
+    const long long a = cs > lo ? cs : lo, z = ce < hi ? ce : hi;
+    m.kc0 = (int)(a - cs);
+    m.nkc = (int)(z - a);
+    m.tile = t;
+    const long long bf = owner(cs), bl = owner(ce - 1);
+    m.nparts = (int)(bl - bf + 1);
+    m.part = (int)((long long)blockIdx.x - bf);
+    ++t;
+    return true;
+  }
+};
+
+struct MmaShared {
+  uint8_t* stage;        // kMStages x kMStageBytes, 1024-aligned
+  uint64_t* full;        // [kMStages] A landed (tx) + B written (2 warp arrivals)
+  uint64_t* empty;       // [kMStages] MMAs of the stage done
+  uint64_t* accfull;     // [2] accumulator buffer ready for the epilogue
+  uint64_t* accempty;    // [2] epilogue done reading the accumulator
+  uint32_t* tmem_base;
+  int* abort_flag;
+  int* misc;             // [8] epilogue scratch (combine block list length ...)
+  int* blist;            // [128] combine block list
+};
+
+KD_DEV MmaShared carve_mma_smem(uint8_t* raw) {
+  MmaShared s;
+  uintptr_t p = (reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023);
+  s.stage = reinterpret_cast<uint8_t*>(p);
+  p += (size_t)kMStages * kMStageBytes;
+  s.full = reinterpret_cast<uint64_t*>(p);
+  s.empty = s.full + kMStages;
+  s.accfull = s.empty + kMStages;
+  s.accempty = s.accfull + 2;
+  s.tmem_base = reinterpret_cast<uint32_t*>(s.accempty + 2);
+  s.abort_flag = reinterpret_cast<int*>(s.tmem_base + 1);
+  s.misc = s.abort_flag + 1;
+  s.blist = s.misc + 8;
+  return s;
+}
+
+KD_DEV bool mwait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, unsigned* err) {
+  if (*abort_flag) return false;
+  if (mbar_wait(bar, parity)) return true;
+  *abort_flag = 1;
+  set_error(err, ERR_WAIT_MMA);
+  return false;
+}
+
+// Plan interface (all methods KD_DEV const):
+//   int num_tiles(); long long tile_start(int t); MUnit tile_unit(int t)   (see CtaUnits)
+//   const CUtensorMap* map(int id)
+//   bool split_b()                 B is a hi/lo pair
+//   const uint16_t* b_row(const MUnit&, int j, int hilo)   token j's bf16 row
+//   bool paired()                  rows are (gate, up) pairs
+//   void epilogue(const MUnit&, int row_in_tile, int j, float v)
+//   void epilogue2(const MUnit&, int pair_in_tile, int j, float g, float u)
+//   float* ws(); unsigned* tile_cnt()            split-K partials / arrivals
+//   bool wants_unit_done(); void unit_done(const MUnit&, MmaShared&)   epilogue warps only
+
+template <class Plan>
+KD_DEV void mma_producer_a(const Plan& plan, MmaShared& sh, unsigned* err) {
+  uint32_t it = 0;
+  CtaUnits<Plan> units(plan);
+  MUnit m;
+  while (units.next(m)) {
+    const CUtensorMap* map = plan.map(m.map);
+    for (int c = 0; c < m.nkc; ++c, ++it) {
+      const int s = it % kMStages;
+      const uint32_t ph = (it / kMStages) & 1u;
+      mwait(&sh.empty[s], ph ^ 1u, sh.abort_flag, err);
+      mbar_arrive_expect_tx(&sh.full[s], kATileBytes);
+      tma_load_2d(sh.stage + (size_t)s * kMStageBytes, map, (m.kc0 + c) * kKChunk, m.row,
+                  &sh.full[s]);
+    }
+  }
+}
+
+// Two warps (64 threads) write the B tile of every stage: token rows j <
+// ntok (zeros up to N), 128 bytes (64 K) each, 16-byte chunk c of row r at
+// r*128 + ((c ^ (r & 7)) * 16) -- the 128-byte swizzle the A tile has.
+template <class Plan>
+KD_DEV void mma_producer_b(const Plan& plan, MmaShared& sh, unsigned* err) {
+  const int t = threadIdx.x - 64;  // 0..63
+  const int nh = plan.split_b() ? 2 : 1;
+  uint32_t it = 0;
+  CtaUnits<Plan> units(plan);
+  MUnit m;
+  while (units.next(m)) {
+    const int N = pad16(m.ntok);
+    for (int c = 0; c < m.nkc; ++c, ++it) {
+      const int s = it % kMStages;
+      const uint32_t ph = (it / kMStages) & 1u;
+      mwait(&sh.empty[s], ph ^ 1u, sh.abort_flag, err);
+      uint8_t* bt = sh.stage + (size_t)s * kMStageBytes + kATileBytes;
+      const int k0 = (m.kc0 + c) * kKChunk;
+      for (int q = t; q < nh * N * 8; q += 64) {
+        const int h = q / (N * 8), r = (q / 8) % N, ch = q % 8;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (r < m.ntok) v = ld_nc_v4(plan.b_row(m, r, h) + k0 + ch * 8);
+        *reinterpret_cast<uint4*>(bt + (size_t)h * N * 128 + r * 128 + ((ch ^ (r & 7)) * 16)) = v;
+      }
+      fence_proxy_async_smem();   // generic-proxy writes -> visible to the tensor core
+      mbar_arrive(&sh.full[s]);
+    }
+  }
+}
+
+template <class Plan>
+KD_DEV void mma_issuer(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigned* err) {
+  const bool split = plan.split_b();
+  uint32_t it = 0, nu_local = 0;
+  CtaUnits<Plan> units(plan);
+  MUnit m;
+  for (; units.next(m); ++nu_local) {
+    const int N = pad16(m.ntok);
+    const uint32_t idesc = idesc_bf16(N);
+    const int buf = nu_local & 1;
+    const uint32_t d = tmem + (uint32_t)(buf * kMaxN);
+    mwait(&sh.accempty[buf], ((nu_local >> 1) & 1u) ^ 1u, sh.abort_flag, err);
+    tc_fence_after();
+    for (int c = 0; c < m.nkc; ++c, ++it) {
+      const int s = it % kMStages;
+      const uint32_t ph = (it / kMStages) & 1u;
+      mwait(&sh.full[s], ph, sh.abort_flag, err);
+      tc_fence_after();
+      const uint32_t a = smem_u32(sh.stage + (size_t)s * kMStageBytes);
+      const uint32_t b = a + kATileBytes;
+#pragma unroll
+      for (int k = 0; k < kKChunk / 16; ++k) {
+        const uint64_t ad = sw128_desc(a + k * 32);
+        mma_bf16(d, ad, sw128_desc(b + k * 32), idesc, c > 0 || k > 0);
+        if (split) mma_bf16(d, ad, sw128_desc(b + N * 128 + k * 32), idesc, true);
+      }
+      mma_commit(&sh.empty[s]);   // the stage is free once these MMAs are done
+    }
+    mma_commit(&sh.accfull[buf]);
+  }
+}
+
+// Epilogue warps (4..7).  Thread = accumulator lane = row of the tile.
+template <class Plan>
+KD_DEV void mma_epilogue(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigned* err) {
+  const int ew = (threadIdx.x >> 5) - 4, lane = threadIdx.x & 31;
+  const int row = ew * 32 + lane;
+  uint32_t nu_local = 0;
+  float v[kMaxN];
+  CtaUnits<Plan> units(plan);
+  MUnit m;
+  for (; units.next(m); ++nu_local) {
+    const int N = pad16(m.ntok);
+    const int buf = nu_local & 1;
+    mwait(&sh.accfull[buf], (nu_local >> 1) & 1u, sh.abort_flag, err);
+    tc_fence_after();
+    const uint32_t ta = tmem + ((uint32_t)(ew * 32) << 16) + (uint32_t)(buf * kMaxN);
+#pragma unroll
+    for (int c = 0; c < kMaxN / 16; ++c)
+      if (c * 16 < N) tmem_ld16(ta + c * 16, v + c * 16);
+    tmem_wait_ld();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sh.accempty[buf]);
+    bool complete = true;
+    if (m.nparts > 1) {
+      // split-K: park this part, the last part to arrive sums them in order
+      const int slot = m.part == 0 ? 1 : 0;
+      float* ws = plan.ws() + (size_t)blockIdx.x * kWsFloatsPerCta +
+                  ((size_t)slot * 128 + row) * kMaxN;
+#pragma unroll
+      for (int j = 0; j < kMaxN; ++j)
+        if (j < m.ntok) ws[j] = v[j];
+      __threadfence();
+      named_bar_sync(2, 128);
+      if (threadIdx.x == 128) {
+        const unsigned prev = atomicAdd(plan.tile_cnt() + m.tile, 1u);
+        const bool last = prev == (unsigned)(m.nparts - 1);
+        if (last) plan.tile_cnt()[m.tile] = 0u;  // every part is in: ready for reuse
+        sh.misc[0] = last;
+      }
+      named_bar_sync(2, 128);
+      complete = sh.misc[0] != 0;
+      if (complete) {
+        __threadfence();
+#pragma unroll
+        for (int j = 0; j < kMaxN; ++j) v[j] = 0.f;
+        const int first = (int)blockIdx.x - m.part;
+        for (int p = 0; p < m.nparts; ++p) {
+          const float* src = plan.ws() + (size_t)(first + p) * kWsFloatsPerCta +
+                             ((size_t)(p == 0 ? 1 : 0) * 128 + row) * kMaxN;
+#pragma unroll
+          for (int j = 0; j < kMaxN; ++j)
+            if (j < m.ntok) v[j] += __ldcg(src + j);
+        }
+      }
+    }
+    if (complete) {
+      if (plan.paired()) {
+#pragma unroll
+        for (int j = 0; j < kMaxN; ++j) {
+          if (j < N) {
+            const float other = __shfl_xor_sync(0xffffffffu, v[j], 1);
+            if (!(lane & 1) && j < m.ntok) plan.epilogue2(m, row >> 1, j, v[j], other);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < kMaxN; ++j)
+          if (j < m.ntok) plan.epilogue(m, row, j, v[j]);
+      }
+      if (plan.wants_unit_done()) {
+        named_bar_sync(2, 128);
+        plan.unit_done(m, sh);
+      }
+    }
+  }
+}
+
+template <class Plan>
+KD_DEV void mma_run(const Plan& plan, uint8_t* smem_raw, unsigned* err) {
+  MmaShared sh = carve_mma_smem(smem_raw);
+  const int warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kMStages; ++i) {
+      mbar_init(&sh.full[i], 1 + 64);  // A transaction arrive + the 64 B threads
+      mbar_init(&sh.empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sh.accfull[i], 1);
+      mbar_init(&sh.accempty[i], 4);
+    }
+    *sh.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(sh.tmem_base, 2 * kMaxN);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *sh.tmem_base;
+  if (warp == 0) {
+    if ((threadIdx.x & 31) == 0) mma_producer_a(plan, sh, err);
+  } else if (warp == 1) {
+    if ((threadIdx.x & 31) == 0) mma_issuer(plan, sh, tmem, err);
+  } else if (warp < 4) {
+    mma_producer_b(plan, sh, err);
+  } else {
+    mma_epilogue(plan, sh, tmem, err);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 2 * kMaxN);
+  }
+}
+
+}  // namespace kd

@@ -1,0 +1,230 @@
+// kd_mma_kernels.cuh -- the layer's projections on the tensor-core engine
+// (kd_mma.cuh), used when a call has enough tokens for the weight tiles to be
+// real dense contractions.  Same outputs as the CUDA-core kernels of
+// kd_kernels.cuh; in addition the producers write the bf16 hi/lo pairs
+// (h1lo, act_hi/act_lo) that the next tensor-core kernel multiplies.
+//
+// Tensor maps (one per weight matrix, box 64 K x 128 rows, 128B swizzle):
+//   0 Wqkv [Nqkv, H]   1 Wo [H, A]   2 routed gate/up [E*2I, H]
+//   3 routed down [E*H, I]   4 shared gate/up [2I, H]   5 shared down [H, I]
+#pragma once
+
+#include "kd_kernels.cuh"
+#include "kd_mma.cuh"
+
+namespace kd {
+
+struct MmaMaps {
+  CUtensorMap m[6];
+};
+
+KD_DEV void store_hilo(uint16_t* hi, uint16_t* lo, size_t o, float v) {
+  const uint16_t h = f32_to_bf16_bits(v);
+  hi[o] = h;
+  lo[o] = f32_to_bf16_bits(v - __uint_as_float((uint32_t)h << 16));
+}
+
+// ------------------------------------------------------------------ QKV + o-proj
+
+struct MmaProjPlan {
+  const LayerDev* L; Acts a; const MmaMaps* maps;
+  int tq, to, cq, co;   // tiles and K chunks per tile of QKV and o-proj
+  KD_DEV int num_tiles() const { return tq + to; }
+  KD_DEV long long tile_start(int t) const {
+    return t <= tq ? (long long)t * cq : (long long)tq * cq + (long long)(t - tq) * co;
+  }
+  KD_DEV MUnit tile_unit(int t) const {
+    MUnit m{};
+    const bool q = t < tq;
+    m.map = q ? 0 : 1;
+    m.lrow = m.row = (q ? t : t - tq) * 128;
+    m.tag = q ? 0 : 1;
+    m.tok0 = 0;
+    m.ntok = a.M;
+    return m;
+  }
+  KD_DEV const CUtensorMap* map(int id) const { return &maps->m[id]; }
+  KD_DEV bool split_b() const { return false; }
+  KD_DEV const uint16_t* b_row(const MUnit& m, int j, int) const {
+    return m.tag == 0 ? a.x + (size_t)j * L->H : a.attn + (size_t)j * L->A;
+  }
+  KD_DEV bool paired() const { return false; }
+  KD_DEV void epilogue(const MUnit& m, int r, int j, float v) const {
+    const int row = m.lrow + r;
+    if (m.tag == 0) {
+      L->qkv[(size_t)j * L->Nqkv + row] = f32_to_bf16_bits(v);
+    } else {
+      const size_t o = (size_t)j * L->H + row;
+      const float h = __uint_as_float((uint32_t)a.x[o] << 16) + v;
+      L->h1f[o] = h;
+      store_hilo(L->h1b, L->h1lo, o, h);
+    }
+  }
+  KD_DEV void epilogue2(const MUnit&, int, int, float, float) const {}
+  KD_DEV float* ws() const { return L->ws_main; }
+  KD_DEV unsigned* tile_cnt() const { return L->tcnt_main; }
+  KD_DEV bool wants_unit_done() const { return false; }
+  KD_DEV void unit_done(const MUnit&, MmaShared&) const {}
+};
+
+__global__ void __launch_bounds__(kMThreads, 1) mma_proj_kernel(LayerDev L, Acts a,
+                                                                const __grid_constant__ MmaMaps maps) {
+  extern __shared__ uint8_t smem[];
+  MmaProjPlan p;
+  p.L = &L; p.a = a; p.maps = &maps;
+  p.tq = L.Nqkv / 128; p.to = L.H / 128; p.cq = L.H / kKChunk; p.co = L.A / kKChunk;
+  pdl_wait();
+  pdl_launch_dependents();
+  mma_run(p, smem, L.err);
+}
+
+// ------------------------------------------------------------------ gate/up
+
+// Routed: tiles of the active experts' interleaved gate/up rows (2I/128 per
+// expert); shared: the shared expert's.  B = h1 as a bf16 hi/lo pair.
+struct MmaGateUpPlan {
+  const LayerDev* L; int M; bool shared; const MmaMaps* maps; Route rt; int n_act;
+  KD_DEV int tiles_per() const { return 2 * L->I / 128; }
+  KD_DEV int num_tiles() const { return (shared ? 1 : n_act) * tiles_per(); }
+  KD_DEV long long tile_start(int t) const { return (long long)t * (L->H / kKChunk); }
+  KD_DEV MUnit tile_unit(int t) const {
+    MUnit m{};
+    const int a = t / tiles_per(), tt = t % tiles_per();
+    if (shared) {
+      m.map = 4; m.row = tt * 128; m.tag = -1; m.tok0 = 0; m.ntok = M;
+    } else {
+      const int e = rt.act[a];
+      m.map = 2; m.row = e * 2 * L->I + tt * 128; m.tag = e;
+      m.tok0 = rt.off[e]; m.ntok = rt.cnt[e];
+    }
+    m.lrow = tt * 128;
+    return m;
+  }
+  KD_DEV const CUtensorMap* map(int id) const { return &maps->m[id]; }
+  KD_DEV bool split_b() const { return true; }
+  KD_DEV const uint16_t* b_row(const MUnit& m, int j, int h) const {
+    const int t = shared ? j : rt.perm[m.tok0 + j] / L->k;
+    return (h ? L->h1lo : L->h1b) + (size_t)t * L->H;
+  }
+  KD_DEV bool paired() const { return true; }
+  KD_DEV void epilogue(const MUnit&, int, int, float) const {}
+  KD_DEV void epilogue2(const MUnit& m, int p, int j, float g, float u) const {
+    const int i = m.lrow / 2 + p;
+    const float v = silu(g) * u;
+    const size_t o = shared ? (size_t)j * L->I + i : (size_t)(m.tok0 + j) * L->I + i;
+    if (shared) {
+      L->act_sh[o] = v;
+      store_hilo(L->act_sh_hi, L->act_sh_lo, o, v);
+    } else {
+      L->act[o] = v;
+      store_hilo(L->act_hi, L->act_lo, o, v);
+    }
+  }
+  KD_DEV float* ws() const { return shared ? L->ws_side : L->ws_main; }
+  KD_DEV unsigned* tile_cnt() const { return shared ? L->tcnt_side : L->tcnt_main; }
+  KD_DEV bool wants_unit_done() const { return false; }
+  KD_DEV void unit_done(const MUnit&, MmaShared&) const {}
+};
+
+__global__ void __launch_bounds__(kMThreads, 1) mma_gateup_kernel(LayerDev L, int M, int shared,
+                                                                  const __grid_constant__ MmaMaps maps) {
+  extern __shared__ uint8_t smem[];
+  MmaGateUpPlan p;
+  p.L = &L; p.M = M; p.shared = shared != 0; p.maps = &maps; p.n_act = 1;
+  if (!shared) {
+    pdl_wait();
+    pdl_launch_dependents();
+    p.rt = carve_route(reinterpret_cast<int*>(smem + kMmaSmem), L.E, M * L.k);
+    route_tokens(L, M, p.rt, blockIdx.x == 0);
+    p.n_act = *p.rt.n_act;
+  }
+  mma_run(p, smem, L.err);
+}
+
+// ------------------------------------------------------------------ down + combine
+
+// Tiles of the active experts' down projections (H/128 per expert), then the
+// shared expert's.  B = the SwiGLU activations as a bf16 hi/lo pair.  A CTA
+// that completes a tile counts its 128 rows into the 64-row blocks; the CTA
+// completing a block (every entry) writes that block of the layer output.
+struct MmaDownPlan {
+  const LayerDev* L; int M; int n_act; const MmaMaps* maps; uint16_t* out;
+  KD_DEV int tiles_per() const { return L->H / 128; }
+  KD_DEV int num_tiles() const { return (n_act + L->S) * tiles_per(); }
+  KD_DEV long long tile_start(int t) const { return (long long)t * (L->I / kKChunk); }
+  KD_DEV MUnit tile_unit(int t) const {
+    MUnit m{};
+    const int a = t / tiles_per(), tt = t % tiles_per();
+    if (a >= n_act) {
+      m.map = 5; m.row = tt * 128; m.tag = -1; m.tok0 = 0; m.ntok = M;
+    } else {
+      const int e = L->active[a];
+      m.map = 3; m.row = e * L->H + tt * 128; m.tag = e;
+      m.tok0 = L->offsets[e]; m.ntok = L->counts[e];
+    }
+    m.lrow = tt * 128;
+    return m;
+  }
+  KD_DEV const CUtensorMap* map(int id) const { return &maps->m[id]; }
+  KD_DEV bool split_b() const { return true; }
+  KD_DEV const uint16_t* b_row(const MUnit& m, int j, int h) const {
+    if (m.tag < 0) return (h ? L->act_sh_lo : L->act_sh_hi) + (size_t)j * L->I;
+    return (h ? L->act_lo : L->act_hi) + (size_t)(m.tok0 + j) * L->I;
+  }
+  KD_DEV bool paired() const { return false; }
+  KD_DEV void epilogue(const MUnit& m, int r, int j, float v) const {
+    const int h = m.lrow + r;
+    if (m.tag < 0) L->ysh[(size_t)j * L->H + h] = v;
+    else L->yr[(size_t)L->perm[m.tok0 + j] * L->H + h] = v;
+  }
+  KD_DEV void epilogue2(const MUnit&, int, int, float, float) const {}
+  KD_DEV float* ws() const { return L->ws_main; }
+  KD_DEV unsigned* tile_cnt() const { return L->tcnt_main; }
+  KD_DEV bool wants_unit_done() const { return true; }
+  // epilogue warps only (128 threads, named barrier 2)
+  KD_DEV void unit_done(const MUnit& m, MmaShared& sh) const {
+    const int target = 64 * (n_act + L->S);
+    const int et = threadIdx.x - 128;
+    if (et == 0) {
+      __threadfence();
+      int nb = 0;
+      for (int b = m.lrow / 64; b < (m.lrow + 128) / 64; ++b) {
+        const unsigned prev = atomicAdd(L->hcnt + b, 64u);
+        if (prev + 64u == (unsigned)target) {
+          L->hcnt[b] = 0u;
+          sh.blist[nb++] = b;
+        }
+      }
+      sh.misc[1] = nb;
+      __threadfence();
+    }
+    named_bar_sync(2, 128);
+    const int nb = sh.misc[1];
+    for (int q = 0; q < nb; ++q) {
+      const int b = sh.blist[q];
+      for (int e = et; e < 64 * M; e += 128) {
+        const int t = e / 64, h = b * 64 + e % 64;
+        const size_t o = (size_t)t * L->H + h;
+        float v = L->h1f[o];
+        if (L->S) v += __ldcg(L->ysh + o);
+        for (int j = 0; j < L->k; ++j)
+          v += L->gates[t * L->k + j] * __ldcg(L->yr + ((size_t)t * L->k + j) * L->H + h);
+        out[o] = f32_to_bf16_bits(v);
+      }
+    }
+    named_bar_sync(2, 128);
+  }
+};
+
+__global__ void __launch_bounds__(kMThreads, 1) mma_down_kernel(LayerDev L, int M, uint16_t* out,
+                                                                const __grid_constant__ MmaMaps maps) {
+  extern __shared__ uint8_t smem[];
+  pdl_wait();
+  pdl_launch_dependents();
+  MmaDownPlan p;
+  p.L = &L; p.M = M; p.out = out; p.maps = &maps;
+  p.n_act = *(volatile int*)L.n_active;
+  mma_run(p, smem, L.err);
+}
+
+}  // namespace kd

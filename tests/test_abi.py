@@ -47,10 +47,11 @@ def test_host_side_argument_errors(kd):
     # invalid configurations are rejected before any device call
     bad = [dict(hidden=100), dict(top_k=0), dict(top_k=9, n_experts=8), dict(max_tokens=65),
            dict(max_tokens=0), dict(wdtype=7), dict(n_shared=2), dict(inter=96), dict(n_experts=2000),
-           dict(hidden=32768)]
+           dict(hidden=32768), dict(mma_min_tokens=-1)]
     for b in bad:
         f = dict(hidden=256, q_heads=4, kv_heads=1, head_dim=64, n_experts=8, top_k=2,
-                 n_shared=1, inter=128, wdtype=0, layer_id=0, max_tokens=4, router_bias=None)
+                 n_shared=1, inter=128, wdtype=0, layer_id=0, max_tokens=4, router_bias=None,
+                 mma_min_tokens=0)
         f.update(b)
         cfg = kd._Config(**f)
         assert L.kd_layer_create(ctypes.byref(cfg), 0, ctypes.byref(h)) == kd.KD_EINVAL, b
