@@ -119,7 +119,8 @@ struct MUnit {
 KD_DEV int pad16(int n) { return (n + 15) & ~15; }
 
 // Stream-K partition of a launch: the K chunks of all tiles, concatenated in
-// tile order, are cut into gridDim.x equal ranges; CTA b takes range b.  A
+// tile order, are cut into min(gridDim.x, chunks) equal ranges; CTA b takes
+// range b.  A
 // tile that straddles ranges is computed in parts (one per CTA, part p by
 // CTA first_owner + p) and summed, in part order, by the part that finishes
 // last.  Only a CTA's first and last unit can be partial, so the partials
@@ -130,14 +131,17 @@ KD_DEV int pad16(int n) { return (n + 15) & ~15; }
 template <class Plan>
 struct CtaUnits {
   const Plan& plan;
-  long long T, lo, hi;
+  long long T, G, lo, hi;
   int t, nt;
   KD_DEV explicit CtaUnits(const Plan& p) : plan(p) {
     nt = plan.num_tiles();
     T = plan.tile_start(nt);
-    const long long G = gridDim.x, b = blockIdx.x;
-    lo = b * T / G;
-    hi = (b + 1) * T / G;
+    // with fewer chunks than CTAs only the first T CTAs get one chunk each, so
+    // that every CTA between two owners of a tile owns part of it
+    G = T < (long long)gridDim.x ? T : (long long)gridDim.x;
+    const long long b = blockIdx.x;
+    lo = b < G ? b * T / G : T;
+    hi = b < G ? (b + 1) * T / G : T;
     // first tile whose chunk range reaches past lo
     int a = 0, z = nt;
     while (a < z) {
@@ -147,11 +151,8 @@ struct CtaUnits {
     }
     t = a;
   }
-  // CTA owning chunk c: the largest b with floor(b*T/G) <= c
-  KD_DEV long long owner(long long c) const {
-    const long long G = gridDim.x;
-    return ((c + 1) * G + T - 1) / T - 1;
-  }
+  // CTA owning chunk c: the largest b < G with floor(b*T/G) <= c
+  KD_DEV long long owner(long long c) const { return ((c + 1) * G + T - 1) / T - 1; }
   KD_DEV bool next(MUnit& m) {
     if (lo >= hi) return false;
     long long cs = 0, ce = 0;
