@@ -241,9 +241,21 @@ KD_DEV void mma_producer_a(const Plan& plan, MmaShared& sh, unsigned* err) {
   }
 }
 
-// Two warps (64 threads) write the B tile of every stage: token rows j <
-// ntok (zeros up to N), 128 bytes (64 K) each, 16-byte chunk c of row r at
-// r*128 + ((c ^ (r & 7)) * 16) -- the 128-byte swizzle the A tile has.
+KD_DEV void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;"
+               ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes) : "memory");
+}
+KD_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+KD_DEV void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// Two warps (64 threads) write the B tile of every stage with cp.async:
+// token rows j < ntok (zero-filled up to N), 128 bytes (64 K) each, 16-byte
+// chunk c of row r at r*128 + ((c ^ (r & 7)) * 16) -- the 128-byte swizzle
+// the A tile has.  A stage is handed to the MMA (proxy fence + arrive) kLag
+// stages later, so that kLag stages of gathers are in flight per thread.
+constexpr int kBLag = 2;
+
 template <class Plan>
 KD_DEV void mma_producer_b(const Plan& plan, MmaShared& sh, unsigned* err) {
   const int t = threadIdx.x - 64;  // 0..63
@@ -261,14 +273,22 @@ KD_DEV void mma_producer_b(const Plan& plan, MmaShared& sh, unsigned* err) {
       const int k0 = (m.kc0 + c) * kKChunk;
       for (int q = t; q < nh * N * 8; q += 64) {
         const int h = q / (N * 8), r = (q / 8) % N, ch = q % 8;
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (r < m.ntok) v = ld_nc_v4(plan.b_row(m, r, h) + k0 + ch * 8);
-        *reinterpret_cast<uint4*>(bt + (size_t)h * N * 128 + r * 128 + ((ch ^ (r & 7)) * 16)) = v;
+        const bool live = r < m.ntok;
+        const uint16_t* src = plan.b_row(m, live ? r : 0, h) + k0 + ch * 8;
+        cp_async16(bt + (size_t)h * N * 128 + r * 128 + ((ch ^ (r & 7)) * 16), src, live ? 16u : 0u);
       }
-      fence_proxy_async_smem();   // generic-proxy writes -> visible to the tensor core
-      mbar_arrive(&sh.full[s]);
+      cp_async_commit();
+      if (it >= (uint32_t)kBLag) {
+        cp_async_wait<kBLag>();
+        fence_proxy_async_smem();   // generic-proxy writes -> visible to the tensor core
+        mbar_arrive(&sh.full[(it - kBLag) % kMStages]);
+      }
     }
   }
+  cp_async_wait<0>();
+  fence_proxy_async_smem();
+  for (uint32_t j = it > (uint32_t)kBLag ? it - kBLag : 0; j < it; ++j)
+    mbar_arrive(&sh.full[j % kMStages]);
 }
 
 template <class Plan>
