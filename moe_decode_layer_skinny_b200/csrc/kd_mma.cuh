@@ -95,14 +95,13 @@ KD_DEV void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "
 // ------------------------------------------------------------------ engine
 
 constexpr int kMThreads = 256;
-constexpr int kMStages = 6;
+constexpr int kMaxMStages = 16;
 constexpr int kATileBytes = 128 * 128;                // 128 rows x 64 bf16
-constexpr int kBTileBytes = 64 * 128 * 2;             // up to 64 tokens x 64 bf16, hi + lo
-constexpr int kMStageBytes = kATileBytes + kBTileBytes;
+constexpr int kMRingBytes = 6 * (kATileBytes + 64 * 128 * 2);  // 192 KB of stages
 constexpr int kMaxN = 64;                             // tokens per MMA (N)
 constexpr int kKChunk = 64;                           // K elements per stage
 constexpr size_t kWsFloatsPerCta = 2 * 128 * 64;     // split-K partial slots of one CTA
-constexpr size_t kMmaSmem = (size_t)kMStages * kMStageBytes + 1024 /*align*/ + 1024 /*barriers, lists*/;
+constexpr size_t kMmaSmem = (size_t)kMRingBytes + 1024 /*align*/ + 1024 /*barriers, lists*/;
 
 // One unit of work: K chunks [kc0, kc0 + nkc) of a 128-row weight tile.
 struct MUnit {
@@ -177,9 +176,10 @@ struct CtaUnits {
 };
 
 struct MmaShared {
-  uint8_t* stage;        // kMStages x kMStageBytes, 1024-aligned
-  uint64_t* full;        // [kMStages] A landed (tx) + B written (2 warp arrivals)
-  uint64_t* empty;       // [kMStages] MMAs of the stage done
+  uint8_t* stage;        // nst x stage_bytes, 1024-aligned
+  int nst, stage_bytes;  // stage count and size (A tile + B tile for the launch's largest N)
+  uint64_t* full;        // [nst] A landed (tx) + B written (64 thread arrivals)
+  uint64_t* empty;       // [nst] MMAs of the stage done
   uint64_t* accfull;     // [2] accumulator buffer ready for the epilogue
   uint64_t* accempty;    // [2] epilogue done reading the accumulator
   uint32_t* tmem_base;
@@ -188,14 +188,19 @@ struct MmaShared {
   int* blist;            // [128] combine block list
 };
 
-KD_DEV MmaShared carve_mma_smem(uint8_t* raw) {
+// The ring holds as many stages as fit: a stage is the 16 KB weight tile plus
+// the B tile for the launch's largest token count (hi + lo when split).
+KD_DEV MmaShared carve_mma_smem(uint8_t* raw, int nmax, bool split) {
   MmaShared s;
+  s.stage_bytes = kATileBytes + pad16(nmax) * 128 * (split ? 2 : 1);
+  s.nst = kMRingBytes / s.stage_bytes;
+  if (s.nst > kMaxMStages) s.nst = kMaxMStages;
   uintptr_t p = (reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023);
   s.stage = reinterpret_cast<uint8_t*>(p);
-  p += (size_t)kMStages * kMStageBytes;
+  p += (size_t)kMRingBytes;
   s.full = reinterpret_cast<uint64_t*>(p);
-  s.empty = s.full + kMStages;
-  s.accfull = s.empty + kMStages;
+  s.empty = s.full + kMaxMStages;
+  s.accfull = s.empty + kMaxMStages;
   s.accempty = s.accfull + 2;
   s.tmem_base = reinterpret_cast<uint32_t*>(s.accempty + 2);
   s.abort_flag = reinterpret_cast<int*>(s.tmem_base + 1);
@@ -231,11 +236,11 @@ KD_DEV void mma_producer_a(const Plan& plan, MmaShared& sh, unsigned* err) {
   while (units.next(m)) {
     const CUtensorMap* map = plan.map(m.map);
     for (int c = 0; c < m.nkc; ++c, ++it) {
-      const int s = it % kMStages;
-      const uint32_t ph = (it / kMStages) & 1u;
+      const int s = it % sh.nst;
+      const uint32_t ph = (it / sh.nst) & 1u;
       mwait(&sh.empty[s], ph ^ 1u, sh.abort_flag, err);
       mbar_arrive_expect_tx(&sh.full[s], kATileBytes);
-      tma_load_2d(sh.stage + (size_t)s * kMStageBytes, map, (m.kc0 + c) * kKChunk, m.row,
+      tma_load_2d(sh.stage + (size_t)s * sh.stage_bytes, map, (m.kc0 + c) * kKChunk, m.row,
                   &sh.full[s]);
     }
   }
@@ -254,7 +259,7 @@ KD_DEV void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : 
 // chunk c of row r at r*128 + ((c ^ (r & 7)) * 16) -- the 128-byte swizzle
 // the A tile has.  A stage is handed to the MMA (proxy fence + arrive) kLag
 // stages later, so that kLag stages of gathers are in flight per thread.
-constexpr int kBLag = 2;
+constexpr int kBLag = 4;   // < the smallest ring (6 stages)
 
 template <class Plan>
 KD_DEV void mma_producer_b(const Plan& plan, MmaShared& sh, unsigned* err) {
@@ -266,10 +271,10 @@ KD_DEV void mma_producer_b(const Plan& plan, MmaShared& sh, unsigned* err) {
   while (units.next(m)) {
     const int N = pad16(m.ntok);
     for (int c = 0; c < m.nkc; ++c, ++it) {
-      const int s = it % kMStages;
-      const uint32_t ph = (it / kMStages) & 1u;
+      const int s = it % sh.nst;
+      const uint32_t ph = (it / sh.nst) & 1u;
       mwait(&sh.empty[s], ph ^ 1u, sh.abort_flag, err);
-      uint8_t* bt = sh.stage + (size_t)s * kMStageBytes + kATileBytes;
+      uint8_t* bt = sh.stage + (size_t)s * sh.stage_bytes + kATileBytes;
       const int k0 = (m.kc0 + c) * kKChunk;
       for (int q = t; q < nh * N * 8; q += 64) {
         const int h = q / (N * 8), r = (q / 8) % N, ch = q % 8;
@@ -281,14 +286,14 @@ KD_DEV void mma_producer_b(const Plan& plan, MmaShared& sh, unsigned* err) {
       if (it >= (uint32_t)kBLag) {
         cp_async_wait<kBLag>();
         fence_proxy_async_smem();   // generic-proxy writes -> visible to the tensor core
-        mbar_arrive(&sh.full[(it - kBLag) % kMStages]);
+        mbar_arrive(&sh.full[(it - kBLag) % sh.nst]);
       }
     }
   }
   cp_async_wait<0>();
   fence_proxy_async_smem();
   for (uint32_t j = it > (uint32_t)kBLag ? it - kBLag : 0; j < it; ++j)
-    mbar_arrive(&sh.full[j % kMStages]);
+    mbar_arrive(&sh.full[j % sh.nst]);
 }
 
 template <class Plan>
@@ -305,11 +310,11 @@ KD_DEV void mma_issuer(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigned*
     mwait(&sh.accempty[buf], ((nu_local >> 1) & 1u) ^ 1u, sh.abort_flag, err);
     tc_fence_after();
     for (int c = 0; c < m.nkc; ++c, ++it) {
-      const int s = it % kMStages;
-      const uint32_t ph = (it / kMStages) & 1u;
+      const int s = it % sh.nst;
+      const uint32_t ph = (it / sh.nst) & 1u;
       mwait(&sh.full[s], ph, sh.abort_flag, err);
       tc_fence_after();
-      const uint32_t a = smem_u32(sh.stage + (size_t)s * kMStageBytes);
+      const uint32_t a = smem_u32(sh.stage + (size_t)s * sh.stage_bytes);
       const uint32_t b = a + kATileBytes;
 #pragma unroll
       for (int k = 0; k < kKChunk / 16; ++k) {
@@ -402,10 +407,10 @@ KD_DEV void mma_epilogue(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigne
 
 template <class Plan>
 KD_DEV void mma_run(const Plan& plan, uint8_t* smem_raw, unsigned* err) {
-  MmaShared sh = carve_mma_smem(smem_raw);
+  MmaShared sh = carve_mma_smem(smem_raw, plan.max_n(), plan.split_b());
   const int warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kMStages; ++i) {
+    for (int i = 0; i < sh.nst; ++i) {
       mbar_init(&sh.full[i], 1 + 64);  // A transaction arrive + the 64 B threads
       mbar_init(&sh.empty[i], 1);
     }

@@ -44,6 +44,7 @@ struct MmaProjPlan {
     return m;
   }
   KD_DEV const CUtensorMap* map(int id) const { return &maps->m[id]; }
+  KD_DEV int max_n() const { return a.M; }
   KD_DEV bool split_b() const { return false; }
   KD_DEV const uint16_t* b_row(const MUnit& m, int j, int) const {
     return m.tag == 0 ? a.x + (size_t)j * L->H : a.attn + (size_t)j * L->A;
@@ -101,6 +102,7 @@ struct MmaGateUpPlan {
     return m;
   }
   KD_DEV const CUtensorMap* map(int id) const { return &maps->m[id]; }
+  KD_DEV int max_n() const { return M; }
   KD_DEV bool split_b() const { return true; }
   KD_DEV const uint16_t* b_row(const MUnit& m, int j, int h) const {
     const int t = shared ? j : rt.perm[m.tok0 + j] / L->k;
@@ -166,6 +168,7 @@ struct MmaDownPlan {
     return m;
   }
   KD_DEV const CUtensorMap* map(int id) const { return &maps->m[id]; }
+  KD_DEV int max_n() const { return M; }
   KD_DEV bool split_b() const { return true; }
   KD_DEV const uint16_t* b_row(const MUnit& m, int j, int h) const {
     if (m.tag < 0) return (h ? L->act_sh_lo : L->act_sh_hi) + (size_t)j * L->I;
