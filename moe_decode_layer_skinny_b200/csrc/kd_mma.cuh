@@ -217,6 +217,22 @@ KD_DEV bool mwait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, unsi
   return false;
 }
 
+// Same for waiters off the critical path (the epilogue): sleep between polls
+// so that their spinning does not take issue slots from the producers.
+KD_DEV bool mwait_lazy(uint64_t* bar, uint32_t parity, volatile int* abort_flag, unsigned* err) {
+  if (*abort_flag) return false;
+  const uint64_t t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity)) {
+    __nanosleep(200);
+    if (globaltimer() - t0 > kWaitLimitNs) {
+      *abort_flag = 1;
+      set_error(err, ERR_WAIT_MMA);
+      return false;
+    }
+  }
+  return true;
+}
+
 // Plan interface (all methods KD_DEV const):
 //   int num_tiles(); long long tile_start(int t); MUnit tile_unit(int t)   (see CtaUnits)
 //   const CUtensorMap* map(int id)
@@ -263,25 +279,36 @@ constexpr int kBLag = 4;   // < the smallest ring (6 stages)
 
 template <class Plan>
 KD_DEV void mma_producer_b(const Plan& plan, MmaShared& sh, unsigned* err) {
-  const int t = threadIdx.x - 64;  // 0..63
+  constexpr int kQ = 2 * kMaxN * 8 / 64;   // 16-byte copies per thread per stage (at most)
+  const int t = threadIdx.x - 64;          // 0..63
   const int nh = plan.split_b() ? 2 : 1;
   uint32_t it = 0;
   CtaUnits<Plan> units(plan);
   MUnit m;
   while (units.next(m)) {
     const int N = pad16(m.ntok);
+    // this thread's copies for the whole unit: source row (+ chunk), smem
+    // offset within the B tile, and byte count (0 = zero fill)
+    const uint16_t* src[kQ];
+    uint32_t off[kQ], nb[kQ];
+#pragma unroll
+    for (int i = 0; i < kQ; ++i) {
+      const int q = t + 64 * i;
+      const int h = q / (N * 8), r = (q / 8) % N, ch = q % 8;
+      const bool live = q < nh * N * 8 && r < m.ntok;
+      src[i] = plan.b_row(m, live ? r : 0, q < nh * N * 8 ? h : 0) + ch * 8;
+      off[i] = (uint32_t)(h * N * 128 + r * 128 + ((ch ^ (r & 7)) * 16));
+      nb[i] = q < nh * N * 8 ? (live ? 16u : 0u) : 0xFFFFFFFFu;   // ~0: no copy
+    }
     for (int c = 0; c < m.nkc; ++c, ++it) {
       const int s = it % sh.nst;
       const uint32_t ph = (it / sh.nst) & 1u;
       mwait(&sh.empty[s], ph ^ 1u, sh.abort_flag, err);
       uint8_t* bt = sh.stage + (size_t)s * sh.stage_bytes + kATileBytes;
       const int k0 = (m.kc0 + c) * kKChunk;
-      for (int q = t; q < nh * N * 8; q += 64) {
-        const int h = q / (N * 8), r = (q / 8) % N, ch = q % 8;
-        const bool live = r < m.ntok;
-        const uint16_t* src = plan.b_row(m, live ? r : 0, h) + k0 + ch * 8;
-        cp_async16(bt + (size_t)h * N * 128 + r * 128 + ((ch ^ (r & 7)) * 16), src, live ? 16u : 0u);
-      }
+#pragma unroll
+      for (int i = 0; i < kQ; ++i)
+        if (nb[i] != 0xFFFFFFFFu) cp_async16(bt + off[i], src[i] + k0, nb[i]);
       cp_async_commit();
       if (it >= (uint32_t)kBLag) {
         cp_async_wait<kBLag>();
@@ -340,7 +367,7 @@ KD_DEV void mma_epilogue(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigne
   for (; units.next(m); ++nu_local) {
     const int N = pad16(m.ntok);
     const int buf = nu_local & 1;
-    mwait(&sh.accfull[buf], (nu_local >> 1) & 1u, sh.abort_flag, err);
+    mwait_lazy(&sh.accfull[buf], (nu_local >> 1) & 1u, sh.abort_flag, err);
     tc_fence_after();
     const uint32_t ta = tmem + ((uint32_t)(ew * 32) << 16) + (uint32_t)(buf * kMaxN);
 #pragma unroll
