@@ -296,6 +296,17 @@ def make_layer(w, layer_id=0):
     return kd.Layer(spec, seed=w.seed)
 
 
+def with_experts(w, n_experts: int):
+    """The workload with fewer routed experts (same shapes per expert, same
+    top-k): a small device footprint for profiling captures."""
+    import dataclasses
+    if not n_experts:
+        return w
+    d = dataclasses.replace(w.dims, n_experts=n_experts)
+    return dataclasses.replace(w, dims=d, name=f"{w.name}_e{n_experts}",
+                               zipf_s=w.zipf_s)
+
+
 def bench_single(w, steps, warmup, flush, pg, local, peak):
     layer = make_layer(w)
     try:
@@ -397,7 +408,7 @@ def run_kd(args):
     peak, peak_src = load_peak()
     flush = L2Flush()
     W = kdgen.WORKLOADS
-    main = W[args.workload]
+    main = with_experts(W[args.workload], args.experts)
     res, layer, x, a, kb, kt = bench_single(main, args.steps, args.warmup, flush, pg, local, peak)
     dev_index = torch.cuda.current_device()
     vis = os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")
@@ -518,6 +529,8 @@ def main():
     ap.add_argument("--workload", default="batch1")
     ap.add_argument("--main-only", action="store_true", help="skip the secondary workloads")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
+    ap.add_argument("--experts", type=int, default=0,
+                    help="profiling only: routed experts of the main workload (default: its own)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
