@@ -39,6 +39,24 @@ PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
 FALLBACK_HBM_GBS = 6650.0
 
 
+def profiled_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of `kernel` from the committed ncu capture, or None
+    when there is none for this kernel/workload or its sources changed since."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            t = json.load(f)
+        if t["kernel"] != kernel or not t["workload"].startswith(workload):
+            return None
+        h = hashlib.sha256()
+        for src in t["source_files"]:
+            with open(os.path.join(ROOT, src), "rb") as f:
+                h.update(f.read())
+        return t["dram_bytes_per_launch"] if h.hexdigest()[:16] == t["source_sha256_16"] else None
+    except Exception:
+        return None
+
+
 def load_peak():
     try:
         with open(PEAKS_PATH) as f:
@@ -454,8 +472,8 @@ def run_kd(args):
     dom = max(KNAMES, key=lambda n: kt[n])
     ach = kb[dom] / (kt[dom] * 1e-3) / 1e9
     out["roofline"] = {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": peak, "unit": "GB/s",
-                       "frac": ach / peak, "traffic": None,
-                       "algorithmic_bytes_per_launch": kb[dom]}
+                       "frac": ach / peak, "traffic": profiled_traffic(dom, main.name),
+                       "algorithmic_bytes_per_launch": kb[dom], "peak_src": peak_src}
     # secondary workloads
     if not args.main_only:
         wl = {}
