@@ -96,10 +96,11 @@ KD_DEV void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "
 
 constexpr int kMThreads = 256;
 constexpr int kMaxMStages = 16;
-constexpr int kATileBytes = 128 * 128;                // 128 rows x 64 bf16
-constexpr int kMRingBytes = 6 * (kATileBytes + 64 * 128 * 2);  // 192 KB of stages
+constexpr int kATileBytes = 128 * 128;                // 128 rows x 64 bf16 (one swizzle atom wide)
+constexpr int kSub = 2;                               // 64-K sub-tiles per stage
+constexpr int kMRingBytes = 3 * kSub * (kATileBytes + 64 * 128 * 2);  // 192 KB of stages
 constexpr int kMaxN = 64;                             // tokens per MMA (N)
-constexpr int kKChunk = 64;                           // K elements per stage
+constexpr int kKChunk = 64 * kSub;                    // K elements per stage
 constexpr size_t kWsFloatsPerCta = 2 * 128 * 64;     // split-K partial slots of one CTA
 constexpr size_t kMmaSmem = (size_t)kMRingBytes + 1024 /*align*/ + 1024 /*barriers, lists*/;
 
@@ -188,11 +189,15 @@ struct MmaShared {
   int* blist;            // [128] combine block list
 };
 
-// The ring holds as many stages as fit: a stage is the 16 KB weight tile plus
-// the B tile for the launch's largest token count (hi + lo when split).
+// The ring holds as many stages as fit.  A stage covers 128 K: kSub weight
+// sub-tiles [128 rows x 64 K] (16 KB each, so every row contributes 256
+// contiguous bytes per stage), then kSub B sub-tiles for the launch's largest
+// token count (hi + lo when split).
+KD_DEV int b_sub_bytes(int n, bool split) { return pad16(n) * 128 * (split ? 2 : 1); }
+
 KD_DEV MmaShared carve_mma_smem(uint8_t* raw, int nmax, bool split) {
   MmaShared s;
-  s.stage_bytes = kATileBytes + pad16(nmax) * 128 * (split ? 2 : 1);
+  s.stage_bytes = kSub * (kATileBytes + b_sub_bytes(nmax, split));
   s.nst = kMRingBytes / s.stage_bytes;
   if (s.nst > kMaxMStages) s.nst = kMaxMStages;
   uintptr_t p = (reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023);
@@ -255,9 +260,11 @@ KD_DEV void mma_producer_a(const Plan& plan, MmaShared& sh, unsigned* err) {
       const int s = it % sh.nst;
       const uint32_t ph = (it / sh.nst) & 1u;
       mwait(&sh.empty[s], ph ^ 1u, sh.abort_flag, err);
-      mbar_arrive_expect_tx(&sh.full[s], kATileBytes);
-      tma_load_2d(sh.stage + (size_t)s * sh.stage_bytes, map, (m.kc0 + c) * kKChunk, m.row,
-                  &sh.full[s]);
+      mbar_arrive_expect_tx(&sh.full[s], kSub * kATileBytes);
+#pragma unroll
+      for (int u = 0; u < kSub; ++u)
+        tma_load_2d(sh.stage + (size_t)s * sh.stage_bytes + u * kATileBytes, map,
+                    (m.kc0 + c) * kKChunk + 64 * u, m.row, &sh.full[s]);
     }
   }
 }
@@ -275,7 +282,7 @@ KD_DEV void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : 
 // chunk c of row r at r*128 + ((c ^ (r & 7)) * 16) -- the 128-byte swizzle
 // the A tile has.  A stage is handed to the MMA (proxy fence + arrive) kLag
 // stages later, so that kLag stages of gathers are in flight per thread.
-constexpr int kBLag = 4;   // < the smallest ring (6 stages)
+constexpr int kBLag = 2;   // < the smallest ring (3 stages)
 
 template <class Plan>
 KD_DEV void mma_producer_b(const Plan& plan, MmaShared& sh, unsigned* err) {
@@ -304,11 +311,15 @@ KD_DEV void mma_producer_b(const Plan& plan, MmaShared& sh, unsigned* err) {
       const int s = it % sh.nst;
       const uint32_t ph = (it / sh.nst) & 1u;
       mwait(&sh.empty[s], ph ^ 1u, sh.abort_flag, err);
-      uint8_t* bt = sh.stage + (size_t)s * sh.stage_bytes + kATileBytes;
-      const int k0 = (m.kc0 + c) * kKChunk;
+      uint8_t* bt = sh.stage + (size_t)s * sh.stage_bytes + kSub * kATileBytes;
+      const int bsub = b_sub_bytes(N, nh == 2);
 #pragma unroll
-      for (int i = 0; i < kQ; ++i)
-        if (nb[i] != 0xFFFFFFFFu) cp_async16(bt + off[i], src[i] + k0, nb[i]);
+      for (int u = 0; u < kSub; ++u) {
+        const int k0 = (m.kc0 + c) * kKChunk + 64 * u;
+#pragma unroll
+        for (int i = 0; i < kQ; ++i)
+          if (nb[i] != 0xFFFFFFFFu) cp_async16(bt + u * bsub + off[i], src[i] + k0, nb[i]);
+      }
       cp_async_commit();
       if (it >= (uint32_t)kBLag) {
         cp_async_wait<kBLag>();
@@ -341,13 +352,18 @@ KD_DEV void mma_issuer(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigned*
       const uint32_t ph = (it / sh.nst) & 1u;
       mwait(&sh.full[s], ph, sh.abort_flag, err);
       tc_fence_after();
-      const uint32_t a = smem_u32(sh.stage + (size_t)s * sh.stage_bytes);
-      const uint32_t b = a + kATileBytes;
+      const uint32_t a0 = smem_u32(sh.stage + (size_t)s * sh.stage_bytes);
+      const uint32_t b0 = a0 + kSub * kATileBytes;
+      const int bsub = b_sub_bytes(N, split);
 #pragma unroll
-      for (int k = 0; k < kKChunk / 16; ++k) {
-        const uint64_t ad = sw128_desc(a + k * 32);
-        mma_bf16(d, ad, sw128_desc(b + k * 32), idesc, c > 0 || k > 0);
-        if (split) mma_bf16(d, ad, sw128_desc(b + N * 128 + k * 32), idesc, true);
+      for (int u = 0; u < kSub; ++u) {
+        const uint32_t a = a0 + u * kATileBytes, b = b0 + u * bsub;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint64_t ad = sw128_desc(a + k * 32);
+          mma_bf16(d, ad, sw128_desc(b + k * 32), idesc, c > 0 || u > 0 || k > 0);
+          if (split) mma_bf16(d, ad, sw128_desc(b + N * 128 + k * 32), idesc, true);
+        }
       }
       mma_commit(&sh.empty[s]);   // the stage is free once these MMAs are done
     }
