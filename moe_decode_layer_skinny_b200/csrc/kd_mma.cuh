@@ -97,10 +97,9 @@ KD_DEV void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "
 constexpr int kMThreads = 256;
 constexpr int kMaxMStages = 16;
 constexpr int kATileBytes = 128 * 128;                // 128 rows x 64 bf16 (one swizzle atom wide)
-constexpr int kSub = 2;                               // 64-K sub-tiles per stage
-constexpr int kMRingBytes = 3 * kSub * (kATileBytes + 64 * 128 * 2);  // 192 KB of stages
+constexpr int kMaxSub = 2;                            // 64-K sub-tiles per stage (at most)
+constexpr int kMRingBytes = 3 * kMaxSub * (kATileBytes + 64 * 128 * 2);  // 192 KB of stages
 constexpr int kMaxN = 64;                             // tokens per MMA (N)
-constexpr int kKChunk = 64 * kSub;                    // K elements per stage
 constexpr size_t kWsFloatsPerCta = 2 * 128 * 64;     // split-K partial slots of one CTA
 constexpr size_t kMmaSmem = (size_t)kMRingBytes + 1024 /*align*/ + 1024 /*barriers, lists*/;
 
@@ -179,6 +178,7 @@ struct CtaUnits {
 struct MmaShared {
   uint8_t* stage;        // nst x stage_bytes, 1024-aligned
   int nst, stage_bytes;  // stage count and size (A tile + B tile for the launch's largest N)
+  int nsub;              // 64-K sub-tiles per stage
   uint64_t* full;        // [nst] A landed (tx) + B written (64 thread arrivals)
   uint64_t* empty;       // [nst] MMAs of the stage done
   uint64_t* accfull;     // [2] accumulator buffer ready for the epilogue
@@ -189,15 +189,21 @@ struct MmaShared {
   int* blist;            // [128] combine block list
 };
 
-// The ring holds as many stages as fit.  A stage covers 128 K: kSub weight
-// sub-tiles [128 rows x 64 K] (16 KB each, so every row contributes 256
-// contiguous bytes per stage), then kSub B sub-tiles for the launch's largest
-// token count (hi + lo when split).
+// The ring holds as many stages as fit.  A stage covers nsub x 64 K: nsub
+// weight sub-tiles [128 rows x 64 K] (16 KB each; with nsub = 2 every row
+// contributes 256 contiguous bytes per stage), then nsub B sub-tiles for the
+// launch's largest token count (hi + lo when split).  nsub is 2 when that
+// still leaves at least 4 stages, else 1.
 KD_DEV int b_sub_bytes(int n, bool split) { return pad16(n) * 128 * (split ? 2 : 1); }
 
-KD_DEV MmaShared carve_mma_smem(uint8_t* raw, int nmax, bool split) {
+KD_DEV int mma_nsub(int nmax, bool split) {
+  return kMRingBytes / (2 * (kATileBytes + b_sub_bytes(nmax, split))) >= 4 ? 2 : 1;
+}
+
+KD_DEV MmaShared carve_mma_smem(uint8_t* raw, int nmax, bool split, int nsub) {
   MmaShared s;
-  s.stage_bytes = kSub * (kATileBytes + b_sub_bytes(nmax, split));
+  s.nsub = nsub;
+  s.stage_bytes = nsub * (kATileBytes + b_sub_bytes(nmax, split));
   s.nst = kMRingBytes / s.stage_bytes;
   if (s.nst > kMaxMStages) s.nst = kMaxMStages;
   uintptr_t p = (reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023);
@@ -239,7 +245,9 @@ KD_DEV bool mwait_lazy(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
 }
 
 // Plan interface (all methods KD_DEV const):
-//   int num_tiles(); long long tile_start(int t); MUnit tile_unit(int t)   (see CtaUnits)
+//   int num_tiles(); long long tile_start(int t); MUnit tile_unit(int t)   (see CtaUnits;
+//   a chunk is 64 * nsub K elements, nsub = mma_nsub(max_n(), split_b()))
+//   int max_n(); int nsub
 //   const CUtensorMap* map(int id)
 //   bool split_b()                 B is a hi/lo pair
 //   const uint16_t* b_row(const MUnit&, int j, int hilo)   token j's bf16 row
@@ -260,11 +268,10 @@ KD_DEV void mma_producer_a(const Plan& plan, MmaShared& sh, unsigned* err) {
       const int s = it % sh.nst;
       const uint32_t ph = (it / sh.nst) & 1u;
       mwait(&sh.empty[s], ph ^ 1u, sh.abort_flag, err);
-      mbar_arrive_expect_tx(&sh.full[s], kSub * kATileBytes);
-#pragma unroll
-      for (int u = 0; u < kSub; ++u)
+      mbar_arrive_expect_tx(&sh.full[s], sh.nsub * kATileBytes);
+      for (int u = 0; u < sh.nsub; ++u)
         tma_load_2d(sh.stage + (size_t)s * sh.stage_bytes + u * kATileBytes, map,
-                    (m.kc0 + c) * kKChunk + 64 * u, m.row, &sh.full[s]);
+                    ((m.kc0 + c) * sh.nsub + u) * 64, m.row, &sh.full[s]);
     }
   }
 }
@@ -311,11 +318,10 @@ KD_DEV void mma_producer_b(const Plan& plan, MmaShared& sh, unsigned* err) {
       const int s = it % sh.nst;
       const uint32_t ph = (it / sh.nst) & 1u;
       mwait(&sh.empty[s], ph ^ 1u, sh.abort_flag, err);
-      uint8_t* bt = sh.stage + (size_t)s * sh.stage_bytes + kSub * kATileBytes;
+      uint8_t* bt = sh.stage + (size_t)s * sh.stage_bytes + sh.nsub * kATileBytes;
       const int bsub = b_sub_bytes(N, nh == 2);
-#pragma unroll
-      for (int u = 0; u < kSub; ++u) {
-        const int k0 = (m.kc0 + c) * kKChunk + 64 * u;
+      for (int u = 0; u < sh.nsub; ++u) {
+        const int k0 = ((m.kc0 + c) * sh.nsub + u) * 64;
 #pragma unroll
         for (int i = 0; i < kQ; ++i)
           if (nb[i] != 0xFFFFFFFFu) cp_async16(bt + u * bsub + off[i], src[i] + k0, nb[i]);
@@ -353,10 +359,9 @@ KD_DEV void mma_issuer(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigned*
       mwait(&sh.full[s], ph, sh.abort_flag, err);
       tc_fence_after();
       const uint32_t a0 = smem_u32(sh.stage + (size_t)s * sh.stage_bytes);
-      const uint32_t b0 = a0 + kSub * kATileBytes;
+      const uint32_t b0 = a0 + sh.nsub * kATileBytes;
       const int bsub = b_sub_bytes(N, split);
-#pragma unroll
-      for (int u = 0; u < kSub; ++u) {
+      for (int u = 0; u < sh.nsub; ++u) {
         const uint32_t a = a0 + u * kATileBytes, b = b0 + u * bsub;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -450,7 +455,7 @@ KD_DEV void mma_epilogue(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigne
 
 template <class Plan>
 KD_DEV void mma_run(const Plan& plan, uint8_t* smem_raw, unsigned* err) {
-  MmaShared sh = carve_mma_smem(smem_raw, plan.max_n(), plan.split_b());
+  MmaShared sh = carve_mma_smem(smem_raw, plan.max_n(), plan.split_b(), plan.nsub);
   const int warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
     for (int i = 0; i < sh.nst; ++i) {

@@ -18,6 +18,19 @@ struct MmaMaps {
   CUtensorMap m[6];
 };
 
+// Largest token count among the active experts (every thread gets it).
+KD_DEV int max_tokens_per_expert(const int* cnt, const int* act, int n_act) {
+  __shared__ int s_max;
+  if (threadIdx.x < 32) {
+    int m = 0;
+    for (int a = threadIdx.x; a < n_act; a += 32) m = max(m, cnt[act[a]]);
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (threadIdx.x == 0) s_max = m;
+  }
+  __syncthreads();
+  return s_max;
+}
+
 KD_DEV void store_hilo(uint16_t* hi, uint16_t* lo, size_t o, float v) {
   const uint16_t h = f32_to_bf16_bits(v);
   hi[o] = h;
@@ -28,6 +41,7 @@ KD_DEV void store_hilo(uint16_t* hi, uint16_t* lo, size_t o, float v) {
 
 struct MmaProjPlan {
   const LayerDev* L; Acts a; const MmaMaps* maps;
+  int nsub;
   int tq, to, cq, co;   // tiles and K chunks per tile of QKV and o-proj
   KD_DEV int num_tiles() const { return tq + to; }
   KD_DEV long long tile_start(int t) const {
@@ -73,7 +87,8 @@ __global__ void __launch_bounds__(kMThreads, 1) mma_proj_kernel(LayerDev L, Acts
   extern __shared__ uint8_t smem[];
   MmaProjPlan p;
   p.L = &L; p.a = a; p.maps = &maps;
-  p.tq = L.Nqkv / 128; p.to = L.H / 128; p.cq = L.H / kKChunk; p.co = L.A / kKChunk;
+  p.nsub = mma_nsub(a.M, false);
+  p.tq = L.Nqkv / 128; p.to = L.H / 128; p.cq = L.H / (64 * p.nsub); p.co = L.A / (64 * p.nsub);
   pdl_wait();
   pdl_launch_dependents();
   mma_run(p, smem, L.err);
@@ -85,9 +100,10 @@ __global__ void __launch_bounds__(kMThreads, 1) mma_proj_kernel(LayerDev L, Acts
 // expert); shared: the shared expert's.  B = h1 as a bf16 hi/lo pair.
 struct MmaGateUpPlan {
   const LayerDev* L; int M; bool shared; const MmaMaps* maps; Route rt; int n_act;
+  int nsub, nmax;
   KD_DEV int tiles_per() const { return 2 * L->I / 128; }
   KD_DEV int num_tiles() const { return (shared ? 1 : n_act) * tiles_per(); }
-  KD_DEV long long tile_start(int t) const { return (long long)t * (L->H / kKChunk); }
+  KD_DEV long long tile_start(int t) const { return (long long)t * (L->H / (64 * nsub)); }
   KD_DEV MUnit tile_unit(int t) const {
     MUnit m{};
     const int a = t / tiles_per(), tt = t % tiles_per();
@@ -102,7 +118,7 @@ struct MmaGateUpPlan {
     return m;
   }
   KD_DEV const CUtensorMap* map(int id) const { return &maps->m[id]; }
-  KD_DEV int max_n() const { return M; }
+  KD_DEV int max_n() const { return nmax; }
   KD_DEV bool split_b() const { return true; }
   KD_DEV const uint16_t* b_row(const MUnit& m, int j, int h) const {
     const int t = shared ? j : rt.perm[m.tok0 + j] / L->k;
@@ -133,13 +149,16 @@ __global__ void __launch_bounds__(kMThreads, 1) mma_gateup_kernel(LayerDev L, in
   extern __shared__ uint8_t smem[];
   MmaGateUpPlan p;
   p.L = &L; p.M = M; p.shared = shared != 0; p.maps = &maps; p.n_act = 1;
+  p.nmax = M;
   if (!shared) {
     pdl_wait();
     pdl_launch_dependents();
     p.rt = carve_route(reinterpret_cast<int*>(smem + kMmaSmem), L.E, M * L.k);
     route_tokens(L, M, p.rt, blockIdx.x == 0);
     p.n_act = *p.rt.n_act;
+    p.nmax = max_tokens_per_expert(p.rt.cnt, p.rt.act, p.n_act);
   }
+  p.nsub = mma_nsub(p.nmax, true);
   mma_run(p, smem, L.err);
 }
 
@@ -151,9 +170,10 @@ __global__ void __launch_bounds__(kMThreads, 1) mma_gateup_kernel(LayerDev L, in
 // completing a block (every entry) writes that block of the layer output.
 struct MmaDownPlan {
   const LayerDev* L; int M; int n_act; const MmaMaps* maps; uint16_t* out;
+  int nsub, nmax;
   KD_DEV int tiles_per() const { return L->H / 128; }
   KD_DEV int num_tiles() const { return (n_act + L->S) * tiles_per(); }
-  KD_DEV long long tile_start(int t) const { return (long long)t * (L->I / kKChunk); }
+  KD_DEV long long tile_start(int t) const { return (long long)t * (L->I / (64 * nsub)); }
   KD_DEV MUnit tile_unit(int t) const {
     MUnit m{};
     const int a = t / tiles_per(), tt = t % tiles_per();
@@ -168,7 +188,7 @@ struct MmaDownPlan {
     return m;
   }
   KD_DEV const CUtensorMap* map(int id) const { return &maps->m[id]; }
-  KD_DEV int max_n() const { return M; }
+  KD_DEV int max_n() const { return nmax; }
   KD_DEV bool split_b() const { return true; }
   KD_DEV const uint16_t* b_row(const MUnit& m, int j, int h) const {
     if (m.tag < 0) return (h ? L->act_sh_lo : L->act_sh_hi) + (size_t)j * L->I;
@@ -227,6 +247,9 @@ __global__ void __launch_bounds__(kMThreads, 1) mma_down_kernel(LayerDev L, int 
   MmaDownPlan p;
   p.L = &L; p.M = M; p.out = out; p.maps = &maps;
   p.n_act = *(volatile int*)L.n_active;
+  p.nmax = max_tokens_per_expert(L.counts, L.active, p.n_act);
+  if (L.S && M > p.nmax) p.nmax = M;
+  p.nsub = mma_nsub(p.nmax, true);
   mma_run(p, smem, L.err);
 }
 
