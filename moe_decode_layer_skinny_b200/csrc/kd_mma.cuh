@@ -283,14 +283,20 @@ KD_DEV void cp_async16(void* dst, const void* src, uint32_t src_bytes) {
 KD_DEV void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 KD_DEV void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+// Arrive on `bar` once every cp.async this thread issued so far has landed
+// (the arrival counts against the barrier's expected count).
+KD_DEV void cp_async_arrive_noinc(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
 
 // Two warps (64 threads) write the B tile of every stage with cp.async:
 // token rows j < ntok (zero-filled up to N), 128 bytes (64 K) each, 16-byte
 // chunk c of row r at r*128 + ((c ^ (r & 7)) * 16) -- the 128-byte swizzle
-// the A tile has.  A stage is handed to the MMA (proxy fence + arrive) kLag
-// stages later, so that kLag stages of gathers are in flight per thread.
-constexpr int kBLag = 2;   // < the smallest ring (3 stages)
-
+// the A tile has.  Each thread's copies of a stage arrive on the stage's full
+// barrier when they land (no thread waits for them), so every stage of the
+// ring can have gathers in flight; the MMA issuer fences the generic-proxy
+// writes against the tensor core after its wait.
 template <class Plan>
 KD_DEV void mma_producer_b(const Plan& plan, MmaShared& sh, unsigned* err) {
   constexpr int kQ = 2 * kMaxN * 8 / 64;   // 16-byte copies per thread per stage (at most)
@@ -326,18 +332,11 @@ KD_DEV void mma_producer_b(const Plan& plan, MmaShared& sh, unsigned* err) {
         for (int i = 0; i < kQ; ++i)
           if (nb[i] != 0xFFFFFFFFu) cp_async16(bt + u * bsub + off[i], src[i] + k0, nb[i]);
       }
-      cp_async_commit();
-      if (it >= (uint32_t)kBLag) {
-        cp_async_wait<kBLag>();
-        fence_proxy_async_smem();   // generic-proxy writes -> visible to the tensor core
-        mbar_arrive(&sh.full[(it - kBLag) % sh.nst]);
-      }
+      cp_async_arrive_noinc(&sh.full[s]);
     }
   }
-  cp_async_wait<0>();
-  fence_proxy_async_smem();
-  for (uint32_t j = it > (uint32_t)kBLag ? it - kBLag : 0; j < it; ++j)
-    mbar_arrive(&sh.full[j % sh.nst]);
+  cp_async_commit();
+  cp_async_wait<0>();   // nothing in flight when the warp leaves
 }
 
 template <class Plan>
@@ -357,6 +356,7 @@ KD_DEV void mma_issuer(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigned*
       const int s = it % sh.nst;
       const uint32_t ph = (it / sh.nst) & 1u;
       mwait(&sh.full[s], ph, sh.abort_flag, err);
+      fence_proxy_async_smem();   // the B gathers (generic proxy) -> tensor core reads
       tc_fence_after();
       const uint32_t a0 = smem_u32(sh.stage + (size_t)s * sh.stage_bytes);
       const uint32_t b0 = a0 + sh.nsub * kATileBytes;
