@@ -170,8 +170,8 @@ int kd_layer_set_timing_events(kd_layer* layer, void* const* events, int n_event
  * of this entry point).  For callers that cannot call cudaMalloc from where
  * they run it -- e.g. a host runtime whose device memory all belongs to
  * another allocator, or a plugin that is handed only its input and output
- * buffers: the scratch this computation needs between its two kernels
- * (router logits and per-expert lists) lives in a file-scope __device__
+ * buffers: the scratch this computation needs between the blocks of its
+ * one launch (router logits, a block counter, the per-expert lists) lives in a file-scope __device__
  * array of fixed size in the library, held by every GPU that loads it until
  * the process exits, instead of a cudaMalloc'd workspace.
  *   router_w      device, [n_experts, hidden] bf16 (wdtype KD_WBF16) or e4m3
@@ -183,7 +183,8 @@ int kd_layer_set_timing_events(kd_layer* layer, void* const* events, int n_event
  *   idx_out       device int32 [M, top_k]: selected experts, descending logit,
  *                 ties -> lower id
  *   gates_out     device fp32 [M, top_k]: softmax renormalised over the top_k
- * Same arithmetic as the router of kd_decode_layer.  Limits: M <= 64
+ * Same arithmetic as the CUDA-core router of kd_decode_layer (the one it
+ * runs for FP8 layers and below the tensor-core token threshold).  Limits: M <= 64
  * (KD_STATIC_MAX_TOKENS), n_experts <= 1024 (KD_STATIC_MAX_EXPERTS),
  * top_k <= 16, hidden a multiple of 128 and <= 8192; larger sizes return
  * KD_ERANGE, bad pointers or shapes KD_EINVAL.  Calls no cudaMalloc /

@@ -83,12 +83,14 @@ struct LayerDev {
   int* counts; int* offsets; int* perm; int* active; int* n_active;
   float* act; float* act_sh;               // [Mmax*k, I] by position, [Mmax, I] (fp32)
   uint16_t* h1lo;                          // [Mmax, H] bf16(h1 - bf16(h1))   (tensor-core path)
+  uint16_t* h1lo2;                         // [Mmax, H] what h1b + h1lo leave of h1 (router)
   uint16_t* act_hi; uint16_t* act_lo;      // [Mmax*k, I] bf16 pair of act    (tensor-core path)
   uint16_t* act_sh_hi; uint16_t* act_sh_lo;// [Mmax, I]
   float* ws_main; float* ws_side;          // split-K partials, main / side stream launches
   unsigned* tcnt_main; unsigned* tcnt_side;// split-K tile arrivals (self-resetting)
   float* yr; float* ysh;                   // [Mmax*k, H] by token*k+slot, [Mmax, H]
   unsigned* hcnt;                          // [H/64] down rows done per block (self-resetting)
+  unsigned* rcnt;                          // router blocks done (self-resetting)
   unsigned* err;
 };
 
@@ -199,63 +201,6 @@ KD_DEV void router_chunk(const uint4 wv, float scale, const float* const* arow, 
   }
 }
 
-template <int WT>
-__global__ void __launch_bounds__(kRouterThreads) router_kernel(LayerDev L, int M) {
-  constexpr int EPC = WT == W_BF16 ? 8 : 16;
-  constexpr int kRouterWChunks = WT == W_BF16 ? 8 : 4;  // 16-byte chunks per lane, H <= 8192
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int rloc = warp >> 2, q = warp & 3;
-  const int row = blockIdx.x * kRouterRows + rloc;
-  const int cq = (L.H * L.eb / 16) / 4;   // chunks per quarter row
-  __shared__ float part[kRouterRows][4][64];
-  // the router weights are static: load them before waiting for h1
-  uint4 w[kRouterWChunks];
-  float sc[kRouterWChunks];
-  if (row < L.E) {
-    const uint8_t* wrow = L.wr + (size_t)row * L.H * L.eb;
-#pragma unroll
-    for (int i = 0; i < kRouterWChunks; ++i) {
-      const int c = lane + 32 * i;
-      if (c < cq) {
-        const int ci = q * cq + c;
-        w[i] = ld_nc_v4(wrow + (size_t)ci * 16);
-        sc[i] = WT == W_FP8 ? __ldg(L.sr + (size_t)(row >> 7) * L.nHb + ((ci * EPC) >> 7)) : 1.f;
-      }
-    }
-  }
-  pdl_wait();
-  pdl_launch_dependents();
-  if (row < L.E) {
-    for (int t0 = 0; t0 < M; t0 += kTT) {
-      const int nt = M - t0 < kTT ? M - t0 : kTT;
-      const float* arow[kTT];
-#pragma unroll
-      for (int t = 0; t < kTT; ++t) arow[t] = L.h1f + (size_t)(t0 + (t < nt ? t : 0)) * L.H;
-      float acc[kTT] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int i = 0; i < kRouterWChunks; ++i) {
-        const int c = lane + 32 * i;
-        if (c < cq) router_chunk<WT>(w[i], sc[i], arow, (q * cq + c) * EPC, nt, acc);
-      }
-#pragma unroll
-      for (int t = 0; t < kTT; ++t) {
-        float v = acc[t];
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-        if (lane == 0 && t < nt) part[rloc][q][t0 + t] = v;
-      }
-    }
-  }
-  __syncthreads();
-  for (int i = threadIdx.x; i < kRouterRows * M; i += kRouterThreads) {
-    const int r = i / M, t = i % M, e = blockIdx.x * kRouterRows + r;
-    if (e < L.E)
-      L.logits[(size_t)t * L.E + e] =
-          ((part[r][0][t] + part[r][1][t]) + (part[r][2][t] + part[r][3][t])) +
-          (L.bias ? L.bias[e] : 0.f);
-  }
-
-}
 
 // ------------------------------------------------------------------ selection + dispatch
 
@@ -286,51 +231,135 @@ KD_DEV Route carve_route(int* base, int E, int Mk) {
   return r;
 }
 
-// Top-k of every token (descending logit, ties -> lower expert id), the
-// softmax renormalised over the selection, and the per-expert token lists.
+// Selection keys: larger key = larger logit, ties -> lower expert id.  The
+// logit's bits are mapped to an unsigned order (sign flipped for positive
+// values, all bits for negative ones) and the expert id complemented below.
+KD_DEV uint64_t route_key(float v, int e) {
+  uint32_t u = __float_as_uint(v);
+  u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return ((uint64_t)u << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)e);
+}
+KD_DEV float key_value(uint64_t key) {
+  uint32_t u = (uint32_t)(key >> 32);
+  u = (u & 0x80000000u) ? (u & 0x7FFFFFFFu) : ~u;
+  return __uint_as_float(u);
+}
+KD_DEV int key_expert(uint64_t key) { return (int)(0xFFFFFFFFu - (uint32_t)key); }
+
+KD_DEV void cas_desc(uint64_t& x, uint64_t& y) {
+  const uint64_t hi = x > y ? x : y, lo = x > y ? y : x;
+  x = hi;
+  y = lo;
+}
+// bitonic sequence -> descending
+template <int N>
+KD_DEV void bitonic_merge_desc(uint64_t (&a)[N]) {
+#pragma unroll
+  for (int st = N / 2; st > 0; st >>= 1)
+#pragma unroll
+    for (int i = 0; i < N; ++i)
+      if (!(i & st)) cas_desc(a[i], a[i + st]);
+}
+// any sequence -> descending (bitonic sort)
+template <int N>
+KD_DEV void bitonic_sort_desc(uint64_t (&a)[N]) {
+#pragma unroll
+  for (int sz = 2; sz <= N; sz <<= 1)
+#pragma unroll
+    for (int st = sz / 2; st > 0; st >>= 1)
+#pragma unroll
+      for (int i = 0; i < N; ++i) {
+        const int l = i ^ st;
+        if (l > i) {
+          if ((i & sz) == 0 || sz == N) cas_desc(a[i], a[l]);
+          else cas_desc(a[l], a[i]);
+        }
+      }
+}
+// a, b descending -> a = the largest N of both, descending
+template <int N>
+KD_DEV void keep_top_desc(uint64_t (&a)[N], const uint64_t (&b)[N]) {
+#pragma unroll
+  for (int i = 0; i < N; ++i) a[i] = a[i] > b[N - 1 - i] ? a[i] : b[N - 1 - i];
+  bitonic_merge_desc(a);
+}
+
+// Top-k of token t by one warp: lane holds the logits of experts lane,
+// lane + 32, ... (PER of them, PER >= E / 32) and sorts their keys into a
+// descending list of LL >= k; five butterfly rounds (partner = lane ^ 1, ^ 2,
+// ..., ^ 16) each keep the largest LL of the two lists, after which every lane
+// holds the token's top LL.  Then the softmax renormalised over the first k.
+template <int PER, int LL>
+KD_DEV void topk_token(const LayerDev& L, const Route& R, int t, bool write_global) {
+  const int lane = threadIdx.x & 31;
+  const int k = L.k, E = L.E;
+  uint64_t a[LL];
+#pragma unroll
+  for (int g = 0; g < (PER + LL - 1) / LL; ++g) {
+    uint64_t b[LL];
+#pragma unroll
+    for (int i = 0; i < LL; ++i) {
+      const int qq = g * LL + i, e = lane + 32 * qq;
+      b[i] = (qq < PER && e < E) ? route_key(L.logits[(size_t)t * E + e], e) : 0ull;
+    }
+    bitonic_sort_desc(b);
+    if (g == 0) {
+#pragma unroll
+      for (int i = 0; i < LL; ++i) a[i] = b[i];
+    } else {
+      keep_top_desc(a, b);
+    }
+  }
+#pragma unroll 1
+  for (int o = 1; o < 32; o <<= 1) {
+    uint64_t b[LL];
+#pragma unroll
+    for (int i = 0; i < LL; ++i) b[i] = __shfl_xor_sync(0xffffffffu, a[i], o);
+    keep_top_desc(a, b);
+  }
+  const float top = key_value(a[0]);
+  float den = 0.f, mysel = 0.f;
+  int mye = 0;
+#pragma unroll
+  for (int i = 0; i < LL; ++i) {
+    if (i < k) {
+      const float v = key_value(a[i]);
+      den += expf(v - top);
+      if (i == lane) {
+        mysel = v;
+        mye = key_expert(a[i]);
+      }
+    }
+  }
+  if (lane < k) {
+    R.sel[t * k + lane] = mye;
+    if (write_global) {
+      L.idx[t * k + lane] = mye;
+      L.gates[t * k + lane] = expf(mysel - top) / den;
+    }
+  }
+}
+
+template <int PER>
+KD_DEV void topk_token_k(const LayerDev& L, const Route& R, int t, bool write_global) {
+  if (L.k <= 8) topk_token<PER, 8>(L, R, t, write_global);
+  else topk_token<PER, 16>(L, R, t, write_global);
+}
+
+// Top-k of every token, the renormalised softmax over each selection, and the
+// per-expert token lists.
 KD_DEV void route_tokens(const LayerDev& L, int M, const Route& R, bool write_global) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nw = blockDim.x >> 5;
   const int k = L.k, E = L.E;
-  // top-k: one warp per token; lane holds logits lane, lane+32, ...
+  const int per = (E + 31) / 32;   // E <= 1024
   for (int t = warp; t < M; t += nw) {
-    float lv[32];
-    const int per = (E + 31) / 32;
-#pragma unroll
-    for (int qq = 0; qq < 32; ++qq) {
-      const int e = lane + 32 * qq;
-      lv[qq] = (qq < per && e < E) ? L.logits[(size_t)t * E + e] : -INFINITY;
-    }
-    unsigned taken = 0u;
-    float top = 0.f, den = 0.f, mysel = 0.f;
-    for (int j = 0; j < k; ++j) {
-      float bv = -INFINITY;
-      int be = 0x7fffffff;
-#pragma unroll
-      for (int qq = 0; qq < 32; ++qq) {
-        const int e = lane + 32 * qq;
-        if (qq < per && e < E && !((taken >> qq) & 1u) && (lv[qq] > bv || (lv[qq] == bv && e < be))) {
-          bv = lv[qq];
-          be = e;
-        }
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-        if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
-      }
-      if ((be & 31) == lane) taken |= 1u << (be >> 5);
-      if (j == 0) top = bv;
-      if (j == lane) mysel = bv;
-      den += expf(bv - top);
-      if (lane == 0) R.sel[t * k + j] = be;
-    }
-    __syncwarp();
-    if (write_global && lane < k) {
-      L.idx[t * k + lane] = R.sel[t * k + lane];
-      L.gates[t * k + lane] = expf(mysel - top) / den;
-    }
+    if (per <= 1) topk_token_k<1>(L, R, t, write_global);
+    else if (per <= 2) topk_token_k<2>(L, R, t, write_global);
+    else if (per <= 4) topk_token_k<4>(L, R, t, write_global);
+    else if (per <= 8) topk_token_k<8>(L, R, t, write_global);
+    else if (per <= 16) topk_token_k<16>(L, R, t, write_global);
+    else topk_token_k<32>(L, R, t, write_global);
   }
   for (int e = threadIdx.x; e < E; e += blockDim.x) R.cnt[e] = 0;
   __syncthreads();
@@ -409,6 +438,98 @@ KD_DEV void route_tokens(const LayerDev& L, int M, const Route& R, bool write_gl
   // restore the exclusive offsets (the walk advanced them to the ends)
   for (int e = threadIdx.x; e < E; e += blockDim.x) R.off[e] -= R.cnt[e];
   __syncthreads();
+}
+
+// Logits done by this block: the block that finishes last (of `nblocks`)
+// selects every token's experts and builds the per-expert token lists in
+// global memory (route scratch in dynamic shared memory).  All threads call.
+KD_DEV void route_last_block(const LayerDev& L, int M, unsigned nblocks) {
+  extern __shared__ int route_smem[];
+  __shared__ int s_last;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const unsigned prev = atomicAdd(L.rcnt, 1u);
+    s_last = prev == nblocks - 1;
+    if (s_last) *L.rcnt = 0u;   // every block is in: ready for the next call
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  const Route R = carve_route(route_smem, L.E, M * L.k);
+  route_tokens(L, M, R, true);
+}
+
+// The routing of the call, as the router left it in global memory, copied
+// into shared memory (all threads call).
+KD_DEV void load_route(const LayerDev& L, int M, const Route& R) {
+  const int E = L.E, Mk = M * L.k;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    R.cnt[e] = L.counts[e];
+    R.off[e] = L.offsets[e];
+    R.act[e] = L.active[e];
+  }
+  for (int c = threadIdx.x; c < Mk; c += blockDim.x) R.perm[c] = L.perm[c];
+  if (threadIdx.x == 0) *R.n_act = *L.n_active;
+  __syncthreads();
+}
+
+template <int WT>
+__global__ void __launch_bounds__(kRouterThreads) router_kernel(LayerDev L, int M) {
+  constexpr int EPC = WT == W_BF16 ? 8 : 16;
+  constexpr int kRouterWChunks = WT == W_BF16 ? 8 : 4;  // 16-byte chunks per lane, H <= 8192
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rloc = warp >> 2, q = warp & 3;
+  const int row = blockIdx.x * kRouterRows + rloc;
+  const int cq = (L.H * L.eb / 16) / 4;   // chunks per quarter row
+  __shared__ float part[kRouterRows][4][64];
+  // the router weights are static: load them before waiting for h1
+  uint4 w[kRouterWChunks];
+  float sc[kRouterWChunks];
+  if (row < L.E) {
+    const uint8_t* wrow = L.wr + (size_t)row * L.H * L.eb;
+#pragma unroll
+    for (int i = 0; i < kRouterWChunks; ++i) {
+      const int c = lane + 32 * i;
+      if (c < cq) {
+        const int ci = q * cq + c;
+        w[i] = ld_nc_v4(wrow + (size_t)ci * 16);
+        sc[i] = WT == W_FP8 ? __ldg(L.sr + (size_t)(row >> 7) * L.nHb + ((ci * EPC) >> 7)) : 1.f;
+      }
+    }
+  }
+  pdl_wait();
+  if (row < L.E) {
+    for (int t0 = 0; t0 < M; t0 += kTT) {
+      const int nt = M - t0 < kTT ? M - t0 : kTT;
+      const float* arow[kTT];
+#pragma unroll
+      for (int t = 0; t < kTT; ++t) arow[t] = L.h1f + (size_t)(t0 + (t < nt ? t : 0)) * L.H;
+      float acc[kTT] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int i = 0; i < kRouterWChunks; ++i) {
+        const int c = lane + 32 * i;
+        if (c < cq) router_chunk<WT>(w[i], sc[i], arow, (q * cq + c) * EPC, nt, acc);
+      }
+#pragma unroll
+      for (int t = 0; t < kTT; ++t) {
+        float v = acc[t];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == 0 && t < nt) part[rloc][q][t0 + t] = v;
+      }
+    }
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < kRouterRows * M; i += kRouterThreads) {
+    const int r = i / M, t = i % M, e = blockIdx.x * kRouterRows + r;
+    if (e < L.E)
+      L.logits[(size_t)t * L.E + e] =
+          ((part[r][0][t] + part[r][1][t]) + (part[r][2][t] + part[r][3][t])) +
+          (L.bias ? L.bias[e] : 0.f);
+  }
+  route_last_block(L, M, gridDim.x);
+  pdl_launch_dependents();
 }
 
 // ------------------------------------------------------------------ experts
@@ -570,7 +691,7 @@ __global__ void __launch_bounds__(kThreads, 1) gateup_kernel(LayerDev L, int M, 
     pdl_wait();
     pdl_launch_dependents();
     p.rt = carve_route(reinterpret_cast<int*>(smem + kStreamSmem), L.E, M * L.k);
-    route_tokens(L, M, p.rt, blockIdx.x == 0);
+    load_route(L, M, p.rt);
     n_act = *p.rt.n_act;
   }
   p.R = expert_range(n_act, L.I);

@@ -167,10 +167,14 @@ static int configure_kernels() {
   KD_CUDA(cudaFuncSetAttribute(gateup_kernel<W_FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   KD_CUDA(cudaFuncSetAttribute(down_kernel<W_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   KD_CUDA(cudaFuncSetAttribute(down_kernel<W_FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  const int rsmem = (int)(sizeof(int) * kRouteSmemInts(1024, 64 * 16));
+  KD_CUDA(cudaFuncSetAttribute(router_kernel<W_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, rsmem));
+  KD_CUDA(cudaFuncSetAttribute(router_kernel<W_FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, rsmem));
   const int msmem = (int)(kMmaSmem + 16 + sizeof(int) * kRouteSmemInts(1024, 64 * 16));
   KD_CUDA(cudaFuncSetAttribute(mma_proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem));
   KD_CUDA(cudaFuncSetAttribute(mma_gateup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem));
   KD_CUDA(cudaFuncSetAttribute(mma_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem));
+  KD_CUDA(cudaFuncSetAttribute(mma_router_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem));
   stream_kernels_configured = true;
   return KD_OK;
 }
@@ -289,7 +293,9 @@ extern "C" int kd_layer_create(const kd_config* cfg, uint64_t seed, kd_layer** o
   TRY(dalloc_t(L, (size_t)M * k * H, &d.yr));
   TRY(dalloc_t(L, (size_t)M * H, &d.ysh));
   TRY(dalloc_t(L, (size_t)H / 64, &d.hcnt));
+  TRY(dalloc_t(L, 1, &d.rcnt));
   TRY(dalloc_t(L, (size_t)M * H, &d.h1lo));
+  TRY(dalloc_t(L, (size_t)M * H, &d.h1lo2));
   TRY(dalloc_t(L, (size_t)M * k * I, &d.act_hi));
   TRY(dalloc_t(L, (size_t)M * k * I, &d.act_lo));
   TRY(dalloc_t(L, (size_t)M * I, &d.act_sh_hi));
@@ -297,7 +303,7 @@ extern "C" int kd_layer_create(const kd_config* cfg, uint64_t seed, kd_layer** o
   TRY(dalloc_t(L, (size_t)L->nsm * kWsFloatsPerCta, &d.ws_main));
   TRY(dalloc_t(L, (size_t)L->nsm * kWsFloatsPerCta, &d.ws_side));
   {
-    const size_t ntile = std::max<size_t>({(size_t)(E + 1) * (H / 128), (size_t)E * (2 * I / 128),
+    const size_t ntile = std::max<size_t>({(size_t)(E + 1) * (H / 128), (size_t)(E + 1) * (2 * I / 128),
                                            (size_t)(Nqkv + H) / 128});
     TRY(dalloc_t(L, ntile, &d.tcnt_main));
     TRY(dalloc_t(L, ntile, &d.tcnt_side));
@@ -305,6 +311,7 @@ extern "C" int kd_layer_create(const kd_config* cfg, uint64_t seed, kd_layer** o
     TRYC(cudaMemset(d.tcnt_side, 0, sizeof(unsigned) * ntile));
   }
   TRYC(cudaMemset(d.hcnt, 0, sizeof(unsigned) * (H / 64)));
+  TRYC(cudaMemset(d.rcnt, 0, sizeof(unsigned)));
   TRY(dalloc_t(L, 1, &d.err));
   TRYC(cudaMemset(d.err, 0, sizeof(unsigned)));
   TRYC(cudaMemset(d.n_active, 0, sizeof(int)));
@@ -336,7 +343,8 @@ extern "C" int kd_layer_create(const kd_config* cfg, uint64_t seed, kd_layer** o
   if (!fp8) {
     bool ok = encode_bf16_map(&L->maps.m[0], wqkv, Nqkv, H) && encode_bf16_map(&L->maps.m[1], wo, H, A) &&
               encode_bf16_map(&L->maps.m[2], wgu, (uint64_t)E * 2 * I, H) &&
-              encode_bf16_map(&L->maps.m[3], wd, (uint64_t)E * H, I);
+              encode_bf16_map(&L->maps.m[3], wd, (uint64_t)E * H, I) &&
+              encode_bf16_map(&L->maps.m[6], wr, E, H);
     if (ok && c.n_shared)
       ok = encode_bf16_map(&L->maps.m[4], wgu_sh, 2 * I, H) && encode_bf16_map(&L->maps.m[5], wd_sh, H, I);
     L->has_maps = ok;
@@ -409,17 +417,28 @@ static int launch_layer(kd_layer* L, void* hidden, const void* attn, int M, cuda
   const size_t msm = kMmaSmem;
   const size_t mroute = kMmaSmem + 16 + sizeof(int) * kRouteSmemInts(d.E, M * d.k);
   if (L->timing) KD_CUDA(cudaEventRecord(L->tev[0], s));
+  // Main stream: projections -> router (logits, selection, token lists in one
+  // launch) -> routed gate/up -> down + combine.  Side stream: the shared
+  // expert's gate/up, from the end of the projections, joined by an event
+  // before the down kernel.  The router releases its dependent launch only
+  // when it is done, so the shared gate/up gets the SMs that the router
+  // leaves free while the router runs.
+  const size_t route_ints = sizeof(int) * kRouteSmemInts(d.E, M * d.k);
   if (mma)
     KD_CUDA(launch(mma_proj_kernel, G, kMThreads, msm, s, pdl_first, d, a, L->maps));
   else
     KD_CUDA(launch(fp8 ? proj_kernel<W_FP8> : proj_kernel<W_BF16>, G, kThreads, sm, s, pdl_first, d, a));
   if (L->timing) KD_CUDA(cudaEventRecord(L->tev[1], s));
   if (d.S) KD_CUDA(cudaEventRecord(L->ev_h1, s));
-  // the router goes first so that its CTAs get SMs before the shared
-  // expert's gate/up (on the side stream) fills them
-  const int rgrid = (d.E + kRouterRows - 1) / kRouterRows;
-  KD_CUDA(launch(fp8 ? router_kernel<W_FP8> : router_kernel<W_BF16>, rgrid, kRouterThreads, 0, s,
-                 !L->timing, d, M));
+  if (mma) {
+    const int rchunks = ((d.E + 127) / 128) * (d.H / (64 * mma_nsub(M, 3)));
+    const int rgrid = std::max(1, std::min(G, rchunks / kRouterChunksPerCta));
+    KD_CUDA(launch(mma_router_kernel, rgrid, kMThreads, mroute, s, !L->timing, d, M, L->maps));
+  } else {
+    const int rgrid = (d.E + kRouterRows - 1) / kRouterRows;
+    KD_CUDA(launch(fp8 ? router_kernel<W_FP8> : router_kernel<W_BF16>, rgrid, kRouterThreads,
+                   route_ints, s, !L->timing, d, M));
+  }
   if (d.S) {
     KD_CUDA(cudaStreamWaitEvent(L->side, L->ev_h1, 0));
     if (mma)
@@ -445,11 +464,12 @@ static int launch_layer(kd_layer* L, void* hidden, const void* attn, int M, cuda
     if (rc != KD_OK) return rc;
     KD_CUDA(cudaEventRecord(ev_join, pf));
   }
+  const bool pdl_down = !L->timing && !d.S && !(next && pf);
   if (mma)
-    KD_CUDA(launch(mma_down_kernel, G, kMThreads, msm, s, !L->timing && !d.S, d, M, a.out, L->maps));
+    KD_CUDA(launch(mma_down_kernel, G, kMThreads, msm, s, pdl_down, d, M, a.out, L->maps));
   else
-    KD_CUDA(launch(fp8 ? down_kernel<W_FP8> : down_kernel<W_BF16>, G, kThreads, sm, s,
-                   !L->timing && !d.S, d, M, a.out));
+    KD_CUDA(launch(fp8 ? down_kernel<W_FP8> : down_kernel<W_BF16>, G, kThreads, sm, s, pdl_down, d,
+                   M, a.out));
   if (L->timing) KD_CUDA(cudaEventRecord(L->tev[4], s));
   if (next && pf) KD_CUDA(cudaStreamWaitEvent(s, ev_join, 0));
   return KD_OK;
@@ -464,6 +484,7 @@ extern "C" int kd_layer_check(kd_layer* L) {
   KD_CUDA(cudaMemset(L->d.err, 0, sizeof(unsigned)));
   // an aborted call may have left arrival counters part-way
   KD_CUDA(cudaMemset(L->d.hcnt, 0, sizeof(unsigned) * (L->d.H / 64)));
+  KD_CUDA(cudaMemset(L->d.rcnt, 0, sizeof(unsigned)));
   if (e & (ERR_WAIT_FULL | ERR_WAIT_EMPTY | ERR_WAIT_MMA))
     return fail(KD_ETIMEOUT, "device: a bounded wait gave up (flags %s0x%lx)", "", (long)e);
   return fail(KD_EDEVICE, "device error flags %s0x%lx", "", (long)e);

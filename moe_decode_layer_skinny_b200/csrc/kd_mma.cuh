@@ -12,9 +12,11 @@
 //               into the stage in the same swizzled K-major layout
 //   warps 4-7   epilogue: tcgen05.ld of the accumulator (lane = weight row),
 //               then the plan's epilogue, or a split-K partial
-// Activations that must stay fp32-accurate (h1, the SwiGLU activations) come
-// as a bf16 pair hi + lo (hi = bf16(v), lo = bf16(v - hi)); both are
-// multiplied into the same accumulator, which keeps ~16 significant bits.
+// Activations that must stay fp32-accurate come as a sum of bf16 terms, all
+// multiplied into the same accumulator: the expert inputs (h1, the SwiGLU
+// activations) as hi + lo (hi = bf16(v), lo = bf16(v - hi): ~16 significant
+// bits); the router's h1 as hi + mid + lo (all 24 bits of the fp32 value; the
+// products with bf16 weights are exact in the fp32 accumulator).
 // Work units are (weight tile, K part); a tile split over several parts is
 // summed in part order by the unit that completes it (deterministic).
 #pragma once
@@ -100,6 +102,7 @@ constexpr int kATileBytes = 128 * 128;                // 128 rows x 64 bf16 (one
 constexpr int kMaxSub = 2;                            // 64-K sub-tiles per stage (at most)
 constexpr int kMRingBytes = 3 * kMaxSub * (kATileBytes + 64 * 128 * 2);  // 192 KB of stages
 constexpr int kMaxN = 64;                             // tokens per MMA (N)
+constexpr int kMaxTerms = 3;                          // bf16 terms of an activation
 constexpr size_t kWsFloatsPerCta = 2 * 128 * 64;     // split-K partial slots of one CTA
 constexpr size_t kMmaSmem = (size_t)kMRingBytes + 1024 /*align*/ + 1024 /*barriers, lists*/;
 
@@ -115,7 +118,7 @@ struct MUnit {
   int lrow;       // first row of the tile in its logical output (epilogue index)
 };
 
-KD_DEV int pad16(int n) { return (n + 15) & ~15; }
+__host__ __device__ inline int pad16(int n) { return (n + 15) & ~15; }
 
 // Stream-K partition of a launch: the K chunks of all tiles, concatenated in
 // tile order, are cut into min(gridDim.x, chunks) equal ranges; CTA b takes
@@ -185,25 +188,25 @@ struct MmaShared {
   uint64_t* accempty;    // [2] epilogue done reading the accumulator
   uint32_t* tmem_base;
   int* abort_flag;
-  int* misc;             // [8] epilogue scratch (combine block list length ...)
+  int* misc;             // [8] epilogue scratch ([1] combine block count, [2] after-run flag)
   int* blist;            // [128] combine block list
 };
 
 // The ring holds as many stages as fit.  A stage covers nsub x 64 K: nsub
 // weight sub-tiles [128 rows x 64 K] (16 KB each; with nsub = 2 every row
 // contributes 256 contiguous bytes per stage), then nsub B sub-tiles for the
-// launch's largest token count (hi + lo when split).  nsub is 2 when that
+// launch's largest token count (one per bf16 term of the activations).  nsub is 2 when that
 // still leaves at least 4 stages, else 1.
-KD_DEV int b_sub_bytes(int n, bool split) { return pad16(n) * 128 * (split ? 2 : 1); }
+__host__ __device__ inline int b_sub_bytes(int n, int terms) { return pad16(n) * 128 * terms; }
 
-KD_DEV int mma_nsub(int nmax, bool split) {
-  return kMRingBytes / (2 * (kATileBytes + b_sub_bytes(nmax, split))) >= 4 ? 2 : 1;
+__host__ __device__ inline int mma_nsub(int nmax, int terms) {
+  return kMRingBytes / (2 * (kATileBytes + b_sub_bytes(nmax, terms))) >= 4 ? 2 : 1;
 }
 
-KD_DEV MmaShared carve_mma_smem(uint8_t* raw, int nmax, bool split, int nsub) {
+KD_DEV MmaShared carve_mma_smem(uint8_t* raw, int nmax, int terms, int nsub) {
   MmaShared s;
   s.nsub = nsub;
-  s.stage_bytes = nsub * (kATileBytes + b_sub_bytes(nmax, split));
+  s.stage_bytes = nsub * (kATileBytes + b_sub_bytes(nmax, terms));
   s.nst = kMRingBytes / s.stage_bytes;
   if (s.nst > kMaxMStages) s.nst = kMaxMStages;
   uintptr_t p = (reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023);
@@ -246,16 +249,18 @@ KD_DEV bool mwait_lazy(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
 
 // Plan interface (all methods KD_DEV const):
 //   int num_tiles(); long long tile_start(int t); MUnit tile_unit(int t)   (see CtaUnits;
-//   a chunk is 64 * nsub K elements, nsub = mma_nsub(max_n(), split_b()))
+//   a chunk is 64 * nsub K elements, nsub = mma_nsub(max_n(), kTerms))
 //   int max_n(); int nsub
 //   const CUtensorMap* map(int id)
-//   bool split_b()                 B is a hi/lo pair
-//   const uint16_t* b_row(const MUnit&, int j, int hilo)   token j's bf16 row
+//   static constexpr int kTerms    bf16 terms of B (1; 2 = hi + lo; 3 = hi + mid + lo)
+//   const uint16_t* b_base(const MUnit&, int h); int b_stride(const MUnit&);
+//   int b_rowidx(const MUnit&, int j)   token j's row of term h: base + rowidx * stride
 //   bool paired()                  rows are (gate, up) pairs
 //   void epilogue(const MUnit&, int row_in_tile, int j, float v)
 //   void epilogue2(const MUnit&, int pair_in_tile, int j, float g, float u)
 //   float* ws(); unsigned* tile_cnt()            split-K partials / arrivals
 //   bool wants_unit_done(); void unit_done(const MUnit&, MmaShared&)   epilogue warps only
+//   void after_run(MmaShared&, uint8_t* smem)   all threads, after the pipeline
 
 template <class Plan>
 KD_DEV void mma_producer_a(const Plan& plan, MmaShared& sh, unsigned* err) {
@@ -293,44 +298,55 @@ KD_DEV void cp_async_arrive_noinc(uint64_t* bar) {
 // Two warps (64 threads) write the B tile of every stage with cp.async:
 // token rows j < ntok (zero-filled up to N), 128 bytes (64 K) each, 16-byte
 // chunk c of row r at r*128 + ((c ^ (r & 7)) * 16) -- the 128-byte swizzle
-// the A tile has.  Each thread's copies of a stage arrive on the stage's full
-// barrier when they land (no thread waits for them), so every stage of the
-// ring can have gathers in flight; the MMA issuer fences the generic-proxy
-// writes against the tensor core after its wait.
+// the A tile has.  Thread t copies chunk t % 8 of rows t / 8, t / 8 + 8, ...
+// (so every row it copies has the same swizzle), for every bf16 term.  Each
+// thread's copies of a stage arrive on the stage's full barrier when they
+// land (no thread waits for them), so every stage of the ring can have
+// gathers in flight; the MMA issuer fences the generic-proxy writes against
+// the tensor core after its wait.
 template <class Plan>
 KD_DEV void mma_producer_b(const Plan& plan, MmaShared& sh, unsigned* err) {
-  constexpr int kQ = 2 * kMaxN * 8 / 64;   // 16-byte copies per thread per stage (at most)
-  const int t = threadIdx.x - 64;          // 0..63
-  const int nh = plan.split_b() ? 2 : 1;
+  constexpr int nh = Plan::kTerms;
+  constexpr int kRows = kMaxN / 8;          // rows per thread (at most)
+  const int t = threadIdx.x - 64;           // 0..63
+  const int ch = t & 7, rg = t >> 3;
+  const uint32_t swz = (uint32_t)((ch ^ rg) * 16);
   uint32_t it = 0;
   CtaUnits<Plan> units(plan);
   MUnit m;
   while (units.next(m)) {
     const int N = pad16(m.ntok);
-    // this thread's copies for the whole unit: source row (+ chunk), smem
-    // offset within the B tile, and byte count (0 = zero fill)
-    const uint16_t* src[kQ];
-    uint32_t off[kQ], nb[kQ];
+    const int nr = N >> 3;
+    const size_t stride = (size_t)plan.b_stride(m);
+    // this thread's sources for the whole unit (byte count 0 = zero fill,
+    // ~0 = no row)
+    const uint16_t* src[nh][kRows];
+    uint32_t nb[kRows];
 #pragma unroll
-    for (int i = 0; i < kQ; ++i) {
-      const int q = t + 64 * i;
-      const int h = q / (N * 8), r = (q / 8) % N, ch = q % 8;
-      const bool live = q < nh * N * 8 && r < m.ntok;
-      src[i] = plan.b_row(m, live ? r : 0, q < nh * N * 8 ? h : 0) + ch * 8;
-      off[i] = (uint32_t)(h * N * 128 + r * 128 + ((ch ^ (r & 7)) * 16));
-      nb[i] = q < nh * N * 8 ? (live ? 16u : 0u) : 0xFFFFFFFFu;   // ~0: no copy
+    for (int i = 0; i < kRows; ++i) {
+      const int r = rg + 8 * i;
+      const bool live = i < nr && r < m.ntok;
+      const size_t ro = live ? (size_t)plan.b_rowidx(m, r) * stride : 0;
+#pragma unroll
+      for (int h = 0; h < nh; ++h) src[h][i] = plan.b_base(m, h) + ro + ch * 8;
+      nb[i] = i < nr ? (live ? 16u : 0u) : 0xFFFFFFFFu;
     }
+    const int bsub = b_sub_bytes(N, nh);
     for (int c = 0; c < m.nkc; ++c, ++it) {
       const int s = it % sh.nst;
       const uint32_t ph = (it / sh.nst) & 1u;
       mwait(&sh.empty[s], ph ^ 1u, sh.abort_flag, err);
-      uint8_t* bt = sh.stage + (size_t)s * sh.stage_bytes + sh.nsub * kATileBytes;
-      const int bsub = b_sub_bytes(N, nh == 2);
+      uint8_t* bt = sh.stage + (size_t)s * sh.stage_bytes + sh.nsub * kATileBytes + swz;
       for (int u = 0; u < sh.nsub; ++u) {
         const int k0 = ((m.kc0 + c) * sh.nsub + u) * 64;
 #pragma unroll
-        for (int i = 0; i < kQ; ++i)
-          if (nb[i] != 0xFFFFFFFFu) cp_async16(bt + u * bsub + off[i], src[i] + k0, nb[i]);
+        for (int i = 0; i < kRows; ++i) {
+          if (nb[i] != 0xFFFFFFFFu) {
+#pragma unroll
+            for (int h = 0; h < nh; ++h)
+              cp_async16(bt + u * bsub + h * N * 128 + (rg + 8 * i) * 128, src[h][i] + k0, nb[i]);
+          }
+        }
       }
       cp_async_arrive_noinc(&sh.full[s]);
     }
@@ -341,7 +357,7 @@ KD_DEV void mma_producer_b(const Plan& plan, MmaShared& sh, unsigned* err) {
 
 template <class Plan>
 KD_DEV void mma_issuer(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigned* err) {
-  const bool split = plan.split_b();
+  constexpr int nterms = Plan::kTerms;
   uint32_t it = 0, nu_local = 0;
   CtaUnits<Plan> units(plan);
   MUnit m;
@@ -360,14 +376,16 @@ KD_DEV void mma_issuer(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigned*
       tc_fence_after();
       const uint32_t a0 = smem_u32(sh.stage + (size_t)s * sh.stage_bytes);
       const uint32_t b0 = a0 + sh.nsub * kATileBytes;
-      const int bsub = b_sub_bytes(N, split);
+      const int bsub = b_sub_bytes(N, nterms);
       for (int u = 0; u < sh.nsub; ++u) {
         const uint32_t a = a0 + u * kATileBytes, b = b0 + u * bsub;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const uint64_t ad = sw128_desc(a + k * 32);
           mma_bf16(d, ad, sw128_desc(b + k * 32), idesc, c > 0 || u > 0 || k > 0);
-          if (split) mma_bf16(d, ad, sw128_desc(b + N * 128 + k * 32), idesc, true);
+#pragma unroll
+          for (int h = 1; h < nterms; ++h)
+            mma_bf16(d, ad, sw128_desc(b + h * N * 128 + k * 32), idesc, true);
         }
       }
       mma_commit(&sh.empty[s]);   // the stage is free once these MMAs are done
@@ -376,13 +394,31 @@ KD_DEV void mma_issuer(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigned*
   }
 }
 
-// Epilogue warps (4..7).  Thread = accumulator lane = row of the tile.
+// The plan's epilogue for 16 accumulator columns (tokens c .. c+15) of this
+// thread's row.
+template <class Plan>
+KD_DEV void emit16(const Plan& plan, const MUnit& m, int row, int lane, int c, const float* v) {
+  if (plan.paired()) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const float other = __shfl_xor_sync(0xffffffffu, v[j], 1);
+      if (!(lane & 1) && c + j < m.ntok) plan.epilogue2(m, row >> 1, c + j, v[j], other);
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      if (c + j < m.ntok) plan.epilogue(m, row, c + j, v[j]);
+  }
+}
+
+// Epilogue warps (4..7).  Thread = accumulator lane = row of the tile.  The
+// accumulator is read 16 columns at a time (a rolled loop: this code runs a
+// few times per unit, so it is kept small for the instruction cache).
 template <class Plan>
 KD_DEV void mma_epilogue(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigned* err) {
   const int ew = (threadIdx.x >> 5) - 4, lane = threadIdx.x & 31;
   const int row = ew * 32 + lane;
   uint32_t nu_local = 0;
-  float v[kMaxN];
   CtaUnits<Plan> units(plan);
   MUnit m;
   for (; units.next(m); ++nu_local) {
@@ -391,22 +427,23 @@ KD_DEV void mma_epilogue(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigne
     mwait_lazy(&sh.accfull[buf], (nu_local >> 1) & 1u, sh.abort_flag, err);
     tc_fence_after();
     const uint32_t ta = tmem + ((uint32_t)(ew * 32) << 16) + (uint32_t)(buf * kMaxN);
-#pragma unroll
-    for (int c = 0; c < kMaxN / 16; ++c)
-      if (c * 16 < N) tmem_ld16(ta + c * 16, v + c * 16);
-    tmem_wait_ld();
-    tc_fence_before();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&sh.accempty[buf]);
     bool complete = true;
+    int first = 0;
     if (m.nparts > 1) {
-      // split-K: park this part, the last part to arrive sums them in order
+      // split-K: park this part, the last part to arrive sums them in order.
+      // A slot is [token][row], so that a warp's 32 rows are one 128-byte line.
       const int slot = m.part == 0 ? 1 : 0;
       float* ws = plan.ws() + (size_t)blockIdx.x * kWsFloatsPerCta +
-                  ((size_t)slot * 128 + row) * kMaxN;
+                  (size_t)slot * 128 * kMaxN + row;
+#pragma unroll 1
+      for (int c = 0; c < N; c += 16) {
+        float v[16];
+        tmem_ld16(ta + c, v);
+        tmem_wait_ld();
 #pragma unroll
-      for (int j = 0; j < kMaxN; ++j)
-        if (j < m.ntok) ws[j] = v[j];
+        for (int j = 0; j < 16; ++j)
+          if (c + j < m.ntok) __stcg(ws + (c + j) * 128, v[j]);
+      }
       __threadfence();
       named_bar_sync(2, 128);
       if (threadIdx.x == 128) {
@@ -417,45 +454,55 @@ KD_DEV void mma_epilogue(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigne
       }
       named_bar_sync(2, 128);
       complete = sh.misc[0] != 0;
-      if (complete) {
-        __threadfence();
-#pragma unroll
-        for (int j = 0; j < kMaxN; ++j) v[j] = 0.f;
-        const int first = (int)blockIdx.x - m.part;
-        for (int p = 0; p < m.nparts; ++p) {
-          const float* src = plan.ws() + (size_t)(first + p) * kWsFloatsPerCta +
-                             ((size_t)(p == 0 ? 1 : 0) * 128 + row) * kMaxN;
-#pragma unroll
-          for (int j = 0; j < kMaxN; ++j)
-            if (j < m.ntok) v[j] += __ldcg(src + j);
-        }
-      }
+      first = (int)blockIdx.x - m.part;
+      if (complete) __threadfence();
     }
     if (complete) {
-      if (plan.paired()) {
+#pragma unroll 1
+      for (int c = 0; c < N; c += 16) {
+        float v[16];
+        if (m.nparts > 1) {
 #pragma unroll
-        for (int j = 0; j < kMaxN; ++j) {
-          if (j < N) {
-            const float other = __shfl_xor_sync(0xffffffffu, v[j], 1);
-            if (!(lane & 1) && j < m.ntok) plan.epilogue2(m, row >> 1, j, v[j], other);
+          for (int j = 0; j < 16; ++j) v[j] = 0.f;
+          // parts added in part order; four parts' loads in flight at a time
+#pragma unroll 1
+          for (int p = 0; p < m.nparts; p += 4) {
+            float t[4][16];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const float* src = plan.ws() + (size_t)(first + p + q) * kWsFloatsPerCta +
+                                 (size_t)(p + q == 0 ? 1 : 0) * 128 * kMaxN + row + c * 128;
+#pragma unroll
+              for (int j = 0; j < 16; ++j)
+                t[q][j] = (p + q < m.nparts && c + j < m.ntok) ? __ldcg(src + j * 128) : 0.f;
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              if (p + q < m.nparts) {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) v[j] += t[q][j];
+              }
           }
+        } else {
+          tmem_ld16(ta + c, v);
+          tmem_wait_ld();
         }
-      } else {
-#pragma unroll
-        for (int j = 0; j < kMaxN; ++j)
-          if (j < m.ntok) plan.epilogue(m, row, j, v[j]);
+        emit16(plan, m, row, lane, c, v);
       }
-      if (plan.wants_unit_done()) {
-        named_bar_sync(2, 128);
-        plan.unit_done(m, sh);
-      }
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sh.accempty[buf]);
+    if (complete && plan.wants_unit_done()) {
+      named_bar_sync(2, 128);
+      plan.unit_done(m, sh);
     }
   }
 }
 
 template <class Plan>
 KD_DEV void mma_run(const Plan& plan, uint8_t* smem_raw, unsigned* err) {
-  MmaShared sh = carve_mma_smem(smem_raw, plan.max_n(), plan.split_b(), plan.nsub);
+  MmaShared sh = carve_mma_smem(smem_raw, plan.max_n(), Plan::kTerms, plan.nsub);
   const int warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
     for (int i = 0; i < sh.nst; ++i) {
@@ -467,6 +514,7 @@ KD_DEV void mma_run(const Plan& plan, uint8_t* smem_raw, unsigned* err) {
       mbar_init(&sh.accempty[i], 4);
     }
     *sh.abort_flag = 0;
+    sh.misc[2] = 0;
     fence_mbar_init();
   }
   if (warp == 1) tmem_alloc(sh.tmem_base, 2 * kMaxN);
@@ -489,6 +537,7 @@ KD_DEV void mma_run(const Plan& plan, uint8_t* smem_raw, unsigned* err) {
     tc_fence_after();
     tmem_dealloc(tmem, 2 * kMaxN);
   }
+  plan.after_run(sh, smem_raw);
 }
 
 }  // namespace kd

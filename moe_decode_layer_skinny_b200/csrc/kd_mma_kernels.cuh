@@ -7,6 +7,7 @@
 // Tensor maps (one per weight matrix, box 64 K x 128 rows, 128B swizzle):
 //   0 Wqkv [Nqkv, H]   1 Wo [H, A]   2 routed gate/up [E*2I, H]
 //   3 routed down [E*H, I]   4 shared gate/up [2I, H]   5 shared down [H, I]
+//   6 router [E, H]
 #pragma once
 
 #include "kd_kernels.cuh"
@@ -14,8 +15,9 @@
 
 namespace kd {
 
+constexpr int kNumMaps = 7;
 struct MmaMaps {
-  CUtensorMap m[6];
+  CUtensorMap m[kNumMaps];
 };
 
 // Largest token count among the active experts (every thread gets it).
@@ -35,6 +37,17 @@ KD_DEV void store_hilo(uint16_t* hi, uint16_t* lo, size_t o, float v) {
   const uint16_t h = f32_to_bf16_bits(v);
   hi[o] = h;
   lo[o] = f32_to_bf16_bits(v - __uint_as_float((uint32_t)h << 16));
+}
+
+// v = hi + mid + lo exactly (each difference is exact in fp32; three 8-bit
+// significands cover fp32's 24).
+KD_DEV void store_hilo3(uint16_t* hi, uint16_t* mid, uint16_t* lo, size_t o, float v) {
+  const uint16_t h = f32_to_bf16_bits(v);
+  const float r1 = v - __uint_as_float((uint32_t)h << 16);
+  const uint16_t m = f32_to_bf16_bits(r1);
+  hi[o] = h;
+  mid[o] = m;
+  lo[o] = f32_to_bf16_bits(r1 - __uint_as_float((uint32_t)m << 16));
 }
 
 // ------------------------------------------------------------------ QKV + o-proj
@@ -59,10 +72,10 @@ struct MmaProjPlan {
   }
   KD_DEV const CUtensorMap* map(int id) const { return &maps->m[id]; }
   KD_DEV int max_n() const { return a.M; }
-  KD_DEV bool split_b() const { return false; }
-  KD_DEV const uint16_t* b_row(const MUnit& m, int j, int) const {
-    return m.tag == 0 ? a.x + (size_t)j * L->H : a.attn + (size_t)j * L->A;
-  }
+  static constexpr int kTerms = 1;
+  KD_DEV const uint16_t* b_base(const MUnit& m, int) const { return m.tag == 0 ? a.x : a.attn; }
+  KD_DEV int b_stride(const MUnit& m) const { return m.tag == 0 ? L->H : L->A; }
+  KD_DEV int b_rowidx(const MUnit&, int j) const { return j; }
   KD_DEV bool paired() const { return false; }
   KD_DEV void epilogue(const MUnit& m, int r, int j, float v) const {
     const int row = m.lrow + r;
@@ -72,7 +85,7 @@ struct MmaProjPlan {
       const size_t o = (size_t)j * L->H + row;
       const float h = __uint_as_float((uint32_t)a.x[o] << 16) + v;
       L->h1f[o] = h;
-      store_hilo(L->h1b, L->h1lo, o, h);
+      store_hilo3(L->h1b, L->h1lo, L->h1lo2, o, h);
     }
   }
   KD_DEV void epilogue2(const MUnit&, int, int, float, float) const {}
@@ -80,6 +93,7 @@ struct MmaProjPlan {
   KD_DEV unsigned* tile_cnt() const { return L->tcnt_main; }
   KD_DEV bool wants_unit_done() const { return false; }
   KD_DEV void unit_done(const MUnit&, MmaShared&) const {}
+  KD_DEV void after_run(MmaShared&, uint8_t*) const {}
 };
 
 __global__ void __launch_bounds__(kMThreads, 1) mma_proj_kernel(LayerDev L, Acts a,
@@ -87,17 +101,87 @@ __global__ void __launch_bounds__(kMThreads, 1) mma_proj_kernel(LayerDev L, Acts
   extern __shared__ uint8_t smem[];
   MmaProjPlan p;
   p.L = &L; p.a = a; p.maps = &maps;
-  p.nsub = mma_nsub(a.M, false);
+  p.nsub = mma_nsub(a.M, 1);
   p.tq = L.Nqkv / 128; p.to = L.H / 128; p.cq = L.H / (64 * p.nsub); p.co = L.A / (64 * p.nsub);
   pdl_wait();
   pdl_launch_dependents();
   mma_run(p, smem, L.err);
 }
 
+// ------------------------------------------------------------------ router
+
+// fp32 router logits: the E router rows (ceil(E/128) tiles, rows past E read
+// as zeros) against h1 as three bf16 terms, so that every product is exact and
+// only the fp32 accumulation rounds.  Launched on a small grid (a few K chunks
+// per CTA) to keep the split-K partial sums short.  The CTA that completes
+// the last tile then selects every token's experts (top-k, renormalised
+// softmax) and builds the per-expert token lists, all within this launch.
+struct MmaRouterPlan {
+  const LayerDev* L; int M; const MmaMaps* maps;
+  int nsub;
+  KD_DEV int num_tiles() const { return (L->E + 127) / 128; }
+  KD_DEV long long tile_start(int t) const { return (long long)t * (L->H / (64 * nsub)); }
+  KD_DEV MUnit tile_unit(int t) const {
+    MUnit m{};
+    m.map = 6; m.lrow = m.row = t * 128; m.tag = 0; m.tok0 = 0; m.ntok = M;
+    return m;
+  }
+  KD_DEV const CUtensorMap* map(int id) const { return &maps->m[id]; }
+  KD_DEV int max_n() const { return M; }
+  static constexpr int kTerms = 3;
+  KD_DEV const uint16_t* b_base(const MUnit&, int h) const {
+    return h == 0 ? L->h1b : h == 1 ? L->h1lo : L->h1lo2;
+  }
+  KD_DEV int b_stride(const MUnit&) const { return L->H; }
+  KD_DEV int b_rowidx(const MUnit&, int j) const { return j; }
+  KD_DEV bool paired() const { return false; }
+  KD_DEV void epilogue(const MUnit& m, int r, int j, float v) const {
+    const int e = m.lrow + r;
+    if (e < L->E) L->logits[(size_t)j * L->E + e] = v + (L->bias ? L->bias[e] : 0.f);
+  }
+  KD_DEV void epilogue2(const MUnit&, int, int, float, float) const {}
+  KD_DEV float* ws() const { return L->ws_main; }
+  KD_DEV unsigned* tile_cnt() const { return L->tcnt_main; }
+  // the CTA that completes the last tile of logits routes the call
+  KD_DEV bool wants_unit_done() const { return true; }
+  KD_DEV void unit_done(const MUnit&, MmaShared& sh) const {
+    __threadfence();
+    named_bar_sync(2, 128);
+    if (threadIdx.x == 128) {
+      const unsigned prev = atomicAdd(L->rcnt, 1u);
+      if (prev == (unsigned)num_tiles() - 1) {
+        *L->rcnt = 0u;
+        sh.misc[2] = 1;
+      }
+    }
+  }
+  KD_DEV void after_run(MmaShared& sh, uint8_t* smem) const {
+    if (!sh.misc[2]) return;
+    __threadfence();
+    const Route R = carve_route(reinterpret_cast<int*>(smem + kMmaSmem), L->E, M * L->k);
+    route_tokens(*L, M, R, true);
+  }
+};
+
+// K chunks each router CTA streams (sets the router launch's grid).
+constexpr int kRouterChunksPerCta = 8;
+
+__global__ void __launch_bounds__(kMThreads, 1) mma_router_kernel(LayerDev L, int M,
+                                                                  const __grid_constant__ MmaMaps maps) {
+  extern __shared__ uint8_t smem[];
+  MmaRouterPlan p;
+  p.L = &L; p.M = M; p.maps = &maps;
+  p.nsub = mma_nsub(M, 3);
+  pdl_wait();
+  mma_run(p, smem, L.err);
+  pdl_launch_dependents();
+}
+
 // ------------------------------------------------------------------ gate/up
 
 // Routed: tiles of the active experts' interleaved gate/up rows (2I/128 per
-// expert); shared: the shared expert's.  B = h1 as a bf16 hi/lo pair.
+// expert); shared: the shared expert's (all M tokens; its own launch on the
+// side stream).  B = h1 as a bf16 hi/lo pair.
 struct MmaGateUpPlan {
   const LayerDev* L; int M; bool shared; const MmaMaps* maps; Route rt; int n_act;
   int nsub, nmax;
@@ -119,21 +203,23 @@ struct MmaGateUpPlan {
   }
   KD_DEV const CUtensorMap* map(int id) const { return &maps->m[id]; }
   KD_DEV int max_n() const { return nmax; }
-  KD_DEV bool split_b() const { return true; }
-  KD_DEV const uint16_t* b_row(const MUnit& m, int j, int h) const {
-    const int t = shared ? j : rt.perm[m.tok0 + j] / L->k;
-    return (h ? L->h1lo : L->h1b) + (size_t)t * L->H;
+  static constexpr int kTerms = 2;
+  KD_DEV const uint16_t* b_base(const MUnit&, int h) const { return h ? L->h1lo : L->h1b; }
+  KD_DEV int b_stride(const MUnit&) const { return L->H; }
+  KD_DEV int b_rowidx(const MUnit& m, int j) const {
+    return shared ? j : rt.perm[m.tok0 + j] / L->k;
   }
   KD_DEV bool paired() const { return true; }
   KD_DEV void epilogue(const MUnit&, int, int, float) const {}
   KD_DEV void epilogue2(const MUnit& m, int p, int j, float g, float u) const {
     const int i = m.lrow / 2 + p;
     const float v = silu(g) * u;
-    const size_t o = shared ? (size_t)j * L->I + i : (size_t)(m.tok0 + j) * L->I + i;
     if (shared) {
+      const size_t o = (size_t)j * L->I + i;
       L->act_sh[o] = v;
       store_hilo(L->act_sh_hi, L->act_sh_lo, o, v);
     } else {
+      const size_t o = (size_t)(m.tok0 + j) * L->I + i;
       L->act[o] = v;
       store_hilo(L->act_hi, L->act_lo, o, v);
     }
@@ -142,6 +228,7 @@ struct MmaGateUpPlan {
   KD_DEV unsigned* tile_cnt() const { return shared ? L->tcnt_side : L->tcnt_main; }
   KD_DEV bool wants_unit_done() const { return false; }
   KD_DEV void unit_done(const MUnit&, MmaShared&) const {}
+  KD_DEV void after_run(MmaShared&, uint8_t*) const {}
 };
 
 __global__ void __launch_bounds__(kMThreads, 1) mma_gateup_kernel(LayerDev L, int M, int shared,
@@ -154,20 +241,23 @@ __global__ void __launch_bounds__(kMThreads, 1) mma_gateup_kernel(LayerDev L, in
     pdl_wait();
     pdl_launch_dependents();
     p.rt = carve_route(reinterpret_cast<int*>(smem + kMmaSmem), L.E, M * L.k);
-    route_tokens(L, M, p.rt, blockIdx.x == 0);
+    load_route(L, M, p.rt);
     p.n_act = *p.rt.n_act;
     p.nmax = max_tokens_per_expert(p.rt.cnt, p.rt.act, p.n_act);
   }
-  p.nsub = mma_nsub(p.nmax, true);
+  p.nsub = mma_nsub(p.nmax, 2);
   mma_run(p, smem, L.err);
 }
 
 // ------------------------------------------------------------------ down + combine
 
-// Tiles of the active experts' down projections (H/128 per expert), then the
-// shared expert's.  B = the SwiGLU activations as a bf16 hi/lo pair.  A CTA
-// that completes a tile counts its 128 rows into the 64-row blocks; the CTA
-// completing a block (every entry) writes that block of the layer output.
+// Tiles of the down projections of the active experts and the shared expert
+// ("entries"), ordered by output row tile first: tile t is row tile
+// t / entries of entry t % entries, so the 64-row output blocks complete one
+// after another through the launch and their combines spread over the CTAs.
+// B = the SwiGLU activations as a bf16 hi/lo pair.  A CTA that completes a
+// tile counts its 128 rows into the 64-row blocks; the CTA completing a block
+// (every entry) writes that block of the layer output.
 struct MmaDownPlan {
   const LayerDev* L; int M; int n_act; const MmaMaps* maps; uint16_t* out;
   int nsub, nmax;
@@ -176,7 +266,7 @@ struct MmaDownPlan {
   KD_DEV long long tile_start(int t) const { return (long long)t * (L->I / (64 * nsub)); }
   KD_DEV MUnit tile_unit(int t) const {
     MUnit m{};
-    const int a = t / tiles_per(), tt = t % tiles_per();
+    const int a = t % (n_act + L->S), tt = t / (n_act + L->S);
     if (a >= n_act) {
       m.map = 5; m.row = tt * 128; m.tag = -1; m.tok0 = 0; m.ntok = M;
     } else {
@@ -189,11 +279,13 @@ struct MmaDownPlan {
   }
   KD_DEV const CUtensorMap* map(int id) const { return &maps->m[id]; }
   KD_DEV int max_n() const { return nmax; }
-  KD_DEV bool split_b() const { return true; }
-  KD_DEV const uint16_t* b_row(const MUnit& m, int j, int h) const {
-    if (m.tag < 0) return (h ? L->act_sh_lo : L->act_sh_hi) + (size_t)j * L->I;
-    return (h ? L->act_lo : L->act_hi) + (size_t)(m.tok0 + j) * L->I;
+  static constexpr int kTerms = 2;
+  KD_DEV const uint16_t* b_base(const MUnit& m, int h) const {
+    if (m.tag < 0) return h ? L->act_sh_lo : L->act_sh_hi;
+    return h ? L->act_lo : L->act_hi;
   }
+  KD_DEV int b_stride(const MUnit&) const { return L->I; }
+  KD_DEV int b_rowidx(const MUnit& m, int j) const { return m.tag < 0 ? j : m.tok0 + j; }
   KD_DEV bool paired() const { return false; }
   KD_DEV void epilogue(const MUnit& m, int r, int j, float v) const {
     const int h = m.lrow + r;
@@ -204,6 +296,7 @@ struct MmaDownPlan {
   KD_DEV float* ws() const { return L->ws_main; }
   KD_DEV unsigned* tile_cnt() const { return L->tcnt_main; }
   KD_DEV bool wants_unit_done() const { return true; }
+  KD_DEV void after_run(MmaShared&, uint8_t*) const {}
   // epilogue warps only (128 threads, named barrier 2)
   KD_DEV void unit_done(const MUnit& m, MmaShared& sh) const {
     const int target = 64 * (n_act + L->S);
@@ -249,7 +342,7 @@ __global__ void __launch_bounds__(kMThreads, 1) mma_down_kernel(LayerDev L, int 
   p.n_act = *(volatile int*)L.n_active;
   p.nmax = max_tokens_per_expert(L.counts, L.active, p.n_act);
   if (L.S && M > p.nmax) p.nmax = M;
-  p.nsub = mma_nsub(p.nmax, true);
+  p.nsub = mma_nsub(p.nmax, 2);
   mma_run(p, smem, L.err);
 }
 

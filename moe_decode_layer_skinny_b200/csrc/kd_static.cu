@@ -31,10 +31,14 @@ constexpr int kMaxExp = KD_STATIC_MAX_EXPERTS;
 constexpr int kMaxK = 16;
 
 // logits [64 x 1024] | counts [1024] | offsets [1025] | active [1024]
-// | perm [64 x 16] | n_active [1] | err [1]       (4-byte words)
+// | perm [64 x 16] | n_active [1] | err [1] | router blocks done [1]   (4-byte words)
 constexpr size_t kWords = (size_t)kMaxTok * kMaxExp + kMaxExp + (kMaxExp + 1) + kMaxExp +
-                          (size_t)kMaxTok * kMaxK + 2;
+                          (size_t)kMaxTok * kMaxK + 3;
 
+// Every scratch word is written before it is read within a call (logits by
+// the logit blocks, lists by the selection), so nothing needs clearing; the
+// block-completion counter starts at zero (static storage) and the last
+// block of every call puts it back to zero.
 static __device__ __align__(256) float g_router_scratch[kWords];
 
 constexpr int kMaxDevices = 64;
@@ -42,15 +46,6 @@ std::mutex g_mu;
 void* g_scratch_ptr[kMaxDevices] = {};
 
 thread_local char g_msg[256];
-
-// Every scratch word is written before it is read within a call (logits by
-// the logit kernel, lists by the selection), so nothing needs clearing.
-__global__ void __launch_bounds__(256) topk_kernel(LayerDev L, int M) {
-  extern __shared__ int route_smem[];
-  const Route R = carve_route(route_smem, L.E, M * L.k);
-  route_tokens(L, M, R, true);
-}
-
 }  // namespace
 
 // kd_last_error() reports these messages too (defined with the layer API).
@@ -121,13 +116,14 @@ extern "C" int kd_router_topk_static(const void* router_w, const float* router_s
   d.active = w + o; o += kMaxExp;
   d.perm = w + o; o += (size_t)kMaxTok * kMaxK;
   d.n_active = w + o; o += 1;
-  d.err = reinterpret_cast<unsigned*>(w + o);
+  d.err = reinterpret_cast<unsigned*>(w + o); o += 1;
+  d.rcnt = reinterpret_cast<unsigned*>(w + o);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // one launch: logits, then the last block selects and builds the lists
   const int rgrid = (n_experts + kRouterRows - 1) / kRouterRows;
-  if (wdtype == KD_WFP8) router_kernel<W_FP8><<<rgrid, kRouterThreads, 0, s>>>(d, M);
-  else router_kernel<W_BF16><<<rgrid, kRouterThreads, 0, s>>>(d, M);
-  const size_t smem = sizeof(int) * kRouteSmemInts(n_experts, M * top_k);
-  topk_kernel<<<1, 256, smem, s>>>(d, M);
+  const size_t smem = sizeof(int) * kRouteSmemInts(n_experts, M * top_k);   // < 48 KB
+  if (wdtype == KD_WFP8) router_kernel<W_FP8><<<rgrid, kRouterThreads, smem, s>>>(d, M);
+  else router_kernel<W_BF16><<<rgrid, kRouterThreads, smem, s>>>(d, M);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     snprintf(g_msg, sizeof g_msg, "kd_router_topk_static: launch: %s", cudaGetErrorString(e));

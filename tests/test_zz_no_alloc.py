@@ -15,7 +15,9 @@ pytestmark = pytest.mark.gpu
 
 
 def _case(kd, torch, dims, wdtype, bias, M):
-    spec = kd.LayerSpec.from_dims(dims, wdtype=wdtype, max_tokens=M, router_bias=bias)
+    # the layer's CUDA-core router (the tensor-core one rounds differently)
+    spec = kd.LayerSpec.from_dims(dims, wdtype=wdtype, max_tokens=M, router_bias=bias,
+                                  mma_min_tokens=1000)
     layer = kd.Layer(spec, seed=0)
     try:
         x = kdgen.activations(0, 0, kdgen.HIDDEN_IN, M, dims.hidden, 0.3)
