@@ -443,7 +443,7 @@ def run_kd(args):
     clocks = cs.summary()
     e2e_times, h2d, d2h = time_layer_e2e(layer, x, a, min(args.steps, 200), args.warmup, flush, pg,
                                          local)
-    launches_per_step = 4 + (1 if main.dims.n_shared else 0)
+    launches_per_step = layer.launches(main.M)
     layer.close()
     ms = res["us_per_layer"] / 1e3
     ms_max = max_over_ranks(pg, ms)

@@ -143,6 +143,11 @@ int kd_layer_read_weight(const kd_layer* layer, int kind, int expert, int row0, 
  * router, shared expert, with FP8 scales) and the bytes of one routed expert. */
 int kd_layer_bytes(const kd_layer* layer, uint64_t* static_bytes, uint64_t* expert_bytes);
 
+/* Number of kernels one kd_decode_layer call with M tokens launches (all of
+ * them this library's).  Returns the count (>= 4), or KD_EINVAL for a null
+ * layer, KD_ERANGE for M outside 1..max_tokens. */
+int kd_layer_launches(const kd_layer* layer, int M);
+
 /* Multi-layer decode step.  kd_stack_create records the layers (not owned)
  * and the token count; kd_stack_run runs layer 0..n-1 in order on `stream`,
  * reading attn_out for layer l at attn_out + l*M*A, and carrying hidden.
@@ -184,7 +189,7 @@ int kd_layer_set_timing_events(kd_layer* layer, void* const* events, int n_event
  *                 ties -> lower id
  *   gates_out     device fp32 [M, top_k]: softmax renormalised over the top_k
  * Same arithmetic as the CUDA-core router of kd_decode_layer (the one it
- * runs for FP8 layers and below the tensor-core token threshold).  Limits: M <= 64
+ * runs below the tensor-core token threshold).  Limits: M <= 64
  * (KD_STATIC_MAX_TOKENS), n_experts <= 1024 (KD_STATIC_MAX_EXPERTS),
  * top_k <= 16, hidden a multiple of 128 and <= 8192; larger sizes return
  * KD_ERANGE, bad pointers or shapes KD_EINVAL.  Calls no cudaMalloc /

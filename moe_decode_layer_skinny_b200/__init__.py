@@ -23,8 +23,8 @@ T_H1F, T_H1B, T_LOGITS, T_IDX, T_GATES, T_COUNTS, T_NACTIVE, T_YSHARED, T_YROUTE
 # every symbol include/kd.h declares
 EXPORTS = ("kd_layer_create", "kd_layer_destroy", "kd_decode_layer", "kd_layer_check",
            "kd_layer_qkv", "kd_layer_prefetch_l2", "kd_layer_debug_tensor", "kd_layer_read_weight",
-           "kd_layer_bytes", "kd_layer_set_timing_events", "kd_stack_create", "kd_stack_run",
-           "kd_stack_destroy", "kd_router_topk_static", "kd_last_error")
+           "kd_layer_bytes", "kd_layer_launches", "kd_layer_set_timing_events", "kd_stack_create",
+           "kd_stack_run", "kd_stack_destroy", "kd_router_topk_static", "kd_last_error")
 N_TIMING_EVENTS = 5
 
 
@@ -64,6 +64,7 @@ def lib() -> ctypes.CDLL:
         L.kd_layer_debug_tensor.argtypes = [vp, i32, ctypes.POINTER(vp)]
         L.kd_layer_read_weight.argtypes = [vp, i32, i32, i32, i32, vp, vp]
         L.kd_layer_bytes.argtypes = [vp, ctypes.POINTER(u64), ctypes.POINTER(u64)]
+        L.kd_layer_launches.argtypes = [vp, ctypes.c_int]
         L.kd_layer_set_timing_events.argtypes = [vp, ctypes.POINTER(vp), i32]
         L.kd_stack_create.argtypes = [ctypes.POINTER(vp), i32, i32, i32, ctypes.POINTER(vp)]
         L.kd_stack_run.argtypes = [vp, vp, vp, vp]
@@ -174,6 +175,13 @@ class Layer:
             raise ValueError("timing events must have been recorded once (torch creates them lazily)")
         arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
         _check(lib().kd_layer_set_timing_events(self._h, arr, len(events)))
+
+    def launches(self, M: int) -> int:
+        """Kernels one decode call with M tokens launches."""
+        n = lib().kd_layer_launches(self._h, M)
+        if n < 0:
+            _check(n)
+        return n
 
     def bytes(self) -> tuple[int, int]:
         a, b = ctypes.c_uint64(), ctypes.c_uint64()

@@ -209,6 +209,7 @@ KD_DEV void router_chunk(const uint4 wv, float scale, const float* const* arow, 
 // to global memory for the down kernel and for inspection.
 struct Route {
   int* sel;      // [M*k] selected expert of (token, slot), descending logit
+  float* gv;     // [M*k] its logit
   int* cnt;      // [E] tokens per expert
   int* off;      // [E] exclusive scan of cnt
   int* act;      // [E] active experts in id order
@@ -217,12 +218,15 @@ struct Route {
   int* wsum;     // [2][32] scan scratch
 };
 
-constexpr size_t kRouteSmemInts(int E, int Mk) { return (size_t)3 * E + 2 * Mk + 1 + 64; }
+__host__ __device__ constexpr size_t kRouteSmemInts(int E, int Mk) {
+  return (size_t)3 * E + 3 * Mk + 1 + 64;
+}
 
 KD_DEV Route carve_route(int* base, int E, int Mk) {
   Route r;
   r.sel = base;
-  r.perm = r.sel + Mk;
+  r.gv = reinterpret_cast<float*>(r.sel + Mk);
+  r.perm = r.sel + 2 * Mk;
   r.cnt = r.perm + Mk;
   r.off = r.cnt + E;
   r.act = r.off + E;
@@ -236,6 +240,7 @@ KD_DEV Route carve_route(int* base, int E, int Mk) {
 // values, all bits for negative ones) and the expert id complemented below.
 KD_DEV uint64_t route_key(float v, int e) {
   uint32_t u = __float_as_uint(v);
+  if ((u << 1) == 0u) u = 0u;   // -0 ranks with +0 (then the lower id wins)
   u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
   return ((uint64_t)u << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)e);
 }
@@ -246,121 +251,90 @@ KD_DEV float key_value(uint64_t key) {
 }
 KD_DEV int key_expert(uint64_t key) { return (int)(0xFFFFFFFFu - (uint32_t)key); }
 
-KD_DEV void cas_desc(uint64_t& x, uint64_t& y) {
-  const uint64_t hi = x > y ? x : y, lo = x > y ? y : x;
-  x = hi;
-  y = lo;
-}
-// bitonic sequence -> descending
-template <int N>
-KD_DEV void bitonic_merge_desc(uint64_t (&a)[N]) {
-#pragma unroll
-  for (int st = N / 2; st > 0; st >>= 1)
-#pragma unroll
-    for (int i = 0; i < N; ++i)
-      if (!(i & st)) cas_desc(a[i], a[i + st]);
-}
-// any sequence -> descending (bitonic sort)
-template <int N>
-KD_DEV void bitonic_sort_desc(uint64_t (&a)[N]) {
-#pragma unroll
-  for (int sz = 2; sz <= N; sz <<= 1)
-#pragma unroll
-    for (int st = sz / 2; st > 0; st >>= 1)
-#pragma unroll
-      for (int i = 0; i < N; ++i) {
-        const int l = i ^ st;
-        if (l > i) {
-          if ((i & sz) == 0 || sz == N) cas_desc(a[i], a[l]);
-          else cas_desc(a[l], a[i]);
-        }
-      }
-}
-// a, b descending -> a = the largest N of both, descending
-template <int N>
-KD_DEV void keep_top_desc(uint64_t (&a)[N], const uint64_t (&b)[N]) {
-#pragma unroll
-  for (int i = 0; i < N; ++i) a[i] = a[i] > b[N - 1 - i] ? a[i] : b[N - 1 - i];
-  bitonic_merge_desc(a);
-}
-
-// Top-k of token t by one warp: lane holds the logits of experts lane,
-// lane + 32, ... (PER of them, PER >= E / 32) and sorts their keys into a
-// descending list of LL >= k; five butterfly rounds (partner = lane ^ 1, ^ 2,
-// ..., ^ 16) each keep the largest LL of the two lists, after which every lane
-// holds the token's top LL.  Then the softmax renormalised over the first k.
-template <int PER, int LL>
-KD_DEV void topk_token(const LayerDev& L, const Route& R, int t, bool write_global) {
-  const int lane = threadIdx.x & 31;
+// Top-k of token t by a group of LPT lanes of a warp (32 / LPT tokens per
+// warp at once): lane l of the group holds the keys of experts l, l + LPT,
+// ... (PER of them, PER * LPT >= E).  k rounds, each: the lane's largest
+// remaining key, the group's largest by a shuffle reduction, and the owner
+// drops it.  Loops that run more than once are rolled, so the code stays
+// small for the instruction cache.  Then the softmax renormalised over the k
+// selected logits (same order and arithmetic in every lane of the group).
+// Groups whose token is past M run on empty keys and write nothing.
+template <int PER, int LPT>
+KD_DEV void topk_group(const LayerDev& L, const float* lg, const Route& R, int t, int M,
+                       bool write_global) {
+  const int sl = threadIdx.x & (LPT - 1);
   const int k = L.k, E = L.E;
-  uint64_t a[LL];
+  const bool act = t < M;
+  uint64_t key[PER];
 #pragma unroll
-  for (int g = 0; g < (PER + LL - 1) / LL; ++g) {
-    uint64_t b[LL];
-#pragma unroll
-    for (int i = 0; i < LL; ++i) {
-      const int qq = g * LL + i, e = lane + 32 * qq;
-      b[i] = (qq < PER && e < E) ? route_key(L.logits[(size_t)t * E + e], e) : 0ull;
-    }
-    bitonic_sort_desc(b);
-    if (g == 0) {
-#pragma unroll
-      for (int i = 0; i < LL; ++i) a[i] = b[i];
-    } else {
-      keep_top_desc(a, b);
-    }
+  for (int qq = 0; qq < PER; ++qq) {
+    const int e = sl + LPT * qq;
+    key[qq] = (act && e < E) ? route_key(lg[(size_t)t * E + e], e) : 0ull;
   }
+  float top = 0.f, den = 0.f;
 #pragma unroll 1
-  for (int o = 1; o < 32; o <<= 1) {
-    uint64_t b[LL];
+  for (int j = 0; j < k; ++j) {
+    uint64_t best = key[0];
 #pragma unroll
-    for (int i = 0; i < LL; ++i) b[i] = __shfl_xor_sync(0xffffffffu, a[i], o);
-    keep_top_desc(a, b);
-  }
-  const float top = key_value(a[0]);
-  float den = 0.f, mysel = 0.f;
-  int mye = 0;
+    for (int qq = 1; qq < PER; ++qq) best = key[qq] > best ? key[qq] : best;
+#pragma unroll 1
+    for (int o = LPT / 2; o > 0; o >>= 1) {
+      const uint64_t other = __shfl_xor_sync(0xffffffffu, best, o);
+      best = other > best ? other : best;
+    }
 #pragma unroll
-  for (int i = 0; i < LL; ++i) {
-    if (i < k) {
-      const float v = key_value(a[i]);
-      den += expf(v - top);
-      if (i == lane) {
-        mysel = v;
-        mye = key_expert(a[i]);
-      }
+    for (int qq = 0; qq < PER; ++qq)
+      if (key[qq] == best) key[qq] = 0ull;   // keys are unique (expert id)
+    const float v = key_value(best);
+    if (j == 0) top = v;
+    den += expf(v - top);
+    if (act && sl == 0) {
+      const int e = key_expert(best);
+      R.sel[t * k + j] = e;
+      R.gv[t * k + j] = v;
+      if (write_global) L.idx[t * k + j] = e;
     }
   }
-  if (lane < k) {
-    R.sel[t * k + lane] = mye;
-    if (write_global) {
-      L.idx[t * k + lane] = mye;
-      L.gates[t * k + lane] = expf(mysel - top) / den;
-    }
-  }
+  __syncwarp();
+  if (act && write_global)
+    for (int j = sl; j < k; j += LPT) L.gates[t * k + j] = expf(R.gv[t * k + j] - top) / den;
 }
 
-template <int PER>
-KD_DEV void topk_token_k(const LayerDev& L, const Route& R, int t, bool write_global) {
-  if (L.k <= 8) topk_token<PER, 8>(L, R, t, write_global);
-  else topk_token<PER, 16>(L, R, t, write_global);
+template <int LPT>
+KD_DEV void topk_tokens(const LayerDev& L, const float* lg, const Route& R, int M,
+                        bool write_global) {
+  constexpr int TPW = 32 / LPT;
+  const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const int g = (threadIdx.x & 31) / LPT;
+  const int per = (L.E + LPT - 1) / LPT;   // <= 32
+  for (int t0 = warp * TPW; t0 < M; t0 += nw * TPW) {
+    const int t = t0 + g;
+    if (per <= 1) topk_group<1, LPT>(L, lg, R, t, M, write_global);
+    else if (per <= 2) topk_group<2, LPT>(L, lg, R, t, M, write_global);
+    else if (per <= 4) topk_group<4, LPT>(L, lg, R, t, M, write_global);
+    else if (per <= 8) topk_group<8, LPT>(L, lg, R, t, M, write_global);
+    else if (per <= 16) topk_group<16, LPT>(L, lg, R, t, M, write_global);
+    else topk_group<32, LPT>(L, lg, R, t, M, write_global);
+  }
 }
 
 // Top-k of every token, the renormalised softmax over each selection, and the
-// per-expert token lists.
-KD_DEV void route_tokens(const LayerDev& L, int M, const Route& R, bool write_global) {
+// per-expert token lists.  lg: the logits [M, E] (global, or a copy in shared
+// memory).
+KD_DEV void route_tokens(const LayerDev& L, const float* lg, int M, const Route& R,
+                         bool write_global) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nw = blockDim.x >> 5;
   const int k = L.k, E = L.E;
-  const int per = (E + 31) / 32;   // E <= 1024
-  for (int t = warp; t < M; t += nw) {
-    if (per <= 1) topk_token_k<1>(L, R, t, write_global);
-    else if (per <= 2) topk_token_k<2>(L, R, t, write_global);
-    else if (per <= 4) topk_token_k<4>(L, R, t, write_global);
-    else if (per <= 8) topk_token_k<8>(L, R, t, write_global);
-    else if (per <= 16) topk_token_k<16>(L, R, t, write_global);
-    else topk_token_k<32>(L, R, t, write_global);
-  }
+  // lanes per token: fewer (more tokens per warp at once) when each warp has
+  // several tokens, but at least E / 32 so that a lane holds <= 32 keys
+  const int tpw = (M + nw - 1) / nw;
+  int lpt = tpw >= 4 ? 8 : tpw >= 2 ? 16 : 32;
+  if (E > 32 * lpt) lpt = E > 512 ? 32 : 16;
+  if (lpt == 8) topk_tokens<8>(L, lg, R, M, write_global);
+  else if (lpt == 16) topk_tokens<16>(L, lg, R, M, write_global);
+  else topk_tokens<32>(L, lg, R, M, write_global);
+  __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) R.cnt[e] = 0;
   __syncthreads();
   const int ncode = M * k;
@@ -457,7 +431,19 @@ KD_DEV void route_last_block(const LayerDev& L, int M, unsigned nblocks) {
   if (!s_last) return;
   __threadfence();
   const Route R = carve_route(route_smem, L.E, M * L.k);
-  route_tokens(L, M, R, true);
+  route_tokens(L, L.logits, M, R, true);
+}
+
+// The routing of the call as the router left it in global memory (only the
+// fields the expert kernels read).
+KD_DEV Route global_route(const LayerDev& L) {
+  Route r{};
+  r.perm = L.perm;
+  r.cnt = L.counts;
+  r.off = L.offsets;
+  r.act = L.active;
+  r.n_act = L.n_active;
+  return r;
 }
 
 // The routing of the call, as the router left it in global memory, copied

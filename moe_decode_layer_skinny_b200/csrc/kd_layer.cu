@@ -114,17 +114,19 @@ static EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D map of a row-major bf16 matrix [rows, K]: box 64 K x 128 rows, 128B swizzle.
-static bool encode_bf16_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t K) {
+// 2-D map of a row-major weight matrix [rows, K] (bf16 or e4m3 codes): box
+// 128 bytes x 128 rows (64 bf16 or 128 e4m3 per row), 128B swizzle.
+static bool encode_weight_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t K, bool fp8) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[2] = {K, rows};
-  const cuuint64_t strides[1] = {K * 2};
-  const cuuint32_t box[2] = {64, 128};
+  const cuuint64_t strides[1] = {K * (fp8 ? 1 : 2)};
+  const cuuint32_t box[2] = {fp8 ? 128u : 64u, 128};
   const cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return fn(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+            const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // Generate one logical [R, K] matrix into `dst` with row stride multiplier
@@ -170,11 +172,14 @@ static int configure_kernels() {
   const int rsmem = (int)(sizeof(int) * kRouteSmemInts(1024, 64 * 16));
   KD_CUDA(cudaFuncSetAttribute(router_kernel<W_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, rsmem));
   KD_CUDA(cudaFuncSetAttribute(router_kernel<W_FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, rsmem));
-  const int msmem = (int)(kMmaSmem + 16 + sizeof(int) * kRouteSmemInts(1024, 64 * 16));
-  KD_CUDA(cudaFuncSetAttribute(mma_proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem));
-  KD_CUDA(cudaFuncSetAttribute(mma_gateup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem));
-  KD_CUDA(cudaFuncSetAttribute(mma_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem));
-  KD_CUDA(cudaFuncSetAttribute(mma_router_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem));
+  const int msmem = (int)kMmaSmem;
+  KD_CUDA(cudaFuncSetAttribute(mma_proj_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem));
+  KD_CUDA(cudaFuncSetAttribute(mma_gateup_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem));
+  KD_CUDA(cudaFuncSetAttribute(mma_down_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem));
+  KD_CUDA(cudaFuncSetAttribute(mma_router_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem));
+  KD_CUDA(cudaFuncSetAttribute(mma_proj_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem));
+  KD_CUDA(cudaFuncSetAttribute(mma_gateup_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem));
+  KD_CUDA(cudaFuncSetAttribute(mma_down_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem));
   stream_kernels_configured = true;
   return KD_OK;
 }
@@ -303,7 +308,7 @@ extern "C" int kd_layer_create(const kd_config* cfg, uint64_t seed, kd_layer** o
   TRY(dalloc_t(L, (size_t)L->nsm * kWsFloatsPerCta, &d.ws_main));
   TRY(dalloc_t(L, (size_t)L->nsm * kWsFloatsPerCta, &d.ws_side));
   {
-    const size_t ntile = std::max<size_t>({(size_t)(E + 1) * (H / 128), (size_t)(E + 1) * (2 * I / 128),
+    const size_t ntile = std::max<size_t>({(size_t)(E + 4) * (H / 128), (size_t)(E + 1) * (2 * I / 128),
                                            (size_t)(Nqkv + H) / 128});
     TRY(dalloc_t(L, ntile, &d.tcnt_main));
     TRY(dalloc_t(L, ntile, &d.tcnt_side));
@@ -340,13 +345,15 @@ extern "C" int kd_layer_create(const kd_config* cfg, uint64_t seed, kd_layer** o
   if (rc != KD_OK) { free_layer(L); return rc; }
   TRYC(se);
 
-  if (!fp8) {
-    bool ok = encode_bf16_map(&L->maps.m[0], wqkv, Nqkv, H) && encode_bf16_map(&L->maps.m[1], wo, H, A) &&
-              encode_bf16_map(&L->maps.m[2], wgu, (uint64_t)E * 2 * I, H) &&
-              encode_bf16_map(&L->maps.m[3], wd, (uint64_t)E * H, I) &&
-              encode_bf16_map(&L->maps.m[6], wr, E, H);
+  {
+    bool ok = encode_weight_map(&L->maps.m[0], wqkv, Nqkv, H, fp8) &&
+              encode_weight_map(&L->maps.m[1], wo, H, A, fp8) &&
+              encode_weight_map(&L->maps.m[2], wgu, (uint64_t)E * 2 * I, H, fp8) &&
+              encode_weight_map(&L->maps.m[3], wd, (uint64_t)E * H, I, fp8) &&
+              encode_weight_map(&L->maps.m[6], wr, E, H, fp8);
     if (ok && c.n_shared)
-      ok = encode_bf16_map(&L->maps.m[4], wgu_sh, 2 * I, H) && encode_bf16_map(&L->maps.m[5], wd_sh, H, I);
+      ok = encode_weight_map(&L->maps.m[4], wgu_sh, 2 * I, H, fp8) &&
+           encode_weight_map(&L->maps.m[5], wd_sh, H, I, fp8);
     L->has_maps = ok;
   }
 
@@ -415,7 +422,7 @@ static int launch_layer(kd_layer* L, void* hidden, const void* attn, int M, cuda
   const size_t sm = kStreamSmem;
   const bool mma = L->has_maps && M >= L->mma_min;
   const size_t msm = kMmaSmem;
-  const size_t mroute = kMmaSmem + 16 + sizeof(int) * kRouteSmemInts(d.E, M * d.k);
+  const int mthreads = fp8 ? kMThreadsF8 : kMThreads;
   if (L->timing) KD_CUDA(cudaEventRecord(L->tev[0], s));
   // Main stream: projections -> router (logits, selection, token lists in one
   // launch) -> routed gate/up -> down + combine.  Side stream: the shared
@@ -425,15 +432,19 @@ static int launch_layer(kd_layer* L, void* hidden, const void* attn, int M, cuda
   // leaves free while the router runs.
   const size_t route_ints = sizeof(int) * kRouteSmemInts(d.E, M * d.k);
   if (mma)
-    KD_CUDA(launch(mma_proj_kernel, G, kMThreads, msm, s, pdl_first, d, a, L->maps));
+    KD_CUDA(launch(fp8 ? mma_proj_kernel<true> : mma_proj_kernel<false>, G, mthreads, msm, s,
+                   pdl_first, d, a, L->maps));
   else
     KD_CUDA(launch(fp8 ? proj_kernel<W_FP8> : proj_kernel<W_BF16>, G, kThreads, sm, s, pdl_first, d, a));
   if (L->timing) KD_CUDA(cudaEventRecord(L->tev[1], s));
   if (d.S) KD_CUDA(cudaEventRecord(L->ev_h1, s));
-  if (mma) {
-    const int rchunks = ((d.E + 127) / 128) * (d.H / (64 * mma_nsub(M, 3)));
-    const int rgrid = std::max(1, std::min(G, rchunks / kRouterChunksPerCta));
-    KD_CUDA(launch(mma_router_kernel, rgrid, kMThreads, mroute, s, !L->timing, d, M, L->maps));
+  // FP8 routers stay on CUDA cores: the tensor-core path rounds each scaled
+  // weight to bf16, which the fp32 router logits cannot afford
+  if (mma && !fp8) {
+    const int rsub = mma_nsub(M, 3);
+    const int rchunks = ((d.E + 127) / 128) * (d.H / (64 * rsub));
+    const int rgrid = std::max(1, std::min(G, rchunks / (kRouterChunksPerCta * 2 / rsub)));
+    KD_CUDA(launch(mma_router_kernel<false>, rgrid, mthreads, msm, s, !L->timing, d, M, L->maps));
   } else {
     const int rgrid = (d.E + kRouterRows - 1) / kRouterRows;
     KD_CUDA(launch(fp8 ? router_kernel<W_FP8> : router_kernel<W_BF16>, rgrid, kRouterThreads,
@@ -442,7 +453,8 @@ static int launch_layer(kd_layer* L, void* hidden, const void* attn, int M, cuda
   if (d.S) {
     KD_CUDA(cudaStreamWaitEvent(L->side, L->ev_h1, 0));
     if (mma)
-      KD_CUDA(launch(mma_gateup_kernel, G, kMThreads, msm, L->side, false, d, M, 1, L->maps));
+      KD_CUDA(launch(fp8 ? mma_gateup_kernel<true> : mma_gateup_kernel<false>, G, mthreads, msm,
+                     L->side, false, d, M, 1, L->maps));
     else
       KD_CUDA(launch(fp8 ? gateup_kernel<W_FP8> : gateup_kernel<W_BF16>, G, kThreads, sm, L->side,
                      false, d, M, 1));
@@ -450,7 +462,8 @@ static int launch_layer(kd_layer* L, void* hidden, const void* attn, int M, cuda
   }
   if (L->timing) KD_CUDA(cudaEventRecord(L->tev[2], s));
   if (mma)
-    KD_CUDA(launch(mma_gateup_kernel, G, kMThreads, mroute, s, !L->timing, d, M, 0, L->maps));
+    KD_CUDA(launch(fp8 ? mma_gateup_kernel<true> : mma_gateup_kernel<false>, G, mthreads, msm, s,
+                   !L->timing, d, M, 0, L->maps));
   else
     KD_CUDA(launch(fp8 ? gateup_kernel<W_FP8> : gateup_kernel<W_BF16>, G, kThreads,
                    gateup_smem(d, M), s, !L->timing, d, M, 0));
@@ -465,9 +478,12 @@ static int launch_layer(kd_layer* L, void* hidden, const void* attn, int M, cuda
     KD_CUDA(cudaEventRecord(ev_join, pf));
   }
   const bool pdl_down = !L->timing && !d.S && !(next && pf);
-  if (mma)
-    KD_CUDA(launch(mma_down_kernel, G, kMThreads, msm, s, pdl_down, d, M, a.out, L->maps));
-  else
+  if (mma) {
+    // tensor-core down writes each expert's outputs; the combine follows
+    KD_CUDA(launch(fp8 ? mma_down_kernel<true> : mma_down_kernel<false>, G, mthreads, msm, s,
+                   pdl_down, d, M, L->maps));
+    KD_CUDA(launch(combine_kernel, 2 * G, 256, 0, s, !L->timing, d, M, a.out));
+  } else
     KD_CUDA(launch(fp8 ? down_kernel<W_FP8> : down_kernel<W_BF16>, G, kThreads, sm, s, pdl_down, d,
                    M, a.out));
   if (L->timing) KD_CUDA(cudaEventRecord(L->tev[4], s));
@@ -606,6 +622,16 @@ extern "C" int kd_layer_read_weight(const kd_layer* L, int kind, int expert, int
                        cudaMemcpyDeviceToHost));
   }
   return KD_OK;
+}
+
+extern "C" int kd_layer_launches(const kd_layer* L, int M) {
+  if (!L) return fail(KD_EINVAL, "kd_layer_launches: null layer%s", "");
+  if (M < 1 || M > L->maxM)
+    return fail(KD_ERANGE, "kd_layer_launches: M=%s%ld outside 1..max_tokens", "", (long)M);
+  const bool mma = L->has_maps && M >= L->mma_min;
+  // projections, router, routed gate/up, down (+ combine on the tensor-core
+  // path), + the shared expert's gate/up
+  return 4 + (mma ? 1 : 0) + (L->d.S ? 1 : 0);
 }
 
 extern "C" int kd_layer_bytes(const kd_layer* L, uint64_t* static_bytes, uint64_t* expert_bytes) {

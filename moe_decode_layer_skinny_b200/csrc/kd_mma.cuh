@@ -97,10 +97,11 @@ KD_DEV void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "
 // ------------------------------------------------------------------ engine
 
 constexpr int kMThreads = 256;
+constexpr int kMThreadsF8 = 384;      // + 4 converter warps (e4m3 -> bf16 A tiles)
 constexpr int kMaxMStages = 16;
 constexpr int kATileBytes = 128 * 128;                // 128 rows x 64 bf16 (one swizzle atom wide)
 constexpr int kMaxSub = 2;                            // 64-K sub-tiles per stage (at most)
-constexpr int kMRingBytes = 3 * kMaxSub * (kATileBytes + 64 * 128 * 2);  // 192 KB of stages
+constexpr int kMRingBytes = 224 * 1024;                // stages (+ 2 KB below: 227 KB per CTA)
 constexpr int kMaxN = 64;                             // tokens per MMA (N)
 constexpr int kMaxTerms = 3;                          // bf16 terms of an activation
 constexpr size_t kWsFloatsPerCta = 2 * 128 * 64;     // split-K partial slots of one CTA
@@ -182,14 +183,19 @@ struct MmaShared {
   uint8_t* stage;        // nst x stage_bytes, 1024-aligned
   int nst, stage_bytes;  // stage count and size (A tile + B tile for the launch's largest N)
   int nsub;              // 64-K sub-tiles per stage
-  uint64_t* full;        // [nst] A landed (tx) + B written (64 thread arrivals)
+  uint64_t* full;        // [nst] A landed (tx, or the converter) + B written (64 arrivals)
   uint64_t* empty;       // [nst] MMAs of the stage done
   uint64_t* accfull;     // [2] accumulator buffer ready for the epilogue
   uint64_t* accempty;    // [2] epilogue done reading the accumulator
+  // FP8 weights: e4m3 tiles land in a ring of their own, the converter warps
+  // turn them into the stage's bf16 A tile
+  uint8_t* raw;          // nraw x kRawBytes
+  int nraw;
+  uint64_t* rfull;       // [nraw] e4m3 tile landed (tx)
+  uint64_t* rempty;      // [nraw] converted
   uint32_t* tmem_base;
   int* abort_flag;
-  int* misc;             // [8] epilogue scratch ([1] combine block count, [2] after-run flag)
-  int* blist;            // [128] combine block list
+  int* misc;             // [8] scratch ([0] split-K last part, [2] after-run flag)
 };
 
 // The ring holds as many stages as fit.  A stage covers nsub x 64 K: nsub
@@ -203,23 +209,38 @@ __host__ __device__ inline int mma_nsub(int nmax, int terms) {
   return kMRingBytes / (2 * (kATileBytes + b_sub_bytes(nmax, terms))) >= 4 ? 2 : 1;
 }
 
-KD_DEV MmaShared carve_mma_smem(uint8_t* raw, int nmax, int terms, int nsub) {
+// FP8 weights: one e4m3 tile [128 rows x 128 K] (one scale block) per stage;
+// the stages are double-buffered and the rest of the ring holds e4m3 tiles.
+constexpr int kRawBytes = 128 * 128;
+
+KD_DEV MmaShared carve_mma_smem(uint8_t* base, int nmax, int terms, int nsub, bool fp8,
+                                int aterms) {
   MmaShared s;
   s.nsub = nsub;
-  s.stage_bytes = nsub * (kATileBytes + b_sub_bytes(nmax, terms));
-  s.nst = kMRingBytes / s.stage_bytes;
-  if (s.nst > kMaxMStages) s.nst = kMaxMStages;
-  uintptr_t p = (reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023);
+  s.stage_bytes = nsub * (aterms * kATileBytes + b_sub_bytes(nmax, terms));
+  uintptr_t p = (reinterpret_cast<uintptr_t>(base) + 1023) & ~uintptr_t(1023);
   s.stage = reinterpret_cast<uint8_t*>(p);
+  if (fp8) {
+    s.nst = 2;
+    s.raw = s.stage + 2 * (size_t)s.stage_bytes;
+    s.nraw = (kMRingBytes - 2 * s.stage_bytes) / kRawBytes;
+    if (s.nraw > kMaxMStages) s.nraw = kMaxMStages;
+  } else {
+    s.nst = kMRingBytes / s.stage_bytes;
+    if (s.nst > kMaxMStages) s.nst = kMaxMStages;
+    s.raw = nullptr;
+    s.nraw = 0;
+  }
   p += (size_t)kMRingBytes;
   s.full = reinterpret_cast<uint64_t*>(p);
   s.empty = s.full + kMaxMStages;
-  s.accfull = s.empty + kMaxMStages;
+  s.rfull = s.empty + kMaxMStages;
+  s.rempty = s.rfull + kMaxMStages;
+  s.accfull = s.rempty + kMaxMStages;
   s.accempty = s.accfull + 2;
   s.tmem_base = reinterpret_cast<uint32_t*>(s.accempty + 2);
   s.abort_flag = reinterpret_cast<int*>(s.tmem_base + 1);
   s.misc = s.abort_flag + 1;
-  s.blist = s.misc + 8;
   return s;
 }
 
@@ -253,6 +274,8 @@ KD_DEV bool mwait_lazy(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
 //   int max_n(); int nsub
 //   const CUtensorMap* map(int id)
 //   static constexpr int kTerms    bf16 terms of B (1; 2 = hi + lo; 3 = hi + mid + lo)
+//   static constexpr bool kFp8     A arrives as e4m3 tiles (converter warps, a_scale)
+//   static constexpr int kATerms   bf16 terms of the converted A tile (1, or 2 = hi + lo)
 //   const uint16_t* b_base(const MUnit&, int h); int b_stride(const MUnit&);
 //   int b_rowidx(const MUnit&, int j)   token j's row of term h: base + rowidx * stride
 //   bool paired()                  rows are (gate, up) pairs
@@ -263,9 +286,35 @@ KD_DEV bool mwait_lazy(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
 //   void after_run(MmaShared&, uint8_t* smem)   all threads, after the pipeline
 
 template <class Plan>
+KD_DEV void mma_producer_a_bf16(const Plan& plan, MmaShared& sh, CtaUnits<Plan>& units,
+                                unsigned* err);
+
+template <class Plan>
 KD_DEV void mma_producer_a(const Plan& plan, MmaShared& sh, unsigned* err) {
   uint32_t it = 0;
   CtaUnits<Plan> units(plan);
+  MUnit m;
+  if constexpr (Plan::kFp8) {
+    // e4m3 tiles [128 rows x 128 K bytes] into the raw ring
+    while (units.next(m)) {
+      const CUtensorMap* map = plan.map(m.map);
+      for (int c = 0; c < m.nkc; ++c, ++it) {
+        const int s = it % sh.nraw;
+        const uint32_t ph = (it / sh.nraw) & 1u;
+        mwait(&sh.rempty[s], ph ^ 1u, sh.abort_flag, err);
+        mbar_arrive_expect_tx(&sh.rfull[s], kRawBytes);
+        tma_load_2d(sh.raw + (size_t)s * kRawBytes, map, (m.kc0 + c) * 128, m.row, &sh.rfull[s]);
+      }
+    }
+  } else {
+    mma_producer_a_bf16(plan, sh, units, err);
+  }
+}
+
+template <class Plan>
+KD_DEV void mma_producer_a_bf16(const Plan& plan, MmaShared& sh, CtaUnits<Plan>& units,
+                                unsigned* err) {
+  uint32_t it = 0;
   MUnit m;
   while (units.next(m)) {
     const CUtensorMap* map = plan.map(m.map);
@@ -336,7 +385,7 @@ KD_DEV void mma_producer_b(const Plan& plan, MmaShared& sh, unsigned* err) {
       const int s = it % sh.nst;
       const uint32_t ph = (it / sh.nst) & 1u;
       mwait(&sh.empty[s], ph ^ 1u, sh.abort_flag, err);
-      uint8_t* bt = sh.stage + (size_t)s * sh.stage_bytes + sh.nsub * kATileBytes + swz;
+      uint8_t* bt = sh.stage + (size_t)s * sh.stage_bytes + sh.nsub * Plan::kATerms * kATileBytes + swz;
       for (int u = 0; u < sh.nsub; ++u) {
         const int k0 = ((m.kc0 + c) * sh.nsub + u) * 64;
 #pragma unroll
@@ -353,6 +402,69 @@ KD_DEV void mma_producer_b(const Plan& plan, MmaShared& sh, unsigned* err) {
   }
   cp_async_commit();
   cp_async_wait<0>();   // nothing in flight when the warp leaves
+}
+
+// FP8 weights: warps 8-11 turn each e4m3 tile of the raw ring into the
+// stage's bf16 A tile (two [128 x 64] sub-tiles in the 128-byte swizzle),
+// multiplied by the tile's block scale (rows alternate gate/up scales when the
+// plan pairs them): v = bf16(decode(e4m3) * scale).  Thread t takes the
+// 16-byte chunks t, t + 128, ... of the 1024 in a tile (row = chunk / 8).
+template <class Plan>
+KD_DEV void mma_converter(const Plan& plan, MmaShared& sh, unsigned* err) {
+  const int ct = threadIdx.x - 256;
+  uint32_t it = 0;
+  CtaUnits<Plan> units(plan);
+  MUnit m;
+  while (units.next(m)) {
+    for (int c = 0; c < m.nkc; ++c, ++it) {
+      const int rs = it % sh.nraw, s = it % sh.nst;
+      mwait(&sh.rfull[rs], (it / sh.nraw) & 1u, sh.abort_flag, err);
+      mwait(&sh.empty[s], ((it / sh.nst) & 1u) ^ 1u, sh.abort_flag, err);
+      const float2 sc = plan.a_scale(m, m.kc0 + c);   // (even rows, odd rows)
+      const uint8_t* raw = sh.raw + (size_t)rs * kRawBytes;
+      uint8_t* dst = sh.stage + (size_t)s * sh.stage_bytes;
+#pragma unroll 1
+      for (int q = 0; q < 8; ++q) {
+        const int p = ct + 128 * q;
+        const int r = p >> 3, j = p & 7, sw = r & 7;
+        const uint4 w = *reinterpret_cast<const uint4*>(raw + r * 128 + ((j ^ sw) << 4));
+        const float f = (r & 1) ? sc.y : sc.x;
+        const uint32_t in[4] = {w.x, w.y, w.z, w.w};
+        float v[16];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          e4m3x4_to_f32(in[u], v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) v[4 * u + i] *= f;
+        }
+        // K bytes 16j .. 16j+15 -> bf16 sub-tile j/4, 16-byte chunks 2(j%4), 2(j%4)+1
+        const int j0 = 2 * (j & 3);
+#pragma unroll
+        for (int at = 0; at < Plan::kATerms; ++at) {
+          uint32_t out[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const uint16_t h0 = f32_to_bf16_bits(v[2 * i]), h1 = f32_to_bf16_bits(v[2 * i + 1]);
+            out[i] = (uint32_t)h0 | ((uint32_t)h1 << 16);
+            if (Plan::kATerms > 1) {   // what this term leaves for the next
+              v[2 * i] -= __uint_as_float((uint32_t)h0 << 16);
+              v[2 * i + 1] -= __uint_as_float((uint32_t)h1 << 16);
+            }
+          }
+          uint8_t* sub = dst + (at * 2 + (j >> 2)) * kATileBytes + r * 128;
+          *reinterpret_cast<uint4*>(sub + ((j0 ^ sw) << 4)) = make_uint4(out[0], out[1], out[2], out[3]);
+          *reinterpret_cast<uint4*>(sub + (((j0 + 1) ^ sw) << 4)) =
+              make_uint4(out[4], out[5], out[6], out[7]);
+        }
+      }
+      fence_proxy_async_smem();   // generic-proxy writes -> visible to the tensor core
+      named_bar_sync(3, 128);
+      if (ct == 0) {
+        mbar_arrive(&sh.rempty[rs]);
+        mbar_arrive(&sh.full[s]);
+      }
+    }
+  }
 }
 
 template <class Plan>
@@ -375,17 +487,20 @@ KD_DEV void mma_issuer(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigned*
       fence_proxy_async_smem();   // the B gathers (generic proxy) -> tensor core reads
       tc_fence_after();
       const uint32_t a0 = smem_u32(sh.stage + (size_t)s * sh.stage_bytes);
-      const uint32_t b0 = a0 + sh.nsub * kATileBytes;
+      const uint32_t b0 = a0 + sh.nsub * Plan::kATerms * kATileBytes;
       const int bsub = b_sub_bytes(N, nterms);
       for (int u = 0; u < sh.nsub; ++u) {
-        const uint32_t a = a0 + u * kATileBytes, b = b0 + u * bsub;
+        const uint32_t b = b0 + u * bsub;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const uint64_t ad = sw128_desc(a + k * 32);
-          mma_bf16(d, ad, sw128_desc(b + k * 32), idesc, c > 0 || u > 0 || k > 0);
 #pragma unroll
-          for (int h = 1; h < nterms; ++h)
-            mma_bf16(d, ad, sw128_desc(b + h * N * 128 + k * 32), idesc, true);
+          for (int at = 0; at < Plan::kATerms; ++at) {
+            const uint64_t ad = sw128_desc(a0 + (at * sh.nsub + u) * kATileBytes + k * 32);
+            mma_bf16(d, ad, sw128_desc(b + k * 32), idesc, c > 0 || u > 0 || k > 0 || at > 0);
+#pragma unroll
+            for (int h = 1; h < nterms; ++h)
+              mma_bf16(d, ad, sw128_desc(b + h * N * 128 + k * 32), idesc, true);
+          }
         }
       }
       mma_commit(&sh.empty[s]);   // the stage is free once these MMAs are done
@@ -502,12 +617,17 @@ KD_DEV void mma_epilogue(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigne
 
 template <class Plan>
 KD_DEV void mma_run(const Plan& plan, uint8_t* smem_raw, unsigned* err) {
-  MmaShared sh = carve_mma_smem(smem_raw, plan.max_n(), Plan::kTerms, plan.nsub);
+  MmaShared sh = carve_mma_smem(smem_raw, plan.max_n(), Plan::kTerms, plan.nsub, Plan::kFp8,
+                                Plan::kATerms);
   const int warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
     for (int i = 0; i < sh.nst; ++i) {
-      mbar_init(&sh.full[i], 1 + 64);  // A transaction arrive + the 64 B threads
+      mbar_init(&sh.full[i], 1 + 64);  // A (transaction arrive or converter) + the 64 B threads
       mbar_init(&sh.empty[i], 1);
+    }
+    for (int i = 0; i < sh.nraw; ++i) {
+      mbar_init(&sh.rfull[i], 1);
+      mbar_init(&sh.rempty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sh.accfull[i], 1);
@@ -528,8 +648,10 @@ KD_DEV void mma_run(const Plan& plan, uint8_t* smem_raw, unsigned* err) {
     if ((threadIdx.x & 31) == 0) mma_issuer(plan, sh, tmem, err);
   } else if (warp < 4) {
     mma_producer_b(plan, sh, err);
-  } else {
+  } else if (warp < 8) {
     mma_epilogue(plan, sh, tmem, err);
+  } else if constexpr (Plan::kFp8) {
+    mma_converter(plan, sh, err);
   }
   tc_fence_before();
   __syncthreads();

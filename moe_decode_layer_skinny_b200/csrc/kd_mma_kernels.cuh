@@ -4,7 +4,8 @@
 // kd_kernels.cuh; in addition the producers write the bf16 hi/lo pairs
 // (h1lo, act_hi/act_lo) that the next tensor-core kernel multiplies.
 //
-// Tensor maps (one per weight matrix, box 64 K x 128 rows, 128B swizzle):
+// Tensor maps (one per weight matrix, 128 rows x 128 bytes per box (64 bf16
+// or 128 e4m3 K values), 128B swizzle):
 //   0 Wqkv [Nqkv, H]   1 Wo [H, A]   2 routed gate/up [E*2I, H]
 //   3 routed down [E*H, I]   4 shared gate/up [2I, H]   5 shared down [H, I]
 //   6 router [E, H]
@@ -20,15 +21,16 @@ struct MmaMaps {
   CUtensorMap m[kNumMaps];
 };
 
-// Largest token count among the active experts (every thread gets it).
+// Largest token count among the active experts (every thread gets it; all
+// threads call).  Lists in global memory: one load round per thread.
 KD_DEV int max_tokens_per_expert(const int* cnt, const int* act, int n_act) {
   __shared__ int s_max;
-  if (threadIdx.x < 32) {
-    int m = 0;
-    for (int a = threadIdx.x; a < n_act; a += 32) m = max(m, cnt[act[a]]);
-    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if (threadIdx.x == 0) s_max = m;
-  }
+  if (threadIdx.x == 0) s_max = 0;
+  __syncthreads();
+  int m = 0;
+  for (int a = threadIdx.x; a < n_act; a += blockDim.x) m = max(m, cnt[act[a]]);
+  for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((threadIdx.x & 31) == 0) atomicMax(&s_max, m);
   __syncthreads();
   return s_max;
 }
@@ -52,7 +54,11 @@ KD_DEV void store_hilo3(uint16_t* hi, uint16_t* mid, uint16_t* lo, size_t o, flo
 
 // ------------------------------------------------------------------ QKV + o-proj
 
+template <bool F8>
 struct MmaProjPlan {
+  static constexpr bool kFp8 = F8;
+  // FP8: the scaled weights as bf16 hi + lo (h1 feeds the fp32 router)
+  static constexpr int kATerms = F8 ? 2 : 1;
   const LayerDev* L; Acts a; const MmaMaps* maps;
   int nsub;
   int tq, to, cq, co;   // tiles and K chunks per tile of QKV and o-proj
@@ -73,6 +79,11 @@ struct MmaProjPlan {
   KD_DEV const CUtensorMap* map(int id) const { return &maps->m[id]; }
   KD_DEV int max_n() const { return a.M; }
   static constexpr int kTerms = 1;
+  KD_DEV float2 a_scale(const MUnit& m, int kc) const {
+    const float sc = m.tag == 0 ? L->sqkv[(size_t)(m.row >> 7) * L->nHb + kc]
+                                : L->so[(size_t)(m.row >> 7) * L->nAb + kc];
+    return make_float2(sc, sc);
+  }
   KD_DEV const uint16_t* b_base(const MUnit& m, int) const { return m.tag == 0 ? a.x : a.attn; }
   KD_DEV int b_stride(const MUnit& m) const { return m.tag == 0 ? L->H : L->A; }
   KD_DEV int b_rowidx(const MUnit&, int j) const { return j; }
@@ -83,7 +94,8 @@ struct MmaProjPlan {
       L->qkv[(size_t)j * L->Nqkv + row] = f32_to_bf16_bits(v);
     } else {
       const size_t o = (size_t)j * L->H + row;
-      const float h = __uint_as_float((uint32_t)a.x[o] << 16) + v;
+      // read-only here (a plain load could not move above the stores below)
+      const float h = __uint_as_float((uint32_t)__ldg(a.x + o) << 16) + v;
       L->h1f[o] = h;
       store_hilo3(L->h1b, L->h1lo, L->h1lo2, o, h);
     }
@@ -96,12 +108,13 @@ struct MmaProjPlan {
   KD_DEV void after_run(MmaShared&, uint8_t*) const {}
 };
 
-__global__ void __launch_bounds__(kMThreads, 1) mma_proj_kernel(LayerDev L, Acts a,
-                                                                const __grid_constant__ MmaMaps maps) {
+template <bool F8>
+__global__ void __launch_bounds__(F8 ? kMThreadsF8 : kMThreads, 1)
+    mma_proj_kernel(LayerDev L, Acts a, const __grid_constant__ MmaMaps maps) {
   extern __shared__ uint8_t smem[];
-  MmaProjPlan p;
+  MmaProjPlan<F8> p;
   p.L = &L; p.a = a; p.maps = &maps;
-  p.nsub = mma_nsub(a.M, 1);
+  p.nsub = F8 ? 2 : mma_nsub(a.M, 1);
   p.tq = L.Nqkv / 128; p.to = L.H / 128; p.cq = L.H / (64 * p.nsub); p.co = L.A / (64 * p.nsub);
   pdl_wait();
   pdl_launch_dependents();
@@ -116,7 +129,10 @@ __global__ void __launch_bounds__(kMThreads, 1) mma_proj_kernel(LayerDev L, Acts
 // per CTA) to keep the split-K partial sums short.  The CTA that completes
 // the last tile then selects every token's experts (top-k, renormalised
 // softmax) and builds the per-expert token lists, all within this launch.
+template <bool F8>
 struct MmaRouterPlan {
+  static constexpr bool kFp8 = F8;
+  static constexpr int kATerms = 1;
   const LayerDev* L; int M; const MmaMaps* maps;
   int nsub;
   KD_DEV int num_tiles() const { return (L->E + 127) / 128; }
@@ -129,6 +145,10 @@ struct MmaRouterPlan {
   KD_DEV const CUtensorMap* map(int id) const { return &maps->m[id]; }
   KD_DEV int max_n() const { return M; }
   static constexpr int kTerms = 3;
+  KD_DEV float2 a_scale(const MUnit& m, int kc) const {
+    const float sc = L->sr[(size_t)(m.row >> 7) * L->nHb + kc];
+    return make_float2(sc, sc);
+  }
   KD_DEV const uint16_t* b_base(const MUnit&, int h) const {
     return h == 0 ? L->h1b : h == 1 ? L->h1lo : L->h1lo2;
   }
@@ -137,7 +157,7 @@ struct MmaRouterPlan {
   KD_DEV bool paired() const { return false; }
   KD_DEV void epilogue(const MUnit& m, int r, int j, float v) const {
     const int e = m.lrow + r;
-    if (e < L->E) L->logits[(size_t)j * L->E + e] = v + (L->bias ? L->bias[e] : 0.f);
+    if (e < L->E) L->logits[(size_t)j * L->E + e] = v + (L->bias ? __ldg(L->bias + e) : 0.f);
   }
   KD_DEV void epilogue2(const MUnit&, int, int, float, float) const {}
   KD_DEV float* ws() const { return L->ws_main; }
@@ -158,20 +178,52 @@ struct MmaRouterPlan {
   KD_DEV void after_run(MmaShared& sh, uint8_t* smem) const {
     if (!sh.misc[2]) return;
     __threadfence();
-    const Route R = carve_route(reinterpret_cast<int*>(smem + kMmaSmem), L->E, M * L->k);
-    route_tokens(*L, M, R, true);
+    // the logits into the (now idle) stage ring in one parallel pass, so that
+    // the per-token selections read shared memory
+    const float* lg = L->logits;
+    const int n = M * L->E;
+    // ring: [logits copy (if it fits)] [routing scratch]
+    const size_t lbytes = ((size_t)n * sizeof(float) + 255) & ~(size_t)255;
+    const size_t rbytes = sizeof(int) * kRouteSmemInts(L->E, M * L->k);
+    const bool copy = lbytes + rbytes <= (size_t)kMRingBytes && (n & 3) == 0;
+    if (copy) {
+      // 16-byte loads, eight in flight per thread (the copy is latency-bound)
+      float4* cp = reinterpret_cast<float4*>(sh.stage);
+      const float4* src = reinterpret_cast<const float4*>(L->logits);
+      const int n4 = n >> 2;
+      for (int i0 = 0; i0 < n4; i0 += 8 * (int)blockDim.x) {
+        float4 t[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int i = i0 + u * (int)blockDim.x + (int)threadIdx.x;
+          if (i < n4) t[u] = __ldcg(src + i);
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int i = i0 + u * (int)blockDim.x + (int)threadIdx.x;
+          if (i < n4) cp[i] = t[u];
+        }
+      }
+      __syncthreads();
+      lg = reinterpret_cast<const float*>(cp);
+    }
+    const Route R = carve_route(reinterpret_cast<int*>(sh.stage + (copy ? lbytes : 0)), L->E,
+                                M * L->k);
+    route_tokens(*L, lg, M, R, true);
   }
 };
 
-// K chunks each router CTA streams (sets the router launch's grid).
+// 128-K chunks each router CTA streams (sets the router launch's grid: more
+// CTAs stream faster, fewer leave fewer split-K partials to add up).
 constexpr int kRouterChunksPerCta = 8;
 
-__global__ void __launch_bounds__(kMThreads, 1) mma_router_kernel(LayerDev L, int M,
-                                                                  const __grid_constant__ MmaMaps maps) {
+template <bool F8>
+__global__ void __launch_bounds__(F8 ? kMThreadsF8 : kMThreads, 1)
+    mma_router_kernel(LayerDev L, int M, const __grid_constant__ MmaMaps maps) {
   extern __shared__ uint8_t smem[];
-  MmaRouterPlan p;
+  MmaRouterPlan<F8> p;
   p.L = &L; p.M = M; p.maps = &maps;
-  p.nsub = mma_nsub(M, 3);
+  p.nsub = F8 ? 2 : mma_nsub(M, 3);
   pdl_wait();
   mma_run(p, smem, L.err);
   pdl_launch_dependents();
@@ -182,7 +234,10 @@ __global__ void __launch_bounds__(kMThreads, 1) mma_router_kernel(LayerDev L, in
 // Routed: tiles of the active experts' interleaved gate/up rows (2I/128 per
 // expert); shared: the shared expert's (all M tokens; its own launch on the
 // side stream).  B = h1 as a bf16 hi/lo pair.
+template <bool F8>
 struct MmaGateUpPlan {
+  static constexpr bool kFp8 = F8;
+  static constexpr int kATerms = 1;
   const LayerDev* L; int M; bool shared; const MmaMaps* maps; Route rt; int n_act;
   int nsub, nmax;
   KD_DEV int tiles_per() const { return 2 * L->I / 128; }
@@ -204,6 +259,13 @@ struct MmaGateUpPlan {
   KD_DEV const CUtensorMap* map(int id) const { return &maps->m[id]; }
   KD_DEV int max_n() const { return nmax; }
   static constexpr int kTerms = 2;
+  // rows alternate gate / up: their own scale tables, logical row block tt / 2
+  KD_DEV float2 a_scale(const MUnit& m, int kc) const {
+    const int tt = m.lrow >> 7;
+    const float* base = shared ? L->sgu_sh : L->sgu + (size_t)m.tag * 2 * L->nIb * L->nHb;
+    const size_t o = (size_t)(tt >> 1) * L->nHb + kc;
+    return make_float2(base[o], base[(size_t)L->nIb * L->nHb + o]);
+  }
   KD_DEV const uint16_t* b_base(const MUnit&, int h) const { return h ? L->h1lo : L->h1b; }
   KD_DEV int b_stride(const MUnit&) const { return L->H; }
   KD_DEV int b_rowidx(const MUnit& m, int j) const {
@@ -231,44 +293,49 @@ struct MmaGateUpPlan {
   KD_DEV void after_run(MmaShared&, uint8_t*) const {}
 };
 
-__global__ void __launch_bounds__(kMThreads, 1) mma_gateup_kernel(LayerDev L, int M, int shared,
-                                                                  const __grid_constant__ MmaMaps maps) {
+template <bool F8>
+__global__ void __launch_bounds__(F8 ? kMThreadsF8 : kMThreads, 1)
+    mma_gateup_kernel(LayerDev L, int M, int shared, const __grid_constant__ MmaMaps maps) {
   extern __shared__ uint8_t smem[];
-  MmaGateUpPlan p;
+  MmaGateUpPlan<F8> p;
   p.L = &L; p.M = M; p.shared = shared != 0; p.maps = &maps; p.n_act = 1;
   p.nmax = M;
   if (!shared) {
     pdl_wait();
     pdl_launch_dependents();
-    p.rt = carve_route(reinterpret_cast<int*>(smem + kMmaSmem), L.E, M * L.k);
-    load_route(L, M, p.rt);
+    p.rt = global_route(L);   // as the router left it (read through L2)
     p.n_act = *p.rt.n_act;
     p.nmax = max_tokens_per_expert(p.rt.cnt, p.rt.act, p.n_act);
   }
-  p.nsub = mma_nsub(p.nmax, 2);
+  p.nsub = F8 ? 2 : mma_nsub(p.nmax, 2);
   mma_run(p, smem, L.err);
 }
 
 // ------------------------------------------------------------------ down + combine
 
-// Tiles of the down projections of the active experts and the shared expert
-// ("entries"), ordered by output row tile first: tile t is row tile
-// t / entries of entry t % entries, so the 64-row output blocks complete one
-// after another through the launch and their combines spread over the CTAs.
-// B = the SwiGLU activations as a bf16 hi/lo pair.  A CTA that completes a
-// tile counts its 128 rows into the 64-row blocks; the CTA completing a block
-// (every entry) writes that block of the layer output.
+// Tiles of the active experts' down projections (H/128 per expert), then the
+// shared expert's, its M tokens cut into groups of at most shchunk (the
+// routed experts' largest token count, rounded up to 16) so that its B tiles
+// are no wider than the routed ones: a wide B tile would shrink every stage's
+// share of weights in the ring.  B = the SwiGLU activations as a bf16 hi/lo
+// pair.  The epilogue writes each expert's rows of its tokens' outputs (yr,
+// ysh); the gate-weighted combine into the layer output is the next launch.
+template <bool F8>
 struct MmaDownPlan {
-  const LayerDev* L; int M; int n_act; const MmaMaps* maps; uint16_t* out;
-  int nsub, nmax;
+  static constexpr bool kFp8 = F8;
+  static constexpr int kATerms = 1;
+  const LayerDev* L; int M; int n_act; const MmaMaps* maps;
+  int nsub, nmax, shchunk, nsh;
   KD_DEV int tiles_per() const { return L->H / 128; }
-  KD_DEV int num_tiles() const { return (n_act + L->S) * tiles_per(); }
+  KD_DEV int num_tiles() const { return (n_act + nsh) * tiles_per(); }
   KD_DEV long long tile_start(int t) const { return (long long)t * (L->I / (64 * nsub)); }
   KD_DEV MUnit tile_unit(int t) const {
     MUnit m{};
-    const int a = t % (n_act + L->S), tt = t / (n_act + L->S);
+    const int a = t / tiles_per(), tt = t % tiles_per();
     if (a >= n_act) {
-      m.map = 5; m.row = tt * 128; m.tag = -1; m.tok0 = 0; m.ntok = M;
+      const int q = a - n_act;
+      m.map = 5; m.row = tt * 128; m.tag = -1;
+      m.tok0 = q * shchunk; m.ntok = min(shchunk, M - m.tok0);
     } else {
       const int e = L->active[a];
       m.map = 3; m.row = e * L->H + tt * 128; m.tag = e;
@@ -280,70 +347,84 @@ struct MmaDownPlan {
   KD_DEV const CUtensorMap* map(int id) const { return &maps->m[id]; }
   KD_DEV int max_n() const { return nmax; }
   static constexpr int kTerms = 2;
+  KD_DEV float2 a_scale(const MUnit& m, int kc) const {
+    const float* base = m.tag < 0 ? L->sd_sh : L->sd + (size_t)m.tag * L->nHb * L->nIb;
+    const float sc = base[(size_t)(m.lrow >> 7) * L->nIb + kc];
+    return make_float2(sc, sc);
+  }
   KD_DEV const uint16_t* b_base(const MUnit& m, int h) const {
     if (m.tag < 0) return h ? L->act_sh_lo : L->act_sh_hi;
     return h ? L->act_lo : L->act_hi;
   }
   KD_DEV int b_stride(const MUnit&) const { return L->I; }
-  KD_DEV int b_rowidx(const MUnit& m, int j) const { return m.tag < 0 ? j : m.tok0 + j; }
+  KD_DEV int b_rowidx(const MUnit& m, int j) const { return m.tok0 + j; }
   KD_DEV bool paired() const { return false; }
   KD_DEV void epilogue(const MUnit& m, int r, int j, float v) const {
     const int h = m.lrow + r;
-    if (m.tag < 0) L->ysh[(size_t)j * L->H + h] = v;
-    else L->yr[(size_t)L->perm[m.tok0 + j] * L->H + h] = v;
+    if (m.tag < 0) L->ysh[(size_t)(m.tok0 + j) * L->H + h] = v;
+    else L->yr[(size_t)__ldg(L->perm + m.tok0 + j) * L->H + h] = v;
   }
   KD_DEV void epilogue2(const MUnit&, int, int, float, float) const {}
   KD_DEV float* ws() const { return L->ws_main; }
   KD_DEV unsigned* tile_cnt() const { return L->tcnt_main; }
-  KD_DEV bool wants_unit_done() const { return true; }
+  KD_DEV bool wants_unit_done() const { return false; }
+  KD_DEV void unit_done(const MUnit&, MmaShared&) const {}
   KD_DEV void after_run(MmaShared&, uint8_t*) const {}
-  // epilogue warps only (128 threads, named barrier 2)
-  KD_DEV void unit_done(const MUnit& m, MmaShared& sh) const {
-    const int target = 64 * (n_act + L->S);
-    const int et = threadIdx.x - 128;
-    if (et == 0) {
-      __threadfence();
-      int nb = 0;
-      for (int b = m.lrow / 64; b < (m.lrow + 128) / 64; ++b) {
-        const unsigned prev = atomicAdd(L->hcnt + b, 64u);
-        if (prev + 64u == (unsigned)target) {
-          L->hcnt[b] = 0u;
-          sh.blist[nb++] = b;
-        }
-      }
-      sh.misc[1] = nb;
-      __threadfence();
-    }
-    named_bar_sync(2, 128);
-    const int nb = sh.misc[1];
-    for (int q = 0; q < nb; ++q) {
-      const int b = sh.blist[q];
-      for (int e = et; e < 64 * M; e += 128) {
-        const int t = e / 64, h = b * 64 + e % 64;
-        const size_t o = (size_t)t * L->H + h;
-        float v = L->h1f[o];
-        if (L->S) v += __ldcg(L->ysh + o);
-        for (int j = 0; j < L->k; ++j)
-          v += L->gates[t * L->k + j] * __ldcg(L->yr + ((size_t)t * L->k + j) * L->H + h);
-        out[o] = f32_to_bf16_bits(v);
-      }
-    }
-    named_bar_sync(2, 128);
-  }
 };
 
-__global__ void __launch_bounds__(kMThreads, 1) mma_down_kernel(LayerDev L, int M, uint16_t* out,
-                                                                const __grid_constant__ MmaMaps maps) {
+template <bool F8>
+__global__ void __launch_bounds__(F8 ? kMThreadsF8 : kMThreads, 1)
+    mma_down_kernel(LayerDev L, int M, const __grid_constant__ MmaMaps maps) {
   extern __shared__ uint8_t smem[];
   pdl_wait();
   pdl_launch_dependents();
-  MmaDownPlan p;
-  p.L = &L; p.M = M; p.out = out; p.maps = &maps;
+  MmaDownPlan<F8> p;
+  p.L = &L; p.M = M; p.maps = &maps;
   p.n_act = *(volatile int*)L.n_active;
   p.nmax = max_tokens_per_expert(L.counts, L.active, p.n_act);
-  if (L.S && M > p.nmax) p.nmax = M;
-  p.nsub = mma_nsub(p.nmax, 2);
+  p.shchunk = M;
+  p.nsh = 0;
+  if (L.S) {
+    p.shchunk = min(M, max(16, pad16(p.nmax)));
+    p.nsh = (M + p.shchunk - 1) / p.shchunk;
+    p.nmax = max(p.nmax, p.shchunk);
+  }
+  p.nsub = F8 ? 2 : mma_nsub(p.nmax, 2);
   mma_run(p, smem, L.err);
+}
+
+}  // namespace kd
+
+namespace kd {
+
+// ------------------------------------------------------------------ combine
+
+// out = bf16(h1 + shared expert + sum_j gate_j * routed expert j), token-major,
+// two outputs per thread per step.  The expert outputs were written by the
+// down launch that precedes this one.
+__global__ void __launch_bounds__(256) combine_kernel(LayerDev L, int M, uint16_t* out) {
+  pdl_wait();
+  const int H2 = L.H / 2, k = L.k;
+  const int n = M * H2;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+    const int t = i / H2, h = 2 * (i - t * H2);
+    const size_t o = (size_t)t * L.H + h;
+    float2 v = __ldcg(reinterpret_cast<const float2*>(L.h1f + o));
+    if (L.S) {
+      const float2 y = __ldcg(reinterpret_cast<const float2*>(L.ysh + o));
+      v.x += y.x;
+      v.y += y.y;
+    }
+    for (int j = 0; j < k; ++j) {
+      const float g = __ldcg(L.gates + t * k + j);
+      const float2 y = __ldcg(reinterpret_cast<const float2*>(L.yr + ((size_t)t * k + j) * L.H + h));
+      v.x += g * y.x;
+      v.y += g * y.y;
+    }
+    const uint32_t pair = (uint32_t)f32_to_bf16_bits(v.x) | ((uint32_t)f32_to_bf16_bits(v.y) << 16);
+    *reinterpret_cast<uint32_t*>(out + o) = pair;
+  }
+  pdl_launch_dependents();
 }
 
 }  // namespace kd

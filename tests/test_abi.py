@@ -60,6 +60,7 @@ def test_host_side_argument_errors(kd):
     assert L.kd_layer_check(None) == kd.KD_EINVAL
     assert L.kd_layer_qkv(None) is None
     assert L.kd_layer_bytes(None, None, None) == kd.KD_EINVAL
+    assert L.kd_layer_launches(None, 1) == kd.KD_EINVAL
     assert L.kd_layer_prefetch_l2(None, 0, None) == kd.KD_EINVAL
     assert L.kd_layer_set_timing_events(None, None, 0) == kd.KD_EINVAL
     assert L.kd_stack_create(None, 0, 1, 0, ctypes.byref(h)) == kd.KD_EINVAL
