@@ -187,6 +187,12 @@ struct MmaShared {
   uint64_t* empty;       // [nst] MMAs of the stage done
   uint64_t* accfull;     // [2] accumulator buffer ready for the epilogue
   uint64_t* accempty;    // [2] epilogue done reading the accumulator
+  // B tiles: inside the stages (bf16 weights; bst = stage, boff = the A
+  // bytes, bfull / bempty = full / empty) or a ring of their own (FP8)
+  uint8_t* bst;
+  int nbst, bst_bytes, boff;
+  uint64_t* bfull;       // [nbst] B written (64 thread arrivals)
+  uint64_t* bempty;      // [nbst] MMAs done with it
   // FP8 weights: e4m3 tiles land in a ring of their own, the converter warps
   // turn them into the stage's bf16 A tile
   uint8_t* raw;          // nraw x kRawBytes
@@ -209,34 +215,53 @@ __host__ __device__ inline int mma_nsub(int nmax, int terms) {
   return kMRingBytes / (2 * (kATileBytes + b_sub_bytes(nmax, terms))) >= 4 ? 2 : 1;
 }
 
-// FP8 weights: one e4m3 tile [128 rows x 128 K] (one scale block) per stage;
-// the stages are double-buffered and the rest of the ring holds e4m3 tiles.
+// FP8 weights: one e4m3 tile [128 rows x 128 K] (one scale block) per stage.
+// The converted A stages are double-buffered; B tiles get a ring of their own
+// (2-8 deep, up to half of what is left) so that the gathers run ahead; the
+// rest holds e4m3 tiles.
 constexpr int kRawBytes = 128 * 128;
 
 KD_DEV MmaShared carve_mma_smem(uint8_t* base, int nmax, int terms, int nsub, bool fp8,
                                 int aterms) {
   MmaShared s;
   s.nsub = nsub;
-  s.stage_bytes = nsub * (aterms * kATileBytes + b_sub_bytes(nmax, terms));
+  s.stage_bytes = nsub * (aterms * kATileBytes + b_sub_bytes(nmax, terms));   // bf16: A + B
   uintptr_t p = (reinterpret_cast<uintptr_t>(base) + 1023) & ~uintptr_t(1023);
   s.stage = reinterpret_cast<uint8_t*>(p);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(p + (size_t)kMRingBytes);
+  s.full = bars;
+  s.empty = s.full + kMaxMStages;
+  s.rfull = s.empty + kMaxMStages;
+  s.rempty = s.rfull + kMaxMStages;
   if (fp8) {
+    s.stage_bytes = nsub * aterms * kATileBytes;
     s.nst = 2;
-    s.raw = s.stage + 2 * (size_t)s.stage_bytes;
-    s.nraw = (kMRingBytes - 2 * s.stage_bytes) / kRawBytes;
+    const int bstage = nsub * b_sub_bytes(nmax, terms);
+    const int rem = kMRingBytes - 2 * s.stage_bytes;
+    int nb = bstage > 0 ? rem / 2 / bstage : 2;
+    nb = nb < 2 ? 2 : (nb > 8 ? 8 : nb);
+    s.bst = s.stage + 2 * (size_t)s.stage_bytes;
+    s.nbst = nb;
+    s.bst_bytes = bstage;
+    s.boff = 0;
+    s.bfull = s.rempty + kMaxMStages;
+    s.bempty = s.bfull + kMaxMStages;
+    s.raw = s.bst + (size_t)nb * bstage;
+    s.nraw = (rem - nb * bstage) / kRawBytes;
     if (s.nraw > kMaxMStages) s.nraw = kMaxMStages;
   } else {
     s.nst = kMRingBytes / s.stage_bytes;
     if (s.nst > kMaxMStages) s.nst = kMaxMStages;
+    s.bst = s.stage;
+    s.nbst = s.nst;
+    s.bst_bytes = s.stage_bytes;
+    s.boff = nsub * aterms * kATileBytes;
+    s.bfull = s.full;
+    s.bempty = s.empty;
     s.raw = nullptr;
     s.nraw = 0;
   }
-  p += (size_t)kMRingBytes;
-  s.full = reinterpret_cast<uint64_t*>(p);
-  s.empty = s.full + kMaxMStages;
-  s.rfull = s.empty + kMaxMStages;
-  s.rempty = s.rfull + kMaxMStages;
-  s.accfull = s.rempty + kMaxMStages;
+  s.accfull = s.rempty + 3 * kMaxMStages;
   s.accempty = s.accfull + 2;
   s.tmem_base = reinterpret_cast<uint32_t*>(s.accempty + 2);
   s.abort_flag = reinterpret_cast<int*>(s.tmem_base + 1);
@@ -382,10 +407,10 @@ KD_DEV void mma_producer_b(const Plan& plan, MmaShared& sh, unsigned* err) {
     }
     const int bsub = b_sub_bytes(N, nh);
     for (int c = 0; c < m.nkc; ++c, ++it) {
-      const int s = it % sh.nst;
-      const uint32_t ph = (it / sh.nst) & 1u;
-      mwait(&sh.empty[s], ph ^ 1u, sh.abort_flag, err);
-      uint8_t* bt = sh.stage + (size_t)s * sh.stage_bytes + sh.nsub * Plan::kATerms * kATileBytes + swz;
+      const int s = it % sh.nbst;
+      const uint32_t ph = (it / sh.nbst) & 1u;
+      mwait(&sh.bempty[s], ph ^ 1u, sh.abort_flag, err);
+      uint8_t* bt = sh.bst + (size_t)s * sh.bst_bytes + sh.boff + swz;
       for (int u = 0; u < sh.nsub; ++u) {
         const int k0 = ((m.kc0 + c) * sh.nsub + u) * 64;
 #pragma unroll
@@ -397,7 +422,7 @@ KD_DEV void mma_producer_b(const Plan& plan, MmaShared& sh, unsigned* err) {
           }
         }
       }
-      cp_async_arrive_noinc(&sh.full[s]);
+      cp_async_arrive_noinc(&sh.bfull[s]);
     }
   }
   cp_async_commit();
@@ -423,8 +448,8 @@ KD_DEV void mma_converter(const Plan& plan, MmaShared& sh, unsigned* err) {
       const float2 sc = plan.a_scale(m, m.kc0 + c);   // (even rows, odd rows)
       const uint8_t* raw = sh.raw + (size_t)rs * kRawBytes;
       uint8_t* dst = sh.stage + (size_t)s * sh.stage_bytes;
-#pragma unroll 1
-      for (int q = 0; q < 8; ++q) {
+#pragma unroll 4
+      for (int q = 0; q < 8; ++q) {   // unrolled: independent chunks overlap their latencies
         const int p = ct + 128 * q;
         const int r = p >> 3, j = p & 7, sw = r & 7;
         const uint4 w = *reinterpret_cast<const uint4*>(raw + r * 128 + ((j ^ sw) << 4));
@@ -444,11 +469,11 @@ KD_DEV void mma_converter(const Plan& plan, MmaShared& sh, unsigned* err) {
           uint32_t out[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            const uint16_t h0 = f32_to_bf16_bits(v[2 * i]), h1 = f32_to_bf16_bits(v[2 * i + 1]);
-            out[i] = (uint32_t)h0 | ((uint32_t)h1 << 16);
+            const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);   // one cvt
+            out[i] = *reinterpret_cast<const uint32_t*>(&h);
             if (Plan::kATerms > 1) {   // what this term leaves for the next
-              v[2 * i] -= __uint_as_float((uint32_t)h0 << 16);
-              v[2 * i + 1] -= __uint_as_float((uint32_t)h1 << 16);
+              v[2 * i] -= __low2float(h);
+              v[2 * i + 1] -= __high2float(h);
             }
           }
           uint8_t* sub = dst + (at * 2 + (j >> 2)) * kATileBytes + r * 128;
@@ -484,10 +509,12 @@ KD_DEV void mma_issuer(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigned*
       const int s = it % sh.nst;
       const uint32_t ph = (it / sh.nst) & 1u;
       mwait(&sh.full[s], ph, sh.abort_flag, err);
+      const int sb = it % sh.nbst;
+      if (Plan::kFp8) mwait(&sh.bfull[sb], (it / sh.nbst) & 1u, sh.abort_flag, err);
       fence_proxy_async_smem();   // the B gathers (generic proxy) -> tensor core reads
       tc_fence_after();
       const uint32_t a0 = smem_u32(sh.stage + (size_t)s * sh.stage_bytes);
-      const uint32_t b0 = a0 + sh.nsub * Plan::kATerms * kATileBytes;
+      const uint32_t b0 = smem_u32(sh.bst + (size_t)sb * sh.bst_bytes) + sh.boff;
       const int bsub = b_sub_bytes(N, nterms);
       for (int u = 0; u < sh.nsub; ++u) {
         const uint32_t b = b0 + u * bsub;
@@ -504,6 +531,7 @@ KD_DEV void mma_issuer(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigned*
         }
       }
       mma_commit(&sh.empty[s]);   // the stage is free once these MMAs are done
+      if (Plan::kFp8) mma_commit(&sh.bempty[sb]);
     }
     mma_commit(&sh.accfull[buf]);
   }
@@ -622,8 +650,15 @@ KD_DEV void mma_run(const Plan& plan, uint8_t* smem_raw, unsigned* err) {
   const int warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
     for (int i = 0; i < sh.nst; ++i) {
-      mbar_init(&sh.full[i], 1 + 64);  // A (transaction arrive or converter) + the 64 B threads
+      // A (transaction arrive, or the converter) + the 64 B threads unless B has its own ring
+      mbar_init(&sh.full[i], Plan::kFp8 ? 1 : 1 + 64);
       mbar_init(&sh.empty[i], 1);
+    }
+    if (Plan::kFp8) {
+      for (int i = 0; i < sh.nbst; ++i) {
+        mbar_init(&sh.bfull[i], 64);
+        mbar_init(&sh.bempty[i], 1);
+      }
     }
     for (int i = 0; i < sh.nraw; ++i) {
       mbar_init(&sh.rfull[i], 1);
