@@ -97,7 +97,7 @@ KD_DEV void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "
 // ------------------------------------------------------------------ engine
 
 constexpr int kMThreads = 256;
-constexpr int kMThreadsF8 = 384;      // + 4 converter warps (e4m3 -> bf16 A tiles)
+constexpr int kMThreadsF8 = 512;      // + 8 converter warps (e4m3 -> bf16 A tiles)
 constexpr int kMaxMStages = 16;
 constexpr int kATileBytes = 128 * 128;                // 128 rows x 64 bf16 (one swizzle atom wide)
 constexpr int kMaxSub = 2;                            // 64-K sub-tiles per stage (at most)
@@ -216,9 +216,9 @@ __host__ __device__ inline int mma_nsub(int nmax, int terms) {
 }
 
 // FP8 weights: one e4m3 tile [128 rows x 128 K] (one scale block) per stage.
-// The converted A stages are double-buffered; B tiles get a ring of their own
-// (2-8 deep, up to half of what is left) so that the gathers run ahead; the
-// rest holds e4m3 tiles.
+// Two or three converted A stages; B tiles get a ring of their own (2-4 deep,
+// up to a third of what is left) so that the gathers run ahead; the rest
+// holds e4m3 tiles.
 constexpr int kRawBytes = 128 * 128;
 
 KD_DEV MmaShared carve_mma_smem(uint8_t* base, int nmax, int terms, int nsub, bool fp8,
@@ -235,12 +235,14 @@ KD_DEV MmaShared carve_mma_smem(uint8_t* base, int nmax, int terms, int nsub, bo
   s.rempty = s.rfull + kMaxMStages;
   if (fp8) {
     s.stage_bytes = nsub * aterms * kATileBytes;
-    s.nst = 2;
+    // three converted stages hide the MMA's completion latency (two hi + lo
+    // stages, which are twice the size)
+    s.nst = aterms == 1 ? 3 : 2;
     const int bstage = nsub * b_sub_bytes(nmax, terms);
-    const int rem = kMRingBytes - 2 * s.stage_bytes;
-    int nb = bstage > 0 ? rem / 2 / bstage : 2;
-    nb = nb < 2 ? 2 : (nb > 8 ? 8 : nb);
-    s.bst = s.stage + 2 * (size_t)s.stage_bytes;
+    const int rem = kMRingBytes - s.nst * s.stage_bytes;
+    int nb = bstage > 0 ? rem / 3 / bstage : 2;
+    nb = nb < 2 ? 2 : (nb > 4 ? 4 : nb);
+    s.bst = s.stage + (size_t)s.nst * s.stage_bytes;
     s.nbst = nb;
     s.bst_bytes = bstage;
     s.boff = 0;
@@ -429,11 +431,12 @@ KD_DEV void mma_producer_b(const Plan& plan, MmaShared& sh, unsigned* err) {
   cp_async_wait<0>();   // nothing in flight when the warp leaves
 }
 
-// FP8 weights: warps 8-11 turn each e4m3 tile of the raw ring into the
+// FP8 weights: warps 8-15 turn each e4m3 tile of the raw ring into the
 // stage's bf16 A tile (two [128 x 64] sub-tiles in the 128-byte swizzle),
 // multiplied by the tile's block scale (rows alternate gate/up scales when the
-// plan pairs them): v = bf16(decode(e4m3) * scale).  Thread t takes the
-// 16-byte chunks t, t + 128, ... of the 1024 in a tile (row = chunk / 8).
+// plan pairs them): v = bf16(decode(e4m3) * scale), or a bf16 hi + lo pair.
+// Thread t takes the 16-byte chunks t, t + 256, ... of the 1024 in a tile
+// (row = chunk / 8).
 template <class Plan>
 KD_DEV void mma_converter(const Plan& plan, MmaShared& sh, unsigned* err) {
   const int ct = threadIdx.x - 256;
@@ -449,8 +452,8 @@ KD_DEV void mma_converter(const Plan& plan, MmaShared& sh, unsigned* err) {
       const uint8_t* raw = sh.raw + (size_t)rs * kRawBytes;
       uint8_t* dst = sh.stage + (size_t)s * sh.stage_bytes;
 #pragma unroll 4
-      for (int q = 0; q < 8; ++q) {   // unrolled: independent chunks overlap their latencies
-        const int p = ct + 128 * q;
+      for (int q = 0; q < 4; ++q) {   // unrolled: independent chunks overlap their latencies
+        const int p = ct + 256 * q;
         const int r = p >> 3, j = p & 7, sw = r & 7;
         const uint4 w = *reinterpret_cast<const uint4*>(raw + r * 128 + ((j ^ sw) << 4));
         const float f = (r & 1) ? sc.y : sc.x;
@@ -483,7 +486,7 @@ KD_DEV void mma_converter(const Plan& plan, MmaShared& sh, unsigned* err) {
         }
       }
       fence_proxy_async_smem();   // generic-proxy writes -> visible to the tensor core
-      named_bar_sync(3, 128);
+      named_bar_sync(3, 256);
       if (ct == 0) {
         mbar_arrive(&sh.rempty[rs]);
         mbar_arrive(&sh.full[s]);

@@ -140,6 +140,13 @@ def test_error_paths(kd):
         assert kd.lib().kd_decode_layer(L.handle, None, a.data_ptr(), 1, None) == kd.KD_EINVAL
         L.decode(h, a, 4)
         L.check()
+        # launches per call: CUDA-core path below 4 tokens, tensor-core path
+        # (+ the combine launch) from 4; + the shared expert's gate/up
+        assert L.launches(1) == 5 and L.launches(3) == 5
+        assert L.launches(4) == 6
+        with pytest.raises(kd.KdError) as ei:
+            L.launches(5)
+        assert ei.value.code == kd.KD_ERANGE
     finally:
         L.close()
 
