@@ -519,19 +519,37 @@ KD_DEV void mma_issuer(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigned*
       const uint32_t a0 = smem_u32(sh.stage + (size_t)s * sh.stage_bytes);
       const uint32_t b0 = smem_u32(sh.bst + (size_t)sb * sh.bst_bytes) + sh.boff;
       const int bsub = b_sub_bytes(N, nterms);
-      for (int u = 0; u < sh.nsub; ++u) {
-        const uint32_t b = b0 + u * bsub;
+      if constexpr (!Plan::kFp8) {
+        for (int u = 0; u < sh.nsub; ++u) {
+          const uint32_t b = b0 + u * bsub;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-#pragma unroll
-          for (int at = 0; at < Plan::kATerms; ++at) {
-            const uint64_t ad = sw128_desc(a0 + (at * sh.nsub + u) * kATileBytes + k * 32);
-            mma_bf16(d, ad, sw128_desc(b + k * 32), idesc, c > 0 || u > 0 || k > 0 || at > 0);
+          for (int k = 0; k < 4; ++k) {
+            const uint64_t ad = sw128_desc(a0 + u * kATileBytes + k * 32);
+            mma_bf16(d, ad, sw128_desc(b + k * 32), idesc, c > 0 || u > 0 || k > 0);
 #pragma unroll
             for (int h = 1; h < nterms; ++h)
               mma_bf16(d, ad, sw128_desc(b + h * N * 128 + k * 32), idesc, true);
           }
         }
+      } else {
+      // FP8: descriptors by adding byte offsets / 16 to the start-address
+      // field (shared addresses < 256 KB: the field never carries); the
+      // issuing thread shares its SM quarter with two converter warps
+      const uint64_t ad0 = sw128_desc(a0), bd0 = sw128_desc(b0);
+      for (int u = 0; u < sh.nsub; ++u) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint64_t bd = bd0 + (uint64_t)((u * bsub + k * 32) >> 4);
+#pragma unroll
+          for (int at = 0; at < Plan::kATerms; ++at) {
+            const uint64_t ad = ad0 + (uint64_t)(((at * sh.nsub + u) * kATileBytes + k * 32) >> 4);
+            mma_bf16(d, ad, bd, idesc, c > 0 || u > 0 || k > 0 || at > 0);
+#pragma unroll
+            for (int h = 1; h < nterms; ++h)
+              mma_bf16(d, ad, bd + (uint64_t)((h * N * 128) >> 4), idesc, true);
+          }
+        }
+      }
       }
       mma_commit(&sh.empty[s]);   // the stage is free once these MMAs are done
       if (Plan::kFp8) mma_commit(&sh.bempty[sb]);

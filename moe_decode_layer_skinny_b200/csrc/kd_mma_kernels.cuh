@@ -258,7 +258,9 @@ struct MmaGateUpPlan {
   }
   KD_DEV const CUtensorMap* map(int id) const { return &maps->m[id]; }
   KD_DEV int max_n() const { return nmax; }
-  static constexpr int kTerms = 2;
+  // bf16 hi + lo activations; with FP8 weights (3e-2 tolerance) the hi term
+  // alone, which halves the MMAs per weight byte
+  static constexpr int kTerms = F8 ? 1 : 2;
   // rows alternate gate / up: their own scale tables, logical row block tt / 2
   KD_DEV float2 a_scale(const MUnit& m, int kc) const {
     const int tt = m.lrow >> 7;
@@ -346,7 +348,9 @@ struct MmaDownPlan {
   }
   KD_DEV const CUtensorMap* map(int id) const { return &maps->m[id]; }
   KD_DEV int max_n() const { return nmax; }
-  static constexpr int kTerms = 2;
+  // bf16 hi + lo activations; with FP8 weights (3e-2 tolerance) the hi term
+  // alone, which halves the MMAs per weight byte
+  static constexpr int kTerms = F8 ? 1 : 2;
   KD_DEV float2 a_scale(const MUnit& m, int kc) const {
     const float* base = m.tag < 0 ? L->sd_sh : L->sd + (size_t)m.tag * L->nHb * L->nIb;
     const float sc = base[(size_t)(m.lrow >> 7) * L->nIb + kc];
