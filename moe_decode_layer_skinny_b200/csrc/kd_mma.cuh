@@ -5,18 +5,20 @@
 // tokens are its N (padded to a multiple of 16), so one kind::f16 MMA of
 // 128 x N x 16 consumes 4 KB of weights.  Per CTA (one per SM), warp roles:
 //   warp 0      TMA producer: 2-D tiled loads (128B swizzle) of the weight tile
-//               [128 rows x 64 K] into a ring of stages
+//               (one or two [128 rows x 64 K] boxes per stage) into a ring
 //   warp 1      MMA issuer: owns the TMEM accumulators (two buffers of N fp32
 //               columns), issues tcgen05.mma, commits stage releases
 //   warps 2-3   B producers: gather the tokens' bf16 rows (64 K at a time)
 //               into the stage in the same swizzled K-major layout
 //   warps 4-7   epilogue: tcgen05.ld of the accumulator (lane = weight row),
 //               then the plan's epilogue, or a split-K partial
+//   warps 8-15  FP8 weights only: e4m3 tiles -> scaled bf16 A tiles
 // Activations that must stay fp32-accurate come as a sum of bf16 terms, all
 // multiplied into the same accumulator: the expert inputs (h1, the SwiGLU
 // activations) as hi + lo (hi = bf16(v), lo = bf16(v - hi): ~16 significant
-// bits); the router's h1 as hi + mid + lo (all 24 bits of the fp32 value; the
-// products with bf16 weights are exact in the fp32 accumulator).
+// bits; hi alone with FP8 weights); the router's h1 as hi + mid + lo (all 24
+// bits of the fp32 value; the products with bf16 weights are exact in the
+// fp32 accumulator).
 // Work units are (weight tile, K part); a tile split over several parts is
 // summed in part order by the unit that completes it (deterministic).
 #pragma once

@@ -1,8 +1,10 @@
 // kd_mma_kernels.cuh -- the layer's projections on the tensor-core engine
 // (kd_mma.cuh), used when a call has enough tokens for the weight tiles to be
-// real dense contractions.  Same outputs as the CUDA-core kernels of
-// kd_kernels.cuh; in addition the producers write the bf16 hi/lo pairs
-// (h1lo, act_hi/act_lo) that the next tensor-core kernel multiplies.
+// real dense contractions: QKV + o-proj, router (logits, selection and token
+// lists in one launch), gate/up, down, and the combine launch.  Same outputs
+// as the CUDA-core kernels of kd_kernels.cuh; in addition the epilogues write
+// the bf16 terms (h1b/h1lo/h1lo2, act_hi/act_lo) that the next tensor-core
+// kernel multiplies.
 //
 // Tensor maps (one per weight matrix, 128 rows x 128 bytes per box (64 bf16
 // or 128 e4m3 K values), 128B swizzle):
