@@ -54,6 +54,7 @@ struct kd_layer {
   int mma_min = 4;       // calls with M >= mma_min use the tensor-core kernels
   bool has_maps = false;
   MmaMaps maps{};
+  size_t ntile = 0;      // split-K tile arrival counters per stream
 };
 
 struct kd_stack {
@@ -310,6 +311,7 @@ extern "C" int kd_layer_create(const kd_config* cfg, uint64_t seed, kd_layer** o
   {
     const size_t ntile = std::max<size_t>({(size_t)(E + 4) * (H / 128), (size_t)(E + 1) * (2 * I / 128),
                                            (size_t)(Nqkv + H) / 128});
+    L->ntile = ntile;
     TRY(dalloc_t(L, ntile, &d.tcnt_main));
     TRY(dalloc_t(L, ntile, &d.tcnt_side));
     TRYC(cudaMemset(d.tcnt_main, 0, sizeof(unsigned) * ntile));
@@ -501,6 +503,8 @@ extern "C" int kd_layer_check(kd_layer* L) {
   // an aborted call may have left arrival counters part-way
   KD_CUDA(cudaMemset(L->d.hcnt, 0, sizeof(unsigned) * (L->d.H / 64)));
   KD_CUDA(cudaMemset(L->d.rcnt, 0, sizeof(unsigned)));
+  KD_CUDA(cudaMemset(L->d.tcnt_main, 0, sizeof(unsigned) * L->ntile));
+  KD_CUDA(cudaMemset(L->d.tcnt_side, 0, sizeof(unsigned) * L->ntile));
   if (e & (ERR_WAIT_FULL | ERR_WAIT_EMPTY | ERR_WAIT_MMA))
     return fail(KD_ETIMEOUT, "device: a bounded wait gave up (flags %s0x%lx)", "", (long)e);
   return fail(KD_EDEVICE, "device error flags %s0x%lx", "", (long)e);
