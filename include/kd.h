@@ -144,8 +144,11 @@ int kd_layer_read_weight(const kd_layer* layer, int kind, int expert, int row0, 
 int kd_layer_bytes(const kd_layer* layer, uint64_t* static_bytes, uint64_t* expert_bytes);
 
 /* Number of kernels one kd_decode_layer call with M tokens launches (all of
- * them this library's).  Returns the count (>= 4), or KD_EINVAL for a null
- * layer, KD_ERANGE for M outside 1..max_tokens. */
+ * them this library's) -- the per-layer kernel count by which the write-ups
+ * compare decode paths (bigchange.ai "where the time went"; wireai.ir
+ * "compressing the decode loop with kernel fusion").  Returns the count
+ * (>= 4), or KD_EINVAL for a null layer, KD_ERANGE for M outside
+ * 1..max_tokens. */
 int kd_layer_launches(const kd_layer* layer, int M);
 
 /* Multi-layer decode step.  kd_stack_create records the layers (not owned)
