@@ -69,7 +69,7 @@ typedef struct kd_config {
   const float* router_bias; /* host [E] additive router bias, or NULL; copied    */
   int mma_min_tokens;/* calls with M >= this use the tensor-core (tcgen05) kernels,
                         smaller M the CUDA-core streaming kernels; 0 = default (4),
-                        > 64 = never.  bf16 weights only (FP8 always streams).    */
+                        > 64 = never.                                           */
 } kd_config;
 
 typedef struct kd_layer kd_layer;
@@ -178,10 +178,11 @@ int kd_layer_set_timing_events(kd_layer* layer, void* const* events, int n_event
  * of this entry point).  For callers that cannot call cudaMalloc from where
  * they run it -- e.g. a host runtime whose device memory all belongs to
  * another allocator, or a plugin that is handed only its input and output
- * buffers: the scratch this computation needs between the blocks of its
- * one launch (router logits, a block counter, the per-expert lists) lives in a file-scope __device__
- * array of fixed size in the library, held by every GPU that loads it until
- * the process exits, instead of a cudaMalloc'd workspace.
+ * buffers: the scratch that the blocks of its one launch hand to each other
+ * (router logits, a block counter, the per-expert lists) lives in a
+ * file-scope __device__ array of fixed size in the library, held by every
+ * GPU that loads it until the process exits, instead of a cudaMalloc'd
+ * workspace.
  *   router_w      device, [n_experts, hidden] bf16 (wdtype KD_WBF16) or e4m3
  *                 codes (KD_WFP8), row-major
  *   router_scales device fp32 [ceil(n_experts/128), hidden/128] for KD_WFP8,
@@ -194,15 +195,21 @@ int kd_layer_set_timing_events(kd_layer* layer, void* const* events, int n_event
  * Same arithmetic as the CUDA-core router of kd_decode_layer (the one it
  * runs below the tensor-core token threshold).  Limits: M <= 64
  * (KD_STATIC_MAX_TOKENS), n_experts <= 1024 (KD_STATIC_MAX_EXPERTS),
- * top_k <= 16, hidden a multiple of 128 and <= 8192; larger sizes return
- * KD_ERANGE, bad pointers or shapes KD_EINVAL.  Calls no cudaMalloc /
- * cudaFree.  The first call on a device looks up the scratch's device
- * address (cudaGetSymbolAddress) for that device and caches it, so make that
- * first call before any stream capture.  All calls share the scratch and it
+ * top_k <= 16, hidden <= 8192 (KD_STATIC_MAX_HIDDEN); larger sizes return
+ * KD_ERANGE; null pointers, hidden not a multiple of 128 or a bad wdtype
+ * KD_EINVAL.  Calls no cudaMalloc / cudaFree.  The first call in a CUDA
+ * context looks up the scratch's device address (cudaGetSymbolAddress) for
+ * that device and caches it with the context, so make that first call
+ * before any stream capture (a call in a new context, e.g. after
+ * cudaDeviceReset, looks it up again).  All calls share the scratch and it
  * keeps the last call's contents; calls that overlap on the GPU (other
- * streams, other threads) race on it. */
+ * streams, other threads) race on it.  Device-side errors are not
+ * reported: the launch has no bounded waits, and the only flag its
+ * selection can raise (an out-of-range expert id, which finite logits
+ * cannot produce) stays in the scratch. */
 #define KD_STATIC_MAX_TOKENS 64
 #define KD_STATIC_MAX_EXPERTS 1024
+#define KD_STATIC_MAX_HIDDEN 8192
 int kd_router_topk_static(const void* router_w, const float* router_scales, int wdtype,
                           const float* router_bias, const float* h1, int M, int hidden,
                           int n_experts, int top_k, int* idx_out, float* gates_out, void* stream);

@@ -18,6 +18,7 @@ SO_PATH = os.path.join(HERE, "libkd.so")
 
 KD_OK, KD_EINVAL, KD_ERANGE, KD_ECUDA, KD_ENOMEM, KD_ETIMEOUT, KD_EDEVICE = 0, -1, -2, -3, -4, -5, -6
 KD_WBF16, KD_WFP8 = 0, 1
+KD_STATIC_MAX_TOKENS, KD_STATIC_MAX_EXPERTS, KD_STATIC_MAX_HIDDEN = 64, 1024, 8192
 T_H1F, T_H1B, T_LOGITS, T_IDX, T_GATES, T_COUNTS, T_NACTIVE, T_YSHARED, T_YROUTED = range(9)
 
 # every symbol include/kd.h declares
@@ -210,7 +211,33 @@ def router_topk_static(router_w, router_scales, wdtype: int, router_bias, h1, M:
                        hidden: int, n_experts: int, top_k: int, idx_out, gates_out,
                        stream=None) -> None:
     """kd_router_topk_static on torch CUDA tensors (or None for the optional
-    ones); allocates no device memory."""
+    ones); allocates no device memory.  The tensors are checked here (device,
+    contiguity, dtype, size) so that a wrong one raises instead of being read
+    or written out of bounds by the kernel."""
+    import torch
+
+    def need(t, name, dtypes, numel):
+        if t is None:
+            raise ValueError(f"router_topk_static: {name} is required")
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"router_topk_static: {name} must be a contiguous CUDA tensor")
+        if t.dtype not in dtypes:
+            raise ValueError(f"router_topk_static: {name} has dtype {t.dtype}, want {dtypes}")
+        if t.numel() < numel:
+            raise ValueError(f"router_topk_static: {name} has {t.numel()} elements, needs {numel}")
+
+    if M >= 1 and n_experts >= 1 and top_k >= 1 and hidden >= 1:
+        wt = (torch.bfloat16, torch.int16, torch.uint16) if wdtype == KD_WBF16 else \
+            (torch.uint8, torch.float8_e4m3fn)
+        need(router_w, "router_w", wt, n_experts * hidden)
+        if wdtype == KD_WFP8:
+            need(router_scales, "router_scales", (torch.float32,),
+                 ((n_experts + 127) // 128) * ((hidden + 127) // 128))
+        if router_bias is not None:
+            need(router_bias, "router_bias", (torch.float32,), n_experts)
+        need(h1, "h1", (torch.float32,), M * hidden)
+        need(idx_out, "idx_out", (torch.int32,), M * top_k)
+        need(gates_out, "gates_out", (torch.float32,), M * top_k)
     ptr = lambda t: None if t is None else t.data_ptr()
     _check(lib().kd_router_topk_static(ptr(router_w), ptr(router_scales), wdtype, ptr(router_bias),
                                        ptr(h1), M, hidden, n_experts, top_k, ptr(idx_out),

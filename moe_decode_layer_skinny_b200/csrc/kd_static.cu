@@ -4,16 +4,24 @@
 // example a host runtime whose device memory is entirely owned by another
 // allocator (a framework's caching allocator, an inference engine that hands
 // plugins only their input and output buffers), or code that may only enqueue
-// work.  The logits and the per-expert lists this router needs between its
-// two kernels live in one file-scope __device__ array of fixed size instead
-// of a cudaMalloc'd workspace.
+// work.  The logits and the per-expert lists that the blocks of this
+// router's one launch hand to each other live in one file-scope __device__
+// array of fixed size instead of a cudaMalloc'd workspace.
 //
 // The array exists once per device for the life of the process.  Host code
 // may not pass the array's name to a kernel (on the host it names a stand-in,
 // not the device address): the device address is looked up with
-// cudaGetSymbolAddress on the first call on each device, with that device
-// current, and cached.  All calls share the array: two calls that overlap on
-// the GPU (different streams, or different host threads) race on it.
+// cudaGetSymbolAddress on the first call in each CUDA context (device), with
+// that device current, and cached together with the context; a call in a new
+// context (after cudaDeviceReset, say) looks it up again.  All calls share
+// the array: two calls that overlap on the GPU (different streams, or
+// different host threads) race on it.
+//
+// Device-side errors are not reported: the launch has no bounded waits, and
+// the one error flag its selection code can raise (an expert id out of range,
+// which finite logits cannot produce) stays in the scratch.  The block
+// counter returns to zero at the end of every launch; a launch cannot stop
+// part-way short of a fault, which loses the context and the array with it.
 #include <cuda_runtime.h>
 
 #include <cstdio>
@@ -29,6 +37,7 @@ namespace {
 constexpr int kMaxTok = KD_STATIC_MAX_TOKENS;
 constexpr int kMaxExp = KD_STATIC_MAX_EXPERTS;
 constexpr int kMaxK = 16;
+constexpr int kMaxHidden = 8192;   // router rows held in registers (16-byte chunks per lane)
 
 // logits [64 x 1024] | counts [1024] | offsets [1025] | active [1024]
 // | perm [64 x 16] | n_active [1] | err [1] | router blocks done [1]   (4-byte words)
@@ -44,6 +53,23 @@ static __device__ __align__(256) float g_router_scratch[kWords];
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 void* g_scratch_ptr[kMaxDevices] = {};
+void* g_scratch_ctx[kMaxDevices] = {};   // the context the cached address belongs to
+
+// cuCtxGetCurrent through the runtime's driver entry point (no libcuda link).
+typedef int (*CtxGetCurrentFn)(void**);
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = nullptr;
+  static bool looked = false;
+  if (!looked) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+    looked = true;
+  }
+  return fn;
+}
 
 thread_local char g_msg[256];
 }  // namespace
@@ -63,16 +89,16 @@ extern "C" int kd_router_topk_static(const void* router_w, const float* router_s
                                      int M, int hidden, int n_experts, int top_k, int* idx_out,
                                      float* gates_out, void* stream) {
   if (!router_w || !h1 || !idx_out || !gates_out || (wdtype == KD_WFP8 && !router_scales) ||
-      (wdtype != KD_WBF16 && wdtype != KD_WFP8) || hidden <= 0 || hidden % 128 ||
-      hidden > 8192 || top_k < 1) {
+      (wdtype != KD_WBF16 && wdtype != KD_WFP8) || hidden <= 0 || hidden % 128 || top_k < 1) {
     snprintf(g_msg, sizeof g_msg, "kd_router_topk_static: null pointer or unsupported shape");
     return fail_static(KD_EINVAL);
   }
-  if (M < 1 || M > kMaxTok || n_experts < top_k || n_experts > kMaxExp || top_k > kMaxK) {
+  if (M < 1 || M > kMaxTok || n_experts < top_k || n_experts > kMaxExp || top_k > kMaxK ||
+      hidden > kMaxHidden) {
     snprintf(g_msg, sizeof g_msg,
-             "kd_router_topk_static: M=%d experts=%d top_k=%d beyond the static limits "
-             "(M <= %d, top_k <= experts <= %d, top_k <= %d)",
-             M, n_experts, top_k, kMaxTok, kMaxExp, kMaxK);
+             "kd_router_topk_static: M=%d experts=%d top_k=%d hidden=%d beyond the static "
+             "limits (M <= %d, top_k <= experts <= %d, top_k <= %d, hidden <= %d)",
+             M, n_experts, top_k, hidden, kMaxTok, kMaxExp, kMaxK, kMaxHidden);
     return fail_static(KD_ERANGE);
   }
   int dev = 0;
@@ -82,8 +108,11 @@ extern "C" int kd_router_topk_static(const void* router_w, const float* router_s
   }
   void* base = nullptr;
   {
+    void* ctx = nullptr;
+    CtxGetCurrentFn cur = ctx_get_current();
+    if (cur) cur(&ctx);
     std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_scratch_ptr[dev]) {
+    if (!g_scratch_ptr[dev] || g_scratch_ctx[dev] != ctx) {
       void* p = nullptr;
       cudaError_t e = cudaGetSymbolAddress(&p, g_router_scratch);
       if (e != cudaSuccess) {
@@ -92,6 +121,7 @@ extern "C" int kd_router_topk_static(const void* router_w, const float* router_s
         return fail_static(KD_ECUDA);
       }
       g_scratch_ptr[dev] = p;
+      g_scratch_ctx[dev] = ctx;
     }
     base = g_scratch_ptr[dev];
   }

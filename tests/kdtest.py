@@ -2,11 +2,22 @@
 and compare it with the CPU oracle.
 
 Tolerances (from the layer's precision contract): per output tensor,
-max|gpu - oracle| / rms(oracle) <= 1e-2 for bf16 weights, 3e-2 for FP8,
-measured beyond the rounding of the exact value into the bf16 output format
-(see rel_err_bf16); the top-k expert ids must match exactly unless the
-oracle's k-th and (k+1)-th logits are closer than 1e-4, in which case that
-token's row is compared with the oracle recomputed under the GPU's selection.
+max|gpu - oracle| / rms(oracle) <= 1e-2 for bf16 weights, 3e-2 for FP8.
+Both outputs (the layer output and qkv) are bf16 by the interface, and the
+correctly rounded bf16 value of the exact result is itself up to half a bf16
+ulp away from it -- up to 2^-9 max|x|, which exceeds 1e-2 rms wherever
+max|x| > 5.1 rms.  So each comparison asserts three things:
+  * raw    max|gpu - oracle| / rms <= tol + max half-ulp(oracle) / rms (the
+           bound every correctly rounded result meets); with strict_raw, the
+           literal bound max|gpu - oracle| / rms <= tol as well;
+  * excess the error beyond that storage rounding (rel_err_bf16) <= tol;
+  * tight  the excess <= TIGHT[wdtype], a bound set from the arithmetic of the
+           kernels (bf16 weights: exact products of hi + lo activation terms,
+           fp32 accumulation; measured ~5e-5), low enough that dropping an
+           activation term (~1e-2) fails.
+The top-k expert ids must match exactly unless the oracle's k-th and
+(k+1)-th logits are closer than 1e-4, in which case that token's row is
+compared with the oracle recomputed under the GPU's selection.
 """
 from __future__ import annotations
 
@@ -16,6 +27,7 @@ import kdgen
 import oracle
 
 TOL = {0: 1e-2, 1: 3e-2}
+TIGHT = {0: 1e-3, 1: 3e-2}
 TIE_GAP = 1e-4
 
 
@@ -45,6 +57,29 @@ def rel_err_bf16(gpu: np.ndarray, ref: np.ndarray) -> float:
     rms = float(np.sqrt(np.mean(ref.astype(np.float64) ** 2)))
     ex = np.abs(gpu.astype(np.float64) - ref) - bf16_half_ulp(ref)
     return float(max(np.max(ex), 0.0)) / max(rms, 1e-300)
+
+
+def rounding_floor(ref: np.ndarray) -> float:
+    """max half-ulp_bf16(ref) / rms(ref): what bf16 storage of the exact value
+    alone may cost."""
+    rms = float(np.sqrt(np.mean(ref.astype(np.float64) ** 2)))
+    return float(np.max(bf16_half_ulp(ref))) / max(rms, 1e-300)
+
+
+def check_output(report: dict, key: str, gpu: np.ndarray, ref: np.ndarray, wdtype: int,
+                 strict_raw: bool) -> None:
+    """Raw, beyond-rounding and tight checks of one bf16 output tensor."""
+    tol = TOL[wdtype]
+    raw = rel_err(gpu, ref)
+    ex = rel_err_bf16(gpu, ref)
+    report[key + "_raw"] = raw
+    report[key] = ex
+    report[key + "_floor"] = rounding_floor(ref)
+    assert ex <= tol, (key, report)
+    assert ex <= TIGHT[wdtype], (key, "beyond-rounding error above the tight bound", report)
+    assert raw <= tol + report[key + "_floor"] * (1 + 1e-9), (key, report)
+    if strict_raw:
+        assert raw <= tol, (key, "raw error above the literal bound", report)
 
 
 def torch_bf16(bits: np.ndarray, device="cuda"):
@@ -115,10 +150,9 @@ def selection_check(gpu_idx: np.ndarray, ref_logits: np.ndarray, ref_idx: np.nda
 
 
 def compare_layer(dims, gpu: dict, x_bits, a_bits, *, wdtype=0, layer_id=0, seed=0, bias=None,
-                  rows=None, check_qkv=True) -> dict:
+                  rows=None, check_qkv=True, strict_raw=False) -> dict:
     """Compare one GPU layer call with the oracle (all rows, or the listed rows,
     each recomputed on its own -- rows are independent)."""
-    tol = TOL[wdtype]
     x = bf16_to_f64(x_bits)
     a = bf16_to_f64(a_bits)
     rows = list(range(x.shape[0])) if rows is None else list(rows)
@@ -146,13 +180,7 @@ def compare_layer(dims, gpu: dict, x_bits, a_bits, *, wdtype=0, layer_id=0, seed
         report["logits"] = rel_err(g["logits"], ref["logits"])
         assert report["h1"] < 1e-4, report
         assert report["logits"] < 1e-3, report
-    out = bf16_to_f64(g["out"])
-    report["out_raw"] = rel_err(out, ref["out"])
-    report["out"] = rel_err_bf16(out, ref["out"])
-    assert report["out"] <= tol, report
+    check_output(report, "out", bf16_to_f64(g["out"]), ref["out"], wdtype, strict_raw)
     if check_qkv:
-        q = bf16_to_f64(g["qkv"])
-        report["qkv_raw"] = rel_err(q, ref["qkv"])
-        report["qkv"] = rel_err_bf16(q, ref["qkv"])
-        assert report["qkv"] <= tol, report
+        check_output(report, "qkv", bf16_to_f64(g["qkv"]), ref["qkv"], wdtype, strict_raw)
     return report

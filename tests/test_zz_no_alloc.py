@@ -3,7 +3,8 @@ device memory (a runtime whose device memory belongs to another allocator, a
 plugin handed only its inputs and outputs).  Its scratch is a fixed
 __device__ array inside the library; here its output is checked, through the
 C ABI, against the router of kd_decode_layer on the same weights and h1, on
-two calls in a row.  This file is collected last on purpose."""
+two calls in a row, and the device's free memory is checked to be the same
+before and after a call.  This file is collected last on purpose."""
 import numpy as np
 import pytest
 
@@ -40,11 +41,17 @@ def _case(kd, torch, dims, wdtype, bias, M):
         b = None if bias is None else torch.from_numpy(np.asarray(bias, np.float32)).cuda()
         idx = torch.full((M, k), -1, dtype=torch.int32, device="cuda")
         gates = torch.zeros((M, k), dtype=torch.float32, device="cuda")
-        for _ in range(2):
+        for call in range(2):
             idx.fill_(-1)
             gates.zero_()
+            torch.cuda.synchronize()
+            free0 = torch.cuda.mem_get_info()[0]
+            alloc0 = torch.cuda.memory_allocated()
             kd.router_topk_static(wr, sc, wdtype, b, h1, M, H, E, k, idx, gates)
             torch.cuda.synchronize()
+            if call == 1:   # the first call may load the library's module
+                assert torch.cuda.mem_get_info()[0] == free0
+            assert torch.cuda.memory_allocated() == alloc0
             assert np.array_equal(idx.cpu().numpy(), ref_idx)
             assert np.abs(gates.cpu().numpy() - ref_gates).max() < 1e-4
     finally:
@@ -66,8 +73,14 @@ def test_static_router_rejects_sizes_beyond_its_scratch(torch_cuda):
     wr = torch.zeros((2048, 256), dtype=torch.bfloat16, device="cuda")
     idx = torch.zeros((65, 16), dtype=torch.int32, device="cuda")
     g = torch.zeros((65, 16), dtype=torch.float32, device="cuda")
-    for M, E, k in [(65, 8, 2), (4, 1025, 2), (4, 64, 17)]:
-        with pytest.raises(kd.KdError) as ei:
-            kd.router_topk_static(wr, None, kd.KD_WBF16, None, h1, M, 256, E, k, idx, g)
-        assert ei.value.code == kd.KD_ERANGE
-        assert "static limits" in str(ei.value)
+    for M, E, k, H in [(65, 8, 2, 256), (4, 1025, 2, 256), (4, 64, 17, 256), (4, 8, 2, 8320)]:
+        # through the C ABI directly (the binding would refuse the short buffers)
+        rc = kd.lib().kd_router_topk_static(wr.data_ptr(), None, kd.KD_WBF16, None, h1.data_ptr(),
+                                            M, H, E, k, idx.data_ptr(), g.data_ptr(), None)
+        assert rc == kd.KD_ERANGE, (M, E, k, H)
+        assert "static limits" in kd.lib().kd_last_error().decode()
+    # the binding checks its tensors before the call
+    with pytest.raises(ValueError):
+        kd.router_topk_static(wr, None, kd.KD_WBF16, None, h1[:, :128], 4, 256, 8, 2, idx, g)
+    with pytest.raises(ValueError):
+        kd.router_topk_static(wr, None, kd.KD_WBF16, None, h1, 4, 256, 8, 2, idx.long(), g)
