@@ -21,6 +21,7 @@ _SRC = [os.path.join(_HERE, "kdgen_host.c"), os.path.join(_HERE, "kd_gen.h")]
 
 # tensor kinds of kd_gen.h
 QKV, OPROJ, ROUTER, GATE, UP, DOWN, HIDDEN_IN, ATTN_OUT = 1, 2, 3, 4, 5, 6, 16, 17
+NORM1, NORM2, KCACHE, VCACHE = 7, 8, 18, 19
 UNIT = float.fromhex("0x1.bb67aep-16")
 W002 = float.fromhex("0x1.1bc77ap-21")
 
@@ -55,6 +56,8 @@ def lib() -> ctypes.CDLL:
         L.kdg_host_zipf_bias.argtypes = [i32, f64, vp]
         L.kdg_host_weight_bf16.argtypes = [u64, u32, u32, u32, i32, i32, vp]
         L.kdg_host_weight_fp8.argtypes = [u64, u32, u32, u32, i32, i32, vp, vp]
+        L.kdg_host_norm_bf16.argtypes = [u64, u32, u32, i32, vp]
+        L.kdg_host_kv_cache.argtypes = [u64, u32, u32, i32, i32, i32, f32, f32, vp]
         _lib = L
     return _lib
 
@@ -116,6 +119,21 @@ def weight_fp8(seed: int, layer: int, kind: int, slot: int, R: int, K: int):
     scales = np.empty(((R + 127) // 128, (K + 127) // 128), np.float32)
     lib().kdg_host_weight_fp8(seed, layer, kind, slot, R, K, _p(codes), _p(scales))
     return codes, scales
+
+
+def norm_bf16(seed: int, layer: int, kind: int, n: int) -> np.ndarray:
+    """RMSNorm gains [n] (kind NORM1 / NORM2) as bf16 bits."""
+    out = np.empty(n, np.uint16)
+    lib().kdg_host_norm_bf16(seed, layer, kind, n, _p(out))
+    return out
+
+
+def kv_cache(seed: int, layer: int, kind: int, n_seq: int, max_ctx: int, width: int,
+             sigma: float, scale: float) -> np.ndarray:
+    """Synthetic e4m3 KV-cache codes [n_seq, max_ctx, width] (kind KCACHE / VCACHE)."""
+    out = np.empty((n_seq, max_ctx, width), np.uint8)
+    lib().kdg_host_kv_cache(seed, layer, kind, n_seq, max_ctx, width, sigma, scale, _p(out))
+    return out
 
 
 def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:

@@ -21,6 +21,7 @@
  *   value           = (float)ih4 * c   -- ONE fp32 multiply, c a fixed fp32 constant
  *                     c = KDG_UNIT  (unit variance) or KDG_W002 (sigma = 0.02)
  *   bf16            = round-to-nearest-even of the fp32 value
+ *   norm weight     = bf16(1 + value), c = KDG_W002 (RMSNorm gains near 1)
  *   FP8 (per logical 128x128 block of a weight matrix)
  *                     amax  = max |value| over the block (fp32, exact)
  *                     scale = amax / 448 (IEEE fp32 division), 1 if amax == 0
@@ -53,7 +54,9 @@
 enum {
   KDG_QKV = 1, KDG_OPROJ = 2, KDG_ROUTER = 3,
   KDG_GATE = 4, KDG_UP = 5, KDG_DOWN = 6,
-  KDG_HIDDEN_IN = 16, KDG_ATTN_OUT = 17
+  KDG_NORM1 = 7, KDG_NORM2 = 8,          /* RMSNorm gains before attention / the MoE */
+  KDG_HIDDEN_IN = 16, KDG_ATTN_OUT = 17,
+  KDG_KCACHE = 18, KDG_VCACHE = 19       /* synthetic KV-cache contents */
 };
 
 /* uid of one tensor: layer in bits 40.., kind in 32..39, expert slot in 0..31
@@ -106,6 +109,15 @@ KDG_FN uint16_t kdg_bf16(float f) {
   uint32_t b = kdg_f32_bits(f);
   b += 0x7FFFu + ((b >> 16) & 1u);
   return (uint16_t)(b >> 16);
+}
+
+/* RMSNorm gain element `index`: bf16(1 + value(sigma 0.02)). */
+KDG_FN uint16_t kdg_norm_bf16(uint64_t stream, uint64_t index) {
+#if defined(__CUDA_ARCH__)
+  return kdg_bf16(__fadd_rn(1.0f, kdg_value(stream, index, KDG_W002)));
+#else
+  return kdg_bf16(1.0f + kdg_value(stream, index, KDG_W002));
+#endif
 }
 
 /* FP8 block scale from a block's amax. */

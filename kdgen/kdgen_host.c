@@ -82,3 +82,22 @@ void kdg_host_weight_fp8(uint64_t seed, uint32_t layer, uint32_t kind, uint32_t 
           codes[(size_t)r * K + c] = kdg_e4m3(kdg_fp8_div(kdg_value(st, (uint64_t)r * K + c, KDG_W002), sc));
     }
 }
+
+/* RMSNorm gains [n] of one layer (kind KDG_NORM1 / KDG_NORM2) as bf16 bits. */
+void kdg_host_norm_bf16(uint64_t seed, uint32_t layer, uint32_t kind, int n, uint16_t* out) {
+  uint64_t st = kdg_stream(seed, kdg_uid(layer, kind, 0));
+  for (int i = 0; i < n; ++i) out[i] = kdg_norm_bf16(st, (uint64_t)i);
+}
+
+/* Synthetic KV-cache contents: e4m3 codes of fp32(sigma * z) / scale for
+ * element ((s * max_ctx + p) * width + c) of one layer's K (KDG_KCACHE) or V
+ * (KDG_VCACHE) cache [n_seq][max_ctx][width], z = ih4 * unit (N(0,1)-like). */
+void kdg_host_kv_cache(uint64_t seed, uint32_t layer, uint32_t kind, int n_seq, int max_ctx,
+                       int width, float sigma, float scale, uint8_t* out) {
+  uint64_t st = kdg_stream(seed, kdg_uid(layer, kind, 0));
+  int64_t n = (int64_t)n_seq * max_ctx * width;
+  for (int64_t i = 0; i < n; ++i) {
+    float v = kdg_value(st, (uint64_t)i, KDG_UNIT) * sigma;
+    out[i] = kdg_e4m3(kdg_fp8_div(v, scale));
+  }
+}

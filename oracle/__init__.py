@@ -39,8 +39,11 @@ class _Cfg(ctypes.Structure):
                 ("layer_id", ctypes.c_int), ("seed", ctypes.c_uint64)]
 
 
+_WNAMES = ("wqkv", "wo", "wr", "wg", "wu", "wd", "g1", "g2")
+
+
 class _W(ctypes.Structure):
-    _fields_ = [(n, ctypes.c_void_p) for n in ("wqkv", "wo", "wr", "wg", "wu", "wd")]
+    _fields_ = [(n, ctypes.c_void_p) for n in _WNAMES]
 
 
 _lib = None
@@ -61,6 +64,18 @@ def lib() -> ctypes.CDLL:
         L.orc_bf16_value.argtypes = [ctypes.c_uint16]
         L.orc_e4m3_value.restype = ctypes.c_double
         L.orc_e4m3_value.argtypes = [ctypes.c_uint8]
+        L.orc_e4m3_code.restype = ctypes.c_uint8
+        L.orc_e4m3_code.argtypes = [ctypes.c_double]
+        L.orc_rmsnorm.restype = None
+        L.orc_rmsnorm.argtypes = [vp, vp, ctypes.c_int, ctypes.c_double, vp]
+        i32, f64 = ctypes.c_int, ctypes.c_double
+        L.orc_attention.restype = i32
+        L.orc_attention.argtypes = [vp, i32, vp, vp, f64, f64, i32, i32, i32, i32, i32, vp, vp, i32,
+                                    vp, i32]
+        L.orc_layer_full.restype = i32
+        L.orc_layer_full.argtypes = [ctypes.POINTER(_Cfg), ctypes.POINTER(_W), vp, vp, i32, vp, vp,
+                                     f64, f64, i32, i32, vp, vp, f64, i32, vp, i32,
+                                     vp, vp, vp, vp, vp, vp, vp, vp]
         _lib = L
     return _lib
 
@@ -98,6 +113,80 @@ def weight_rows(dims, kind: int, expert: int, row0: int, nrows: int, wdtype=0, l
     return out
 
 
+def _weights_ptr(weights, keep):
+    if weights is None:
+        return None
+    arrs = {k: np.ascontiguousarray(weights[k], np.float64) for k in _WNAMES if k in weights}
+    keep.append(arrs)
+    return ctypes.byref(_W(*(arrs[k].ctypes.data if k in arrs else None for k in _WNAMES)))
+
+
+def e4m3_code(v: float) -> int:
+    return int(lib().orc_e4m3_code(float(v)))
+
+
+def rmsnorm(x, gamma, eps: float) -> np.ndarray:
+    """RMSNorm of each row of x [.., n] with gain gamma [n]."""
+    x = np.ascontiguousarray(x, np.float64)
+    g = np.ascontiguousarray(gamma, np.float64)
+    flat = x.reshape(-1, x.shape[-1])
+    out = np.empty_like(flat)
+    for i in range(flat.shape[0]):
+        lib().orc_rmsnorm(_p(flat[i]), _p(g), flat.shape[1], eps, _p(out[i]))
+    return out.reshape(x.shape)
+
+
+def attention(q, kc, vc, k_scale, v_scale, hq, hkv, hd, seq, pos) -> np.ndarray:
+    """Attention of rows q [M, hq*hd] over e4m3 caches kc, vc [n_seq, max_ctx, hkv*hd]."""
+    q = np.ascontiguousarray(q, np.float64)
+    kc = np.ascontiguousarray(kc, np.uint8)
+    vc = np.ascontiguousarray(vc, np.uint8)
+    seq = np.ascontiguousarray(seq, np.int32)
+    pos = np.ascontiguousarray(pos, np.int32)
+    M = q.shape[0]
+    out = np.zeros((M, hq * hd))
+    rc = lib().orc_attention(_p(q), q.shape[1], _p(kc), _p(vc), k_scale, v_scale, kc.shape[0],
+                             kc.shape[1], hq, hkv, hd, _p(seq), _p(pos), M, _p(out), hq * hd)
+    if rc != 0:
+        raise ValueError("orc_attention: bad arguments")
+    return out
+
+
+def layer_full(dims, x, kc, vc, k_scale, v_scale, seq, pos, *, wdtype=0, layer_id=0, seed=0,
+               eps=1e-6, bias=None, weights=None, keep_new_kv=False, forced_idx=None,
+               nthreads=None) -> dict:
+    """The full decode layer (RMSNorm, QKV, FP8-cache attention, o-proj +
+    residual, RMSNorm, MoE) for M tokens; kc / vc [n_seq, max_ctx, kv_heads*hd]
+    e4m3 codes are copied, and the copies (with the new tokens' codes) are
+    returned as "kc" / "vc"."""
+    x = np.ascontiguousarray(x, np.float64)
+    M = x.shape[0]
+    kc = np.array(kc, np.uint8, copy=True, order="C")
+    vc = np.array(vc, np.uint8, copy=True, order="C")
+    seq = np.ascontiguousarray(seq, np.int32)
+    pos = np.ascontiguousarray(pos, np.int32)
+    c = _cfg(dims, wdtype, layer_id, seed)
+    keep = []
+    wp = _weights_ptr(weights, keep)
+    b = None if bias is None else np.ascontiguousarray(bias, np.float64)
+    f = None if forced_idx is None else np.ascontiguousarray(forced_idx, np.int32)
+    if nthreads is None:
+        nthreads = os.cpu_count() or 1
+    res = {"qkv": np.zeros((M, dims.nqkv)), "attn": np.zeros((M, dims.attn)),
+           "h1": np.zeros((M, dims.hidden)), "v": np.zeros((M, dims.hidden)),
+           "logits": np.zeros((M, dims.n_experts)), "idx": np.zeros((M, dims.top_k), np.int32),
+           "gates": np.zeros((M, dims.top_k)), "out": np.zeros((M, dims.hidden))}
+    rc = lib().orc_layer_full(ctypes.byref(c), wp, _p(b), _p(x), M, _p(kc), _p(vc), k_scale,
+                              v_scale, kc.shape[0], kc.shape[1], _p(seq), _p(pos), eps,
+                              1 if keep_new_kv else 0, _p(f), nthreads, _p(res["qkv"]),
+                              _p(res["attn"]), _p(res["h1"]), _p(res["v"]), _p(res["logits"]),
+                              _p(res["idx"]), _p(res["gates"]), _p(res["out"]))
+    if rc != 0:
+        raise ValueError("orc_layer_full: bad arguments")
+    res["kc"], res["vc"] = kc, vc
+    return res
+
+
 def layer(dims, x, attn, *, wdtype=0, layer_id=0, seed=0, bias=None, weights=None,
           forced_idx=None, ksplit=1, nthreads=None, want_qkv=True) -> dict:
     """Evaluate one layer for M tokens.
@@ -113,11 +202,7 @@ def layer(dims, x, attn, *, wdtype=0, layer_id=0, seed=0, bias=None, weights=Non
     assert x.shape == (M, dims.hidden) and attn.shape == (M, dims.attn)
     c = _cfg(dims, wdtype, layer_id, seed)
     keep = []
-    wp = None
-    if weights is not None:
-        arrs = {k: np.ascontiguousarray(weights[k], np.float64) for k in ("wqkv", "wo", "wr", "wg", "wu", "wd")}
-        keep.append(arrs)
-        wp = ctypes.byref(_W(*(arrs[k].ctypes.data for k in ("wqkv", "wo", "wr", "wg", "wu", "wd"))))
+    wp = _weights_ptr(weights, keep)
     b = None if bias is None else np.ascontiguousarray(bias, np.float64)
     f = None if forced_idx is None else np.ascontiguousarray(forced_idx, np.int32)
     if nthreads is None:

@@ -55,6 +55,8 @@ typedef struct orc_weights {
   const double* wg;    /* [n_shared+E, I, H] */
   const double* wu;    /* [n_shared+E, I, H] */
   const double* wd;    /* [n_shared+E, H, I] */
+  const double* g1;    /* [H] RMSNorm gain before attention (full layer), or NULL */
+  const double* g2;    /* [H] RMSNorm gain before the MoE (full layer), or NULL   */
 } orc_weights;
 
 /* One layer for M tokens.  Returns 0, or -1 on bad arguments.
@@ -79,9 +81,54 @@ int orc_layer(const orc_cfg* cfg, const orc_weights* w, const double* bias,
 int orc_weight_rows(const orc_cfg* cfg, int kind, int expert, int row0,
                     int nrows, double* dst);
 
-/* This file's own decoders of the two storage formats. */
+/* This file's own decoders of the two storage formats, and its e4m3 encoder
+ * (round to nearest even, saturating at +-448), written from the format. */
 double orc_bf16_value(uint16_t bits);
 double orc_e4m3_value(uint8_t code);
+uint8_t orc_e4m3_code(double v);
+
+/* ---------------------------------------------------------------- full layer
+ * The decode layer with its attention half (an extension beyond the chain
+ * above: the pages name the attention core with an FP8 KV cache among the
+ * steps of decode -- bigchange.ai "where the time went" -- and the input
+ * projections feeding it -- wireai.ir "4 key changes", item 1).  Pre-norm
+ * residual form, for token t of sequence seq[t] at position pos[t]:
+ *
+ *   u_t   = RMSNorm(x_t) g1          RMSNorm(z) = z / sqrt(mean(z^2) + eps)
+ *   qkv_t = Wqkv u_t = (q_t [Hq x hd], k_t [Hkv x hd], v_t [Hkv x hd])
+ *   K[seq, pos] = e4m3(k_t / k_scale),  V[seq, pos] = e4m3(v_t / v_scale)
+ *   o_t,h = sum_{j <= pos} softmax_j(q_t,h . K'_j,g / sqrt(hd)) V'_j,g,
+ *           K' = k_scale dec(K), V' = v_scale dec(V), g = h / (Hq / Hkv)
+ *   h1_t  = x_t + Wo o_t
+ *   v_t   = RMSNorm(h1_t) g2
+ *   out_t = h1_t + F_shared(v_t) + sum_{e in S_t} g_e F_e(v_t),  S_t, g from Wr v_t + b
+ *
+ * Every new key and value is written before any token attends, so tokens of
+ * one sequence at consecutive positions (a speculative-verify step) see each
+ * other causally.  No positional rotation is applied. */
+
+/* RMSNorm of one row: y = x / sqrt(sum(x^2)/n + eps) * gamma. */
+void orc_rmsnorm(const double* x, const double* gamma, int n, double eps, double* y);
+
+/* Attention of M tokens over an e4m3 KV cache [n_seq][max_ctx][Hkv][hd]
+ * (codes as given, the new tokens' included).  q row t at q + t*ldq, output
+ * row t at out + t*ldo.  Returns 0, or -1 on bad arguments. */
+int orc_attention(const double* q, int ldq, const uint8_t* kc, const uint8_t* vc, double k_scale,
+                  double v_scale, int n_seq, int max_ctx, int Hq, int Hkv, int hd,
+                  const int* seq, const int* pos, int M, double* out, int ldo);
+
+/* The full layer.  kc / vc are read and (unless keep_new_kv) the new tokens'
+ * codes written at (seq[t], pos[t]); with keep_new_kv the codes already there
+ * are used (the GPU's, for parity checks).  Gains from w->g1 / w->g2 or the
+ * generator (kinds KDG_NORM1 / KDG_NORM2).  Outputs (any may be NULL except
+ * out): qkv [M,Nqkv], attn [M,A], h1 [M,H], v [M,H] (the MoE input), logits,
+ * idx, gates, out [M,H]. */
+int orc_layer_full(const orc_cfg* cfg, const orc_weights* w, const double* bias, const double* x,
+                   int M, uint8_t* kc, uint8_t* vc, double k_scale, double v_scale, int n_seq,
+                   int max_ctx, const int* seq, const int* pos, double eps, int keep_new_kv,
+                   const int* forced_idx, int nthreads, double* qkv_out, double* attn_out,
+                   double* h1_out, double* v_out, double* logits_out, int* idx_out,
+                   double* gates_out, double* out);
 
 #ifdef __cplusplus
 }
