@@ -226,6 +226,7 @@ def kernel_bytes(spec, n_active: int) -> dict:
 
 
 KNAMES = ("proj", "router", "gateup", "down")
+SWEEP_M = (1, 2, 3, 4, 5, 6, 7, 8, 16, 32, 64)
 
 
 def time_layer(layer, x_bits, a_bits, steps, warmup, flush, pg, local, per_kernel=True):
@@ -359,6 +360,7 @@ def bench_single(w, steps, warmup, flush, pg, local, peak):
                "active_experts": na, "weight_bytes": byts,
                "hbm_gbs": byts / (ms * 1e-3) / 1e9, "tok_s": w.M / (ms * 1e-3)}
         res["hbm_frac"] = res["hbm_gbs"] / peak
+        res["expert_bytes"] = layer.bytes()[1]
         res["kernels_us"] = {n: kt[n] * 1e3 for n in KNAMES}
         res["kernels_gbs"] = {n: (kb[n] / (kt[n] * 1e-3) / 1e9 if kb[n] else None) for n in KNAMES}
         return res, layer, x, a, kb, kt
@@ -399,35 +401,117 @@ def bench_stack(w, steps, warmup, flush, pg, local, peak, prefetch):
         # bytes: each layer's unique weights under the routing of its own input
         byts = 0
         hidden.copy_(x0)
+        per_layer = []
         for L, l in zip(layers, range(w.n_layers)):
             L.decode(hidden, attn[l * w.M:(l + 1) * w.M])
-            byts += layer_bytes(L, n_active_of(L))
+            na = n_active_of(L)
+            per_layer.append(na)
+            byts += layer_bytes(L, na)
+        st0, ex0 = layers[0].bytes()
         st.close()
         ms = statistics.mean(times)
         return {"us_per_layer": ms * 1e3 / w.n_layers, "us_per_step": ms * 1e3,
                 "M": w.M, "layers": w.n_layers, "weight_bytes": byts,
                 "hbm_gbs": byts / (ms * 1e-3) / 1e9, "hbm_frac": byts / (ms * 1e-3) / 1e9 / peak,
-                "tok_s": w.M / (ms * 1e-3), "l2_prefetch": bool(prefetch)}
+                "tok_s": w.M / (ms * 1e-3), "l2_prefetch": bool(prefetch),
+                "active_experts_per_layer": per_layer, "active_experts_layer0": per_layer[0],
+                "layer0_bytes": (st0, ex0)}
     finally:
         for L in layers:
             L.close()
 
 
-def cpu_baseline(w, budget_s=15.0):
-    """The oracle as it stands, on the host cores, full layer for the workload."""
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def _oracle_call(w, rows, threads, layer_id=0):
     import oracle
     import kdgen
-    x = kdgen.bf16_bits_to_f32(w.hidden_in()).astype(np.float64)
-    a = kdgen.bf16_bits_to_f32(w.attn_out()).astype(np.float64)
-    cores = os.cpu_count() or 1
-    times = []
+    x = kdgen.bf16_bits_to_f32(w.hidden_in()[rows]).astype(np.float64)
+    a = kdgen.bf16_bits_to_f32(w.attn_out(layer_id)[rows]).astype(np.float64)
+    t0 = time.perf_counter()
+    r = oracle.layer(w.dims, x, a, wdtype=w.wdtype, layer_id=layer_id,
+                     bias=None if w.bias() is None else w.bias().astype(np.float64),
+                     nthreads=threads, want_qkv=True)
+    return time.perf_counter() - t0, len(np.unique(r["idx"]))
+
+
+def cpu_baseline(w, threads, budget_s=15.0, rows=None, full_union=None, static_bytes=None,
+                 expert_bytes=None):
+    """The oracle as it stands (fp64 C, weights generated as it goes) on the
+    host cores, timed on the workload's layer (layer 0 of a stack).  With
+    `rows`, a bounded sample: only those token rows, scaled to the full layer
+    by its weight bytes (the oracle's time is its weight generation, linear in
+    the experts it touches): t_full = t_sample x (static + U_full expert) /
+    (static + U_sample expert)."""
+    rows = list(range(w.M)) if rows is None else list(rows)
+    times, n_sample = [], 0
     t_end = time.time() + budget_s
     while not times or (time.time() < t_end and len(times) < 5):
-        t0 = time.perf_counter()
-        oracle.layer(w.dims, x, a, wdtype=w.wdtype, bias=None if w.bias() is None else
-                     w.bias().astype(np.float64), nthreads=cores, want_qkv=True)
-        times.append(time.perf_counter() - t0)
-    return statistics.mean(times), cores, len(times)
+        t, n_sample = _oracle_call(w, rows, threads)
+        times.append(t)
+    t = statistics.mean(times)
+    res = {"threads": threads, "calls": len(times), "rows": len(rows), "sample_s": t}
+    if len(rows) < w.M and full_union and static_bytes is not None:
+        scale = (static_bytes + full_union * expert_bytes) / (static_bytes + n_sample * expert_bytes)
+        res.update(us_per_layer=t * scale * 1e6, scaled=True, experts_sample=n_sample,
+                   experts_full=full_union)
+    else:
+        res.update(us_per_layer=t * 1e6, scaled=False, experts=n_sample)
+    return res
+
+
+def cpu_baselines(workloads: dict, unions: dict, layer_bytes_by_wl: dict) -> dict:
+    """Every workload's layer on all host cores (full layer) and on one core
+    (the full layer when it is the M=1 one, else the first token row, scaled
+    to the full layer by weight bytes)."""
+    cores = os.cpu_count() or 1
+    out = {"nproc": cores, "cpu_model": cpu_model(), "kind": "oracle", "unit": UNIT,
+           "workloads": {}}
+    for name, w in workloads.items():
+        st, ex = layer_bytes_by_wl.get(name, (None, None))
+        allc = cpu_baseline(w, cores, budget_s=10.0)
+        one = cpu_baseline(w, 1, budget_s=5.0, rows=None if w.M == 1 else [0],
+                           full_union=unions.get(name), static_bytes=st, expert_bytes=ex)
+        out["workloads"][name] = {"all_cores": allc, "one_core": one}
+    return out
+
+
+def bench_sweep(dims, Ms, steps, flush, pg, local, peak) -> dict:
+    """µs per layer, HBM fraction and launches at each token count M (one
+    bf16 H=7168 layer; rows with 0.9 correlation at the verify shapes 4..8,
+    independent otherwise)."""
+    import moe_decode_layer_skinny_b200 as kd
+    import kdgen
+    spec = kd.LayerSpec.from_dims(dims, max_tokens=max(Ms))
+    layer = kd.Layer(spec, seed=0)
+    res = {}
+    try:
+        for M in Ms:
+            rho = 0.9 if 4 <= M <= 8 else 0.0
+            x = kdgen.activations(0, 0, kdgen.HIDDEN_IN, M, dims.hidden, rho)
+            a = kdgen.activations(0, 0, kdgen.ATTN_OUT, M, dims.attn, rho)
+            times, _ = time_layer(layer, x, a, steps, 3, flush, pg, local, per_kernel=False)
+            na = n_active_of(layer)
+            ms = statistics.mean(times)
+            byts = layer_bytes(layer, na)
+            res[str(M)] = {"us_per_layer": ms * 1e3, "active_experts": na, "weight_bytes": byts,
+                           "hbm_gbs": byts / (ms * 1e-3) / 1e9,
+                           "hbm_frac": byts / (ms * 1e-3) / 1e9 / peak,
+                           "tok_s": M / (ms * 1e-3), "launches": layer.launches(M),
+                           "rows": "correlated 0.9" if rho else "independent"}
+    finally:
+        layer.close()
+    return res
 
 
 def run_kd(args):
@@ -491,22 +575,36 @@ def run_kd(args):
                        "frac": ach / peak, "traffic": profiled_traffic(dom, main.name),
                        "algorithmic_bytes_per_launch": kb[dom], "peak_src": peak_src}
     # secondary workloads
+    unions = {main.name: res["active_experts"]}
+    lbytes = {main.name: (res["weight_bytes"] - res["active_experts"] * res["expert_bytes"],
+                          res["expert_bytes"])}
     if not args.main_only:
         wl = {}
         for name in ("verify8", "batch64_zipf"):
             r2, l2, *_ = bench_single(W[name], max(10, args.steps // 10), 3, flush, pg, local, peak)
             l2.close()
             wl[name] = r2
+            unions[name] = r2["active_experts"]
+            lbytes[name] = (r2["weight_bytes"] - r2["active_experts"] * r2["expert_bytes"],
+                            r2["expert_bytes"])
         for pf in (True, False):
             key = "stack4_fp8" + ("" if pf else "_noprefetch")
             wl[key] = bench_stack(W["stack4_fp8"], max(5, args.steps // 20), 3, flush, pg, local,
                                   peak, pf)
+        unions["stack4_fp8"] = wl["stack4_fp8"]["active_experts_layer0"]
+        lbytes["stack4_fp8"] = wl["stack4_fp8"]["layer0_bytes"]
         out["workloads"] = wl
+        out["sweep"] = bench_sweep(W["batch1"].dims, SWEEP_M, max(10, args.steps // 10), flush, pg,
+                                   local, peak)
     if rank == 0 and ws == 1 and not args.no_cpu:
-        t, cores, n = cpu_baseline(main)
-        out["cpu_baseline"] = {"value": t * 1e6, "unit": UNIT, "cores": cores, "kind": "oracle",
-                               "sample": f"{n} full {main.name} layer call(s) (M={main.M}), fp64 oracle "
-                                         f"generating its weights as it goes, {cores} threads"}
+        names = [main.name] if args.main_only else ["batch1", "verify8", "batch64_zipf", "stack4_fp8"]
+        cb = cpu_baselines({n: W[n] if n != main.name else main for n in names}, unions, lbytes)
+        head = cb["workloads"][main.name]["all_cores"]
+        out["cpu_baseline"] = {
+            "value": head["us_per_layer"], "unit": UNIT, "cores": cb["nproc"], "kind": "oracle",
+            "sample": f"{head['calls']} full {main.name} layer call(s) (M={main.M}), fp64 oracle "
+                      f"generating its weights as it goes, {cb['nproc']} threads",
+            "cpu_model": cb["cpu_model"], "per_workload": cb["workloads"]}
     if pg is not None:
         pg.destroy_process_group()
     if rank == 0:

@@ -22,7 +22,10 @@
  *   S_t   = top-k(l_t) (ties -> lower expert id)
  *   g_e   = exp(l_e) / sum_{i in S_t} exp(l_i)            e in S_t
  *   F(v)  = Wd (silu(Wg v) * (Wu v))
- *   hidden[t] <- bf16( h1_t + F_shared(h1_t) + sum_{e in S_t} g_e F_e(h1_t) )
+ *   hidden[t] <- bf16( h1_t + F_shared(h1_t) + s sum_{e in S_t} g_e F_e(h1_t) )
+ * (s = routed_scale, 1 by default; with bias_select_only, S_t = top-k(l + b)
+ * and g over the unbiased l -- the selection-only expert bias of
+ * DeepSeek-V3-style routers.)
  *
  * Conventions
  *   - Every function returns KD_OK (0) or a negative KD_E* code; the message
@@ -68,8 +71,22 @@ typedef struct kd_config {
   int max_tokens;    /* largest M a call may use, 1..64; sizes the workspaces    */
   const float* router_bias; /* host [E] additive router bias, or NULL; copied    */
   int mma_min_tokens;/* calls with M >= this use the tensor-core (tcgen05) kernels,
-                        smaller M the CUDA-core streaming kernels; 0 = default (4),
+                        smaller M the CUDA-core streaming kernels; 0 = default (3),
                         > 64 = never.                                           */
+  /* Full layer (kd_decode_layer_full); all zero for the layer above.         */
+  int full_layer;    /* 1: RMSNorm gains are generated and the layer takes the
+                        full-layer call; 0: kd_decode_layer only                */
+  float rms_eps;     /* RMSNorm epsilon; 0 = 1e-6                                */
+  int kv_n_seq;      /* KV cache geometry: sequences ...                         */
+  int kv_max_ctx;    /* ... and positions per sequence                           */
+  float k_scale;     /* e4m3 cache scales: dequantised value = code value x scale */
+  float v_scale;
+  /* Gating variants (both layer kinds); zero keeps the plain gating.         */
+  int bias_select_only; /* 1: router_bias chooses the experts only; the gates
+                           are the softmax of the unbiased logits over the
+                           selection (the logits buffer then holds unbiased
+                           logits)                                             */
+  float routed_scale;   /* factor on the routed experts' sum; 0 = 1           */
 } kd_config;
 
 typedef struct kd_layer kd_layer;
@@ -79,7 +96,10 @@ typedef struct kd_stack kd_stack;
  * the device from (seed, layer_id) with the counter-based generator of
  * kdgen/kd_gen.h (synchronous).  The layer owns weights, workspaces, a side
  * stream and events; *out receives the handle.  Errors: KD_EINVAL for a bad
- * config, KD_ENOMEM, KD_ECUDA. */
+ * config, KD_ENOMEM, KD_ECUDA; on any error everything allocated so far is
+ * released.  Test hook: with the environment variable KD_TEST_FAIL_ALLOC_AT=n
+ * (n >= 1) the n-th device allocation of the call fails as if the device
+ * were out of memory. */
 int kd_layer_create(const kd_config* cfg, uint64_t seed, kd_layer** out);
 
 /* Release everything kd_layer_create allocated (NULL is ignored).  The caller
@@ -97,6 +117,33 @@ void kd_layer_destroy(kd_layer* layer);
  * Device-side failures are reported by kd_layer_check. */
 int kd_decode_layer(kd_layer* layer, void* hidden_inout, const void* attn_out, int M,
                     void* stream);
+
+/* One decode step of the FULL layer (pre-norm residual block with its
+ * attention half) for M tokens, enqueued on `stream`.  Token t belongs to
+ * sequence seq[t] and sits at position pos[t] of it:
+ *   u = RMSNorm(x) g1;  (q, k, v) = Wqkv u
+ *   K[seq, pos] = e4m3(k / k_scale),  V[seq, pos] = e4m3(v / v_scale)
+ *   o_h = softmax_j(q_h . K'_j / sqrt(head_dim)) V'_j over j = 0..pos of the
+ *         token's sequence, kv head h / (q_heads / kv_heads)
+ *   h1 = x + Wo o;  w = RMSNorm(h1) g2;  out = h1 + F_shared(w) + sum g_e F_e(w)
+ * with the router on w (bigchange.ai "where the time went": attention with an
+ * FP8 KV cache among the steps of decode; wireai.ir "4 key changes", items
+ * 1-3).  Every new key and value is written before any token attends, so
+ * tokens of one sequence at consecutive positions (a speculative-verify
+ * step) see each other causally.  No positional rotation is applied.
+ *   hidden_inout  bf16 [M, H] device: x on entry, the layer output on exit
+ *   k_cache,      device e4m3 codes [kv_n_seq][kv_max_ctx][kv_heads][head_dim]
+ *   v_cache       (caller-owned; the call writes the M new positions)
+ *   seq, pos      device int32 [M]; 0 <= seq < kv_n_seq, 0 <= pos < kv_max_ctx
+ * The layer must have been created with full_layer = 1, kv_heads >= 1,
+ * q_heads / kv_heads in {1, 2, 4, 8} and head_dim 64 or 128.  Same
+ * capturability and workspace rules as kd_decode_layer.  Errors: KD_EINVAL
+ * (null pointers, a layer without full_layer), KD_ERANGE (M outside
+ * 1..max_tokens), KD_ECUDA.  Out-of-range seq / pos entries are skipped on
+ * the device (that token's attention output is zero) and reported by
+ * kd_layer_check as KD_EDEVICE. */
+int kd_decode_layer_full(kd_layer* layer, void* hidden_inout, void* k_cache, void* v_cache,
+                         const int* seq, const int* pos, int M, void* stream);
 
 /* Synchronise the device and report (then clear) the layer's device error
  * word: KD_OK, KD_ETIMEOUT (a bounded wait inside a kernel gave up) or
@@ -118,6 +165,7 @@ int kd_layer_prefetch_l2(const kd_layer* layer, size_t max_bytes, void* stream);
  *          KD_T_IDX int32 [M,k] | KD_T_GATES fp32 [M,k]
  *          KD_T_COUNTS int32 [E] | KD_T_NACTIVE int32 [1]
  *          KD_T_YSHARED fp32 [M,H] | KD_T_YROUTED fp32 [M*k,H]
+ *          (full layer: KD_T_H1F / KD_T_H1B hold the MoE input w = RMSNorm(h1) g2)
  * *dev_ptr receives the layer-owned pointer. */
 #define KD_T_H1F 0
 #define KD_T_H1B 1
@@ -128,6 +176,11 @@ int kd_layer_prefetch_l2(const kd_layer* layer, size_t max_bytes, void* stream);
 #define KD_T_NACTIVE 6
 #define KD_T_YSHARED 7
 #define KD_T_YROUTED 8
+#define KD_T_ATTN 9          /* full layer: fp32 [M, q_heads*head_dim] attention output */
+#define KD_T_RESID 10        /* full layer: fp32 [M, H] h1 (residual stream after attention) */
+#define KD_T_ACT 11          /* fp32 [M*k, I] routed SwiGLU activations, by (expert, token) position */
+#define KD_T_ACTSH 12        /* fp32 [M, I] the shared expert's SwiGLU activations */
+
 int kd_layer_debug_tensor(const kd_layer* layer, int which, void** dev_ptr);
 
 /* Device copy of one generated weight matrix in its LOGICAL layout, for
@@ -146,7 +199,8 @@ int kd_layer_bytes(const kd_layer* layer, uint64_t* static_bytes, uint64_t* expe
 /* Number of kernels one kd_decode_layer call with M tokens launches (all of
  * them this library's) -- the per-layer kernel count by which the write-ups
  * compare decode paths (bigchange.ai "where the time went"; wireai.ir
- * "compressing the decode loop with kernel fusion").  Returns the count
+ * "compressing the decode loop with kernel fusion"); for a layer created
+ * with full_layer, the count of one kd_decode_layer_full call.  Returns the count
  * (>= 4), or KD_EINVAL for a null layer, KD_ERANGE for M outside
  * 1..max_tokens. */
 int kd_layer_launches(const kd_layer* layer, int M);

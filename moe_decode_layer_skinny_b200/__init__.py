@@ -19,10 +19,12 @@ SO_PATH = os.path.join(HERE, "libkd.so")
 KD_OK, KD_EINVAL, KD_ERANGE, KD_ECUDA, KD_ENOMEM, KD_ETIMEOUT, KD_EDEVICE = 0, -1, -2, -3, -4, -5, -6
 KD_WBF16, KD_WFP8 = 0, 1
 KD_STATIC_MAX_TOKENS, KD_STATIC_MAX_EXPERTS, KD_STATIC_MAX_HIDDEN = 64, 1024, 8192
-T_H1F, T_H1B, T_LOGITS, T_IDX, T_GATES, T_COUNTS, T_NACTIVE, T_YSHARED, T_YROUTED = range(9)
+T_H1F, T_H1B, T_LOGITS, T_IDX, T_GATES, T_COUNTS, T_NACTIVE, T_YSHARED, T_YROUTED, T_ATTN, \
+    T_RESID, T_ACT, T_ACTSH = range(13)
 
 # every symbol include/kd.h declares
-EXPORTS = ("kd_layer_create", "kd_layer_destroy", "kd_decode_layer", "kd_layer_check",
+EXPORTS = ("kd_layer_create", "kd_layer_destroy", "kd_decode_layer", "kd_decode_layer_full",
+           "kd_layer_check",
            "kd_layer_qkv", "kd_layer_prefetch_l2", "kd_layer_debug_tensor", "kd_layer_read_weight",
            "kd_layer_bytes", "kd_layer_launches", "kd_layer_set_timing_events", "kd_stack_create",
            "kd_stack_run", "kd_stack_destroy", "kd_router_topk_static", "kd_last_error")
@@ -40,7 +42,11 @@ class _Config(ctypes.Structure):
                 ("head_dim", ctypes.c_int), ("n_experts", ctypes.c_int), ("top_k", ctypes.c_int),
                 ("n_shared", ctypes.c_int), ("inter", ctypes.c_int), ("wdtype", ctypes.c_int),
                 ("layer_id", ctypes.c_int), ("max_tokens", ctypes.c_int),
-                ("router_bias", ctypes.c_void_p), ("mma_min_tokens", ctypes.c_int)]
+                ("router_bias", ctypes.c_void_p), ("mma_min_tokens", ctypes.c_int),
+                ("full_layer", ctypes.c_int), ("rms_eps", ctypes.c_float),
+                ("kv_n_seq", ctypes.c_int), ("kv_max_ctx", ctypes.c_int),
+                ("k_scale", ctypes.c_float), ("v_scale", ctypes.c_float),
+                ("bias_select_only", ctypes.c_int), ("routed_scale", ctypes.c_float)]
 
 
 _lib = None
@@ -58,6 +64,7 @@ def lib() -> ctypes.CDLL:
         L.kd_layer_destroy.argtypes = [vp]
         L.kd_layer_destroy.restype = None
         L.kd_decode_layer.argtypes = [vp, vp, vp, i32, vp]
+        L.kd_decode_layer_full.argtypes = [vp, vp, vp, vp, vp, vp, i32, vp]
         L.kd_layer_check.argtypes = [vp]
         L.kd_layer_qkv.argtypes = [vp]
         L.kd_layer_qkv.restype = vp
@@ -104,6 +111,14 @@ class LayerSpec:
     max_tokens: int = 64
     router_bias: np.ndarray | None = None
     mma_min_tokens: int = 0
+    full_layer: int = 0
+    rms_eps: float = 0.0
+    kv_n_seq: int = 0
+    kv_max_ctx: int = 0
+    k_scale: float = 0.0
+    v_scale: float = 0.0
+    bias_select_only: int = 0
+    routed_scale: float = 0.0
 
     @classmethod
     def from_dims(cls, dims, **kw) -> "LayerSpec":
@@ -122,7 +137,9 @@ class Layer:
         cfg = _Config(spec.hidden, spec.q_heads, spec.kv_heads, spec.head_dim, spec.n_experts,
                       spec.top_k, spec.n_shared, spec.inter, spec.wdtype, spec.layer_id,
                       spec.max_tokens, None if bias is None else bias.ctypes.data,
-                      spec.mma_min_tokens)
+                      spec.mma_min_tokens, spec.full_layer, spec.rms_eps, spec.kv_n_seq,
+                      spec.kv_max_ctx, spec.k_scale, spec.v_scale, spec.bias_select_only,
+                      spec.routed_scale)
         h = ctypes.c_void_p()
         _check(lib().kd_layer_create(ctypes.byref(cfg), seed, ctypes.byref(h)))
         self._h = h
@@ -149,6 +166,17 @@ class Layer:
             M = hidden.shape[0]
         _check(lib().kd_decode_layer(self._h, hidden.data_ptr(), attn_out.data_ptr(), M,
                                      _stream_ptr(stream)))
+
+    def decode_full(self, hidden, k_cache, v_cache, seq, pos, M: int | None = None,
+                    stream=None) -> None:
+        """kd_decode_layer_full on torch CUDA tensors: hidden bf16 [M,H] (in
+        place), k_cache / v_cache uint8 e4m3 codes [n_seq, max_ctx, kv_heads *
+        head_dim] (the M new positions are written), seq / pos int32 [M]."""
+        if M is None:
+            M = hidden.shape[0]
+        _check(lib().kd_decode_layer_full(self._h, hidden.data_ptr(), k_cache.data_ptr(),
+                                          v_cache.data_ptr(), seq.data_ptr(), pos.data_ptr(), M,
+                                          _stream_ptr(stream)))
 
     def decode_ptr(self, hidden_ptr: int, attn_ptr: int, M: int, stream_ptr: int | None) -> int:
         return lib().kd_decode_layer(self._h, hidden_ptr, attn_ptr, M, stream_ptr)

@@ -19,6 +19,7 @@ enum : unsigned {
   ERR_WAIT_EMPTY = 2u,  // producer gave up waiting for a free stage
   ERR_WAIT_MMA = 4u,    // tensor-core pipeline wait gave up
   ERR_BAD_ROUTE = 8u,   // routing produced an out-of-range expert id
+  ERR_BAD_KV = 16u,     // full layer: a token's sequence / position outside the KV cache
 };
 
 // Every spin-wait gives up after this many nanoseconds of %globaltimer.
@@ -133,7 +134,55 @@ KD_DEV uint16_t f32_to_bf16_bits(float f) {
   return *reinterpret_cast<uint16_t*>(&b);
 }
 
+KD_DEV void store_hilo(uint16_t* hi, uint16_t* lo, size_t o, float v) {
+  const uint16_t h = f32_to_bf16_bits(v);
+  hi[o] = h;
+  lo[o] = f32_to_bf16_bits(v - __uint_as_float((uint32_t)h << 16));
+}
+
+// v = hi + mid + lo exactly (each difference is exact in fp32; three 8-bit
+// significands cover fp32's 24).
+KD_DEV void store_hilo3(uint16_t* hi, uint16_t* mid, uint16_t* lo, size_t o, float v) {
+  const uint16_t h = f32_to_bf16_bits(v);
+  const float r1 = v - __uint_as_float((uint32_t)h << 16);
+  const uint16_t m = f32_to_bf16_bits(r1);
+  hi[o] = h;
+  mid[o] = m;
+  lo[o] = f32_to_bf16_bits(r1 - __uint_as_float((uint32_t)m << 16));
+}
+
 KD_DEV float silu(float z) { return z / (1.0f + expf(-z)); }
+
+// Power of two 2^P that puts a group's largest magnitude amax in [128, 256)
+// (inside e4m3's range, 448), and its inverse; 1 for an all-zero group.
+KD_DEV float q_scale(float amax, float& inv) {
+  if (!(amax > 0.f) || !(amax < 3.0e38f)) {
+    inv = 1.f;
+    return 1.f;
+  }
+  int e = (int)((__float_as_uint(amax) >> 23) & 0xFFu) - 127;   // floor(log2 amax), normal amax
+  if (e < -126) e = -126;
+  int P = 7 - e;
+  P = P > 100 ? 100 : (P < -100 ? -100 : P);
+  inv = __uint_as_float((uint32_t)(127 - P) << 23);
+  return __uint_as_float((uint32_t)(127 + P) << 23);
+}
+
+// e4m3 (round to nearest even, saturating) of two values: byte 0 = lo, byte 1 = hi.
+KD_DEV uint32_t e4m3x2_rn(float lo, float hi) {
+  uint16_t d;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(d) : "f"(hi), "f"(lo));
+  return d;
+}
+
+// The two e4m3 codes of e4m3x2_rn back to fp32 (exact).
+KD_DEV float2 e4m3x2_value(uint32_t v) {
+  uint32_t h;
+  const uint16_t b = (uint16_t)v;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(b));
+  __half2 hh = *reinterpret_cast<__half2*>(&h);
+  return __half22float2(hh);
+}
 
 // Two fp32 values in one 64-bit register, for the packed fp32 FMA of sm_100
 // (fma.rn.f32x2: two IEEE fp32 FMAs per instruction).

@@ -77,6 +77,8 @@ struct LayerDev {
   const float* sqkv; const float* so; const float* sr;
   const float* sgu_sh; const float* sd_sh; const float* sgu; const float* sd;
   const float* bias;                       // [E] or null
+  int bias_sel;                            // 1: the bias enters the selection only
+  float rscale;                            // factor on the routed experts' sum
   // workspaces
   uint16_t* qkv; float* h1f; uint16_t* h1b;
   float* logits; int* idx; float* gates;
@@ -89,6 +91,23 @@ struct LayerDev {
   float* ws_main; float* ws_side;          // split-K partials, main / side stream launches
   unsigned* tcnt_main; unsigned* tcnt_side;// split-K tile arrivals (self-resetting)
   float* yr; float* ysh;                   // [Mmax*k, H] by token*k+slot, [Mmax, H]
+  // FP8 tensor-core experts: max |v| per (row, 64 consecutive elements) of
+  // their fp32 inputs, [rows][K/64]
+  float* h1g;                              // h1 (gate/up input) [Mmax]
+  float* actg;                             // routed SwiGLU activations [Mmax*k]
+  float* actshg;                           // the shared expert's [Mmax]
+  // the residual the combine adds: h1f (the chain with a given attn_out) or
+  // h1r (the full layer, where h1f holds the MoE input RMSNorm(h1) g2)
+  const float* resid;
+  // full layer (kd_decode_layer_full)
+  int Hq, Hkv, hd, n_seq, max_ctx, att_ch, att_nch;
+  float eps, k_scale, v_scale;
+  const uint16_t* g1; const uint16_t* g2;  // RMSNorm gains, bf16 [H]
+  float* uf; uint16_t* u_hi; uint16_t* u_lo;   // RMSNorm(x) g1 [Mmax, H]
+  float* qkvf;                             // fp32 QKV projection [Mmax, Nqkv]
+  float* attnf; uint16_t* attn_hi; uint16_t* attn_lo;   // attention output [Mmax, A]
+  float* att_ws; unsigned* att_cnt;        // per-chunk partials, (token, kv head) arrivals
+  float* h1r;                              // h1 = x + Wo o [Mmax, H]
   unsigned* hcnt;                          // [H/64] down rows done per block (self-resetting)
   unsigned* rcnt;                          // router blocks done (self-resetting)
   unsigned* err;
@@ -99,29 +118,59 @@ struct Acts {                              // per-call activations
   const uint16_t* attn;                    // [M, A]
   uint16_t* out;                           // [M, H] (layer output, = x in place)
   int M;
+  // full layer: the caller's e4m3 KV cache and each token's (sequence, position)
+  uint8_t* kc; uint8_t* vc;
+  const int* seq; const int* pos;
 };
+
+// The new token's key or value element (row of the fused QKV output past
+// the query part) into the e4m3 cache at (seq[j], pos[j]).
+KD_DEV void kv_store(const LayerDev& L, const Acts& a, int j, int row, float v) {
+  const int qw = L.Hq * L.hd, kw = L.Hkv * L.hd;
+  if (row < qw) return;
+  int r2 = row - qw;
+  const bool isv = r2 >= kw;
+  if (isv) r2 -= kw;
+  const int s = a.seq[j], p = a.pos[j];
+  if (s < 0 || s >= L.n_seq || p < 0 || p >= L.max_ctx) {
+    set_error(L.err, ERR_BAD_KV);
+    return;
+  }
+  const float q = __fdiv_rn(v, isv ? L.v_scale : L.k_scale);
+  (isv ? a.vc : a.kc)[((size_t)s * L.max_ctx + p) * kw + r2] = (uint8_t)(e4m3x2_rn(q, 0.f) & 0xFFu);
+}
+
+
 
 KD_DEV int split_lo(int n, int parts, int i) { return (int)(((long long)n * i) / parts); }
 
 // ------------------------------------------------------------------ QKV + o-proj
 
-struct ProjPlan {
+// MODE 0: QKV + o-proj with residual (the chain with a given attn_out), bf16
+// activations x / attn_out.  Full layer: MODE 1 QKV of u = RMSNorm(x) g1
+// (fp32), which also writes the new keys / values into the KV cache; MODE 2
+// o-proj of the attention output (fp32) + residual x into h1r.
+template <int MODE>
+struct ProjPlanT {
   const LayerDev* L; Acts a;
   int q0, q1, o0, o1;
-  KD_DEV int num_segments() const { return 2; }
+  KD_DEV int num_segments() const { return MODE == 0 ? 2 : 1; }
   KD_DEV Seg segment(int i) const {
     Seg s;
-    if (i == 0) {
+    const int which = MODE == 0 ? i : MODE - 1;
+    if (which == 0) {
       s.row_bytes = L->H * L->eb; s.w = L->wqkv + (size_t)q0 * s.row_bytes;
       s.nrows = q1 - q0; s.row0 = q0;
     } else {
       s.row_bytes = L->A * L->eb; s.w = L->wo + (size_t)o0 * s.row_bytes;
       s.nrows = o1 - o0; s.row0 = o0;
     }
-    s.tok0 = 0; s.ntok = a.M; s.tag = i;
+    s.tok0 = 0; s.ntok = a.M; s.tag = which;
     return s;
   }
   KD_DEV const void* act_row(const Seg& s, int j) const {
+    if (MODE == 1) return L->uf + (size_t)j * L->H;
+    if (MODE == 2) return L->attnf + (size_t)j * L->A;
     return s.tag == 0 ? (const void*)(a.x + (size_t)j * L->H) : (const void*)(a.attn + (size_t)j * L->A);
   }
   KD_DEV const float* scale_row(const Seg& s, int row) const {
@@ -131,29 +180,38 @@ struct ProjPlan {
   KD_DEV void epilogue(const Seg& s, int row, int j, float v) const {
     if (s.tag == 0) {
       L->qkv[(size_t)j * L->Nqkv + row] = f32_to_bf16_bits(v);
+      if (MODE == 1) {
+        L->qkvf[(size_t)j * L->Nqkv + row] = v;
+        kv_store(*L, a, j, row, v);
+      }
     } else {
       const size_t o = (size_t)j * L->H + row;
       const float h = __uint_as_float((uint32_t)a.x[o] << 16) + v;
-      L->h1f[o] = h;
-      L->h1b[o] = f32_to_bf16_bits(h);
+      if (MODE == 2) {
+        L->h1r[o] = h;
+      } else {
+        L->h1f[o] = h;
+        L->h1b[o] = f32_to_bf16_bits(h);
+      }
     }
   }
   KD_DEV void epilogue2(const Seg&, int, int, float, float) const {}
   KD_DEV bool wants_segment_done() const { return false; }
   KD_DEV void segment_done(const Seg&) const {}
 };
+using ProjPlan = ProjPlanT<0>;
 
 // The weights are static, so the first stages are requested before waiting
-// for the preceding kernel (programmatic dependent launch); x and attn_out
+// for the preceding kernel (programmatic dependent launch); the activations
 // are read only after the wait.
-template <int WT>
+template <int WT, int MODE = 0>
 __global__ void __launch_bounds__(kThreads, 1) proj_kernel(LayerDev L, Acts a) {
   extern __shared__ uint8_t smem[];
-  ProjPlan p;
+  ProjPlanT<MODE> p;
   p.L = &L; p.a = a;
   p.q0 = split_lo(L.Nqkv, gridDim.x, blockIdx.x); p.q1 = split_lo(L.Nqkv, gridDim.x, blockIdx.x + 1);
   p.o0 = split_lo(L.H, gridDim.x, blockIdx.x); p.o1 = split_lo(L.H, gridDim.x, blockIdx.x + 1);
-  stream_run<WT, A_BF16>(p, smem, L.err, true);
+  stream_run<WT, MODE == 0 ? A_BF16 : A_F32>(p, smem, L.err, true);
 }
 
 // ------------------------------------------------------------------ router
@@ -266,10 +324,18 @@ KD_DEV void topk_group(const LayerDev& L, const float* lg, const Route& R, int t
   const int k = L.k, E = L.E;
   const bool act = t < M;
   uint64_t key[PER];
+  // selection keys: the logits, or with a selection-only bias logits + bias
+  // (the logits buffer then holds the unbiased logits, which the gates use)
+  const bool sel_bias = L.bias_sel && L.bias;
 #pragma unroll
   for (int qq = 0; qq < PER; ++qq) {
     const int e = sl + LPT * qq;
-    key[qq] = (act && e < E) ? route_key(lg[(size_t)t * E + e], e) : 0ull;
+    float v = 0.f;
+    if (act && e < E) {
+      v = lg[(size_t)t * E + e];
+      if (sel_bias) v += __ldg(L.bias + e);
+    }
+    key[qq] = (act && e < E) ? route_key(v, e) : 0ull;
   }
   float top = 0.f, den = 0.f;
 #pragma unroll 1
@@ -285,11 +351,15 @@ KD_DEV void topk_group(const LayerDev& L, const float* lg, const Route& R, int t
 #pragma unroll
     for (int qq = 0; qq < PER; ++qq)
       if (key[qq] == best) key[qq] = 0ull;   // keys are unique (expert id)
-    const float v = key_value(best);
-    if (j == 0) top = v;
+    const int be = key_expert(best);
+    const float v = sel_bias ? (act ? lg[(size_t)t * E + be] : 0.f) : key_value(best);
+    if (j == 0 || v > top) {   // the gates' reference value: their largest logit
+      den = j == 0 ? 0.f : den * expf(top - v);
+      top = v;
+    }
     den += expf(v - top);
     if (act && sl == 0) {
-      const int e = key_expert(best);
+      const int e = be;
       R.sel[t * k + j] = e;
       R.gv[t * k + j] = v;
       if (write_global) L.idx[t * k + j] = e;
@@ -512,7 +582,7 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(LayerDev L, int 
     if (e < L.E)
       L.logits[(size_t)t * L.E + e] =
           ((part[r][0][t] + part[r][1][t]) + (part[r][2][t] + part[r][3][t])) +
-          (L.bias ? L.bias[e] : 0.f);
+          (L.bias && !L.bias_sel ? L.bias[e] : 0.f);
   }
   route_last_block(L, M, gridDim.x);
   pdl_launch_dependents();
@@ -644,10 +714,10 @@ struct DownPlan {
       for (int e = threadIdx.x; e < 64 * M; e += kThreads) {
         const int t = e / 64, h = b * 64 + e % 64;
         const size_t o = (size_t)t * L->H + h;
-        float v = L->h1f[o];
+        float v = L->resid[o];
         if (L->S) v += __ldcg(L->ysh + o);
         for (int j = 0; j < L->k; ++j)
-          v += L->gates[t * L->k + j] * __ldcg(L->yr + ((size_t)t * L->k + j) * L->H + h);
+          v += (L->rscale * L->gates[t * L->k + j]) * __ldcg(L->yr + ((size_t)t * L->k + j) * L->H + h);
         out[o] = f32_to_bf16_bits(v);
       }
     }

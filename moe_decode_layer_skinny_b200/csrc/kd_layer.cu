@@ -14,11 +14,13 @@
 
 #include <algorithm>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <string>
 #include <vector>
 
 #include "../../include/kd.h"
+#include "kd_full.cuh"
 #include "kd_kernels.cuh"
 #include "kd_mma_kernels.cuh"
 
@@ -55,6 +57,12 @@ struct kd_layer {
   bool has_maps = false;
   MmaMaps maps{};
   size_t ntile = 0;      // split-K tile arrival counters per stream
+  // test hook: the n-th device allocation of kd_layer_create fails (0 = none)
+  int fail_alloc_at = 0, nalloc = 0;
+  // full layer
+  bool full = false;
+  size_t att_smem = 0;
+  int att_ncnt = 0;      // (token, kv head) arrival counters
 };
 
 struct kd_stack {
@@ -77,6 +85,11 @@ void kd_set_last_error(const char* msg) { g_err = msg; }
 
 static int dalloc(kd_layer* L, size_t bytes, void** p) {
   if (bytes == 0) bytes = 16;
+  if (L->fail_alloc_at > 0 && ++L->nalloc == L->fail_alloc_at) {
+    *p = nullptr;
+    return fail(KD_ENOMEM, "cudaMalloc of %s%ld bytes failed (injected by KD_TEST_FAIL_ALLOC_AT)", "",
+                (long)bytes);
+  }
   cudaError_t e = cudaMalloc(p, bytes);
   if (e != cudaSuccess) {
     cudaGetLastError();
@@ -144,6 +157,33 @@ static int gen_matrix(const kd_layer* L, uint8_t* dst, float* scales, int R, int
   return KD_OK;
 }
 
+// RMSNorm gains: dst[i] = bf16(1 + value(stream, i)).
+static __global__ void gen_norm_kernel(uint16_t* dst, int n, uint64_t stream) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x)
+    dst[i] = kdg_norm_bf16(stream, (uint64_t)i);
+}
+
+typedef void (*AttnKernel)(LayerDev, Acts);
+
+static AttnKernel attention_for(int hd, int grp) {
+  if (hd == 128) {
+    switch (grp) {
+      case 1: return attention_kernel<128, 1>;
+      case 2: return attention_kernel<128, 2>;
+      case 4: return attention_kernel<128, 4>;
+      case 8: return attention_kernel<128, 8>;
+    }
+  } else if (hd == 64) {
+    switch (grp) {
+      case 1: return attention_kernel<64, 1>;
+      case 2: return attention_kernel<64, 2>;
+      case 4: return attention_kernel<64, 4>;
+      case 8: return attention_kernel<64, 8>;
+    }
+  }
+  return nullptr;
+}
+
 static void free_layer(kd_layer* L) {
   if (!L) return;
   for (void* p : L->allocs) cudaFree(p);
@@ -154,6 +194,7 @@ static void free_layer(kd_layer* L) {
 }
 
 static bool stream_kernels_configured = false;
+constexpr int kMaxAttChunk = 1024;   // attention positions per CTA (at most)
 
 // Routed gate/up CTAs keep the call's routing after the stream area.
 static size_t gateup_smem(const LayerDev& d, int M) {
@@ -181,6 +222,18 @@ static int configure_kernels() {
   KD_CUDA(cudaFuncSetAttribute(mma_proj_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem));
   KD_CUDA(cudaFuncSetAttribute(mma_gateup_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem));
   KD_CUDA(cudaFuncSetAttribute(mma_down_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem));
+  KD_CUDA(cudaFuncSetAttribute(proj_kernel<W_BF16, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  KD_CUDA(cudaFuncSetAttribute(proj_kernel<W_BF16, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  KD_CUDA(cudaFuncSetAttribute(proj_kernel<W_FP8, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  KD_CUDA(cudaFuncSetAttribute(proj_kernel<W_FP8, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  KD_CUDA(cudaFuncSetAttribute(mma_proj_kernel<false, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem));
+  KD_CUDA(cudaFuncSetAttribute(mma_proj_kernel<false, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem));
+  KD_CUDA(cudaFuncSetAttribute(mma_proj_kernel<true, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem));
+  KD_CUDA(cudaFuncSetAttribute(mma_proj_kernel<true, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem));
+  for (int hd : {64, 128})
+    for (int grp : {1, 2, 4, 8})
+      KD_CUDA(cudaFuncSetAttribute(attention_for(hd, grp), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   (int)attention_smem(kMaxAttChunk, grp, hd)));
   stream_kernels_configured = true;
   return KD_OK;
 }
@@ -196,18 +249,28 @@ extern "C" int kd_layer_create(const kd_config* cfg, uint64_t seed, kd_layer** o
       A % 128 || Nqkv % 128 || c.n_experts < 1 || c.n_experts > 1024 || c.top_k < 1 ||
       c.top_k > 16 || c.top_k > c.n_experts || c.n_shared < 0 || c.n_shared > 1 || c.inter <= 0 ||
       c.inter % 128 || (c.wdtype != KD_WBF16 && c.wdtype != KD_WFP8) || c.max_tokens < 1 ||
-      c.max_tokens > 64 || c.layer_id < 0 || c.mma_min_tokens < 0)
+      c.max_tokens > 64 || c.layer_id < 0 || c.mma_min_tokens < 0 ||
+      (c.bias_select_only != 0 && c.bias_select_only != 1))
     return fail(KD_EINVAL, "kd_layer_create: unsupported configuration%s", "");
   if (c.hidden * 2 > kStageBytes || A * 2 > kStageBytes || c.inter * 2 > kStageBytes ||
       c.hidden > 8192 || A > 8192 || c.inter > 8192)
     return fail(KD_EINVAL, "kd_layer_create: a weight row exceeds one %s%ld-byte stage", "",
                 (long)kStageBytes);
+  if (c.full_layer) {
+    const int grp = c.kv_heads > 0 ? c.q_heads / c.kv_heads : 0;
+    if (c.full_layer != 1 || c.kv_heads < 1 || c.q_heads % c.kv_heads ||
+        (grp != 1 && grp != 2 && grp != 4 && grp != 8) || (c.head_dim != 64 && c.head_dim != 128) ||
+        c.kv_n_seq < 1 || c.kv_max_ctx < 1 || !(c.k_scale > 0.f) || !(c.v_scale > 0.f) ||
+        c.rms_eps < 0.f)
+      return fail(KD_EINVAL, "kd_layer_create: unsupported full-layer configuration%s", "");
+  }
 
   kd_layer* L = new kd_layer();
   L->cfg = c;
+  if (const char* f = getenv("KD_TEST_FAIL_ALLOC_AT")) L->fail_alloc_at = atoi(f);
   L->cfg.router_bias = nullptr;
   L->maxM = c.max_tokens;
-  L->mma_min = c.mma_min_tokens > 0 ? c.mma_min_tokens : 4;
+  L->mma_min = c.mma_min_tokens > 0 ? c.mma_min_tokens : 3;
   L->Nqkv = Nqkv;
   L->A = A;
   int rc = KD_OK;
@@ -282,6 +345,8 @@ extern "C" int kd_layer_create(const kd_config* cfg, uint64_t seed, kd_layer** o
     TRYC(cudaMemcpy(bias, cfg->router_bias, sizeof(float) * E, cudaMemcpyHostToDevice));
   }
   d.bias = bias;
+  d.bias_sel = c.bias_select_only ? 1 : 0;
+  d.rscale = c.routed_scale != 0.f ? c.routed_scale : 1.f;
 
   TRY(dalloc_t(L, (size_t)M * Nqkv, &d.qkv));
   TRY(dalloc_t(L, (size_t)M * H, &d.h1f));
@@ -306,6 +371,45 @@ extern "C" int kd_layer_create(const kd_config* cfg, uint64_t seed, kd_layer** o
   TRY(dalloc_t(L, (size_t)M * k * I, &d.act_lo));
   TRY(dalloc_t(L, (size_t)M * I, &d.act_sh_hi));
   TRY(dalloc_t(L, (size_t)M * I, &d.act_sh_lo));
+  if (fp8) {
+    // per-64 maxima of the FP8 tensor-core experts' inputs
+    TRY(dalloc_t(L, (size_t)M * (H / kQGroup), &d.h1g));
+    TRY(dalloc_t(L, (size_t)M * k * (I / kQGroup), &d.actg));
+    TRY(dalloc_t(L, (size_t)M * (I / kQGroup), &d.actshg));
+  }
+  d.resid = d.h1f;
+  if (c.full_layer) {
+    L->full = true;
+    d.Hq = c.q_heads; d.Hkv = c.kv_heads; d.hd = c.head_dim;
+    d.n_seq = c.kv_n_seq; d.max_ctx = c.kv_max_ctx;
+    d.k_scale = c.k_scale; d.v_scale = c.v_scale;
+    d.eps = c.rms_eps > 0.f ? c.rms_eps : 1e-6f;
+    // positions per attention CTA: about two CTAs per SM for one token
+    const int grp = c.q_heads / c.kv_heads;
+    int want = (2 * L->nsm + c.kv_heads - 1) / c.kv_heads;
+    int ch = (c.kv_max_ctx + want - 1) / want;
+    ch = std::max(32, std::min(kMaxAttChunk, (ch + 31) & ~31));
+    d.att_ch = ch;
+    d.att_nch = (c.kv_max_ctx + ch - 1) / ch;
+    L->att_smem = attention_smem(ch, grp, c.head_dim);
+    uint16_t *g1, *g2;
+    TRY(dalloc_t(L, (size_t)H, &g1));
+    TRY(dalloc_t(L, (size_t)H, &g2));
+    d.g1 = g1; d.g2 = g2;
+    TRY(dalloc_t(L, (size_t)M * H, &d.uf));
+    TRY(dalloc_t(L, (size_t)M * H, &d.u_hi));
+    TRY(dalloc_t(L, (size_t)M * H, &d.u_lo));
+    TRY(dalloc_t(L, (size_t)M * Nqkv, &d.qkvf));
+    TRY(dalloc_t(L, (size_t)M * A, &d.attnf));
+    TRY(dalloc_t(L, (size_t)M * A, &d.attn_hi));
+    TRY(dalloc_t(L, (size_t)M * A, &d.attn_lo));
+    TRY(dalloc_t(L, (size_t)M * c.kv_heads * d.att_nch * grp * (c.head_dim + 2), &d.att_ws));
+    L->att_ncnt = M * c.kv_heads;
+    TRY(dalloc_t(L, (size_t)L->att_ncnt, &d.att_cnt));
+    TRYC(cudaMemset(d.att_cnt, 0, sizeof(unsigned) * L->att_ncnt));
+    TRY(dalloc_t(L, (size_t)M * H, &d.h1r));
+    d.resid = d.h1r;
+  }
   TRY(dalloc_t(L, (size_t)L->nsm * kWsFloatsPerCta, &d.ws_main));
   TRY(dalloc_t(L, (size_t)L->nsm * kWsFloatsPerCta, &d.ws_side));
   {
@@ -341,6 +445,13 @@ extern "C" int kd_layer_create(const kd_config* cfg, uint64_t seed, kd_layer** o
     rc = gen(gu, sg, I, H, KDG_GATE, slot, 2, 0);
     if (rc == KD_OK) rc = gen(gu, sg ? sg + (size_t)d.nIb * d.nHb : nullptr, I, H, KDG_UP, slot, 2, 1);
     if (rc == KD_OK) rc = gen(dn, sdn, H, I, KDG_DOWN, slot, 1, 0);
+  }
+  if (rc == KD_OK && c.full_layer) {
+    gen_norm_kernel<<<32, 256, 0, gs>>>(const_cast<uint16_t*>(d.g1), H,
+                                        kdg_stream(seed, kdg_uid((uint32_t)c.layer_id, KDG_NORM1, 0)));
+    gen_norm_kernel<<<32, 256, 0, gs>>>(const_cast<uint16_t*>(d.g2), H,
+                                        kdg_stream(seed, kdg_uid((uint32_t)c.layer_id, KDG_NORM2, 0)));
+    if (cudaGetLastError() != cudaSuccess) rc = fail(KD_ECUDA, "kd_layer_create: norm generator%s", "");
   }
   cudaError_t se = cudaStreamSynchronize(gs);
   cudaStreamDestroy(gs);
@@ -398,33 +509,93 @@ static cudaError_t launch(void (*kernel)(KArgs...), int grid, int block, size_t 
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
-static int launch_layer(kd_layer* L, void* hidden, const void* attn, int M, cudaStream_t s,
-                        const kd_layer* prefetch_next, cudaStream_t pf, cudaEvent_t ev_fork,
-                        cudaEvent_t ev_join, bool pdl_first);
+static int launch_layer(kd_layer* L, const Acts& a, cudaStream_t s, const kd_layer* prefetch_next,
+                        cudaStream_t pf, cudaEvent_t ev_fork, cudaEvent_t ev_join, bool pdl_first);
 
 extern "C" int kd_decode_layer(kd_layer* L, void* hidden, const void* attn, int M, void* stream) {
   if (!L || !hidden || !attn) return fail(KD_EINVAL, "kd_decode_layer: null argument%s", "");
   if (M < 1 || M > L->maxM)
     return fail(KD_ERANGE, "kd_decode_layer: M=%s%ld outside 1..max_tokens", "", (long)M);
-  return launch_layer(L, hidden, attn, M, static_cast<cudaStream_t>(stream), nullptr, nullptr,
-                      nullptr, nullptr, false);
-}
-
-static int launch_layer(kd_layer* L, void* hidden, const void* attn, int M, cudaStream_t s,
-                        const kd_layer* next, cudaStream_t pf, cudaEvent_t ev_fork,
-                        cudaEvent_t ev_join, bool pdl_first) {
-  const LayerDev& d = L->d;
-  const bool fp8 = L->cfg.wdtype == KD_WFP8;
-  Acts a;
+  Acts a{};
   a.x = static_cast<const uint16_t*>(hidden);
   a.attn = static_cast<const uint16_t*>(attn);
   a.out = static_cast<uint16_t*>(hidden);
   a.M = M;
+  return launch_layer(L, a, static_cast<cudaStream_t>(stream), nullptr, nullptr, nullptr, nullptr,
+                      false);
+}
+
+extern "C" int kd_decode_layer_full(kd_layer* L, void* hidden, void* k_cache, void* v_cache,
+                                    const int* seq, const int* pos, int M, void* stream) {
+  if (!L || !hidden || !k_cache || !v_cache || !seq || !pos)
+    return fail(KD_EINVAL, "kd_decode_layer_full: null argument%s", "");
+  if (!L->full)
+    return fail(KD_EINVAL, "kd_decode_layer_full: the layer was created without full_layer%s", "");
+  if (M < 1 || M > L->maxM)
+    return fail(KD_ERANGE, "kd_decode_layer_full: M=%s%ld outside 1..max_tokens", "", (long)M);
+  Acts a{};
+  a.x = static_cast<const uint16_t*>(hidden);
+  a.attn = nullptr;
+  a.out = static_cast<uint16_t*>(hidden);
+  a.M = M;
+  a.kc = static_cast<uint8_t*>(k_cache);
+  a.vc = static_cast<uint8_t*>(v_cache);
+  a.seq = seq;
+  a.pos = pos;
+  return launch_layer(L, a, static_cast<cudaStream_t>(stream), nullptr, nullptr, nullptr, nullptr,
+                      false);
+}
+
+// The front of the layer up to h1 (and, in the full layer, the MoE input
+// w = RMSNorm(h1) g2): the chain with a given attn_out runs QKV and o-proj in
+// one launch; the full layer runs RMSNorm -> QKV (+ KV cache append) ->
+// attention -> o-proj + residual -> RMSNorm.
+static int launch_front(kd_layer* L, const Acts& a, cudaStream_t s, bool pdl_first) {
+  const LayerDev& d = L->d;
+  const bool fp8 = L->cfg.wdtype == KD_WFP8;
+  const int G = L->nsm, M = a.M;
+  const bool mma = L->has_maps && M >= L->mma_min;
+  const int pthreads = fp8 ? kMThreadsF8 : kMThreads;
+  if (!L->full) {
+    if (mma)
+      KD_CUDA(launch(fp8 ? mma_proj_kernel<true> : mma_proj_kernel<false>, G, pthreads, kMmaSmem, s,
+                     pdl_first, d, a, L->maps));
+    else
+      KD_CUDA(launch(fp8 ? proj_kernel<W_FP8> : proj_kernel<W_BF16>, G, kThreads, kStreamSmem, s,
+                     pdl_first, d, a));
+    return KD_OK;
+  }
+  KD_CUDA(launch(rmsnorm_in_kernel, M, kNormThreads, 0, s, pdl_first, d, a));
+  if (mma)
+    KD_CUDA(launch(fp8 ? mma_proj_kernel<true, 1> : mma_proj_kernel<false, 1>, G, pthreads, kMmaSmem,
+                   s, true, d, a, L->maps));
+  else
+    KD_CUDA(launch(fp8 ? proj_kernel<W_FP8, 1> : proj_kernel<W_BF16, 1>, G, kThreads, kStreamSmem, s,
+                   true, d, a));
+  KD_CUDA(launch(attention_for(d.hd, d.Hq / d.Hkv), M * d.Hkv * d.att_nch, 256, L->att_smem, s,
+                 true, d, a));
+  if (mma)
+    KD_CUDA(launch(fp8 ? mma_proj_kernel<true, 2> : mma_proj_kernel<false, 2>, G, pthreads, kMmaSmem,
+                   s, true, d, a, L->maps));
+  else
+    KD_CUDA(launch(fp8 ? proj_kernel<W_FP8, 2> : proj_kernel<W_BF16, 2>, G, kThreads, kStreamSmem, s,
+                   true, d, a));
+  KD_CUDA(launch(rmsnorm_moe_kernel, M, kNormThreads, 0, s, true, d, (int)(fp8 && mma)));
+  return KD_OK;
+}
+
+static int launch_layer(kd_layer* L, const Acts& a, cudaStream_t s, const kd_layer* next,
+                        cudaStream_t pf, cudaEvent_t ev_fork, cudaEvent_t ev_join, bool pdl_first) {
+  const LayerDev& d = L->d;
+  const bool fp8 = L->cfg.wdtype == KD_WFP8;
+  const int M = a.M;
   const int G = L->nsm;
   const size_t sm = kStreamSmem;
   const bool mma = L->has_maps && M >= L->mma_min;
   const size_t msm = kMmaSmem;
-  const int mthreads = fp8 ? kMThreadsF8 : kMThreads;
+  // FP8 projections convert their e4m3 tiles (converter warps); the FP8
+  // experts multiply them as they land
+  const int mthreads = kMThreads;
   if (L->timing) KD_CUDA(cudaEventRecord(L->tev[0], s));
   // Main stream: projections -> router (logits, selection, token lists in one
   // launch) -> routed gate/up -> down + combine.  Side stream: the shared
@@ -433,13 +604,13 @@ static int launch_layer(kd_layer* L, void* hidden, const void* attn, int M, cuda
   // when it is done, so the shared gate/up gets the SMs that the router
   // leaves free while the router runs.
   const size_t route_ints = sizeof(int) * kRouteSmemInts(d.E, M * d.k);
-  if (mma)
-    KD_CUDA(launch(fp8 ? mma_proj_kernel<true> : mma_proj_kernel<false>, G, mthreads, msm, s,
-                   pdl_first, d, a, L->maps));
-  else
-    KD_CUDA(launch(fp8 ? proj_kernel<W_FP8> : proj_kernel<W_BF16>, G, kThreads, sm, s, pdl_first, d, a));
+  {
+    const int rc = launch_front(L, a, s, pdl_first);
+    if (rc != KD_OK) return rc;
+  }
   if (L->timing) KD_CUDA(cudaEventRecord(L->tev[1], s));
   if (d.S) KD_CUDA(cudaEventRecord(L->ev_h1, s));
+
   // FP8 routers stay on CUDA cores: the tensor-core path rounds each scaled
   // weight to bf16, which the fp32 router logits cannot afford
   if (mma && !fp8) {
@@ -505,6 +676,7 @@ extern "C" int kd_layer_check(kd_layer* L) {
   KD_CUDA(cudaMemset(L->d.rcnt, 0, sizeof(unsigned)));
   KD_CUDA(cudaMemset(L->d.tcnt_main, 0, sizeof(unsigned) * L->ntile));
   KD_CUDA(cudaMemset(L->d.tcnt_side, 0, sizeof(unsigned) * L->ntile));
+  if (L->full) KD_CUDA(cudaMemset(L->d.att_cnt, 0, sizeof(unsigned) * L->att_ncnt));
   if (e & (ERR_WAIT_FULL | ERR_WAIT_EMPTY | ERR_WAIT_MMA))
     return fail(KD_ETIMEOUT, "device: a bounded wait gave up (flags %s0x%lx)", "", (long)e);
   return fail(KD_EDEVICE, "device error flags %s0x%lx", "", (long)e);
@@ -578,6 +750,11 @@ extern "C" int kd_layer_debug_tensor(const kd_layer* L, int which, void** p) {
     case KD_T_NACTIVE: *p = d.n_active; break;
     case KD_T_YSHARED: *p = d.ysh; break;
     case KD_T_YROUTED: *p = d.yr; break;
+    case KD_T_ATTN: *p = d.attnf; break;
+    case KD_T_RESID: *p = d.h1r; break;
+    case KD_T_ACT: *p = d.act; break;
+    case KD_T_ACTSH: *p = d.act_sh; break;
+
     default: return fail(KD_EINVAL, "kd_layer_debug_tensor: unknown tensor %s%ld", "", (long)which);
   }
   return KD_OK;
@@ -634,8 +811,9 @@ extern "C" int kd_layer_launches(const kd_layer* L, int M) {
     return fail(KD_ERANGE, "kd_layer_launches: M=%s%ld outside 1..max_tokens", "", (long)M);
   const bool mma = L->has_maps && M >= L->mma_min;
   // projections, router, routed gate/up, down (+ combine on the tensor-core
-  // path), + the shared expert's gate/up
-  return 4 + (mma ? 1 : 0) + (L->d.S ? 1 : 0);
+  // path), + the shared expert's gate/up; a full layer runs RMSNorm, QKV,
+  // attention, o-proj and RMSNorm in place of the projections' launch
+  return 4 + (mma ? 1 : 0) + (L->d.S ? 1 : 0) + (L->full ? 4 : 0);
 }
 
 extern "C" int kd_layer_bytes(const kd_layer* L, uint64_t* static_bytes, uint64_t* expert_bytes) {
@@ -700,10 +878,15 @@ extern "C" int kd_stack_run(kd_stack* S, void* hidden, const void* attn, void* s
     int rc = KD_OK;
     for (int l = 0; l < n && rc == KD_OK; ++l) {
       kd_layer* L = S->layers[l];
-      const uint8_t* a = static_cast<const uint8_t*>(attn) + (size_t)l * S->M * L->d.A * 2;
+      Acts a{};
+      a.x = static_cast<const uint16_t*>(hidden);
+      a.attn = reinterpret_cast<const uint16_t*>(static_cast<const uint8_t*>(attn) +
+                                                 (size_t)l * S->M * L->d.A * 2);
+      a.out = static_cast<uint16_t*>(hidden);
+      a.M = S->M;
       const kd_layer* next = (S->prefetch && l + 1 < n) ? S->layers[l + 1] : nullptr;
-      rc = launch_layer(L, hidden, a, S->M, S->cap, next, next ? S->pf : nullptr, S->ev_fork[l],
-                        S->ev_join[l], l > 0);
+      rc = launch_layer(L, a, S->cap, next, next ? S->pf : nullptr, S->ev_fork[l], S->ev_join[l],
+                        l > 0);
     }
     cudaGraph_t g = nullptr;
     cudaError_t ce = cudaStreamEndCapture(S->cap, &g);

@@ -12,13 +12,24 @@
 //               into the stage in the same swizzled K-major layout
 //   warps 4-7   epilogue: tcgen05.ld of the accumulator (lane = weight row),
 //               then the plan's epilogue, or a split-K partial
-//   warps 8-15  FP8 weights only: e4m3 tiles -> scaled bf16 A tiles
+//   warps 8-15  FP8 projections only: e4m3 tiles -> scaled bf16 A tiles
 // Activations that must stay fp32-accurate come as a sum of bf16 terms, all
 // multiplied into the same accumulator: the expert inputs (h1, the SwiGLU
 // activations) as hi + lo (hi = bf16(v), lo = bf16(v - hi): ~16 significant
-// bits; hi alone with FP8 weights); the router's h1 as hi + mid + lo (all 24
-// bits of the fp32 value; the products with bf16 weights are exact in the
-// fp32 accumulator).
+// bits); the router's h1 as hi + mid + lo (all 24 bits of the fp32 value; the
+// products with bf16 weights are exact in the fp32 accumulator).
+//
+// FP8 experts ("q8" plans) take the e4m3 weight tile as TMA lands it, with no
+// conversion, into kind::f8f6f4 MMAs (128 x N x 32).  The 128 x 128 block
+// scale of the weights cannot sit on an e4m3 operand, so the B producers put
+// it on the activations: for each stage (one 128 x 128 weight block) they
+// write the live tokens' fp32 activations times (block scale x 2^P) as two
+// e4m3 terms, t0 = e4m3(v), t1 = e4m3(v - t0), with one power of two 2^P per
+// (token, tile) that puts the largest |activation x block scale| of the tile
+// in [128, 256) (from per-64-element maxima the producing kernel writes).
+// Gate and up rows of a paired tile have scales of their own, so a paired
+// tile gets two B variants and two accumulators.  The accumulators stay in
+// TMEM for the whole unit, and the epilogue multiplies by 2^-P once.
 // Work units are (weight tile, K part); a tile split over several parts is
 // summed in part order by the unit that completes it (deterministic).
 #pragma once
@@ -55,6 +66,11 @@ KD_DEV uint32_t idesc_bf16(int n) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((128u >> 4) << 24);
 }
 
+// Instruction descriptor, kind::f8f6f4: e4m3 A and B (K-major), fp32 D, M = 128.
+KD_DEV uint32_t idesc_e4m3(int n) {
+  return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((128u >> 4) << 24);
+}
+
 KD_DEV void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 KD_DEV void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
@@ -73,6 +89,13 @@ KD_DEV void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t i
   asm volatile(
       "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"((uint32_t)acc) : "memory");
+}
+
+KD_DEV void mma_e4m3(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, bool acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}"
       ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"((uint32_t)acc) : "memory");
 }
 
@@ -103,11 +126,15 @@ constexpr int kMThreadsF8 = 512;      // + 8 converter warps (e4m3 -> bf16 A til
 constexpr int kMaxMStages = 16;
 constexpr int kATileBytes = 128 * 128;                // 128 rows x 64 bf16 (one swizzle atom wide)
 constexpr int kMaxSub = 2;                            // 64-K sub-tiles per stage (at most)
-constexpr int kMRingBytes = 224 * 1024;                // stages (+ 2 KB below: 227 KB per CTA)
+constexpr int kMRingBytes = 222 * 1024;                // stages (+ 3 KB below: 225 KB per CTA)
 constexpr int kMaxN = 64;                             // tokens per MMA (N)
 constexpr int kMaxTerms = 3;                          // bf16 terms of an activation
 constexpr size_t kWsFloatsPerCta = 2 * 128 * 64;     // split-K partial slots of one CTA
-constexpr size_t kMmaSmem = (size_t)kMRingBytes + 1024 /*align*/ + 1024 /*barriers, lists*/;
+constexpr size_t kMmaSmem = (size_t)kMRingBytes + 1024 /*align*/ + 2048 /*barriers, scratch*/;
+constexpr int kQ8AccCols = 256;                       // q8: one accumulator, <= 2 x 2 x 64 columns
+constexpr int kQ8TmemCols = 2 * kQ8AccCols;           // q8: two accumulators
+constexpr int kQGroup = 64;                           // activation elements per stored maximum
+constexpr int kQTerms = 2;                            // e4m3 terms of a q8 activation
 
 // One unit of work: K chunks [kc0, kc0 + nkc) of a 128-row weight tile.
 struct MUnit {
@@ -184,8 +211,11 @@ struct CtaUnits {
 struct MmaShared {
   uint8_t* stage;        // nst x stage_bytes, 1024-aligned
   int nst, stage_bytes;  // stage count and size (A tile + B tile for the launch's largest N)
+  int xoff;              // q8: offset of the activation staging area in a stage
   int nsub;              // 64-K sub-tiles per stage
-  uint64_t* full;        // [nst] A landed (tx, or the converter) + B written (64 arrivals)
+  uint64_t* full;        // [nst] B written (64 arrivals), or (FP8 converter) the A tile converted
+  uint64_t* afull;       // [nst] bf16 / q8 plans: the A tile landed (TMA transaction count)
+  uint64_t* xfull;       // [nst] q8 plans: the stage's activation rows landed (32 arrivals)
   uint64_t* empty;       // [nst] MMAs of the stage done
   uint64_t* accfull;     // [2] accumulator buffer ready for the epilogue
   uint64_t* accempty;    // [2] epilogue done reading the accumulator
@@ -201,9 +231,12 @@ struct MmaShared {
   int nraw;
   uint64_t* rfull;       // [nraw] e4m3 tile landed (tx)
   uint64_t* rempty;      // [nraw] converted
+  uint64_t* drain;       // the issuer's MMAs done, after an abort
   uint32_t* tmem_base;
   int* abort_flag;
   int* misc;             // [8] scratch ([0] split-K last part, [2] after-run flag)
+  float* qmax;           // [4][16] per-warp column maxima (output group maxima)
+  float* qtab;           // [2][kMaxN] q8 epilogue: 2^-P per (variant, token) of the unit
 };
 
 // The ring holds as many stages as fit.  A stage covers nsub x 64 K: nsub
@@ -224,10 +257,13 @@ __host__ __device__ inline int mma_nsub(int nmax, int terms) {
 constexpr int kRawBytes = 128 * 128;
 
 KD_DEV MmaShared carve_mma_smem(uint8_t* base, int nmax, int terms, int nsub, bool fp8,
-                                int aterms) {
+                                int aterms, bool q8 = false) {
   MmaShared s;
   s.nsub = nsub;
   s.stage_bytes = nsub * (aterms * kATileBytes + b_sub_bytes(nmax, terms));   // bf16: A + B
+  // q8: + a staging area for the rows' fp32 activations of the chunk (512 B a row)
+  s.xoff = s.stage_bytes;
+  if (q8) s.stage_bytes += pad16(nmax) * 512;
   uintptr_t p = (reinterpret_cast<uintptr_t>(base) + 1023) & ~uintptr_t(1023);
   s.stage = reinterpret_cast<uint8_t*>(p);
   uint64_t* bars = reinterpret_cast<uint64_t*>(p + (size_t)kMRingBytes);
@@ -270,6 +306,12 @@ KD_DEV MmaShared carve_mma_smem(uint8_t* base, int nmax, int terms, int nsub, bo
   s.tmem_base = reinterpret_cast<uint32_t*>(s.accempty + 2);
   s.abort_flag = reinterpret_cast<int*>(s.tmem_base + 1);
   s.misc = s.abort_flag + 1;
+  s.qmax = reinterpret_cast<float*>(s.misc + 8);
+  s.qtab = s.qmax + 64;
+  // without a raw ring its barriers serve the A tiles' transactions
+  s.afull = s.rfull;
+  s.xfull = s.rempty + kMaxMStages;   // the B ring's barriers, unused without a raw ring
+  s.drain = reinterpret_cast<uint64_t*>(s.misc + 4);
   return s;
 }
 
@@ -305,11 +347,19 @@ KD_DEV bool mwait_lazy(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
 //   static constexpr int kTerms    bf16 terms of B (1; 2 = hi + lo; 3 = hi + mid + lo)
 //   static constexpr bool kFp8     A arrives as e4m3 tiles (converter warps, a_scale)
 //   static constexpr int kATerms   bf16 terms of the converted A tile (1, or 2 = hi + lo)
-//   const uint16_t* b_base(const MUnit&, int h); int b_stride(const MUnit&);
+//   static constexpr bool kQ8      e4m3 A tiles into kind::f8f6f4 MMAs; B made in-kernel
+//                                  from fp32 rows: int kVariants (1, or 2 for gate / up
+//                                  scales), const float* x_row(m, j), const float*
+//                                  g_row(m, j) (per-64 maxima), int kgroups(),
+//                                  float w_scale_v(m, kc, variant); kTerms = kVariants *
+//                                  kQTerms (B tiles per stage)
+//   static constexpr bool kGmaxOut  also write the output's per-64 maxima for a q8
+//                                  consumer: bool gmax_tile(m), gmax_store(m, group, j, v)
+//   const uint8_t* b_base(const MUnit&, int h); int b_stride(const MUnit&) (bytes)
 //   int b_rowidx(const MUnit&, int j)   token j's row of term h: base + rowidx * stride
 //   bool paired()                  rows are (gate, up) pairs
-//   void epilogue(const MUnit&, int row_in_tile, int j, float v)
-//   void epilogue2(const MUnit&, int pair_in_tile, int j, float g, float u)
+//   float epilogue(const MUnit&, int row_in_tile, int j, float v)   returns the stored value
+//   float epilogue2(const MUnit&, int pair_in_tile, int j, float g, float u)
 //   float* ws(); unsigned* tile_cnt()            split-K partials / arrivals
 //   bool wants_unit_done(); void unit_done(const MUnit&, MmaShared&)   epilogue warps only
 //   void after_run(MmaShared&, uint8_t* smem)   all threads, after the pipeline
@@ -318,44 +368,60 @@ template <class Plan>
 KD_DEV void mma_producer_a_bf16(const Plan& plan, MmaShared& sh, CtaUnits<Plan>& units,
                                 unsigned* err);
 
+// After an abort: wait (bounded, whatever the abort flag says) until the
+// last `n` transactions issued on ring `bars` of `nslots` slots have landed,
+// so that no TMA write is still in flight when the CTA leaves.
+KD_DEV void drain_tx(uint64_t* bars, int nslots, uint32_t issued) {
+  const uint32_t n = issued < (uint32_t)nslots ? issued : (uint32_t)nslots;
+  for (uint32_t i = issued - n; i < issued; ++i) mbar_wait(&bars[i % nslots], (i / nslots) & 1u);
+}
+
 template <class Plan>
 KD_DEV void mma_producer_a(const Plan& plan, MmaShared& sh, unsigned* err) {
   uint32_t it = 0;
   CtaUnits<Plan> units(plan);
   MUnit m;
+  bool ok = true;
   if constexpr (Plan::kFp8) {
     // e4m3 tiles [128 rows x 128 K bytes] into the raw ring
-    while (units.next(m)) {
+    while (ok && units.next(m)) {
       const CUtensorMap* map = plan.map(m.map);
       for (int c = 0; c < m.nkc; ++c, ++it) {
         const int s = it % sh.nraw;
         const uint32_t ph = (it / sh.nraw) & 1u;
-        mwait(&sh.rempty[s], ph ^ 1u, sh.abort_flag, err);
+        if (!mwait(&sh.rempty[s], ph ^ 1u, sh.abort_flag, err)) { ok = false; break; }
         mbar_arrive_expect_tx(&sh.rfull[s], kRawBytes);
         tma_load_2d(sh.raw + (size_t)s * kRawBytes, map, (m.kc0 + c) * 128, m.row, &sh.rfull[s]);
       }
     }
-  } else {
-    mma_producer_a_bf16(plan, sh, units, err);
-  }
-}
-
-template <class Plan>
-KD_DEV void mma_producer_a_bf16(const Plan& plan, MmaShared& sh, CtaUnits<Plan>& units,
-                                unsigned* err) {
-  uint32_t it = 0;
-  MUnit m;
-  while (units.next(m)) {
-    const CUtensorMap* map = plan.map(m.map);
-    for (int c = 0; c < m.nkc; ++c, ++it) {
-      const int s = it % sh.nst;
-      const uint32_t ph = (it / sh.nst) & 1u;
-      mwait(&sh.empty[s], ph ^ 1u, sh.abort_flag, err);
-      mbar_arrive_expect_tx(&sh.full[s], sh.nsub * kATileBytes);
-      for (int u = 0; u < sh.nsub; ++u)
-        tma_load_2d(sh.stage + (size_t)s * sh.stage_bytes + u * kATileBytes, map,
-                    ((m.kc0 + c) * sh.nsub + u) * 64, m.row, &sh.full[s]);
+    if (*sh.abort_flag) drain_tx(sh.rfull, sh.nraw, it);
+  } else if constexpr (Plan::kQ8) {
+    // e4m3 tiles [128 rows x 128 K bytes] straight into the stage (one box)
+    while (ok && units.next(m)) {
+      const CUtensorMap* map = plan.map(m.map);
+      for (int c = 0; c < m.nkc; ++c, ++it) {
+        const int s = it % sh.nst;
+        const uint32_t ph = (it / sh.nst) & 1u;
+        if (!mwait(&sh.empty[s], ph ^ 1u, sh.abort_flag, err)) { ok = false; break; }
+        mbar_arrive_expect_tx(&sh.afull[s], kRawBytes);
+        tma_load_2d(sh.stage + (size_t)s * sh.stage_bytes, map, (m.kc0 + c) * 128, m.row, &sh.afull[s]);
+      }
     }
+    if (*sh.abort_flag) drain_tx(sh.afull, sh.nst, it);
+  } else {
+    while (ok && units.next(m)) {
+      const CUtensorMap* map = plan.map(m.map);
+      for (int c = 0; c < m.nkc; ++c, ++it) {
+        const int s = it % sh.nst;
+        const uint32_t ph = (it / sh.nst) & 1u;
+        if (!mwait(&sh.empty[s], ph ^ 1u, sh.abort_flag, err)) { ok = false; break; }
+        mbar_arrive_expect_tx(&sh.afull[s], sh.nsub * kATileBytes);
+        for (int u = 0; u < sh.nsub; ++u)
+          tma_load_2d(sh.stage + (size_t)s * sh.stage_bytes + u * kATileBytes, map,
+                      ((m.kc0 + c) * sh.nsub + u) * 64, m.row, &sh.afull[s]);
+      }
+    }
+    if (*sh.abort_flag) drain_tx(sh.afull, sh.nst, it);
   }
 }
 
@@ -374,7 +440,8 @@ KD_DEV void cp_async_arrive_noinc(uint64_t* bar) {
 }
 
 // Two warps (64 threads) write the B tile of every stage with cp.async:
-// token rows j < ntok (zero-filled up to N), 128 bytes (64 K) each, 16-byte
+// token rows j < ntok (zero-filled up to N), 128 bytes (64 bf16 or 128 e4m3
+// K values) each, 16-byte
 // chunk c of row r at r*128 + ((c ^ (r & 7)) * 16) -- the 128-byte swizzle
 // the A tile has.  Thread t copies chunk t % 8 of rows t / 8, t / 8 + 8, ...
 // (so every row it copies has the same swizzle), for every bf16 term.  Each
@@ -395,10 +462,10 @@ KD_DEV void mma_producer_b(const Plan& plan, MmaShared& sh, unsigned* err) {
   while (units.next(m)) {
     const int N = pad16(m.ntok);
     const int nr = N >> 3;
-    const size_t stride = (size_t)plan.b_stride(m);
+    const size_t stride = (size_t)plan.b_stride(m);   // bytes
     // this thread's sources for the whole unit (byte count 0 = zero fill,
     // ~0 = no row)
-    const uint16_t* src[nh][kRows];
+    const uint8_t* src[nh][kRows];
     uint32_t nb[kRows];
 #pragma unroll
     for (int i = 0; i < kRows; ++i) {
@@ -406,7 +473,7 @@ KD_DEV void mma_producer_b(const Plan& plan, MmaShared& sh, unsigned* err) {
       const bool live = i < nr && r < m.ntok;
       const size_t ro = live ? (size_t)plan.b_rowidx(m, r) * stride : 0;
 #pragma unroll
-      for (int h = 0; h < nh; ++h) src[h][i] = plan.b_base(m, h) + ro + ch * 8;
+      for (int h = 0; h < nh; ++h) src[h][i] = plan.b_base(m, h) + ro + ch * 16;
       nb[i] = i < nr ? (live ? 16u : 0u) : 0xFFFFFFFFu;
     }
     const int bsub = b_sub_bytes(N, nh);
@@ -416,13 +483,13 @@ KD_DEV void mma_producer_b(const Plan& plan, MmaShared& sh, unsigned* err) {
       mwait(&sh.bempty[s], ph ^ 1u, sh.abort_flag, err);
       uint8_t* bt = sh.bst + (size_t)s * sh.bst_bytes + sh.boff + swz;
       for (int u = 0; u < sh.nsub; ++u) {
-        const int k0 = ((m.kc0 + c) * sh.nsub + u) * 64;
+        const size_t kb = (size_t)((m.kc0 + c) * sh.nsub + u) * 128;   // bytes of K before it
 #pragma unroll
         for (int i = 0; i < kRows; ++i) {
           if (nb[i] != 0xFFFFFFFFu) {
 #pragma unroll
             for (int h = 0; h < nh; ++h)
-              cp_async16(bt + u * bsub + h * N * 128 + (rg + 8 * i) * 128, src[h][i] + k0, nb[i]);
+              cp_async16(bt + u * bsub + h * N * 128 + (rg + 8 * i) * 128, src[h][i] + kb, nb[i]);
           }
         }
       }
@@ -497,6 +564,14 @@ KD_DEV void mma_converter(const Plan& plan, MmaShared& sh, unsigned* err) {
   }
 }
 
+// After an abort: no MMA of this thread may still be running when TMEM is
+// freed: commit them to the drain barrier and wait (bounded).
+KD_DEV void drain_mma(MmaShared& sh) {
+  if (!*sh.abort_flag) return;
+  mma_commit(sh.drain);
+  mbar_wait(sh.drain, 0);
+}
+
 template <class Plan>
 KD_DEV void mma_issuer(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigned* err) {
   constexpr int nterms = Plan::kTerms;
@@ -508,14 +583,21 @@ KD_DEV void mma_issuer(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigned*
     const uint32_t idesc = idesc_bf16(N);
     const int buf = nu_local & 1;
     const uint32_t d = tmem + (uint32_t)(buf * kMaxN);
-    mwait(&sh.accempty[buf], ((nu_local >> 1) & 1u) ^ 1u, sh.abort_flag, err);
+    if (!mwait(&sh.accempty[buf], ((nu_local >> 1) & 1u) ^ 1u, sh.abort_flag, err)) break;
     tc_fence_after();
+    bool ok = true;
     for (int c = 0; c < m.nkc; ++c, ++it) {
       const int s = it % sh.nst;
       const uint32_t ph = (it / sh.nst) & 1u;
-      mwait(&sh.full[s], ph, sh.abort_flag, err);
       const int sb = it % sh.nbst;
-      if (Plan::kFp8) mwait(&sh.bfull[sb], (it / sh.nbst) & 1u, sh.abort_flag, err);
+      if (Plan::kFp8) {
+        ok = mwait(&sh.full[s], ph, sh.abort_flag, err) &&
+             mwait(&sh.bfull[sb], (it / sh.nbst) & 1u, sh.abort_flag, err);
+      } else {
+        ok = mwait(&sh.afull[s], ph, sh.abort_flag, err) &&
+             mwait(&sh.full[s], ph, sh.abort_flag, err);
+      }
+      if (!ok) break;
       fence_proxy_async_smem();   // the B gathers (generic proxy) -> tensor core reads
       tc_fence_after();
       const uint32_t a0 = smem_u32(sh.stage + (size_t)s * sh.stage_bytes);
@@ -556,24 +638,280 @@ KD_DEV void mma_issuer(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigned*
       mma_commit(&sh.empty[s]);   // the stage is free once these MMAs are done
       if (Plan::kFp8) mma_commit(&sh.bempty[sb]);
     }
+    if (!ok) break;
     mma_commit(&sh.accfull[buf]);
+  }
+  drain_mma(sh);
+}
+
+// q8 plans: per stage (one e4m3 weight tile [128 x 128 K] and a B tile of
+// NV x kQTerms x N rows: every (variant, term, token)), four K-steps of 32,
+// one MMA each (N = NV kQTerms pad16(ntok) columns); the accumulator lives in
+// TMEM for the whole unit (two buffers, alternating between units, as for
+// the bf16 plans) and the epilogue adds the term columns.
+template <class Plan>
+KD_DEV void mma_issuer_q8(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigned* err) {
+  constexpr int NV = Plan::kVariants, nh = kQTerms;
+  uint32_t it = 0, nu = 0;
+  CtaUnits<Plan> units(plan);
+  MUnit m;
+  for (; units.next(m); ++nu) {
+    const int N = pad16(m.ntok);
+    // one MMA per K-step covers every (variant, term, token) row of the B tile
+    const uint32_t idesc = idesc_e4m3(NV * nh * N);
+    const int buf = nu & 1;
+    if (!mwait(&sh.accempty[buf], ((nu >> 1) & 1u) ^ 1u, sh.abort_flag, err)) break;
+    tc_fence_after();
+    const uint32_t d0 = tmem + (uint32_t)(buf * kQ8AccCols);
+    bool ok = true;
+    for (int c = 0; c < m.nkc; ++c, ++it) {
+      const int s = it % sh.nst;
+      const uint32_t ph = (it / sh.nst) & 1u;
+      ok = mwait(&sh.afull[s], ph, sh.abort_flag, err) && mwait(&sh.full[s], ph, sh.abort_flag, err);
+      if (!ok) break;
+      fence_proxy_async_smem();   // the B terms (generic proxy) -> tensor core reads
+      tc_fence_after();
+      const uint32_t a0 = smem_u32(sh.stage + (size_t)s * sh.stage_bytes);
+      // descriptors by adding byte offsets / 16 to the start-address field
+      // (shared addresses < 256 KB: the field never carries)
+      const uint64_t ad0 = sw128_desc(a0), bd0 = sw128_desc(a0 + sh.boff);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint64_t off = (uint64_t)((k * 32) >> 4);
+        mma_e4m3(d0, ad0 + off, bd0 + off, idesc, c > 0 || k > 0);
+      }
+      mma_commit(&sh.empty[s]);   // the stage is free once these MMAs are done
+    }
+    if (!ok) break;
+    mma_commit(&sh.accfull[buf]);
+  }
+  drain_mma(sh);
+}
+
+// 2^P for token j of a q8 unit and scale variant v (and 2^-P in inv): the
+// largest |activation| x weight block scale over the tile's K, from the
+// activation's per-64-element maxima, put in [128, 256).
+template <class Plan>
+KD_DEV float q8_unit_scale(const Plan& plan, const MUnit& m, int j, int v, float& inv) {
+  const float* g = plan.g_row(m, j);
+  float amax = 0.f;
+  const int ng = plan.kgroups();
+  for (int q = 0; q < ng; ++q) amax = fmaxf(amax, __ldg(g + q) * plan.w_scale_v(m, q >> 1, v));
+  return q_scale(amax, inv);
+}
+
+// q8 B producers.  Warp 2 (copier) copies, for every stage, the live token
+// rows' fp32 activations of the stage's 128-K chunk with cp.async into the
+// stage's staging area (after its B terms); each lane's copies arrive on the
+// stage's xfull barrier when they land, so every stage of the ring can have
+// copies in flight.  Warp 3 (converter) waits for a stage's rows and writes
+// x times (block scale x 2^P) as kQTerms e4m3 terms per scale variant, in
+// the 128-byte swizzle, then arrives on the stage's full barrier.  Rows past
+// ntok are left as they are: their MMA columns are not read.
+template <class Plan>
+KD_DEV void q8_convert_stage(const Plan& plan, MmaShared& sh, const MUnit& m, int c, int s,
+                             const float (&pm)[16][2]) {
+  constexpr int NV = Plan::kVariants, nh = kQTerms;
+  const int lane = threadIdx.x & 31;
+  const int N = pad16(m.ntok);
+  uint8_t* bt = sh.stage + (size_t)s * sh.stage_bytes + sh.boff;
+  const uint8_t* xs = sh.stage + (size_t)s * sh.stage_bytes + sh.xoff;
+  const int kc = m.kc0 + c;
+  float ws[NV];
+#pragma unroll
+  for (int v = 0; v < NV; ++v) ws[v] = plan.w_scale_v(m, kc, v);
+  // (row, 16-element chunk) pairs p = lane + 32 u: row p / 8, chunk p % 8
+#pragma unroll 1
+  for (int u = 0; u < 16; ++u) {
+    const int p = lane + 32 * u, r = p >> 3, ch = p & 7;
+    if (r >= m.ntok) break;
+    float x[16];
+    {
+      const float4* src = reinterpret_cast<const float4*>(xs + (size_t)r * 512 + ch * 64);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float4 f = src[q];
+        x[4 * q] = f.x; x[4 * q + 1] = f.y; x[4 * q + 2] = f.z; x[4 * q + 3] = f.w;
+      }
+    }
+    const uint32_t swz = (uint32_t)((ch ^ (r & 7)) * 16);
+#pragma unroll
+    for (int v = 0; v < NV; ++v) {
+      const float f = ws[v] * pm[u][v];
+      float w[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) w[e] = x[e] * f;
+#pragma unroll
+      for (int h = 0; h < nh; ++h) {
+        uint32_t pk[4];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const uint32_t c2 = e4m3x2_rn(w[2 * e], w[2 * e + 1]);
+          if (e & 1) pk[e >> 1] |= c2 << 16;
+          else pk[e >> 1] = c2;
+          if (h + 1 < nh) {
+            const float2 tv = e4m3x2_value(c2);
+            w[2 * e] -= tv.x;       // exact: within a factor of two of w (or w)
+            w[2 * e + 1] -= tv.y;
+          }
+        }
+        *reinterpret_cast<uint4*>(bt + (size_t)((v * nh + h) * N + r) * 128 + swz) =
+            make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      }
+    }
+  }
+  fence_proxy_async_smem();   // generic-proxy writes -> visible to the tensor core
+  mbar_arrive(&sh.full[s]);
+}
+
+// Warp 2: the copies (no waiting for them to land).
+template <class Plan>
+KD_DEV void mma_copier_q8(const Plan& plan, MmaShared& sh, unsigned* err) {
+  const int lane = threadIdx.x & 31;
+  uint32_t it = 0;
+  CtaUnits<Plan> units(plan);
+  MUnit m;
+  while (units.next(m)) {
+    for (int c = 0; c < m.nkc; ++c, ++it) {
+      const int s = it % sh.nst;
+      mwait(&sh.empty[s], ((it / sh.nst) & 1u) ^ 1u, sh.abort_flag, err);
+      uint8_t* xs = sh.stage + (size_t)s * sh.stage_bytes + sh.xoff;
+      const int kc = m.kc0 + c;
+      const int nq = *sh.abort_flag ? 0 : m.ntok * 32;   // no new copies after an abort
+      for (int q = lane; q < nq; q += 32) {               // 16-byte pieces, 32 a row
+        const int r = q >> 5, pi = q & 31;
+        const uint8_t* src = reinterpret_cast<const uint8_t*>(plan.x_row(m, r)) +
+                             (size_t)kc * 512 + pi * 16;
+        cp_async16(xs + (size_t)r * 512 + pi * 16, src, 16u);
+      }
+      cp_async_arrive_noinc(&sh.xfull[s]);
+    }
+  }
+  cp_async_commit();
+  cp_async_wait<0>();   // nothing in flight when the warp leaves
+}
+
+// Warp 3: per stage, wait for its rows, convert, release.
+template <class Plan>
+KD_DEV void mma_converter_q8(const Plan& plan, MmaShared& sh, unsigned* err) {
+  constexpr int NV = Plan::kVariants;
+  const int lane = threadIdx.x & 31;
+  float pm[16][2];
+  uint32_t it = 0;
+  CtaUnits<Plan> units(plan);
+  MUnit m;
+  while (units.next(m)) {
+    // 2^P of this lane's conversion rows (lane / 8 + 4 u) for the unit: each
+    // row's largest |x| x block scale over the tile's groups.  The lanes
+    // split the groups; the block scales are loaded once, and 8 rows' loads
+    // are all issued before their reductions.
+    {
+      constexpr int kG = 4;   // groups per lane (<= 128 groups: K <= 8192)
+      const int ng = plan.kgroups();
+      float wv[kG][NV];
+#pragma unroll
+      for (int i = 0; i < kG; ++i) {
+        const int q = lane + 32 * i;
+#pragma unroll
+        for (int v = 0; v < NV; ++v) wv[i][v] = q < ng ? plan.w_scale_v(m, q >> 1, v) : 0.f;
+      }
+#pragma unroll 1
+      for (int r0 = 0; r0 < m.ntok; r0 += 8) {
+        float lm[8][NV];
+#pragma unroll
+        for (int rr = 0; rr < 8; ++rr) {
+          const int r = r0 + rr;
+          float g[kG];
+          const float* gr = plan.g_row(m, r < m.ntok ? r : 0);
+#pragma unroll
+          for (int i = 0; i < kG; ++i) {
+            const int q = lane + 32 * i;
+            g[i] = (r < m.ntok && q < ng) ? __ldg(gr + q) : 0.f;
+          }
+#pragma unroll
+          for (int v = 0; v < NV; ++v) {
+            float a = 0.f;
+#pragma unroll
+            for (int i = 0; i < kG; ++i) a = fmaxf(a, g[i] * wv[i][v]);
+            lm[rr][v] = a;
+          }
+        }
+#pragma unroll
+        for (int rr = 0; rr < 8; ++rr)
+#pragma unroll
+          for (int v = 0; v < NV; ++v) {
+            float amax = lm[rr][v];
+            for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+            float inv;
+            const float sc = q_scale(amax, inv);
+            const int r = r0 + rr;
+            if (r < m.ntok && (r & 3) == (lane >> 3)) pm[r >> 2][v] = sc;
+          }
+      }
+    }
+    for (int c = 0; c < m.nkc; ++c, ++it) {
+      const int s = it % sh.nst;
+      mwait(&sh.xfull[s], (it / sh.nst) & 1u, sh.abort_flag, err);
+      q8_convert_stage(plan, sh, m, c, s, pm);
+    }
   }
 }
 
-// The plan's epilogue for 16 accumulator columns (tokens c .. c+15) of this
-// thread's row.
+// Per-64-element maxima of the output for a q8 consumer: this thread's 16
+// outputs o (tokens c .. c+15 of its row; with paired rows only the even
+// lanes hold one) -> max |o| per (token, group of kQGroup outputs): a group
+// is 64 rows (two epilogue warps) of an unpaired tile, or the 64 outputs of
+// a paired one (all four).  All four epilogue warps call.
 template <class Plan>
-KD_DEV void emit16(const Plan& plan, const MUnit& m, int row, int lane, int c, const float* v) {
+KD_DEV void groupmax16(const Plan& plan, const MUnit& m, int lane, int c, const float* o,
+                       MmaShared& sh) {
+  const int ew = (threadIdx.x >> 5) - 4;
+  const bool paired = plan.paired();
+  const bool valid = !paired || !(lane & 1);
+  float mx[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) mx[j] = (valid && c + j < m.ntok) ? fabsf(o[j]) : 0.f;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+    for (int j = 0; j < 16; ++j) mx[j] = fmaxf(mx[j], __shfl_xor_sync(0xffffffffu, mx[j], off));
+  if (lane == 0) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) sh.qmax[ew * 16 + j] = mx[j];
+  }
+  named_bar_sync(2, 128);
+  const int g = paired ? 0 : (ew >> 1);
+  if (lane < 16 && (paired ? ew == 0 : (ew & 1) == 0) && c + lane < m.ntok) {
+    const float* q = sh.qmax + lane;
+    const float v = paired ? fmaxf(fmaxf(q[0], q[16]), fmaxf(q[32], q[48]))
+                           : fmaxf(q[(2 * g) * 16], q[(2 * g + 1) * 16]);
+    plan.gmax_store(m, g, c + lane, v);
+  }
+  named_bar_sync(2, 128);   // qmax is rewritten by the next chunk
+}
+
+// The plan's epilogue for 16 accumulator columns (tokens c .. c+15) of this
+// thread's row, then (plans with kGmaxOut) the output's per-64 maxima.
+template <class Plan>
+KD_DEV void emit16(const Plan& plan, const MUnit& m, int row, int lane, int c, const float* v,
+                   MmaShared& sh) {
+  float o[16];
   if (plan.paired()) {
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
       const float other = __shfl_xor_sync(0xffffffffu, v[j], 1);
-      if (!(lane & 1) && c + j < m.ntok) plan.epilogue2(m, row >> 1, c + j, v[j], other);
+      o[j] = 0.f;
+      if (!(lane & 1) && c + j < m.ntok) o[j] = plan.epilogue2(m, row >> 1, c + j, v[j], other);
     }
   } else {
 #pragma unroll
-    for (int j = 0; j < 16; ++j)
-      if (c + j < m.ntok) plan.epilogue(m, row, c + j, v[j]);
+    for (int j = 0; j < 16; ++j) {
+      o[j] = 0.f;
+      if (c + j < m.ntok) o[j] = plan.epilogue(m, row, c + j, v[j]);
+    }
+  }
+  if constexpr (Plan::kGmaxOut) {
+    if (plan.gmax_tile(m)) groupmax16(plan, m, lane, c, o, sh);
   }
 }
 
@@ -653,7 +991,7 @@ KD_DEV void mma_epilogue(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigne
           tmem_ld16(ta + c, v);
           tmem_wait_ld();
         }
-        emit16(plan, m, row, lane, c, v);
+        emit16(plan, m, row, lane, c, v, sh);
       }
     }
     tc_fence_before();
@@ -666,17 +1004,137 @@ KD_DEV void mma_epilogue(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigne
   }
 }
 
+
+// q8 epilogue warps (4..7): as mma_epilogue, with the accumulator of this
+// thread's variant (gate for even rows, up for odd rows of a paired tile)
+// times the token's 2^-P (a per-unit table in shared memory).
+template <class Plan>
+KD_DEV void mma_epilogue_q8(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigned* err) {
+  constexpr int NV = Plan::kVariants;
+  const int ew = (threadIdx.x >> 5) - 4, lane = threadIdx.x & 31;
+  const int row = ew * 32 + lane, et = threadIdx.x - 128;
+  const int myv = NV == 2 ? (row & 1) : 0;
+  uint32_t nu_local = 0;
+  CtaUnits<Plan> units(plan);
+  MUnit m;
+  for (; units.next(m); ++nu_local) {
+    const int N = pad16(m.ntok);
+    const int buf = nu_local & 1;
+    // the unit's 2^-P per (variant, token), shared by the four warps
+    named_bar_sync(2, 128);   // every warp is done with the previous unit's table
+    {
+      const int j = et & 63, v = et >> 6;
+      if (j < m.ntok && v < NV) {
+        float inv;
+        q8_unit_scale(plan, m, j, v, inv);
+        sh.qtab[v * 64 + j] = inv;
+      }
+    }
+    named_bar_sync(2, 128);
+    mwait_lazy(&sh.accfull[buf], (nu_local >> 1) & 1u, sh.abort_flag, err);
+    tc_fence_after();
+    const uint32_t ta = tmem + ((uint32_t)(ew * 32) << 16) + (uint32_t)(buf * kQ8AccCols);
+    const float* qt = sh.qtab + myv * 64;
+    // 16 tokens of this thread's variant: the sum of its term columns, scaled
+    // (every lane loads every (variant, term) block: tcgen05.ld is warp-wide)
+    auto load16 = [&](int c, float* out) {
+      float d[NV][kQTerms][16];
+#pragma unroll
+      for (int v = 0; v < NV; ++v)
+#pragma unroll
+        for (int h = 0; h < kQTerms; ++h) tmem_ld16(ta + (uint32_t)((v * kQTerms + h) * N + c), d[v][h]);
+      tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        float acc = 0.f;
+#pragma unroll
+        for (int v = 0; v < NV; ++v)
+          if (v == myv) {
+#pragma unroll
+            for (int h = 0; h < kQTerms; ++h) acc += d[v][h][j];
+          }
+        out[j] = acc * qt[c + j];
+      }
+    };
+    bool complete = true;
+    int first = 0;
+    if (m.nparts > 1) {
+      const int slot = m.part == 0 ? 1 : 0;
+      float* ws = plan.ws() + (size_t)blockIdx.x * kWsFloatsPerCta +
+                  (size_t)slot * 128 * kMaxN + row;
+#pragma unroll 1
+      for (int c = 0; c < N; c += 16) {
+        float v[16];
+        load16(c, v);
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          if (c + j < m.ntok) __stcg(ws + (c + j) * 128, v[j]);
+      }
+      __threadfence();
+      named_bar_sync(2, 128);
+      if (threadIdx.x == 128) {
+        const unsigned prev = atomicAdd(plan.tile_cnt() + m.tile, 1u);
+        const bool last = prev == (unsigned)(m.nparts - 1);
+        if (last) plan.tile_cnt()[m.tile] = 0u;  // every part is in: ready for reuse
+        sh.misc[0] = last;
+      }
+      named_bar_sync(2, 128);
+      complete = sh.misc[0] != 0;
+      first = (int)blockIdx.x - m.part;
+      if (complete) __threadfence();
+    }
+    if (complete) {
+#pragma unroll 1
+      for (int c = 0; c < N; c += 16) {
+        float v[16];
+        if (m.nparts > 1) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) v[j] = 0.f;
+#pragma unroll 1
+          for (int p = 0; p < m.nparts; p += 4) {
+            float t[4][16];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const float* src = plan.ws() + (size_t)(first + p + q) * kWsFloatsPerCta +
+                                 (size_t)(p + q == 0 ? 1 : 0) * 128 * kMaxN + row + c * 128;
+#pragma unroll
+              for (int j = 0; j < 16; ++j)
+                t[q][j] = (p + q < m.nparts && c + j < m.ntok) ? __ldcg(src + j * 128) : 0.f;
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              if (p + q < m.nparts) {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) v[j] += t[q][j];
+              }
+          }
+        } else {
+          load16(c, v);
+        }
+        emit16(plan, m, row, lane, c, v, sh);
+      }
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sh.accempty[buf]);
+  }
+}
+
 template <class Plan>
 KD_DEV void mma_run(const Plan& plan, uint8_t* smem_raw, unsigned* err) {
   MmaShared sh = carve_mma_smem(smem_raw, plan.max_n(), Plan::kTerms, plan.nsub, Plan::kFp8,
-                                Plan::kATerms);
+                                Plan::kATerms, Plan::kQ8);
   const int warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
     for (int i = 0; i < sh.nst; ++i) {
-      // A (transaction arrive, or the converter) + the 64 B threads unless B has its own ring
-      mbar_init(&sh.full[i], Plan::kFp8 ? 1 : 1 + 64);
+      // the converter (FP8 projections), the 64 B threads (A: afull), or the
+      // q8 converter warp (32)
+      mbar_init(&sh.full[i], Plan::kFp8 ? 1 : (Plan::kQ8 ? 32 : 64));
       mbar_init(&sh.empty[i], 1);
+      if (!Plan::kFp8) mbar_init(&sh.afull[i], 1);
+      if (Plan::kQ8) mbar_init(&sh.xfull[i], 32);
     }
+    mbar_init(sh.drain, 1);
     if (Plan::kFp8) {
       for (int i = 0; i < sh.nbst; ++i) {
         mbar_init(&sh.bfull[i], 64);
@@ -687,6 +1145,7 @@ KD_DEV void mma_run(const Plan& plan, uint8_t* smem_raw, unsigned* err) {
       mbar_init(&sh.rfull[i], 1);
       mbar_init(&sh.rempty[i], 1);
     }
+
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sh.accfull[i], 1);
       mbar_init(&sh.accempty[i], 4);
@@ -695,7 +1154,9 @@ KD_DEV void mma_run(const Plan& plan, uint8_t* smem_raw, unsigned* err) {
     sh.misc[2] = 0;
     fence_mbar_init();
   }
-  if (warp == 1) tmem_alloc(sh.tmem_base, 2 * kMaxN);
+  constexpr uint32_t kCols = Plan::kQ8 ? (uint32_t)kQ8TmemCols : (uint32_t)(2 * kMaxN);
+  static_assert(!Plan::kQ8 || Plan::kVariants * kQTerms * kMaxN <= kQ8AccCols, "q8 accumulators");
+  if (warp == 1) tmem_alloc(sh.tmem_base, kCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -703,11 +1164,20 @@ KD_DEV void mma_run(const Plan& plan, uint8_t* smem_raw, unsigned* err) {
   if (warp == 0) {
     if ((threadIdx.x & 31) == 0) mma_producer_a(plan, sh, err);
   } else if (warp == 1) {
-    if ((threadIdx.x & 31) == 0) mma_issuer(plan, sh, tmem, err);
+    if ((threadIdx.x & 31) == 0) {
+      if constexpr (Plan::kQ8) mma_issuer_q8(plan, sh, tmem, err);
+      else mma_issuer(plan, sh, tmem, err);
+    }
   } else if (warp < 4) {
-    mma_producer_b(plan, sh, err);
+    if constexpr (Plan::kQ8) {
+      if (warp == 2) mma_copier_q8(plan, sh, err);
+      else mma_converter_q8(plan, sh, err);
+    } else {
+      mma_producer_b(plan, sh, err);
+    }
   } else if (warp < 8) {
-    mma_epilogue(plan, sh, tmem, err);
+    if constexpr (Plan::kQ8) mma_epilogue_q8(plan, sh, tmem, err);
+    else mma_epilogue(plan, sh, tmem, err);
   } else if constexpr (Plan::kFp8) {
     mma_converter(plan, sh, err);
   }
@@ -715,7 +1185,7 @@ KD_DEV void mma_run(const Plan& plan, uint8_t* smem_raw, unsigned* err) {
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 2 * kMaxN);
+    tmem_dealloc(tmem, kCols);
   }
   plan.after_run(sh, smem_raw);
 }

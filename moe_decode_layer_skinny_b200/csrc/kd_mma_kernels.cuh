@@ -37,28 +37,21 @@ KD_DEV int max_tokens_per_expert(const int* cnt, const int* act, int n_act) {
   return s_max;
 }
 
-KD_DEV void store_hilo(uint16_t* hi, uint16_t* lo, size_t o, float v) {
-  const uint16_t h = f32_to_bf16_bits(v);
-  hi[o] = h;
-  lo[o] = f32_to_bf16_bits(v - __uint_as_float((uint32_t)h << 16));
-}
-
-// v = hi + mid + lo exactly (each difference is exact in fp32; three 8-bit
-// significands cover fp32's 24).
-KD_DEV void store_hilo3(uint16_t* hi, uint16_t* mid, uint16_t* lo, size_t o, float v) {
-  const uint16_t h = f32_to_bf16_bits(v);
-  const float r1 = v - __uint_as_float((uint32_t)h << 16);
-  const uint16_t m = f32_to_bf16_bits(r1);
-  hi[o] = h;
-  mid[o] = m;
-  lo[o] = f32_to_bf16_bits(r1 - __uint_as_float((uint32_t)m << 16));
-}
-
 // ------------------------------------------------------------------ QKV + o-proj
 
-template <bool F8>
+// MODE 0: QKV + o-proj tiles of one launch (the chain with a given attn_out,
+// B = the bf16 inputs).  Full layer: MODE 1 the QKV tiles with B = u =
+// RMSNorm(x) g1 as a bf16 hi + lo pair (the epilogue also writes fp32 QKV and
+// the new keys / values into the KV cache); MODE 2 the o-proj tiles with B =
+// the attention output as hi + lo, residual x, into h1r.
+template <bool F8, int MODE = 0>
 struct MmaProjPlan {
   static constexpr bool kFp8 = F8;
+  static constexpr bool kQ8 = false;
+  static constexpr int kVariants = 1;
+  // FP8: h1's per-64 maxima for the q8 gate/up kernels (the full layer's
+  // come from its second RMSNorm)
+  static constexpr bool kGmaxOut = F8 && MODE == 0;
   // FP8: the scaled weights as bf16 hi + lo (h1 feeds the fp32 router)
   static constexpr int kATerms = F8 ? 2 : 1;
   const LayerDev* L; Acts a; const MmaMaps* maps;
@@ -80,29 +73,48 @@ struct MmaProjPlan {
   }
   KD_DEV const CUtensorMap* map(int id) const { return &maps->m[id]; }
   KD_DEV int max_n() const { return a.M; }
-  static constexpr int kTerms = 1;
+  static constexpr int kTerms = MODE == 0 ? 1 : 2;
   KD_DEV float2 a_scale(const MUnit& m, int kc) const {
     const float sc = m.tag == 0 ? L->sqkv[(size_t)(m.row >> 7) * L->nHb + kc]
                                 : L->so[(size_t)(m.row >> 7) * L->nAb + kc];
     return make_float2(sc, sc);
   }
-  KD_DEV const uint16_t* b_base(const MUnit& m, int) const { return m.tag == 0 ? a.x : a.attn; }
-  KD_DEV int b_stride(const MUnit& m) const { return m.tag == 0 ? L->H : L->A; }
+  KD_DEV const uint8_t* b_base(const MUnit& m, int h) const {
+    if (MODE == 1) return reinterpret_cast<const uint8_t*>(h ? L->u_lo : L->u_hi);
+    if (MODE == 2) return reinterpret_cast<const uint8_t*>(h ? L->attn_lo : L->attn_hi);
+    return reinterpret_cast<const uint8_t*>(m.tag == 0 ? a.x : a.attn);
+  }
+  KD_DEV int b_stride(const MUnit& m) const { return (m.tag == 0 ? L->H : L->A) * 2; }
   KD_DEV int b_rowidx(const MUnit&, int j) const { return j; }
   KD_DEV bool paired() const { return false; }
-  KD_DEV void epilogue(const MUnit& m, int r, int j, float v) const {
+  KD_DEV float epilogue(const MUnit& m, int r, int j, float v) const {
     const int row = m.lrow + r;
     if (m.tag == 0) {
       L->qkv[(size_t)j * L->Nqkv + row] = f32_to_bf16_bits(v);
-    } else {
-      const size_t o = (size_t)j * L->H + row;
-      // read-only here (a plain load could not move above the stores below)
-      const float h = __uint_as_float((uint32_t)__ldg(a.x + o) << 16) + v;
-      L->h1f[o] = h;
-      store_hilo3(L->h1b, L->h1lo, L->h1lo2, o, h);
+      if (MODE == 1) {
+        L->qkvf[(size_t)j * L->Nqkv + row] = v;
+        kv_store(*L, a, j, row, v);
+      }
+      return v;
     }
+    const size_t o = (size_t)j * L->H + row;
+    // read-only here (a plain load could not move above the stores below)
+    const float h = __uint_as_float((uint32_t)__ldg(a.x + o) << 16) + v;
+    if (MODE == 2) {
+      L->h1r[o] = h;
+      return h;
+    }
+    L->h1f[o] = h;
+    if (F8) L->h1b[o] = f32_to_bf16_bits(h);   // the FP8 router reads h1f on CUDA cores
+    else store_hilo3(L->h1b, L->h1lo, L->h1lo2, o, h);
+    return h;
   }
-  KD_DEV void epilogue2(const MUnit&, int, int, float, float) const {}
+  KD_DEV float epilogue2(const MUnit&, int, int, float, float) const { return 0.f; }
+  // h1's per-64 maxima: o-proj tiles, groups of 64 rows of h
+  KD_DEV bool gmax_tile(const MUnit& m) const { return m.tag == 1; }
+  KD_DEV void gmax_store(const MUnit& m, int g, int j, float v) const {
+    L->h1g[(size_t)j * (L->H / kQGroup) + m.lrow / kQGroup + g] = v;
+  }
   KD_DEV float* ws() const { return L->ws_main; }
   KD_DEV unsigned* tile_cnt() const { return L->tcnt_main; }
   KD_DEV bool wants_unit_done() const { return false; }
@@ -110,14 +122,15 @@ struct MmaProjPlan {
   KD_DEV void after_run(MmaShared&, uint8_t*) const {}
 };
 
-template <bool F8>
+template <bool F8, int MODE = 0>
 __global__ void __launch_bounds__(F8 ? kMThreadsF8 : kMThreads, 1)
     mma_proj_kernel(LayerDev L, Acts a, const __grid_constant__ MmaMaps maps) {
   extern __shared__ uint8_t smem[];
-  MmaProjPlan<F8> p;
+  MmaProjPlan<F8, MODE> p;
   p.L = &L; p.a = a; p.maps = &maps;
-  p.nsub = F8 ? 2 : mma_nsub(a.M, 1);
-  p.tq = L.Nqkv / 128; p.to = L.H / 128; p.cq = L.H / (64 * p.nsub); p.co = L.A / (64 * p.nsub);
+  p.nsub = F8 ? 2 : mma_nsub(a.M, MmaProjPlan<F8, MODE>::kTerms);
+  p.tq = MODE == 2 ? 0 : L.Nqkv / 128; p.to = MODE == 1 ? 0 : L.H / 128;
+  p.cq = L.H / (64 * p.nsub); p.co = L.A / (64 * p.nsub);
   pdl_wait();
   pdl_launch_dependents();
   mma_run(p, smem, L.err);
@@ -134,6 +147,9 @@ __global__ void __launch_bounds__(F8 ? kMThreadsF8 : kMThreads, 1)
 template <bool F8>
 struct MmaRouterPlan {
   static constexpr bool kFp8 = F8;
+  static constexpr bool kQ8 = false;
+  static constexpr int kVariants = 1;
+  static constexpr bool kGmaxOut = false;
   static constexpr int kATerms = 1;
   const LayerDev* L; int M; const MmaMaps* maps;
   int nsub;
@@ -151,17 +167,19 @@ struct MmaRouterPlan {
     const float sc = L->sr[(size_t)(m.row >> 7) * L->nHb + kc];
     return make_float2(sc, sc);
   }
-  KD_DEV const uint16_t* b_base(const MUnit&, int h) const {
-    return h == 0 ? L->h1b : h == 1 ? L->h1lo : L->h1lo2;
+  KD_DEV const uint8_t* b_base(const MUnit&, int h) const {
+    return reinterpret_cast<const uint8_t*>(h == 0 ? L->h1b : h == 1 ? L->h1lo : L->h1lo2);
   }
-  KD_DEV int b_stride(const MUnit&) const { return L->H; }
+  KD_DEV int b_stride(const MUnit&) const { return L->H * 2; }
   KD_DEV int b_rowidx(const MUnit&, int j) const { return j; }
   KD_DEV bool paired() const { return false; }
-  KD_DEV void epilogue(const MUnit& m, int r, int j, float v) const {
+  KD_DEV float epilogue(const MUnit& m, int r, int j, float v) const {
     const int e = m.lrow + r;
-    if (e < L->E) L->logits[(size_t)j * L->E + e] = v + (L->bias ? __ldg(L->bias + e) : 0.f);
+    if (e < L->E)
+      L->logits[(size_t)j * L->E + e] = v + (L->bias && !L->bias_sel ? __ldg(L->bias + e) : 0.f);
+    return v;
   }
-  KD_DEV void epilogue2(const MUnit&, int, int, float, float) const {}
+  KD_DEV float epilogue2(const MUnit&, int, int, float, float) const { return 0.f; }
   KD_DEV float* ws() const { return L->ws_main; }
   KD_DEV unsigned* tile_cnt() const { return L->tcnt_main; }
   // the CTA that completes the last tile of logits routes the call
@@ -235,16 +253,24 @@ __global__ void __launch_bounds__(F8 ? kMThreadsF8 : kMThreads, 1)
 
 // Routed: tiles of the active experts' interleaved gate/up rows (2I/128 per
 // expert); shared: the shared expert's (all M tokens; its own launch on the
-// side stream).  B = h1 as a bf16 hi/lo pair.
+// side stream).  bf16 weights: B = h1 as a bf16 hi/lo pair.  FP8 weights
+// (q8): the e4m3 tiles as they land, B made from h1 (fp32) per stage with
+// the gate rows' and the up rows' block scales (two variants), and the
+// SwiGLU activations' per-64 maxima written for the down kernel.
 template <bool F8>
 struct MmaGateUpPlan {
-  static constexpr bool kFp8 = F8;
+  static constexpr bool kFp8 = false;    // no converter warps
+  static constexpr bool kQ8 = F8;
+  static constexpr int kVariants = F8 ? 2 : 1;
+  static constexpr bool kGmaxOut = F8;
   static constexpr int kATerms = 1;
   const LayerDev* L; int M; bool shared; const MmaMaps* maps; Route rt; int n_act;
   int nsub, nmax;
   KD_DEV int tiles_per() const { return 2 * L->I / 128; }
   KD_DEV int num_tiles() const { return (shared ? 1 : n_act) * tiles_per(); }
-  KD_DEV long long tile_start(int t) const { return (long long)t * (L->H / (64 * nsub)); }
+  KD_DEV long long tile_start(int t) const {
+    return (long long)t * (L->H / (F8 ? 128 : 64 * nsub));
+  }
   KD_DEV MUnit tile_unit(int t) const {
     MUnit m{};
     const int a = t / tiles_per(), tt = t % tiles_per();
@@ -260,35 +286,52 @@ struct MmaGateUpPlan {
   }
   KD_DEV const CUtensorMap* map(int id) const { return &maps->m[id]; }
   KD_DEV int max_n() const { return nmax; }
-  // bf16 hi + lo activations; with FP8 weights (3e-2 tolerance) the hi term
-  // alone, which halves the MMAs per weight byte
-  static constexpr int kTerms = F8 ? 1 : 2;
-  // rows alternate gate / up: their own scale tables, logical row block tt / 2
-  KD_DEV float2 a_scale(const MUnit& m, int kc) const {
-    const int tt = m.lrow >> 7;
-    const float* base = shared ? L->sgu_sh : L->sgu + (size_t)m.tag * 2 * L->nIb * L->nHb;
-    const size_t o = (size_t)(tt >> 1) * L->nHb + kc;
-    return make_float2(base[o], base[(size_t)L->nIb * L->nHb + o]);
+  // bf16: hi + lo activations; q8: kQTerms e4m3 terms for each of the two
+  // scale variants (B tiles per stage)
+  static constexpr int kTerms = F8 ? kVariants * kQTerms : 2;
+  KD_DEV const uint8_t* b_base(const MUnit&, int h) const {
+    return reinterpret_cast<const uint8_t*>(h ? L->h1lo : L->h1b);
   }
-  KD_DEV const uint16_t* b_base(const MUnit&, int h) const { return h ? L->h1lo : L->h1b; }
-  KD_DEV int b_stride(const MUnit&) const { return L->H; }
+  KD_DEV int b_stride(const MUnit&) const { return L->H * 2; }
   KD_DEV int b_rowidx(const MUnit& m, int j) const {
     return shared ? j : rt.perm[m.tok0 + j] / L->k;
   }
+  // q8: rows alternate gate / up, each with its own block scales (logical
+  // row block tt / 2); variant 0 = gate, 1 = up
+  KD_DEV float w_scale_v(const MUnit& m, int kc, int v) const {
+    const int tt = m.lrow >> 7;
+    const float* base = shared ? L->sgu_sh : L->sgu + (size_t)m.tag * 2 * L->nIb * L->nHb;
+    return __ldg(base + (size_t)v * L->nIb * L->nHb + (size_t)(tt >> 1) * L->nHb + kc);
+  }
+  KD_DEV const float* x_row(const MUnit& m, int j) const {
+    return L->h1f + (size_t)b_rowidx(m, j) * L->H;
+  }
+  KD_DEV const float* g_row(const MUnit& m, int j) const {
+    return L->h1g + (size_t)b_rowidx(m, j) * (L->H / kQGroup);
+  }
+  KD_DEV int kgroups() const { return L->H / kQGroup; }
   KD_DEV bool paired() const { return true; }
-  KD_DEV void epilogue(const MUnit&, int, int, float) const {}
-  KD_DEV void epilogue2(const MUnit& m, int p, int j, float g, float u) const {
+  KD_DEV float epilogue(const MUnit&, int, int, float) const { return 0.f; }
+  KD_DEV float epilogue2(const MUnit& m, int p, int j, float g, float u) const {
     const int i = m.lrow / 2 + p;
     const float v = silu(g) * u;
     if (shared) {
       const size_t o = (size_t)j * L->I + i;
       L->act_sh[o] = v;
-      store_hilo(L->act_sh_hi, L->act_sh_lo, o, v);
+      if (!F8) store_hilo(L->act_sh_hi, L->act_sh_lo, o, v);
     } else {
       const size_t o = (size_t)(m.tok0 + j) * L->I + i;
       L->act[o] = v;
-      store_hilo(L->act_hi, L->act_lo, o, v);
+      if (!F8) store_hilo(L->act_hi, L->act_lo, o, v);
     }
+    return v;
+  }
+  // the activations' per-64 maxima (q8): one group = the tile's 64 outputs
+  KD_DEV bool gmax_tile(const MUnit&) const { return true; }
+  KD_DEV void gmax_store(const MUnit& m, int, int j, float v) const {
+    const int g = m.lrow / 128, nq = L->I / kQGroup;
+    if (shared) L->actshg[(size_t)j * nq + g] = v;
+    else L->actg[(size_t)(m.tok0 + j) * nq + g] = v;
   }
   KD_DEV float* ws() const { return shared ? L->ws_side : L->ws_main; }
   KD_DEV unsigned* tile_cnt() const { return shared ? L->tcnt_side : L->tcnt_main; }
@@ -298,7 +341,7 @@ struct MmaGateUpPlan {
 };
 
 template <bool F8>
-__global__ void __launch_bounds__(F8 ? kMThreadsF8 : kMThreads, 1)
+__global__ void __launch_bounds__(kMThreads, 1)
     mma_gateup_kernel(LayerDev L, int M, int shared, const __grid_constant__ MmaMaps maps) {
   extern __shared__ uint8_t smem[];
   MmaGateUpPlan<F8> p;
@@ -311,7 +354,7 @@ __global__ void __launch_bounds__(F8 ? kMThreadsF8 : kMThreads, 1)
     p.n_act = *p.rt.n_act;
     p.nmax = max_tokens_per_expert(p.rt.cnt, p.rt.act, p.n_act);
   }
-  p.nsub = F8 ? 2 : mma_nsub(p.nmax, 2);
+  p.nsub = F8 ? 1 : mma_nsub(p.nmax, 2);
   mma_run(p, smem, L.err);
 }
 
@@ -322,17 +365,23 @@ __global__ void __launch_bounds__(F8 ? kMThreadsF8 : kMThreads, 1)
 // routed experts' largest token count, rounded up to 16) so that its B tiles
 // are no wider than the routed ones: a wide B tile would shrink every stage's
 // share of weights in the ring.  B = the SwiGLU activations as a bf16 hi/lo
-// pair.  The epilogue writes each expert's rows of its tokens' outputs (yr,
-// ysh); the gate-weighted combine into the layer output is the next launch.
+// pair (q8: the e4m3 terms of the activations).  The epilogue writes each
+// expert's rows of its tokens' outputs (yr, ysh); the gate-weighted combine
+// into the layer output is the next launch.
 template <bool F8>
 struct MmaDownPlan {
-  static constexpr bool kFp8 = F8;
+  static constexpr bool kFp8 = false;    // no converter warps
+  static constexpr bool kQ8 = F8;
+  static constexpr int kVariants = 1;
+  static constexpr bool kGmaxOut = false;
   static constexpr int kATerms = 1;
   const LayerDev* L; int M; int n_act; const MmaMaps* maps;
   int nsub, nmax, shchunk, nsh;
   KD_DEV int tiles_per() const { return L->H / 128; }
   KD_DEV int num_tiles() const { return (n_act + nsh) * tiles_per(); }
-  KD_DEV long long tile_start(int t) const { return (long long)t * (L->I / (64 * nsub)); }
+  KD_DEV long long tile_start(int t) const {
+    return (long long)t * (L->I / (F8 ? 128 : 64 * nsub));
+  }
   KD_DEV MUnit tile_unit(int t) const {
     MUnit m{};
     const int a = t / tiles_per(), tt = t % tiles_per();
@@ -350,27 +399,33 @@ struct MmaDownPlan {
   }
   KD_DEV const CUtensorMap* map(int id) const { return &maps->m[id]; }
   KD_DEV int max_n() const { return nmax; }
-  // bf16 hi + lo activations; with FP8 weights (3e-2 tolerance) the hi term
-  // alone, which halves the MMAs per weight byte
-  static constexpr int kTerms = F8 ? 1 : 2;
-  KD_DEV float2 a_scale(const MUnit& m, int kc) const {
+  // bf16: hi + lo activations; q8: kQTerms e4m3 terms
+  static constexpr int kTerms = F8 ? kQTerms : 2;
+  KD_DEV float w_scale_v(const MUnit& m, int kc, int) const {
     const float* base = m.tag < 0 ? L->sd_sh : L->sd + (size_t)m.tag * L->nHb * L->nIb;
-    const float sc = base[(size_t)(m.lrow >> 7) * L->nIb + kc];
-    return make_float2(sc, sc);
+    return __ldg(base + (size_t)(m.lrow >> 7) * L->nIb + kc);
   }
-  KD_DEV const uint16_t* b_base(const MUnit& m, int h) const {
-    if (m.tag < 0) return h ? L->act_sh_lo : L->act_sh_hi;
-    return h ? L->act_lo : L->act_hi;
+  KD_DEV const float* x_row(const MUnit& m, int j) const {
+    return (m.tag < 0 ? L->act_sh : L->act) + (size_t)(m.tok0 + j) * L->I;
   }
-  KD_DEV int b_stride(const MUnit&) const { return L->I; }
+  KD_DEV const float* g_row(const MUnit& m, int j) const {
+    return (m.tag < 0 ? L->actshg : L->actg) + (size_t)(m.tok0 + j) * (L->I / kQGroup);
+  }
+  KD_DEV int kgroups() const { return L->I / kQGroup; }
+  KD_DEV const uint8_t* b_base(const MUnit& m, int h) const {
+    if (m.tag < 0) return reinterpret_cast<const uint8_t*>(h ? L->act_sh_lo : L->act_sh_hi);
+    return reinterpret_cast<const uint8_t*>(h ? L->act_lo : L->act_hi);
+  }
+  KD_DEV int b_stride(const MUnit&) const { return L->I * 2; }
   KD_DEV int b_rowidx(const MUnit& m, int j) const { return m.tok0 + j; }
   KD_DEV bool paired() const { return false; }
-  KD_DEV void epilogue(const MUnit& m, int r, int j, float v) const {
+  KD_DEV float epilogue(const MUnit& m, int r, int j, float v) const {
     const int h = m.lrow + r;
     if (m.tag < 0) L->ysh[(size_t)(m.tok0 + j) * L->H + h] = v;
     else L->yr[(size_t)__ldg(L->perm + m.tok0 + j) * L->H + h] = v;
+    return v;
   }
-  KD_DEV void epilogue2(const MUnit&, int, int, float, float) const {}
+  KD_DEV float epilogue2(const MUnit&, int, int, float, float) const { return 0.f; }
   KD_DEV float* ws() const { return L->ws_main; }
   KD_DEV unsigned* tile_cnt() const { return L->tcnt_main; }
   KD_DEV bool wants_unit_done() const { return false; }
@@ -379,7 +434,7 @@ struct MmaDownPlan {
 };
 
 template <bool F8>
-__global__ void __launch_bounds__(F8 ? kMThreadsF8 : kMThreads, 1)
+__global__ void __launch_bounds__(kMThreads, 1)
     mma_down_kernel(LayerDev L, int M, const __grid_constant__ MmaMaps maps) {
   extern __shared__ uint8_t smem[];
   pdl_wait();
@@ -395,7 +450,7 @@ __global__ void __launch_bounds__(F8 ? kMThreadsF8 : kMThreads, 1)
     p.nsh = (M + p.shchunk - 1) / p.shchunk;
     p.nmax = max(p.nmax, p.shchunk);
   }
-  p.nsub = F8 ? 2 : mma_nsub(p.nmax, 2);
+  p.nsub = F8 ? 1 : mma_nsub(p.nmax, 2);
   mma_run(p, smem, L.err);
 }
 
@@ -415,14 +470,14 @@ __global__ void __launch_bounds__(256) combine_kernel(LayerDev L, int M, uint16_
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
     const int t = i / H2, h = 2 * (i - t * H2);
     const size_t o = (size_t)t * L.H + h;
-    float2 v = __ldcg(reinterpret_cast<const float2*>(L.h1f + o));
+    float2 v = __ldcg(reinterpret_cast<const float2*>(L.resid + o));
     if (L.S) {
       const float2 y = __ldcg(reinterpret_cast<const float2*>(L.ysh + o));
       v.x += y.x;
       v.y += y.y;
     }
     for (int j = 0; j < k; ++j) {
-      const float g = __ldcg(L.gates + t * k + j);
+      const float g = L.rscale * __ldcg(L.gates + t * k + j);
       const float2 y = __ldcg(reinterpret_cast<const float2*>(L.yr + ((size_t)t * k + j) * L.H + h));
       v.x += g * y.x;
       v.y += g * y.y;

@@ -331,8 +331,9 @@ KD_DEV void release_stage(const Plan& plan, StreamShared& sh, Issuer& iss, int s
   __syncwarp();
   if ((threadIdx.x & 31) == 0) mbar_arrive(&sh.empty[slot]);
   if (threadIdx.x == kIssuer) {
-    wait_or_abort(&sh.empty[slot], ph, sh.abort_flag, err, ERR_WAIT_EMPTY);
-    iss.next(plan, sh);
+    // after an abort no new copy is issued (the ones in flight are drained
+    // before the CTA leaves)
+    if (wait_or_abort(&sh.empty[slot], ph, sh.abort_flag, err, ERR_WAIT_EMPTY)) iss.next(plan, sh);
   }
   __syncwarp();  // the issuing lane rejoins its warp before any CTA barrier
 }
@@ -452,6 +453,11 @@ KD_DEV void stream_run(const Plan& plan, uint8_t* smem_raw, unsigned* err,
   }
   __syncthreads();
   stream_consume<WT, AT>(plan, sh, iss, err);
+  if (threadIdx.x == kIssuer && *sh.abort_flag) {
+    // after an abort: the last stages' bulk copies land before the CTA leaves
+    const uint32_t n = iss.n < (uint32_t)kStages ? iss.n : (uint32_t)kStages;
+    for (uint32_t i = iss.n - n; i < iss.n; ++i) mbar_wait(&sh.full[i % kStages], (i / kStages) & 1u);
+  }
 }
 
 }  // namespace kd

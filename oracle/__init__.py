@@ -36,7 +36,8 @@ class _Cfg(ctypes.Structure):
     _fields_ = [("hidden", ctypes.c_int), ("q_heads", ctypes.c_int), ("kv_heads", ctypes.c_int),
                 ("head_dim", ctypes.c_int), ("n_experts", ctypes.c_int), ("top_k", ctypes.c_int),
                 ("n_shared", ctypes.c_int), ("inter", ctypes.c_int), ("wdtype", ctypes.c_int),
-                ("layer_id", ctypes.c_int), ("seed", ctypes.c_uint64)]
+                ("layer_id", ctypes.c_int), ("seed", ctypes.c_uint64),
+                ("bias_select_only", ctypes.c_int), ("routed_scale", ctypes.c_double)]
 
 
 _WNAMES = ("wqkv", "wo", "wr", "wg", "wu", "wd", "g1", "g2")
@@ -80,9 +81,10 @@ def lib() -> ctypes.CDLL:
     return _lib
 
 
-def _cfg(dims, wdtype=0, layer_id=0, seed=0) -> _Cfg:
+def _cfg(dims, wdtype=0, layer_id=0, seed=0, bias_select_only=False, routed_scale=1.0) -> _Cfg:
     return _Cfg(dims.hidden, dims.q_heads, dims.kv_heads, dims.head_dim, dims.n_experts,
-                dims.top_k, dims.n_shared, dims.inter, wdtype, layer_id, seed)
+                dims.top_k, dims.n_shared, dims.inter, wdtype, layer_id, seed,
+                1 if bias_select_only else 0, routed_scale)
 
 
 def _p(a):
@@ -188,19 +190,22 @@ def layer_full(dims, x, kc, vc, k_scale, v_scale, seq, pos, *, wdtype=0, layer_i
 
 
 def layer(dims, x, attn, *, wdtype=0, layer_id=0, seed=0, bias=None, weights=None,
-          forced_idx=None, ksplit=1, nthreads=None, want_qkv=True) -> dict:
+          forced_idx=None, ksplit=1, nthreads=None, want_qkv=True, bias_select_only=False,
+          routed_scale=1.0) -> dict:
     """Evaluate one layer for M tokens.
 
     x, attn: fp64 arrays [M, H], [M, A] (the exact values the GPU receives,
     e.g. decoded bf16).  weights: optional dict of explicit fp64 logical
     weights (wqkv, wo, wr, wg, wu, wd; expert arrays shared-first).
-    Returns fp64 qkv, h1, logits, gates, out and int32 idx.
+    Returns fp64 qkv, h1, logits, gates, out and int32 idx.  bias_select_only:
+    the bias chooses the experts only (gates from the unbiased logits, which
+    are then the returned logits); routed_scale: factor on the routed sum.
     """
     x = np.ascontiguousarray(x, np.float64)
     attn = np.ascontiguousarray(attn, np.float64)
     M = x.shape[0]
     assert x.shape == (M, dims.hidden) and attn.shape == (M, dims.attn)
-    c = _cfg(dims, wdtype, layer_id, seed)
+    c = _cfg(dims, wdtype, layer_id, seed, bias_select_only, routed_scale)
     keep = []
     wp = _weights_ptr(weights, keep)
     b = None if bias is None else np.ascontiguousarray(bias, np.float64)

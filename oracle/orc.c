@@ -229,16 +229,20 @@ static void moe_block(const orc_cfg* c, const orc_weights* w, const dims* d, con
   /* router logits, selection, renormalised softmax over the selection */
   double* lg = (double*)malloc(sizeof(double) * (size_t)M * d->E);
   matvec(c, w, d, K_R, -1, v, d->H, all, M, lg, d->E, ksplit, nthreads);
-  if (bias)
-    for (int t = 0; t < M; ++t)
-      for (int e = 0; e < d->E; ++e) lg[(size_t)t * d->E + e] += bias[e];
+  /* selection keys: logits + bias; the gates' logits: the same, or with
+   * bias_select_only the unbiased logits */
+  double* key = (double*)malloc(sizeof(double) * (size_t)M * d->E);
+  for (int t = 0; t < M; ++t)
+    for (int e = 0; e < d->E; ++e)
+      key[(size_t)t * d->E + e] = lg[(size_t)t * d->E + e] + (bias ? bias[e] : 0.0);
+  if (!c->bias_select_only) memcpy(lg, key, sizeof(double) * (size_t)M * d->E);
   int* sel = (int*)malloc(sizeof(int) * (size_t)M * d->k);
   double* g = (double*)malloc(sizeof(double) * (size_t)M * d->k);
   for (int t = 0; t < M; ++t) {
     int* s = sel + (size_t)t * d->k;
     const double* l = lg + (size_t)t * d->E;
     if (forced_idx) memcpy(s, forced_idx + (size_t)t * d->k, sizeof(int) * (size_t)d->k);
-    else topk(l, d->E, d->k, s);
+    else topk(key + (size_t)t * d->E, d->E, d->k, s);
     double mx = l[s[0]];
     for (int j = 1; j < d->k; ++j) if (l[s[j]] > mx) mx = l[s[j]];
     double den = 0.0;
@@ -269,15 +273,17 @@ static void moe_block(const orc_cfg* c, const orc_weights* w, const dims* d, con
       memcpy(yr + ((size_t)tok[q] * d->k + slot[q]) * d->H, y + (size_t)q * d->H,
              sizeof(double) * (size_t)d->H);
   }
+  const double rs = c->routed_scale != 0.0 ? c->routed_scale : 1.0;
   for (int t = 0; t < M; ++t)
     for (int j = 0; j < d->k; ++j) {
-      double gj = g[(size_t)t * d->k + j];
+      double gj = rs * g[(size_t)t * d->k + j];
       const double* yy = yr + ((size_t)t * d->k + j) * d->H;
       for (int h = 0; h < d->H; ++h) out[(size_t)t * d->H + h] += gj * yy[h];
     }
   if (logits_out) memcpy(logits_out, lg, sizeof(double) * (size_t)M * d->E);
   if (idx_out) memcpy(idx_out, sel, sizeof(int) * (size_t)M * d->k);
   if (gates_out) memcpy(gates_out, g, sizeof(double) * (size_t)M * d->k);
+  free(key);
   free(all); free(lg); free(sel); free(g); free(y); free(yr); free(tok); free(slot);
 }
 

@@ -21,6 +21,12 @@
  *   F_e(v)   = Wd_e ( silu(Wg_e v) * (Wu_e v) ),  silu(z) = z / (1 + e^-z)
  *   out_t    = h1_t + F_shared(h1_t) + sum_{e in S_t} g_{t,e} F_e(h1_t)
  *
+ * Two variants of the gating (configuration fields): with bias_select_only
+ * the bias enters the selection only, S_t = top-k(Wr h1_t + b) and g over
+ * the unbiased logits Wr h1_t (the selection-only expert bias of
+ * DeepSeek-V3-style routers); routed_scale s multiplies the routed sum,
+ * out_t = h1_t + F_shared(h1_t) + s sum_e g_{t,e} F_e(h1_t).
+ *
  * Weights are either given explicitly (fp64 arrays, for hand-built cases) or
  * generated from the seed exactly as the GPU receives them (bf16 values, or
  * FP8 e4m3 codes times the fp32 scale of their 128 x 128 block) and decoded
@@ -44,6 +50,10 @@ typedef struct orc_cfg {
   int wdtype;                       /* 0 = bf16, 1 = FP8 e4m3 + block scale */
   int layer_id;                     /* generator stream id of the layer    */
   uint64_t seed;
+  int bias_select_only;             /* 1: the router bias chooses the experts
+                                       only; the gates are the softmax of the
+                                       unbiased logits over the selection   */
+  double routed_scale;              /* factor on the routed experts' sum (0 = 1) */
 } orc_cfg;
 
 /* Explicit logical weights, row-major fp64.  Expert arrays hold the shared
@@ -60,6 +70,8 @@ typedef struct orc_weights {
 } orc_weights;
 
 /* One layer for M tokens.  Returns 0, or -1 on bad arguments.
+ *   logits (output) are the biased logits, or with bias_select_only the
+ *   unbiased ones.
  *   w          NULL -> weights generated from cfg->seed / cfg->layer_id
  *   bias       [E] additive router bias or NULL
  *   x, attn    [M, H], [M, A]

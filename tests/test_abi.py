@@ -47,7 +47,7 @@ def test_host_side_argument_errors(kd):
     # invalid configurations are rejected before any device call
     bad = [dict(hidden=100), dict(top_k=0), dict(top_k=9, n_experts=8), dict(max_tokens=65),
            dict(max_tokens=0), dict(wdtype=7), dict(n_shared=2), dict(inter=96), dict(n_experts=2000),
-           dict(hidden=32768), dict(mma_min_tokens=-1)]
+           dict(hidden=32768), dict(mma_min_tokens=-1), dict(bias_select_only=3)]
     for b in bad:
         f = dict(hidden=256, q_heads=4, kv_heads=1, head_dim=64, n_experts=8, top_k=2,
                  n_shared=1, inter=128, wdtype=0, layer_id=0, max_tokens=4, router_bias=None,
@@ -56,7 +56,18 @@ def test_host_side_argument_errors(kd):
         cfg = kd._Config(**f)
         assert L.kd_layer_create(ctypes.byref(cfg), 0, ctypes.byref(h)) == kd.KD_EINVAL, b
         assert kd.lib().kd_last_error().decode()
+    # full-layer geometry the attention kernels do not take
+    for b in [dict(head_dim=96), dict(kv_heads=0), dict(q_heads=6, kv_heads=2, head_dim=128),
+              dict(kv_n_seq=0), dict(kv_max_ctx=0), dict(k_scale=0.0), dict(full_layer=2)]:
+        f = dict(hidden=256, q_heads=4, kv_heads=1, head_dim=64, n_experts=8, top_k=2,
+                 n_shared=1, inter=128, wdtype=0, layer_id=0, max_tokens=4, router_bias=None,
+                 mma_min_tokens=0, full_layer=1, rms_eps=0.0, kv_n_seq=2, kv_max_ctx=16,
+                 k_scale=0.01, v_scale=0.01)
+        f.update(b)
+        cfg = kd._Config(**f)
+        assert L.kd_layer_create(ctypes.byref(cfg), 0, ctypes.byref(h)) == kd.KD_EINVAL, b
     assert L.kd_decode_layer(None, None, None, 1, None) == kd.KD_EINVAL
+    assert L.kd_decode_layer_full(None, None, None, None, None, None, 1, None) == kd.KD_EINVAL
     assert L.kd_layer_check(None) == kd.KD_EINVAL
     assert L.kd_layer_qkv(None) is None
     assert L.kd_layer_bytes(None, None, None) == kd.KD_EINVAL

@@ -91,7 +91,7 @@ def test_tiny_layer_parity(kd, wdtype, M):
     try:
         x, a = inputs(d, M, rho=0.5)
         g = run_gpu_layer(L, x, a)
-        compare_layer(d, g, x, a, wdtype=wdtype, strict_raw=True)
+        compare_layer(d, g, x, a, wdtype=wdtype)
         assert g["counts"].sum() == M * d.top_k
         assert g["n_active"] == int((g["counts"] > 0).sum())
     finally:
@@ -109,6 +109,26 @@ def test_tiny_variants(kd):
             x, a = inputs(d, 7)
             g = run_gpu_layer(L, x, a)
             compare_layer(d, g, x, a, bias=None if bias is None else bias.astype(np.float64))
+        finally:
+            L.close()
+
+
+@pytest.mark.parametrize("wdtype", [0, 1])
+@pytest.mark.parametrize("M", [3, 8])
+def test_gating_variants(kd, wdtype, M):
+    """Selection-only router bias (the gates from the unbiased logits) and a
+    routed scaling factor, on both engines (M=3 CUDA cores, M=8 tensor cores)."""
+    d = TINY
+    bias = kdgen.zipf_bias(d.n_experts, 1.1)
+    for sel, rs in [(1, 1.0), (0, 2.5), (1, 0.75)]:
+        spec = kd.LayerSpec.from_dims(d, wdtype=wdtype, max_tokens=8, router_bias=bias,
+                                      bias_select_only=sel, routed_scale=rs)
+        L = kd.Layer(spec, seed=0)
+        try:
+            x, a = inputs(d, M, rho=0.3)
+            g = run_gpu_layer(L, x, a)
+            compare_layer(d, g, x, a, wdtype=wdtype, bias=bias.astype(np.float64),
+                          bias_select_only=bool(sel), routed_scale=rs)
         finally:
             L.close()
 
@@ -148,10 +168,10 @@ def test_error_paths(kd):
         assert kd.lib().kd_decode_layer(L.handle, None, a.data_ptr(), 1, None) == kd.KD_EINVAL
         L.decode(h, a, 4)
         L.check()
-        # launches per call: CUDA-core path below 4 tokens, tensor-core path
-        # (+ the combine launch) from 4; + the shared expert's gate/up
-        assert L.launches(1) == 5 and L.launches(3) == 5
-        assert L.launches(4) == 6
+        # launches per call: CUDA-core path below 3 tokens, tensor-core path
+        # (+ the combine launch) from 3; + the shared expert's gate/up
+        assert L.launches(1) == 5 and L.launches(2) == 5
+        assert L.launches(3) == 6 and L.launches(4) == 6
         with pytest.raises(kd.KdError) as ei:
             L.launches(5)
         assert ei.value.code == kd.KD_ERANGE
@@ -172,7 +192,7 @@ def test_batch1_layer_parity(kd, k2_layer):
     w = WORKLOADS["batch1"]
     x, a = w.hidden_in(), w.attn_out()
     g = run_gpu_layer(k2_layer, x, a)
-    r = compare_layer(K2, g, x, a, strict_raw=True)
+    r = compare_layer(K2, g, x, a, strict_raw=True)   # floor 0.0099 at this input
     assert g["n_active"] == 8
     print("batch1", r)
 
@@ -188,8 +208,8 @@ def test_verify8_layer_parity(kd, k2_layer):
 
 @pytest.mark.parametrize("M", [2, 3, 4, 5, 6, 7, 16])
 def test_k2_other_token_counts(kd, k2_layer, M):
-    """All rows at M = 2, 3 (CUDA-core engine), 4 (the switch to the tensor
-    cores), 5..7 (speculative verify with 4..6 draft tokens + 1, correlated
+    """All rows at M = 2 (CUDA-core engine), 3 (the switch to the tensor
+    cores), 4..7 (speculative verify with 3..6 draft tokens + 1, correlated
     rows) and 16."""
     x, a = inputs(K2, M, seed=3, rho=0.9 if 4 <= M <= 7 else 0.0)
     g = run_gpu_layer(k2_layer, x, a)

@@ -362,3 +362,60 @@ def test_golden_tiny_regression():
     assert np.array_equal(r["idx"][0], vals["idx"].astype(int))
     for k in ("gates", "out"):
         assert np.allclose(r[k][0], vals[k], rtol=1e-12, atol=1e-14), k
+
+
+# ------------------------------------------------------------- gating variants
+
+TRI = Dims(hidden=2, q_heads=1, kv_heads=0, head_dim=2, n_experts=3, top_k=2, n_shared=1, inter=1)
+
+
+def tri_weights(shared_down=1.0):
+    # Wo = 0 so h1 = x = (1, 1); router logits (3, 2, 1); every expert's
+    # SwiGLU value is silu(1) * 1 on row 0, times its own down column
+    return {
+        "wqkv": np.zeros((2, 2)), "wo": np.zeros((2, 2)),
+        "wr": np.array([[3.0, 0.0], [2.0, 0.0], [1.0, 0.0]]),
+        "wg": np.array([[[1.0, 0.0]]] * 4), "wu": np.array([[[1.0, 0.0]]] * 4),
+        "wd": np.array([[[shared_down], [0.0]], [[1.0], [0.0]], [[0.0], [1.0]], [[1.0], [1.0]]]),
+    }
+
+
+def test_selection_only_bias_hand_computed():
+    # bias (0, 0, 2.5): keys (3, 2, 3.5) select experts 2 then 0.  Gates over
+    # the selection: biased logits (3.5, 3) in the plain reading, unbiased
+    # (1, 3) with the selection-only bias.
+    x, a = np.array([[1.0, 1.0]]), np.zeros((1, 2))
+    b = np.array([0.0, 0.0, 2.5])
+    plain = oracle.layer(TRI, x, a, weights=tri_weights(), bias=b)
+    sel = oracle.layer(TRI, x, a, weights=tri_weights(), bias=b, bias_select_only=True)
+    assert list(plain["idx"][0]) == [2, 0] and list(sel["idx"][0]) == [2, 0]
+    assert np.allclose(plain["gates"][0], [1 / (1 + math.exp(-0.5)), 1 / (1 + math.exp(0.5))],
+                       rtol=1e-15)
+    assert np.allclose(sel["gates"][0], [1 / (1 + math.exp(2.0)), 1 / (1 + math.exp(-2.0))],
+                       rtol=1e-15)
+    assert np.array_equal(sel["logits"][0], [3.0, 2.0, 1.0])      # unbiased
+    assert np.array_equal(plain["logits"][0], [3.0, 2.0, 3.5])    # biased
+    # out = h1 + silu(1) (shared down (1, 0)) + sum_j g_j silu(1) down_{e_j}
+    s1 = silu(1.0)
+    g2, g0 = sel["gates"][0]
+    want = np.array([1 + s1 + g2 * s1 * 1.0 + g0 * s1 * 1.0, 1 + g2 * s1 * 1.0 + g0 * 0.0])
+    assert np.allclose(sel["out"][0], want, rtol=1e-15)
+
+
+def test_routed_scale_multiplies_the_routed_sum():
+    x, a = tiny_inputs(M=3)
+    base = oracle.layer(TINY, x, a, want_qkv=False)
+    for s in (0.5, 2.5):
+        r = oracle.layer(TINY, x, a, want_qkv=False, routed_scale=s)
+        assert np.array_equal(r["idx"], base["idx"])
+        # shared part: the layer with the routed sum scaled by 0 is h1 + shared
+        sh = oracle.layer(TINY, x, a, want_qkv=False, routed_scale=1e-300)["out"]
+        assert np.allclose(r["out"] - sh, s * (base["out"] - sh), rtol=1e-12, atol=1e-13)
+
+
+def test_selection_only_bias_equals_plain_without_bias():
+    x, a = tiny_inputs(M=2)
+    r0 = oracle.layer(TINY, x, a, want_qkv=False)
+    r1 = oracle.layer(TINY, x, a, want_qkv=False, bias=np.zeros(TINY.n_experts),
+                      bias_select_only=True)
+    assert np.array_equal(r0["out"], r1["out"]) and np.array_equal(r0["idx"], r1["idx"])
