@@ -261,9 +261,10 @@ KD_DEV MmaShared carve_mma_smem(uint8_t* base, int nmax, int terms, int nsub, bo
   MmaShared s;
   s.nsub = nsub;
   s.stage_bytes = nsub * (aterms * kATileBytes + b_sub_bytes(nmax, terms));   // bf16: A + B
-  // q8: + a staging area for the rows' fp32 activations of the chunk (512 B a row)
+  // q8: + a staging area for the rows' fp32 activations of the chunk (512 B a
+  // row, for the launch's largest token count; stages stay 1024-aligned)
   s.xoff = s.stage_bytes;
-  if (q8) s.stage_bytes += pad16(nmax) * 512;
+  if (q8) s.stage_bytes += ((nmax + 1) / 2) * 1024;
   uintptr_t p = (reinterpret_cast<uintptr_t>(base) + 1023) & ~uintptr_t(1023);
   s.stage = reinterpret_cast<uint8_t*>(p);
   uint64_t* bars = reinterpret_cast<uint64_t*>(p + (size_t)kMRingBytes);
