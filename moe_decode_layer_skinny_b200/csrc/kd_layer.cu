@@ -594,8 +594,10 @@ static int launch_layer(kd_layer* L, const Acts& a, cudaStream_t s, const kd_lay
   const bool mma = L->has_maps && M >= L->mma_min;
   const size_t msm = kMmaSmem;
   // FP8 projections convert their e4m3 tiles (converter warps); the FP8
-  // experts multiply them as they land
+  // experts multiply them as they land (with kQ8Conv converter warps for
+  // their activation terms)
   const int mthreads = kMThreads;
+  const int ethreads = fp8 ? kMThreadsQ8 : kMThreads;
   if (L->timing) KD_CUDA(cudaEventRecord(L->tev[0], s));
   // Main stream: projections -> router (logits, selection, token lists in one
   // launch) -> routed gate/up -> down + combine.  Side stream: the shared
@@ -626,7 +628,7 @@ static int launch_layer(kd_layer* L, const Acts& a, cudaStream_t s, const kd_lay
   if (d.S) {
     KD_CUDA(cudaStreamWaitEvent(L->side, L->ev_h1, 0));
     if (mma)
-      KD_CUDA(launch(fp8 ? mma_gateup_kernel<true> : mma_gateup_kernel<false>, G, mthreads, msm,
+      KD_CUDA(launch(fp8 ? mma_gateup_kernel<true> : mma_gateup_kernel<false>, G, ethreads, msm,
                      L->side, false, d, M, 1, L->maps));
     else
       KD_CUDA(launch(fp8 ? gateup_kernel<W_FP8> : gateup_kernel<W_BF16>, G, kThreads, sm, L->side,
@@ -635,7 +637,7 @@ static int launch_layer(kd_layer* L, const Acts& a, cudaStream_t s, const kd_lay
   }
   if (L->timing) KD_CUDA(cudaEventRecord(L->tev[2], s));
   if (mma)
-    KD_CUDA(launch(fp8 ? mma_gateup_kernel<true> : mma_gateup_kernel<false>, G, mthreads, msm, s,
+    KD_CUDA(launch(fp8 ? mma_gateup_kernel<true> : mma_gateup_kernel<false>, G, ethreads, msm, s,
                    !L->timing, d, M, 0, L->maps));
   else
     KD_CUDA(launch(fp8 ? gateup_kernel<W_FP8> : gateup_kernel<W_BF16>, G, kThreads,
@@ -653,7 +655,7 @@ static int launch_layer(kd_layer* L, const Acts& a, cudaStream_t s, const kd_lay
   const bool pdl_down = !L->timing && !d.S && !(next && pf);
   if (mma) {
     // tensor-core down writes each expert's outputs; the combine follows
-    KD_CUDA(launch(fp8 ? mma_down_kernel<true> : mma_down_kernel<false>, G, mthreads, msm, s,
+    KD_CUDA(launch(fp8 ? mma_down_kernel<true> : mma_down_kernel<false>, G, ethreads, msm, s,
                    pdl_down, d, M, L->maps));
     KD_CUDA(launch(combine_kernel, 2 * G, 256, 0, s, !L->timing, d, M, a.out));
   } else

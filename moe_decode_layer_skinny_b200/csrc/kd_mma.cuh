@@ -9,10 +9,12 @@
 //   warp 1      MMA issuer: owns the TMEM accumulators (two buffers of N fp32
 //               columns), issues tcgen05.mma, commits stage releases
 //   warps 2-3   B producers: gather the tokens' bf16 rows (64 K at a time)
-//               into the stage in the same swizzled K-major layout
+//               into the stage in the same swizzled K-major layout (q8
+//               plans: warp 2 copies the fp32 rows, warp 3 converts them)
 //   warps 4-7   epilogue: tcgen05.ld of the accumulator (lane = weight row),
 //               then the plan's epilogue, or a split-K partial
 //   warps 8-15  FP8 projections only: e4m3 tiles -> scaled bf16 A tiles
+//   warp 8      q8 plans: the second converter (the two take alternate stages)
 // Activations that must stay fp32-accurate come as a sum of bf16 terms, all
 // multiplied into the same accumulator: the expert inputs (h1, the SwiGLU
 // activations) as hi + lo (hi = bf16(v), lo = bf16(v - hi): ~16 significant
@@ -123,6 +125,8 @@ KD_DEV void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "
 
 constexpr int kMThreads = 256;
 constexpr int kMThreadsF8 = 512;      // + 8 converter warps (e4m3 -> bf16 A tiles)
+constexpr int kQ8Conv = 2;            // q8 converter warps (warp 3, then warps 8 ..)
+constexpr int kMThreadsQ8 = kMThreads + 32 * (kQ8Conv - 1);
 constexpr int kMaxMStages = 16;
 constexpr int kATileBytes = 128 * 128;                // 128 rows x 64 bf16 (one swizzle atom wide)
 constexpr int kMaxSub = 2;                            // 64-K sub-tiles per stage (at most)
@@ -130,7 +134,7 @@ constexpr int kMRingBytes = 222 * 1024;                // stages (+ 3 KB below: 
 constexpr int kMaxN = 64;                             // tokens per MMA (N)
 constexpr int kMaxTerms = 3;                          // bf16 terms of an activation
 constexpr size_t kWsFloatsPerCta = 2 * 128 * 64;     // split-K partial slots of one CTA
-constexpr size_t kMmaSmem = (size_t)kMRingBytes + 1024 /*align*/ + 2048 /*barriers, scratch*/;
+constexpr size_t kMmaSmem = (size_t)kMRingBytes + 1024 /*align*/ + 3072 /*barriers, scratch*/;
 constexpr int kQ8AccCols = 256;                       // q8: one accumulator, <= 2 x 2 x 64 columns
 constexpr int kQ8TmemCols = 2 * kQ8AccCols;           // q8: two accumulators
 constexpr int kQGroup = 64;                           // activation elements per stored maximum
@@ -237,6 +241,7 @@ struct MmaShared {
   int* misc;             // [8] scratch ([0] split-K last part, [2] after-run flag)
   float* qmax;           // [4][16] per-warp column maxima (output group maxima)
   float* qtab;           // [2][kMaxN] q8 epilogue: 2^-P per (variant, token) of the unit
+  float* cpm;            // [kQ8Conv][2][kMaxN] q8 converters: 2^P per (variant, token) of the unit
 };
 
 // The ring holds as many stages as fit.  A stage covers nsub x 64 K: nsub
@@ -309,6 +314,7 @@ KD_DEV MmaShared carve_mma_smem(uint8_t* base, int nmax, int terms, int nsub, bo
   s.misc = s.abort_flag + 1;
   s.qmax = reinterpret_cast<float*>(s.misc + 8);
   s.qtab = s.qmax + 64;
+  s.cpm = s.qtab + 2 * kMaxN;   // ends below 2.7 KB of the 3 KB region
   // without a raw ring its barriers serve the A tiles' transactions
   s.afull = s.rfull;
   s.xfull = s.rempty + kMaxMStages;   // the B ring's barriers, unused without a raw ring
@@ -316,7 +322,12 @@ KD_DEV MmaShared carve_mma_smem(uint8_t* base, int nmax, int terms, int nsub, bo
   return s;
 }
 
+// A role's wait on a pipeline barrier: true once the phase completed; false
+// after an abort (another role gave up) or after the time limit (this one
+// gives up: it raises the abort flag and records the error).  A phase that
+// has already completed is taken without reading the flag.
 KD_DEV bool mwait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, unsigned* err) {
+  if (mbar_try_wait(bar, parity)) return true;
   if (*abort_flag) return false;
   if (mbar_wait(bar, parity)) return true;
   *abort_flag = 1;
@@ -653,7 +664,9 @@ KD_DEV void mma_issuer(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigned*
 template <class Plan>
 KD_DEV void mma_issuer_q8(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigned* err) {
   constexpr int NV = Plan::kVariants, nh = kQTerms;
-  uint32_t it = 0, nu = 0;
+  uint32_t nu = 0, ph = 0;
+  int s = 0;
+  const uint32_t ring0 = smem_u32(sh.stage);
   CtaUnits<Plan> units(plan);
   MUnit m;
   for (; units.next(m); ++nu) {
@@ -665,14 +678,13 @@ KD_DEV void mma_issuer_q8(const Plan& plan, MmaShared& sh, uint32_t tmem, unsign
     tc_fence_after();
     const uint32_t d0 = tmem + (uint32_t)(buf * kQ8AccCols);
     bool ok = true;
-    for (int c = 0; c < m.nkc; ++c, ++it) {
-      const int s = it % sh.nst;
-      const uint32_t ph = (it / sh.nst) & 1u;
+    for (int c = 0; c < m.nkc; ++c) {
       ok = mwait(&sh.afull[s], ph, sh.abort_flag, err) && mwait(&sh.full[s], ph, sh.abort_flag, err);
       if (!ok) break;
-      fence_proxy_async_smem();   // the B terms (generic proxy) -> tensor core reads
+      // (the converter fenced its B writes against the async proxy before
+      // its arrival)
       tc_fence_after();
-      const uint32_t a0 = smem_u32(sh.stage + (size_t)s * sh.stage_bytes);
+      const uint32_t a0 = ring0 + (uint32_t)(s * sh.stage_bytes);
       // descriptors by adding byte offsets / 16 to the start-address field
       // (shared addresses < 256 KB: the field never carries)
       const uint64_t ad0 = sw128_desc(a0), bd0 = sw128_desc(a0 + sh.boff);
@@ -682,6 +694,7 @@ KD_DEV void mma_issuer_q8(const Plan& plan, MmaShared& sh, uint32_t tmem, unsign
         mma_e4m3(d0, ad0 + off, bd0 + off, idesc, c > 0 || k > 0);
       }
       mma_commit(&sh.empty[s]);   // the stage is free once these MMAs are done
+      if (++s == sh.nst) { s = 0; ph ^= 1u; }
     }
     if (!ok) break;
     mma_commit(&sh.accfull[buf]);
@@ -705,13 +718,18 @@ KD_DEV float q8_unit_scale(const Plan& plan, const MUnit& m, int j, int v, float
 // rows' fp32 activations of the stage's 128-K chunk with cp.async into the
 // stage's staging area (after its B terms); each lane's copies arrive on the
 // stage's xfull barrier when they land, so every stage of the ring can have
-// copies in flight.  Warp 3 (converter) waits for a stage's rows and writes
-// x times (block scale x 2^P) as kQTerms e4m3 terms per scale variant, in
-// the 128-byte swizzle, then arrives on the stage's full barrier.  Rows past
-// ntok are left as they are: their MMA columns are not read.
+// copies in flight.  The converter warps (kQ8Conv of them, alternate stages)
+// wait for a stage's rows and write x times (block scale x 2^P) as kQTerms
+// e4m3 terms per scale variant, in the 128-byte swizzle, then arrive on the
+// stage's full barrier.  Rows past ntok are left as they are: their MMA
+// columns are not read.
+//
+// One stage by one converter warp: (row, 8-element piece) pairs p = lane +
+// 32 u, row p / 16, piece p % 16 (K elements 8 (p % 16) ..), so that every
+// lane has work from two tokens up; pm = the warp's 2^P table of the unit.
 template <class Plan>
 KD_DEV void q8_convert_stage(const Plan& plan, MmaShared& sh, const MUnit& m, int c, int s,
-                             const float (&pm)[16][2]) {
+                             const float* pm) {
   constexpr int NV = Plan::kVariants, nh = kQTerms;
   const int lane = threadIdx.x & 31;
   const int N = pad16(m.ntok);
@@ -721,32 +739,30 @@ KD_DEV void q8_convert_stage(const Plan& plan, MmaShared& sh, const MUnit& m, in
   float ws[NV];
 #pragma unroll
   for (int v = 0; v < NV; ++v) ws[v] = plan.w_scale_v(m, kc, v);
-  // (row, 16-element chunk) pairs p = lane + 32 u: row p / 8, chunk p % 8
+  const int np = m.ntok * 16;
 #pragma unroll 1
-  for (int u = 0; u < 16; ++u) {
-    const int p = lane + 32 * u, r = p >> 3, ch = p & 7;
-    if (r >= m.ntok) break;
-    float x[16];
+  for (int p = lane; p < np; p += 32) {
+    const int r = p >> 4, pc = p & 15;
+    float x[8];
     {
-      const float4* src = reinterpret_cast<const float4*>(xs + (size_t)r * 512 + ch * 64);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float4 f = src[q];
-        x[4 * q] = f.x; x[4 * q + 1] = f.y; x[4 * q + 2] = f.z; x[4 * q + 3] = f.w;
-      }
+      const float4* src = reinterpret_cast<const float4*>(xs + (size_t)r * 512 + pc * 32);
+      const float4 f0 = src[0], f1 = src[1];
+      x[0] = f0.x; x[1] = f0.y; x[2] = f0.z; x[3] = f0.w;
+      x[4] = f1.x; x[5] = f1.y; x[6] = f1.z; x[7] = f1.w;
     }
-    const uint32_t swz = (uint32_t)((ch ^ (r & 7)) * 16);
+    // 16-byte chunk pc / 2 of the row, swizzled; this piece is its half pc % 2
+    const uint32_t off = (uint32_t)((((pc >> 1) ^ (r & 7)) << 4) | ((pc & 1) << 3));
 #pragma unroll
     for (int v = 0; v < NV; ++v) {
-      const float f = ws[v] * pm[u][v];
-      float w[16];
+      const float f = ws[v] * pm[v * kMaxN + r];
+      float w[8];
 #pragma unroll
-      for (int e = 0; e < 16; ++e) w[e] = x[e] * f;
+      for (int e = 0; e < 8; ++e) w[e] = x[e] * f;
 #pragma unroll
       for (int h = 0; h < nh; ++h) {
-        uint32_t pk[4];
+        uint32_t pk[2];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
+        for (int e = 0; e < 4; ++e) {
           const uint32_t c2 = e4m3x2_rn(w[2 * e], w[2 * e + 1]);
           if (e & 1) pk[e >> 1] |= c2 << 16;
           else pk[e >> 1] = c2;
@@ -756,8 +772,8 @@ KD_DEV void q8_convert_stage(const Plan& plan, MmaShared& sh, const MUnit& m, in
             w[2 * e + 1] -= tv.y;
           }
         }
-        *reinterpret_cast<uint4*>(bt + (size_t)((v * nh + h) * N + r) * 128 + swz) =
-            make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        *reinterpret_cast<uint2*>(bt + (size_t)((v * nh + h) * N + r) * 128 + off) =
+            make_uint2(pk[0], pk[1]);
       }
     }
   }
@@ -792,20 +808,23 @@ KD_DEV void mma_copier_q8(const Plan& plan, MmaShared& sh, unsigned* err) {
   cp_async_wait<0>();   // nothing in flight when the warp leaves
 }
 
-// Warp 3: per stage, wait for its rows, convert, release.
+// Converter warp cw (warp 3, then warps 8 ..): per unit, the 2^P table of
+// its tokens; then, for each stage of the unit that is its own (stage
+// counter mod kQ8Conv), wait for the rows, convert, release.
 template <class Plan>
-KD_DEV void mma_converter_q8(const Plan& plan, MmaShared& sh, unsigned* err) {
+KD_DEV void mma_converter_q8(const Plan& plan, MmaShared& sh, int cw, unsigned* err) {
   constexpr int NV = Plan::kVariants;
   const int lane = threadIdx.x & 31;
-  float pm[16][2];
+  float* pm = sh.cpm + cw * 2 * kMaxN;
   uint32_t it = 0;
   CtaUnits<Plan> units(plan);
   MUnit m;
   while (units.next(m)) {
-    // 2^P of this lane's conversion rows (lane / 8 + 4 u) for the unit: each
-    // row's largest |x| x block scale over the tile's groups.  The lanes
-    // split the groups; the block scales are loaded once, and 8 rows' loads
-    // are all issued before their reductions.
+    // 2^P per (variant, token) of the unit: each token's largest |x| x block
+    // scale over the tile's groups.  The lanes split the groups; the block
+    // scales are loaded once, and 8 rows' loads are all issued before their
+    // reductions.
+    __syncwarp();   // the previous unit's conversions are done with the table
     {
       constexpr int kG = 4;   // groups per lane (<= 128 groups: K <= 8192)
       const int ng = plan.kgroups();
@@ -845,12 +864,13 @@ KD_DEV void mma_converter_q8(const Plan& plan, MmaShared& sh, unsigned* err) {
             for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
             float inv;
             const float sc = q_scale(amax, inv);
-            const int r = r0 + rr;
-            if (r < m.ntok && (r & 3) == (lane >> 3)) pm[r >> 2][v] = sc;
+            if (lane == rr && r0 + rr < m.ntok) pm[v * kMaxN + r0 + rr] = sc;
           }
       }
     }
+    __syncwarp();
     for (int c = 0; c < m.nkc; ++c, ++it) {
+      if ((int)(it % kQ8Conv) != cw) continue;
       const int s = it % sh.nst;
       mwait(&sh.xfull[s], (it / sh.nst) & 1u, sh.abort_flag, err);
       q8_convert_stage(plan, sh, m, c, s, pm);
@@ -1172,7 +1192,7 @@ KD_DEV void mma_run(const Plan& plan, uint8_t* smem_raw, unsigned* err) {
   } else if (warp < 4) {
     if constexpr (Plan::kQ8) {
       if (warp == 2) mma_copier_q8(plan, sh, err);
-      else mma_converter_q8(plan, sh, err);
+      else mma_converter_q8(plan, sh, 0, err);
     } else {
       mma_producer_b(plan, sh, err);
     }
@@ -1181,6 +1201,8 @@ KD_DEV void mma_run(const Plan& plan, uint8_t* smem_raw, unsigned* err) {
     else mma_epilogue(plan, sh, tmem, err);
   } else if constexpr (Plan::kFp8) {
     mma_converter(plan, sh, err);
+  } else if constexpr (Plan::kQ8) {
+    mma_converter_q8(plan, sh, warp - 7, err);   // warps 8 ..
   }
   tc_fence_before();
   __syncthreads();

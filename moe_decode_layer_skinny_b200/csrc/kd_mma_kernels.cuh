@@ -341,7 +341,7 @@ struct MmaGateUpPlan {
 };
 
 template <bool F8>
-__global__ void __launch_bounds__(kMThreads, 1)
+__global__ void __launch_bounds__(F8 ? kMThreadsQ8 : kMThreads, 1)
     mma_gateup_kernel(LayerDev L, int M, int shared, const __grid_constant__ MmaMaps maps) {
   extern __shared__ uint8_t smem[];
   MmaGateUpPlan<F8> p;
@@ -434,7 +434,7 @@ struct MmaDownPlan {
 };
 
 template <bool F8>
-__global__ void __launch_bounds__(kMThreads, 1)
+__global__ void __launch_bounds__(F8 ? kMThreadsQ8 : kMThreads, 1)
     mma_down_kernel(LayerDev L, int M, const __grid_constant__ MmaMaps maps) {
   extern __shared__ uint8_t smem[];
   pdl_wait();
