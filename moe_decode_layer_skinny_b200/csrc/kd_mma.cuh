@@ -139,6 +139,7 @@ constexpr int kQ8AccCols = 256;                       // q8: one accumulator, <=
 constexpr int kQ8TmemCols = 2 * kQ8AccCols;           // q8: two accumulators
 constexpr int kQGroup = 64;                           // activation elements per stored maximum
 constexpr int kQTerms = 2;                            // e4m3 terms of a q8 activation
+constexpr int kQ8XBudget = 40 * 1024;                 // q8: bytes of the activation-row ring
 
 // One unit of work: K chunks [kc0, kc0 + nkc) of a 128-row weight tile.
 struct MUnit {
@@ -215,11 +216,15 @@ struct CtaUnits {
 struct MmaShared {
   uint8_t* stage;        // nst x stage_bytes, 1024-aligned
   int nst, stage_bytes;  // stage count and size (A tile + B tile for the launch's largest N)
-  int xoff;              // q8: offset of the activation staging area in a stage
+  // q8: a ring of its own for the activation rows of a stage (the copier
+  // refills a slot once a converter is done with it, ahead of the MMAs)
+  uint8_t* xring;
+  int nxs, xslot;
   int nsub;              // 64-K sub-tiles per stage
   uint64_t* full;        // [nst] B written (64 arrivals), or (FP8 converter) the A tile converted
   uint64_t* afull;       // [nst] bf16 / q8 plans: the A tile landed (TMA transaction count)
-  uint64_t* xfull;       // [nst] q8 plans: the stage's activation rows landed (32 arrivals)
+  uint64_t* xfull;       // [nxs] q8 plans: a slot's activation rows landed (32 arrivals)
+  uint64_t* xempty;      // [nxs] q8 plans: a converter is done with the slot (32 arrivals)
   uint64_t* empty;       // [nst] MMAs of the stage done
   uint64_t* accfull;     // [2] accumulator buffer ready for the epilogue
   uint64_t* accempty;    // [2] epilogue done reading the accumulator
@@ -266,10 +271,16 @@ KD_DEV MmaShared carve_mma_smem(uint8_t* base, int nmax, int terms, int nsub, bo
   MmaShared s;
   s.nsub = nsub;
   s.stage_bytes = nsub * (aterms * kATileBytes + b_sub_bytes(nmax, terms));   // bf16: A + B
-  // q8: + a staging area for the rows' fp32 activations of the chunk (512 B a
-  // row, for the launch's largest token count; stages stay 1024-aligned)
-  s.xoff = s.stage_bytes;
-  if (q8) s.stage_bytes += ((nmax + 1) / 2) * 1024;
+  // q8: slots for the rows' fp32 activations of a 128-K chunk (512 B a row,
+  // for the launch's largest token count), as many as fit kQ8XBudget (2 ..
+  // kMaxMStages), after the stages
+  s.xslot = 0;
+  s.nxs = 0;
+  if (q8) {
+    s.xslot = ((nmax + 1) / 2) * 1024;
+    const int nx = kQ8XBudget / s.xslot;
+    s.nxs = nx < 2 ? 2 : (nx > kMaxMStages ? kMaxMStages : nx);
+  }
   uintptr_t p = (reinterpret_cast<uintptr_t>(base) + 1023) & ~uintptr_t(1023);
   s.stage = reinterpret_cast<uint8_t*>(p);
   uint64_t* bars = reinterpret_cast<uint64_t*>(p + (size_t)kMRingBytes);
@@ -296,7 +307,7 @@ KD_DEV MmaShared carve_mma_smem(uint8_t* base, int nmax, int terms, int nsub, bo
     s.nraw = (rem - nb * bstage) / kRawBytes;
     if (s.nraw > kMaxMStages) s.nraw = kMaxMStages;
   } else {
-    s.nst = kMRingBytes / s.stage_bytes;
+    s.nst = (kMRingBytes - s.nxs * s.xslot) / s.stage_bytes;
     if (s.nst > kMaxMStages) s.nst = kMaxMStages;
     s.bst = s.stage;
     s.nbst = s.nst;
@@ -317,7 +328,10 @@ KD_DEV MmaShared carve_mma_smem(uint8_t* base, int nmax, int terms, int nsub, bo
   s.cpm = s.qtab + 2 * kMaxN;   // ends below 2.7 KB of the 3 KB region
   // without a raw ring its barriers serve the A tiles' transactions
   s.afull = s.rfull;
-  s.xfull = s.rempty + kMaxMStages;   // the B ring's barriers, unused without a raw ring
+  // q8: the B ring's barriers, unused without a raw ring
+  s.xring = s.stage + (size_t)s.nst * s.stage_bytes;
+  s.xfull = s.rempty + kMaxMStages;
+  s.xempty = s.xfull + kMaxMStages;
   s.drain = reinterpret_cast<uint64_t*>(s.misc + 4);
   return s;
 }
@@ -576,17 +590,29 @@ KD_DEV void mma_converter(const Plan& plan, MmaShared& sh, unsigned* err) {
   }
 }
 
-// After an abort: no MMA of this thread may still be running when TMEM is
-// freed: commit them to the drain barrier and wait (bounded).
-KD_DEV void drain_mma(MmaShared& sh) {
+// After an abort: no MMA of the issuing lane may still be running when TMEM
+// is freed: it commits them to the drain barrier and waits (bounded).
+KD_DEV void drain_mma(MmaShared& sh, bool issuing_lane) {
   if (!*sh.abort_flag) return;
-  mma_commit(sh.drain);
-  mbar_wait(sh.drain, 0);
+  if (issuing_lane) {
+    mma_commit(sh.drain);
+    mbar_wait(sh.drain, 0);
+  }
+  __syncwarp();
+}
+
+// The issuer runs on a whole warp with uniform control flow, so that the
+// operand descriptors are warp-uniform values; lane 0 issues the MMAs and
+// the commits.  Every lane waits; a wait counts as done only if it is done
+// for all of them.
+KD_DEV bool mwait_warp(uint64_t* bar, uint32_t parity, volatile int* abort_flag, unsigned* err) {
+  return __all_sync(0xffffffffu, mwait(bar, parity, abort_flag, err));
 }
 
 template <class Plan>
 KD_DEV void mma_issuer(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigned* err) {
   constexpr int nterms = Plan::kTerms;
+  const bool issue = (threadIdx.x & 31) == 0;
   uint32_t it = 0, nu_local = 0;
   CtaUnits<Plan> units(plan);
   MUnit m;
@@ -595,7 +621,7 @@ KD_DEV void mma_issuer(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigned*
     const uint32_t idesc = idesc_bf16(N);
     const int buf = nu_local & 1;
     const uint32_t d = tmem + (uint32_t)(buf * kMaxN);
-    if (!mwait(&sh.accempty[buf], ((nu_local >> 1) & 1u) ^ 1u, sh.abort_flag, err)) break;
+    if (!mwait_warp(&sh.accempty[buf], ((nu_local >> 1) & 1u) ^ 1u, sh.abort_flag, err)) break;
     tc_fence_after();
     bool ok = true;
     for (int c = 0; c < m.nkc; ++c, ++it) {
@@ -603,11 +629,11 @@ KD_DEV void mma_issuer(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigned*
       const uint32_t ph = (it / sh.nst) & 1u;
       const int sb = it % sh.nbst;
       if (Plan::kFp8) {
-        ok = mwait(&sh.full[s], ph, sh.abort_flag, err) &&
-             mwait(&sh.bfull[sb], (it / sh.nbst) & 1u, sh.abort_flag, err);
+        ok = mwait_warp(&sh.full[s], ph, sh.abort_flag, err) &&
+             mwait_warp(&sh.bfull[sb], (it / sh.nbst) & 1u, sh.abort_flag, err);
       } else {
-        ok = mwait(&sh.afull[s], ph, sh.abort_flag, err) &&
-             mwait(&sh.full[s], ph, sh.abort_flag, err);
+        ok = mwait_warp(&sh.afull[s], ph, sh.abort_flag, err) &&
+             mwait_warp(&sh.full[s], ph, sh.abort_flag, err);
       }
       if (!ok) break;
       fence_proxy_async_smem();   // the B gathers (generic proxy) -> tensor core reads
@@ -615,23 +641,24 @@ KD_DEV void mma_issuer(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigned*
       const uint32_t a0 = smem_u32(sh.stage + (size_t)s * sh.stage_bytes);
       const uint32_t b0 = smem_u32(sh.bst + (size_t)sb * sh.bst_bytes) + sh.boff;
       const int bsub = b_sub_bytes(N, nterms);
-      if constexpr (!Plan::kFp8) {
+      // descriptors by adding byte offsets / 16 to the start-address field
+      // (shared addresses < 256 KB: the field never carries)
+      const uint64_t ad0 = sw128_desc(a0), bd0 = sw128_desc(b0);
+      if (!issue) {
+      } else if constexpr (!Plan::kFp8) {
         for (int u = 0; u < sh.nsub; ++u) {
-          const uint32_t b = b0 + u * bsub;
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            const uint64_t ad = sw128_desc(a0 + u * kATileBytes + k * 32);
-            mma_bf16(d, ad, sw128_desc(b + k * 32), idesc, c > 0 || u > 0 || k > 0);
+            const uint64_t ad = ad0 + (uint64_t)((u * kATileBytes + k * 32) >> 4);
+            const uint64_t bd = bd0 + (uint64_t)((u * bsub + k * 32) >> 4);
+            mma_bf16(d, ad, bd, idesc, c > 0 || u > 0 || k > 0);
 #pragma unroll
             for (int h = 1; h < nterms; ++h)
-              mma_bf16(d, ad, sw128_desc(b + h * N * 128 + k * 32), idesc, true);
+              mma_bf16(d, ad, bd + (uint64_t)((h * N * 128) >> 4), idesc, true);
           }
         }
       } else {
-      // FP8: descriptors by adding byte offsets / 16 to the start-address
-      // field (shared addresses < 256 KB: the field never carries); the
-      // issuing thread shares its SM quarter with two converter warps
-      const uint64_t ad0 = sw128_desc(a0), bd0 = sw128_desc(b0);
+      // FP8 projections: the A terms of the converted tile
       for (int u = 0; u < sh.nsub; ++u) {
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -647,13 +674,17 @@ KD_DEV void mma_issuer(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigned*
         }
       }
       }
-      mma_commit(&sh.empty[s]);   // the stage is free once these MMAs are done
-      if (Plan::kFp8) mma_commit(&sh.bempty[sb]);
+      if (issue) {
+        mma_commit(&sh.empty[s]);   // the stage is free once these MMAs are done
+        if (Plan::kFp8) mma_commit(&sh.bempty[sb]);
+      }
+      __syncwarp();
     }
     if (!ok) break;
-    mma_commit(&sh.accfull[buf]);
+    if (issue) mma_commit(&sh.accfull[buf]);
+    __syncwarp();
   }
-  drain_mma(sh);
+  drain_mma(sh, issue);
 }
 
 // q8 plans: per stage (one e4m3 weight tile [128 x 128 K] and a B tile of
@@ -664,6 +695,7 @@ KD_DEV void mma_issuer(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigned*
 template <class Plan>
 KD_DEV void mma_issuer_q8(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigned* err) {
   constexpr int NV = Plan::kVariants, nh = kQTerms;
+  const bool issue = (threadIdx.x & 31) == 0;
   uint32_t nu = 0, ph = 0;
   int s = 0;
   const uint32_t ring0 = smem_u32(sh.stage);
@@ -674,12 +706,13 @@ KD_DEV void mma_issuer_q8(const Plan& plan, MmaShared& sh, uint32_t tmem, unsign
     // one MMA per K-step covers every (variant, term, token) row of the B tile
     const uint32_t idesc = idesc_e4m3(NV * nh * N);
     const int buf = nu & 1;
-    if (!mwait(&sh.accempty[buf], ((nu >> 1) & 1u) ^ 1u, sh.abort_flag, err)) break;
+    if (!mwait_warp(&sh.accempty[buf], ((nu >> 1) & 1u) ^ 1u, sh.abort_flag, err)) break;
     tc_fence_after();
     const uint32_t d0 = tmem + (uint32_t)(buf * kQ8AccCols);
     bool ok = true;
     for (int c = 0; c < m.nkc; ++c) {
-      ok = mwait(&sh.afull[s], ph, sh.abort_flag, err) && mwait(&sh.full[s], ph, sh.abort_flag, err);
+      ok = mwait_warp(&sh.afull[s], ph, sh.abort_flag, err) &&
+           mwait_warp(&sh.full[s], ph, sh.abort_flag, err);
       if (!ok) break;
       // (the converter fenced its B writes against the async proxy before
       // its arrival)
@@ -688,18 +721,22 @@ KD_DEV void mma_issuer_q8(const Plan& plan, MmaShared& sh, uint32_t tmem, unsign
       // descriptors by adding byte offsets / 16 to the start-address field
       // (shared addresses < 256 KB: the field never carries)
       const uint64_t ad0 = sw128_desc(a0), bd0 = sw128_desc(a0 + sh.boff);
+      if (issue) {
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const uint64_t off = (uint64_t)((k * 32) >> 4);
-        mma_e4m3(d0, ad0 + off, bd0 + off, idesc, c > 0 || k > 0);
+        for (int k = 0; k < 4; ++k) {
+          const uint64_t off = (uint64_t)((k * 32) >> 4);
+          mma_e4m3(d0, ad0 + off, bd0 + off, idesc, c > 0 || k > 0);
+        }
+        mma_commit(&sh.empty[s]);   // the stage is free once these MMAs are done
       }
-      mma_commit(&sh.empty[s]);   // the stage is free once these MMAs are done
+      __syncwarp();
       if (++s == sh.nst) { s = 0; ph ^= 1u; }
     }
     if (!ok) break;
-    mma_commit(&sh.accfull[buf]);
+    if (issue) mma_commit(&sh.accfull[buf]);
+    __syncwarp();
   }
-  drain_mma(sh);
+  drain_mma(sh, issue);
 }
 
 // 2^P for token j of a q8 unit and scale variant v (and 2^-P in inv): the
@@ -715,26 +752,28 @@ KD_DEV float q8_unit_scale(const Plan& plan, const MUnit& m, int j, int v, float
 }
 
 // q8 B producers.  Warp 2 (copier) copies, for every stage, the live token
-// rows' fp32 activations of the stage's 128-K chunk with cp.async into the
-// stage's staging area (after its B terms); each lane's copies arrive on the
-// stage's xfull barrier when they land, so every stage of the ring can have
-// copies in flight.  The converter warps (kQ8Conv of them, alternate stages)
-// wait for a stage's rows and write x times (block scale x 2^P) as kQTerms
-// e4m3 terms per scale variant, in the 128-byte swizzle, then arrive on the
-// stage's full barrier.  Rows past ntok are left as they are: their MMA
-// columns are not read.
+// rows' fp32 activations of the stage's 128-K chunk with cp.async into a slot
+// of the activation ring; each lane's copies arrive on the slot's xfull
+// barrier when they land.  The slots are refilled as soon as a converter has
+// read them, so the copies run ahead of the weight stages and their latency
+// stays off the MMAs' path.  The converter warps (kQ8Conv of them, alternate
+// stages) wait for a stage's rows and for its B tile to be free (the MMAs of
+// its previous use done), write x times (block scale x 2^P) as kQTerms e4m3
+// terms per scale variant, in the 128-byte swizzle, release the slot, and
+// arrive on the stage's full barrier.  Rows past ntok are left as they are:
+// their MMA columns are not read.
 //
 // One stage by one converter warp: (row, 8-element piece) pairs p = lane +
 // 32 u, row p / 16, piece p % 16 (K elements 8 (p % 16) ..), so that every
 // lane has work from two tokens up; pm = the warp's 2^P table of the unit.
 template <class Plan>
 KD_DEV void q8_convert_stage(const Plan& plan, MmaShared& sh, const MUnit& m, int c, int s,
-                             const float* pm) {
+                             int xsl, const float* pm) {
   constexpr int NV = Plan::kVariants, nh = kQTerms;
   const int lane = threadIdx.x & 31;
   const int N = pad16(m.ntok);
   uint8_t* bt = sh.stage + (size_t)s * sh.stage_bytes + sh.boff;
-  const uint8_t* xs = sh.stage + (size_t)s * sh.stage_bytes + sh.xoff;
+  const uint8_t* xs = sh.xring + (size_t)xsl * sh.xslot;
   const int kc = m.kc0 + c;
   float ws[NV];
 #pragma unroll
@@ -777,7 +816,8 @@ KD_DEV void q8_convert_stage(const Plan& plan, MmaShared& sh, const MUnit& m, in
       }
     }
   }
-  fence_proxy_async_smem();   // generic-proxy writes -> visible to the tensor core
+  mbar_arrive(&sh.xempty[xsl]);   // the rows are read: the copier may refill the slot
+  fence_proxy_async_smem();       // generic-proxy writes -> visible to the tensor core
   mbar_arrive(&sh.full[s]);
 }
 
@@ -789,19 +829,24 @@ KD_DEV void mma_copier_q8(const Plan& plan, MmaShared& sh, unsigned* err) {
   CtaUnits<Plan> units(plan);
   MUnit m;
   while (units.next(m)) {
+    // the unit's row sources (lane j: rows j and j + 32), resolved once per
+    // unit and handed out per stage by shuffles
+    const unsigned long long r0 =
+        lane < m.ntok ? reinterpret_cast<unsigned long long>(plan.x_row(m, lane)) : 0ull;
+    const unsigned long long r1 =
+        lane + 32 < m.ntok ? reinterpret_cast<unsigned long long>(plan.x_row(m, lane + 32)) : 0ull;
     for (int c = 0; c < m.nkc; ++c, ++it) {
-      const int s = it % sh.nst;
-      mwait(&sh.empty[s], ((it / sh.nst) & 1u) ^ 1u, sh.abort_flag, err);
-      uint8_t* xs = sh.stage + (size_t)s * sh.stage_bytes + sh.xoff;
-      const int kc = m.kc0 + c;
-      const int nq = *sh.abort_flag ? 0 : m.ntok * 32;   // no new copies after an abort
-      for (int q = lane; q < nq; q += 32) {               // 16-byte pieces, 32 a row
-        const int r = q >> 5, pi = q & 31;
-        const uint8_t* src = reinterpret_cast<const uint8_t*>(plan.x_row(m, r)) +
-                             (size_t)kc * 512 + pi * 16;
-        cp_async16(xs + (size_t)r * 512 + pi * 16, src, 16u);
+      const int xsl = it % sh.nxs;
+      mwait(&sh.xempty[xsl], ((it / sh.nxs) & 1u) ^ 1u, sh.abort_flag, err);
+      uint8_t* xs = sh.xring + (size_t)xsl * sh.xslot;
+      const size_t ko = (size_t)(m.kc0 + c) * 512 + lane * 16;
+      // no new copies after an abort (one read of the flag for the warp)
+      const int nr = __shfl_sync(0xffffffffu, *sh.abort_flag ? 0 : m.ntok, 0);
+      for (int r = 0; r < nr; ++r) {   // lane = 16-byte piece of the 512-byte row
+        const unsigned long long src = __shfl_sync(0xffffffffu, r < 32 ? r0 : r1, r & 31);
+        cp_async16(xs + (size_t)r * 512 + lane * 16, reinterpret_cast<const uint8_t*>(src) + ko, 16u);
       }
-      cp_async_arrive_noinc(&sh.xfull[s]);
+      cp_async_arrive_noinc(&sh.xfull[xsl]);
     }
   }
   cp_async_commit();
@@ -871,9 +916,10 @@ KD_DEV void mma_converter_q8(const Plan& plan, MmaShared& sh, int cw, unsigned* 
     __syncwarp();
     for (int c = 0; c < m.nkc; ++c, ++it) {
       if ((int)(it % kQ8Conv) != cw) continue;
-      const int s = it % sh.nst;
-      mwait(&sh.xfull[s], (it / sh.nst) & 1u, sh.abort_flag, err);
-      q8_convert_stage(plan, sh, m, c, s, pm);
+      const int s = it % sh.nst, xsl = it % sh.nxs;
+      mwait(&sh.xfull[xsl], (it / sh.nxs) & 1u, sh.abort_flag, err);
+      mwait(&sh.empty[s], ((it / sh.nst) & 1u) ^ 1u, sh.abort_flag, err);
+      q8_convert_stage(plan, sh, m, c, s, xsl, pm);
     }
   }
 }
@@ -1153,7 +1199,10 @@ KD_DEV void mma_run(const Plan& plan, uint8_t* smem_raw, unsigned* err) {
       mbar_init(&sh.full[i], Plan::kFp8 ? 1 : (Plan::kQ8 ? 32 : 64));
       mbar_init(&sh.empty[i], 1);
       if (!Plan::kFp8) mbar_init(&sh.afull[i], 1);
-      if (Plan::kQ8) mbar_init(&sh.xfull[i], 32);
+    }
+    for (int i = 0; i < sh.nxs; ++i) {
+      mbar_init(&sh.xfull[i], 32);
+      mbar_init(&sh.xempty[i], 32);
     }
     mbar_init(sh.drain, 1);
     if (Plan::kFp8) {
@@ -1185,10 +1234,8 @@ KD_DEV void mma_run(const Plan& plan, uint8_t* smem_raw, unsigned* err) {
   if (warp == 0) {
     if ((threadIdx.x & 31) == 0) mma_producer_a(plan, sh, err);
   } else if (warp == 1) {
-    if ((threadIdx.x & 31) == 0) {
-      if constexpr (Plan::kQ8) mma_issuer_q8(plan, sh, tmem, err);
-      else mma_issuer(plan, sh, tmem, err);
-    }
+    if constexpr (Plan::kQ8) mma_issuer_q8(plan, sh, tmem, err);
+    else mma_issuer(plan, sh, tmem, err);
   } else if (warp < 4) {
     if constexpr (Plan::kQ8) {
       if (warp == 2) mma_copier_q8(plan, sh, err);

@@ -360,7 +360,7 @@ __global__ void __launch_bounds__(F8 ? kMThreadsQ8 : kMThreads, 1)
 
 // ------------------------------------------------------------------ down + combine
 
-// Tiles of the active experts' down projections (H/128 per expert), then the
+// Tiles of the active experts' down projections (H/128 per expert) and the
 // shared expert's, its M tokens cut into groups of at most shchunk (the
 // routed experts' largest token count, rounded up to 16) so that its B tiles
 // are no wider than the routed ones: a wide B tile would shrink every stage's
@@ -382,11 +382,18 @@ struct MmaDownPlan {
   KD_DEV long long tile_start(int t) const {
     return (long long)t * (L->I / (F8 ? 128 : 64 * nsub));
   }
+  // The shared expert's tiles are spread evenly through the sequence (tile t
+  // is one iff floor((t + 1) S / NT) > floor(t S / NT), S of the NT tiles), so
+  // that the CTAs' contiguous ranges share its wider token groups.
   KD_DEV MUnit tile_unit(int t) const {
     MUnit m{};
-    const int a = t / tiles_per(), tt = t % tiles_per();
-    if (a >= n_act) {
-      const int q = a - n_act;
+    const long long NT = num_tiles(), S = (long long)nsh * tiles_per();
+    const int sb = (int)((long long)t * S / NT);   // shared tiles before t
+    const bool sh = (int)((long long)(t + 1) * S / NT) > sb;
+    const int idx = sh ? sb : t - sb;
+    const int a = idx / tiles_per(), tt = idx % tiles_per();
+    if (sh) {
+      const int q = a;
       m.map = 5; m.row = tt * 128; m.tag = -1;
       m.tok0 = q * shchunk; m.ntok = min(shchunk, M - m.tok0);
     } else {
