@@ -30,8 +30,11 @@
 // (token, tile) that puts the largest |activation x block scale| of the tile
 // in [128, 256) (from per-64-element maxima the producing kernel writes).
 // Gate and up rows of a paired tile have scales of their own, so a paired
-// tile gets two B variants and two accumulators.  The accumulators stay in
-// TMEM for the whole unit, and the epilogue multiplies by 2^-P once.
+// tile gets two B variants.  The B rows are token-major, C = variants x terms
+// rows a token (row j C + v kQTerms + h), so that one MMA of N = pad16(C ntok)
+// covers them all with little padding.  The accumulators stay in TMEM for the
+// whole unit, and the epilogue adds a token's term columns and multiplies by
+// 2^-P once.
 // Work units are (weight tile, K part); a tile split over several parts is
 // summed in part order by the unit that completes it (deterministic).
 #pragma once
@@ -271,6 +274,7 @@ KD_DEV MmaShared carve_mma_smem(uint8_t* base, int nmax, int terms, int nsub, bo
   MmaShared s;
   s.nsub = nsub;
   s.stage_bytes = nsub * (aterms * kATileBytes + b_sub_bytes(nmax, terms));   // bf16: A + B
+  if (q8) s.stage_bytes = kATileBytes + pad16(terms * nmax) * 128;           // A + packed B
   // q8: slots for the rows' fp32 activations of a 128-K chunk (512 B a row,
   // for the launch's largest token count), as many as fit kQ8XBudget (2 ..
   // kMaxMStages), after the stages
@@ -590,29 +594,18 @@ KD_DEV void mma_converter(const Plan& plan, MmaShared& sh, unsigned* err) {
   }
 }
 
-// After an abort: no MMA of the issuing lane may still be running when TMEM
-// is freed: it commits them to the drain barrier and waits (bounded).
-KD_DEV void drain_mma(MmaShared& sh, bool issuing_lane) {
+// After an abort: no MMA of the issuing thread may still be running when
+// TMEM is freed: it commits them to the drain barrier and waits (bounded).
+KD_DEV void drain_mma(MmaShared& sh) {
   if (!*sh.abort_flag) return;
-  if (issuing_lane) {
-    mma_commit(sh.drain);
-    mbar_wait(sh.drain, 0);
-  }
-  __syncwarp();
+  mma_commit(sh.drain);
+  mbar_wait(sh.drain, 0);
 }
 
-// The issuer runs on a whole warp with uniform control flow, so that the
-// operand descriptors are warp-uniform values; lane 0 issues the MMAs and
-// the commits.  Every lane waits; a wait counts as done only if it is done
-// for all of them.
-KD_DEV bool mwait_warp(uint64_t* bar, uint32_t parity, volatile int* abort_flag, unsigned* err) {
-  return __all_sync(0xffffffffu, mwait(bar, parity, abort_flag, err));
-}
 
 template <class Plan>
 KD_DEV void mma_issuer(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigned* err) {
   constexpr int nterms = Plan::kTerms;
-  const bool issue = (threadIdx.x & 31) == 0;
   uint32_t it = 0, nu_local = 0;
   CtaUnits<Plan> units(plan);
   MUnit m;
@@ -621,7 +614,7 @@ KD_DEV void mma_issuer(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigned*
     const uint32_t idesc = idesc_bf16(N);
     const int buf = nu_local & 1;
     const uint32_t d = tmem + (uint32_t)(buf * kMaxN);
-    if (!mwait_warp(&sh.accempty[buf], ((nu_local >> 1) & 1u) ^ 1u, sh.abort_flag, err)) break;
+    if (!mwait(&sh.accempty[buf], ((nu_local >> 1) & 1u) ^ 1u, sh.abort_flag, err)) break;
     tc_fence_after();
     bool ok = true;
     for (int c = 0; c < m.nkc; ++c, ++it) {
@@ -629,11 +622,11 @@ KD_DEV void mma_issuer(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigned*
       const uint32_t ph = (it / sh.nst) & 1u;
       const int sb = it % sh.nbst;
       if (Plan::kFp8) {
-        ok = mwait_warp(&sh.full[s], ph, sh.abort_flag, err) &&
-             mwait_warp(&sh.bfull[sb], (it / sh.nbst) & 1u, sh.abort_flag, err);
+        ok = mwait(&sh.full[s], ph, sh.abort_flag, err) &&
+             mwait(&sh.bfull[sb], (it / sh.nbst) & 1u, sh.abort_flag, err);
       } else {
-        ok = mwait_warp(&sh.afull[s], ph, sh.abort_flag, err) &&
-             mwait_warp(&sh.full[s], ph, sh.abort_flag, err);
+        ok = mwait(&sh.afull[s], ph, sh.abort_flag, err) &&
+             mwait(&sh.full[s], ph, sh.abort_flag, err);
       }
       if (!ok) break;
       fence_proxy_async_smem();   // the B gathers (generic proxy) -> tensor core reads
@@ -641,24 +634,23 @@ KD_DEV void mma_issuer(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigned*
       const uint32_t a0 = smem_u32(sh.stage + (size_t)s * sh.stage_bytes);
       const uint32_t b0 = smem_u32(sh.bst + (size_t)sb * sh.bst_bytes) + sh.boff;
       const int bsub = b_sub_bytes(N, nterms);
-      // descriptors by adding byte offsets / 16 to the start-address field
-      // (shared addresses < 256 KB: the field never carries)
-      const uint64_t ad0 = sw128_desc(a0), bd0 = sw128_desc(b0);
-      if (!issue) {
-      } else if constexpr (!Plan::kFp8) {
+      if constexpr (!Plan::kFp8) {
         for (int u = 0; u < sh.nsub; ++u) {
+          const uint32_t b = b0 + u * bsub;
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
-            const uint64_t ad = ad0 + (uint64_t)((u * kATileBytes + k * 32) >> 4);
-            const uint64_t bd = bd0 + (uint64_t)((u * bsub + k * 32) >> 4);
-            mma_bf16(d, ad, bd, idesc, c > 0 || u > 0 || k > 0);
+            const uint64_t ad = sw128_desc(a0 + u * kATileBytes + k * 32);
+            mma_bf16(d, ad, sw128_desc(b + k * 32), idesc, c > 0 || u > 0 || k > 0);
 #pragma unroll
             for (int h = 1; h < nterms; ++h)
-              mma_bf16(d, ad, bd + (uint64_t)((h * N * 128) >> 4), idesc, true);
+              mma_bf16(d, ad, sw128_desc(b + h * N * 128 + k * 32), idesc, true);
           }
         }
       } else {
-      // FP8 projections: the A terms of the converted tile
+      // FP8: descriptors by adding byte offsets / 16 to the start-address
+      // field (shared addresses < 256 KB: the field never carries); the
+      // issuing thread shares its SM quarter with two converter warps
+      const uint64_t ad0 = sw128_desc(a0), bd0 = sw128_desc(b0);
       for (int u = 0; u < sh.nsub; ++u) {
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -674,17 +666,13 @@ KD_DEV void mma_issuer(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigned*
         }
       }
       }
-      if (issue) {
-        mma_commit(&sh.empty[s]);   // the stage is free once these MMAs are done
-        if (Plan::kFp8) mma_commit(&sh.bempty[sb]);
-      }
-      __syncwarp();
+      mma_commit(&sh.empty[s]);   // the stage is free once these MMAs are done
+      if (Plan::kFp8) mma_commit(&sh.bempty[sb]);
     }
     if (!ok) break;
-    if (issue) mma_commit(&sh.accfull[buf]);
-    __syncwarp();
+    mma_commit(&sh.accfull[buf]);
   }
-  drain_mma(sh, issue);
+  drain_mma(sh);
 }
 
 // q8 plans: per stage (one e4m3 weight tile [128 x 128 K] and a B tile of
@@ -695,24 +683,22 @@ KD_DEV void mma_issuer(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigned*
 template <class Plan>
 KD_DEV void mma_issuer_q8(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigned* err) {
   constexpr int NV = Plan::kVariants, nh = kQTerms;
-  const bool issue = (threadIdx.x & 31) == 0;
   uint32_t nu = 0, ph = 0;
   int s = 0;
   const uint32_t ring0 = smem_u32(sh.stage);
   CtaUnits<Plan> units(plan);
   MUnit m;
   for (; units.next(m); ++nu) {
-    const int N = pad16(m.ntok);
-    // one MMA per K-step covers every (variant, term, token) row of the B tile
-    const uint32_t idesc = idesc_e4m3(NV * nh * N);
+    // one MMA per K-step covers every (token, variant, term) row of the B tile
+    const uint32_t idesc = idesc_e4m3(pad16(NV * nh * m.ntok));
     const int buf = nu & 1;
-    if (!mwait_warp(&sh.accempty[buf], ((nu >> 1) & 1u) ^ 1u, sh.abort_flag, err)) break;
+    if (!mwait(&sh.accempty[buf], ((nu >> 1) & 1u) ^ 1u, sh.abort_flag, err)) break;
     tc_fence_after();
     const uint32_t d0 = tmem + (uint32_t)(buf * kQ8AccCols);
     bool ok = true;
     for (int c = 0; c < m.nkc; ++c) {
-      ok = mwait_warp(&sh.afull[s], ph, sh.abort_flag, err) &&
-           mwait_warp(&sh.full[s], ph, sh.abort_flag, err);
+      ok = mwait(&sh.afull[s], ph, sh.abort_flag, err) &&
+           mwait(&sh.full[s], ph, sh.abort_flag, err);
       if (!ok) break;
       // (the converter fenced its B writes against the async proxy before
       // its arrival)
@@ -721,22 +707,18 @@ KD_DEV void mma_issuer_q8(const Plan& plan, MmaShared& sh, uint32_t tmem, unsign
       // descriptors by adding byte offsets / 16 to the start-address field
       // (shared addresses < 256 KB: the field never carries)
       const uint64_t ad0 = sw128_desc(a0), bd0 = sw128_desc(a0 + sh.boff);
-      if (issue) {
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const uint64_t off = (uint64_t)((k * 32) >> 4);
-          mma_e4m3(d0, ad0 + off, bd0 + off, idesc, c > 0 || k > 0);
-        }
-        mma_commit(&sh.empty[s]);   // the stage is free once these MMAs are done
+      for (int k = 0; k < 4; ++k) {
+        const uint64_t off = (uint64_t)((k * 32) >> 4);
+        mma_e4m3(d0, ad0 + off, bd0 + off, idesc, c > 0 || k > 0);
       }
-      __syncwarp();
+      mma_commit(&sh.empty[s]);   // the stage is free once these MMAs are done
       if (++s == sh.nst) { s = 0; ph ^= 1u; }
     }
     if (!ok) break;
-    if (issue) mma_commit(&sh.accfull[buf]);
-    __syncwarp();
+    mma_commit(&sh.accfull[buf]);
   }
-  drain_mma(sh, issue);
+  drain_mma(sh);
 }
 
 // 2^P for token j of a q8 unit and scale variant v (and 2^-P in inv): the
@@ -769,9 +751,8 @@ KD_DEV float q8_unit_scale(const Plan& plan, const MUnit& m, int j, int v, float
 template <class Plan>
 KD_DEV void q8_convert_stage(const Plan& plan, MmaShared& sh, const MUnit& m, int c, int s,
                              int xsl, const float* pm) {
-  constexpr int NV = Plan::kVariants, nh = kQTerms;
+  constexpr int NV = Plan::kVariants, nh = kQTerms, C = NV * nh;
   const int lane = threadIdx.x & 31;
-  const int N = pad16(m.ntok);
   uint8_t* bt = sh.stage + (size_t)s * sh.stage_bytes + sh.boff;
   const uint8_t* xs = sh.xring + (size_t)xsl * sh.xslot;
   const int kc = m.kc0 + c;
@@ -789,8 +770,6 @@ KD_DEV void q8_convert_stage(const Plan& plan, MmaShared& sh, const MUnit& m, in
       x[0] = f0.x; x[1] = f0.y; x[2] = f0.z; x[3] = f0.w;
       x[4] = f1.x; x[5] = f1.y; x[6] = f1.z; x[7] = f1.w;
     }
-    // 16-byte chunk pc / 2 of the row, swizzled; this piece is its half pc % 2
-    const uint32_t off = (uint32_t)((((pc >> 1) ^ (r & 7)) << 4) | ((pc & 1) << 3));
 #pragma unroll
     for (int v = 0; v < NV; ++v) {
       const float f = ws[v] * pm[v * kMaxN + r];
@@ -811,8 +790,10 @@ KD_DEV void q8_convert_stage(const Plan& plan, MmaShared& sh, const MUnit& m, in
             w[2 * e + 1] -= tv.y;
           }
         }
-        *reinterpret_cast<uint2*>(bt + (size_t)((v * nh + h) * N + r) * 128 + off) =
-            make_uint2(pk[0], pk[1]);
+        // B row b, 16-byte chunk pc / 2 (swizzled), this piece its half pc % 2
+        const int b = r * C + v * nh + h;
+        const uint32_t off = (uint32_t)((((pc >> 1) ^ (b & 7)) << 4) | ((pc & 1) << 3));
+        *reinterpret_cast<uint2*>(bt + (size_t)b * 128 + off) = make_uint2(pk[0], pk[1]);
       }
     }
   }
@@ -1086,6 +1067,7 @@ KD_DEV void mma_epilogue_q8(const Plan& plan, MmaShared& sh, uint32_t tmem, unsi
   MUnit m;
   for (; units.next(m); ++nu_local) {
     const int N = pad16(m.ntok);
+    const int NC = pad16(NV * kQTerms * m.ntok);   // accumulator columns
     const int buf = nu_local & 1;
     // the unit's 2^-P per (variant, token), shared by the four warps
     named_bar_sync(2, 128);   // every warp is done with the previous unit's table
@@ -1102,23 +1084,31 @@ KD_DEV void mma_epilogue_q8(const Plan& plan, MmaShared& sh, uint32_t tmem, unsi
     tc_fence_after();
     const uint32_t ta = tmem + ((uint32_t)(ew * 32) << 16) + (uint32_t)(buf * kQ8AccCols);
     const float* qt = sh.qtab + myv * 64;
-    // 16 tokens of this thread's variant: the sum of its term columns, scaled
-    // (every lane loads every (variant, term) block: tcgen05.ld is warp-wide)
+    // 16 tokens c .. c+15 of this thread's variant: the sum of its term
+    // columns (token j's C columns start at j C), scaled.  C loads of 16
+    // columns; every lane loads every column (tcgen05.ld is warp-wide).
     auto load16 = [&](int c, float* out) {
-      float d[NV][kQTerms][16];
+      constexpr int C = NV * kQTerms, TPL = 16 / C;   // tokens per 16-column load
+      float d[C][16];
 #pragma unroll
-      for (int v = 0; v < NV; ++v)
+      for (int q = 0; q < C; ++q) {
+        if ((c + q * TPL) * C < NC) {
+          tmem_ld16(ta + (uint32_t)((c * C) + 16 * q), d[q]);
+        } else {
 #pragma unroll
-        for (int h = 0; h < kQTerms; ++h) tmem_ld16(ta + (uint32_t)((v * kQTerms + h) * N + c), d[v][h]);
+          for (int i = 0; i < 16; ++i) d[q][i] = 0.f;   // tokens past ntok
+        }
+      }
       tmem_wait_ld();
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
+        const int q = j / TPL, base = (j % TPL) * C;
         float acc = 0.f;
 #pragma unroll
         for (int v = 0; v < NV; ++v)
           if (v == myv) {
 #pragma unroll
-            for (int h = 0; h < kQTerms; ++h) acc += d[v][h][j];
+            for (int h = 0; h < kQTerms; ++h) acc += d[q][base + v * kQTerms + h];
           }
         out[j] = acc * qt[c + j];
       }
@@ -1234,8 +1224,10 @@ KD_DEV void mma_run(const Plan& plan, uint8_t* smem_raw, unsigned* err) {
   if (warp == 0) {
     if ((threadIdx.x & 31) == 0) mma_producer_a(plan, sh, err);
   } else if (warp == 1) {
-    if constexpr (Plan::kQ8) mma_issuer_q8(plan, sh, tmem, err);
-    else mma_issuer(plan, sh, tmem, err);
+    if ((threadIdx.x & 31) == 0) {
+      if constexpr (Plan::kQ8) mma_issuer_q8(plan, sh, tmem, err);
+      else mma_issuer(plan, sh, tmem, err);
+    }
   } else if (warp < 4) {
     if constexpr (Plan::kQ8) {
       if (warp == 2) mma_copier_q8(plan, sh, err);
