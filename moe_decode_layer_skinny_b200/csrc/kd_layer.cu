@@ -597,7 +597,8 @@ static int launch_layer(kd_layer* L, const Acts& a, cudaStream_t s, const kd_lay
   // experts multiply them as they land (with kQ8Conv converter warps for
   // their activation terms)
   const int mthreads = kMThreads;
-  const int ethreads = fp8 ? kMThreadsQ8 : kMThreads;
+  const int gthreads = fp8 ? q8_threads(kGateUpConv) : kMThreads;
+  const int dthreads = fp8 ? q8_threads(kDownConv) : kMThreads;
   if (L->timing) KD_CUDA(cudaEventRecord(L->tev[0], s));
   // Main stream: projections -> router (logits, selection, token lists in one
   // launch) -> routed gate/up -> down + combine.  Side stream: the shared
@@ -628,7 +629,7 @@ static int launch_layer(kd_layer* L, const Acts& a, cudaStream_t s, const kd_lay
   if (d.S) {
     KD_CUDA(cudaStreamWaitEvent(L->side, L->ev_h1, 0));
     if (mma)
-      KD_CUDA(launch(fp8 ? mma_gateup_kernel<true> : mma_gateup_kernel<false>, G, ethreads, msm,
+      KD_CUDA(launch(fp8 ? mma_gateup_kernel<true> : mma_gateup_kernel<false>, G, gthreads, msm,
                      L->side, false, d, M, 1, L->maps));
     else
       KD_CUDA(launch(fp8 ? gateup_kernel<W_FP8> : gateup_kernel<W_BF16>, G, kThreads, sm, L->side,
@@ -637,7 +638,7 @@ static int launch_layer(kd_layer* L, const Acts& a, cudaStream_t s, const kd_lay
   }
   if (L->timing) KD_CUDA(cudaEventRecord(L->tev[2], s));
   if (mma)
-    KD_CUDA(launch(fp8 ? mma_gateup_kernel<true> : mma_gateup_kernel<false>, G, ethreads, msm, s,
+    KD_CUDA(launch(fp8 ? mma_gateup_kernel<true> : mma_gateup_kernel<false>, G, gthreads, msm, s,
                    !L->timing, d, M, 0, L->maps));
   else
     KD_CUDA(launch(fp8 ? gateup_kernel<W_FP8> : gateup_kernel<W_BF16>, G, kThreads,
@@ -655,7 +656,7 @@ static int launch_layer(kd_layer* L, const Acts& a, cudaStream_t s, const kd_lay
   const bool pdl_down = !L->timing && !d.S && !(next && pf);
   if (mma) {
     // tensor-core down writes each expert's outputs; the combine follows
-    KD_CUDA(launch(fp8 ? mma_down_kernel<true> : mma_down_kernel<false>, G, ethreads, msm, s,
+    KD_CUDA(launch(fp8 ? mma_down_kernel<true> : mma_down_kernel<false>, G, dthreads, msm, s,
                    pdl_down, d, M, L->maps));
     KD_CUDA(launch(combine_kernel, 2 * G, 256, 0, s, !L->timing, d, M, a.out));
   } else

@@ -14,7 +14,8 @@
 //   warps 4-7   epilogue: tcgen05.ld of the accumulator (lane = weight row),
 //               then the plan's epilogue, or a split-K partial
 //   warps 8-15  FP8 projections only: e4m3 tiles -> scaled bf16 A tiles
-//   warp 8      q8 plans: the second converter (the two take alternate stages)
+//   warps 8 ..  q8 plans: the other converters (the kQ8Conv converters take
+//               stages in turn)
 // Activations that must stay fp32-accurate come as a sum of bf16 terms, all
 // multiplied into the same accumulator: the expert inputs (h1, the SwiGLU
 // activations) as hi + lo (hi = bf16(v), lo = bf16(v - hi): ~16 significant
@@ -128,8 +129,9 @@ KD_DEV void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "
 
 constexpr int kMThreads = 256;
 constexpr int kMThreadsF8 = 512;      // + 8 converter warps (e4m3 -> bf16 A tiles)
-constexpr int kQ8Conv = 2;            // q8 converter warps (warp 3, then warps 8 ..)
-constexpr int kMThreadsQ8 = kMThreads + 32 * (kQ8Conv - 1);
+constexpr int kQ8Conv = 4;            // q8: most converter warps (warp 3, then warps 8 ..)
+// q8 plans: threads of a CTA with `conv` converter warps (Plan::kConv)
+constexpr int q8_threads(int conv) { return 32 * (8 + conv - 1); }
 constexpr int kMaxMStages = 16;
 constexpr int kATileBytes = 128 * 128;                // 128 rows x 64 bf16 (one swizzle atom wide)
 constexpr int kMaxSub = 2;                            // 64-K sub-tiles per stage (at most)
@@ -137,7 +139,8 @@ constexpr int kMRingBytes = 222 * 1024;                // stages (+ 3 KB below: 
 constexpr int kMaxN = 64;                             // tokens per MMA (N)
 constexpr int kMaxTerms = 3;                          // bf16 terms of an activation
 constexpr size_t kWsFloatsPerCta = 2 * 128 * 64;     // split-K partial slots of one CTA
-constexpr size_t kMmaSmem = (size_t)kMRingBytes + 1024 /*align*/ + 3072 /*barriers, scratch*/;
+constexpr size_t kMmaSmem = (size_t)kMRingBytes + 1024 /*align*/ + 3840 /*barriers, scratch*/;
+static_assert(kMmaSmem + 64 <= 227 * 1024, "shared memory per CTA (with the kernels' static bytes)");
 constexpr int kQ8AccCols = 256;                       // q8: one accumulator, <= 2 x 2 x 64 columns
 constexpr int kQ8TmemCols = 2 * kQ8AccCols;           // q8: two accumulators
 constexpr int kQGroup = 64;                           // activation elements per stored maximum
@@ -223,6 +226,11 @@ struct MmaShared {
   // refills a slot once a converter is done with it, ahead of the MMAs)
   uint8_t* xring;
   int nxs, xslot;
+  // q8: converters that take stages (<= kQ8Conv, nxs and nst).  A converter
+  // takes every nconv-th stage and waits for it by phase parity, which stays
+  // unambiguous only while no slot or stage comes round twice between two of
+  // its stages; the rest idle.
+  int nconv;
   int nsub;              // 64-K sub-tiles per stage
   uint64_t* full;        // [nst] B written (64 arrivals), or (FP8 converter) the A tile converted
   uint64_t* afull;       // [nst] bf16 / q8 plans: the A tile landed (TMA transaction count)
@@ -270,7 +278,7 @@ __host__ __device__ inline int mma_nsub(int nmax, int terms) {
 constexpr int kRawBytes = 128 * 128;
 
 KD_DEV MmaShared carve_mma_smem(uint8_t* base, int nmax, int terms, int nsub, bool fp8,
-                                int aterms, bool q8 = false) {
+                                int aterms, bool q8 = false, int conv = 0) {
   MmaShared s;
   s.nsub = nsub;
   s.stage_bytes = nsub * (aterms * kATileBytes + b_sub_bytes(nmax, terms));   // bf16: A + B
@@ -280,6 +288,7 @@ KD_DEV MmaShared carve_mma_smem(uint8_t* base, int nmax, int terms, int nsub, bo
   // kMaxMStages), after the stages
   s.xslot = 0;
   s.nxs = 0;
+  s.nconv = 0;
   if (q8) {
     s.xslot = ((nmax + 1) / 2) * 1024;
     const int nx = kQ8XBudget / s.xslot;
@@ -313,6 +322,8 @@ KD_DEV MmaShared carve_mma_smem(uint8_t* base, int nmax, int terms, int nsub, bo
   } else {
     s.nst = (kMRingBytes - s.nxs * s.xslot) / s.stage_bytes;
     if (s.nst > kMaxMStages) s.nst = kMaxMStages;
+    s.nconv = conv < s.nxs ? conv : s.nxs;
+    if (s.nconv > s.nst) s.nconv = s.nst;
     s.bst = s.stage;
     s.nbst = s.nst;
     s.bst_bytes = s.stage_bytes;
@@ -329,7 +340,7 @@ KD_DEV MmaShared carve_mma_smem(uint8_t* base, int nmax, int terms, int nsub, bo
   s.misc = s.abort_flag + 1;
   s.qmax = reinterpret_cast<float*>(s.misc + 8);
   s.qtab = s.qmax + 64;
-  s.cpm = s.qtab + 2 * kMaxN;   // ends below 2.7 KB of the 3 KB region
+  s.cpm = s.qtab + 2 * kMaxN;   // ends below 3.7 KB of the 3.75 KB region
   // without a raw ring its barriers serve the A tiles' transactions
   s.afull = s.rfull;
   // q8: the B ring's barriers, unused without a raw ring
@@ -378,6 +389,7 @@ KD_DEV bool mwait_lazy(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
 //   static constexpr bool kFp8     A arrives as e4m3 tiles (converter warps, a_scale)
 //   static constexpr int kATerms   bf16 terms of the converted A tile (1, or 2 = hi + lo)
 //   static constexpr bool kQ8      e4m3 A tiles into kind::f8f6f4 MMAs; B made in-kernel
+//   static constexpr int kConv     q8: converter warps (<= kQ8Conv; the CTA has q8_threads(kConv))
 //                                  from fp32 rows: int kVariants (1, or 2 for gate / up
 //                                  scales), const float* x_row(m, j), const float*
 //                                  g_row(m, j) (per-64 maxima), int kgroups(),
@@ -806,7 +818,8 @@ KD_DEV void q8_convert_stage(const Plan& plan, MmaShared& sh, const MUnit& m, in
 template <class Plan>
 KD_DEV void mma_copier_q8(const Plan& plan, MmaShared& sh, unsigned* err) {
   const int lane = threadIdx.x & 31;
-  uint32_t it = 0;
+  int xsl = 0;         // slot of the stage counter
+  uint32_t xph = 0;    // and its phase
   CtaUnits<Plan> units(plan);
   MUnit m;
   while (units.next(m)) {
@@ -816,9 +829,8 @@ KD_DEV void mma_copier_q8(const Plan& plan, MmaShared& sh, unsigned* err) {
         lane < m.ntok ? reinterpret_cast<unsigned long long>(plan.x_row(m, lane)) : 0ull;
     const unsigned long long r1 =
         lane + 32 < m.ntok ? reinterpret_cast<unsigned long long>(plan.x_row(m, lane + 32)) : 0ull;
-    for (int c = 0; c < m.nkc; ++c, ++it) {
-      const int xsl = it % sh.nxs;
-      mwait(&sh.xempty[xsl], ((it / sh.nxs) & 1u) ^ 1u, sh.abort_flag, err);
+    for (int c = 0; c < m.nkc; ++c) {
+      mwait(&sh.xempty[xsl], xph ^ 1u, sh.abort_flag, err);
       uint8_t* xs = sh.xring + (size_t)xsl * sh.xslot;
       const size_t ko = (size_t)(m.kc0 + c) * 512 + lane * 16;
       // no new copies after an abort (one read of the flag for the warp)
@@ -828,28 +840,31 @@ KD_DEV void mma_copier_q8(const Plan& plan, MmaShared& sh, unsigned* err) {
         cp_async16(xs + (size_t)r * 512 + lane * 16, reinterpret_cast<const uint8_t*>(src) + ko, 16u);
       }
       cp_async_arrive_noinc(&sh.xfull[xsl]);
+      if (++xsl == sh.nxs) { xsl = 0; xph ^= 1u; }
     }
   }
   cp_async_commit();
   cp_async_wait<0>();   // nothing in flight when the warp leaves
 }
 
-// Converter warp cw (warp 3, then warps 8 ..): per unit, the 2^P table of
-// its tokens; then, for each stage of the unit that is its own (stage
-// counter mod kQ8Conv), wait for the rows, convert, release.
+// Converter warp cw (warp 3, then warps 8 ..), one of nconv: per unit, the
+// 2^P table of its tokens (each token's largest |x| x block scale over the
+// tile's groups, put in [128, 256) by q_scale) in a table of its own; then,
+// for each stage of the unit that is its own (stage counter mod nconv), wait
+// for the rows and for the stage's B tile, convert, release.  The lanes split
+// the groups; the block scales are loaded once, and 8 rows' loads are all
+// issued before their reductions.
 template <class Plan>
 KD_DEV void mma_converter_q8(const Plan& plan, MmaShared& sh, int cw, unsigned* err) {
   constexpr int NV = Plan::kVariants;
   const int lane = threadIdx.x & 31;
+  if (cw >= sh.nconv) return;
   float* pm = sh.cpm + cw * 2 * kMaxN;
-  uint32_t it = 0;
+  int own = 0, s = 0, xsl = 0;   // the stage counter's owner, stage, slot
+  uint32_t sph = 0, xph = 0;     // and their phases
   CtaUnits<Plan> units(plan);
   MUnit m;
   while (units.next(m)) {
-    // 2^P per (variant, token) of the unit: each token's largest |x| x block
-    // scale over the tile's groups.  The lanes split the groups; the block
-    // scales are loaded once, and 8 rows' loads are all issued before their
-    // reductions.
     __syncwarp();   // the previous unit's conversions are done with the table
     {
       constexpr int kG = 4;   // groups per lane (<= 128 groups: K <= 8192)
@@ -895,12 +910,16 @@ KD_DEV void mma_converter_q8(const Plan& plan, MmaShared& sh, int cw, unsigned* 
       }
     }
     __syncwarp();
-    for (int c = 0; c < m.nkc; ++c, ++it) {
-      if ((int)(it % kQ8Conv) != cw) continue;
-      const int s = it % sh.nst, xsl = it % sh.nxs;
-      mwait(&sh.xfull[xsl], (it / sh.nxs) & 1u, sh.abort_flag, err);
-      mwait(&sh.empty[s], ((it / sh.nst) & 1u) ^ 1u, sh.abort_flag, err);
-      q8_convert_stage(plan, sh, m, c, s, xsl, pm);
+    // stage / slot indices and phases kept as counters (no divisions)
+    for (int c = 0; c < m.nkc; ++c) {
+      if (own == cw) {
+        mwait(&sh.xfull[xsl], xph, sh.abort_flag, err);
+        mwait(&sh.empty[s], sph ^ 1u, sh.abort_flag, err);
+        q8_convert_stage(plan, sh, m, c, s, xsl, pm);
+      }
+      if (++own == sh.nconv) own = 0;
+      if (++s == sh.nst) { s = 0; sph ^= 1u; }
+      if (++xsl == sh.nxs) { xsl = 0; xph ^= 1u; }
     }
   }
 }
@@ -1180,7 +1199,7 @@ KD_DEV void mma_epilogue_q8(const Plan& plan, MmaShared& sh, uint32_t tmem, unsi
 template <class Plan>
 KD_DEV void mma_run(const Plan& plan, uint8_t* smem_raw, unsigned* err) {
   MmaShared sh = carve_mma_smem(smem_raw, plan.max_n(), Plan::kTerms, plan.nsub, Plan::kFp8,
-                                Plan::kATerms, Plan::kQ8);
+                                Plan::kATerms, Plan::kQ8, Plan::kConv);
   const int warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
     for (int i = 0; i < sh.nst; ++i) {
@@ -1241,7 +1260,7 @@ KD_DEV void mma_run(const Plan& plan, uint8_t* smem_raw, unsigned* err) {
   } else if constexpr (Plan::kFp8) {
     mma_converter(plan, sh, err);
   } else if constexpr (Plan::kQ8) {
-    mma_converter_q8(plan, sh, warp - 7, err);   // warps 8 ..
+    mma_converter_q8(plan, sh, warp - 7, err);   // warps 8 .. 8 + kConv - 2
   }
   tc_fence_before();
   __syncthreads();

@@ -18,6 +18,12 @@
 
 namespace kd {
 
+// q8 converter warps of the expert kernels: the gate/up B tiles carry two
+// scale variants (four e4m3 rows a token), the down ones one (two rows)
+constexpr int kGateUpConv = 3;
+constexpr int kDownConv = 2;
+static_assert(kGateUpConv <= kQ8Conv && kDownConv <= kQ8Conv, "q8 converter tables");
+
 constexpr int kNumMaps = 7;
 struct MmaMaps {
   CUtensorMap m[kNumMaps];
@@ -48,6 +54,7 @@ template <bool F8, int MODE = 0>
 struct MmaProjPlan {
   static constexpr bool kFp8 = F8;
   static constexpr bool kQ8 = false;
+  static constexpr int kConv = 0;
   static constexpr int kVariants = 1;
   // FP8: h1's per-64 maxima for the q8 gate/up kernels (the full layer's
   // come from its second RMSNorm)
@@ -148,6 +155,7 @@ template <bool F8>
 struct MmaRouterPlan {
   static constexpr bool kFp8 = F8;
   static constexpr bool kQ8 = false;
+  static constexpr int kConv = 0;
   static constexpr int kVariants = 1;
   static constexpr bool kGmaxOut = false;
   static constexpr int kATerms = 1;
@@ -261,6 +269,7 @@ template <bool F8>
 struct MmaGateUpPlan {
   static constexpr bool kFp8 = false;    // no converter warps
   static constexpr bool kQ8 = F8;
+  static constexpr int kConv = F8 ? kGateUpConv : 0;   // q8 converter warps
   static constexpr int kVariants = F8 ? 2 : 1;
   static constexpr bool kGmaxOut = F8;
   static constexpr int kATerms = 1;
@@ -341,7 +350,7 @@ struct MmaGateUpPlan {
 };
 
 template <bool F8>
-__global__ void __launch_bounds__(F8 ? kMThreadsQ8 : kMThreads, 1)
+__global__ void __launch_bounds__(F8 ? q8_threads(kGateUpConv) : kMThreads, 1)
     mma_gateup_kernel(LayerDev L, int M, int shared, const __grid_constant__ MmaMaps maps) {
   extern __shared__ uint8_t smem[];
   MmaGateUpPlan<F8> p;
@@ -372,6 +381,7 @@ template <bool F8>
 struct MmaDownPlan {
   static constexpr bool kFp8 = false;    // no converter warps
   static constexpr bool kQ8 = F8;
+  static constexpr int kConv = F8 ? kDownConv : 0;   // q8 converter warps
   static constexpr int kVariants = 1;
   static constexpr bool kGmaxOut = false;
   static constexpr int kATerms = 1;
@@ -441,7 +451,7 @@ struct MmaDownPlan {
 };
 
 template <bool F8>
-__global__ void __launch_bounds__(F8 ? kMThreadsQ8 : kMThreads, 1)
+__global__ void __launch_bounds__(F8 ? q8_threads(kDownConv) : kMThreads, 1)
     mma_down_kernel(LayerDev L, int M, const __grid_constant__ MmaMaps maps) {
   extern __shared__ uint8_t smem[];
   pdl_wait();
