@@ -87,6 +87,17 @@ typedef struct kd_config {
                            selection (the logits buffer then holds unbiased
                            logits)                                             */
   float routed_scale;   /* factor on the routed experts' sum; 0 = 1           */
+  /* Tensor parallelism: this layer is shard tp_rank of tp_size (0 or 1 = the
+     whole layer).  A shard holds q heads [r Hq/R, (r+1) Hq/R) with the kv
+     heads they read (QKV rows, o-proj input columns), router rows
+     [r E/R, (r+1) E/R) and intermediate rows [r I/R, (r+1) I/R) of every
+     expert; it runs the kd_tp_* calls below, not kd_decode_layer.
+     Requires q_heads, E and I divisible by tp_size, I/tp_size and the shard's
+     o-proj columns multiples of 128; with FP8 weights also E/tp_size and
+     head_dim multiples of 128 (the 128 x 128 scale blocks stay whole); no
+     full layer.  Otherwise KD_EINVAL.                                        */
+  int tp_rank;
+  int tp_size;
 } kd_config;
 
 typedef struct kd_layer kd_layer;
@@ -144,6 +155,39 @@ int kd_decode_layer(kd_layer* layer, void* hidden_inout, const void* attn_out, i
  * kd_layer_check as KD_EDEVICE. */
 int kd_decode_layer_full(kd_layer* layer, void* hidden_inout, void* k_cache, void* v_cache,
                          const int* seq, const int* pos, int M, void* stream);
+
+/* ---------------------------------------------------------------- tensor parallel
+ * One decode step of a sharded layer (kd_config.tp_size = R > 1) is four
+ * calls, with three exchanges between the R shards' calls done by the caller
+ * (NCCL, or any other all-reduce / all-gather; the ranks' order of
+ * additions is theirs).  The sharding follows wireai.ir "vLLM Blackwell Kimi
+ * decode", section "4 key changes", items 2 (o-proj partial sums reduced
+ * across GPUs with the residual) and 3 (router scores split among the
+ * tensor-parallel ranks).  Exchange buffers (kd_tp_buffers) are
+ * layer-owned device memory, fp32 row-major:
+ *   p        [M, H]        o-proj partial sum, then (after the caller's
+ *                          all-reduce, in place) the sum over shards
+ *   lshard   [M, E/R]      this shard's router logits
+ *   lfull    [M, E]        all shards' logits side by side, shard r in
+ *                          columns [r E/R, (r+1) E/R) (the caller's all-gather)
+ *   y        [M, H]        expert partial sum, then (all-reduce, in place) the
+ *                          sum over shards
+ * Calls (all enqueue on `stream`; M in 1..max_tokens, else KD_ERANGE):
+ *   kd_tp_attn     hidden bf16 [M, H] and attn bf16 [M, q_heads head_dim]
+ *                  (the whole attention output; the shard reads its heads'
+ *                  columns) -> its QKV rows (kd_layer_qkv: bf16 [M, rows],
+ *                  q rows of its heads, then k and v of its kv heads) and p.
+ *   kd_tp_router   hidden and the summed p -> h1 = x + p (kept), lshard.
+ *   kd_tp_moe      lfull -> the selection (identical on every shard), the
+ *                  shard's rows of every selected and shared expert -> y
+ *                  (without h1).
+ *   kd_tp_combine  the summed y -> hidden = bf16(h1 + y), in place.
+ * Errors: KD_EINVAL (null or unsharded layer), KD_ERANGE, KD_ECUDA. */
+int kd_tp_buffers(const kd_layer* layer, float** p, float** lshard, float** lfull, float** y);
+int kd_tp_attn(kd_layer* layer, const void* hidden, const void* attn, int M, void* stream);
+int kd_tp_router(kd_layer* layer, const void* hidden, int M, void* stream);
+int kd_tp_moe(kd_layer* layer, int M, void* stream);
+int kd_tp_combine(kd_layer* layer, void* hidden, int M, void* stream);
 
 /* Synchronise the device and report (then clear) the layer's device error
  * word: KD_OK, KD_ETIMEOUT (a bounded wait inside a kernel gave up) or

@@ -27,7 +27,8 @@ EXPORTS = ("kd_layer_create", "kd_layer_destroy", "kd_decode_layer", "kd_decode_
            "kd_layer_check",
            "kd_layer_qkv", "kd_layer_prefetch_l2", "kd_layer_debug_tensor", "kd_layer_read_weight",
            "kd_layer_bytes", "kd_layer_launches", "kd_layer_set_timing_events", "kd_stack_create",
-           "kd_stack_run", "kd_stack_destroy", "kd_router_topk_static", "kd_last_error")
+           "kd_stack_run", "kd_stack_destroy", "kd_router_topk_static", "kd_last_error",
+           "kd_tp_buffers", "kd_tp_attn", "kd_tp_router", "kd_tp_moe", "kd_tp_combine")
 N_TIMING_EVENTS = 5
 
 
@@ -46,7 +47,8 @@ class _Config(ctypes.Structure):
                 ("full_layer", ctypes.c_int), ("rms_eps", ctypes.c_float),
                 ("kv_n_seq", ctypes.c_int), ("kv_max_ctx", ctypes.c_int),
                 ("k_scale", ctypes.c_float), ("v_scale", ctypes.c_float),
-                ("bias_select_only", ctypes.c_int), ("routed_scale", ctypes.c_float)]
+                ("bias_select_only", ctypes.c_int), ("routed_scale", ctypes.c_float),
+                ("tp_rank", ctypes.c_int), ("tp_size", ctypes.c_int)]
 
 
 _lib = None
@@ -80,6 +82,12 @@ def lib() -> ctypes.CDLL:
         L.kd_stack_destroy.restype = None
         L.kd_router_topk_static.argtypes = [vp, vp, i32, vp, vp, i32, i32, i32, i32, vp, vp, vp]
         L.kd_last_error.restype = ctypes.c_char_p
+        fpp = ctypes.POINTER(vp)
+        L.kd_tp_buffers.argtypes = [vp, fpp, fpp, fpp, fpp]
+        L.kd_tp_attn.argtypes = [vp, vp, vp, i32, vp]
+        L.kd_tp_router.argtypes = [vp, vp, i32, vp]
+        L.kd_tp_moe.argtypes = [vp, i32, vp]
+        L.kd_tp_combine.argtypes = [vp, vp, i32, vp]
         _lib = L
     return _lib
 
@@ -119,6 +127,8 @@ class LayerSpec:
     v_scale: float = 0.0
     bias_select_only: int = 0
     routed_scale: float = 0.0
+    tp_rank: int = 0
+    tp_size: int = 0
 
     @classmethod
     def from_dims(cls, dims, **kw) -> "LayerSpec":
@@ -139,7 +149,7 @@ class Layer:
                       spec.max_tokens, None if bias is None else bias.ctypes.data,
                       spec.mma_min_tokens, spec.full_layer, spec.rms_eps, spec.kv_n_seq,
                       spec.kv_max_ctx, spec.k_scale, spec.v_scale, spec.bias_select_only,
-                      spec.routed_scale)
+                      spec.routed_scale, spec.tp_rank, spec.tp_size)
         h = ctypes.c_void_p()
         _check(lib().kd_layer_create(ctypes.byref(cfg), seed, ctypes.byref(h)))
         self._h = h
@@ -177,6 +187,29 @@ class Layer:
         _check(lib().kd_decode_layer_full(self._h, hidden.data_ptr(), k_cache.data_ptr(),
                                           v_cache.data_ptr(), seq.data_ptr(), pos.data_ptr(), M,
                                           _stream_ptr(stream)))
+
+    # ---- tensor-parallel shard (spec.tp_size > 1): the four phases of
+    # kd_tp_*; the exchanges between them are the caller's (tp.decode_tp)
+    def tp_buffers(self) -> dict:
+        """Device pointers of the shard's fp32 exchange buffers (kd_tp_buffers)."""
+        ptrs = [ctypes.c_void_p() for _ in range(4)]
+        _check(lib().kd_tp_buffers(self._h, *[ctypes.byref(p) for p in ptrs]))
+        return dict(zip(("p", "lshard", "lfull", "y"), (p.value for p in ptrs)))
+
+    def tp_attn(self, hidden, attn, M: int | None = None, stream=None) -> None:
+        M = hidden.shape[0] if M is None else M
+        _check(lib().kd_tp_attn(self._h, hidden.data_ptr(), attn.data_ptr(), M, _stream_ptr(stream)))
+
+    def tp_router(self, hidden, M: int | None = None, stream=None) -> None:
+        M = hidden.shape[0] if M is None else M
+        _check(lib().kd_tp_router(self._h, hidden.data_ptr(), M, _stream_ptr(stream)))
+
+    def tp_moe(self, M: int, stream=None) -> None:
+        _check(lib().kd_tp_moe(self._h, M, _stream_ptr(stream)))
+
+    def tp_combine(self, hidden, M: int | None = None, stream=None) -> None:
+        M = hidden.shape[0] if M is None else M
+        _check(lib().kd_tp_combine(self._h, hidden.data_ptr(), M, _stream_ptr(stream)))
 
     def decode_ptr(self, hidden_ptr: int, attn_ptr: int, M: int, stream_ptr: int | None) -> int:
         return lib().kd_decode_layer(self._h, hidden_ptr, attn_ptr, M, stream_ptr)

@@ -19,22 +19,30 @@ namespace kd {
 
 // ------------------------------------------------------------------ generator
 
-// dst[(r*row_mult + row_off) * K + c] = bf16(value(stream, r*K + c)), r < R.
+// Rows [lr0, lr0 + R) x columns [lc0, lc0 + K) of a logical matrix with LK
+// columns (the whole matrix: lr0 = lc0 = 0, LK = K; a tensor-parallel shard:
+// its rows or columns):
+// dst[(r*row_mult + row_off) * K + c] = bf16(value(stream, (lr0 + r) LK + lc0 + c)).
 static __global__ void gen_bf16_kernel(uint16_t* __restrict__ dst, int R, int K, uint64_t stream,
-                                int row_mult, int row_off) {
+                                int row_mult, int row_off, uint64_t lr0, uint64_t lc0,
+                                uint64_t LK) {
   const uint64_t n = (uint64_t)R * (uint64_t)K;
   for (uint64_t i = (uint64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
        i += (uint64_t)gridDim.x * blockDim.x) {
     const uint64_t r = i / (uint64_t)K, c = i - r * (uint64_t)K;
-    dst[(r * row_mult + row_off) * (uint64_t)K + c] = kdg_bf16(kdg_value(stream, i, KDG_W002));
+    dst[(r * row_mult + row_off) * (uint64_t)K + c] =
+        kdg_bf16(kdg_value(stream, (lr0 + r) * LK + lc0 + c, KDG_W002));
   }
 }
 
 // One 128x128 block per CTA (256 threads): amax -> scale -> e4m3 codes.
-// scales: [ceil(R/128), ceil(K/128)] table of this logical matrix.
+// scales: [ceil(R/128), ceil(K/128)] table of these rows and columns.  The
+// logical offsets (as for gen_bf16_kernel) are multiples of 128, so that every
+// block is a block of the logical matrix.
 static __global__ void __launch_bounds__(256) gen_fp8_kernel(uint8_t* __restrict__ dst,
                                                       float* __restrict__ scales, int R, int K,
-                                                      uint64_t stream, int row_mult, int row_off) {
+                                                      uint64_t stream, int row_mult, int row_off,
+                                                      uint64_t lr0, uint64_t lc0, uint64_t LK) {
   const int kb = blockIdx.x, rb = blockIdx.y, nkb = gridDim.x;
   __shared__ float wmax[8];
   float v[64];
@@ -45,7 +53,7 @@ static __global__ void __launch_bounds__(256) gen_fp8_kernel(uint8_t* __restrict
     const int r = rb * 128 + (e >> 7), c = kb * 128 + (e & 127);
     v[q] = 0.f;
     if (r < R && c < K) {
-      v[q] = kdg_value(stream, (uint64_t)r * (uint64_t)K + (uint64_t)c, KDG_W002);
+      v[q] = kdg_value(stream, (lr0 + (uint64_t)r) * LK + lc0 + (uint64_t)c, KDG_W002);
       amax = fmaxf(amax, fabsf(v[q]));
     }
   }
@@ -70,6 +78,15 @@ static __global__ void __launch_bounds__(256) gen_fp8_kernel(uint8_t* __restrict
 struct LayerDev {
   int H, A, Nqkv, E, k, I, S, eb;       // eb = weight element bytes (2 bf16, 1 fp8)
   int nHb, nAb, nIb;                    // 128-blocks along H, A, I
+  // Tensor-parallel shard (tp = 1): A, Nqkv and I are the shard's, E stays
+  // the number of experts the selection runs over, Er the router rows of this
+  // layer (E unsharded), attn_ld the row stride of the attention input (its
+  // full width); the o-proj epilogue then writes the partial sum alone, the
+  // router no selection, and the combine the fp32 expert sum into tp_y.
+  int Er, attn_ld, tp;
+  float* tp_y;                          // [Mmax, H] expert partial sum (shards)
+  float* tp_lfull;                      // [Mmax, E] gathered logits (shards)
+  const float* rbias;                   // bias of the router rows (bias + first row)
   // weights (physical layouts; see kd_layer.cu)
   const uint8_t* wqkv; const uint8_t* wo; const uint8_t* wr;
   const uint8_t* wgu_sh; const uint8_t* wd_sh;
@@ -171,7 +188,8 @@ struct ProjPlanT {
   KD_DEV const void* act_row(const Seg& s, int j) const {
     if (MODE == 1) return L->uf + (size_t)j * L->H;
     if (MODE == 2) return L->attnf + (size_t)j * L->A;
-    return s.tag == 0 ? (const void*)(a.x + (size_t)j * L->H) : (const void*)(a.attn + (size_t)j * L->A);
+    return s.tag == 0 ? (const void*)(a.x + (size_t)j * L->H)
+                      : (const void*)(a.attn + (size_t)j * L->attn_ld);
   }
   KD_DEV const float* scale_row(const Seg& s, int row) const {
     return s.tag == 0 ? L->sqkv + (size_t)(row >> 7) * L->nHb : L->so + (size_t)(row >> 7) * L->nAb;
@@ -186,6 +204,10 @@ struct ProjPlanT {
       }
     } else {
       const size_t o = (size_t)j * L->H + row;
+      if (MODE == 0 && L->tp) {   // a shard's o-proj partial sum
+        L->h1f[o] = v;
+        return;
+      }
       const float h = __uint_as_float((uint32_t)a.x[o] << 16) + v;
       if (MODE == 2) {
         L->h1r[o] = h;
@@ -542,7 +564,7 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(LayerDev L, int 
   // the router weights are static: load them before waiting for h1
   uint4 w[kRouterWChunks];
   float sc[kRouterWChunks];
-  if (row < L.E) {
+  if (row < L.Er) {
     const uint8_t* wrow = L.wr + (size_t)row * L.H * L.eb;
 #pragma unroll
     for (int i = 0; i < kRouterWChunks; ++i) {
@@ -555,7 +577,7 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(LayerDev L, int 
     }
   }
   pdl_wait();
-  if (row < L.E) {
+  if (row < L.Er) {
     for (int t0 = 0; t0 < M; t0 += kTT) {
       const int nt = M - t0 < kTT ? M - t0 : kTT;
       const float* arow[kTT];
@@ -579,12 +601,12 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(LayerDev L, int 
   __syncthreads();
   for (int i = threadIdx.x; i < kRouterRows * M; i += kRouterThreads) {
     const int r = i / M, t = i % M, e = blockIdx.x * kRouterRows + r;
-    if (e < L.E)
-      L.logits[(size_t)t * L.E + e] =
+    if (e < L.Er)
+      L.logits[(size_t)t * L.Er + e] =
           ((part[r][0][t] + part[r][1][t]) + (part[r][2][t] + part[r][3][t])) +
-          (L.bias && !L.bias_sel ? L.bias[e] : 0.f);
+          (L.rbias && !L.bias_sel ? L.rbias[e] : 0.f);
   }
-  route_last_block(L, M, gridDim.x);
+  if (!L.tp) route_last_block(L, M, gridDim.x);   // a shard's selection runs on all shards' logits
   pdl_launch_dependents();
 }
 
@@ -714,11 +736,12 @@ struct DownPlan {
       for (int e = threadIdx.x; e < 64 * M; e += kThreads) {
         const int t = e / 64, h = b * 64 + e % 64;
         const size_t o = (size_t)t * L->H + h;
-        float v = L->resid[o];
+        float v = L->tp_y ? 0.f : L->resid[o];
         if (L->S) v += __ldcg(L->ysh + o);
         for (int j = 0; j < L->k; ++j)
           v += (L->rscale * L->gates[t * L->k + j]) * __ldcg(L->yr + ((size_t)t * L->k + j) * L->H + h);
-        out[o] = f32_to_bf16_bits(v);
+        if (L->tp_y) L->tp_y[o] = v;   // a shard's expert partial sum
+        else out[o] = f32_to_bf16_bits(v);
       }
     }
     named_bar_sync(1, kThreads);  // s_list / s_n are reused by the next segment

@@ -51,6 +51,8 @@ struct kd_layer {
   cudaEvent_t ev_h1 = nullptr, ev_sh = nullptr;
   uint64_t static_bytes = 0, expert_bytes = 0;
   int Nqkv = 0, A = 0;
+  bool tp = false;       // a tensor-parallel shard (kd_tp_* calls)
+  int attn_col0 = 0;     // a shard's first attention-output column
   cudaEvent_t tev[KD_N_TIMING_EVENTS] = {};  // profiling hook (kd_layer_set_timing_events)
   bool timing = false;
   int mma_min = 4;       // calls with M >= mma_min use the tensor-core kernels
@@ -143,15 +145,21 @@ static bool encode_weight_map(CUtensorMap* m, const void* base, uint64_t rows, u
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Generate one logical [R, K] matrix into `dst` with row stride multiplier
-// (physical row = r*mult + off); FP8 writes its block scales to `scales`.
+// Generate rows [lr0, lr0 + R) x columns [lc0, lc0 + K) of one logical
+// matrix with LK columns (LK = 0: the whole [R, K] matrix) into `dst` with
+// row stride multiplier (physical row = r*mult + off); FP8 writes its block
+// scales to `scales`.
 static int gen_matrix(const kd_layer* L, uint8_t* dst, float* scales, int R, int K, uint64_t seed,
-                      uint32_t kind, uint32_t slot, int mult, int off, cudaStream_t s) {
+                      uint32_t kind, uint32_t slot, int mult, int off, cudaStream_t s,
+                      int lr0 = 0, int lc0 = 0, int LK = 0) {
   const uint64_t st = kdg_stream(seed, kdg_uid((uint32_t)L->cfg.layer_id, kind, slot));
+  const uint64_t lk = LK ? (uint64_t)LK : (uint64_t)K;
   if (L->cfg.wdtype == KD_WBF16) {
-    gen_bf16_kernel<<<L->nsm * 8, 256, 0, s>>>(reinterpret_cast<uint16_t*>(dst), R, K, st, mult, off);
+    gen_bf16_kernel<<<L->nsm * 8, 256, 0, s>>>(reinterpret_cast<uint16_t*>(dst), R, K, st, mult, off,
+                                               (uint64_t)lr0, (uint64_t)lc0, lk);
   } else {
-    gen_fp8_kernel<<<dim3(ceil128(K), ceil128(R)), 256, 0, s>>>(dst, scales, R, K, st, mult, off);
+    gen_fp8_kernel<<<dim3(ceil128(K), ceil128(R)), 256, 0, s>>>(dst, scales, R, K, st, mult, off,
+                                                                (uint64_t)lr0, (uint64_t)lc0, lk);
   }
   KD_CUDA(cudaGetLastError());
   return KD_OK;
@@ -214,6 +222,7 @@ static int configure_kernels() {
   const int rsmem = (int)(sizeof(int) * kRouteSmemInts(1024, 64 * 16));
   KD_CUDA(cudaFuncSetAttribute(router_kernel<W_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, rsmem));
   KD_CUDA(cudaFuncSetAttribute(router_kernel<W_FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, rsmem));
+  KD_CUDA(cudaFuncSetAttribute(tp_route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, rsmem));
   const int msmem = (int)kMmaSmem;
   KD_CUDA(cudaFuncSetAttribute(mma_proj_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem));
   KD_CUDA(cudaFuncSetAttribute(mma_gateup_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem));
@@ -256,6 +265,22 @@ extern "C" int kd_layer_create(const kd_config* cfg, uint64_t seed, kd_layer** o
       c.hidden > 8192 || A > 8192 || c.inter > 8192)
     return fail(KD_EINVAL, "kd_layer_create: a weight row exceeds one %s%ld-byte stage", "",
                 (long)kStageBytes);
+  const int R = c.tp_size > 1 ? c.tp_size : 1, tr = c.tp_size > 1 ? c.tp_rank : 0;
+  if (c.tp_size < 0 || c.tp_rank < 0 || (c.tp_size <= 1 && c.tp_rank != 0) || tr >= R)
+    return fail(KD_EINVAL, "kd_layer_create: bad tensor-parallel rank%s", "");
+  if (R > 1) {
+    const bool fp8 = c.wdtype == KD_WFP8;
+    // q heads per rank and the kv heads they read (all ranks alike: a rank's
+    // q heads never straddle two kv-head groups unevenly)
+    const int qr = c.q_heads / R, grp = c.kv_heads > 0 ? c.q_heads / c.kv_heads : 0;
+    const bool even = grp > 0 && qr > 0 && (qr % grp == 0 || grp % qr == 0);
+    const int kvr = even ? (qr >= grp ? qr / grp : 1) : 0;
+    if (!even || ((qr + 2 * kvr) * c.head_dim) % 128 ||
+        c.kv_heads < 1 || c.q_heads % c.kv_heads || c.q_heads % R || c.n_experts % R ||
+        c.inter % R || (c.inter / R) % 128 || (c.q_heads / R * c.head_dim) % 128 || c.full_layer ||
+        (fp8 && ((c.n_experts / R) % 128 || c.head_dim % 128)))
+      return fail(KD_EINVAL, "kd_layer_create: unsupported tensor-parallel sharding%s", "");
+  }
   if (c.full_layer) {
     const int grp = c.kv_heads > 0 ? c.q_heads / c.kv_heads : 0;
     if (c.full_layer != 1 || c.kv_heads < 1 || c.q_heads % c.kv_heads ||
@@ -271,8 +296,18 @@ extern "C" int kd_layer_create(const kd_config* cfg, uint64_t seed, kd_layer** o
   L->cfg.router_bias = nullptr;
   L->maxM = c.max_tokens;
   L->mma_min = c.mma_min_tokens > 0 ? c.mma_min_tokens : 3;
-  L->Nqkv = Nqkv;
-  L->A = A;
+  // tensor-parallel shard: its q heads [q0, q1), the kv heads they read
+  // [k0, k1), router rows [e0, e0 + Er), expert rows [i0, i0 + Ir)
+  const int q0 = c.q_heads * tr / R, q1 = c.q_heads * (tr + 1) / R;
+  const int grpq = c.kv_heads > 0 ? c.q_heads / c.kv_heads : 1;
+  const int k0 = R > 1 ? q0 / grpq : 0, k1 = R > 1 ? (q1 - 1) / grpq + 1 : c.kv_heads;
+  const int Ar = (q1 - q0) * c.head_dim;
+  const int Nr = (q1 - q0 + 2 * (k1 - k0)) * c.head_dim;
+  const int Er = c.n_experts / R, e0 = Er * tr, Ir = c.inter / R, i0 = Ir * tr;
+  L->tp = R > 1;
+  L->attn_col0 = q0 * c.head_dim;
+  L->Nqkv = Nr;
+  L->A = Ar;
   int rc = KD_OK;
 #define TRY(x)                 \
   do {                         \
@@ -298,18 +333,22 @@ extern "C" int kd_layer_create(const kd_config* cfg, uint64_t seed, kd_layer** o
   TRY(configure_kernels());
 
   LayerDev& d = L->d;
-  const int H = c.hidden, E = c.n_experts, I = c.inter, k = c.top_k, M = c.max_tokens;
+  // (a shard: A, Nqkv, I its own; E the experts the selection runs over; the
+  // router generates Er rows)
+  const int H = c.hidden, E = c.n_experts, k = c.top_k, M = c.max_tokens;
+  const int I = Ir, A_ = Ar, Nq = Nr;
   const int eb = c.wdtype == KD_WBF16 ? 2 : 1;
   const bool fp8 = c.wdtype == KD_WFP8;
-  d.H = H; d.A = A; d.Nqkv = Nqkv; d.E = E; d.k = k; d.I = I; d.S = c.n_shared; d.eb = eb;
-  d.nHb = ceil128(H); d.nAb = ceil128(A); d.nIb = ceil128(I);
+  d.H = H; d.A = A_; d.Nqkv = Nq; d.E = E; d.k = k; d.I = I; d.S = c.n_shared; d.eb = eb;
+  d.nHb = ceil128(H); d.nAb = ceil128(A_); d.nIb = ceil128(I);
+  d.Er = Er; d.attn_ld = A; d.tp = L->tp ? 1 : 0;
 
   uint8_t *wqkv, *wo, *wr, *wgu_sh = nullptr, *wd_sh = nullptr, *wgu, *wd;
   float *sqkv = nullptr, *so = nullptr, *sr = nullptr, *sgu_sh = nullptr, *sd_sh = nullptr,
         *sgu = nullptr, *sd = nullptr;
-  TRY(dalloc_t(L, (size_t)Nqkv * H * eb, &wqkv));
-  TRY(dalloc_t(L, (size_t)H * A * eb, &wo));
-  TRY(dalloc_t(L, (size_t)E * H * eb, &wr));
+  TRY(dalloc_t(L, (size_t)Nq * H * eb, &wqkv));
+  TRY(dalloc_t(L, (size_t)H * A_ * eb, &wo));
+  TRY(dalloc_t(L, (size_t)Er * H * eb, &wr));
   const size_t gu_bytes = (size_t)2 * I * H * eb, dn_bytes = (size_t)H * I * eb;
   if (c.n_shared) {
     TRY(dalloc_t(L, gu_bytes, &wgu_sh));
@@ -319,9 +358,9 @@ extern "C" int kd_layer_create(const kd_config* cfg, uint64_t seed, kd_layer** o
   TRY(dalloc_t(L, dn_bytes * E, &wd));
   const size_t n_sgu = (size_t)2 * d.nIb * d.nHb, n_sd = (size_t)d.nHb * d.nIb;
   if (fp8) {
-    TRY(dalloc_t(L, (size_t)ceil128(Nqkv) * d.nHb, &sqkv));
+    TRY(dalloc_t(L, (size_t)ceil128(Nq) * d.nHb, &sqkv));
     TRY(dalloc_t(L, (size_t)d.nHb * d.nAb, &so));
-    TRY(dalloc_t(L, (size_t)ceil128(E) * d.nHb, &sr));
+    TRY(dalloc_t(L, (size_t)ceil128(Er) * d.nHb, &sr));
     if (c.n_shared) {
       TRY(dalloc_t(L, n_sgu, &sgu_sh));
       TRY(dalloc_t(L, n_sd, &sd_sh));
@@ -333,10 +372,10 @@ extern "C" int kd_layer_create(const kd_config* cfg, uint64_t seed, kd_layer** o
   d.sqkv = sqkv; d.so = so; d.sr = sr; d.sgu_sh = sgu_sh; d.sd_sh = sd_sh; d.sgu = sgu; d.sd = sd;
 
   const size_t sc = fp8 ? sizeof(float) : 0;
-  L->static_bytes = (size_t)Nqkv * H * eb + (size_t)H * A * eb + (size_t)E * H * eb +
+  L->static_bytes = (size_t)Nq * H * eb + (size_t)H * A_ * eb + (size_t)Er * H * eb +
                     (c.n_shared ? gu_bytes + dn_bytes : 0) +
-                    sc * ((size_t)ceil128(Nqkv) * d.nHb + (size_t)d.nHb * d.nAb +
-                          (size_t)ceil128(E) * d.nHb + (c.n_shared ? n_sgu + n_sd : 0));
+                    sc * ((size_t)ceil128(Nq) * d.nHb + (size_t)d.nHb * d.nAb +
+                          (size_t)ceil128(Er) * d.nHb + (c.n_shared ? n_sgu + n_sd : 0));
   L->expert_bytes = gu_bytes + dn_bytes + sc * (n_sgu + n_sd);
 
   float* bias = nullptr;
@@ -345,10 +384,11 @@ extern "C" int kd_layer_create(const kd_config* cfg, uint64_t seed, kd_layer** o
     TRYC(cudaMemcpy(bias, cfg->router_bias, sizeof(float) * E, cudaMemcpyHostToDevice));
   }
   d.bias = bias;
+  d.rbias = bias ? bias + e0 : nullptr;
   d.bias_sel = c.bias_select_only ? 1 : 0;
   d.rscale = c.routed_scale != 0.f ? c.routed_scale : 1.f;
 
-  TRY(dalloc_t(L, (size_t)M * Nqkv, &d.qkv));
+  TRY(dalloc_t(L, (size_t)M * Nq, &d.qkv));
   TRY(dalloc_t(L, (size_t)M * H, &d.h1f));
   TRY(dalloc_t(L, (size_t)M * H, &d.h1b));
   TRY(dalloc_t(L, (size_t)M * E, &d.logits));
@@ -378,6 +418,10 @@ extern "C" int kd_layer_create(const kd_config* cfg, uint64_t seed, kd_layer** o
     TRY(dalloc_t(L, (size_t)M * (I / kQGroup), &d.actshg));
   }
   d.resid = d.h1f;
+  if (L->tp) {
+    TRY(dalloc_t(L, (size_t)M * H, &d.tp_y));
+    TRY(dalloc_t(L, (size_t)M * E, &d.tp_lfull));
+  }
   if (c.full_layer) {
     L->full = true;
     d.Hq = c.q_heads; d.Hkv = c.kv_heads; d.hd = c.head_dim;
@@ -414,7 +458,7 @@ extern "C" int kd_layer_create(const kd_config* cfg, uint64_t seed, kd_layer** o
   TRY(dalloc_t(L, (size_t)L->nsm * kWsFloatsPerCta, &d.ws_side));
   {
     const size_t ntile = std::max<size_t>({(size_t)(E + 4) * (H / 128), (size_t)(E + 1) * (2 * I / 128),
-                                           (size_t)(Nqkv + H) / 128});
+                                           (size_t)(Nq + H) / 128});
     L->ntile = ntile;
     TRY(dalloc_t(L, ntile, &d.tcnt_main));
     TRY(dalloc_t(L, ntile, &d.tcnt_side));
@@ -433,18 +477,35 @@ extern "C" int kd_layer_create(const kd_config* cfg, uint64_t seed, kd_layer** o
   TRYC(cudaStreamCreateWithFlags(&gs, cudaStreamNonBlocking));
   auto gen = [&](uint8_t* dst, float* s, int R, int K, uint32_t kind, uint32_t slot, int mult,
                  int off) { return gen_matrix(L, dst, s, R, K, seed, kind, slot, mult, off, gs); };
-  rc = gen(wqkv, sqkv, Nqkv, H, KDG_QKV, 0, 1, 0);
-  if (rc == KD_OK) rc = gen(wo, so, H, A, KDG_OPROJ, 0, 1, 0);
-  if (rc == KD_OK) rc = gen(wr, sr, E, H, KDG_ROUTER, 0, 1, 0);
+  if (!L->tp) {
+    rc = gen(wqkv, sqkv, Nq, H, KDG_QKV, 0, 1, 0);
+  } else {
+    // a shard's QKV rows: its q heads, then k and v of the kv heads they read
+    const int hd = c.head_dim;
+    const int seg_l[3] = {q0 * hd, (c.q_heads + k0) * hd, (c.q_heads + c.kv_heads + k0) * hd};
+    const int seg_n[3] = {(q1 - q0) * hd, (k1 - k0) * hd, (k1 - k0) * hd};
+    int r0 = 0;
+    for (int g = 0; g < 3 && rc == KD_OK; ++g) {
+      rc = gen_matrix(L, wqkv + (size_t)r0 * H * eb, sqkv ? sqkv + (size_t)(r0 / 128) * d.nHb : nullptr,
+                      seg_n[g], H, seed, KDG_QKV, 0, 1, 0, gs, seg_l[g], 0, H);
+      r0 += seg_n[g];
+    }
+  }
+  if (rc == KD_OK)
+    rc = gen_matrix(L, wo, so, H, A_, seed, KDG_OPROJ, 0, 1, 0, gs, 0, L->attn_col0, A);
+  if (rc == KD_OK) rc = gen_matrix(L, wr, sr, Er, H, seed, KDG_ROUTER, 0, 1, 0, gs, e0, 0, H);
   for (int e = (c.n_shared ? -1 : 0); e < E && rc == KD_OK; ++e) {
     uint8_t* gu = e < 0 ? wgu_sh : wgu + (size_t)e * gu_bytes;
     uint8_t* dn = e < 0 ? wd_sh : wd + (size_t)e * dn_bytes;
     float* sg = fp8 ? (e < 0 ? sgu_sh : sgu + (size_t)e * n_sgu) : nullptr;
     float* sdn = fp8 ? (e < 0 ? sd_sh : sd + (size_t)e * n_sd) : nullptr;
     const uint32_t slot = (uint32_t)(e + 1);
-    rc = gen(gu, sg, I, H, KDG_GATE, slot, 2, 0);
-    if (rc == KD_OK) rc = gen(gu, sg ? sg + (size_t)d.nIb * d.nHb : nullptr, I, H, KDG_UP, slot, 2, 1);
-    if (rc == KD_OK) rc = gen(dn, sdn, H, I, KDG_DOWN, slot, 1, 0);
+    // (a shard: intermediate rows [i0, i0 + I) of gate and up, those columns of down)
+    rc = gen_matrix(L, gu, sg, I, H, seed, KDG_GATE, slot, 2, 0, gs, i0, 0, H);
+    if (rc == KD_OK)
+      rc = gen_matrix(L, gu, sg ? sg + (size_t)d.nIb * d.nHb : nullptr, I, H, seed, KDG_UP, slot, 2, 1,
+                      gs, i0, 0, H);
+    if (rc == KD_OK) rc = gen_matrix(L, dn, sdn, H, I, seed, KDG_DOWN, slot, 1, 0, gs, 0, i0, c.inter);
   }
   if (rc == KD_OK && c.full_layer) {
     gen_norm_kernel<<<32, 256, 0, gs>>>(const_cast<uint16_t*>(d.g1), H,
@@ -459,11 +520,11 @@ extern "C" int kd_layer_create(const kd_config* cfg, uint64_t seed, kd_layer** o
   TRYC(se);
 
   {
-    bool ok = encode_weight_map(&L->maps.m[0], wqkv, Nqkv, H, fp8) &&
-              encode_weight_map(&L->maps.m[1], wo, H, A, fp8) &&
+    bool ok = encode_weight_map(&L->maps.m[0], wqkv, Nq, H, fp8) &&
+              encode_weight_map(&L->maps.m[1], wo, H, A_, fp8) &&
               encode_weight_map(&L->maps.m[2], wgu, (uint64_t)E * 2 * I, H, fp8) &&
               encode_weight_map(&L->maps.m[3], wd, (uint64_t)E * H, I, fp8) &&
-              encode_weight_map(&L->maps.m[6], wr, E, H, fp8);
+              encode_weight_map(&L->maps.m[6], wr, Er, H, fp8);
     if (ok && c.n_shared)
       ok = encode_weight_map(&L->maps.m[4], wgu_sh, 2 * I, H, fp8) &&
            encode_weight_map(&L->maps.m[5], wd_sh, H, I, fp8);
@@ -514,6 +575,7 @@ static int launch_layer(kd_layer* L, const Acts& a, cudaStream_t s, const kd_lay
 
 extern "C" int kd_decode_layer(kd_layer* L, void* hidden, const void* attn, int M, void* stream) {
   if (!L || !hidden || !attn) return fail(KD_EINVAL, "kd_decode_layer: null argument%s", "");
+  if (L->tp) return fail(KD_EINVAL, "kd_decode_layer: a tensor-parallel shard takes kd_tp_*%s", "");
   if (M < 1 || M > L->maxM)
     return fail(KD_ERANGE, "kd_decode_layer: M=%s%ld outside 1..max_tokens", "", (long)M);
   Acts a{};
@@ -664,6 +726,106 @@ static int launch_layer(kd_layer* L, const Acts& a, cudaStream_t s, const kd_lay
                    M, a.out));
   if (L->timing) KD_CUDA(cudaEventRecord(L->tev[4], s));
   if (next && pf) KD_CUDA(cudaStreamWaitEvent(s, ev_join, 0));
+  return KD_OK;
+}
+
+// ------------------------------------------------------------------ tensor parallel
+
+static int tp_args(const kd_layer* L, int M, const char* fn) {
+  if (!L || !L->tp) return fail(KD_EINVAL, "%s: not a tensor-parallel shard", fn);
+  if (M < 1 || M > L->maxM) return fail(KD_ERANGE, "%s: M outside 1..max_tokens", fn);
+  return KD_OK;
+}
+
+extern "C" int kd_tp_buffers(const kd_layer* L, float** p, float** lshard, float** lfull, float** y) {
+  if (!L || !L->tp || !p || !lshard || !lfull || !y)
+    return fail(KD_EINVAL, "kd_tp_buffers: bad arguments%s", "");
+  *p = L->d.h1f;
+  *lshard = L->d.logits;
+  *lfull = L->d.tp_lfull;
+  *y = L->d.tp_y;
+  return KD_OK;
+}
+
+// Phase 1: the shard's QKV rows and o-proj partial sum (into h1f).
+extern "C" int kd_tp_attn(kd_layer* L, const void* hidden, const void* attn, int M, void* stream) {
+  int rc = tp_args(L, M, "kd_tp_attn");
+  if (rc != KD_OK) return rc;
+  if (!hidden || !attn) return fail(KD_EINVAL, "kd_tp_attn: null argument%s", "");
+  Acts a{};
+  a.x = static_cast<const uint16_t*>(hidden);
+  a.attn = static_cast<const uint16_t*>(attn) + L->attn_col0;   // row stride: d.attn_ld
+  a.M = M;
+  return launch_front(L, a, static_cast<cudaStream_t>(stream), false);
+}
+
+// Phase 2: h1 = x + the summed partials; the shard's router logits.
+extern "C" int kd_tp_router(kd_layer* L, const void* hidden, int M, void* stream) {
+  int rc = tp_args(L, M, "kd_tp_router");
+  if (rc != KD_OK) return rc;
+  if (!hidden) return fail(KD_EINVAL, "kd_tp_router: null argument%s", "");
+  const LayerDev& d = L->d;
+  const bool fp8 = L->cfg.wdtype == KD_WFP8;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int ng = M * (d.H / 64);
+  KD_CUDA(launch(tp_h1_kernel, (ng + 255) / 256, 256, 0, s, false, d,
+                 static_cast<const uint16_t*>(hidden), M, (int)fp8));
+  const int rgrid = (d.Er + kRouterRows - 1) / kRouterRows;
+  KD_CUDA(launch(fp8 ? router_kernel<W_FP8> : router_kernel<W_BF16>, rgrid, kRouterThreads, 0, s,
+                 false, d, M));
+  return KD_OK;
+}
+
+// Phase 3: the selection from the gathered logits, then the shard's rows of
+// the experts (shared on the side stream, as in the whole layer) -> tp_y.
+extern "C" int kd_tp_moe(kd_layer* L, int M, void* stream) {
+  int rc = tp_args(L, M, "kd_tp_moe");
+  if (rc != KD_OK) return rc;
+  const LayerDev& d = L->d;
+  const bool fp8 = L->cfg.wdtype == KD_WFP8;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int G = L->nsm;
+  const bool mma = L->has_maps && M >= L->mma_min;
+  const size_t route_ints = sizeof(int) * kRouteSmemInts(d.E, M * d.k);
+  KD_CUDA(launch(tp_route_kernel, 1, kRouterThreads, route_ints, s, false, d, M));
+  const int gthreads = fp8 ? q8_threads(kGateUpConv) : kMThreads;
+  const int dthreads = fp8 ? q8_threads(kDownConv) : kMThreads;
+  if (d.S) {
+    KD_CUDA(cudaEventRecord(L->ev_h1, s));
+    KD_CUDA(cudaStreamWaitEvent(L->side, L->ev_h1, 0));
+    if (mma)
+      KD_CUDA(launch(fp8 ? mma_gateup_kernel<true> : mma_gateup_kernel<false>, G, gthreads, kMmaSmem,
+                     L->side, false, d, M, 1, L->maps));
+    else
+      KD_CUDA(launch(fp8 ? gateup_kernel<W_FP8> : gateup_kernel<W_BF16>, G, kThreads, kStreamSmem,
+                     L->side, false, d, M, 1));
+    KD_CUDA(cudaEventRecord(L->ev_sh, L->side));
+  }
+  if (mma)
+    KD_CUDA(launch(fp8 ? mma_gateup_kernel<true> : mma_gateup_kernel<false>, G, gthreads, kMmaSmem, s,
+                   false, d, M, 0, L->maps));
+  else
+    KD_CUDA(launch(fp8 ? gateup_kernel<W_FP8> : gateup_kernel<W_BF16>, G, kThreads,
+                   gateup_smem(d, M), s, false, d, M, 0));
+  if (d.S) KD_CUDA(cudaStreamWaitEvent(s, L->ev_sh, 0));
+  if (mma) {
+    KD_CUDA(launch(fp8 ? mma_down_kernel<true> : mma_down_kernel<false>, G, dthreads, kMmaSmem, s,
+                   false, d, M, L->maps));
+    KD_CUDA(launch(combine_kernel, 2 * G, 256, 0, s, false, d, M, (uint16_t*)nullptr));
+  } else {
+    KD_CUDA(launch(fp8 ? down_kernel<W_FP8> : down_kernel<W_BF16>, G, kThreads, kStreamSmem, s, false,
+                   d, M, (uint16_t*)nullptr));
+  }
+  return KD_OK;
+}
+
+// Phase 4: hidden = bf16(h1 + the summed expert partials).
+extern "C" int kd_tp_combine(kd_layer* L, void* hidden, int M, void* stream) {
+  int rc = tp_args(L, M, "kd_tp_combine");
+  if (rc != KD_OK) return rc;
+  if (!hidden) return fail(KD_EINVAL, "kd_tp_combine: null argument%s", "");
+  KD_CUDA(launch(tp_final_kernel, 2 * L->nsm, 256, 0, static_cast<cudaStream_t>(stream), false, L->d,
+                 static_cast<uint16_t*>(hidden), M));
   return KD_OK;
 }
 
@@ -833,6 +995,7 @@ extern "C" int kd_stack_create(kd_layer* const* layers, int n, int M, int prefet
   *out = nullptr;
   for (int i = 0; i < n; ++i) {
     if (!layers[i]) return fail(KD_EINVAL, "kd_stack_create: null layer%s", "");
+    if (layers[i]->tp) return fail(KD_EINVAL, "kd_stack_create: a tensor-parallel shard%s", "");
     if (M < 1 || M > layers[i]->maxM)
       return fail(KD_ERANGE, "kd_stack_create: M=%s%ld outside a layer's 1..max_tokens", "", (long)M);
     if (layers[i]->d.H != layers[0]->d.H || layers[i]->d.A != layers[0]->d.A)

@@ -91,7 +91,9 @@ struct MmaProjPlan {
     if (MODE == 2) return reinterpret_cast<const uint8_t*>(h ? L->attn_lo : L->attn_hi);
     return reinterpret_cast<const uint8_t*>(m.tag == 0 ? a.x : a.attn);
   }
-  KD_DEV int b_stride(const MUnit& m) const { return (m.tag == 0 ? L->H : L->A) * 2; }
+  KD_DEV int b_stride(const MUnit& m) const {
+    return (m.tag == 0 ? L->H : (MODE == 0 ? L->attn_ld : L->A)) * 2;
+  }
   KD_DEV int b_rowidx(const MUnit&, int j) const { return j; }
   KD_DEV bool paired() const { return false; }
   KD_DEV float epilogue(const MUnit& m, int r, int j, float v) const {
@@ -105,6 +107,10 @@ struct MmaProjPlan {
       return v;
     }
     const size_t o = (size_t)j * L->H + row;
+    if (MODE == 0 && L->tp) {   // a shard's o-proj partial sum
+      L->h1f[o] = v;
+      return v;
+    }
     // read-only here (a plain load could not move above the stores below)
     const float h = __uint_as_float((uint32_t)__ldg(a.x + o) << 16) + v;
     if (MODE == 2) {
@@ -487,7 +493,7 @@ __global__ void __launch_bounds__(256) combine_kernel(LayerDev L, int M, uint16_
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
     const int t = i / H2, h = 2 * (i - t * H2);
     const size_t o = (size_t)t * L.H + h;
-    float2 v = __ldcg(reinterpret_cast<const float2*>(L.resid + o));
+    float2 v = L.tp_y ? make_float2(0.f, 0.f) : __ldcg(reinterpret_cast<const float2*>(L.resid + o));
     if (L.S) {
       const float2 y = __ldcg(reinterpret_cast<const float2*>(L.ysh + o));
       v.x += y.x;
@@ -499,10 +505,54 @@ __global__ void __launch_bounds__(256) combine_kernel(LayerDev L, int M, uint16_
       v.x += g * y.x;
       v.y += g * y.y;
     }
+    if (L.tp_y) {   // a shard's expert partial sum
+      *reinterpret_cast<float2*>(L.tp_y + o) = v;
+      continue;
+    }
     const uint32_t pair = (uint32_t)f32_to_bf16_bits(v.x) | ((uint32_t)f32_to_bf16_bits(v.y) << 16);
     *reinterpret_cast<uint32_t*>(out + o) = pair;
   }
   pdl_launch_dependents();
+}
+
+// ------------------------------------------------------------------ tensor-parallel shard
+
+// h1 = x + (the o-proj partial sums of all shards, summed in place in h1f by
+// the caller), and the copies of h1 the later kernels read: bf16 (FP8
+// weights) or the bf16 hi + mid + lo terms, and for FP8 the per-64 maxima.
+// One thread per (token, 64 consecutive elements).
+__global__ void __launch_bounds__(256) tp_h1_kernel(LayerDev L, const uint16_t* x, int M, int fp8) {
+  static_assert(kQGroup == 64, "one thread per group of maxima");
+  const int ng = L.H / 64;
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= M * ng) return;
+  const int t = i / ng, g = i - t * ng;
+  float mx = 0.f;
+  for (int u = 0; u < 64; ++u) {
+    const size_t o = (size_t)t * L.H + g * 64 + u;
+    const float h = __uint_as_float((uint32_t)x[o] << 16) + L.h1f[o];
+    L.h1f[o] = h;
+    if (fp8) L.h1b[o] = f32_to_bf16_bits(h);
+    else store_hilo3(L.h1b, L.h1lo, L.h1lo2, o, h);
+    mx = fmaxf(mx, fabsf(h));
+  }
+  if (fp8 && L.h1g) L.h1g[(size_t)t * (L.H / kQGroup) + g] = mx;
+}
+
+// The selection, softmax and token lists of a shard from the gathered logits
+// (one CTA; the same on every shard).
+__global__ void __launch_bounds__(kRouterThreads) tp_route_kernel(LayerDev L, int M) {
+  extern __shared__ int route_smem[];
+  const Route R = carve_route(route_smem, L.E, M * L.k);
+  route_tokens(L, L.tp_lfull, M, R, true);
+}
+
+// hidden = bf16(h1 + the expert partial sums of all shards).
+__global__ void __launch_bounds__(256) tp_final_kernel(LayerDev L, uint16_t* out, int M) {
+  const size_t n = (size_t)M * L.H;
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (size_t)gridDim.x * blockDim.x)
+    out[i] = f32_to_bf16_bits(L.h1f[i] + L.tp_y[i]);
 }
 
 }  // namespace kd

@@ -137,6 +137,8 @@ extern "C" int kd_router_topk_static(const void* router_w, const float* router_s
   d.wr = static_cast<const uint8_t*>(router_w);
   d.sr = router_scales;
   d.bias = router_bias;
+  d.rbias = router_bias;
+  d.Er = n_experts;
   d.bias_sel = 0;
   d.rscale = 1.f;
   d.h1f = const_cast<float*>(h1);

@@ -71,3 +71,50 @@ def decode_tp(shard: ShardOps, hidden, attn, group=None):
     dist.all_reduce(y, op=dist.ReduceOp.SUM, group=group)
     shard.combine(y, hidden)
     return hidden
+
+
+class _DeviceArray:
+    """A layer-owned device buffer as a CUDA array interface (fp32, 2-D)."""
+
+    def __init__(self, ptr: int, shape):
+        self.__cuda_array_interface__ = {"shape": tuple(shape), "typestr": "<f4",
+                                         "data": (int(ptr), False), "version": 3, "strides": None}
+
+
+class CudaShard:
+    """ShardOps on one tensor-parallel shard of the CUDA layer (a
+    ``moe_decode_layer_skinny_b200.Layer`` created with tp_rank / tp_size):
+    the phases are its kd_tp_* calls; the partial sums live in the layer's
+    exchange buffers, which the collectives reduce in place."""
+
+    def __init__(self, layer, M: int):
+        import torch
+        self.layer, self.M = layer, M
+        s = layer.spec
+        R = s.tp_size
+        b = layer.tp_buffers()
+        dev = torch.device("cuda", torch.cuda.current_device())
+        self.p = torch.as_tensor(_DeviceArray(b["p"], (M, s.hidden)), device=dev)
+        self.lshard = torch.as_tensor(_DeviceArray(b["lshard"], (M, s.n_experts // R)), device=dev)
+        self.lfull = torch.as_tensor(_DeviceArray(b["lfull"], (M, s.n_experts)), device=dev)
+        self.y = torch.as_tensor(_DeviceArray(b["y"], (M, s.hidden)), device=dev)
+
+    def attn_partial(self, hidden, attn):
+        self.layer.tp_attn(hidden, attn, self.M)
+        return self.p
+
+    def router_shard(self, hidden, p_sum):
+        if p_sum.data_ptr() != self.p.data_ptr():
+            self.p.copy_(p_sum)
+        self.layer.tp_router(hidden, self.M)
+        return self.lshard
+
+    def moe_partial(self, logits):
+        self.lfull.copy_(logits)
+        self.layer.tp_moe(self.M)
+        return self.y
+
+    def combine(self, y_sum, hidden):
+        if y_sum.data_ptr() != self.y.data_ptr():
+            self.y.copy_(y_sum)
+        self.layer.tp_combine(hidden, self.M)

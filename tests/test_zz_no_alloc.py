@@ -5,6 +5,8 @@ __device__ array inside the library; here its output is checked, through the
 C ABI, against the router of kd_decode_layer on the same weights and h1, on
 two calls in a row, and the device's free memory is checked to be the same
 before and after a call.  This file is collected last on purpose."""
+import gc
+
 import numpy as np
 import pytest
 
@@ -44,6 +46,7 @@ def _case(kd, torch, dims, wdtype, bias, M):
         for call in range(2):
             idx.fill_(-1)
             gates.zero_()
+            gc.collect()   # objects of earlier tests freed now, not inside the window
             torch.cuda.synchronize()
             free0 = torch.cuda.mem_get_info()[0]
             alloc0 = torch.cuda.memory_allocated()
