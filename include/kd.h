@@ -108,9 +108,13 @@ typedef struct kd_stack kd_stack;
  * kdgen/kd_gen.h (synchronous).  The layer owns weights, workspaces, a side
  * stream and events; *out receives the handle.  Errors: KD_EINVAL for a bad
  * config, KD_ENOMEM, KD_ECUDA; on any error everything allocated so far is
- * released.  Test hook: with the environment variable KD_TEST_FAIL_ALLOC_AT=n
+ * released.  Test hooks: with the environment variable KD_TEST_FAIL_ALLOC_AT=n
  * (n >= 1) the n-th device allocation of the call fails as if the device
- * were out of memory. */
+ * were out of memory; with KD_TEST_STALL_WAIT=1 the layer's tensor-core
+ * kernels first wait on a pipeline barrier that nothing completes, so that
+ * the bounded wait gives up after its limit (2 s), the kernel stops its roles
+ * and returns, and kd_layer_check reports KD_ETIMEOUT (the layer stays
+ * usable; the calls' outputs are then undefined). */
 int kd_layer_create(const kd_config* cfg, uint64_t seed, kd_layer** out);
 
 /* Release everything kd_layer_create allocated (NULL is ignored).  The caller

@@ -84,6 +84,7 @@ struct LayerDev {
   // full width); the o-proj epilogue then writes the partial sum alone, the
   // router no selection, and the combine the fp32 expert sum into tp_y.
   int Er, attn_ld, tp;
+  int test_stall;                       // test hook: tensor-core kernels stall first (bounded)
   float* tp_y;                          // [Mmax, H] expert partial sum (shards)
   float* tp_lfull;                      // [Mmax, E] gathered logits (shards)
   const float* rbias;                   // bias of the router rows (bias + first row)

@@ -293,6 +293,7 @@ extern "C" int kd_layer_create(const kd_config* cfg, uint64_t seed, kd_layer** o
   kd_layer* L = new kd_layer();
   L->cfg = c;
   if (const char* f = getenv("KD_TEST_FAIL_ALLOC_AT")) L->fail_alloc_at = atoi(f);
+  if (const char* f = getenv("KD_TEST_STALL_WAIT")) L->d.test_stall = atoi(f) == 1;
   L->cfg.router_bias = nullptr;
   L->maxM = c.max_tokens;
   L->mma_min = c.mma_min_tokens > 0 ? c.mma_min_tokens : 3;

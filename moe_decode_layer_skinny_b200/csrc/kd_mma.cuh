@@ -1240,6 +1240,10 @@ KD_DEV void mma_run(const Plan& plan, uint8_t* smem_raw, unsigned* err) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *sh.tmem_base;
+  // test hook: one wait that nothing completes (the drain barrier, which is
+  // only ever committed after an abort); it gives up after the limit and
+  // raises the abort flag, and the roles below stop at their first blocked wait
+  if (plan.L->test_stall && threadIdx.x == 32) mwait(sh.drain, 0, sh.abort_flag, err);
   if (warp == 0) {
     if ((threadIdx.x & 31) == 0) mma_producer_a(plan, sh, err);
   } else if (warp == 1) {
