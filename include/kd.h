@@ -249,7 +249,7 @@ int kd_layer_bytes(const kd_layer* layer, uint64_t* static_bytes, uint64_t* expe
  * compare decode paths (bigchange.ai "where the time went"; wireai.ir
  * "compressing the decode loop with kernel fusion"); for a layer created
  * with full_layer, the count of one kd_decode_layer_full call.  Returns the count
- * (>= 4), or KD_EINVAL for a null layer, KD_ERANGE for M outside
+ * (>= 5), or KD_EINVAL for a null layer, KD_ERANGE for M outside
  * 1..max_tokens. */
 int kd_layer_launches(const kd_layer* layer, int M);
 

@@ -126,7 +126,6 @@ struct LayerDev {
   float* attnf; uint16_t* attn_hi; uint16_t* attn_lo;   // attention output [Mmax, A]
   float* att_ws; unsigned* att_cnt;        // per-chunk partials, (token, kv head) arrivals
   float* h1r;                              // h1 = x + Wo o [Mmax, H]
-  unsigned* hcnt;                          // [H/64] down rows done per block (self-resetting)
   unsigned* rcnt;                          // router blocks done (self-resetting)
   unsigned* err;
 };
@@ -248,6 +247,7 @@ __global__ void __launch_bounds__(kThreads, 1) proj_kernel(LayerDev L, Acts a) {
 // routed-expert kernel.
 constexpr int kRouterThreads = 256;
 constexpr int kRouterRows = 2;
+constexpr int kCoreRouterMaxM = 8;   // bf16 layers: the CUDA-core router up to this many tokens
 
 // Accumulate one 16-byte weight chunk against up to kTT fp32 activation rows.
 template <int WT>
@@ -673,8 +673,6 @@ struct GateUpPlan {
 // expert, in one launch.
 struct DownPlan {
   const LayerDev* L; int M; int n_act; ExpertRange R;
-  uint16_t* out;                 // layer output [M, H] bf16
-  int* s_list; int* s_n;         // shared scratch: blocks this CTA completes
   KD_DEV int num_segments() const { return R.num_segments(); }
   KD_DEV Seg segment(int i) const {
     int a, u0, u1;
@@ -707,46 +705,8 @@ struct DownPlan {
     else L->yr[(size_t)L->perm[s.tok0 + j] * L->H + h] = v;
   }
   KD_DEV void epilogue2(const Seg&, int, int, float, float) const {}
-  KD_DEV bool wants_segment_done() const { return true; }
-
-  // Count the segment's rows into their 64-row blocks; the CTA whose rows
-  // complete a block (every routed entry and the shared one) writes that
-  // block of the layer output:
-  //   out[t, h] = bf16(h1[t, h] + ysh[t, h] + sum_j g[t, j] yr[t*k + j, h])
-  // with the terms added in this fixed order.
-  KD_DEV void segment_done(const Seg& s) const {
-    const int target = 64 * (n_act + L->S);
-    if (threadIdx.x == 0) {
-      *s_n = 0;
-      __threadfence();
-      for (int b = s.row0 / 64; b * 64 < s.row0 + s.nrows; ++b) {
-        const int lo = b * 64 > s.row0 ? b * 64 : s.row0;
-        const int hi = (b + 1) * 64 < s.row0 + s.nrows ? (b + 1) * 64 : s.row0 + s.nrows;
-        const unsigned prev = atomicAdd(L->hcnt + b, (unsigned)(hi - lo));
-        if (prev + (unsigned)(hi - lo) == (unsigned)target) {
-          L->hcnt[b] = 0u;  // every contribution is in: ready for the next call
-          s_list[(*s_n)++] = b;
-        }
-      }
-      __threadfence();
-    }
-    named_bar_sync(1, kThreads);
-    const int nb = *s_n;
-    for (int q = 0; q < nb; ++q) {
-      const int b = s_list[q];
-      for (int e = threadIdx.x; e < 64 * M; e += kThreads) {
-        const int t = e / 64, h = b * 64 + e % 64;
-        const size_t o = (size_t)t * L->H + h;
-        float v = L->tp_y ? 0.f : L->resid[o];
-        if (L->S) v += __ldcg(L->ysh + o);
-        for (int j = 0; j < L->k; ++j)
-          v += (L->rscale * L->gates[t * L->k + j]) * __ldcg(L->yr + ((size_t)t * L->k + j) * L->H + h);
-        if (L->tp_y) L->tp_y[o] = v;   // a shard's expert partial sum
-        else out[o] = f32_to_bf16_bits(v);
-      }
-    }
-    named_bar_sync(1, kThreads);  // s_list / s_n are reused by the next segment
-  }
+  KD_DEV bool wants_segment_done() const { return false; }
+  KD_DEV void segment_done(const Seg&) const {}
 };
 
 KD_DEV ExpertRange expert_range(int n_act, int per) {
@@ -779,14 +739,12 @@ __global__ void __launch_bounds__(kThreads, 1) gateup_kernel(LayerDev L, int M, 
 }
 
 template <int WT>
-__global__ void __launch_bounds__(kThreads, 1) down_kernel(LayerDev L, int M, uint16_t* out) {
+__global__ void __launch_bounds__(kThreads, 1) down_kernel(LayerDev L, int M) {
   extern __shared__ uint8_t smem[];
-  __shared__ int s_list[128];
-  __shared__ int s_n;
   pdl_wait();
   pdl_launch_dependents();
   DownPlan p;
-  p.L = &L; p.M = M; p.out = out; p.s_list = s_list; p.s_n = &s_n;
+  p.L = &L; p.M = M;
   p.n_act = *(volatile int*)L.n_active;
   p.R = expert_range(p.n_act + L.S, L.H);
   stream_run<WT, A_F32>(p, smem, L.err, false);

@@ -404,7 +404,6 @@ extern "C" int kd_layer_create(const kd_config* cfg, uint64_t seed, kd_layer** o
   TRY(dalloc_t(L, (size_t)M * I, &d.act_sh));
   TRY(dalloc_t(L, (size_t)M * k * H, &d.yr));
   TRY(dalloc_t(L, (size_t)M * H, &d.ysh));
-  TRY(dalloc_t(L, (size_t)H / 64, &d.hcnt));
   TRY(dalloc_t(L, 1, &d.rcnt));
   TRY(dalloc_t(L, (size_t)M * H, &d.h1lo));
   TRY(dalloc_t(L, (size_t)M * H, &d.h1lo2));
@@ -466,7 +465,6 @@ extern "C" int kd_layer_create(const kd_config* cfg, uint64_t seed, kd_layer** o
     TRYC(cudaMemset(d.tcnt_main, 0, sizeof(unsigned) * ntile));
     TRYC(cudaMemset(d.tcnt_side, 0, sizeof(unsigned) * ntile));
   }
-  TRYC(cudaMemset(d.hcnt, 0, sizeof(unsigned) * (H / 64)));
   TRYC(cudaMemset(d.rcnt, 0, sizeof(unsigned)));
   TRY(dalloc_t(L, 1, &d.err));
   TRYC(cudaMemset(d.err, 0, sizeof(unsigned)));
@@ -678,8 +676,10 @@ static int launch_layer(kd_layer* L, const Acts& a, cudaStream_t s, const kd_lay
   if (d.S) KD_CUDA(cudaEventRecord(L->ev_h1, s));
 
   // FP8 routers stay on CUDA cores: the tensor-core path rounds each scaled
-  // weight to bf16, which the fp32 router logits cannot afford
-  if (mma && !fp8) {
+  // weight to bf16, which the fp32 router logits cannot afford.  Up to
+  // kCoreRouterMaxM tokens the CUDA-core router (one CTA per two experts) is
+  // also the faster one: the tensor-core router's small grid is a latency chain.
+  if (mma && !fp8 && M > kCoreRouterMaxM) {
     const int rsub = mma_nsub(M, 3);
     const int rchunks = ((d.E + 127) / 128) * (d.H / (64 * rsub));
     const int rgrid = std::max(1, std::min(G, rchunks / (kRouterChunksPerCta * 2 / rsub)));
@@ -722,9 +722,12 @@ static int launch_layer(kd_layer* L, const Acts& a, cudaStream_t s, const kd_lay
     KD_CUDA(launch(fp8 ? mma_down_kernel<true> : mma_down_kernel<false>, G, dthreads, msm, s,
                    pdl_down, d, M, L->maps));
     KD_CUDA(launch(combine_kernel, 2 * G, 256, 0, s, !L->timing, d, M, a.out));
-  } else
+  } else {
+    // the CUDA-core down writes each expert's outputs too; the combine follows
     KD_CUDA(launch(fp8 ? down_kernel<W_FP8> : down_kernel<W_BF16>, G, kThreads, sm, s, pdl_down, d,
-                   M, a.out));
+                   M));
+    KD_CUDA(launch(combine_kernel, 2 * G, 256, 0, s, !L->timing, d, M, a.out));
+  }
   if (L->timing) KD_CUDA(cudaEventRecord(L->tev[4], s));
   if (next && pf) KD_CUDA(cudaStreamWaitEvent(s, ev_join, 0));
   return KD_OK;
@@ -815,7 +818,8 @@ extern "C" int kd_tp_moe(kd_layer* L, int M, void* stream) {
     KD_CUDA(launch(combine_kernel, 2 * G, 256, 0, s, false, d, M, (uint16_t*)nullptr));
   } else {
     KD_CUDA(launch(fp8 ? down_kernel<W_FP8> : down_kernel<W_BF16>, G, kThreads, kStreamSmem, s, false,
-                   d, M, (uint16_t*)nullptr));
+                   d, M));
+    KD_CUDA(launch(combine_kernel, 2 * G, 256, 0, s, false, d, M, (uint16_t*)nullptr));
   }
   return KD_OK;
 }
@@ -838,7 +842,6 @@ extern "C" int kd_layer_check(kd_layer* L) {
   if (e == 0) return KD_OK;
   KD_CUDA(cudaMemset(L->d.err, 0, sizeof(unsigned)));
   // an aborted call may have left arrival counters part-way
-  KD_CUDA(cudaMemset(L->d.hcnt, 0, sizeof(unsigned) * (L->d.H / 64)));
   KD_CUDA(cudaMemset(L->d.rcnt, 0, sizeof(unsigned)));
   KD_CUDA(cudaMemset(L->d.tcnt_main, 0, sizeof(unsigned) * L->ntile));
   KD_CUDA(cudaMemset(L->d.tcnt_side, 0, sizeof(unsigned) * L->ntile));
@@ -975,11 +978,10 @@ extern "C" int kd_layer_launches(const kd_layer* L, int M) {
   if (!L) return fail(KD_EINVAL, "kd_layer_launches: null layer%s", "");
   if (M < 1 || M > L->maxM)
     return fail(KD_ERANGE, "kd_layer_launches: M=%s%ld outside 1..max_tokens", "", (long)M);
-  const bool mma = L->has_maps && M >= L->mma_min;
-  // projections, router, routed gate/up, down (+ combine on the tensor-core
-  // path), + the shared expert's gate/up; a full layer runs RMSNorm, QKV,
-  // attention, o-proj and RMSNorm in place of the projections' launch
-  return 4 + (mma ? 1 : 0) + (L->d.S ? 1 : 0) + (L->full ? 4 : 0);
+  // projections, router, routed gate/up, down, combine, + the shared
+  // expert's gate/up; a full layer runs RMSNorm, QKV, attention, o-proj and
+  // RMSNorm in place of the projections' launch (the same for every M)
+  return 5 + (L->d.S ? 1 : 0) + (L->full ? 4 : 0);
 }
 
 extern "C" int kd_layer_bytes(const kd_layer* L, uint64_t* static_bytes, uint64_t* expert_bytes) {

@@ -235,7 +235,7 @@ def test_full_layer_entry_point_errors(kd):
         with pytest.raises(kd.KdError) as ei:
             L.decode_full(h, c, c, i, i, 5)
         assert ei.value.code == kd.KD_ERANGE
-        assert L.launches(1) == 9 and L.launches(3) == 10
+        assert L.launches(1) == 10 and L.launches(3) == 10
     finally:
         L.close()
 

@@ -168,9 +168,9 @@ def test_error_paths(kd):
         assert kd.lib().kd_decode_layer(L.handle, None, a.data_ptr(), 1, None) == kd.KD_EINVAL
         L.decode(h, a, 4)
         L.check()
-        # launches per call: CUDA-core path below 3 tokens, tensor-core path
-        # (+ the combine launch) from 3; + the shared expert's gate/up
-        assert L.launches(1) == 5 and L.launches(2) == 5
+        # launches per call: projections, router, gate/up, down, combine, +
+        # the shared expert's gate/up, on either path
+        assert L.launches(1) == 6 and L.launches(2) == 6
         assert L.launches(3) == 6 and L.launches(4) == 6
         with pytest.raises(kd.KdError) as ei:
             L.launches(5)
