@@ -98,6 +98,12 @@ typedef struct kd_config {
      full layer.  Otherwise KD_EINVAL.                                        */
   int tp_rank;
   int tp_size;
+  /* FP8 expert activations on the tensor cores: e4m3 terms of each activation
+     (times its 128 x 128 weight block's scale and a power of two per token
+     and tile): 0 or 2 = two terms (~8 significant bits); 1 = one term (W8A8,
+     ~4 significant bits, larger error).  Ignored for bf16 weights; other
+     values KD_EINVAL.                                                        */
+  int fp8_act_terms;
 } kd_config;
 
 typedef struct kd_layer kd_layer;

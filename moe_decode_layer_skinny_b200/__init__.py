@@ -48,7 +48,8 @@ class _Config(ctypes.Structure):
                 ("kv_n_seq", ctypes.c_int), ("kv_max_ctx", ctypes.c_int),
                 ("k_scale", ctypes.c_float), ("v_scale", ctypes.c_float),
                 ("bias_select_only", ctypes.c_int), ("routed_scale", ctypes.c_float),
-                ("tp_rank", ctypes.c_int), ("tp_size", ctypes.c_int)]
+                ("tp_rank", ctypes.c_int), ("tp_size", ctypes.c_int),
+                ("fp8_act_terms", ctypes.c_int)]
 
 
 _lib = None
@@ -129,6 +130,7 @@ class LayerSpec:
     routed_scale: float = 0.0
     tp_rank: int = 0
     tp_size: int = 0
+    fp8_act_terms: int = 0
 
     @classmethod
     def from_dims(cls, dims, **kw) -> "LayerSpec":
@@ -149,7 +151,7 @@ class Layer:
                       spec.max_tokens, None if bias is None else bias.ctypes.data,
                       spec.mma_min_tokens, spec.full_layer, spec.rms_eps, spec.kv_n_seq,
                       spec.kv_max_ctx, spec.k_scale, spec.v_scale, spec.bias_select_only,
-                      spec.routed_scale, spec.tp_rank, spec.tp_size)
+                      spec.routed_scale, spec.tp_rank, spec.tp_size, spec.fp8_act_terms)
         h = ctypes.c_void_p()
         _check(lib().kd_layer_create(ctypes.byref(cfg), seed, ctypes.byref(h)))
         self._h = h

@@ -52,6 +52,7 @@ struct kd_layer {
   uint64_t static_bytes = 0, expert_bytes = 0;
   int Nqkv = 0, A = 0;
   bool tp = false;       // a tensor-parallel shard (kd_tp_* calls)
+  bool w8a8 = false;     // FP8 experts with one e4m3 activation term
   int attn_col0 = 0;     // a shard's first attention-output column
   cudaEvent_t tev[KD_N_TIMING_EVENTS] = {};  // profiling hook (kd_layer_set_timing_events)
   bool timing = false;
@@ -231,6 +232,8 @@ static int configure_kernels() {
   KD_CUDA(cudaFuncSetAttribute(mma_proj_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem));
   KD_CUDA(cudaFuncSetAttribute(mma_gateup_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem));
   KD_CUDA(cudaFuncSetAttribute(mma_down_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem));
+  KD_CUDA(cudaFuncSetAttribute(mma_gateup_kernel<true, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem));
+  KD_CUDA(cudaFuncSetAttribute(mma_down_kernel<true, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem));
   KD_CUDA(cudaFuncSetAttribute(proj_kernel<W_BF16, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   KD_CUDA(cudaFuncSetAttribute(proj_kernel<W_BF16, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   KD_CUDA(cudaFuncSetAttribute(proj_kernel<W_FP8, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
@@ -259,7 +262,8 @@ extern "C" int kd_layer_create(const kd_config* cfg, uint64_t seed, kd_layer** o
       c.top_k > 16 || c.top_k > c.n_experts || c.n_shared < 0 || c.n_shared > 1 || c.inter <= 0 ||
       c.inter % 128 || (c.wdtype != KD_WBF16 && c.wdtype != KD_WFP8) || c.max_tokens < 1 ||
       c.max_tokens > 64 || c.layer_id < 0 || c.mma_min_tokens < 0 ||
-      (c.bias_select_only != 0 && c.bias_select_only != 1))
+      (c.bias_select_only != 0 && c.bias_select_only != 1) || c.fp8_act_terms < 0 ||
+      c.fp8_act_terms > 2)
     return fail(KD_EINVAL, "kd_layer_create: unsupported configuration%s", "");
   if (c.hidden * 2 > kStageBytes || A * 2 > kStageBytes || c.inter * 2 > kStageBytes ||
       c.hidden > 8192 || A > 8192 || c.inter > 8192)
@@ -294,6 +298,7 @@ extern "C" int kd_layer_create(const kd_config* cfg, uint64_t seed, kd_layer** o
   L->cfg = c;
   if (const char* f = getenv("KD_TEST_FAIL_ALLOC_AT")) L->fail_alloc_at = atoi(f);
   if (const char* f = getenv("KD_TEST_STALL_WAIT")) L->d.test_stall = atoi(f) == 1;
+  L->w8a8 = c.fp8_act_terms == 1;
   L->cfg.router_bias = nullptr;
   L->maxM = c.max_tokens;
   L->mma_min = c.mma_min_tokens > 0 ? c.mma_min_tokens : 3;
@@ -607,6 +612,18 @@ extern "C" int kd_decode_layer_full(kd_layer* L, void* hidden, void* k_cache, vo
                       false);
 }
 
+// The tensor-core expert kernels for the layer's weight format.
+using GateupMmaFn = void (*)(LayerDev, int, int, const MmaMaps);
+using DownMmaFn = void (*)(LayerDev, int, const MmaMaps);
+static GateupMmaFn gateup_mma_for(const kd_layer* L) {
+  if (L->cfg.wdtype != KD_WFP8) return mma_gateup_kernel<false>;
+  return L->w8a8 ? mma_gateup_kernel<true, 1> : mma_gateup_kernel<true>;
+}
+static DownMmaFn down_mma_for(const kd_layer* L) {
+  if (L->cfg.wdtype != KD_WFP8) return mma_down_kernel<false>;
+  return L->w8a8 ? mma_down_kernel<true, 1> : mma_down_kernel<true>;
+}
+
 // The front of the layer up to h1 (and, in the full layer, the MoE input
 // w = RMSNorm(h1) g2): the chain with a given attn_out runs QKV and o-proj in
 // one launch; the full layer runs RMSNorm -> QKV (+ KV cache append) ->
@@ -692,7 +709,7 @@ static int launch_layer(kd_layer* L, const Acts& a, cudaStream_t s, const kd_lay
   if (d.S) {
     KD_CUDA(cudaStreamWaitEvent(L->side, L->ev_h1, 0));
     if (mma)
-      KD_CUDA(launch(fp8 ? mma_gateup_kernel<true> : mma_gateup_kernel<false>, G, gthreads, msm,
+      KD_CUDA(launch(gateup_mma_for(L), G, gthreads, msm,
                      L->side, false, d, M, 1, L->maps));
     else
       KD_CUDA(launch(fp8 ? gateup_kernel<W_FP8> : gateup_kernel<W_BF16>, G, kThreads, sm, L->side,
@@ -701,7 +718,7 @@ static int launch_layer(kd_layer* L, const Acts& a, cudaStream_t s, const kd_lay
   }
   if (L->timing) KD_CUDA(cudaEventRecord(L->tev[2], s));
   if (mma)
-    KD_CUDA(launch(fp8 ? mma_gateup_kernel<true> : mma_gateup_kernel<false>, G, gthreads, msm, s,
+    KD_CUDA(launch(gateup_mma_for(L), G, gthreads, msm, s,
                    !L->timing, d, M, 0, L->maps));
   else
     KD_CUDA(launch(fp8 ? gateup_kernel<W_FP8> : gateup_kernel<W_BF16>, G, kThreads,
@@ -719,7 +736,7 @@ static int launch_layer(kd_layer* L, const Acts& a, cudaStream_t s, const kd_lay
   const bool pdl_down = !L->timing && !d.S && !(next && pf);
   if (mma) {
     // tensor-core down writes each expert's outputs; the combine follows
-    KD_CUDA(launch(fp8 ? mma_down_kernel<true> : mma_down_kernel<false>, G, dthreads, msm, s,
+    KD_CUDA(launch(down_mma_for(L), G, dthreads, msm, s,
                    pdl_down, d, M, L->maps));
     KD_CUDA(launch(combine_kernel, 2 * G, 256, 0, s, !L->timing, d, M, a.out));
   } else {
@@ -798,7 +815,7 @@ extern "C" int kd_tp_moe(kd_layer* L, int M, void* stream) {
     KD_CUDA(cudaEventRecord(L->ev_h1, s));
     KD_CUDA(cudaStreamWaitEvent(L->side, L->ev_h1, 0));
     if (mma)
-      KD_CUDA(launch(fp8 ? mma_gateup_kernel<true> : mma_gateup_kernel<false>, G, gthreads, kMmaSmem,
+      KD_CUDA(launch(gateup_mma_for(L), G, gthreads, kMmaSmem,
                      L->side, false, d, M, 1, L->maps));
     else
       KD_CUDA(launch(fp8 ? gateup_kernel<W_FP8> : gateup_kernel<W_BF16>, G, kThreads, kStreamSmem,
@@ -806,14 +823,14 @@ extern "C" int kd_tp_moe(kd_layer* L, int M, void* stream) {
     KD_CUDA(cudaEventRecord(L->ev_sh, L->side));
   }
   if (mma)
-    KD_CUDA(launch(fp8 ? mma_gateup_kernel<true> : mma_gateup_kernel<false>, G, gthreads, kMmaSmem, s,
+    KD_CUDA(launch(gateup_mma_for(L), G, gthreads, kMmaSmem, s,
                    false, d, M, 0, L->maps));
   else
     KD_CUDA(launch(fp8 ? gateup_kernel<W_FP8> : gateup_kernel<W_BF16>, G, kThreads,
                    gateup_smem(d, M), s, false, d, M, 0));
   if (d.S) KD_CUDA(cudaStreamWaitEvent(s, L->ev_sh, 0));
   if (mma) {
-    KD_CUDA(launch(fp8 ? mma_down_kernel<true> : mma_down_kernel<false>, G, dthreads, kMmaSmem, s,
+    KD_CUDA(launch(down_mma_for(L), G, dthreads, kMmaSmem, s,
                    false, d, M, L->maps));
     KD_CUDA(launch(combine_kernel, 2 * G, 256, 0, s, false, d, M, (uint16_t*)nullptr));
   } else {

@@ -144,7 +144,8 @@ static_assert(kMmaSmem + 64 <= 227 * 1024, "shared memory per CTA (with the kern
 constexpr int kQ8AccCols = 256;                       // q8: one accumulator, <= 2 x 2 x 64 columns
 constexpr int kQ8TmemCols = 2 * kQ8AccCols;           // q8: two accumulators
 constexpr int kQGroup = 64;                           // activation elements per stored maximum
-constexpr int kQTerms = 2;                            // e4m3 terms of a q8 activation
+constexpr int kQTerms = 2;                            // e4m3 terms of a q8 activation (at most;
+                                                      // a plan's kQT: 2, or 1 for W8A8)
 constexpr int kQ8XBudget = 40 * 1024;                 // q8: bytes of the activation-row ring
 
 // One unit of work: K chunks [kc0, kc0 + nkc) of a 128-row weight tile.
@@ -694,7 +695,7 @@ KD_DEV void mma_issuer(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigned*
 // the bf16 plans) and the epilogue adds the term columns.
 template <class Plan>
 KD_DEV void mma_issuer_q8(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigned* err) {
-  constexpr int NV = Plan::kVariants, nh = kQTerms;
+  constexpr int NV = Plan::kVariants, nh = Plan::kQT;
   uint32_t nu = 0, ph = 0;
   int s = 0;
   const uint32_t ring0 = smem_u32(sh.stage);
@@ -763,7 +764,7 @@ KD_DEV float q8_unit_scale(const Plan& plan, const MUnit& m, int j, int v, float
 template <class Plan>
 KD_DEV void q8_convert_stage(const Plan& plan, MmaShared& sh, const MUnit& m, int c, int s,
                              int xsl, const float* pm) {
-  constexpr int NV = Plan::kVariants, nh = kQTerms, C = NV * nh;
+  constexpr int NV = Plan::kVariants, nh = Plan::kQT, C = NV * nh;
   const int lane = threadIdx.x & 31;
   uint8_t* bt = sh.stage + (size_t)s * sh.stage_bytes + sh.boff;
   const uint8_t* xs = sh.xring + (size_t)xsl * sh.xslot;
@@ -1086,7 +1087,7 @@ KD_DEV void mma_epilogue_q8(const Plan& plan, MmaShared& sh, uint32_t tmem, unsi
   MUnit m;
   for (; units.next(m); ++nu_local) {
     const int N = pad16(m.ntok);
-    const int NC = pad16(NV * kQTerms * m.ntok);   // accumulator columns
+    const int NC = pad16(NV * Plan::kQT * m.ntok);   // accumulator columns
     const int buf = nu_local & 1;
     // the unit's 2^-P per (variant, token), shared by the four warps
     named_bar_sync(2, 128);   // every warp is done with the previous unit's table
@@ -1107,7 +1108,7 @@ KD_DEV void mma_epilogue_q8(const Plan& plan, MmaShared& sh, uint32_t tmem, unsi
     // columns (token j's C columns start at j C), scaled.  C loads of 16
     // columns; every lane loads every column (tcgen05.ld is warp-wide).
     auto load16 = [&](int c, float* out) {
-      constexpr int C = NV * kQTerms, TPL = 16 / C;   // tokens per 16-column load
+      constexpr int C = NV * Plan::kQT, TPL = 16 / C;   // tokens per 16-column load
       float d[C][16];
 #pragma unroll
       for (int q = 0; q < C; ++q) {
@@ -1127,7 +1128,7 @@ KD_DEV void mma_epilogue_q8(const Plan& plan, MmaShared& sh, uint32_t tmem, unsi
         for (int v = 0; v < NV; ++v)
           if (v == myv) {
 #pragma unroll
-            for (int h = 0; h < kQTerms; ++h) acc += d[q][base + v * kQTerms + h];
+            for (int h = 0; h < Plan::kQT; ++h) acc += d[q][base + v * Plan::kQT + h];
           }
         out[j] = acc * qt[c + j];
       }

@@ -271,8 +271,9 @@ __global__ void __launch_bounds__(F8 ? kMThreadsF8 : kMThreads, 1)
 // (q8): the e4m3 tiles as they land, B made from h1 (fp32) per stage with
 // the gate rows' and the up rows' block scales (two variants), and the
 // SwiGLU activations' per-64 maxima written for the down kernel.
-template <bool F8>
+template <bool F8, int NT = kQTerms>
 struct MmaGateUpPlan {
+  static constexpr int kQT = NT;         // q8: e4m3 terms of an activation (1: W8A8)
   static constexpr bool kFp8 = false;    // no converter warps
   static constexpr bool kQ8 = F8;
   static constexpr int kConv = F8 ? kGateUpConv : 0;   // q8 converter warps
@@ -301,9 +302,9 @@ struct MmaGateUpPlan {
   }
   KD_DEV const CUtensorMap* map(int id) const { return &maps->m[id]; }
   KD_DEV int max_n() const { return nmax; }
-  // bf16: hi + lo activations; q8: kQTerms e4m3 terms for each of the two
+  // bf16: hi + lo activations; q8: NT e4m3 terms for each of the two
   // scale variants (B tiles per stage)
-  static constexpr int kTerms = F8 ? kVariants * kQTerms : 2;
+  static constexpr int kTerms = F8 ? kVariants * NT : 2;
   KD_DEV const uint8_t* b_base(const MUnit&, int h) const {
     return reinterpret_cast<const uint8_t*>(h ? L->h1lo : L->h1b);
   }
@@ -355,11 +356,11 @@ struct MmaGateUpPlan {
   KD_DEV void after_run(MmaShared&, uint8_t*) const {}
 };
 
-template <bool F8>
+template <bool F8, int NT = kQTerms>
 __global__ void __launch_bounds__(F8 ? q8_threads(kGateUpConv) : kMThreads, 1)
     mma_gateup_kernel(LayerDev L, int M, int shared, const __grid_constant__ MmaMaps maps) {
   extern __shared__ uint8_t smem[];
-  MmaGateUpPlan<F8> p;
+  MmaGateUpPlan<F8, NT> p;
   p.L = &L; p.M = M; p.shared = shared != 0; p.maps = &maps; p.n_act = 1;
   p.nmax = M;
   if (!shared) {
@@ -383,8 +384,9 @@ __global__ void __launch_bounds__(F8 ? q8_threads(kGateUpConv) : kMThreads, 1)
 // pair (q8: the e4m3 terms of the activations).  The epilogue writes each
 // expert's rows of its tokens' outputs (yr, ysh); the gate-weighted combine
 // into the layer output is the next launch.
-template <bool F8>
+template <bool F8, int NT = kQTerms>
 struct MmaDownPlan {
+  static constexpr int kQT = NT;         // q8: e4m3 terms of an activation (1: W8A8)
   static constexpr bool kFp8 = false;    // no converter warps
   static constexpr bool kQ8 = F8;
   static constexpr int kConv = F8 ? kDownConv : 0;   // q8 converter warps
@@ -399,13 +401,13 @@ struct MmaDownPlan {
     return (long long)t * (L->I / (F8 ? 128 : 64 * nsub));
   }
   // The shared expert's tiles are spread evenly through the sequence (tile t
-  // is one iff floor((t + 1) S / NT) > floor(t S / NT), S of the NT tiles), so
+  // is one iff floor((t + 1) S / T) > floor(t S / T), S of the T tiles), so
   // that the CTAs' contiguous ranges share its wider token groups.
   KD_DEV MUnit tile_unit(int t) const {
     MUnit m{};
-    const long long NT = num_tiles(), S = (long long)nsh * tiles_per();
-    const int sb = (int)((long long)t * S / NT);   // shared tiles before t
-    const bool sh = (int)((long long)(t + 1) * S / NT) > sb;
+    const long long T = num_tiles(), S = (long long)nsh * tiles_per();
+    const int sb = (int)((long long)t * S / T);   // shared tiles before t
+    const bool sh = (int)((long long)(t + 1) * S / T) > sb;
     const int idx = sh ? sb : t - sb;
     const int a = idx / tiles_per(), tt = idx % tiles_per();
     if (sh) {
@@ -422,8 +424,8 @@ struct MmaDownPlan {
   }
   KD_DEV const CUtensorMap* map(int id) const { return &maps->m[id]; }
   KD_DEV int max_n() const { return nmax; }
-  // bf16: hi + lo activations; q8: kQTerms e4m3 terms
-  static constexpr int kTerms = F8 ? kQTerms : 2;
+  // bf16: hi + lo activations; q8: NT e4m3 terms
+  static constexpr int kTerms = F8 ? NT : 2;
   KD_DEV float w_scale_v(const MUnit& m, int kc, int) const {
     const float* base = m.tag < 0 ? L->sd_sh : L->sd + (size_t)m.tag * L->nHb * L->nIb;
     return __ldg(base + (size_t)(m.lrow >> 7) * L->nIb + kc);
@@ -456,13 +458,13 @@ struct MmaDownPlan {
   KD_DEV void after_run(MmaShared&, uint8_t*) const {}
 };
 
-template <bool F8>
+template <bool F8, int NT = kQTerms>
 __global__ void __launch_bounds__(F8 ? q8_threads(kDownConv) : kMThreads, 1)
     mma_down_kernel(LayerDev L, int M, const __grid_constant__ MmaMaps maps) {
   extern __shared__ uint8_t smem[];
   pdl_wait();
   pdl_launch_dependents();
-  MmaDownPlan<F8> p;
+  MmaDownPlan<F8, NT> p;
   p.L = &L; p.M = M; p.maps = &maps;
   p.n_act = *(volatile int*)L.n_active;
   p.nmax = max_tokens_per_expert(L.counts, L.active, p.n_act);

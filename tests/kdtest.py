@@ -27,8 +27,14 @@ import numpy as np
 import kdgen
 import oracle
 
-TOL = {0: 1e-2, 1: 3e-2}
-TIGHT = {0: 1e-3, 1: 3e-2}
+# key 2: FP8 weights with one e4m3 term per expert activation (W8A8): each
+# activation carries one e4m3 rounding (relative <= 2^-4, rms 2^-4 / sqrt(3)
+# for a uniform rounding error) at each of the two expert matrices, so the
+# output's error is bounded in rms, not elementwise: rms(gpu - oracle) <= 2^-4
+# rms(oracle) (sqrt(2) x 2^-4 / sqrt(3) ~ 0.051 for two independent stages),
+# and its largest element within 8 such rms (a sanity bound).
+TOL = {0: 1e-2, 1: 3e-2, 2: 2.0 ** -4}
+TIGHT = {0: 1e-3, 1: 3e-2, 2: 2.0 ** -4}
 TIE_GAP = 1e-4
 
 
@@ -73,6 +79,14 @@ def check_output(report: dict, key: str, gpu: np.ndarray, ref: np.ndarray, wdtyp
     strict_raw: assert the literal raw bound (None: wherever the correctly
     rounded result meets it)."""
     tol = TOL[wdtype]
+    if wdtype == 2:   # W8A8: the rms bound (see TOL)
+        err = gpu.astype(np.float64) - ref
+        rms = float(np.sqrt(np.mean(ref.astype(np.float64) ** 2)))
+        report[key + "_rms"] = float(np.sqrt(np.mean(err ** 2))) / rms
+        report[key + "_raw"] = rel_err(gpu, ref)
+        assert report[key + "_rms"] <= tol, (key, report)
+        assert report[key + "_raw"] <= 8 * tol, (key, report)
+        return
     raw = rel_err(gpu, ref)
     ex = rel_err_bf16(gpu, ref)
     report[key + "_raw"] = raw
@@ -160,7 +174,7 @@ def selection_check(gpu_idx: np.ndarray, ref_logits: np.ndarray, ref_idx: np.nda
 
 def compare_layer(dims, gpu: dict, x_bits, a_bits, *, wdtype=0, layer_id=0, seed=0, bias=None,
                   rows=None, check_qkv=True, strict_raw=None, bias_select_only=False,
-                  routed_scale=1.0) -> dict:
+                  routed_scale=1.0, tol_key=None) -> dict:
     """Compare one GPU layer call with the oracle (all rows, or the listed rows,
     each recomputed on its own -- rows are independent)."""
     x = bf16_to_f64(x_bits)
@@ -192,7 +206,8 @@ def compare_layer(dims, gpu: dict, x_bits, a_bits, *, wdtype=0, layer_id=0, seed
         report["logits"] = rel_err(g["logits"], ref["logits"])
         assert report["h1"] < 1e-4, report
         assert report["logits"] < 1e-3, report
-    check_output(report, "out", bf16_to_f64(g["out"]), ref["out"], wdtype, strict_raw)
-    if check_qkv:
+    tk = wdtype if tol_key is None else tol_key
+    check_output(report, "out", bf16_to_f64(g["out"]), ref["out"], tk, strict_raw)
+    if check_qkv:   # (the projections are the same for W8A8)
         check_output(report, "qkv", bf16_to_f64(g["qkv"]), ref["qkv"], wdtype, strict_raw)
     return report

@@ -133,6 +133,25 @@ def test_gating_variants(kd, wdtype, M):
             L.close()
 
 
+@pytest.mark.parametrize("dims,M,rows", [(TINY, 8, None), (K2, 32, [0, 7, 19, 31])])
+def test_w8a8_experts(kd, dims, M, rows):
+    """FP8 expert weights with one e4m3 term per activation (W8A8) on the
+    tensor cores: the output's rms error within one e4m3 rounding (2^-4) of
+    its rms; the same selection; the projections as with two terms."""
+    spec = kd.LayerSpec.from_dims(dims, wdtype=1, max_tokens=M, fp8_act_terms=1)
+    L = kd.Layer(spec, seed=0)
+    try:
+        x, a = inputs(dims, M, rho=0.3)
+        g = run_gpu_layer(L, x, a)
+        r = compare_layer(dims, g, x, a, wdtype=1, rows=rows, tol_key=2)
+        print("w8a8", dims.hidden, M, r)
+    finally:
+        L.close()
+    with pytest.raises(kd.KdError) as e:
+        kd.Layer(kd.LayerSpec.from_dims(TINY, wdtype=1, max_tokens=4, fp8_act_terms=3))
+    assert e.value.code == kd.KD_EINVAL
+
+
 def test_determinism_and_in_place(kd):
     import torch
     d = TINY
