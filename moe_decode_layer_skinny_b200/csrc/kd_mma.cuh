@@ -143,6 +143,11 @@ constexpr size_t kMmaSmem = (size_t)kMRingBytes + 1024 /*align*/ + 3840 /*barrie
 static_assert(kMmaSmem + 64 <= 227 * 1024, "shared memory per CTA (with the kernels' static bytes)");
 constexpr int kQ8AccCols = 256;                       // q8: one accumulator, <= 2 x 2 x 64 columns
 constexpr int kQ8TmemCols = 2 * kQ8AccCols;           // q8: two accumulators
+// bf16 plans: one accumulator holds every B term's columns side by side
+// (term h of token j in column h N + j, N = pad16(ntok)), <= 3 x 64 columns;
+// two buffers kBfAccCols apart in the 512 columns the CTA allocates
+constexpr int kBfAccCols = 256;
+static_assert(kMaxTerms * kMaxN <= kBfAccCols, "bf16 accumulators");
 constexpr int kQGroup = 64;                           // activation elements per stored maximum
 constexpr int kQTerms = 2;                            // e4m3 terms of a q8 activation (at most;
                                                       // a plan's kQT: 2, or 1 for W8A8)
@@ -625,8 +630,11 @@ KD_DEV void mma_issuer(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigned*
   for (; units.next(m); ++nu_local) {
     const int N = pad16(m.ntok);
     const uint32_t idesc = idesc_bf16(N);
+    // bf16 weights: one MMA per K-step for all terms (their B rows lie one
+    // after another: N' = nterms N columns, summed by the epilogue)
+    const uint32_t idesc_all = idesc_bf16(nterms * N);
     const int buf = nu_local & 1;
-    const uint32_t d = tmem + (uint32_t)(buf * kMaxN);
+    const uint32_t d = tmem + (uint32_t)(buf * kBfAccCols);
     if (!mwait(&sh.accempty[buf], ((nu_local >> 1) & 1u) ^ 1u, sh.abort_flag, err)) break;
     tc_fence_after();
     bool ok = true;
@@ -651,13 +659,9 @@ KD_DEV void mma_issuer(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigned*
         for (int u = 0; u < sh.nsub; ++u) {
           const uint32_t b = b0 + u * bsub;
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint64_t ad = sw128_desc(a0 + u * kATileBytes + k * 32);
-            mma_bf16(d, ad, sw128_desc(b + k * 32), idesc, c > 0 || u > 0 || k > 0);
-#pragma unroll
-            for (int h = 1; h < nterms; ++h)
-              mma_bf16(d, ad, sw128_desc(b + h * N * 128 + k * 32), idesc, true);
-          }
+          for (int k = 0; k < 4; ++k)
+            mma_bf16(d, sw128_desc(a0 + u * kATileBytes + k * 32), sw128_desc(b + k * 32), idesc_all,
+                     c > 0 || u > 0 || k > 0);
         }
       } else {
       // FP8: descriptors by adding byte offsets / 16 to the start-address
@@ -998,7 +1002,23 @@ KD_DEV void mma_epilogue(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigne
     const int buf = nu_local & 1;
     mwait_lazy(&sh.accfull[buf], (nu_local >> 1) & 1u, sh.abort_flag, err);
     tc_fence_after();
-    const uint32_t ta = tmem + ((uint32_t)(ew * 32) << 16) + (uint32_t)(buf * kMaxN);
+    const uint32_t ta = tmem + ((uint32_t)(ew * 32) << 16) + (uint32_t)(buf * kBfAccCols);
+    // 16 tokens of the accumulator: the sum of the terms' column blocks
+    // (bf16 weights; the FP8 projections accumulate their terms in the MMAs)
+    auto acc16 = [&](int c, float* v) {
+      constexpr int NT = Plan::kFp8 ? 1 : Plan::kTerms;
+      float t[NT][16];
+#pragma unroll
+      for (int h = 0; h < NT; ++h) tmem_ld16(ta + (uint32_t)(h * N + c), t[h]);
+      tmem_wait_ld();
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        float a = t[0][j];
+#pragma unroll
+        for (int h = 1; h < NT; ++h) a += t[h][j];
+        v[j] = a;
+      }
+    };
     bool complete = true;
     int first = 0;
     if (m.nparts > 1) {
@@ -1010,8 +1030,7 @@ KD_DEV void mma_epilogue(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigne
 #pragma unroll 1
       for (int c = 0; c < N; c += 16) {
         float v[16];
-        tmem_ld16(ta + c, v);
-        tmem_wait_ld();
+        acc16(c, v);
 #pragma unroll
         for (int j = 0; j < 16; ++j)
           if (c + j < m.ntok) __stcg(ws + (c + j) * 128, v[j]);
@@ -1056,8 +1075,7 @@ KD_DEV void mma_epilogue(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigne
               }
           }
         } else {
-          tmem_ld16(ta + c, v);
-          tmem_wait_ld();
+          acc16(c, v);
         }
         emit16(plan, m, row, lane, c, v, sh);
       }
@@ -1234,7 +1252,7 @@ KD_DEV void mma_run(const Plan& plan, uint8_t* smem_raw, unsigned* err) {
     sh.misc[2] = 0;
     fence_mbar_init();
   }
-  constexpr uint32_t kCols = Plan::kQ8 ? (uint32_t)kQ8TmemCols : (uint32_t)(2 * kMaxN);
+  constexpr uint32_t kCols = Plan::kQ8 ? (uint32_t)kQ8TmemCols : (uint32_t)(2 * kBfAccCols);
   static_assert(!Plan::kQ8 || Plan::kVariants * kQTerms * kMaxN <= kQ8AccCols, "q8 accumulators");
   if (warp == 1) tmem_alloc(sh.tmem_base, kCols);
   tc_fence_before();
