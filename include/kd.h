@@ -71,8 +71,8 @@ typedef struct kd_config {
   int max_tokens;    /* largest M a call may use, 1..64; sizes the workspaces    */
   const float* router_bias; /* host [E] additive router bias, or NULL; copied    */
   int mma_min_tokens;/* calls with M >= this use the tensor-core (tcgen05) kernels,
-                        smaller M the CUDA-core streaming kernels; 0 = default (3),
-                        > 64 = never.                                           */
+                        smaller M the CUDA-core streaming kernels; 0 = default (1:
+                        the tensor cores for every M), > 64 = never.            */
   /* Full layer (kd_decode_layer_full); all zero for the layer above.         */
   int full_layer;    /* 1: RMSNorm gains are generated and the layer takes the
                         full-layer call; 0: kd_decode_layer only                */

@@ -301,7 +301,7 @@ extern "C" int kd_layer_create(const kd_config* cfg, uint64_t seed, kd_layer** o
   L->w8a8 = c.fp8_act_terms == 1;
   L->cfg.router_bias = nullptr;
   L->maxM = c.max_tokens;
-  L->mma_min = c.mma_min_tokens > 0 ? c.mma_min_tokens : 3;
+  L->mma_min = c.mma_min_tokens > 0 ? c.mma_min_tokens : 1;
   // tensor-parallel shard: its q heads [q0, q1), the kv heads they read
   // [k0, k1), router rows [e0, e0 + Er), expert rows [i0, i0 + Ir)
   const int q0 = c.q_heads * tr / R, q1 = c.q_heads * (tr + 1) / R;

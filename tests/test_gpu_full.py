@@ -40,11 +40,11 @@ def kv_scales(dims):
     return float(np.float32(4 * sigma / 448)), float(np.float32(4 * sigma / 448)), sigma
 
 
-def make_full(kd, dims, n_seq, max_ctx, wdtype=0, max_tokens=8, layer_id=0):
+def make_full(kd, dims, n_seq, max_ctx, wdtype=0, max_tokens=8, layer_id=0, mma_min=0):
     ks, vs, _ = kv_scales(dims)
     spec = kd.LayerSpec.from_dims(dims, wdtype=wdtype, layer_id=layer_id, max_tokens=max_tokens,
                                   full_layer=1, kv_n_seq=n_seq, kv_max_ctx=max_ctx, k_scale=ks,
-                                  v_scale=vs)
+                                  v_scale=vs, mma_min_tokens=mma_min)
     return kd.Layer(spec, seed=0)
 
 
@@ -156,10 +156,10 @@ LAYOUTS = {
 @pytest.mark.parametrize("layout", ["ragged", "verify"])
 def test_full_tiny(kd, wdtype, M, layout):
     """Tiny dims (2 kv heads of 2 query heads, head_dim 64), a 300-position
-    cache (ten attention chunks), both engines (M < 3 CUDA cores, M >= 3
-    tensor cores)."""
+    cache (ten attention chunks), both engines (the CUDA-core kernels for
+    M = 1 and 3, the tensor cores for 5 and 8)."""
     n_seq, ctx = 3, 300
-    L = make_full(kd, TINYF, n_seq, ctx, wdtype=wdtype)
+    L = make_full(kd, TINYF, n_seq, ctx, wdtype=wdtype, mma_min=4)
     try:
         x = kdgen.activations(0, 0, kdgen.HIDDEN_IN, M, TINYF.hidden, 0.3)
         kc0, vc0 = cache_inputs(TINYF, n_seq, ctx)

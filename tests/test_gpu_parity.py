@@ -32,9 +32,14 @@ def kd(torch_cuda):
     return kd
 
 
-def make_layer(kd, dims, wdtype=0, layer_id=0, bias=None, max_tokens=64, seed=0):
+# engines: "tensor" = the default (tcgen05 kernels for every M), "cores" =
+# the CUDA-core streaming kernels (mma_min_tokens beyond any M)
+ENGINE_MMA_MIN = {"tensor": 0, "cores": 1000}
+
+
+def make_layer(kd, dims, wdtype=0, layer_id=0, bias=None, max_tokens=64, seed=0, engine="tensor"):
     spec = kd.LayerSpec.from_dims(dims, wdtype=wdtype, layer_id=layer_id, max_tokens=max_tokens,
-                                  router_bias=bias)
+                                  router_bias=bias, mma_min_tokens=ENGINE_MMA_MIN[engine])
     return kd.Layer(spec, seed=seed)
 
 
@@ -84,10 +89,12 @@ def test_device_weights_match_generator_k2_sampled(kd):
 # ---------------------------------------------------------------- tiny layer
 
 @pytest.mark.parametrize("wdtype", [0, 1])
-@pytest.mark.parametrize("M", [1, 2, 3, 5, 8, 13, 32, 64])
-def test_tiny_layer_parity(kd, wdtype, M):
+@pytest.mark.parametrize("M,engine", [(1, "tensor"), (2, "tensor"), (3, "tensor"), (5, "tensor"),
+                                      (8, "tensor"), (13, "tensor"), (32, "tensor"), (64, "tensor"),
+                                      (1, "cores"), (2, "cores"), (3, "cores"), (5, "cores")])
+def test_tiny_layer_parity(kd, wdtype, M, engine):
     d = TINY
-    L = make_layer(kd, d, wdtype=wdtype)
+    L = make_layer(kd, d, wdtype=wdtype, engine=engine)
     try:
         x, a = inputs(d, M, rho=0.5)
         g = run_gpu_layer(L, x, a)
@@ -114,15 +121,16 @@ def test_tiny_variants(kd):
 
 
 @pytest.mark.parametrize("wdtype", [0, 1])
-@pytest.mark.parametrize("M", [3, 8])
-def test_gating_variants(kd, wdtype, M):
+@pytest.mark.parametrize("M,engine", [(3, "cores"), (8, "tensor"), (2, "tensor")])
+def test_gating_variants(kd, wdtype, M, engine):
     """Selection-only router bias (the gates from the unbiased logits) and a
-    routed scaling factor, on both engines (M=3 CUDA cores, M=8 tensor cores)."""
+    routed scaling factor, on both engines."""
     d = TINY
     bias = kdgen.zipf_bias(d.n_experts, 1.1)
     for sel, rs in [(1, 1.0), (0, 2.5), (1, 0.75)]:
         spec = kd.LayerSpec.from_dims(d, wdtype=wdtype, max_tokens=8, router_bias=bias,
-                                      bias_select_only=sel, routed_scale=rs)
+                                      bias_select_only=sel, routed_scale=rs,
+                                      mma_min_tokens=ENGINE_MMA_MIN[engine])
         L = kd.Layer(spec, seed=0)
         try:
             x, a = inputs(d, M, rho=0.3)
@@ -216,6 +224,24 @@ def test_batch1_layer_parity(kd, k2_layer):
     print("batch1", r)
 
 
+def test_k2_cuda_core_engine(kd):
+    """The CUDA-core streaming kernels (mma_min_tokens beyond any M) on the
+    H=7168 layer: batch 1, and two tokens; every row against the oracle."""
+    L = make_layer(kd, K2, max_tokens=2, engine="cores")
+    try:
+        w = WORKLOADS["batch1"]
+        x, a = w.hidden_in(), w.attn_out()
+        g = run_gpu_layer(L, x, a)
+        r = compare_layer(K2, g, x, a, strict_raw=True)   # floor 0.0099 at this input
+        assert g["n_active"] == 8
+        print("batch1 cores", r)
+        x, a = inputs(K2, 2, seed=3)
+        g = run_gpu_layer(L, x, a)
+        print("M=2 cores", compare_layer(K2, g, x, a))
+    finally:
+        L.close()
+
+
 def test_verify8_layer_parity(kd, k2_layer):
     w = WORKLOADS["verify8"]
     x, a = w.hidden_in(), w.attn_out()
@@ -227,9 +253,8 @@ def test_verify8_layer_parity(kd, k2_layer):
 
 @pytest.mark.parametrize("M", [2, 3, 4, 5, 6, 7, 16])
 def test_k2_other_token_counts(kd, k2_layer, M):
-    """All rows at M = 2 (CUDA-core engine), 3 (the switch to the tensor
-    cores), 4..7 (speculative verify with 3..6 draft tokens + 1, correlated
-    rows) and 16."""
+    """All rows at M = 2, 3, 4..7 (speculative verify with 3..6 draft tokens
+    + 1, correlated rows) and 16."""
     x, a = inputs(K2, M, seed=3, rho=0.9 if 4 <= M <= 7 else 0.0)
     g = run_gpu_layer(k2_layer, x, a)
     r = compare_layer(K2, g, x, a, check_qkv=True)

@@ -73,12 +73,14 @@ def _qkv_of(kd, dims, layers, M):
     return full
 
 
-@pytest.mark.parametrize("R,M,wdtype", [(2, 1, 0), (4, 1, 0), (2, 2, 0), (2, 8, 0), (4, 8, 0),
-                                        (4, 16, 0)])
-def test_tp_small(kd, R, M, wdtype):
+# mma_min: 0 = the tensor-core kernels, 1000 = the CUDA-core kernels
+@pytest.mark.parametrize("R,M,mma_min", [(2, 1, 1000), (4, 1, 1000), (2, 2, 1000), (2, 1, 0),
+                                         (2, 8, 0), (4, 8, 0), (4, 16, 0)])
+def test_tp_small(kd, R, M, mma_min):
+    wdtype = 0
     x = kdgen.activations(0, 0, kdgen.HIDDEN_IN, M, SMALL.hidden)
     a = kdgen.activations(0, 0, kdgen.ATTN_OUT, M, SMALL.attn)
-    layers = _shards(kd, SMALL, R, M, wdtype=wdtype)
+    layers = _shards(kd, SMALL, R, M, wdtype=wdtype, mma_min_tokens=mma_min)
     try:
         out, logits, _ = run_tp(kd, layers, x, a)
         # every rank ends with the same hidden state
@@ -122,9 +124,9 @@ def test_tp_fp8(kd, M):
 
 
 def test_tp_k2(kd):
-    """Full-size shards (H=7168, 256 experts, I=2048) over 2 ranks at M=1
-    (CUDA-core kernels) and M=8 (tensor cores): the same selection as the
-    unsharded GPU layer, and every output row and QKV row against the oracle."""
+    """Full-size shards (H=7168, 256 experts, I=2048) over 2 ranks at M=1 and
+    M=8: the same selection as the unsharded GPU layer, and every output row
+    and QKV row against the oracle."""
     K2 = kdgen.K2
     for M in (1, 8):
         x = kdgen.activations(0, 0, kdgen.HIDDEN_IN, M, K2.hidden)
