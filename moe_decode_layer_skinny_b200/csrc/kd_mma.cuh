@@ -624,7 +624,10 @@ KD_DEV void drain_mma(MmaShared& sh) {
 template <class Plan>
 KD_DEV void mma_issuer(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigned* err) {
   constexpr int nterms = Plan::kTerms;
-  uint32_t it = 0, nu_local = 0;
+  uint32_t nu_local = 0;
+  int s = 0, sb = 0;            // stage and B slot of the stage counter
+  uint32_t ph = 0, bph = 0;     // and their phases (counters, no divisions)
+  const uint32_t ring0 = smem_u32(sh.stage), bring0 = smem_u32(sh.bst) + sh.boff;
   CtaUnits<Plan> units(plan);
   MUnit m;
   for (; units.next(m); ++nu_local) {
@@ -638,13 +641,10 @@ KD_DEV void mma_issuer(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigned*
     if (!mwait(&sh.accempty[buf], ((nu_local >> 1) & 1u) ^ 1u, sh.abort_flag, err)) break;
     tc_fence_after();
     bool ok = true;
-    for (int c = 0; c < m.nkc; ++c, ++it) {
-      const int s = it % sh.nst;
-      const uint32_t ph = (it / sh.nst) & 1u;
-      const int sb = it % sh.nbst;
+    for (int c = 0; c < m.nkc; ++c) {
       if (Plan::kFp8) {
         ok = mwait(&sh.full[s], ph, sh.abort_flag, err) &&
-             mwait(&sh.bfull[sb], (it / sh.nbst) & 1u, sh.abort_flag, err);
+             mwait(&sh.bfull[sb], bph, sh.abort_flag, err);
       } else {
         ok = mwait(&sh.afull[s], ph, sh.abort_flag, err) &&
              mwait(&sh.full[s], ph, sh.abort_flag, err);
@@ -652,8 +652,8 @@ KD_DEV void mma_issuer(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigned*
       if (!ok) break;
       fence_proxy_async_smem();   // the B gathers (generic proxy) -> tensor core reads
       tc_fence_after();
-      const uint32_t a0 = smem_u32(sh.stage + (size_t)s * sh.stage_bytes);
-      const uint32_t b0 = smem_u32(sh.bst + (size_t)sb * sh.bst_bytes) + sh.boff;
+      const uint32_t a0 = ring0 + (uint32_t)(s * sh.stage_bytes);
+      const uint32_t b0 = bring0 + (uint32_t)(sb * sh.bst_bytes);
       const int bsub = b_sub_bytes(N, nterms);
       if constexpr (!Plan::kFp8) {
         for (int u = 0; u < sh.nsub; ++u) {
@@ -685,6 +685,8 @@ KD_DEV void mma_issuer(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigned*
       }
       mma_commit(&sh.empty[s]);   // the stage is free once these MMAs are done
       if (Plan::kFp8) mma_commit(&sh.bempty[sb]);
+      if (++s == sh.nst) { s = 0; ph ^= 1u; }
+      if (++sb == sh.nbst) { sb = 0; bph ^= 1u; }
     }
     if (!ok) break;
     mma_commit(&sh.accfull[buf]);
