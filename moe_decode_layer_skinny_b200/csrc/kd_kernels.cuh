@@ -243,8 +243,8 @@ __global__ void __launch_bounds__(kThreads, 1) proj_kernel(LayerDev L, Acts a) {
 // Each lane loads its weight chunks (16 bytes each, up to 8) before waiting
 // for h1 (the router weights are static), then forms partial dot products
 // with the h1 rows of 4 tokens at a time; the four quarters are added in a
-// fixed order.  The selection itself (route_tokens) runs at the start of the
-// routed-expert kernel.
+// fixed order.  The CTA that finishes last then runs the selection
+// (route_tokens) for every token.
 constexpr int kRouterThreads = 256;
 constexpr int kRouterRows = 2;
 constexpr int kCoreRouterMaxM = 8;   // bf16 layers: the CUDA-core router up to this many tokens
@@ -285,9 +285,9 @@ KD_DEV void router_chunk(const uint4 wv, float scale, const float* const* arow, 
 
 // ------------------------------------------------------------------ selection + dispatch
 
-// Routing of the call in shared memory, built by every routed-expert CTA from
-// the logits (redundantly: no grid-wide serialisation); CTA 0 also writes it
-// to global memory for the down kernel and for inspection.
+// Routing of the call in shared memory, built by the router's last CTA from
+// the logits (and written to global memory for the expert kernels); the
+// CUDA-core gate/up kernel copies it back into shared memory.
 struct Route {
   int* sel;      // [M*k] selected expert of (token, slot), descending logit
   float* gv;     // [M*k] its logit
@@ -297,10 +297,20 @@ struct Route {
   int* perm;     // [M*k] token*k + slot, sorted by (expert, token*k + slot)
   int* n_act;    // [1]
   int* wsum;     // [2][32] scan scratch
+  int* wc;       // [kWalkWarps][E] the selection's per-warp expert counts (selection only)
 };
 
+// Warps that place the codes into the per-expert lists (contiguous ranges of
+// codes, one per warp).
+constexpr int kWalkWarps = 8;
+
+// Ints of a Route in shared memory; the selection (route_tokens) also needs
+// its per-warp counts after it.
 __host__ __device__ constexpr size_t kRouteSmemInts(int E, int Mk) {
   return (size_t)3 * E + 3 * Mk + 1 + 64;
+}
+__host__ __device__ constexpr size_t kSelectSmemInts(int E, int Mk) {
+  return kRouteSmemInts(E, Mk) + (size_t)kWalkWarps * E;
 }
 
 KD_DEV Route carve_route(int* base, int E, int Mk) {
@@ -313,102 +323,102 @@ KD_DEV Route carve_route(int* base, int E, int Mk) {
   r.act = r.off + E;
   r.n_act = r.act + E;
   r.wsum = r.n_act + 1;
+  r.wc = r.wsum + 64;
   return r;
 }
 
-// Selection keys: larger key = larger logit, ties -> lower expert id.  The
-// logit's bits are mapped to an unsigned order (sign flipped for positive
-// values, all bits for negative ones) and the expert id complemented below.
-KD_DEV uint64_t route_key(float v, int e) {
+// A logit's bits as an unsigned order (sign flipped for positive values, all
+// bits for negative ones; -0 ranks with +0) and back.
+KD_DEV uint32_t order_bits(float v) {
   uint32_t u = __float_as_uint(v);
-  if ((u << 1) == 0u) u = 0u;   // -0 ranks with +0 (then the lower id wins)
-  u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-  return ((uint64_t)u << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)e);
+  if ((u << 1) == 0u) u = 0u;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
-KD_DEV float key_value(uint64_t key) {
-  uint32_t u = (uint32_t)(key >> 32);
-  u = (u & 0x80000000u) ? (u & 0x7FFFFFFFu) : ~u;
-  return __uint_as_float(u);
+KD_DEV float order_value(uint32_t u) {
+  return __uint_as_float((u & 0x80000000u) ? (u & 0x7FFFFFFFu) : ~u);
 }
-KD_DEV int key_expert(uint64_t key) { return (int)(0xFFFFFFFFu - (uint32_t)key); }
 
-// Top-k of token t by a group of LPT lanes of a warp (32 / LPT tokens per
-// warp at once): lane l of the group holds the keys of experts l, l + LPT,
-// ... (PER of them, PER * LPT >= E).  k rounds, each: the lane's largest
-// remaining key, the group's largest by a shuffle reduction, and the owner
-// drops it.  Loops that run more than once are rolled, so the code stays
-// small for the instruction cache.  Then the softmax renormalised over the k
-// selected logits (same order and arithmetic in every lane of the group).
-// Groups whose token is past M run on empty keys and write nothing.
-template <int PER, int LPT>
-KD_DEV void topk_group(const LayerDev& L, const float* lg, const Route& R, int t, int M,
-                       bool write_global) {
-  const int sl = threadIdx.x & (LPT - 1);
+// Top-k of token t by one warp: lane l holds the logits of experts l, l + 32,
+// ... (PER of them, PER * 32 >= E) and their selection keys (order bits of
+// the logit, plus the bias when it only steers the selection).  A selection
+// key ranks by value, then by lower expert id.  Each lane keeps its best
+// remaining candidate; a round takes the warp's best with two warp
+// reductions (redux.sync max: the order bits, then among the lanes holding
+// that value the complemented expert id), and the lane that held it drops it
+// and finds its next best.  Then the softmax renormalised over the k
+// selected logits, in the same order and arithmetic in every lane.
+template <int PER>
+KD_DEV void topk_warp(const LayerDev& L, const float* lg, const Route& R, int t,
+                      bool write_global) {
+  const int lane = threadIdx.x & 31;
   const int k = L.k, E = L.E;
-  const bool act = t < M;
-  uint64_t key[PER];
-  // selection keys: the logits, or with a selection-only bias logits + bias
-  // (the logits buffer then holds the unbiased logits, which the gates use)
+  // with a selection-only bias the logits buffer holds the unbiased logits,
+  // which the gates use
   const bool sel_bias = L.bias_sel && L.bias;
+  float raw[PER];
+  uint32_t hk[PER];
+  unsigned live = 0;   // bit qq: expert lane + 32 qq is still a candidate
 #pragma unroll
   for (int qq = 0; qq < PER; ++qq) {
-    const int e = sl + LPT * qq;
-    float v = 0.f;
-    if (act && e < E) {
-      v = lg[(size_t)t * E + e];
-      if (sel_bias) v += __ldg(L.bias + e);
-    }
-    key[qq] = (act && e < E) ? route_key(v, e) : 0ull;
+    const int e = lane + 32 * qq;
+    raw[qq] = e < E ? lg[(size_t)t * E + e] : 0.f;
   }
+#pragma unroll
+  for (int qq = 0; qq < PER; ++qq) {
+    const int e = lane + 32 * qq;
+    hk[qq] = order_bits(raw[qq] + (sel_bias && e < E ? __ldg(L.bias + e) : 0.f));
+    if (e < E) live |= 1u << qq;
+  }
+  uint32_t bh = 0;   // this lane's best remaining key: order bits and slot
+  int bq = -1;
+  auto lane_best = [&]() {
+    bh = 0;
+    bq = -1;
+#pragma unroll
+    for (int qq = 0; qq < PER; ++qq)
+      if (((live >> qq) & 1u) && (bq < 0 || hk[qq] > bh)) { bh = hk[qq]; bq = qq; }
+  };
+  lane_best();
   float top = 0.f, den = 0.f;
 #pragma unroll 1
   for (int j = 0; j < k; ++j) {
-    uint64_t best = key[0];
+    const uint32_t lo = bq >= 0 ? ~(uint32_t)(lane + 32 * bq) : 0u;
+    const uint32_t bhi = __reduce_max_sync(0xffffffffu, bh);
+    const uint32_t blo = __reduce_max_sync(0xffffffffu, bh == bhi ? lo : 0u);
+    const int be = (int)~blo;
+    float w = 0.f;   // the winner's unbiased logit, in the lane that held it
+    if (lane == (be & 31)) {
 #pragma unroll
-    for (int qq = 1; qq < PER; ++qq) best = key[qq] > best ? key[qq] : best;
-#pragma unroll 1
-    for (int o = LPT / 2; o > 0; o >>= 1) {
-      const uint64_t other = __shfl_xor_sync(0xffffffffu, best, o);
-      best = other > best ? other : best;
+      for (int qq = 0; qq < PER; ++qq)
+        if (qq == bq) w = raw[qq];
+      live &= ~(1u << bq);
+      lane_best();
     }
-#pragma unroll
-    for (int qq = 0; qq < PER; ++qq)
-      if (key[qq] == best) key[qq] = 0ull;   // keys are unique (expert id)
-    const int be = key_expert(best);
-    const float v = sel_bias ? (act ? lg[(size_t)t * E + be] : 0.f) : key_value(best);
+    const float v = sel_bias ? __shfl_sync(0xffffffffu, w, be & 31) : order_value(bhi);
     if (j == 0 || v > top) {   // the gates' reference value: their largest logit
       den = j == 0 ? 0.f : den * expf(top - v);
       top = v;
     }
     den += expf(v - top);
-    if (act && sl == 0) {
-      const int e = be;
-      R.sel[t * k + j] = e;
+    if (lane == 0) {
+      R.sel[t * k + j] = be;
       R.gv[t * k + j] = v;
-      if (write_global) L.idx[t * k + j] = e;
     }
   }
   __syncwarp();
-  if (act && write_global)
-    for (int j = sl; j < k; j += LPT) L.gates[t * k + j] = expf(R.gv[t * k + j] - top) / den;
+  if (write_global)
+    for (int j = lane; j < k; j += 32) {
+      L.idx[t * k + j] = R.sel[t * k + j];
+      L.gates[t * k + j] = expf(R.gv[t * k + j] - top) / den;
+    }
 }
 
-template <int LPT>
+// Every token's top-k, one token per warp at a time.
+template <int PER>
 KD_DEV void topk_tokens(const LayerDev& L, const float* lg, const Route& R, int M,
                         bool write_global) {
-  constexpr int TPW = 32 / LPT;
-  const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  const int g = (threadIdx.x & 31) / LPT;
-  const int per = (L.E + LPT - 1) / LPT;   // <= 32
-  for (int t0 = warp * TPW; t0 < M; t0 += nw * TPW) {
-    const int t = t0 + g;
-    if (per <= 1) topk_group<1, LPT>(L, lg, R, t, M, write_global);
-    else if (per <= 2) topk_group<2, LPT>(L, lg, R, t, M, write_global);
-    else if (per <= 4) topk_group<4, LPT>(L, lg, R, t, M, write_global);
-    else if (per <= 8) topk_group<8, LPT>(L, lg, R, t, M, write_global);
-    else if (per <= 16) topk_group<16, LPT>(L, lg, R, t, M, write_global);
-    else topk_group<32, LPT>(L, lg, R, t, M, write_global);
-  }
+  for (int t = threadIdx.x >> 5; t < M; t += blockDim.x >> 5)
+    topk_warp<PER>(L, lg, R, t, write_global);
 }
 
 // Top-k of every token, the renormalised softmax over each selection, and the
@@ -417,24 +427,46 @@ KD_DEV void topk_tokens(const LayerDev& L, const float* lg, const Route& R, int 
 KD_DEV void route_tokens(const LayerDev& L, const float* lg, int M, const Route& R,
                          bool write_global) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nw = blockDim.x >> 5;
   const int k = L.k, E = L.E;
-  // lanes per token: fewer (more tokens per warp at once) when each warp has
-  // several tokens, but at least E / 32 so that a lane holds <= 32 keys
-  const int tpw = (M + nw - 1) / nw;
-  int lpt = tpw >= 4 ? 8 : tpw >= 2 ? 16 : 32;
-  if (E > 32 * lpt) lpt = E > 512 ? 32 : 16;
-  if (lpt == 8) topk_tokens<8>(L, lg, R, M, write_global);
-  else if (lpt == 16) topk_tokens<16>(L, lg, R, M, write_global);
+  // keys per lane: the smallest of 4, 8, 16, 32 that covers E (E <= 1024)
+  if (E <= 128) topk_tokens<4>(L, lg, R, M, write_global);
+  else if (E <= 256) topk_tokens<8>(L, lg, R, M, write_global);
+  else if (E <= 512) topk_tokens<16>(L, lg, R, M, write_global);
   else topk_tokens<32>(L, lg, R, M, write_global);
   __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x) R.cnt[e] = 0;
-  __syncthreads();
+  // The codes (token * k + slot) in nwalk contiguous ranges of whole 32-code
+  // steps, one per warp.  A step ranks the codes of equal experts with a
+  // match; its lowest lane per expert does the bookkeeping.
   const int ncode = M * k;
-  for (int c = threadIdx.x; c < ncode; c += blockDim.x) {
-    const int e = R.sel[c];
-    if (e < 0 || e >= E) set_error(L.err, ERR_BAD_ROUTE);
-    else atomicAdd(&R.cnt[e], 1);
+  const int nwalk = min(kWalkWarps, (int)(blockDim.x >> 5));
+  const int span = ((ncode + nwalk - 1) / nwalk + 31) & ~31;
+  for (int i = threadIdx.x; i < nwalk * E; i += blockDim.x) R.wc[i] = 0;
+  __syncthreads();
+  // each warp counts its range's codes per expert
+  if (warp < nwalk) {
+    int* wc = R.wc + warp * E;
+    const int c1 = min(ncode, (warp + 1) * span);
+    for (int c0 = warp * span; c0 < c1; c0 += 32) {
+      const int c = c0 + lane;
+      const int se = c < c1 ? R.sel[c] : 0;
+      const bool live = c < c1 && se >= 0 && se < E;
+      if (c < c1 && !live) set_error(L.err, ERR_BAD_ROUTE);
+      const int e = live ? se : -1 - lane;   // unique dummies
+      const unsigned same = __match_any_sync(0xffffffffu, e);
+      if (live && (same & ((1u << lane) - 1u)) == 0) wc[e] += __popc(same);
+      __syncwarp();
+    }
+  }
+  __syncthreads();
+  // per expert: its count, and each warp's first place among its codes
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = 0;
+    for (int w = 0; w < nwalk; ++w) {
+      const int n = R.wc[w * E + e];
+      R.wc[w * E + e] = run;
+      run += n;
+    }
+    R.cnt[e] = run;
   }
   __syncthreads();
   // block-wide exclusive scans of cnt and of (cnt > 0): each thread owns
@@ -484,26 +516,27 @@ KD_DEV void route_tokens(const LayerDev& L, const float* lg, int M, const Route&
     }
   }
   __syncthreads();
-  // positions in (expert, code) order: one warp walks the codes 32 at a time
-  if (warp == 0) {
-    for (int c0 = 0; c0 < ncode; c0 += 32) {
+  // positions in (expert, code) order: each warp places its range's codes
+  if (warp < nwalk) {
+    int* wc = R.wc + warp * E;
+    const int c1 = min(ncode, (warp + 1) * span);
+    for (int c0 = warp * span; c0 < c1; c0 += 32) {
       const int c = c0 + lane;
-      const int e = c < ncode ? R.sel[c] : -1 - lane;  // unique dummies
+      const int se = c < c1 ? R.sel[c] : 0;
+      const bool live = c < c1 && se >= 0 && se < E;
+      const int e = live ? se : -1 - lane;
       const unsigned same = __match_any_sync(0xffffffffu, e);
       const int rank = __popc(same & ((1u << lane) - 1u));
-      const int base = (c < ncode && e >= 0 && e < E) ? R.off[e] : 0;
-      __syncwarp();
-      if (c < ncode && e >= 0 && e < E) {
-        R.perm[base + rank] = c;
-        if (write_global) L.perm[base + rank] = c;
-        if (rank == 0) R.off[e] = base + __popc(same);
+      if (live) {
+        const int pos = R.off[e] + wc[e] + rank;
+        R.perm[pos] = c;
+        if (write_global) L.perm[pos] = c;
       }
+      __syncwarp();
+      if (live && rank == 0) wc[e] += __popc(same);
       __syncwarp();
     }
   }
-  __syncthreads();
-  // restore the exclusive offsets (the walk advanced them to the ends)
-  for (int e = threadIdx.x; e < E; e += blockDim.x) R.off[e] -= R.cnt[e];
   __syncthreads();
 }
 

@@ -220,7 +220,7 @@ static int configure_kernels() {
   KD_CUDA(cudaFuncSetAttribute(gateup_kernel<W_FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   KD_CUDA(cudaFuncSetAttribute(down_kernel<W_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
   KD_CUDA(cudaFuncSetAttribute(down_kernel<W_FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-  const int rsmem = (int)(sizeof(int) * kRouteSmemInts(1024, 64 * 16));
+  const int rsmem = (int)(sizeof(int) * kSelectSmemInts(1024, 64 * 16));
   KD_CUDA(cudaFuncSetAttribute(router_kernel<W_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, rsmem));
   KD_CUDA(cudaFuncSetAttribute(router_kernel<W_FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, rsmem));
   KD_CUDA(cudaFuncSetAttribute(tp_route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, rsmem));
@@ -684,7 +684,7 @@ static int launch_layer(kd_layer* L, const Acts& a, cudaStream_t s, const kd_lay
   // before the down kernel.  The router releases its dependent launch only
   // when it is done, so the shared gate/up gets the SMs that the router
   // leaves free while the router runs.
-  const size_t route_ints = sizeof(int) * kRouteSmemInts(d.E, M * d.k);
+  const size_t route_ints = sizeof(int) * kSelectSmemInts(d.E, M * d.k);
   {
     const int rc = launch_front(L, a, s, pdl_first);
     if (rc != KD_OK) return rc;
@@ -807,7 +807,7 @@ extern "C" int kd_tp_moe(kd_layer* L, int M, void* stream) {
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int G = L->nsm;
   const bool mma = L->has_maps && M >= L->mma_min;
-  const size_t route_ints = sizeof(int) * kRouteSmemInts(d.E, M * d.k);
+  const size_t route_ints = sizeof(int) * kSelectSmemInts(d.E, M * d.k);
   KD_CUDA(launch(tp_route_kernel, 1, kRouterThreads, route_ints, s, false, d, M));
   const int gthreads = fp8 ? q8_threads(kGateUpConv) : kMThreads;
   const int dthreads = fp8 ? q8_threads(kDownConv) : kMThreads;

@@ -966,6 +966,18 @@ KD_DEV void groupmax16(const Plan& plan, const MUnit& m, int lane, int c, const 
 
 // The plan's epilogue for 16 accumulator columns (tokens c .. c+15) of this
 // thread's row, then (plans with kGmaxOut) the output's per-64 maxima.
+// Plans whose epilogue reads an input per output (a residual) provide
+// epilogue_in(m, row, j), and emit16 loads the 16 tokens' inputs before the
+// first store (the loads could not move above stores to memory that may alias).
+template <class P, class = void>
+struct HasEpilogueIn {
+  static constexpr bool value = false;
+};
+template <class P>
+struct HasEpilogueIn<P, decltype((void)&P::epilogue_in)> {
+  static constexpr bool value = true;
+};
+
 template <class Plan>
 KD_DEV void emit16(const Plan& plan, const MUnit& m, int row, int lane, int c, const float* v,
                    MmaShared& sh) {
@@ -976,6 +988,15 @@ KD_DEV void emit16(const Plan& plan, const MUnit& m, int row, int lane, int c, c
       const float other = __shfl_xor_sync(0xffffffffu, v[j], 1);
       o[j] = 0.f;
       if (!(lane & 1) && c + j < m.ntok) o[j] = plan.epilogue2(m, row >> 1, c + j, v[j], other);
+    }
+  } else if constexpr (HasEpilogueIn<Plan>::value) {
+    float in[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) in[j] = c + j < m.ntok ? plan.epilogue_in(m, row, c + j) : 0.f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      o[j] = 0.f;
+      if (c + j < m.ntok) o[j] = plan.epilogue(m, row, c + j, v[j], in[j]);
     }
   } else {
 #pragma unroll

@@ -96,7 +96,12 @@ struct MmaProjPlan {
   }
   KD_DEV int b_rowidx(const MUnit&, int j) const { return j; }
   KD_DEV bool paired() const { return false; }
-  KD_DEV float epilogue(const MUnit& m, int r, int j, float v) const {
+  // the residual x of an o-proj output (none for QKV rows and shard partials)
+  KD_DEV float epilogue_in(const MUnit& m, int r, int j) const {
+    if (m.tag == 0 || (MODE == 0 && L->tp)) return 0.f;
+    return __uint_as_float((uint32_t)__ldg(a.x + (size_t)j * L->H + m.lrow + r) << 16);
+  }
+  KD_DEV float epilogue(const MUnit& m, int r, int j, float v, float xin) const {
     const int row = m.lrow + r;
     if (m.tag == 0) {
       L->qkv[(size_t)j * L->Nqkv + row] = f32_to_bf16_bits(v);
@@ -111,8 +116,7 @@ struct MmaProjPlan {
       L->h1f[o] = v;
       return v;
     }
-    // read-only here (a plain load could not move above the stores below)
-    const float h = __uint_as_float((uint32_t)__ldg(a.x + o) << 16) + v;
+    const float h = xin + v;
     if (MODE == 2) {
       L->h1r[o] = h;
       return h;
@@ -187,10 +191,14 @@ struct MmaRouterPlan {
   KD_DEV int b_stride(const MUnit&) const { return L->H * 2; }
   KD_DEV int b_rowidx(const MUnit&, int j) const { return j; }
   KD_DEV bool paired() const { return false; }
-  KD_DEV float epilogue(const MUnit& m, int r, int j, float v) const {
+  // the logit bias of the row (added when it is part of the logits)
+  KD_DEV float epilogue_in(const MUnit& m, int r, int) const {
     const int e = m.lrow + r;
-    if (e < L->E)
-      L->logits[(size_t)j * L->E + e] = v + (L->bias && !L->bias_sel ? __ldg(L->bias + e) : 0.f);
+    return e < L->E && L->bias && !L->bias_sel ? __ldg(L->bias + e) : 0.f;
+  }
+  KD_DEV float epilogue(const MUnit& m, int r, int j, float v, float b) const {
+    const int e = m.lrow + r;
+    if (e < L->E) L->logits[(size_t)j * L->E + e] = v + b;
     return v;
   }
   KD_DEV float epilogue2(const MUnit&, int, int, float, float) const { return 0.f; }
@@ -218,7 +226,7 @@ struct MmaRouterPlan {
     const int n = M * L->E;
     // ring: [logits copy (if it fits)] [routing scratch]
     const size_t lbytes = ((size_t)n * sizeof(float) + 255) & ~(size_t)255;
-    const size_t rbytes = sizeof(int) * kRouteSmemInts(L->E, M * L->k);
+    const size_t rbytes = sizeof(int) * kSelectSmemInts(L->E, M * L->k);
     const bool copy = lbytes + rbytes <= (size_t)kMRingBytes && (n & 3) == 0;
     if (copy) {
       // 16-byte loads, eight in flight per thread (the copy is latency-bound)

@@ -155,10 +155,20 @@ extern "C" int kd_router_topk_static(const void* router_w, const float* router_s
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   // one launch: logits, then the last block selects and builds the lists
   const int rgrid = (n_experts + kRouterRows - 1) / kRouterRows;
-  const size_t smem = sizeof(int) * kRouteSmemInts(n_experts, M * top_k);   // < 48 KB
+  const size_t smem = sizeof(int) * kSelectSmemInts(n_experts, M * top_k);   // <= 57.6 KB
+  // the limit for the largest configuration (the layer sets the same one: a
+  // kernel's attribute is shared by every caller in the process)
+  const int smax = (int)(sizeof(int) * kSelectSmemInts(KD_STATIC_MAX_EXPERTS, kMaxTok * kMaxK));
+  cudaError_t e = wdtype == KD_WFP8
+      ? cudaFuncSetAttribute(router_kernel<W_FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smax)
+      : cudaFuncSetAttribute(router_kernel<W_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smax);
+  if (e != cudaSuccess) {
+    snprintf(g_msg, sizeof g_msg, "kd_router_topk_static: shared memory: %s", cudaGetErrorString(e));
+    return fail_static(KD_ECUDA);
+  }
   if (wdtype == KD_WFP8) router_kernel<W_FP8><<<rgrid, kRouterThreads, smem, s>>>(d, M);
   else router_kernel<W_BF16><<<rgrid, kRouterThreads, smem, s>>>(d, M);
-  cudaError_t e = cudaGetLastError();
+  e = cudaGetLastError();
   if (e != cudaSuccess) {
     snprintf(g_msg, sizeof g_msg, "kd_router_topk_static: launch: %s", cudaGetErrorString(e));
     return fail_static(KD_ECUDA);

@@ -141,6 +141,27 @@ def test_gating_variants(kd, wdtype, M, engine):
             L.close()
 
 
+@pytest.mark.parametrize("E,k,M,sel", [(384, 8, 8, 1), (384, 8, 40, 0), (640, 16, 5, 1),
+                                        (1024, 16, 64, 0)])
+def test_wide_router_layers(kd, E, k, M, sel):
+    """More experts than 256 (a lane of the selection holds 16 or 32 logits),
+    top-16, up to 64 tokens: the layer against the oracle, on the CUDA-core
+    router (M <= 8) and the tensor-core router, with a selection-only or a
+    logit bias."""
+    from kdgen import Dims
+    d = Dims(hidden=256, q_heads=2, kv_heads=1, head_dim=128, n_experts=E, top_k=k, n_shared=1,
+             inter=128)
+    bias = kdgen.zipf_bias(E, 0.3)
+    spec = kd.LayerSpec.from_dims(d, max_tokens=64, router_bias=bias, bias_select_only=sel)
+    L = kd.Layer(spec, seed=3)
+    try:
+        x, a = inputs(d, M, rho=0.2, seed=5)
+        g = run_gpu_layer(L, x, a)
+        compare_layer(d, g, x, a, seed=3, bias=bias.astype(np.float64), bias_select_only=bool(sel))
+    finally:
+        L.close()
+
+
 @pytest.mark.parametrize("dims,M,rows", [(TINY, 8, None), (K2, 32, [0, 7, 19, 31])])
 def test_w8a8_experts(kd, dims, M, rows):
     """FP8 expert weights with one e4m3 term per activation (W8A8) on the
