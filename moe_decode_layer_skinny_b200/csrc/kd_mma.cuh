@@ -990,9 +990,9 @@ KD_DEV void emit16(const Plan& plan, const MUnit& m, int row, int lane, int c, c
       if (!(lane & 1) && c + j < m.ntok) o[j] = plan.epilogue2(m, row >> 1, c + j, v[j], other);
     }
   } else if constexpr (HasEpilogueIn<Plan>::value) {
-    float in[16];
+    decltype(plan.epilogue_in(m, row, 0)) in[16];
 #pragma unroll
-    for (int j = 0; j < 16; ++j) in[j] = c + j < m.ntok ? plan.epilogue_in(m, row, c + j) : 0.f;
+    for (int j = 0; j < 16; ++j) in[j] = c + j < m.ntok ? plan.epilogue_in(m, row, c + j) : 0;
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
       o[j] = 0.f;

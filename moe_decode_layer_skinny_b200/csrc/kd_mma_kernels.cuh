@@ -452,10 +452,15 @@ struct MmaDownPlan {
   KD_DEV int b_stride(const MUnit&) const { return L->I * 2; }
   KD_DEV int b_rowidx(const MUnit& m, int j) const { return m.tok0 + j; }
   KD_DEV bool paired() const { return false; }
-  KD_DEV float epilogue(const MUnit& m, int r, int j, float v) const {
+  // a routed output's (token, slot) code (loaded for 16 tokens before their
+  // stores)
+  KD_DEV int epilogue_in(const MUnit& m, int, int j) const {
+    return m.tag < 0 ? 0 : __ldg(L->perm + m.tok0 + j);
+  }
+  KD_DEV float epilogue(const MUnit& m, int r, int j, float v, int code) const {
     const int h = m.lrow + r;
     if (m.tag < 0) L->ysh[(size_t)(m.tok0 + j) * L->H + h] = v;
-    else L->yr[(size_t)__ldg(L->perm + m.tok0 + j) * L->H + h] = v;
+    else L->yr[(size_t)code * L->H + h] = v;
     return v;
   }
   KD_DEV float epilogue2(const MUnit&, int, int, float, float) const { return 0.f; }
