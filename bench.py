@@ -587,8 +587,11 @@ def run_kd(args):
             unions[name] = r2["active_experts"]
             lbytes[name] = (r2["weight_bytes"] - r2["active_experts"] * r2["expert_bytes"],
                             r2["expert_bytes"])
-        for pf in (True, False):
-            key = "stack4_fp8" + ("" if pf else "_noprefetch")
+        # the stack without and with the next layer's static weights prefetched
+        # into L2 on a side stream (the pages' option; measured slightly slower
+        # here, so the plain chain is the workload's line)
+        for pf in (False, True):
+            key = "stack4_fp8" + ("_prefetch" if pf else "")
             wl[key] = bench_stack(W["stack4_fp8"], max(5, args.steps // 20), 3, flush, pg, local,
                                   peak, pf)
         unions["stack4_fp8"] = wl["stack4_fp8"]["active_experts_layer0"]

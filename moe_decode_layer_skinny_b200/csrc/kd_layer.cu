@@ -708,8 +708,12 @@ static int launch_layer(kd_layer* L, const Acts& a, cudaStream_t s, const kd_lay
   }
   if (d.S) {
     KD_CUDA(cudaStreamWaitEvent(L->side, L->ev_h1, 0));
+    // one CTA fewer than SMs: the router's last CTA holds its SM for the
+    // selection, and a shared gate/up CTA waiting for that SM would start
+    // (and end) late and delay the routed gate/up CTA that follows it there
+    // (per-CTA clocks: routed starts spread 75-87 us -> 75-76 us at batch 1)
     if (mma)
-      KD_CUDA(launch(gateup_mma_for(L), G, gthreads, msm,
+      KD_CUDA(launch(gateup_mma_for(L), std::max(1, G - 1), gthreads, msm,
                      L->side, false, d, M, 1, L->maps));
     else
       KD_CUDA(launch(fp8 ? gateup_kernel<W_FP8> : gateup_kernel<W_BF16>, G, kThreads, sm, L->side,
