@@ -309,9 +309,9 @@ KD_DEV MmaShared carve_mma_smem(uint8_t* base, int nmax, int terms, int nsub, bo
   s.rempty = s.rfull + kMaxMStages;
   if (fp8) {
     s.stage_bytes = nsub * aterms * kATileBytes;
-    // three converted stages hide the MMA's completion latency (two hi + lo
-    // stages, which are twice the size)
-    s.nst = aterms == 1 ? 3 : 2;
+    // three converted stages hide the MMA's completion latency (measured: a
+    // fourth, which leaves fewer e4m3 slots in flight, is slower)
+    s.nst = 3;
     const int bstage = nsub * b_sub_bytes(nmax, terms);
     const int rem = kMRingBytes - s.nst * s.stage_bytes;
     int nb = bstage > 0 ? rem / 3 / bstage : 2;
@@ -392,8 +392,12 @@ KD_DEV bool mwait_lazy(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
 //   int max_n(); int nsub
 //   const CUtensorMap* map(int id)
 //   static constexpr int kTerms    bf16 terms of B (1; 2 = hi + lo; 3 = hi + mid + lo)
-//   static constexpr bool kFp8     A arrives as e4m3 tiles (converter warps, a_scale)
-//   static constexpr int kATerms   bf16 terms of the converted A tile (1, or 2 = hi + lo)
+//   static constexpr int kGatherTerms  (optional, default kTerms) B terms gathered
+//                                  from memory; FP8 plans' converter rewrites B
+//   static constexpr bool kFp8     A arrives as e4m3 tiles; converter warps write
+//                                  them as bf16 (exact) and B as kTerms bf16 terms
+//                                  of (gathered sum) x a_scale
+//   static constexpr int kATerms   bf16 terms of the converted A tile (1)
 //   static constexpr bool kQ8      e4m3 A tiles into kind::f8f6f4 MMAs; B made in-kernel
 //   static constexpr int kConv     q8: converter warps (<= kQ8Conv; the CTA has q8_threads(kConv))
 //                                  from fp32 rows: int kVariants (1, or 2 for gate / up
@@ -487,6 +491,16 @@ KD_DEV void cp_async_arrive_noinc(uint64_t* bar) {
                : "memory");
 }
 
+// B terms a plan gathers from memory (kGatherTerms, else all kTerms).
+template <class P, class = void>
+struct GatherTerms {
+  static constexpr int value = P::kTerms;
+};
+template <class P>
+struct GatherTerms<P, decltype((void)P::kGatherTerms)> {
+  static constexpr int value = P::kGatherTerms;
+};
+
 // Two warps (64 threads) write the B tile of every stage with cp.async:
 // token rows j < ntok (zero-filled up to N), 128 bytes (64 bf16 or 128 e4m3
 // K values) each, 16-byte
@@ -500,6 +514,7 @@ KD_DEV void cp_async_arrive_noinc(uint64_t* bar) {
 template <class Plan>
 KD_DEV void mma_producer_b(const Plan& plan, MmaShared& sh, unsigned* err) {
   constexpr int nh = Plan::kTerms;
+  constexpr int ng = GatherTerms<Plan>::value;   // terms copied (<= nh)
   constexpr int kRows = kMaxN / 8;          // rows per thread (at most)
   const int t = threadIdx.x - 64;           // 0..63
   const int ch = t & 7, rg = t >> 3;
@@ -513,7 +528,7 @@ KD_DEV void mma_producer_b(const Plan& plan, MmaShared& sh, unsigned* err) {
     const size_t stride = (size_t)plan.b_stride(m);   // bytes
     // this thread's sources for the whole unit (byte count 0 = zero fill,
     // ~0 = no row)
-    const uint8_t* src[nh][kRows];
+    const uint8_t* src[ng][kRows];
     uint32_t nb[kRows];
 #pragma unroll
     for (int i = 0; i < kRows; ++i) {
@@ -521,7 +536,7 @@ KD_DEV void mma_producer_b(const Plan& plan, MmaShared& sh, unsigned* err) {
       const bool live = i < nr && r < m.ntok;
       const size_t ro = live ? (size_t)plan.b_rowidx(m, r) * stride : 0;
 #pragma unroll
-      for (int h = 0; h < nh; ++h) src[h][i] = plan.b_base(m, h) + ro + ch * 16;
+      for (int h = 0; h < ng; ++h) src[h][i] = plan.b_base(m, h) + ro + ch * 16;
       nb[i] = i < nr ? (live ? 16u : 0u) : 0xFFFFFFFFu;
     }
     const int bsub = b_sub_bytes(N, nh);
@@ -536,7 +551,7 @@ KD_DEV void mma_producer_b(const Plan& plan, MmaShared& sh, unsigned* err) {
         for (int i = 0; i < kRows; ++i) {
           if (nb[i] != 0xFFFFFFFFu) {
 #pragma unroll
-            for (int h = 0; h < nh; ++h)
+            for (int h = 0; h < ng; ++h)
               cp_async16(bt + u * bsub + h * N * 128 + (rg + 8 * i) * 128, src[h][i] + kb, nb[i]);
           }
         }
@@ -549,23 +564,31 @@ KD_DEV void mma_producer_b(const Plan& plan, MmaShared& sh, unsigned* err) {
 }
 
 // FP8 weights: warps 8-15 turn each e4m3 tile of the raw ring into the
-// stage's bf16 A tile (two [128 x 64] sub-tiles in the 128-byte swizzle),
-// multiplied by the tile's block scale (rows alternate gate/up scales when the
-// plan pairs them): v = bf16(decode(e4m3) * scale), or a bf16 hi + lo pair.
-// Thread t takes the 16-byte chunks t, t + 256, ... of the 1024 in a tile
-// (row = chunk / 8).
+// stage's bf16 A tile (two [128 x 64] sub-tiles in the 128-byte swizzle):
+// bf16(decode(e4m3)), exact (every e4m3 value is a bf16 value).  The tile's
+// block scale goes on B instead: once the stage's B rows have landed, the
+// same warps replace them in place by the kTerms bf16 terms of (the sum of
+// the gathered terms) x scale, so that each product is a weight times an
+// activation term.  A: thread t takes the 16-byte chunks t, t + 256, ... of
+// the 1024 in a tile (row = chunk / 8).  B: the 16-byte chunks of one term
+// (the terms lie N rows apart, so a chunk's swizzled place is the same in
+// every term), in turn.
 template <class Plan>
 KD_DEV void mma_converter(const Plan& plan, MmaShared& sh, unsigned* err) {
+  constexpr int nh = Plan::kTerms, ng = GatherTerms<Plan>::value;
+  static_assert(Plan::kATerms == 1 && !Plan::kQ8, "FP8 converter: one exact A term");
   const int ct = threadIdx.x - 256;
   uint32_t it = 0;
   CtaUnits<Plan> units(plan);
   MUnit m;
   while (units.next(m)) {
+    const int N = pad16(m.ntok);
+    const int bsub = b_sub_bytes(N, nh);
+    const int nchunk = sh.nsub * N * 8;   // 16-byte chunks of one B term per stage
     for (int c = 0; c < m.nkc; ++c, ++it) {
-      const int rs = it % sh.nraw, s = it % sh.nst;
+      const int rs = it % sh.nraw, s = it % sh.nst, sb = it % sh.nbst;
       mwait(&sh.rfull[rs], (it / sh.nraw) & 1u, sh.abort_flag, err);
       mwait(&sh.empty[s], ((it / sh.nst) & 1u) ^ 1u, sh.abort_flag, err);
-      const float2 sc = plan.a_scale(m, m.kc0 + c);   // (even rows, odd rows)
       const uint8_t* raw = sh.raw + (size_t)rs * kRawBytes;
       uint8_t* dst = sh.stage + (size_t)s * sh.stage_bytes;
 #pragma unroll 4
@@ -573,33 +596,55 @@ KD_DEV void mma_converter(const Plan& plan, MmaShared& sh, unsigned* err) {
         const int p = ct + 256 * q;
         const int r = p >> 3, j = p & 7, sw = r & 7;
         const uint4 w = *reinterpret_cast<const uint4*>(raw + r * 128 + ((j ^ sw) << 4));
-        const float f = (r & 1) ? sc.y : sc.x;
         const uint32_t in[4] = {w.x, w.y, w.z, w.w};
-        float v[16];
+        uint32_t out[8];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          e4m3x4_to_f32(in[u], v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) v[4 * u + i] *= f;
+          float v0, v1, v2, v3;
+          e4m3x4_to_f32(in[u], v0, v1, v2, v3);
+          const __nv_bfloat162 h0 = __floats2bfloat162_rn(v0, v1), h1 = __floats2bfloat162_rn(v2, v3);
+          out[2 * u] = *reinterpret_cast<const uint32_t*>(&h0);
+          out[2 * u + 1] = *reinterpret_cast<const uint32_t*>(&h1);
         }
         // K bytes 16j .. 16j+15 -> bf16 sub-tile j/4, 16-byte chunks 2(j%4), 2(j%4)+1
         const int j0 = 2 * (j & 3);
+        uint8_t* sub = dst + (j >> 2) * kATileBytes + r * 128;
+        *reinterpret_cast<uint4*>(sub + ((j0 ^ sw) << 4)) = make_uint4(out[0], out[1], out[2], out[3]);
+        *reinterpret_cast<uint4*>(sub + (((j0 + 1) ^ sw) << 4)) =
+            make_uint4(out[4], out[5], out[6], out[7]);
+      }
+      // B: (gathered terms) x scale -> nh bf16 terms, in place
+      mwait(&sh.bfull[sb], (it / sh.nbst) & 1u, sh.abort_flag, err);
+      const float sc = plan.a_scale(m, m.kc0 + c).x;
+      uint8_t* bt = sh.bst + (size_t)sb * sh.bst_bytes + sh.boff;
+      for (int p = ct; p < nchunk; p += 256) {
+        const int u = p / (N * 8);
+        uint8_t* c0 = bt + u * bsub + (p - u * N * 8) * 16;
+        float v[8];
 #pragma unroll
-        for (int at = 0; at < Plan::kATerms; ++at) {
-          uint32_t out[8];
+        for (int h = 0; h < ng; ++h) {
+          const uint4 t = *reinterpret_cast<const uint4*>(c0 + h * N * 128);
+          const uint32_t tw[4] = {t.x, t.y, t.z, t.w};
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);   // one cvt
-            out[i] = *reinterpret_cast<const uint32_t*>(&h);
-            if (Plan::kATerms > 1) {   // what this term leaves for the next
-              v[2 * i] -= __low2float(h);
-              v[2 * i + 1] -= __high2float(h);
-            }
+          for (int i = 0; i < 4; ++i) {
+            const float lo = __uint_as_float(tw[i] << 16), hi = __uint_as_float(tw[i] & 0xFFFF0000u);
+            v[2 * i] = h ? v[2 * i] + lo : lo;
+            v[2 * i + 1] = h ? v[2 * i + 1] + hi : hi;
           }
-          uint8_t* sub = dst + (at * 2 + (j >> 2)) * kATileBytes + r * 128;
-          *reinterpret_cast<uint4*>(sub + ((j0 ^ sw) << 4)) = make_uint4(out[0], out[1], out[2], out[3]);
-          *reinterpret_cast<uint4*>(sub + (((j0 + 1) ^ sw) << 4)) =
-              make_uint4(out[4], out[5], out[6], out[7]);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[i] *= sc;
+#pragma unroll
+        for (int h = 0; h < nh; ++h) {
+          uint32_t o[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const __nv_bfloat162 b2 = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+            o[i] = *reinterpret_cast<const uint32_t*>(&b2);
+            v[2 * i] -= __low2float(b2);   // what this term leaves for the next
+            v[2 * i + 1] -= __high2float(b2);
+          }
+          *reinterpret_cast<uint4*>(c0 + h * N * 128) = make_uint4(o[0], o[1], o[2], o[3]);
         }
       }
       fence_proxy_async_smem();   // generic-proxy writes -> visible to the tensor core
@@ -632,9 +677,8 @@ KD_DEV void mma_issuer(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigned*
   MUnit m;
   for (; units.next(m); ++nu_local) {
     const int N = pad16(m.ntok);
-    const uint32_t idesc = idesc_bf16(N);
-    // bf16 weights: one MMA per K-step for all terms (their B rows lie one
-    // after another: N' = nterms N columns, summed by the epilogue)
+    // one MMA per K-step for all B terms (their rows lie one after another:
+    // N' = nterms N columns, summed by the epilogue)
     const uint32_t idesc_all = idesc_bf16(nterms * N);
     const int buf = nu_local & 1;
     const uint32_t d = tmem + (uint32_t)(buf * kBfAccCols);
@@ -664,22 +708,17 @@ KD_DEV void mma_issuer(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigned*
                      c > 0 || u > 0 || k > 0);
         }
       } else {
-      // FP8: descriptors by adding byte offsets / 16 to the start-address
-      // field (shared addresses < 256 KB: the field never carries); the
-      // issuing thread shares its SM quarter with two converter warps
+      // FP8: the converted A tile (one exact term) against every B term in
+      // one MMA per K-step, as for bf16 weights; descriptors by adding byte
+      // offsets / 16 to the start-address field (shared addresses < 256 KB:
+      // the field never carries)
       const uint64_t ad0 = sw128_desc(a0), bd0 = sw128_desc(b0);
       for (int u = 0; u < sh.nsub; ++u) {
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const uint64_t bd = bd0 + (uint64_t)((u * bsub + k * 32) >> 4);
-#pragma unroll
-          for (int at = 0; at < Plan::kATerms; ++at) {
-            const uint64_t ad = ad0 + (uint64_t)(((at * sh.nsub + u) * kATileBytes + k * 32) >> 4);
-            mma_bf16(d, ad, bd, idesc, c > 0 || u > 0 || k > 0 || at > 0);
-#pragma unroll
-            for (int h = 1; h < nterms; ++h)
-              mma_bf16(d, ad, bd + (uint64_t)((h * N * 128) >> 4), idesc, true);
-          }
+          const uint64_t ad = ad0 + (uint64_t)((u * kATileBytes + k * 32) >> 4);
+          mma_bf16(d, ad, bd, idesc_all, c > 0 || u > 0 || k > 0);
         }
       }
       }
@@ -1026,10 +1065,9 @@ KD_DEV void mma_epilogue(const Plan& plan, MmaShared& sh, uint32_t tmem, unsigne
     mwait_lazy(&sh.accfull[buf], (nu_local >> 1) & 1u, sh.abort_flag, err);
     tc_fence_after();
     const uint32_t ta = tmem + ((uint32_t)(ew * 32) << 16) + (uint32_t)(buf * kBfAccCols);
-    // 16 tokens of the accumulator: the sum of the terms' column blocks
-    // (bf16 weights; the FP8 projections accumulate their terms in the MMAs)
+    // 16 tokens of the accumulator: the sum of the B terms' column blocks
     auto acc16 = [&](int c, float* v) {
-      constexpr int NT = Plan::kFp8 ? 1 : Plan::kTerms;
+      constexpr int NT = Plan::kTerms;
       float t[NT][16];
 #pragma unroll
       for (int h = 0; h < NT; ++h) tmem_ld16(ta + (uint32_t)(h * N + c), t[h]);

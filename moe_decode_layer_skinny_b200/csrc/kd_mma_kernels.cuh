@@ -59,8 +59,10 @@ struct MmaProjPlan {
   // FP8: h1's per-64 maxima for the q8 gate/up kernels (the full layer's
   // come from its second RMSNorm)
   static constexpr bool kGmaxOut = F8 && MODE == 0;
-  // FP8: the scaled weights as bf16 hi + lo (h1 feeds the fp32 router)
-  static constexpr int kATerms = F8 ? 2 : 1;
+  // FP8: the converter writes the e4m3 tile as bf16 (exact, one term) and
+  // puts the block scale on B: (x s) as a bf16 hi + lo pair, so that the
+  // products stay exact to ~16 bits (h1 feeds the fp32 router)
+  static constexpr int kATerms = 1;
   const LayerDev* L; Acts a; const MmaMaps* maps;
   int nsub;
   int tq, to, cq, co;   // tiles and K chunks per tile of QKV and o-proj
@@ -80,7 +82,10 @@ struct MmaProjPlan {
   }
   KD_DEV const CUtensorMap* map(int id) const { return &maps->m[id]; }
   KD_DEV int max_n() const { return a.M; }
-  static constexpr int kTerms = MODE == 0 ? 1 : 2;
+  static constexpr int kTerms = MODE == 0 && !F8 ? 1 : 2;
+  // B terms gathered from memory (FP8, MODE 0: x; the converter writes the
+  // scaled hi + lo over it)
+  static constexpr int kGatherTerms = MODE == 0 ? 1 : 2;
   KD_DEV float2 a_scale(const MUnit& m, int kc) const {
     const float sc = m.tag == 0 ? L->sqkv[(size_t)(m.row >> 7) * L->nHb + kc]
                                 : L->so[(size_t)(m.row >> 7) * L->nAb + kc];
