@@ -147,7 +147,7 @@ def test_wide_router_layers(kd, E, k, M, sel):
     """More experts than 256 (a lane of the selection holds 16 or 32 logits),
     top-16, up to 64 tokens: the layer against the oracle, on the CUDA-core
     router (M <= 8) and the tensor-core router, with a selection-only or a
-    logit bias."""
+    logit bias.  Every row; the oracle takes 0.02-0.11 s per case."""
     from kdgen import Dims
     d = Dims(hidden=256, q_heads=2, kv_heads=1, head_dim=128, n_experts=E, top_k=k, n_shared=1,
              inter=128)
