@@ -83,13 +83,9 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_moe_kernel(LayerDev L, i
     const float w1 = __fmul_rn(__fmul_rn(h[i + 1], r), __uint_as_float((uint32_t)L.g2[i + 1] << 16));
     L.h1f[o] = w0;
     L.h1f[o + 1] = w1;
-    if (!fp8) {
-      store_hilo3(L.h1b, L.h1lo, L.h1lo2, o, w0);
-      store_hilo3(L.h1b, L.h1lo, L.h1lo2, o + 1, w1);
-      continue;
-    }
-    L.h1b[o] = f32_to_bf16_bits(w0);
-    L.h1b[o + 1] = f32_to_bf16_bits(w1);
+    store_hilo3(L.h1b, L.h1lo, L.h1lo2, o, w0);
+    store_hilo3(L.h1b, L.h1lo, L.h1lo2, o + 1, w1);
+    if (!fp8) continue;
     float mx = fmaxf(fabsf(w0), fabsf(w1));
     for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
     if (lane == 0) L.h1g[(size_t)t * (H / kQGroup) + g] = mx;

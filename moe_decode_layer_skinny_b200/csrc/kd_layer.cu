@@ -229,6 +229,7 @@ static int configure_kernels() {
   KD_CUDA(cudaFuncSetAttribute(mma_gateup_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem));
   KD_CUDA(cudaFuncSetAttribute(mma_down_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem));
   KD_CUDA(cudaFuncSetAttribute(mma_router_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem));
+  KD_CUDA(cudaFuncSetAttribute(mma_router_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem));
   KD_CUDA(cudaFuncSetAttribute(mma_proj_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem));
   KD_CUDA(cudaFuncSetAttribute(mma_gateup_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem));
   KD_CUDA(cudaFuncSetAttribute(mma_down_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, msmem));
@@ -692,15 +693,18 @@ static int launch_layer(kd_layer* L, const Acts& a, cudaStream_t s, const kd_lay
   if (L->timing) KD_CUDA(cudaEventRecord(L->tev[1], s));
   if (d.S) KD_CUDA(cudaEventRecord(L->ev_h1, s));
 
-  // FP8 routers stay on CUDA cores: the tensor-core path rounds each scaled
-  // weight to bf16, which the fp32 router logits cannot afford.  Up to
-  // kCoreRouterMaxM tokens the CUDA-core router (one CTA per two experts) is
-  // also the faster one: the tensor-core router's small grid is a latency chain.
-  if (mma && !fp8 && M > kCoreRouterMaxM) {
-    const int rsub = mma_nsub(M, 3);
+  // Up to kCoreRouterMaxM tokens the CUDA-core router (one CTA per two
+  // experts) is the faster one: the tensor-core router's small grid is a
+  // latency chain.  FP8 router weights go to the tensor cores as exact bf16
+  // with the block scale on h1's three terms (the converter warps).
+  if (mma && M > kCoreRouterMaxM) {
+    const int rsub = fp8 ? 2 : mma_nsub(M, 3);
     const int rchunks = ((d.E + 127) / 128) * (d.H / (64 * rsub));
     const int rgrid = std::max(1, std::min(G, rchunks / (kRouterChunksPerCta * 2 / rsub)));
-    KD_CUDA(launch(mma_router_kernel<false>, rgrid, mthreads, msm, s, !L->timing, d, M, L->maps));
+    if (fp8)
+      KD_CUDA(launch(mma_router_kernel<true>, rgrid, kMThreadsF8, msm, s, !L->timing, d, M, L->maps));
+    else
+      KD_CUDA(launch(mma_router_kernel<false>, rgrid, mthreads, msm, s, !L->timing, d, M, L->maps));
   } else {
     const int rgrid = (d.E + kRouterRows - 1) / kRouterRows;
     KD_CUDA(launch(fp8 ? router_kernel<W_FP8> : router_kernel<W_BF16>, rgrid, kRouterThreads,

@@ -127,8 +127,7 @@ struct MmaProjPlan {
       return h;
     }
     L->h1f[o] = h;
-    if (F8) L->h1b[o] = f32_to_bf16_bits(h);   // the FP8 router reads h1f on CUDA cores
-    else store_hilo3(L->h1b, L->h1lo, L->h1lo2, o, h);
+    store_hilo3(L->h1b, L->h1lo, L->h1lo2, o, h);   // the tensor-core router's three terms
     return h;
   }
   KD_DEV float epilogue2(const MUnit&, int, int, float, float) const { return 0.f; }
