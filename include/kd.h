@@ -301,7 +301,9 @@ int kd_layer_set_timing_events(kd_layer* layer, void* const* events, int n_event
  *                 ties -> lower id
  *   gates_out     device fp32 [M, top_k]: softmax renormalised over the top_k
  * Same arithmetic as the CUDA-core router of kd_decode_layer (the one it
- * runs below the tensor-core token threshold).  Limits: M <= 64
+ * runs for up to 8 tokens); each call raises that kernel's dynamic shared
+ * memory limit to the largest size these limits need (cudaFuncSetAttribute,
+ * not an allocation).  Limits: M <= 64
  * (KD_STATIC_MAX_TOKENS), n_experts <= 1024 (KD_STATIC_MAX_EXPERTS),
  * top_k <= 16, hidden <= 8192 (KD_STATIC_MAX_HIDDEN); larger sizes return
  * KD_ERANGE; null pointers, hidden not a multiple of 128 or a bad wdtype
